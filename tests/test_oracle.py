@@ -295,6 +295,10 @@ def test_zero_down_projection_makes_block_identity(moe):
     # X1 = X0, X2 = X1 + X0, X3 = X2, X4 = X3 + X2, X5 = X4 (the last layer takes no inter-residual)
     for l, c in enumerate([1, 1, 2, 2, 4, 4]):
         assert np.array_equal(hist[l], c * X), l
+    # L = 4 is a multiple of the gap: the last layer still takes no inter-residual
+    hist4 = O.stack_forward(X, cfg.with_(L=4), lambda l, s, j: w[(l, s, j)])["hist"]
+    for l, c in enumerate([1, 1, 2, 2, 2]):
+        assert np.array_equal(hist4[l], c * X), l
 
 
 def test_per_bank_isolation():
