@@ -1,0 +1,184 @@
+/*
+ * tm.h -- C ABI of the B200 TokenMixer-Large forward library (libtm.so).
+ *
+ * The library runs the forward pass of the TokenMixer-Large block and stack on
+ * one B200 (sm_100a).  Sources for what each call computes:
+ *   [digest] "TokenMixer-Large: Scaling Up Large Ranking Models in Industrial
+ *            Recommenders", paper digest of arXiv 2602.06563, sections 2.2-2.5;
+ *   [readme] "tokenmixerlarge" README of the TensorFlow/Keras reproduction,
+ *            block diagram and the list of paper-faithful choices.
+ *
+ * Conventions shared by every call:
+ *   - Every tensor pointer is caller-owned DEVICE memory, 16-byte aligned, in
+ *     row-major (C) order with the shape given beside it.  The library never
+ *     allocates device memory and never frees caller memory; scratch space is
+ *     the caller's `workspace`, sized by the *_workspace_bytes queries.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls only
+ *     enqueue work: nothing synchronises except tm_get_device_error.
+ *   - Storage dtype is tm_shape.dtype (fp32 or bf16) for activations and FFN
+ *     weights; router weights are always fp32; accumulation is always fp32;
+ *     stores to bf16 round to nearest-even.
+ *   - Weights are [out, in] ("K-major"): a hidden unit's gate row is contiguous
+ *     over the input width.
+ *   - Host-side validation runs before any launch.  On TM_ERR_INVALID_ARG,
+ *     TM_ERR_UNSUPPORTED or TM_ERR_WORKSPACE nothing is launched and no output
+ *     is touched.  A kernel that hits a bounded-wait timeout or a bounds check
+ *     records it in a device error word (it never traps); read it with
+ *     tm_get_device_error.
+ *   - Results are deterministic: the same inputs give the same output bits.
+ *   - Calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef TM_H_
+#define TM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TM_OK = 0,
+    TM_ERR_INVALID_ARG = 1,     /* bad shape, null or misaligned pointer */
+    TM_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. a width the kernels lack) */
+    TM_ERR_WORKSPACE = 3,       /* workspace null or smaller than the query returned */
+    TM_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed */
+    TM_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded wait ran out (reported by tm_get_device_error) */
+    TM_ERR_DEVICE_BOUNDS = 6    /* a kernel's bounds check fired (reported by tm_get_device_error) */
+} tm_status;
+
+typedef enum { TM_F32 = 0, TM_BF16 = 1 } tm_dtype;
+
+/* How a sub-layer sees its input rows and writes its output.
+ *   TM_LAYOUT_ROWS : x, residual and y are [B, banks, width] (for the reverting
+ *                    sub-layer that is [B, T, D] with banks = T, width = D).
+ *   TM_LAYOUT_MIXED: x, residual and y are token tensors [B, T, D]; the rows are
+ *                    Mix(x) (banks = H, width = T*D/H, [digest] 2.3.1 Eq. 9-11)
+ *                    and the output rows are written back through Revert
+ *                    (Eq. 13-15), so Mix/Revert are never materialised.      */
+typedef enum { TM_LAYOUT_ROWS = 0, TM_LAYOUT_MIXED = 1 } tm_layout;
+
+/* Token tensor X in R[B, T, D] ([digest] 2.2, Eq. 4), H heads with D % H == 0,
+ * RMSNorm epsilon (added inside the square root). */
+typedef struct { int B, T, D, H; tm_dtype dtype; float eps; } tm_shape;
+
+/* Per-token SwiGLU bank ([digest] 2.3.2, Eq. 17-18, no bias): one weight set per
+ * bank.  w_gate, w_up: [banks, hidden, width]; w_down: [banks, width, hidden]. */
+typedef struct {
+    int banks, width, hidden;
+    const void *w_gate, *w_up, *w_down;
+} tm_swiglu_w;
+
+/* Sparse-Pertoken MoE bank ([digest] 2.4, Eq. 19-21): per bank, an fp32 router
+ * w_router [banks, E, width], E routed SwiGLU experts we_gate/we_up
+ * [banks, E, hidden_e, width], we_down [banks, E, width, hidden_e], and one
+ * always-on shared expert ws_gate/ws_up [banks, hidden_s, width], ws_down
+ * [banks, width, hidden_s] (hidden_s == 0: no shared expert, ws_* ignored).
+ * Output = alpha * sum_{top-k e} softmax(router logits)_e * Expert_e + Shared. */
+typedef struct {
+    int banks, width, E, k, hidden_e, hidden_s;
+    float alpha;
+    const float *w_router;
+    const void *we_gate, *we_up, *we_down;
+    const void *ws_gate, *ws_up, *ws_down;
+} tm_moe_w;
+
+/* One sub-layer: RMSNorm gain [width] (NULL = all ones) and its FFN bank. */
+typedef struct {
+    const void *norm_gain;
+    int is_moe;            /* 0: dense (uses .dense), 1: MoE (uses .moe) */
+    tm_swiglu_w dense;
+    tm_moe_w moe;
+} tm_sublayer;
+
+/* One block: the mixing sub-layer (banks = H, width = T*D/H) and the reverting
+ * sub-layer (banks = T, width = D). */
+typedef struct { tm_sublayer mix, rev; } tm_block;
+
+/* Static string for a status code. */
+const char *tm_status_string(tm_status s);
+
+/* Library ABI version (major * 100 + minor). */
+int tm_version(void);
+
+/* Workspace bytes needed by tm_pertoken_swiglu / tm_sparse_pertoken_moe for this
+ * sub-layer and layout (0 if the arguments are invalid). */
+size_t tm_sublayer_workspace_bytes(const tm_shape *shape, tm_layout layout, const tm_sublayer *sub);
+
+/* Workspace bytes needed by tm_route_topk. */
+size_t tm_route_workspace_bytes(const tm_shape *shape, tm_layout layout, const tm_moe_w *w);
+
+/* Workspace bytes needed by tm_block_forward (L = 1) or tm_stack_forward. */
+size_t tm_workspace_bytes(const tm_shape *shape, const tm_block *blocks, int L, int inter_residual_gap);
+
+/* Group-wise tokenizer stub ([digest] 2.2.1-2.2.2, Eq. 2-4), one bias-free linear
+ * layer per group: X[b,0] = w_global . concat_g groups[b,g]  (the global token),
+ * X[b,t] = w_group[t-1] . groups[b,t-1] for t = 1..T-1.
+ * groups [B, T-1, dg]; w_group [T-1, D, dg]; w_global [D, (T-1)*dg]; X_out [B,T,D].
+ * A boundary utility (plain CUDA-core kernel), not part of the timed path. */
+tm_status tm_tokenize_stub(const void *groups, const void *w_group, const void *w_global, int dg,
+                           const tm_shape *shape, void *X_out, void *stream);
+
+/* Mix ([digest] 2.3.1, Eq. 9-11): Hm[b, h, t*dh + j] = X[b, t, h*dh + j],
+ * X [B,T,D] -> Hm [B, H, T*D/H].  A test/API utility: the fused path never calls it. */
+tm_status tm_mix(const void *X, void *Hm, const tm_shape *shape, void *stream);
+
+/* Revert ([digest] 2.3.1, Eq. 13-15), the inverse of Mix: Hm [B,H,T*D/H] -> X [B,T,D]. */
+tm_status tm_revert(const void *Hm, void *X, const tm_shape *shape, void *stream);
+
+/* Router of a Sparse-Pertoken MoE sub-layer ([digest] 2.4.1 Eq. 19, 2.4.3 Eq. 21)
+ * plus the expert-first bucketing that [digest] 2.5.1 calls MoEPermute.
+ * For every row r = (b, bank): n = RMSNorm(row) * gain; logits = w_router[bank] . n
+ * in fp32; p = softmax over all E; the k largest p (ties: lower expert index) in
+ * descending order.  Outputs:
+ *   topk_idx   [B, banks, k] int32  chosen experts
+ *   topk_gate  [B, banks, k] fp32   alpha * p of each chosen expert (no renormalisation)
+ *   inv_rms    [B, banks]    fp32   1/sqrt(mean(row^2) + eps)   (may be NULL)
+ *   bucket_offsets [banks*E + 1] int32  start of group g = bank*E + e in bucket_rows
+ *   bucket_rows    [B*banks*k]   int32  sample index b of every routed row, grouped by
+ *                                       (bank, expert), ascending b inside a group
+ *   slot_of        [B, banks, k] int32  position in bucket_rows of (b, bank, j)
+ * x and layout as in tm_layout. */
+tm_status tm_route_topk(const void *x, tm_layout layout, const tm_shape *shape, const void *norm_gain,
+                        const tm_moe_w *w, int32_t *topk_idx, float *topk_gate, float *inv_rms,
+                        int32_t *bucket_offsets, int32_t *bucket_rows, int32_t *slot_of,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* Dense per-token SwiGLU sub-layer with pre-RMSNorm and residual
+ * ([readme] block diagram; [digest] 2.3.2-2.3.3):
+ *   y_row = SwiGLU_bank(RMSNorm(x_row) * gain) + residual_row
+ * residual may be NULL (no residual) and has the layout of y.  y must not alias x. */
+tm_status tm_pertoken_swiglu(const void *x, const void *residual, tm_layout layout, const tm_shape *shape,
+                             const void *norm_gain, const tm_swiglu_w *w, void *y,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/* Sparse-Pertoken MoE sub-layer ([digest] 2.4, Eq. 19-21) with pre-RMSNorm and residual:
+ *   y_row = alpha * sum_{top-k e} p_e * Expert_{bank,e}(n) + Shared_bank(n) + residual_row.
+ * Routing as in tm_route_topk; the combine is a fixed-order fp32 sum (deterministic). */
+tm_status tm_sparse_pertoken_moe(const void *x, const void *residual, tm_layout layout, const tm_shape *shape,
+                                 const void *norm_gain, const tm_moe_w *w, void *y,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/* One TokenMixer-Large block ([readme] block diagram; [digest] Eq. 9-16, pre-norm reading):
+ *   H = Mix(X); H_next = FFN_mix(Norm(H)) + H; X_rev = Revert(H_next);
+ *   Y = FFN_rev(Norm(X_rev)) + X.
+ * X, Y [B,T,D]; X_revert_opt [B,T,D] receives X_rev when not NULL. */
+tm_status tm_block_forward(const void *X, const tm_block *block, const tm_shape *shape, void *Y,
+                           void *X_revert_opt, void *workspace, size_t workspace_bytes, void *stream);
+
+/* L blocks with the inter-residual of [digest] 2.3.4 ([readme]: "at gap 2, excluded
+ * from the final layer"): X_l = Block_l(X_{l-1}); X_l += X_{l-gap} when gap > 0,
+ * l % gap == 0 and l < L (layers counted from 1).  Y = X_L.  Y must not alias X. */
+tm_status tm_stack_forward(const void *X, const tm_block *blocks, int L, int inter_residual_gap,
+                           const tm_shape *shape, void *Y, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/* Synchronises `stream`, returns the first device-side error recorded since the
+ * last call (TM_OK if none) and clears it. */
+tm_status tm_get_device_error(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TM_H_ */

@@ -128,3 +128,17 @@ def stack(X, T, D, H, eps, L, gap, specs, weights):
             Y = [[[Y[b][t][d] + prev[b][t][d] for d in range(D)] for t in range(T)] for b in range(len(Y))]
         hist.append(Y)
     return hist[-1]
+
+
+def tokenize(groups, w_group, w_global):
+    """Scalar loops: X[b][0][d] = sum_{i,c} w_global[d][i*dg + c] * groups[b][i][c];
+    X[b][i+1][d] = sum_c w_group[i][d][c] * groups[b][i][c]."""
+    B, G, dg = len(groups), len(groups[0]), len(groups[0][0])
+    D = len(w_group[0])
+    X = []
+    for b in range(B):
+        toks = [[sum(w_global[d][i * dg + c] * groups[b][i][c] for i in range(G) for c in range(dg)) for d in range(D)]]
+        for i in range(G):
+            toks.append([sum(w_group[i][d][c] * groups[b][i][c] for c in range(dg)) for d in range(D)])
+        X.append(toks)
+    return X

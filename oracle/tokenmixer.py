@@ -218,3 +218,20 @@ def stack_forward(X: np.ndarray, cfg, bank_w: Callable[[int, int, int], Weights]
         hist.append(Xl)
         blocks.append(b if keep else {"mix": b["mix"], "rev": b["rev"]})
     return {"Y": hist[-1], "hist": hist, "blocks": blocks}
+
+
+# ------------------------------------------------------------------ tokenizer stub
+def tokenize(groups: np.ndarray, w_group: np.ndarray, w_global: np.ndarray) -> np.ndarray:
+    """Group-wise tokens plus a global token.  [digest] 2.2.1-2.2.2, Eq. 2-4.
+
+    Each group MLP is read as one bias-free linear layer (the pages leave its depth open).
+    groups [B, G, dg]; w_group [G, D, dg]; w_global [D, G*dg]  ->  X [B, G+1, D] with
+    the global token first (Eq. 4 lists X_G before the group tokens).
+    """
+    B, G, dg = groups.shape
+    D = w_group.shape[1]
+    X = np.empty((B, G + 1, D))
+    X[:, 0, :] = groups.reshape(B, G * dg) @ w_global.T           # Eq. 3
+    for i in range(G):
+        X[:, i + 1, :] = groups[:, i, :] @ w_group[i].T            # Eq. 2
+    return X

@@ -332,3 +332,22 @@ def test_samples_are_independent():
     perm = np.array([4, 1, 5, 0, 3, 2])
     assert np.allclose(O.stack_forward(X[perm], cfg, get)["Y"], full[perm], rtol=1e-13, atol=1e-14)
     assert np.allclose(O.stack_forward(X[2:3], cfg, get)["Y"], full[2:3], rtol=1e-13, atol=1e-14)
+
+
+def test_tokenize_matches_bruteforce_and_identity():
+    rng = np.random.default_rng(26)
+    g = rng.standard_normal((3, 4, 5))
+    wg = rng.standard_normal((4, 6, 5))
+    wG = rng.standard_normal((6, 20))
+    got = O.tokenize(g, wg, wG)
+    assert got.shape == (3, 5, 6)
+    assert np.allclose(got, np.array(brute.tokenize(g.tolist(), wg.tolist(), wG.tolist())), rtol=1e-13, atol=1e-13)
+    # identity group maps copy each group; a global map picking element c of group i puts it at d
+    gi = rng.standard_normal((2, 3, 4))
+    eye = np.stack([np.eye(4)] * 3)
+    wsel = np.zeros((4, 12))
+    wsel[0, 5] = wsel[1, 0] = wsel[2, 11] = wsel[3, 6] = 1.0
+    X = O.tokenize(gi, eye, wsel)
+    assert np.array_equal(X[:, 1:, :], gi)
+    flat = gi.reshape(2, 12)
+    assert np.array_equal(X[:, 0, :], flat[:, [5, 0, 11, 6]])
