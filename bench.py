@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Throughput of the TokenMixer-Large forward on B200 (one JSON line on rank 0).
+
+A step is one tm_stack_forward over one batch of the dense bf16 block workload
+(B=4096 samples, T=16 tokens, D=256, H=16 heads, per-token SwiGLU hidden 1024 in
+both sub-layers, L=1) with synthetic inputs and random weights already resident in
+HBM.  Each timed step is bracketed by CUDA events on the launching stream; a 256 MB
+write between steps flushes the 126 MB L2, so every step starts cold.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+N > 1 (under torchrun): every rank runs its own batch (weak scaling, no data-path
+collective); the step time is the max over ranks.  --impl reference times the CPU
+float64 oracle on the host cores (rank 0 only) on a bounded sample of the workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import tm_synth as S  # noqa: E402
+
+METRIC = "samples/sec & TFLOP/s of TokenMixer-Large fwd, % of B200 bf16 TC roofline"
+DEFAULT_WORKLOAD = "dense_block_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["tm_gemm.cuh", "tm_device.cuh", "tm_gemm.cu", "tm_kernels.cu", "tm_api.cu"]
+
+
+def describe(cfg) -> str:
+    def ffn(s):
+        if s.is_moe:
+            return f"MoE E={s.E} k={s.k} Fe={s.hidden_e} Fs={s.hidden_s} alpha={s.alpha:g}"
+        return f"SwiGLU F={s.hidden}"
+    return (f"{cfg.name}: B={cfg.B} T={cfg.T} D={cfg.D} H={cfg.H} L={cfg.L} gap={cfg.gap} {cfg.dtype}; "
+            f"mix {ffn(cfg.mix)}; rev {ffn(cfg.rev)}")
+
+
+def sublayer_flops_per_sample(cfg, sub) -> float:
+    """Algorithmic flops of one sub-layer per sample: only the work the method performs
+    (the k chosen experts, the shared expert, the router); Mix/Revert 0, RMSNorm not counted."""
+    s, W, banks = cfg.ffn(sub), cfg.width(sub), cfg.banks(sub)
+    if s.is_moe:
+        return banks * (s.k * 6.0 * W * s.hidden_e + 6.0 * W * s.hidden_s + 2.0 * W * s.E)
+    return banks * 6.0 * W * s.hidden
+
+
+def flops_per_sample(cfg) -> float:
+    return cfg.L * (sublayer_flops_per_sample(cfg, 0) + sublayer_flops_per_sample(cfg, 1))
+
+
+def swiglu_gemm_flops(cfg, B) -> list:
+    """Algorithmic flops of each gemm_swiglu launch of one step, in launch order."""
+    out = []
+    for _ in range(cfg.L):
+        for sub in (0, 1):
+            s, W, banks = cfg.ffn(sub), cfg.width(sub), cfg.banks(sub)
+            if s.is_moe:
+                out.append(B * banks * s.k * 4.0 * W * s.hidden_e)        # routed experts
+                out.append(B * banks * 4.0 * W * s.hidden_s)              # shared expert
+            else:
+                out.append(B * banks * 4.0 * W * s.hidden)
+    return out
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "token_sparse_moe_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on these kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("kernel_hash") != kernel_hash():
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.f is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.f.flush()
+        with open(self.f.name) as g:
+            rows = [l.strip().split(", ") for l in g if l.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def time_oracle(cfg, budget_s: float, max_samples: int):
+    """Oracle samples/s on the host cores over a bounded sample (weights drawn beforehand)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    get = oracle.synth_banks(cfg)
+    for l in range(cfg.L):
+        for sub in (0, 1):
+            for j in range(cfg.banks(sub)):
+                get(l, sub, j)
+    n = min(max_samples, cfg.B)
+    X = S.to_f64(S.make_x(cfg, np.arange(n)))
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle.stack_forward(X, cfg, get)
+        done += n
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return done / dt, {"cores": int(threads), "samples": done, "seconds": dt, "per_call": n}
+
+
+def run_reference(args, cfg, rank):
+    if rank != 0:
+        return
+    steps, warm = args.steps_ref, max(1, min(args.warmup, 1))
+    import oracle
+    get = oracle.synth_banks(cfg)
+    for l in range(cfg.L):
+        for sub in (0, 1):
+            for j in range(cfg.banks(sub)):
+                get(l, sub, j)
+    n = min(args.ref_samples, cfg.B)
+    X = S.to_f64(S.make_x(cfg, np.arange(n)))
+    for _ in range(warm):
+        oracle.stack_forward(X, cfg, get)
+    t = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        oracle.stack_forward(X, cfg, get)
+        t.append(time.perf_counter() - t0)
+    from threadpoolctl import threadpool_info
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    sec = sum(t)
+    value = n * steps / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "samples/s", "n_gpus": args.gpus,
+        "steps": steps, "warmup": warm, "ms_per_step": 1e3 * sec / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(cfg), "global_batch": n, "parallelism": "host cores",
+                   "step": f"oracle stack forward on the first {n} samples of the batch"},
+        "tflops": flops_per_sample(cfg) * value / 1e12,
+        "cpu_baseline": {"value": value, "unit": "samples/s", "cores": int(threads), "kind": "oracle",
+                         "sample": f"{steps} steps x {n} samples of {cfg.name}"},
+        "e2e": {"value": value, "unit": "samples/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from token_sparse_moe_b200 import api
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    blocks = api.blocks_from_synth(cfg, dev)
+    sh = api.config_shape(cfg)
+    run = api.StackRunner(blocks, sh, cfg.gap, dev)
+    X = api.to_device(S.make_x(cfg.with_(seed=cfg.seed + rank)), dev)
+    Y = torch.empty_like(X)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    K, W = args.steps, args.warmup
+
+    with torch.cuda.stream(stream):
+        for _ in range(W):
+            flush.zero_()
+            run(X, Y, stream)
+        stream.synchronize()
+        api.get_device_error(stream)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        n0 = api.launch_count()
+        api.profile_start()
+        with ClockSampler(local_rank) as clk:
+            t_wall = time.perf_counter()
+            for i in range(K):
+                flush.zero_()
+                ev[i][0].record(stream)
+                run(X, Y, stream)
+                ev[i][1].record(stream)
+            stream.synchronize()
+            t_wall = time.perf_counter() - t_wall
+        kern = api.profile_stop()
+        launches = api.launch_count() - n0
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        api.get_device_error(stream)
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+
+    mean_ms = sum(step_ms) / K
+    if world > 1:
+        t = torch.tensor([mean_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        mean_ms = float(t.item())
+
+    # end to end through the public API: pinned host X -> device -> forward -> pinned host Y
+    Ke = min(K, args.e2e_steps)
+    Xh = X.cpu().pin_memory()
+    Yh = torch.empty_like(Xh).pin_memory()
+    Xd = torch.empty_like(X)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            run.run_host(Xh, Yh, Xd, Y, stream)
+        stream.synchronize()
+        eve = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+        for i in range(Ke):
+            flush.zero_()
+            eve[i][0].record(stream)
+            run.run_host(Xh, Yh, Xd, Y, stream)
+            eve[i][1].record(stream)
+        stream.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in eve) / Ke
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    io_bytes = X.numel() * X.element_size()
+
+    if rank != 0:
+        return
+    pk, pk_src = peaks()
+    total_samples = cfg.B * world
+    value = total_samples / (mean_ms / 1e3)
+    tflops = flops_per_sample(cfg) * value / 1e12
+    # dominant kernel: largest share of device time in the timed region
+    dom = max(kern.items(), key=lambda kv: kv[1]["total_ms"]) if kern else (None, None)
+    roof = None
+    if dom[0] == "gemm_swiglu":
+        per_step = swiglu_gemm_flops(cfg, cfg.B)
+        per_launch = sum(per_step) / len(per_step)
+        avg_ms = dom[1]["total_ms"] / dom[1]["launches"]
+        ach = per_launch / (avg_ms / 1e3) / 1e12
+        tr = traffic_for("gemm_swiglu", cfg.name)
+        roof = {"kernel": "gemm_swiglu", "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"], "traffic": tr,
+                "peak_source": f"{pk_src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)" if pk_src == "measured"
+                else "fallback 1.59 PFLOP/s", "flops_per_launch": per_launch, "avg_launch_ms": avg_ms}
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, info = time_oracle(cfg, args.cpu_seconds, args.cpu_samples)
+        cpu = {"value": v, "unit": "samples/s", "cores": info["cores"], "kind": "oracle",
+               "sample": f"{info['samples']} samples ({info['per_call']} per oracle call) of {cfg.name}, "
+                         f"{info['seconds']:.1f} s of host time"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "samples/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded normal inputs, random-init weights of the workload's shapes)",
+        "config": {"workload": describe(cfg), "global_batch": total_samples, "seq_len": cfg.T,
+                   "parallelism": f"dp{world} (independent batches, no data-path collective)",
+                   "l2": "flushed by a 256 MB write between timed steps (outside the step events)"},
+        "tflops": tflops, "tc_roofline_frac": tflops / pk["bf16_tflops"],
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": total_samples / (e2e_ms / 1e3), "unit": "samples/s", "h2d_bytes_per_step": io_bytes,
+                "d2h_bytes_per_step": io_bytes, "ms_per_step": e2e_ms, "steps": Ke},
+        "gpu_launches": int(launches),
+        "launches_per_step": launches / K,
+        "kernels": {k: {"launches": v["launches"], "avg_ms": v["total_ms"] / v["launches"],
+                        "share": v["total_ms"] / sum(x["total_ms"] for x in kern.values())}
+                    for k, v in sorted(kern.items(), key=lambda kv: -kv[1]["total_ms"])},
+        "clocks": clk.summary(),
+        "wall_s_timed": t_wall,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(S.CONFIGS))
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-samples", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-samples", type=int, default=128)
+    ap.add_argument("--steps-ref", type=int, default=None)
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = S.CONFIGS[args.workload]
+    if args.impl == "reference":
+        args.steps_ref = args.steps_ref or min(args.steps, 20)
+        run_reference(args, cfg, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, cfg, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

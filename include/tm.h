@@ -34,6 +34,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define TM_API __attribute__((visibility("default")))
+#else
+#define TM_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -97,35 +103,35 @@ typedef struct {
 typedef struct { tm_sublayer mix, rev; } tm_block;
 
 /* Static string for a status code. */
-const char *tm_status_string(tm_status s);
+TM_API const char *tm_status_string(tm_status s);
 
 /* Library ABI version (major * 100 + minor). */
-int tm_version(void);
+TM_API int tm_version(void);
 
 /* Workspace bytes needed by tm_pertoken_swiglu / tm_sparse_pertoken_moe for this
  * sub-layer and layout (0 if the arguments are invalid). */
-size_t tm_sublayer_workspace_bytes(const tm_shape *shape, tm_layout layout, const tm_sublayer *sub);
+TM_API size_t tm_sublayer_workspace_bytes(const tm_shape *shape, tm_layout layout, const tm_sublayer *sub);
 
 /* Workspace bytes needed by tm_route_topk. */
-size_t tm_route_workspace_bytes(const tm_shape *shape, tm_layout layout, const tm_moe_w *w);
+TM_API size_t tm_route_workspace_bytes(const tm_shape *shape, tm_layout layout, const tm_moe_w *w);
 
 /* Workspace bytes needed by tm_block_forward (L = 1) or tm_stack_forward. */
-size_t tm_workspace_bytes(const tm_shape *shape, const tm_block *blocks, int L, int inter_residual_gap);
+TM_API size_t tm_workspace_bytes(const tm_shape *shape, const tm_block *blocks, int L, int inter_residual_gap);
 
 /* Group-wise tokenizer stub ([digest] 2.2.1-2.2.2, Eq. 2-4), one bias-free linear
  * layer per group: X[b,0] = w_global . concat_g groups[b,g]  (the global token),
  * X[b,t] = w_group[t-1] . groups[b,t-1] for t = 1..T-1.
  * groups [B, T-1, dg]; w_group [T-1, D, dg]; w_global [D, (T-1)*dg]; X_out [B,T,D].
  * A boundary utility (plain CUDA-core kernel), not part of the timed path. */
-tm_status tm_tokenize_stub(const void *groups, const void *w_group, const void *w_global, int dg,
+TM_API tm_status tm_tokenize_stub(const void *groups, const void *w_group, const void *w_global, int dg,
                            const tm_shape *shape, void *X_out, void *stream);
 
 /* Mix ([digest] 2.3.1, Eq. 9-11): Hm[b, h, t*dh + j] = X[b, t, h*dh + j],
  * X [B,T,D] -> Hm [B, H, T*D/H].  A test/API utility: the fused path never calls it. */
-tm_status tm_mix(const void *X, void *Hm, const tm_shape *shape, void *stream);
+TM_API tm_status tm_mix(const void *X, void *Hm, const tm_shape *shape, void *stream);
 
 /* Revert ([digest] 2.3.1, Eq. 13-15), the inverse of Mix: Hm [B,H,T*D/H] -> X [B,T,D]. */
-tm_status tm_revert(const void *Hm, void *X, const tm_shape *shape, void *stream);
+TM_API tm_status tm_revert(const void *Hm, void *X, const tm_shape *shape, void *stream);
 
 /* Router of a Sparse-Pertoken MoE sub-layer ([digest] 2.4.1 Eq. 19, 2.4.3 Eq. 21)
  * plus the expert-first bucketing that [digest] 2.5.1 calls MoEPermute.
@@ -140,7 +146,7 @@ tm_status tm_revert(const void *Hm, void *X, const tm_shape *shape, void *stream
  *                                       (bank, expert), ascending b inside a group
  *   slot_of        [B, banks, k] int32  position in bucket_rows of (b, bank, j)
  * x and layout as in tm_layout. */
-tm_status tm_route_topk(const void *x, tm_layout layout, const tm_shape *shape, const void *norm_gain,
+TM_API tm_status tm_route_topk(const void *x, tm_layout layout, const tm_shape *shape, const void *norm_gain,
                         const tm_moe_w *w, int32_t *topk_idx, float *topk_gate, float *inv_rms,
                         int32_t *bucket_offsets, int32_t *bucket_rows, int32_t *slot_of,
                         void *workspace, size_t workspace_bytes, void *stream);
@@ -149,14 +155,14 @@ tm_status tm_route_topk(const void *x, tm_layout layout, const tm_shape *shape, 
  * ([readme] block diagram; [digest] 2.3.2-2.3.3):
  *   y_row = SwiGLU_bank(RMSNorm(x_row) * gain) + residual_row
  * residual may be NULL (no residual) and has the layout of y.  y must not alias x. */
-tm_status tm_pertoken_swiglu(const void *x, const void *residual, tm_layout layout, const tm_shape *shape,
+TM_API tm_status tm_pertoken_swiglu(const void *x, const void *residual, tm_layout layout, const tm_shape *shape,
                              const void *norm_gain, const tm_swiglu_w *w, void *y,
                              void *workspace, size_t workspace_bytes, void *stream);
 
 /* Sparse-Pertoken MoE sub-layer ([digest] 2.4, Eq. 19-21) with pre-RMSNorm and residual:
  *   y_row = alpha * sum_{top-k e} p_e * Expert_{bank,e}(n) + Shared_bank(n) + residual_row.
  * Routing as in tm_route_topk; the combine is a fixed-order fp32 sum (deterministic). */
-tm_status tm_sparse_pertoken_moe(const void *x, const void *residual, tm_layout layout, const tm_shape *shape,
+TM_API tm_status tm_sparse_pertoken_moe(const void *x, const void *residual, tm_layout layout, const tm_shape *shape,
                                  const void *norm_gain, const tm_moe_w *w, void *y,
                                  void *workspace, size_t workspace_bytes, void *stream);
 
@@ -164,19 +170,41 @@ tm_status tm_sparse_pertoken_moe(const void *x, const void *residual, tm_layout 
  *   H = Mix(X); H_next = FFN_mix(Norm(H)) + H; X_rev = Revert(H_next);
  *   Y = FFN_rev(Norm(X_rev)) + X.
  * X, Y [B,T,D]; X_revert_opt [B,T,D] receives X_rev when not NULL. */
-tm_status tm_block_forward(const void *X, const tm_block *block, const tm_shape *shape, void *Y,
+TM_API tm_status tm_block_forward(const void *X, const tm_block *block, const tm_shape *shape, void *Y,
                            void *X_revert_opt, void *workspace, size_t workspace_bytes, void *stream);
 
 /* L blocks with the inter-residual of [digest] 2.3.4 ([readme]: "at gap 2, excluded
  * from the final layer"): X_l = Block_l(X_{l-1}); X_l += X_{l-gap} when gap > 0,
  * l % gap == 0 and l < L (layers counted from 1).  Y = X_L.  Y must not alias X. */
-tm_status tm_stack_forward(const void *X, const tm_block *blocks, int L, int inter_residual_gap,
+TM_API tm_status tm_stack_forward(const void *X, const tm_block *blocks, int L, int inter_residual_gap,
                            const tm_shape *shape, void *Y, void *workspace, size_t workspace_bytes,
                            void *stream);
 
+/* Per-kernel timing of the library's own launches (tracing). */
+typedef struct {
+    char name[48];       /* kernel family, e.g. "gemm_swiglu" */
+    int launches;        /* launches recorded between start and stop */
+    double total_ms;     /* sum of their CUDA-event durations on the launching stream */
+} tm_kernel_time;
+
+/* Start recording a CUDA event pair around every kernel the library launches from now on. */
+TM_API tm_status tm_profile_start(void);
+
+/* Stop recording, synchronise the device, and fold the recorded launches into at most
+ * max_entries per-kernel totals in `out` (count written to *n_entries). */
+TM_API tm_status tm_profile_stop(tm_kernel_time *out, int max_entries, int *n_entries);
+
+/* Text of the most recent CUDA error the library saw, with the step that failed ("" if none).
+ * Setting TM_DEBUG_SYNC=1 in the environment makes every launch synchronise so that a
+ * failing kernel is named here (debugging only: it serialises the host and the GPU). */
+TM_API const char *tm_last_cuda_error(void);
+
+/* Number of kernels this library has launched in this process (always counted). */
+TM_API unsigned long long tm_launch_count(void);
+
 /* Synchronises `stream`, returns the first device-side error recorded since the
  * last call (TM_OK if none) and clears it. */
-tm_status tm_get_device_error(void *stream);
+TM_API tm_status tm_get_device_error(void *stream);
 
 #ifdef __cplusplus
 }

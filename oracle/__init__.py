@@ -11,8 +11,8 @@ import numpy as np
 
 import tm_synth
 from . import tokenmixer
-from .tokenmixer import (block_forward, mix, revert, rmsnorm, route, silu, softmax, sp_moe,
-                         sp_moe_dense_masked, stack_forward, sublayer, swiglu, topk)
+from .tokenmixer import (block_forward, mix, revert, rmsnorm, round_bf16, route, silu, softmax, sp_moe,
+                         sp_moe_dense_masked, stack_forward, storage_round, sublayer, swiglu, topk)
 
 
 def synth_banks(cfg, down_scale=None, cache=True):
@@ -26,7 +26,7 @@ def synth_banks(cfg, down_scale=None, cache=True):
     return lru_cache(maxsize=None)(get) if cache else get
 
 
-def run_stack(cfg, samples=None, down_scale=None, gains=None, cache=True, keep=False):
+def run_stack(cfg, samples=None, down_scale=None, gains=None, cache=True, keep=False, storage=None):
     """Oracle stack forward of a synthetic workload on the given samples (default: all)."""
     X = tm_synth.to_f64(tm_synth.make_x(cfg, samples))
-    return stack_forward(X, cfg, synth_banks(cfg, down_scale, cache), gains=gains, keep=keep)
+    return stack_forward(X, cfg, synth_banks(cfg, down_scale, cache), gains=gains, keep=keep, storage=storage)

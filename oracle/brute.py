@@ -89,8 +89,11 @@ def _ffn_row(n, bw, j, spec):
     return _swiglu_row(n, bw["w_gate"][j], bw["w_up"][j], bw["w_down"][j])
 
 
-def block(X, T, D, H, eps, spec_mix, w_mix, spec_rev, w_rev, gain_mix=None, gain_rev=None):
-    """One block on nested-list X[b][t][d]; returns X_next as nested lists."""
+def block(X, T, D, H, eps, spec_mix, w_mix, spec_rev, w_rev, gain_mix=None, gain_rev=None, rnd=None, extra=None):
+    """One block on nested-list X[b][t][d]; returns X_next as nested lists.  `rnd` (a scalar
+    rounding function) is applied to the stored X_revert and to the block output after
+    `extra` (the inter-residual term) is added."""
+    rnd = rnd or (lambda v: v)
     B = len(X)
     dh = D // H
     W = T * dh
@@ -104,30 +107,42 @@ def block(X, T, D, H, eps, spec_mix, w_mix, spec_rev, w_rev, gain_mix=None, gain
             rows.append([y[c] + row[c] for c in range(W)])
         Hn.append(rows)
     # revert: X_rev[b][t][h*dh + j] = H_next[b][h][t*dh + j]  (Eq. 13-15)
-    Xr = [[[Hn[b][d // dh][t * dh + d % dh] for d in range(D)] for t in range(T)] for b in range(B)]
+    Xr = [[[rnd(Hn[b][d // dh][t * dh + d % dh]) for d in range(D)] for t in range(T)] for b in range(B)]
     # reverting sub-layer, residual to the block input X
     out = []
     for b in range(B):
         toks = []
         for t in range(T):
             y = _ffn_row(_norm_row(Xr[b][t], eps, gain_rev), w_rev, t, spec_rev)
-            toks.append([y[d] + X[b][t][d] for d in range(D)])
+            toks.append([rnd(y[d] + X[b][t][d] + (extra[b][t][d] if extra is not None else 0.0)) for d in range(D)])
         out.append(toks)
     return out
 
 
-def stack(X, T, D, H, eps, L, gap, specs, weights):
+def stack(X, T, D, H, eps, L, gap, specs, weights, rnd=None):
     """specs[l] = (spec_mix, spec_rev), weights[l] = (w_mix, w_rev); inter-residual per the
     reading X_l += X_{l-gap} when l % gap == 0 and l < L."""
     hist = [X]
     for l in range(1, L + 1):
         (sm, sr), (wm, wr) = specs[l - 1], weights[l - 1]
-        Y = block(hist[-1], T, D, H, eps, sm, wm, sr, wr)
-        if gap > 0 and l % gap == 0 and l < L:
-            prev = hist[l - gap]
-            Y = [[[Y[b][t][d] + prev[b][t][d] for d in range(D)] for t in range(T)] for b in range(len(Y))]
+        extra = hist[l - gap] if (gap > 0 and l % gap == 0 and l < L) else None
+        Y = block(hist[-1], T, D, H, eps, sm, wm, sr, wr, rnd=rnd, extra=extra)
         hist.append(Y)
     return hist[-1]
+
+
+def round_bf16(v):
+    """Nearest-even value with 8 significant bits, by scalar arithmetic."""
+    if v == 0.0 or not math.isfinite(v):
+        return v
+    m, e = math.frexp(v)
+    q = math.ldexp(1.0, e - 8)
+    n = v / q
+    f = math.floor(n)
+    d = n - f
+    if d > 0.5 or (d == 0.5 and f % 2 == 1):
+        f += 1
+    return f * q
 
 
 def tokenize(groups, w_group, w_global):

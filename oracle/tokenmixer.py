@@ -23,7 +23,12 @@ reason in the design notes of the repository):
   * routing: softmax over all E logits, top-k by probability with ties to the
     lower expert index, gate = alpha * p (no renormalisation after top-k),
     E routed experts plus one always-on shared expert;
-  * inter-residual: after block l, X_l += X_{l-gap} when l % gap == 0 and l < L.
+  * inter-residual: after block l, X_l += X_{l-gap} when l % gap == 0 and l < L;
+  * storage (optional): a model whose dtype is bf16 (or fp32) keeps the tensors it hands
+    from one sub-layer to the next in that dtype -- X_revert, and each block output after
+    its inter-residual.  With storage="bf16" / "f32" the oracle rounds exactly those
+    tensors to nearest-even in that format; every other step stays float64.  Routing
+    decisions in deeper layers then see the same stored inputs the model defines.
 """
 from __future__ import annotations
 
@@ -156,6 +161,26 @@ def sp_moe_dense_masked(n: np.ndarray, bw: Weights, k: int, alpha: float) -> np.
     return out
 
 
+# ------------------------------------------------------------------ storage rounding
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Nearest-even bf16 value (8 significant bits) of each float64, computed in float64."""
+    m, e = np.frexp(x)                     # x = m * 2**e, 0.5 <= |m| < 1
+    q = np.ldexp(1.0, e - 8)               # spacing of 8-significant-bit values at |x|
+    r = np.round(x / q) * q                # np.round: half to even
+    return np.where(x == 0, x, r)
+
+
+def storage_round(storage):
+    """Rounding applied to the tensors a model of this dtype stores between sub-layers."""
+    if storage in (None, "f64"):
+        return lambda a: a
+    if storage == "bf16":
+        return round_bf16
+    if storage == "f32":
+        return lambda a: a.astype(np.float32).astype(np.float64)
+    raise ValueError(storage)
+
+
 # ------------------------------------------------------------------ sub-layer / block / stack
 def sublayer(rows: np.ndarray, bank_w: Callable[[int], Weights], spec, eps: float,
              gain: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
@@ -186,35 +211,39 @@ def sublayer(rows: np.ndarray, bank_w: Callable[[int], Weights], spec, eps: floa
 
 
 def block_forward(X: np.ndarray, cfg, layer: int, bank_w: Callable[[int, int, int], Weights],
-                  gains=(None, None)) -> Dict[str, np.ndarray]:
+                  gains=(None, None), extra: Optional[np.ndarray] = None, storage=None) -> Dict[str, np.ndarray]:
     """One TokenMixer-Large block on X [R, T, D].  [readme] block diagram; [digest] Eq. 9-16.
 
         H      = Mix(X)
         H_next = FFN_mix(Norm(H)) + H
         X_rev  = Revert(H_next)
-        X_next = FFN_rev(Norm(X_rev)) + X      (residual to the block input)
+        X_next = FFN_rev(Norm(X_rev)) + X  (+ extra)   (residual to the block input; extra is
+                                                         the inter-residual term of the stack)
+    X_rev and X_next are the stored tensors that `storage` rounds.
     """
+    rnd = storage_round(storage)
     Hm = mix(X, cfg.H)
     s_mix = sublayer(Hm, lambda j: bank_w(layer, 0, j), cfg.mix, cfg.eps, gains[0])
     Hn = s_mix["out"] + Hm
-    Xr = revert(Hn, cfg.T)
+    Xr = rnd(revert(Hn, cfg.T))
     s_rev = sublayer(Xr, lambda j: bank_w(layer, 1, j), cfg.rev, cfg.eps, gains[1])
     Xn = s_rev["out"] + X
-    return {"Hm": Hm, "Hn": Hn, "Xr": Xr, "Y": Xn, "mix": s_mix, "rev": s_rev}
+    if extra is not None:
+        Xn = Xn + extra
+    return {"Hm": Hm, "Hn": Hn, "Xr": Xr, "Y": rnd(Xn), "mix": s_mix, "rev": s_rev}
 
 
 def stack_forward(X: np.ndarray, cfg, bank_w: Callable[[int, int, int], Weights],
-                  gains: Optional[List] = None, keep: bool = False) -> Dict[str, object]:
+                  gains: Optional[List] = None, keep: bool = False, storage=None) -> Dict[str, object]:
     """L blocks with the inter-residual.  [digest] 2.3.4; [readme] "inter-residual at gap 2
     with the last layer excluded":  X_l = Block_l(X_{l-1}); X_l += X_{l-gap} when
     gap > 0, l % gap == 0 and l < L (layers counted from 1)."""
     hist = [X]
     blocks = []
     for l in range(1, cfg.L + 1):
-        b = block_forward(hist[-1], cfg, l - 1, bank_w, gains[l - 1] if gains else (None, None))
+        extra = hist[l - cfg.gap] if (cfg.gap > 0 and l % cfg.gap == 0 and l < cfg.L) else None
+        b = block_forward(hist[-1], cfg, l - 1, bank_w, gains[l - 1] if gains else (None, None), extra, storage)
         Xl = b["Y"]
-        if cfg.gap > 0 and l % cfg.gap == 0 and l < cfg.L:
-            Xl = Xl + hist[l - cfg.gap]
         hist.append(Xl)
         blocks.append(b if keep else {"mix": b["mix"], "rev": b["rev"]})
     return {"Y": hist[-1], "hist": hist, "blocks": blocks}

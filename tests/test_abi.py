@@ -1,0 +1,147 @@
+"""The C ABI on the CPU: the library loads, exports every entry point include/tm.h
+declares, its struct layouts match the C compiler's, and host-side validation and
+workspace queries answer without touching a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import tm_synth as S
+from token_sparse_moe_b200 import _abi as A
+from token_sparse_moe_b200 import api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tm.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"TM_API[^;]*?\b(tm_\w+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(A.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = A.load()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", A.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (tm_\w+)", out))
+    assert set(declared_functions()) <= exported
+    assert lib.tm_version() == 100
+
+
+def test_struct_layout_matches_c(tmp_path):
+    src = tmp_path / "layout.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <stddef.h>
+#include "tm.h"
+#define P(T, f) printf(#T "." #f " %zu\n", offsetof(T, f));
+int main(void) {
+  printf("tm_shape %zu\ntm_swiglu_w %zu\ntm_moe_w %zu\ntm_sublayer %zu\ntm_block %zu\n",
+         sizeof(tm_shape), sizeof(tm_swiglu_w), sizeof(tm_moe_w), sizeof(tm_sublayer), sizeof(tm_block));
+  P(tm_shape, eps) P(tm_swiglu_w, w_gate) P(tm_swiglu_w, w_down) P(tm_moe_w, alpha) P(tm_moe_w, w_router)
+  P(tm_moe_w, ws_down) P(tm_sublayer, dense) P(tm_sublayer, moe) P(tm_block, rev)
+  return 0;
+}
+''')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = dict(l.split() for l in subprocess.run([str(exe)], capture_output=True, text=True).stdout.splitlines())
+    want = {
+        "tm_shape": ctypes.sizeof(A.tm_shape), "tm_swiglu_w": ctypes.sizeof(A.tm_swiglu_w),
+        "tm_moe_w": ctypes.sizeof(A.tm_moe_w), "tm_sublayer": ctypes.sizeof(A.tm_sublayer),
+        "tm_block": ctypes.sizeof(A.tm_block),
+        "tm_shape.eps": A.tm_shape.eps.offset, "tm_swiglu_w.w_gate": A.tm_swiglu_w.w_gate.offset,
+        "tm_swiglu_w.w_down": A.tm_swiglu_w.w_down.offset, "tm_moe_w.alpha": A.tm_moe_w.alpha.offset,
+        "tm_moe_w.w_router": A.tm_moe_w.w_router.offset, "tm_moe_w.ws_down": A.tm_moe_w.ws_down.offset,
+        "tm_sublayer.dense": A.tm_sublayer.dense.offset, "tm_sublayer.moe": A.tm_sublayer.moe.offset,
+        "tm_block.rev": A.tm_block.rev.offset,
+    }
+    assert {k: int(v) for k, v in got.items()} == want
+
+
+def test_status_strings():
+    lib = A.load()
+    assert lib.tm_status_string(0) == b"ok"
+    assert lib.tm_status_string(3) == b"workspace missing or too small"
+
+
+class _FakeTensor:
+    """Stands in for a device tensor in host-only calls: only its address is passed."""
+
+    def __init__(self, addr=0x10000):
+        self.addr = addr
+
+    def data_ptr(self):
+        return self.addr
+
+
+def _fake_sub(cfg, sub):
+    spec = cfg.ffn(sub)
+    names = (["w_router", "we_gate", "we_up", "we_down", "ws_gate", "ws_up", "ws_down"] if spec.is_moe
+             else ["w_gate", "w_up", "w_down"])
+    t = {n: _FakeTensor(0x100000 * (i + 1)) for i, n in enumerate(names)}
+    if spec.is_moe:
+        return api.SubLayer(True, cfg.banks(sub), cfg.width(sub), t, E=spec.E, k=spec.k, hidden_e=spec.hidden_e,
+                            hidden_s=spec.hidden_s, alpha=spec.alpha)
+    return api.SubLayer(False, cfg.banks(sub), cfg.width(sub), t, hidden=spec.hidden)
+
+
+@pytest.mark.parametrize("name", S.CONFIG_ORDER)
+def test_workspace_queries(name):
+    cfg = S.CONFIGS[name]
+    sh = api.config_shape(cfg)
+    blocks = [api.Block(_fake_sub(cfg, 0), _fake_sub(cfg, 1)) for _ in range(cfg.L)]
+    n = api.workspace_bytes(sh, blocks, cfg.gap)
+    tok = cfg.B * cfg.T * cfg.D * (2 if cfg.dtype == "bf16" else 4)
+    assert n > tok
+    m = api.sublayer_workspace_bytes(sh, A.TM_LAYOUT_MIXED, blocks[0].mix)
+    r = api.sublayer_workspace_bytes(sh, A.TM_LAYOUT_ROWS, blocks[0].rev)
+    assert n >= max(m, r) + tok
+    if cfg.mix.is_moe:
+        w = blocks[0].mix.moe_c()
+        assert A.load().tm_route_workspace_bytes(ctypes.byref(sh), A.TM_LAYOUT_MIXED, ctypes.byref(w)) > 0
+
+
+def test_host_validation_rejects_before_launch():
+    lib = A.load()
+    cfg = S.CONFIGS["dense_block_bf16"]
+    sub = _fake_sub(cfg, 0)
+    w = sub.dense_c()
+    good = api.config_shape(cfg)
+    bad = api.shape(cfg.B, cfg.T, 250, cfg.H, "bf16")          # D % H != 0
+    x, y, ws = ctypes.c_void_p(0x200000), ctypes.c_void_p(0x400000), ctypes.c_void_p(0x800000)
+    assert lib.tm_pertoken_swiglu(x, None, A.TM_LAYOUT_MIXED, ctypes.byref(bad), None, ctypes.byref(w), y, ws, 1 << 30,
+                                  None) == A.TM_ERR_INVALID_ARG
+    # workspace too small
+    assert lib.tm_pertoken_swiglu(x, None, A.TM_LAYOUT_MIXED, ctypes.byref(good), None, ctypes.byref(w), y, ws, 16,
+                                  None) == A.TM_ERR_WORKSPACE
+    # misaligned output
+    assert lib.tm_pertoken_swiglu(x, None, A.TM_LAYOUT_MIXED, ctypes.byref(good), None, ctypes.byref(w),
+                                  ctypes.c_void_p(0x400002), ws, 1 << 30, None) == A.TM_ERR_INVALID_ARG
+    # mixed layout needs banks == H
+    w2 = A.tm_swiglu_w(cfg.H + 1, cfg.W, 1024, 0x100000, 0x200000, 0x300000)
+    assert lib.tm_pertoken_swiglu(x, None, A.TM_LAYOUT_MIXED, ctypes.byref(good), None, ctypes.byref(w2), y, ws,
+                                  1 << 30, None) == A.TM_ERR_INVALID_ARG
+    # hidden not a multiple of the 64-wide K slab
+    w3 = A.tm_swiglu_w(cfg.H, cfg.W, 1000, 0x100000, 0x200000, 0x300000)
+    assert lib.tm_pertoken_swiglu(x, None, A.TM_LAYOUT_MIXED, ctypes.byref(good), None, ctypes.byref(w3), y, ws,
+                                  1 << 30, None) == A.TM_ERR_UNSUPPORTED
+    # MoE: k > E
+    mcfg = S.CONFIGS["moe_stack_bf16"]
+    msub = _fake_sub(mcfg, 0)
+    mw = msub.moe_c()
+    mw.k = 9
+    msh = api.config_shape(mcfg)
+    assert lib.tm_sparse_pertoken_moe(x, None, A.TM_LAYOUT_MIXED, ctypes.byref(msh), None, ctypes.byref(mw), y, ws,
+                                      1 << 30, None) == A.TM_ERR_INVALID_ARG
+    # stack: bad gap / L
+    blocks = (A.tm_block * 1)(api.Block(sub, _fake_sub(cfg, 1)).c())
+    assert lib.tm_stack_forward(x, blocks, 0, 0, ctypes.byref(good), y, ws, 1 << 30, None) == A.TM_ERR_INVALID_ARG
+    assert lib.tm_stack_forward(x, blocks, 1, 0, ctypes.byref(good), x, ws, 1 << 30, None) == A.TM_ERR_INVALID_ARG

@@ -1,0 +1,270 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle, element by
+element on the same seeded inputs.
+
+Small cases span several 128-row tiles with a ragged tail and every kernel path
+(TMA Mix map, 3-D row map, cp.async gather, each output tile width, fp32 CUDA-core
+path).  The full-size workloads run the whole batch on the GPU and compare a
+deterministic sample subset (first and last sample included) with the oracle;
+samples are independent, so the subset's rows are exact oracle outputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tm_synth as S
+from oracle import tokenmixer as O
+from tm_synth import FFNSpec
+from token_sparse_moe_b200 import TMError, api
+from token_sparse_moe_b200 import _abi as A
+
+from parity_util import (BF16_TOL, F32_TOL, GAP_TOL, check_buckets, check_routing, check_stack, err, err_bf16,
+                         err_delta, err_f32, err_moe_delta, oracle_sublayer, rms, routed_abs_contrib, to_np, tol)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def small(name, B, T, D, H, dtype, mix, rev, L=1, gap=0):
+    return S.Config(name, B=B, T=T, D=D, H=H, L=L, dtype=dtype, mix=mix, rev=rev, gap=gap)
+
+
+def moe(E, k, Fe, Fs, alpha=None):
+    return FFNSpec("moe", E=E, k=k, hidden_e=Fe, hidden_s=Fs, alpha=float(E) / k if alpha is None else alpha)
+
+
+DENSE_SMALL = [
+    # dh = 16: Mix read through the 4-D tensor map; rows through the 3-D map; 300 rows = 2 full tiles + 44
+    small("dense_sq", 300, 16, 256, 16, "bf16", FFNSpec("dense", hidden=384), FFNSpec("dense", hidden=256)),
+    # dh = 48: three 16-column Mix boxes per head; hidden 192/320 -> 64-wide hidden tiles; rev width 384 -> 192-wide
+    small("dense_ns", 200, 16, 384, 8, "bf16", FFNSpec("dense", hidden=192), FFNSpec("dense", hidden=320)),
+    # fp32 CUDA-core path
+    small("dense_f32", 150, 8, 64, 8, "f32", FFNSpec("dense", hidden=128), FFNSpec("dense", hidden=96)),
+]
+MOE_SMALL = [
+    small("moe_sq", 300, 16, 256, 16, "bf16", moe(8, 2, 128, 128, 4.0), moe(4, 1, 64, 192, 4.0)),
+    small("moe_ns", 260, 8, 384, 4, "bf16", moe(16, 4, 128, 256), moe(6, 3, 64, 64)),
+    small("moe_f32", 150, 8, 64, 8, "f32", moe(4, 2, 64, 32), moe(8, 3, 32, 64)),
+]
+
+
+def dev(arr):
+    return api.to_device(arr, DEV)
+
+
+def inputs(cfg):
+    X = S.make_x(cfg)
+    R = S.make_x(cfg.with_(seed=cfg.seed + 17))
+    return X, R
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("T,D,H", [(16, 256, 16), (16, 384, 8), (8, 64, 8), (32, 512, 32), (48, 768, 48), (5, 40, 10)])
+def test_mix_revert_bit_exact(dtype, T, D, H):
+    cfg = small("m", 37, T, D, H, dtype, FFNSpec("dense", hidden=64), FFNSpec("dense", hidden=64))
+    X = S.make_x(cfg)
+    Hm = api.mix(dev(X), H)
+    ref = O.mix(S.to_f64(X), H)
+    assert np.array_equal(to_np(Hm), ref)
+    back = api.revert(Hm, T)
+    assert np.array_equal(to_np(back), S.to_f64(X))
+
+
+def check_outputs(cfg, y, o, x, down_scale):
+    """Small-init workloads: the stated measure (fp32: max relative error, bf16: max abs / rms).
+    Down weights at std x 1 (the FFN term is as large as the residual, so outputs cancel to
+    near zero in places and reach |y| ~ 8 in others): the FFN's own error beyond one ulp of
+    the stored output, relative to rms(o - x), at the dtype's tolerance."""
+    if down_scale is None:
+        assert err(cfg.dtype, y, o) <= tol(cfg.dtype), err(cfg.dtype, y, o)
+    else:
+        assert err_delta(y, o, x, cfg.dtype) <= tol(cfg.dtype), err_delta(y, o, x, cfg.dtype)
+
+
+def _run_sub(cfg, sub, X, R, down_scale=None, with_gain=False):
+    sw = api.sublayer_from_synth(cfg, 0, sub, DEV, down_scale, with_gain)
+    sh = api.config_shape(cfg)
+    layout = A.TM_LAYOUT_MIXED if sub == 0 else A.TM_LAYOUT_ROWS
+    fn = api.sparse_pertoken_moe if sw.is_moe else api.pertoken_swiglu
+    y = fn(dev(X), dev(R), layout, sh, sw)
+    api.get_device_error()
+    return to_np(y), sw
+
+
+def _oracle_sub(cfg, sub, X, R, down_scale=None, with_gain=False):
+    X64, R64 = S.to_f64(X), S.to_f64(R)
+    g = S.to_f64(S.gain(cfg, 0, sub)) if with_gain else None
+    if sub == 0:
+        rows = O.mix(X64, cfg.H)
+        r = oracle_sublayer(cfg, 0, 0, rows, down_scale, g)
+        return O.revert(r["out"] + O.mix(R64, cfg.H), cfg.T), r, rows
+    r = oracle_sublayer(cfg, 0, 1, X64, down_scale, g)
+    return r["out"] + R64, r, X64
+
+
+@pytest.mark.parametrize("down_scale", [None, 1.0])
+@pytest.mark.parametrize("sub", [0, 1])
+@pytest.mark.parametrize("cfg", DENSE_SMALL, ids=lambda c: c.name)
+def test_dense_sublayer(cfg, sub, down_scale):
+    X, R = inputs(cfg)
+    y, _ = _run_sub(cfg, sub, X, R, down_scale)
+    o, _, _ = _oracle_sub(cfg, sub, X, R, down_scale)
+    R64 = S.to_f64(R)
+    check_outputs(cfg, y, o, R64, down_scale)
+
+
+@pytest.mark.parametrize("sub", [0, 1])
+@pytest.mark.parametrize("cfg", MOE_SMALL, ids=lambda c: c.name)
+def test_route_topk(cfg, sub):
+    X, _ = inputs(cfg)
+    sw = api.sublayer_from_synth(cfg, 0, sub, DEV)
+    layout = A.TM_LAYOUT_MIXED if sub == 0 else A.TM_LAYOUT_ROWS
+    r = api.route_topk(dev(X), layout, api.config_shape(cfg), sw)
+    api.get_device_error()
+    X64 = S.to_f64(X)
+    rows = O.mix(X64, cfg.H) if sub == 0 else X64
+    info = oracle_sublayer(cfg, 0, sub, rows)
+    spec = cfg.ffn(sub)
+    idx = r["idx"].cpu().numpy()
+    bad, near = check_routing(idx, r["gate"].cpu().numpy(), info, spec.alpha, spec.E)
+    assert bad == 0, f"{bad} rows routed differently outside near ties ({near} near-tie rows)"
+    inv = 1.0 / np.sqrt(np.mean(rows * rows, axis=-1) + cfg.eps)
+    assert np.allclose(r["inv_rms"].cpu().numpy(), inv, rtol=1e-5)
+    check_buckets(idx, r["offsets"].cpu().numpy(), r["rows"].cpu().numpy(), r["slot_of"].cpu().numpy(), spec.E)
+
+
+@pytest.mark.parametrize("down_scale", [None, 1.0])
+@pytest.mark.parametrize("sub", [0, 1])
+@pytest.mark.parametrize("cfg", MOE_SMALL, ids=lambda c: c.name)
+def test_moe_sublayer(cfg, sub, down_scale):
+    X, R = inputs(cfg)
+    y, sw = _run_sub(cfg, sub, X, R, down_scale)
+    o, info, rows = _oracle_sub(cfg, sub, X, R, down_scale)
+    layout = A.TM_LAYOUT_MIXED if sub == 0 else A.TM_LAYOUT_ROWS
+    gi = api.route_topk(dev(X), layout, api.config_shape(cfg), sw)["idx"].cpu().numpy()
+    flip = np.any(np.sort(gi, -1) != np.sort(info["idx"], -1), axis=-1)            # [B, banks]
+    assert np.all(info["gap"][flip] < GAP_TOL), "routing differs outside a near tie"
+    if down_scale is None:
+        assert err(cfg.dtype, y, o) <= tol(cfg.dtype), err(cfg.dtype, y, o)
+        return
+    # FFN term as large as the residual: per element, the FFN's error beyond the output's own
+    # ulp and the bf16 rounding of the routed expert rows must stay within tol * rms(o - x).
+    # Samples where a near tie flipped an expert carry a different (valid) expert: left out.
+    keep = ~np.any(flip, axis=1)
+    c = routed_abs_contrib(cfg, 0, sub, rows, down_scale)
+    if sub == 0:
+        c = O.revert(c, cfg.T)
+    R64 = S.to_f64(R)
+    e = err_moe_delta(y[keep], o[keep], R64[keep], c[keep], cfg.dtype)
+    assert e <= tol(cfg.dtype), e
+
+
+@pytest.mark.parametrize("cfg", [DENSE_SMALL[0], MOE_SMALL[0], DENSE_SMALL[2]], ids=lambda c: c.name)
+def test_norm_gain(cfg):
+    X, R = inputs(cfg)
+    for sub in (0, 1):
+        y, _ = _run_sub(cfg, sub, X, R, 1.0, with_gain=True)
+        o, _, rows = _oracle_sub(cfg, sub, X, R, 1.0, with_gain=True)
+        if cfg.ffn(sub).is_moe:
+            # the gain is folded into the bf16 gate and up weights: two more roundings of at
+            # most 2^-8 each on every expert's output, routed and shared, on top of the slot one
+            g = S.to_f64(S.gain(cfg, 0, sub))
+            c = routed_abs_contrib(cfg, 0, sub, rows, 1.0, g)
+            call = routed_abs_contrib(cfg, 0, sub, rows, 1.0, g, include_shared=True)
+            if sub == 0:
+                c, call = O.revert(c, cfg.T), O.revert(call, cfg.T)
+            e = err_moe_delta(y, o, S.to_f64(R), c, cfg.dtype, extra=2 * 2.0 ** -8 * call)
+            assert e <= tol(cfg.dtype), e
+        else:
+            check_outputs(cfg, y, o, S.to_f64(R), 1.0)
+
+
+def _stack_gpu(cfg, down_scale=None, samples=None):
+    blocks = api.blocks_from_synth(cfg, DEV, down_scale)
+    sh = api.config_shape(cfg)
+    X = S.make_x(cfg)
+    Y = api.stack_forward(dev(X), blocks, cfg.gap, sh)
+    api.get_device_error()
+    Y = to_np(Y)
+    return Y if samples is None else Y[samples]
+
+
+@pytest.mark.parametrize("cfg", [
+    small("stack_moe", 200, 16, 256, 16, "bf16", moe(8, 2, 128, 128), moe(8, 2, 128, 128), L=4, gap=2),
+    small("stack_dense", 200, 16, 256, 16, "bf16", FFNSpec("dense", hidden=256), FFNSpec("dense", hidden=256), L=5, gap=2),
+    small("stack_f32_moe", 130, 8, 64, 8, "f32", moe(4, 2, 64, 64), moe(4, 1, 32, 32), L=3, gap=2),
+], ids=lambda c: c.name)
+def test_small_stack_with_inter_residual(cfg):
+    y = _stack_gpu(cfg)
+    check_stack(cfg, y)
+
+
+def test_fp32_stack_tiny_config_full():
+    cfg = S.CONFIGS["tiny_f32_dense"]
+    y = _stack_gpu(cfg)
+    _, _, o = check_stack(cfg, y)
+    assert err_f32(y, o) <= F32_TOL
+    assert err_delta(y, o, S.to_f64(S.make_x(cfg)), "f32") <= 1e-3
+
+
+@pytest.mark.parametrize("name,n", [("dense_block_bf16", 256), ("nonsquare_dense_bf16", 128), ("moe_stack_bf16", 48)])
+def test_full_size_config(name, n):
+    cfg = S.CONFIGS[name]
+    samples = S.subsample(cfg.B, n)
+    y = _stack_gpu(cfg, samples=samples)
+    check_stack(cfg, y, samples)
+
+
+def test_block_forward_matches_stack_and_returns_revert():
+    cfg = DENSE_SMALL[0]
+    X, _ = inputs(cfg)
+    blocks = api.blocks_from_synth(cfg, DEV)
+    sh = api.config_shape(cfg)
+    Xd = dev(X)
+    Xr = torch.empty_like(Xd)
+    Y = api.block_forward(Xd, blocks[0], sh, X_revert=Xr)
+    api.get_device_error()
+    b = O.block_forward(S.to_f64(X), cfg, 0, oracle.synth_banks(cfg), storage="bf16")
+    assert err_bf16(to_np(Y), b["Y"]) <= BF16_TOL
+    assert err_bf16(to_np(Xr), b["Xr"]) <= BF16_TOL
+    assert np.array_equal(to_np(api.stack_forward(Xd, blocks, 0, sh)), to_np(Y))
+
+
+def test_deterministic_bits():
+    cfg = MOE_SMALL[0].with_(L=2, gap=2)
+    blocks = api.blocks_from_synth(cfg, DEV)
+    sh = api.config_shape(cfg)
+    X = dev(S.make_x(cfg))
+    run = api.StackRunner(blocks, sh, cfg.gap, DEV)
+    Y1 = run(X, torch.empty_like(X)).clone()
+    Y2 = run(X, torch.empty_like(X))
+    torch.cuda.synchronize()
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+
+
+def test_tokenize_stub():
+    rng = np.random.default_rng(3)
+    B, G, dg, D = 33, 5, 24, 64
+    g = rng.standard_normal((B, G, dg)).astype(np.float32)
+    wg = rng.standard_normal((G, D, dg)).astype(np.float32)
+    wG = rng.standard_normal((D, G * dg)).astype(np.float32)
+    X = api.tokenize_stub(dev(g), dev(wg), dev(wG), D, 8)
+    ref = O.tokenize(g.astype(np.float64), wg.astype(np.float64), wG.astype(np.float64))
+    assert err_f32(to_np(X), ref) <= F32_TOL
+
+
+def test_workspace_too_small_is_reported():
+    cfg = DENSE_SMALL[0]
+    X, R = inputs(cfg)
+    sw = api.sublayer_from_synth(cfg, 0, 0, DEV)
+    small_ws = torch.empty(1024, dtype=torch.uint8, device=DEV)
+    with pytest.raises(TMError) as e:
+        lib = api.lib()
+        import ctypes
+        sh = api.config_shape(cfg)
+        w = sw.dense_c()
+        y = torch.empty((cfg.B, cfg.T, cfg.D), dtype=torch.bfloat16, device=DEV)
+        A.check(lib.tm_pertoken_swiglu(api._p(dev(X)), None, A.TM_LAYOUT_MIXED, ctypes.byref(sh), None,
+                                       ctypes.byref(w), api._p(y), api._p(small_ws), 1024, api._s(None)), "call")
+    assert e.value.status == A.TM_ERR_WORKSPACE
+    api.get_device_error()

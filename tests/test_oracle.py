@@ -351,3 +351,42 @@ def test_tokenize_matches_bruteforce_and_identity():
     assert np.array_equal(X[:, 1:, :], gi)
     flat = gi.reshape(2, 12)
     assert np.array_equal(X[:, 0, :], flat[:, [5, 0, 11, 6]])
+
+
+def test_round_bf16_matches_bit_rounding_and_scalar_form():
+    import tm_synth
+    rng = np.random.default_rng(30)
+    v = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-6, 6, 20000),
+                        [0.0, 1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -1.0 - 2 ** -8, 255.5, 256.5]])
+    v32 = v.astype(np.float32)                               # values exactly representable in fp32
+    bits = tm_synth.bf16_to_f32(tm_synth.bf16_bits(v32)).astype(np.float64)
+    assert np.array_equal(O.round_bf16(v32.astype(np.float64)), bits)
+    assert all(brute.round_bf16(float(x)) == float(r) for x, r in zip(v32[:500], bits[:500]))
+    assert O.round_bf16(np.array([1.0 + 2 ** -8]))[0] == 1.0                 # tie to even
+    assert O.round_bf16(np.array([1.0 + 3 * 2 ** -8]))[0] == 1.0 + 2 ** -6   # tie to even (up)
+
+
+@pytest.mark.parametrize("moe", [False, True])
+def test_stack_with_storage_rounding_matches_bruteforce(moe):
+    cfg = _tiny_cfg(2, 4, 2, moe, L=3, gap=2)
+    rng = np.random.default_rng(31)
+    w = _tiny_weights(cfg, rng, down=0.5)
+    X = O.round_bf16(rng.standard_normal((2, 2, 4)))
+    got = O.stack_forward(X, cfg, lambda l, s, j: w[(l, s, j)], storage="bf16")["Y"]
+    specs = [(cfg.mix, cfg.rev)] * 3
+    wl = [(_as_lists(cfg, w, l, 0), _as_lists(cfg, w, l, 1)) for l in range(3)]
+    ref = brute.stack(X.tolist(), 2, 4, 2, cfg.eps, 3, 2, specs, wl, rnd=brute.round_bf16)
+    assert np.allclose(got, np.array(ref), rtol=0, atol=1e-12)
+    assert np.array_equal(got, O.round_bf16(got))                           # the output is a stored tensor
+    plain = O.stack_forward(X, cfg, lambda l, s, j: w[(l, s, j)])["Y"]
+    assert 0 < np.max(np.abs(plain - got)) < 0.5                            # a rounding-size perturbation
+
+
+def test_storage_rounding_keeps_zero_down_identity():
+    cfg = _tiny_cfg(4, 8, 2, True, L=4, gap=2)
+    rng = np.random.default_rng(32)
+    w = _tiny_weights(cfg, rng, down=0.0)
+    X = O.round_bf16(rng.standard_normal((3, 4, 8)))
+    hist = O.stack_forward(X, cfg, lambda l, s, j: w[(l, s, j)], storage="bf16")["hist"]
+    for l, c in enumerate([1, 1, 2, 2, 2]):
+        assert np.array_equal(hist[l], c * X), l

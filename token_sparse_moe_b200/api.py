@@ -1,0 +1,270 @@
+"""Python binding of libtm.so with the same call names as include/tm.h.
+
+Argument marshalling only: every step of the forward runs in the library's CUDA
+kernels.  PyTorch supplies device memory (outputs and workspaces are allocated
+here, by the caller side of the C ABI) and the CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import _abi as A
+
+_DT = {torch.float32: A.TM_F32, torch.bfloat16: A.TM_BF16}
+_TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def lib():
+    return A.load()
+
+
+def shape(B: int, T: int, D: int, H: int, dtype, eps: float = 1e-6) -> A.tm_shape:
+    dt = _DT[dtype] if isinstance(dtype, torch.dtype) else (A.TM_BF16 if dtype == "bf16" else A.TM_F32)
+    return A.tm_shape(B, T, D, H, dt, eps)
+
+
+def to_device(arr: np.ndarray, device) -> torch.Tensor:
+    """Storage array from tm_synth (uint16 = bf16 bits, float32) -> device tensor of the same bits."""
+    if arr.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(arr)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(np.ascontiguousarray(arr)).to(device)
+
+
+# ------------------------------------------------------------------ weights
+@dataclass
+class SubLayer:
+    """Device weights of one sub-layer plus its C descriptor (keeps the tensors alive)."""
+    is_moe: bool
+    banks: int
+    width: int
+    tensors: Dict[str, torch.Tensor]
+    hidden: int = 0
+    E: int = 0
+    k: int = 0
+    hidden_e: int = 0
+    hidden_s: int = 0
+    alpha: float = 0.0
+    gain: Optional[torch.Tensor] = None
+
+    def moe_c(self) -> A.tm_moe_w:
+        t = self.tensors
+        return A.tm_moe_w(self.banks, self.width, self.E, self.k, self.hidden_e, self.hidden_s, self.alpha,
+                          _p(t["w_router"]), _p(t["we_gate"]), _p(t["we_up"]), _p(t["we_down"]),
+                          _p(t.get("ws_gate")), _p(t.get("ws_up")), _p(t.get("ws_down")))
+
+    def dense_c(self) -> A.tm_swiglu_w:
+        t = self.tensors
+        return A.tm_swiglu_w(self.banks, self.width, self.hidden, _p(t["w_gate"]), _p(t["w_up"]), _p(t["w_down"]))
+
+    def c(self) -> A.tm_sublayer:
+        s = A.tm_sublayer()
+        s.norm_gain = _p(self.gain)
+        s.is_moe = 1 if self.is_moe else 0
+        if self.is_moe:
+            s.moe = self.moe_c()
+        else:
+            s.dense = self.dense_c()
+        return s
+
+
+@dataclass
+class Block:
+    mix: SubLayer
+    rev: SubLayer
+
+    def c(self) -> A.tm_block:
+        return A.tm_block(self.mix.c(), self.rev.c())
+
+
+def sublayer_from_synth(cfg, layer: int, sub: int, device, down_scale=None, with_gain: bool = False) -> SubLayer:
+    import tm_synth
+    spec = cfg.ffn(sub)
+    w = tm_synth.sublayer_weights(cfg, layer, sub, down_scale)
+    t = {k: to_device(v, device) for k, v in w.items()}
+    g = to_device(tm_synth.gain(cfg, layer, sub), device) if with_gain else None
+    if spec.is_moe:
+        return SubLayer(True, cfg.banks(sub), cfg.width(sub), t, E=spec.E, k=spec.k, hidden_e=spec.hidden_e,
+                        hidden_s=spec.hidden_s, alpha=spec.alpha, gain=g)
+    return SubLayer(False, cfg.banks(sub), cfg.width(sub), t, hidden=spec.hidden, gain=g)
+
+
+def blocks_from_synth(cfg, device, down_scale=None) -> List[Block]:
+    return [Block(sublayer_from_synth(cfg, l, 0, device, down_scale), sublayer_from_synth(cfg, l, 1, device, down_scale))
+            for l in range(cfg.L)]
+
+
+def config_shape(cfg) -> A.tm_shape:
+    return shape(cfg.B, cfg.T, cfg.D, cfg.H, cfg.dtype, cfg.eps)
+
+
+# ------------------------------------------------------------------ calls
+def _ws(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
+    if workspace is not None and workspace.numel() >= nbytes:
+        return workspace
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def mix(X: torch.Tensor, H: int, stream=None) -> torch.Tensor:
+    B, T, D = X.shape
+    out = torch.empty((B, H, T * D // H), dtype=X.dtype, device=X.device)
+    sh = shape(B, T, D, H, X.dtype)
+    A.check(lib().tm_mix(_p(X), _p(out), ctypes.byref(sh), _s(stream)), "tm_mix")
+    return out
+
+
+def revert(Hm: torch.Tensor, T: int, stream=None) -> torch.Tensor:
+    B, H, W = Hm.shape
+    D = W * H // T
+    out = torch.empty((B, T, D), dtype=Hm.dtype, device=Hm.device)
+    sh = shape(B, T, D, H, Hm.dtype)
+    A.check(lib().tm_revert(_p(Hm), _p(out), ctypes.byref(sh), _s(stream)), "tm_revert")
+    return out
+
+
+def tokenize_stub(groups: torch.Tensor, w_group: torch.Tensor, w_global: torch.Tensor, D: int, H: int,
+                  stream=None) -> torch.Tensor:
+    B, G, dg = groups.shape
+    out = torch.empty((B, G + 1, D), dtype=groups.dtype, device=groups.device)
+    sh = shape(B, G + 1, D, H, groups.dtype)
+    A.check(lib().tm_tokenize_stub(_p(groups), _p(w_group), _p(w_global), dg, ctypes.byref(sh), _p(out), _s(stream)),
+            "tm_tokenize_stub")
+    return out
+
+
+def route_topk(x: torch.Tensor, layout: int, sh: A.tm_shape, sub: SubLayer, workspace=None, stream=None) -> dict:
+    w = sub.moe_c()
+    B, banks, k, E = sh.B, sub.banks, sub.k, sub.E
+    dev = x.device
+    out = {
+        "idx": torch.empty((B, banks, k), dtype=torch.int32, device=dev),
+        "gate": torch.empty((B, banks, k), dtype=torch.float32, device=dev),
+        "inv_rms": torch.empty((B, banks), dtype=torch.float32, device=dev),
+        "offsets": torch.empty(banks * E + 1, dtype=torch.int32, device=dev),
+        "rows": torch.empty(B * banks * k, dtype=torch.int32, device=dev),
+        "slot_of": torch.empty((B, banks, k), dtype=torch.int32, device=dev),
+    }
+    nb = lib().tm_route_workspace_bytes(ctypes.byref(sh), layout, ctypes.byref(w))
+    if nb == 0:
+        raise A.TMError(A.TM_ERR_INVALID_ARG, "tm_route_workspace_bytes")
+    ws = _ws(nb, dev, workspace)
+    A.check(lib().tm_route_topk(_p(x), layout, ctypes.byref(sh), _p(sub.gain), ctypes.byref(w), _p(out["idx"]),
+                                _p(out["gate"]), _p(out["inv_rms"]), _p(out["offsets"]), _p(out["rows"]),
+                                _p(out["slot_of"]), _p(ws), ws.numel(), _s(stream)), "tm_route_topk")
+    return out
+
+
+def sublayer_workspace_bytes(sh: A.tm_shape, layout: int, sub: SubLayer) -> int:
+    c = sub.c()
+    n = lib().tm_sublayer_workspace_bytes(ctypes.byref(sh), layout, ctypes.byref(c))
+    if n == 0:
+        raise A.TMError(A.TM_ERR_INVALID_ARG, "tm_sublayer_workspace_bytes")
+    return n
+
+
+def _out_like(x: torch.Tensor, layout: int, sh: A.tm_shape, sub: SubLayer) -> torch.Tensor:
+    if layout == A.TM_LAYOUT_MIXED:
+        return torch.empty((sh.B, sh.T, sh.D), dtype=x.dtype, device=x.device)
+    return torch.empty((sh.B, sub.banks, sub.width), dtype=x.dtype, device=x.device)
+
+
+def pertoken_swiglu(x, residual, layout: int, sh: A.tm_shape, sub: SubLayer, y=None, workspace=None, stream=None):
+    y = _out_like(x, layout, sh, sub) if y is None else y
+    ws = _ws(sublayer_workspace_bytes(sh, layout, sub), x.device, workspace)
+    w = sub.dense_c()
+    A.check(lib().tm_pertoken_swiglu(_p(x), _p(residual), layout, ctypes.byref(sh), _p(sub.gain), ctypes.byref(w),
+                                     _p(y), _p(ws), ws.numel(), _s(stream)), "tm_pertoken_swiglu")
+    return y
+
+
+def sparse_pertoken_moe(x, residual, layout: int, sh: A.tm_shape, sub: SubLayer, y=None, workspace=None, stream=None):
+    y = _out_like(x, layout, sh, sub) if y is None else y
+    ws = _ws(sublayer_workspace_bytes(sh, layout, sub), x.device, workspace)
+    w = sub.moe_c()
+    A.check(lib().tm_sparse_pertoken_moe(_p(x), _p(residual), layout, ctypes.byref(sh), _p(sub.gain),
+                                         ctypes.byref(w), _p(y), _p(ws), ws.numel(), _s(stream)),
+            "tm_sparse_pertoken_moe")
+    return y
+
+
+def workspace_bytes(sh: A.tm_shape, blocks: Sequence[Block], gap: int = 0) -> int:
+    arr = (A.tm_block * len(blocks))(*[b.c() for b in blocks])
+    n = lib().tm_workspace_bytes(ctypes.byref(sh), arr, len(blocks), gap)
+    if n == 0:
+        raise A.TMError(A.TM_ERR_INVALID_ARG, "tm_workspace_bytes")
+    return n
+
+
+def block_forward(X, block: Block, sh: A.tm_shape, Y=None, X_revert=None, workspace=None, stream=None):
+    Y = torch.empty_like(X) if Y is None else Y
+    c = block.c()
+    ws = _ws(workspace_bytes(sh, [block]), X.device, workspace)
+    A.check(lib().tm_block_forward(_p(X), ctypes.byref(c), ctypes.byref(sh), _p(Y), _p(X_revert), _p(ws), ws.numel(),
+                                   _s(stream)), "tm_block_forward")
+    return Y
+
+
+class StackRunner:
+    """Holds the C block array and a workspace so repeated stack forwards launch with no allocation."""
+
+    def __init__(self, blocks: Sequence[Block], sh: A.tm_shape, gap: int, device):
+        self.blocks = list(blocks)
+        self.sh = sh
+        self.gap = gap
+        self.arr = (A.tm_block * len(self.blocks))(*[b.c() for b in self.blocks])
+        self.ws = torch.empty(workspace_bytes(sh, self.blocks, gap), dtype=torch.uint8, device=device)
+
+    def __call__(self, X: torch.Tensor, Y: torch.Tensor, stream=None) -> torch.Tensor:
+        A.check(lib().tm_stack_forward(_p(X), self.arr, len(self.blocks), self.gap, ctypes.byref(self.sh), _p(Y),
+                                       _p(self.ws), self.ws.numel(), _s(stream)), "tm_stack_forward")
+        return Y
+
+
+    def run_host(self, X_host: torch.Tensor, Y_host: torch.Tensor, X_dev: torch.Tensor, Y_dev: torch.Tensor,
+                 stream=None) -> torch.Tensor:
+        """End to end on one stream: pinned host X -> device, stack forward, device -> pinned host Y."""
+        s = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(s):
+            X_dev.copy_(X_host, non_blocking=True)
+            self(X_dev, Y_dev, s)
+            Y_host.copy_(Y_dev, non_blocking=True)
+        return Y_host
+
+
+def stack_forward(X, blocks: Sequence[Block], gap: int, sh: A.tm_shape, Y=None, stream=None):
+    Y = torch.empty_like(X) if Y is None else Y
+    return StackRunner(blocks, sh, gap, X.device)(X, Y, stream)
+
+
+def profile_start() -> None:
+    A.check(lib().tm_profile_start(), "tm_profile_start")
+
+
+def profile_stop(max_entries: int = 64) -> Dict[str, dict]:
+    """Per-kernel {launches, total_ms} recorded since profile_start (CUDA events on the launch stream)."""
+    arr = (A.tm_kernel_time * max_entries)()
+    n = ctypes.c_int(0)
+    A.check(lib().tm_profile_stop(arr, max_entries, ctypes.byref(n)), "tm_profile_stop")
+    return {arr[i].name.decode(): {"launches": arr[i].launches, "total_ms": arr[i].total_ms} for i in range(n.value)}
+
+
+def launch_count() -> int:
+    return int(lib().tm_launch_count())
+
+
+def get_device_error(stream=None) -> None:
+    A.check(lib().tm_get_device_error(_s(stream)), "device")

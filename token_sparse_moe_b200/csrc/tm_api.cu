@@ -1,0 +1,687 @@
+// tm_api.cu -- host side of the C ABI declared in include/tm.h: validation, workspace
+// carving, TMA tensor maps and the launch sequence of every call.  Nothing here
+// allocates device memory or synchronises (except tm_get_device_error).
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "tm.h"
+#include "tm_internal.h"
+
+namespace tml {
+namespace {
+
+// ------------------------------------------------------------------ small utilities
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct Carve {
+    uint8_t* base;
+    size_t off = 0;
+    template <class T>
+    T* take(size_t n) {
+        off = align256(off);
+        T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+        off += n * sizeof(T);
+        return p;
+    }
+};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// bf16 tensor map; dims/box innermost first, strides in bytes for dims 1..r-1.  The box's
+// inner extent always equals the swizzle span (128 B with SWIZZLE_128B, 32 B with SWIZZLE_32B).
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+              const uint32_t* box, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// [rows, cols] row-major bf16 matrix, box = 64 columns x box_rows rows
+bool map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    uint64_t dims[2] = {cols, rows};
+    uint64_t strides[1] = {cols * 2};
+    uint32_t box[2] = {64, box_rows};
+    return make_map(m, base, 2, dims, strides, box);
+}
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (!cache[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+
+tm_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return TM_OK;
+    note_cuda_error("launch", e);
+    return TM_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ geometry and validation
+struct Geo {
+    int B, banks, W, dtype;
+    size_t esz;
+    float eps;
+    RowMap map;
+};
+
+tm_status check_shape(const tm_shape* s) {
+    if (!s) return TM_ERR_INVALID_ARG;
+    if (s->B <= 0 || s->T <= 0 || s->D <= 0 || s->H <= 0 || s->D % s->H != 0) return TM_ERR_INVALID_ARG;
+    if (s->dtype != TM_F32 && s->dtype != TM_BF16) return TM_ERR_INVALID_ARG;
+    if (!(s->eps >= 0.f) || !isfinite(s->eps)) return TM_ERR_INVALID_ARG;
+    return TM_OK;
+}
+
+// Geometry of a sub-layer with `banks` banks of width `width` seen through `layout`.
+tm_status make_geo(const tm_shape* s, int layout, int banks, int width, Geo* g) {
+    tm_status st = check_shape(s);
+    if (st != TM_OK) return st;
+    const int dh = s->D / s->H;
+    if (layout == TM_LAYOUT_MIXED) {
+        if (banks != s->H || width != s->T * dh) return TM_ERR_INVALID_ARG;
+    } else if (layout == TM_LAYOUT_ROWS) {
+        if (banks <= 0 || width <= 0) return TM_ERR_INVALID_ARG;
+    } else {
+        return TM_ERR_INVALID_ARG;
+    }
+    const int V = s->dtype == TM_BF16 ? 8 : 4;   // elements per 16-byte vector
+    if (width % V != 0) return TM_ERR_UNSUPPORTED;
+    if (layout == TM_LAYOUT_MIXED && dh % V != 0) return TM_ERR_UNSUPPORTED;
+    g->B = s->B;
+    g->banks = banks;
+    g->W = width;
+    g->dtype = s->dtype;
+    g->esz = s->dtype == TM_BF16 ? 2 : 4;
+    g->eps = s->eps;
+    g->map = RowMap{layout == TM_LAYOUT_MIXED ? 1 : 0, banks, width, s->T, s->D, dh};
+    return TM_OK;
+}
+
+// K and N granularity of the GEMMs: 64 for the tcgen05 path (64-wide K slabs), 32 for fp32.
+int gran(const Geo& g) { return g.dtype == TM_BF16 ? 64 : 32; }
+
+tm_status check_dense(const Geo& g, const tm_swiglu_w* w) {
+    if (!w || w->banks != g.banks || w->width != g.W || w->hidden <= 0) return TM_ERR_INVALID_ARG;
+    if (!w->w_gate || !w->w_up || !w->w_down) return TM_ERR_INVALID_ARG;
+    if (!al16(w->w_gate) || !al16(w->w_up) || !al16(w->w_down)) return TM_ERR_INVALID_ARG;
+    if (w->hidden % gran(g) || g.W % gran(g)) return TM_ERR_UNSUPPORTED;
+    return TM_OK;
+}
+
+tm_status check_moe(const Geo& g, const tm_moe_w* w) {
+    if (!w || w->banks != g.banks || w->width != g.W) return TM_ERR_INVALID_ARG;
+    if (w->E < 1 || w->k < 1 || w->k > w->E || w->hidden_e <= 0 || w->hidden_s < 0) return TM_ERR_INVALID_ARG;
+    if (!isfinite(w->alpha)) return TM_ERR_INVALID_ARG;
+    if (w->E > 32 || w->k > 8) return TM_ERR_UNSUPPORTED;
+    if ((size_t)w->banks * w->E > 4096) return TM_ERR_UNSUPPORTED;
+    if ((size_t)w->E * w->width * 4 > 200 * 1024) return TM_ERR_UNSUPPORTED;   // router weights staged in smem
+    if (!w->w_router || !w->we_gate || !w->we_up || !w->we_down) return TM_ERR_INVALID_ARG;
+    if (!al16(w->w_router) || !al16(w->we_gate) || !al16(w->we_up) || !al16(w->we_down)) return TM_ERR_INVALID_ARG;
+    if (w->hidden_s > 0) {
+        if (!w->ws_gate || !w->ws_up || !w->ws_down) return TM_ERR_INVALID_ARG;
+        if (!al16(w->ws_gate) || !al16(w->ws_up) || !al16(w->ws_down)) return TM_ERR_INVALID_ARG;
+        if (w->hidden_s % gran(g)) return TM_ERR_UNSUPPORTED;
+    }
+    if (w->hidden_e % gran(g) || g.W % gran(g)) return TM_ERR_UNSUPPORTED;
+    return TM_OK;
+}
+
+// ------------------------------------------------------------------ GEMM helpers
+int pick_bn_swiglu(int F) { return F % 128 == 0 ? 256 : 128; }
+int pick_bn_out(int W) { return W % 256 == 0 ? 256 : (W % 192 == 0 ? 192 : 128); }
+
+// The A operand of GEMM1 read straight from x: a 3-D map over [B, banks, W] rows, or the 4-D Mix
+// map (j16, q, t, b) over the token tensor, q = the 16-column piece of a token (head h owns
+// q = h*dh/16 .. h*dh/16 + dh/16 - 1), when the head width is a multiple of 16.
+int gemm1_amode(const Geo& g) {
+    if (g.map.layout == 0) return A_TMA_3D;
+    return (g.map.dh % 16 == 0) ? A_TMA_MIX : A_GATHER;
+}
+bool gemm1_amap(const Geo& g, const void* x, int amode, CUtensorMap* m) {
+    if (amode == A_TMA_3D) {
+        uint64_t dims[3] = {(uint64_t)g.W, (uint64_t)g.banks, (uint64_t)g.B};
+        uint64_t strides[2] = {(uint64_t)g.W * 2, (uint64_t)g.banks * g.W * 2};
+        uint32_t box[3] = {64, 1, 128};
+        return make_map(m, x, 3, dims, strides, box);
+    }
+    if (amode == A_TMA_MIX) {
+        const RowMap& r = g.map;
+        uint64_t dims[4] = {16, (uint64_t)r.D / 16, (uint64_t)r.T, (uint64_t)g.B};
+        uint64_t strides[3] = {32, (uint64_t)r.D * 2, (uint64_t)r.T * r.D * 2};
+        uint32_t box[4] = {16, 1, 1, 128};
+        return make_map(m, x, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B);
+    }
+    memset(m, 0, sizeof(*m));
+    return true;
+}
+
+GemmParams base_params(const Geo& g) {
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.banks = g.banks;
+    p.rows = g.B;
+    p.groups = g.banks;
+    p.E = 1;
+    p.amap = g.map;
+    p.omap = g.map;
+    p.pos_limit = g.B * g.banks;
+    return p;
+}
+
+int dense_grid(const GemmParams& p) {
+    const long tiles = (long)p.groups * ((p.rows + 127) / 128) * p.n_tiles;
+    return (int)(tiles < num_sms() ? tiles : num_sms());
+}
+
+// SwiGLU GEMM1 over x (dense groups = banks, rows = B): hidden [banks*B, F]
+tm_status gemm1_dense(const Geo& g, const void* x, const void* wg, const void* wu, int F, const float* inv_rms,
+                      void* hidden, cudaStream_t st) {
+    GemmParams p = base_params(g);
+    p.sched = 0;
+    p.K = g.W;
+    p.N = 2 * F;
+    p.inv_rms = inv_rms;
+    p.out = (__nv_bfloat16*)hidden;
+    p.out_ld = F;
+    p.out_elems = (size_t)g.banks * g.B * F;
+    p.a_ptr = (const __nv_bfloat16*)x;
+    if (g.dtype == TM_F32) {
+        p.n_tiles = F / 32;
+        SimtGemmArgs a{p, (const float*)x, (const float*)wg, (const float*)wu};
+        return cuda_status(launch_simt_gemm(EPI_SWIGLU, a, p.groups * ((p.rows + 127) / 128) * p.n_tiles, st));
+    }
+    const int bn = pick_bn_swiglu(F);
+    p.n_tiles = p.N / bn;
+    const int am = gemm1_amode(g);
+    CUtensorMap ma, mg, mu;
+    if (!gemm1_amap(g, x, am, &ma)) return TM_ERR_CUDA;
+    if (!map_2d(&mg, wg, (uint64_t)g.banks * F, g.W, bn / 2) || !map_2d(&mu, wu, (uint64_t)g.banks * F, g.W, bn / 2))
+        return TM_ERR_CUDA;
+    return cuda_status(launch_grouped_gemm(bn, am, EPI_SWIGLU, ma, mg, mu, p, dense_grid(p), st));
+}
+
+// GEMM2 over dense hidden rows [banks*B, F] with the residual / combine epilogue into y (omap).
+tm_status gemm2_dense(const Geo& g, const void* hidden, const void* wd, int F, int epi, const void* resid,
+                      const void* extra, void* y, const float* gate, const int* slot_of, const void* slots, int k,
+                      cudaStream_t st) {
+    GemmParams p = base_params(g);
+    p.sched = 0;
+    p.K = F;
+    p.N = g.W;
+    p.out = (__nv_bfloat16*)y;
+    p.out_elems = (size_t)g.B * g.banks * g.W;
+    p.resid = (const __nv_bfloat16*)resid;
+    p.extra = (const __nv_bfloat16*)extra;
+    p.gate = gate;
+    p.slot_of = slot_of;
+    p.slots = (const __nv_bfloat16*)slots;
+    p.k = k;
+    if (epi == EPI_COMBINE) p.pos_limit = g.B * g.banks * k;   // slot rows
+    if (g.dtype == TM_F32) {
+        p.n_tiles = g.W / 32;
+        SimtGemmArgs a{p, (const float*)hidden, (const float*)wd, nullptr};
+        return cuda_status(launch_simt_gemm(epi, a, p.groups * ((p.rows + 127) / 128) * p.n_tiles, st));
+    }
+    const int bn = pick_bn_out(g.W);
+    p.n_tiles = g.W / bn;
+    CUtensorMap ma, mb;
+    if (!map_2d(&ma, hidden, (uint64_t)g.banks * g.B, F, 128) || !map_2d(&mb, wd, (uint64_t)g.banks * g.W, F, bn))
+        return TM_ERR_CUDA;
+    return cuda_status(launch_grouped_gemm(bn, A_TMA_2D, epi, ma, mb, mb, p, dense_grid(p), st));
+}
+
+// ------------------------------------------------------------------ dense sub-layer
+struct DenseWs {
+    float* inv_rms;
+    void* hidden;
+    void* wg;
+    void* wu;
+};
+DenseWs carve_dense(Carve& c, const Geo& g, int F, bool gain) {
+    DenseWs w;
+    w.inv_rms = c.take<float>((size_t)g.B * g.banks);
+    w.hidden = c.take<uint8_t>((size_t)g.banks * g.B * F * g.esz);
+    w.wg = gain ? c.take<uint8_t>((size_t)g.banks * F * g.W * g.esz) : nullptr;
+    w.wu = gain ? c.take<uint8_t>((size_t)g.banks * F * g.W * g.esz) : nullptr;
+    return w;
+}
+
+tm_status run_dense(const Geo& g, const void* x, const void* resid, const void* extra, const void* gain,
+                    const tm_swiglu_w* w, void* y, void* ws, size_t wsb, cudaStream_t st) {
+    Carve c{(uint8_t*)ws};
+    DenseWs d = carve_dense(c, g, w->hidden, gain != nullptr);
+    if (!ws || wsb < c.off || !al16(ws)) return TM_ERR_WORKSPACE;
+    const void* wg = w->w_gate;
+    const void* wu = w->w_up;
+    tm_status s;
+    if (gain) {
+        const size_t rows = (size_t)g.banks * w->hidden;
+        if ((s = cuda_status(launch_fold_gain(g.dtype, wg, gain, d.wg, rows, g.W, st))) != TM_OK) return s;
+        if ((s = cuda_status(launch_fold_gain(g.dtype, wu, gain, d.wu, rows, g.W, st))) != TM_OK) return s;
+        wg = d.wg;
+        wu = d.wu;
+    }
+    if ((s = cuda_status(launch_rms(g.dtype, x, g.map, g.B, g.eps, d.inv_rms, st))) != TM_OK) return s;
+    if ((s = gemm1_dense(g, x, wg, wu, w->hidden, d.inv_rms, d.hidden, st)) != TM_OK) return s;
+    return gemm2_dense(g, d.hidden, w->w_down, w->hidden, EPI_RESID, resid, extra, y, nullptr, nullptr, nullptr, 0, st);
+}
+
+// ------------------------------------------------------------------ MoE sub-layer
+struct MoeWs {
+    float* inv_rms;
+    int32_t *idx, *slot_of, *bucket_rows, *offsets, *tile_start, *counts;
+    float* gate;
+    void *hidden_r, *slots, *hidden_s;
+    void *weg, *weu, *wsg, *wsu;
+};
+MoeWs carve_moe(Carve& c, const Geo& g, const tm_moe_w* w, bool gain) {
+    MoeWs m;
+    const size_t rows = (size_t)g.B * g.banks;
+    const size_t routed = rows * w->k;
+    const int nchunks = (g.B + kRouterChunk - 1) / kRouterChunk;
+    const size_t G = (size_t)g.banks * w->E;
+    m.inv_rms = c.take<float>(rows);
+    m.idx = c.take<int32_t>(routed);
+    m.gate = c.take<float>(routed);
+    m.slot_of = c.take<int32_t>(routed);
+    m.bucket_rows = c.take<int32_t>(routed);
+    m.offsets = c.take<int32_t>(G + 1);
+    m.tile_start = c.take<int32_t>(G + 1);
+    m.counts = c.take<int32_t>((size_t)g.banks * nchunks * w->E);
+    m.hidden_r = c.take<uint8_t>(routed * w->hidden_e * g.esz);
+    m.slots = c.take<uint8_t>(routed * g.W * g.esz);
+    m.hidden_s = w->hidden_s > 0 ? c.take<uint8_t>(rows * w->hidden_s * g.esz) : nullptr;
+    m.weg = gain ? c.take<uint8_t>(G * w->hidden_e * g.W * g.esz) : nullptr;
+    m.weu = gain ? c.take<uint8_t>(G * w->hidden_e * g.W * g.esz) : nullptr;
+    m.wsg = gain && w->hidden_s ? c.take<uint8_t>((size_t)g.banks * w->hidden_s * g.W * g.esz) : nullptr;
+    m.wsu = gain && w->hidden_s ? c.take<uint8_t>((size_t)g.banks * w->hidden_s * g.W * g.esz) : nullptr;
+    return m;
+}
+
+struct RouteOut {
+    int32_t *idx, *offsets, *tile_start, *bucket_rows, *slot_of, *counts;
+    float *gate, *inv_rms;
+};
+
+tm_status run_route(const Geo& g, const void* x, const void* gain, const tm_moe_w* w, const RouteOut& r,
+                    cudaStream_t st) {
+    tm_status s;
+    if ((s = cuda_status(launch_router(g.dtype, x, g.map, g.B, g.eps, gain, w->w_router, w->E, w->k, w->alpha, r.idx,
+                                       r.gate, r.inv_rms, r.counts, st))) != TM_OK)
+        return s;
+    const int nchunks = (g.B + kRouterChunk - 1) / kRouterChunk;
+    if ((s = cuda_status(launch_offsets(r.counts, r.counts, g.banks, nchunks, w->E, r.offsets, r.tile_start, st))) !=
+        TM_OK)
+        return s;
+    return cuda_status(launch_scatter(r.idx, r.counts, r.offsets, g.B, g.banks, w->E, w->k, r.bucket_rows, r.slot_of, st));
+}
+
+tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* extra, const void* gain,
+                  const tm_moe_w* w, void* y, void* ws, size_t wsb, cudaStream_t st) {
+    Carve c{(uint8_t*)ws};
+    MoeWs m = carve_moe(c, g, w, gain != nullptr);
+    if (!ws || wsb < c.off || !al16(ws)) return TM_ERR_WORKSPACE;
+    if (w->hidden_s == 0) return TM_ERR_UNSUPPORTED;
+    const void *weg = w->we_gate, *weu = w->we_up, *wsg = w->ws_gate, *wsu = w->ws_up;
+    tm_status s;
+    const size_t G = (size_t)g.banks * w->E;
+    if (gain) {
+        if ((s = cuda_status(launch_fold_gain(g.dtype, weg, gain, m.weg, G * w->hidden_e, g.W, st))) != TM_OK) return s;
+        if ((s = cuda_status(launch_fold_gain(g.dtype, weu, gain, m.weu, G * w->hidden_e, g.W, st))) != TM_OK) return s;
+        if ((s = cuda_status(launch_fold_gain(g.dtype, wsg, gain, m.wsg, (size_t)g.banks * w->hidden_s, g.W, st))) != TM_OK)
+            return s;
+        if ((s = cuda_status(launch_fold_gain(g.dtype, wsu, gain, m.wsu, (size_t)g.banks * w->hidden_s, g.W, st))) != TM_OK)
+            return s;
+        weg = m.weg; weu = m.weu; wsg = m.wsg; wsu = m.wsu;
+    }
+    RouteOut r{m.idx, m.offsets, m.tile_start, m.bucket_rows, m.slot_of, m.counts, m.gate, m.inv_rms};
+    if ((s = run_route(g, x, gain, w, r, st)) != TM_OK) return s;
+
+    const size_t routed = (size_t)g.B * g.banks * w->k;
+    const int Fe = w->hidden_e;
+    // routed experts, GEMM1 + SwiGLU over the buckets (rows gathered through the row map)
+    GemmParams p = base_params(g);
+    p.sched = 1;
+    p.groups = (int)G;
+    p.E = w->E;
+    p.row_start = m.offsets;
+    p.tile_start = m.tile_start;
+    p.bucket_rows = m.bucket_rows;
+    p.pos_limit = (int)routed;
+    p.K = g.W;
+    p.N = 2 * Fe;
+    p.inv_rms = m.inv_rms;
+    p.out = (__nv_bfloat16*)m.hidden_r;
+    p.out_ld = Fe;
+    p.out_elems = routed * Fe;
+    p.a_ptr = (const __nv_bfloat16*)x;
+    const long max_mt = (long)(routed / 128) + (long)G;
+    if (g.dtype == TM_F32) {
+        p.n_tiles = Fe / 32;
+        SimtGemmArgs a{p, (const float*)x, (const float*)weg, (const float*)weu};
+        if ((s = cuda_status(launch_simt_gemm(EPI_SWIGLU, a, (int)(max_mt * p.n_tiles), st))) != TM_OK) return s;
+    } else {
+        const int bn = pick_bn_swiglu(Fe);
+        p.n_tiles = p.N / bn;
+        CUtensorMap none, mg, mu;
+        memset(&none, 0, sizeof(none));
+        if (!map_2d(&mg, weg, G * Fe, g.W, bn / 2) || !map_2d(&mu, weu, G * Fe, g.W, bn / 2)) return TM_ERR_CUDA;
+        const long grid = max_mt * p.n_tiles < num_sms() ? max_mt * p.n_tiles : num_sms();
+        if ((s = cuda_status(launch_grouped_gemm(bn, A_GATHER, EPI_SWIGLU, none, mg, mu, p, (int)grid, st))) != TM_OK)
+            return s;
+    }
+    // shared expert GEMM1 (dense rows)
+    if ((s = gemm1_dense(g, x, wsg, wsu, w->hidden_s, m.inv_rms, m.hidden_s, st)) != TM_OK) return s;
+    // routed experts GEMM2 -> slot rows
+    p.K = Fe;
+    p.N = g.W;
+    p.out = (__nv_bfloat16*)m.slots;
+    p.out_ld = g.W;
+    p.out_elems = routed * g.W;
+    if (g.dtype == TM_F32) {
+        p.n_tiles = g.W / 32;
+        SimtGemmArgs a{p, (const float*)m.hidden_r, (const float*)w->we_down, nullptr};
+        if ((s = cuda_status(launch_simt_gemm(EPI_SLOT, a, (int)(max_mt * p.n_tiles), st))) != TM_OK) return s;
+    } else {
+        const int bn = pick_bn_out(g.W);
+        p.n_tiles = g.W / bn;
+        CUtensorMap ma, mb;
+        if (!map_2d(&ma, m.hidden_r, routed, Fe, 128) || !map_2d(&mb, w->we_down, G * g.W, Fe, bn)) return TM_ERR_CUDA;
+        const long grid = max_mt * p.n_tiles < num_sms() ? max_mt * p.n_tiles : num_sms();
+        if ((s = cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SLOT, ma, mb, mb, p, (int)grid, st))) != TM_OK)
+            return s;
+    }
+    // shared expert GEMM2 + deterministic combine + residual(s), stored through the row map
+    return gemm2_dense(g, m.hidden_s, w->ws_down, w->hidden_s, EPI_COMBINE, resid, extra, y, m.gate, m.slot_of,
+                       m.slots, w->k, st);
+}
+
+// ------------------------------------------------------------------ sub-layer dispatch
+int sub_banks(const tm_sublayer* s) { return s->is_moe ? s->moe.banks : s->dense.banks; }
+int sub_width(const tm_sublayer* s) { return s->is_moe ? s->moe.width : s->dense.width; }
+
+tm_status check_sublayer(const tm_shape* shape, int layout, const tm_sublayer* sub, Geo* g) {
+    if (!sub) return TM_ERR_INVALID_ARG;
+    tm_status s = make_geo(shape, layout, sub_banks(sub), sub_width(sub), g);
+    if (s != TM_OK) return s;
+    if (sub->norm_gain && !al16(sub->norm_gain)) return TM_ERR_INVALID_ARG;
+    if (sub->is_moe) {
+        s = check_moe(*g, &sub->moe);
+        if (s == TM_OK && sub->moe.hidden_s == 0) s = TM_ERR_UNSUPPORTED;
+        return s;
+    }
+    return check_dense(*g, &sub->dense);
+}
+
+size_t sublayer_ws(const Geo& g, const tm_sublayer* sub) {
+    Carve c{nullptr};
+    if (sub->is_moe) carve_moe(c, g, &sub->moe, sub->norm_gain != nullptr);
+    else carve_dense(c, g, sub->dense.hidden, sub->norm_gain != nullptr);
+    return align256(c.off);
+}
+
+tm_status run_sublayer(const Geo& g, const void* x, const void* resid, const void* extra, const tm_sublayer* sub,
+                       void* y, void* ws, size_t wsb, cudaStream_t st) {
+    if (sub->is_moe) return run_moe(g, x, resid, extra, sub->norm_gain, &sub->moe, y, ws, wsb, st);
+    return run_dense(g, x, resid, extra, sub->norm_gain, &sub->dense, y, ws, wsb, st);
+}
+
+// block geometry: mixing sub-layer (MIXED, banks H) and reverting sub-layer (ROWS, banks T, width D)
+tm_status check_block(const tm_shape* s, const tm_block* b, Geo* gm, Geo* gr) {
+    if (!b) return TM_ERR_INVALID_ARG;
+    tm_status st = check_sublayer(s, TM_LAYOUT_MIXED, &b->mix, gm);
+    if (st != TM_OK) return st;
+    st = check_sublayer(s, TM_LAYOUT_ROWS, &b->rev, gr);
+    if (st != TM_OK) return st;
+    if (gr->banks != s->T || gr->W != s->D) return TM_ERR_INVALID_ARG;
+    return TM_OK;
+}
+
+size_t stack_ws(const tm_shape* s, const tm_block* blocks, int L, int gap, bool* ok) {
+    size_t sub = 0;
+    for (int l = 0; l < L; ++l) {
+        Geo gm, gr;
+        if (check_block(s, &blocks[l], &gm, &gr) != TM_OK) { *ok = false; return 0; }
+        const size_t a = sublayer_ws(gm, &blocks[l].mix), b = sublayer_ws(gr, &blocks[l].rev);
+        sub = a > sub ? a : sub;
+        sub = b > sub ? b : sub;
+    }
+    *ok = true;
+    const size_t tok = align256((size_t)s->B * s->T * s->D * (s->dtype == TM_BF16 ? 2 : 4));
+    const int ring = L > 1 ? (gap > 0 ? gap + 1 : 2) : 0;
+    return tok * (1 + ring) + sub;
+}
+
+tm_status run_block(const tm_shape* s, const tm_block* b, const void* X, const void* extra, void* Y, void* Xr,
+                    void* sub_ws, size_t sub_wsb, cudaStream_t st) {
+    Geo gm, gr;
+    tm_status r = check_block(s, b, &gm, &gr);
+    if (r != TM_OK) return r;
+    // H_next = FFN_mix(Norm(Mix(X))) + Mix(X), written through Revert straight into X_rev
+    if ((r = run_sublayer(gm, X, X, nullptr, &b->mix, Xr, sub_ws, sub_wsb, st)) != TM_OK) return r;
+    // Y = FFN_rev(Norm(X_rev)) + X (+ inter-residual)
+    return run_sublayer(gr, Xr, X, extra, &b->rev, Y, sub_ws, sub_wsb, st);
+}
+
+}  // namespace
+}  // namespace tml
+
+using namespace tml;
+
+extern "C" {
+
+const char* tm_status_string(tm_status s) {
+    switch (s) {
+        case TM_OK: return "ok";
+        case TM_ERR_INVALID_ARG: return "invalid argument";
+        case TM_ERR_UNSUPPORTED: return "unsupported configuration";
+        case TM_ERR_WORKSPACE: return "workspace missing or too small";
+        case TM_ERR_CUDA: return "CUDA error";
+        case TM_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        case TM_ERR_DEVICE_BOUNDS: return "device bounds check failed";
+    }
+    return "unknown status";
+}
+
+int tm_version(void) { return 100; }
+
+size_t tm_sublayer_workspace_bytes(const tm_shape* shape, tm_layout layout, const tm_sublayer* sub) {
+    Geo g;
+    if (check_sublayer(shape, layout, sub, &g) != TM_OK) return 0;
+    return sublayer_ws(g, sub);
+}
+
+size_t tm_route_workspace_bytes(const tm_shape* shape, tm_layout layout, const tm_moe_w* w) {
+    Geo g;
+    if (!w || make_geo(shape, layout, w->banks, w->width, &g) != TM_OK || check_moe(g, w) != TM_OK) return 0;
+    const int nchunks = (g.B + kRouterChunk - 1) / kRouterChunk;
+    return align256((size_t)g.banks * nchunks * w->E * sizeof(int32_t)) + align256(((size_t)g.banks * w->E + 1) * 4);
+}
+
+size_t tm_workspace_bytes(const tm_shape* shape, const tm_block* blocks, int L, int gap) {
+    if (!blocks || L < 1 || gap < 0) return 0;
+    bool ok = false;
+    const size_t n = stack_ws(shape, blocks, L, gap, &ok);
+    return ok ? n : 0;
+}
+
+tm_status tm_tokenize_stub(const void* groups, const void* w_group, const void* w_global, int dg,
+                           const tm_shape* shape, void* X_out, void* stream) {
+    tm_status s = check_shape(shape);
+    if (s != TM_OK) return s;
+    if (!groups || !w_global || !X_out || dg <= 0 || shape->T < 2) return TM_ERR_INVALID_ARG;
+    if (!w_group) return TM_ERR_INVALID_ARG;
+    return cuda_status(launch_tokenize(shape->dtype, groups, w_group, w_global, dg, shape->B, shape->T, shape->D, X_out,
+                                       (cudaStream_t)stream));
+}
+
+tm_status tm_mix(const void* X, void* Hm, const tm_shape* shape, void* stream) {
+    tm_status s = check_shape(shape);
+    if (s != TM_OK) return s;
+    if (!X || !Hm || X == Hm) return TM_ERR_INVALID_ARG;
+    return cuda_status(launch_permute(shape->dtype, X, Hm, shape->B, shape->T, shape->D, shape->H, true,
+                                      (cudaStream_t)stream));
+}
+
+tm_status tm_revert(const void* Hm, void* X, const tm_shape* shape, void* stream) {
+    tm_status s = check_shape(shape);
+    if (s != TM_OK) return s;
+    if (!X || !Hm || X == Hm) return TM_ERR_INVALID_ARG;
+    return cuda_status(launch_permute(shape->dtype, Hm, X, shape->B, shape->T, shape->D, shape->H, false,
+                                      (cudaStream_t)stream));
+}
+
+tm_status tm_route_topk(const void* x, tm_layout layout, const tm_shape* shape, const void* norm_gain,
+                        const tm_moe_w* w, int32_t* topk_idx, float* topk_gate, float* inv_rms,
+                        int32_t* bucket_offsets, int32_t* bucket_rows, int32_t* slot_of, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+    Geo g;
+    if (!w) return TM_ERR_INVALID_ARG;
+    tm_status s = make_geo(shape, layout, w->banks, w->width, &g);
+    if (s != TM_OK) return s;
+    if ((s = check_moe(g, w)) != TM_OK) return s;
+    if (!x || !al16(x) || !topk_idx || !topk_gate || !bucket_offsets || !bucket_rows || !slot_of)
+        return TM_ERR_INVALID_ARG;
+    if (norm_gain && !al16(norm_gain)) return TM_ERR_INVALID_ARG;
+    const size_t need = tm_route_workspace_bytes(shape, layout, w);
+    if (!workspace || workspace_bytes < need || !al16(workspace)) return TM_ERR_WORKSPACE;
+    Carve c{(uint8_t*)workspace};
+    const int nchunks = (g.B + kRouterChunk - 1) / kRouterChunk;
+    int32_t* counts = c.take<int32_t>((size_t)g.banks * nchunks * w->E);
+    int32_t* tiles = c.take<int32_t>((size_t)g.banks * w->E + 1);
+    RouteOut r{topk_idx, bucket_offsets, tiles, bucket_rows, slot_of, counts, topk_gate, inv_rms};
+    return run_route(g, x, norm_gain, w, r, (cudaStream_t)stream);
+}
+
+tm_status tm_pertoken_swiglu(const void* x, const void* residual, tm_layout layout, const tm_shape* shape,
+                             const void* norm_gain, const tm_swiglu_w* w, void* y, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    tm_sublayer sub;
+    memset(&sub, 0, sizeof(sub));
+    if (!w) return TM_ERR_INVALID_ARG;
+    sub.norm_gain = norm_gain;
+    sub.is_moe = 0;
+    sub.dense = *w;
+    Geo g;
+    tm_status s = check_sublayer(shape, layout, &sub, &g);
+    if (s != TM_OK) return s;
+    if (!x || !y || !al16(x) || !al16(y) || x == y || (residual && !al16(residual))) return TM_ERR_INVALID_ARG;
+    return run_sublayer(g, x, residual, nullptr, &sub, y, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+tm_status tm_sparse_pertoken_moe(const void* x, const void* residual, tm_layout layout, const tm_shape* shape,
+                                 const void* norm_gain, const tm_moe_w* w, void* y, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    tm_sublayer sub;
+    memset(&sub, 0, sizeof(sub));
+    if (!w) return TM_ERR_INVALID_ARG;
+    sub.norm_gain = norm_gain;
+    sub.is_moe = 1;
+    sub.moe = *w;
+    Geo g;
+    tm_status s = check_sublayer(shape, layout, &sub, &g);
+    if (s != TM_OK) return s;
+    if (!x || !y || !al16(x) || !al16(y) || x == y || (residual && !al16(residual))) return TM_ERR_INVALID_ARG;
+    return run_sublayer(g, x, residual, nullptr, &sub, y, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+tm_status tm_block_forward(const void* X, const tm_block* block, const tm_shape* shape, void* Y, void* X_revert_opt,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    bool ok = false;
+    const size_t need = block ? stack_ws(shape, block, 1, 0, &ok) : 0;
+    if (!ok) {
+        Geo a, b;
+        tm_status s = check_block(shape, block, &a, &b);
+        return s == TM_OK ? TM_ERR_INVALID_ARG : s;
+    }
+    if (!X || !Y || X == Y || !al16(X) || !al16(Y) || (X_revert_opt && !al16(X_revert_opt))) return TM_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < need || !al16(workspace)) return TM_ERR_WORKSPACE;
+    Carve c{(uint8_t*)workspace};
+    const size_t tok = (size_t)shape->B * shape->T * shape->D * (shape->dtype == TM_BF16 ? 2 : 4);
+    void* xr = c.take<uint8_t>(tok);
+    if (X_revert_opt) xr = X_revert_opt;
+    c.off = align256(c.off);
+    return run_block(shape, block, X, nullptr, Y, xr, (uint8_t*)workspace + c.off, workspace_bytes - c.off,
+                     (cudaStream_t)stream);
+}
+
+tm_status tm_stack_forward(const void* X, const tm_block* blocks, int L, int gap, const tm_shape* shape, void* Y,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    if (!blocks || L < 1 || gap < 0) return TM_ERR_INVALID_ARG;
+    bool ok = false;
+    const size_t need = stack_ws(shape, blocks, L, gap, &ok);
+    if (!ok) {
+        for (int l = 0; l < L; ++l) {
+            Geo a, b;
+            tm_status s = check_block(shape, &blocks[l], &a, &b);
+            if (s != TM_OK) return s;
+        }
+        return TM_ERR_INVALID_ARG;
+    }
+    if (!X || !Y || X == Y || !al16(X) || !al16(Y)) return TM_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < need || !al16(workspace)) return TM_ERR_WORKSPACE;
+    const size_t tok = (size_t)shape->B * shape->T * shape->D * (shape->dtype == TM_BF16 ? 2 : 4);
+    Carve c{(uint8_t*)workspace};
+    void* xr = c.take<uint8_t>(tok);
+    const int R = L > 1 ? (gap > 0 ? gap + 1 : 2) : 0;
+    void* ring[64];
+    if (R > 64) return TM_ERR_UNSUPPORTED;
+    for (int i = 0; i < R; ++i) ring[i] = c.take<uint8_t>(tok);
+    c.off = align256(c.off);
+    void* sub_ws = (uint8_t*)workspace + c.off;
+    const size_t sub_wsb = workspace_bytes - c.off;
+    cudaStream_t st = (cudaStream_t)stream;
+    // X_l for l >= 1 lives in ring[l % R] (the last one in Y); X_0 is the caller's X
+    auto xl = [&](int l) -> const void* { return l == 0 ? X : (l == L ? Y : ring[l % R]); };
+    for (int l = 1; l <= L; ++l) {
+        const void* in = xl(l - 1);
+        void* out = l == L ? Y : ring[l % R];
+        const void* extra = (gap > 0 && l % gap == 0 && l < L) ? xl(l - gap) : nullptr;
+        tm_status s = run_block(shape, &blocks[l - 1], in, extra, out, xr, sub_ws, sub_wsb, st);
+        if (s != TM_OK) return s;
+    }
+    return TM_OK;
+}
+
+tm_status tm_get_device_error(void* stream) {
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) { note_cuda_error("tm_get_device_error: stream synchronize", e); return TM_ERR_CUDA; }
+    unsigned int h[2] = {0, 0};
+    e = cudaMemcpyFromSymbol(h, g_error, sizeof(h));
+    if (e != cudaSuccess) { note_cuda_error("tm_get_device_error: read error word", e); return TM_ERR_CUDA; }
+    if (h[0] == 0) return TM_OK;
+    char where[64];
+    snprintf(where, sizeof(where), "device error %u at site 0x%x", h[0], h[1]);
+    note_cuda_error(where, cudaErrorUnknown);
+    const unsigned int z[2] = {0, 0};
+    e = cudaMemcpyToSymbol(g_error, z, sizeof(z));
+    if (e != cudaSuccess) { note_cuda_error("tm_get_device_error: clear error word", e); return TM_ERR_CUDA; }
+    return h[0] == ERR_TIMEOUT ? TM_ERR_DEVICE_TIMEOUT : TM_ERR_DEVICE_BOUNDS;
+}
+
+}  // extern "C"

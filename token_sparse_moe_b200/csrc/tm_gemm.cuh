@@ -1,0 +1,459 @@
+// tm_gemm.cuh -- the grouped bf16 GEMM on tcgen05 tensor cores that carries every
+// per-token FFN of the TokenMixer-Large forward.
+//
+// One persistent kernel shape serves four jobs, chosen at compile time:
+//   EPI_SWIGLU : hidden = silu(s * A Wg^T) * (s * A Wu^T)   (GEMM1 of a SwiGLU bank,
+//                s = per-row 1/rms, i.e. the pre-RMSNorm folded into the epilogue)
+//   EPI_RESID  : y = A Wd^T + residual (+ inter-residual), stored through the row map
+//                (for mixed rows this store IS the Revert permutation)
+//   EPI_SLOT   : slot row = A Wd^T (a routed expert's output, bf16)
+//   EPI_COMBINE: y = A Ws^T + sum_j gate_j * slot_j + residual (+ inter-residual):
+//                shared expert GEMM2 plus the MoE combine, in fixed order
+// A operand sources: a plain 2-D TMA map (hidden rows), a 3-D TMA map over
+// [B, banks, W] rows, a 4-D TMA map that reads mixed rows straight out of the token
+// tensor (Mix folded into the tensor map: each 16-column piece of a mixed row is a
+// 32-byte run of one token, fetched as a 128-row box with 32-byte swizzle), or a
+// cp.async row gather (routed rows).
+//
+// Tile: 128 rows x BN columns, K in 64-wide slabs with 128-byte swizzle.  Warp roles:
+// warp 0 TMA producer, warp 1 MMA issuer (one thread) and TMEM owner, warps 2-5
+// epilogue (TMEM lane quarter = warp % 4), warps 6-9 row gatherers (gather mode).
+// TMEM holds two accumulators so the epilogue of tile i overlaps the MMAs of i+1.
+#pragma once
+#include "tm_device.cuh"
+
+namespace tml {
+
+enum AMode : int { A_TMA_2D = 0, A_TMA_3D = 1, A_TMA_MIX = 2, A_GATHER = 3 };
+enum Epi : int { EPI_SWIGLU = 0, EPI_RESID = 1, EPI_SLOT = 2, EPI_COMBINE = 3 };
+
+// Where element c of the row (sample b, bank) of a sub-layer lives in a tensor.
+//   layout 0 (rows):  [B, banks, W]
+//   layout 1 (mixed): token tensor [B, T, D]; c = t*dh + j  ->  [b, t, bank*dh + j]
+struct RowMap {
+    int layout, banks, W, T, D, dh;
+};
+__host__ __device__ __forceinline__ size_t row_elem(const RowMap& m, int b, int bank, int c) {
+    if (m.layout == 0) return ((size_t)b * m.banks + bank) * m.W + c;
+    const int t = c / m.dh;
+    const int j = c - t * m.dh;
+    return ((size_t)b * m.T + t) * m.D + (size_t)bank * m.dh + j;
+}
+
+struct GemmParams {
+    // tile space
+    int sched;                 // 0: groups of `rows` rows (dense banks); 1: bucketed (routed experts)
+    int groups;                // number of groups (sched 1: banks * E)
+    int rows;                  // sched 0: rows per group (= B)
+    int banks;                 // sub-layer banks
+    int E;                     // sched 1: experts per bank (bank = g / E)
+    const int* row_start;      // sched 1: [groups+1] first row position of each group
+    const int* tile_start;     // sched 1: [groups+1] prefix of 128-row tiles per group
+    const int* bucket_rows;    // sched 1: sample index of each row position
+    int pos_limit;             // row positions in hidden / slot buffers (bounds check)
+    size_t out_elems;          // elements of `out` (and of resid / extra for the row-map epilogues)
+    int K, N, n_tiles;         // reduction length, output columns per group, N / BN
+    // gathered A
+    const __nv_bfloat16* a_ptr;
+    RowMap amap;
+    // epilogue
+    const float* inv_rms;      // [B * banks]
+    __nv_bfloat16* out;        // hidden / slot rows [row positions, out_ld] or y (omap)
+    int out_ld;
+    const __nv_bfloat16* resid;
+    const __nv_bfloat16* extra;
+    RowMap omap;
+    const float* gate;         // combine: [B, banks, k]
+    const int* slot_of;        // combine: [B, banks, k]
+    const __nv_bfloat16* slots;// combine: [row positions, W]
+    int k;
+};
+
+template <int BN, int AMODE>
+struct GemmCfg {
+    static constexpr int BM = 128, BK = 64;
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 192 ? 5 : 6);
+    static constexpr int NWARPS = AMODE == A_GATHER ? 10 : 6;
+    static constexpr int NTHREADS = NWARPS * 32;
+    static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+};
+
+struct TileInfo {
+    int g, m, n, row0, nrows;
+};
+
+__device__ __forceinline__ int total_tiles(const GemmParams& p) {
+    if (p.sched == 0) return p.groups * ((p.rows + 127) / 128) * p.n_tiles;
+    return __ldg(&p.tile_start[p.groups]) * p.n_tiles;
+}
+
+__device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int t) {
+    TileInfo ti;
+    const int gm = t / p.n_tiles;
+    ti.n = t - gm * p.n_tiles;
+    if (p.sched == 0) {
+        const int mt = (p.rows + 127) / 128;
+        ti.g = gm / mt;
+        ti.m = gm - ti.g * mt;
+        ti.row0 = ti.g * p.rows + ti.m * 128;
+        ti.nrows = min(128, p.rows - ti.m * 128);
+    } else {
+        int lo = 0, hi = p.groups;   // invariant: tile_start[lo] <= gm < tile_start[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(&p.tile_start[mid]) <= gm) lo = mid; else hi = mid;
+        }
+        ti.g = lo;
+        ti.m = gm - __ldg(&p.tile_start[lo]);
+        ti.row0 = __ldg(&p.row_start[lo]) + ti.m * 128;
+        ti.nrows = min(128, __ldg(&p.row_start[lo + 1]) - ti.row0);
+    }
+    return ti;
+}
+
+// Bounded wait that also gives up as soon as another role of the CTA has given up.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              unsigned where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_error(ERR_TIMEOUT, where);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+template <int BN, int AMODE, int EPI>
+__global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
+    using C = GemmCfg<BN, AMODE>;
+    constexpr int STAGES = C::STAGES;
+    const int ntile = total_tiles(p);
+    if ((int)blockIdx.x >= ntile) return;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* acc_full = empty + STAGES;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int KB = p.K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], AMODE == A_GATHER ? 1 + 128 : 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_base_smem, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_base_smem;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            if (AMODE != A_GATHER) tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB0);
+            if (EPI == EPI_SWIGLU) tma_prefetch_desc(&tmB1);
+            int s = 0;
+            uint32_t ph = 0;
+            for (int t = blockIdx.x; t < ntile; t += gridDim.x) {
+                const TileInfo ti = decode_tile(p, t);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x100)) goto producer_done;
+                    uint8_t* sa = smem + s * C::STAGE_BYTES;
+                    uint8_t* sb = sa + C::A_BYTES;
+                    mbar_arrive_expect_tx(&full[s], (AMODE == A_GATHER ? 0 : C::A_BYTES) + C::B_BYTES);
+                    if (AMODE == A_TMA_2D) {
+                        tma_load_2d(sa, &tmA, &full[s], kb * 64, ti.row0);
+                    } else if (AMODE == A_TMA_3D) {
+                        tma_load_3d(sa, &tmA, &full[s], kb * 64, ti.g, ti.m * 128);
+                    } else if (AMODE == A_TMA_MIX) {
+                        // mixed-row columns c16*16 .. +15 = token t, head piece jj of head ti.g
+                        const int per = p.amap.dh >> 4;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int c16 = kb * 4 + i;
+                            const int t = c16 / per, jj = c16 - t * per;
+                            tma_load_4d(sa + i * 4096, &tmA, &full[s], 0, ti.g * per + jj, t, ti.m * 128);
+                        }
+                    }
+                    if (EPI == EPI_SWIGLU) {
+                        const int F = p.N >> 1;
+                        const int r0 = ti.g * F + ti.n * (BN / 2);
+                        tma_load_2d(sb, &tmB0, &full[s], kb * 64, r0);
+                        tma_load_2d(sb + (BN / 2) * 128, &tmB1, &full[s], kb * 64, r0);
+                    } else {
+                        tma_load_2d(sb, &tmB0, &full[s], kb * 64, ti.g * p.N + ti.n * BN);
+                    }
+                    if (++s == STAGES) { s = 0; ph ^= 1; }
+                }
+            }
+        }
+    producer_done:;
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16(128, BN);
+            int s = 0;
+            uint32_t ph = 0;
+            int lt = 0;
+            for (int t = blockIdx.x; t < ntile; t += gridDim.x, ++lt) {
+                const int buf = lt & 1;
+                const uint32_t aph = (lt >> 1) & 1;
+                if (!wait_or_abort(&acc_empty[buf], aph ^ 1, abort_flag, 0x200)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + buf * BN;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!wait_or_abort(&full[s], ph, abort_flag, 0x201)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+                    const uint32_t sb = sa + C::A_BYTES;
+                    const uint64_t ad = umma_sdesc_sw128(sa);
+                    const uint64_t bd = umma_sdesc_sw128(sb);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        // A: one 32-byte-swizzled 4 KB sub-slab per K step (mixed rows) or the
+                        // 128-byte-swizzled 64-wide slab advanced by 32 bytes per K step
+                        const uint64_t a_k = AMODE == A_TMA_MIX ? umma_sdesc_sw32(sa + kk * 4096) : ad + 2 * kk;
+                        umma_bf16(d, a_k, bd + 2 * kk, idesc, (kb | kk) != 0);
+                    }
+                    umma_commit(&empty[s]);
+                    if (++s == STAGES) { s = 0; ph ^= 1; }
+                }
+                if (!ok) break;
+                umma_commit(&acc_full[buf]);
+            }
+            // every MMA this thread issued must be complete before TMEM is released
+            umma_commit(drain);
+            wait_or_abort(drain, 0, abort_flag, 0x202);
+        }
+    } else if (warp >= 2 && warp < 6) {
+        // ---------------------------------------------------------------- epilogue
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        int lt = 0;
+        for (int t = blockIdx.x; t < ntile; t += gridDim.x, ++lt) {
+            const TileInfo ti = decode_tile(p, t);
+            const int buf = lt & 1;
+            const uint32_t aph = (lt >> 1) & 1;
+            if (!wait_or_abort(&acc_full[buf], aph, abort_flag, 0x300)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + buf * BN;
+            bool valid = r < ti.nrows;
+            const int pos = ti.row0 + r;                      // row position (hidden / slot index)
+            int b, bank;
+            if (p.sched == 0) {
+                b = ti.m * 128 + r;
+                bank = ti.g;
+            } else {
+                b = valid ? __ldg(&p.bucket_rows[pos]) : 0;
+                bank = ti.g / p.E;
+            }
+            if (valid && (b < 0 || b >= p.rows || pos < 0 || pos >= p.pos_limit)) {
+                record_error(ERR_BOUNDS, 0x310);
+                valid = false;
+            }
+            if (valid && EPI != EPI_RESID && EPI != EPI_COMBINE &&
+                (size_t)(pos + 1) * p.out_ld > p.out_elems) {
+                record_error(ERR_BOUNDS, 0x312);
+                valid = false;
+            }
+            if (EPI == EPI_SWIGLU) {
+                const float sc = valid ? __ldg(&p.inv_rms[(size_t)b * p.banks + bank]) : 0.f;
+                __nv_bfloat16* dst = p.out + (size_t)pos * p.out_ld + ti.n * (BN / 2);
+#pragma unroll 1
+                for (int c = 0; c < BN / 2; c += 32) {
+                    float gv[32], uv[32];
+                    tmem_ld32(taddr + c, gv);
+                    tmem_ld32(taddr + BN / 2 + c, uv);
+                    if (valid) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float h0 = silu_f(sc * gv[2 * i]) * (sc * uv[2 * i]);
+                            const float h1 = silu_f(sc * gv[2 * i + 1]) * (sc * uv[2 * i + 1]);
+                            pk[i] = pack_bf16x2(h0, h1);
+                        }
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+            } else if (EPI == EPI_SLOT) {
+                __nv_bfloat16* dst = p.out + (size_t)pos * p.out_ld + ti.n * BN;
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    float v[32];
+                    tmem_ld32(taddr + c, v);
+                    if (valid) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            d4[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                                               pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+                    }
+                }
+            } else {   // EPI_RESID / EPI_COMBINE
+                int spos[8];
+                float sg[8];
+                if (EPI == EPI_COMBINE) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        spos[j] = 0;
+                        sg[j] = 0.f;
+                        if (j < p.k && valid) {
+                            const size_t e = ((size_t)b * p.banks + bank) * p.k + j;
+                            spos[j] = __ldg(&p.slot_of[e]);
+                            sg[j] = __ldg(&p.gate[e]);
+                            if (spos[j] < 0 || spos[j] >= p.pos_limit) {
+                                record_error(ERR_BOUNDS, 0x311);
+                                spos[j] = 0;
+                                sg[j] = 0.f;
+                            }
+                        }
+                    }
+                }
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    float v[32];
+                    tmem_ld32(taddr + c, v);
+                    if (!valid) continue;
+                    const int col0 = ti.n * BN + c;
+                    if (EPI == EPI_COMBINE) {
+                        for (int j = 0; j < p.k; ++j) {
+                            const uint4* s4 = reinterpret_cast<const uint4*>(p.slots + (size_t)spos[j] * p.omap.W + col0);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const uint4 w = __ldg(s4 + i);
+                                const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    v[8 * i + 2 * e] += sg[j] * bf16_lo(wv[e]);
+                                    v[8 * i + 2 * e + 1] += sg[j] * bf16_hi(wv[e]);
+                                }
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const size_t off = row_elem(p.omap, b, bank, col0 + 8 * i);
+                        if (off + 8 > p.out_elems) {
+                            record_error(ERR_BOUNDS, 0x313);
+                            continue;
+                        }
+                        float o[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) o[e] = v[8 * i + e];
+                        if (p.resid) {
+                            const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.resid + off));
+                            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) { o[2 * e] += bf16_lo(wv[e]); o[2 * e + 1] += bf16_hi(wv[e]); }
+                        }
+                        if (p.extra) {
+                            const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.extra + off));
+                            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) { o[2 * e] += bf16_lo(wv[e]); o[2 * e + 1] += bf16_hi(wv[e]); }
+                        }
+                        *reinterpret_cast<uint4*>(p.out + off) =
+                            make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                                       pack_bf16x2(o[6], o[7]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+    } else if (AMODE == A_GATHER) {
+        // ---------------------------------------------------------------- row gatherers (warps 6-9)
+        // Thread gt copies 16-byte chunk (gt % 8) of rows (gt / 8) + 16 * i, i = 0..7, into the
+        // 128-byte-swizzled K-major A slab; copies land asynchronously and are published to the
+        // MMA one stage late (commit group, wait, proxy fence, arrive).
+        const int gt = threadIdx.x - 6 * 32;
+        const int chunk = gt & 7;
+        const int rsub = gt >> 3;
+        int s = 0, pend_s = -1;
+        uint32_t ph = 0;
+        for (int t = blockIdx.x; t < ntile; t += gridDim.x) {
+            const TileInfo ti = decode_tile(p, t);
+            int rb[8];
+            int bank = p.sched == 0 ? ti.g : ti.g / p.E;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int rr = rsub + 16 * i;
+                rb[i] = -1;
+                if (rr < ti.nrows) rb[i] = p.sched == 0 ? ti.m * 128 + rr : __ldg(&p.bucket_rows[ti.row0 + rr]);
+                if (rb[i] >= p.rows) {
+                    record_error(ERR_BOUNDS, 0x410);
+                    rb[i] = -1;
+                }
+            }
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x400)) goto gather_done;
+                const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+                const int col = kb * 64 + chunk * 8;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int rr = rsub + 16 * i;
+                    const uint32_t dst = sa + rr * 128 + ((chunk ^ (rr & 7)) << 4);
+                    const __nv_bfloat16* src = rb[i] >= 0 ? p.a_ptr + row_elem(p.amap, rb[i], bank, col) : p.a_ptr;
+                    cp_async_16(dst, src, rb[i] >= 0 ? 16u : 0u);
+                }
+                asm volatile("cp.async.commit_group;" ::: "memory");
+                if (pend_s >= 0) {
+                    asm volatile("cp.async.wait_group 1;" ::: "memory");
+                    fence_proxy_async_smem();
+                    mbar_arrive(&full[pend_s]);
+                }
+                pend_s = s;
+                if (++s == STAGES) { s = 0; ph ^= 1; }
+            }
+        }
+    gather_done:
+        cp_async_wait_all();
+        if (pend_s >= 0) {
+            fence_proxy_async_smem();
+            mbar_arrive(&full[pend_s]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace tml

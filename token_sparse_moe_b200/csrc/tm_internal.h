@@ -1,0 +1,61 @@
+// tm_internal.h -- host-side declarations shared by the library's .cu files.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "tm_gemm.cuh"
+
+namespace tml {
+
+constexpr int kRouterChunk = 128;
+
+// Counts the launch and, while profiling is on, brackets it with a CUDA event pair.
+class ProfileScope {
+   public:
+    ProfileScope(const char* name, cudaStream_t st);
+    ~ProfileScope();
+
+   private:
+    cudaStream_t st_;
+    int ev_;
+    const char* name_;
+};
+void note_cuda_error(const char* where, cudaError_t e);   // samples per router block: one bucketing chunk
+
+// ---- tcgen05 grouped GEMM (bf16) ------------------------------------------------
+// a_mode: AMode; epi: Epi; bn: tile width.  maps are passed by value into the kernel.
+cudaError_t launch_grouped_gemm(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
+                                const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st);
+bool grouped_gemm_supported(int bn, int a_mode, int epi);
+int grouped_gemm_smem(int bn, int a_mode);
+
+// ---- CUDA-core kernels ------------------------------------------------------------
+// dtype: 0 fp32, 1 bf16.
+cudaError_t launch_rms(int dtype, const void* x, RowMap m, int B, float eps, float* inv_rms, cudaStream_t st);
+cudaError_t launch_router(int dtype, const void* x, RowMap m, int B, float eps, const void* gain, const float* w_router,
+                          int E, int k, float alpha, int32_t* idx, float* gate, float* inv_rms, int32_t* counts,
+                          cudaStream_t st);
+cudaError_t launch_offsets(const int32_t* counts_in, int32_t* chunk_prefix, int banks, int nchunks, int E,
+                           int32_t* bucket_offsets, int32_t* tile_start, cudaStream_t st);
+cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, const int32_t* bucket_offsets, int B,
+                           int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st);
+cudaError_t launch_permute(int dtype, const void* src, void* dst, int B, int T, int D, int H, bool to_mixed,
+                           cudaStream_t st);
+cudaError_t launch_fold_gain(int dtype, const void* w, const void* gain, void* out, size_t rows, int width,
+                             cudaStream_t st);
+cudaError_t launch_tokenize(int dtype, const void* groups, const void* w_group, const void* w_global, int dg, int B,
+                            int T, int D, void* X, cudaStream_t st);
+
+// fp32 CUDA-core grouped GEMM with the same tile space and epilogues as the tcgen05 one.
+// A is x (gathered through amap) when epi == EPI_SWIGLU, else hidden rows [positions, K].
+struct SimtGemmArgs {
+    GemmParams p;            // pointer fields reinterpret bf16 as float
+    const float* a;          // x or hidden
+    const float* w0;         // gate / down
+    const float* w1;         // up (SwiGLU)
+};
+cudaError_t launch_simt_gemm(int epi, const SimtGemmArgs& a, int max_tiles, cudaStream_t st);
+
+}  // namespace tml

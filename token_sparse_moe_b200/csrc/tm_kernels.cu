@@ -1,0 +1,538 @@
+// tm_kernels.cu -- CUDA-core kernels of the TokenMixer-Large forward:
+//   * per-row RMSNorm statistics (1/rms) for dense sub-layers,
+//   * the MoE router (fp32 logits, softmax, top-k, alpha-scaled gates) with the
+//     per-chunk expert histogram, the offsets scan and the stable scatter that
+//     together give the expert-first row buckets ("MoEPermute" in the
+//     TokenMixer-Large digest, section 2.5.1),
+//   * Mix / Revert as plain permutations (API utilities; the GEMM path never calls them),
+//   * the gain fold, the tokenizer stub, and the fp32 grouped GEMM used for fp32 tensors.
+#include "tm_internal.h"
+
+namespace tml {
+
+
+// ------------------------------------------------------------------ vector loads
+template <typename T> struct Vec;
+template <> struct Vec<float> {
+    static constexpr int N = 4;
+    __device__ static void load(const float* p, float* o) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+        o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+    }
+};
+template <> struct Vec<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ static void load(const __nv_bfloat16* p, float* o) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { o[2 * i] = bf16_lo(w[i]); o[2 * i + 1] = bf16_hi(w[i]); }
+    }
+};
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ void from_f(float v, float* d) { *d = v; }
+__device__ __forceinline__ void from_f(float v, __nv_bfloat16* d) { *d = __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// ------------------------------------------------------------------ RMS statistics
+// inv_rms[b * banks + bank] = 1 / sqrt(mean(row^2) + eps), one warp per row.
+template <typename T>
+__global__ void rms_kernel(const T* __restrict__ x, RowMap m, int B, float eps, float* __restrict__ inv_rms) {
+    constexpr int V = Vec<T>::N;
+    const int lane = threadIdx.x & 31;
+    const int nrows = B * m.banks;
+    const int wstride = gridDim.x * (blockDim.x >> 5);
+    for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < nrows; row += wstride) {
+        const int b = row / m.banks, bank = row - b * m.banks;
+        float ss = 0.f;
+        for (int c = lane * V; c < m.W; c += 32 * V) {
+            float v[V];
+            Vec<T>::load(x + row_elem(m, b, bank, c), v);
+#pragma unroll
+            for (int i = 0; i < V; ++i) ss = fmaf(v[i], v[i], ss);
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) inv_rms[row] = 1.0f / sqrtf(ss / (float)m.W + eps);
+    }
+}
+
+// ------------------------------------------------------------------ router
+// Block (bank = blockIdx.y, chunk = blockIdx.x) routes samples [chunk*128, chunk*128 + 128) of
+// one bank.  Each warp handles R rows at a time; every lane accumulates partial dot products
+// for all experts, then a butterfly reduction gives every lane the totals.
+template <typename T, int EMAX, int R>
+__global__ void __launch_bounds__(256) router_kernel(const T* __restrict__ x, RowMap m, int B, float eps,
+                                                     const T* __restrict__ gain, const float* __restrict__ w_router,
+                                                     int E, int k, float alpha, int32_t* __restrict__ idx,
+                                                     float* __restrict__ gate, float* __restrict__ inv_rms,
+                                                     int32_t* __restrict__ counts) {
+    constexpr int V = Vec<T>::N;
+    extern __shared__ float wr[];   // [E][W], gain folded in
+    __shared__ int cnt[EMAX];
+    const int bank = blockIdx.y, chunk = blockIdx.x, W = m.W;
+    for (int i = threadIdx.x; i < E * W; i += blockDim.x) {
+        const int c = i % W;
+        const float g = gain ? to_f(gain[c]) : 1.0f;
+        wr[i] = w_router[(size_t)bank * E * W + i] * g;
+    }
+    if (threadIdx.x < EMAX) cnt[threadIdx.x] = 0;
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int ROWS_PER_WARP = kRouterChunk / 8;
+    for (int g0 = 0; g0 < ROWS_PER_WARP; g0 += R) {
+        int bs[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) bs[r] = chunk * kRouterChunk + warp * ROWS_PER_WARP + g0 + r;
+        float acc[R][EMAX];
+        float ss[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            ss[r] = 0.f;
+#pragma unroll
+            for (int e = 0; e < EMAX; ++e) acc[r][e] = 0.f;
+        }
+        for (int c = lane * V; c < W; c += 32 * V) {
+            float xv[R][V];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                if (bs[r] < B) {
+                    Vec<T>::load(x + row_elem(m, bs[r], bank, c), xv[r]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < V; ++i) xv[r][i] = 0.f;
+                }
+#pragma unroll
+                for (int i = 0; i < V; ++i) ss[r] = fmaf(xv[r][i], xv[r][i], ss[r]);
+            }
+#pragma unroll
+            for (int e = 0; e < EMAX; ++e) {
+                if (e < E) {
+                    const float* wp = wr + e * W + c;
+#pragma unroll
+                    for (int i = 0; i < V; ++i) {
+                        const float w = wp[i];
+#pragma unroll
+                        for (int r = 0; r < R; ++r) acc[r][e] = fmaf(w, xv[r][i], acc[r][e]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            ss[r] = warp_sum(ss[r]);
+#pragma unroll
+            for (int e = 0; e < EMAX; ++e)
+                if (e < E) acc[r][e] = warp_sum(acc[r][e]);
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int b = bs[r];
+            if (b >= B) continue;
+            const float irs = 1.0f / sqrtf(ss[r] / (float)W + eps);
+            float z[EMAX];
+            float zmax = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < EMAX; ++e) {
+                z[e] = e < E ? acc[r][e] * irs : -INFINITY;
+                zmax = fmaxf(zmax, z[e]);
+            }
+            float sum = 0.f;
+            float pe[EMAX];
+#pragma unroll
+            for (int e = 0; e < EMAX; ++e) {
+                pe[e] = e < E ? expf(z[e] - zmax) : 0.f;
+                sum += pe[e];
+            }
+            const float inv_sum = 1.0f / sum;
+            uint32_t taken = 0;
+            const size_t rowi = (size_t)b * m.banks + bank;
+            for (int j = 0; j < k; ++j) {
+                int best = -1;
+                float bz = -INFINITY, bp = 0.f;
+#pragma unroll
+                for (int e = 0; e < EMAX; ++e) {
+                    if (e < E && !((taken >> e) & 1u) && (best < 0 || z[e] > bz)) { best = e; bz = z[e]; bp = pe[e]; }
+                }
+                taken |= 1u << best;
+                if (lane == 0) {
+                    idx[rowi * k + j] = best;
+                    gate[rowi * k + j] = alpha * (bp * inv_sum);
+                    atomicAdd(&cnt[best], 1);
+                }
+            }
+            if (lane == 0 && inv_rms) inv_rms[rowi] = irs;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < E) counts[((size_t)bank * gridDim.x + chunk) * E + threadIdx.x] = cnt[threadIdx.x];
+}
+
+// counts [banks][nchunks][E] -> (in place) exclusive prefix over chunks, plus the group
+// offsets and the 128-row tile prefix over groups g = bank*E + e.  One block.
+__global__ void __launch_bounds__(1024) offsets_kernel(int32_t* counts, int banks, int nchunks, int E,
+                                                       int32_t* bucket_offsets, int32_t* tile_start) {
+    __shared__ int tot[4096];
+    const int G = banks * E;
+    for (int g = threadIdx.x; g < G; g += blockDim.x) {
+        const int bank = g / E, e = g - bank * E;
+        int run = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const size_t i = ((size_t)bank * nchunks + c) * E + e;
+            const int v = counts[i];
+            counts[i] = run;
+            run += v;
+        }
+        tot[g] = run;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const int per = (G + 31) / 32;
+        const int lo = min(G, lane * per), hi = min(G, lo + per);
+        int s1 = 0, s2 = 0;
+        for (int g = lo; g < hi; ++g) { s1 += tot[g]; s2 += (tot[g] + 127) / 128; }
+        int e1 = s1, e2 = s2;   // inclusive scan across lanes
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int a = __shfl_up_sync(0xffffffffu, e1, o), b2 = __shfl_up_sync(0xffffffffu, e2, o);
+            if (lane >= o) { e1 += a; e2 += b2; }
+        }
+        int r1 = e1 - s1, r2 = e2 - s2;
+        for (int g = lo; g < hi; ++g) {
+            bucket_offsets[g] = r1;
+            tile_start[g] = r2;
+            r1 += tot[g];
+            r2 += (tot[g] + 127) / 128;
+        }
+        if (lane == 31) { bucket_offsets[G] = e1; tile_start[G] = e2; }
+    }
+}
+
+// Stable scatter: position of (b, bank, j) = group offset + earlier chunks + earlier rows of
+// this chunk routed to the same expert (warp ballots keep ascending b).
+__global__ void __launch_bounds__(kRouterChunk) scatter_kernel(const int32_t* __restrict__ idx,
+                                                               const int32_t* __restrict__ chunk_prefix,
+                                                               const int32_t* __restrict__ bucket_offsets, int B,
+                                                               int banks, int E, int k, int32_t* __restrict__ bucket_rows,
+                                                               int32_t* __restrict__ slot_of) {
+    __shared__ int wcount[kRouterChunk / 32][64];
+    const int bank = blockIdx.y, chunk = blockIdx.x, nchunks = gridDim.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = chunk * kRouterChunk + threadIdx.x;
+    const bool valid = b < B;
+    const size_t rowi = (size_t)b * banks + bank;
+    int my[8], rank[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { my[j] = -1; rank[j] = 0; }
+    if (valid)
+        for (int j = 0; j < k; ++j) my[j] = idx[rowi * k + j];
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int e = 0; e < E; ++e) {
+        bool has = false;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) has |= (my[j] == e);
+        const unsigned bal = __ballot_sync(0xffffffffu, has);
+        if (lane == 0) wcount[warp][e] = __popc(bal);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (my[j] == e) rank[j] = __popc(bal & lt_mask);
+    }
+    __syncthreads();
+    if (!valid) return;
+    const int limit = B * banks * k;
+    for (int j = 0; j < k; ++j) {
+        const int e = my[j];
+        if (e < 0 || e >= E) {
+            record_error(ERR_BOUNDS, 0x500);
+            continue;
+        }
+        int pos = bucket_offsets[bank * E + e] + chunk_prefix[((size_t)bank * nchunks + chunk) * E + e] + rank[j];
+        for (int w = 0; w < warp; ++w) pos += wcount[w][e];
+        if (pos < 0 || pos >= limit) {
+            record_error(ERR_BOUNDS, 0x501);
+            continue;
+        }
+        slot_of[rowi * k + j] = pos;
+        bucket_rows[pos] = b;
+    }
+}
+
+// ------------------------------------------------------------------ Mix / Revert utilities
+template <typename T>
+__global__ void permute_kernel(const T* __restrict__ src, T* __restrict__ dst, int B, int T_, int D, int H,
+                               bool to_mixed) {
+    const size_t total = (size_t)B * T_ * D;
+    const int dh = D / H;
+    for (size_t o = blockIdx.x * (size_t)blockDim.x + threadIdx.x; o < total; o += (size_t)gridDim.x * blockDim.x) {
+        const size_t b = o / ((size_t)T_ * D);
+        const int rem = (int)(o - b * (size_t)T_ * D);
+        const int t = rem / D, d = rem - t * D;
+        const int h = d / dh, j = d - h * dh;
+        const size_t mo = (b * H + h) * (size_t)T_ * dh + (size_t)t * dh + j;   // Hm[b, h, t*dh + j]
+        if (to_mixed) dst[mo] = src[o]; else dst[o] = src[mo];
+    }
+}
+
+template <typename T>
+__global__ void fold_gain_kernel(const T* __restrict__ w, const T* __restrict__ gain, T* __restrict__ out, size_t n,
+                                 int width) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        from_f(to_f(w[i]) * to_f(gain[i % width]), &out[i]);
+}
+
+template <typename T>
+__global__ void tokenize_kernel(const T* __restrict__ groups, const T* __restrict__ w_group,
+                                const T* __restrict__ w_global, int dg, int B, int T_, int D, T* __restrict__ X) {
+    const int G = T_ - 1;
+    const size_t total = (size_t)B * T_ * D;
+    for (size_t o = blockIdx.x * (size_t)blockDim.x + threadIdx.x; o < total; o += (size_t)gridDim.x * blockDim.x) {
+        const size_t b = o / ((size_t)T_ * D);
+        const int rem = (int)(o - b * (size_t)T_ * D);
+        const int t = rem / D, d = rem - t * D;
+        float acc = 0.f;
+        const T* gb = groups + b * (size_t)G * dg;
+        if (t == 0) {
+            const T* wrow = w_global + (size_t)d * G * dg;
+            for (int i = 0; i < G * dg; ++i) acc = fmaf(to_f(wrow[i]), to_f(gb[i]), acc);
+        } else {
+            const T* wrow = w_group + ((size_t)(t - 1) * D + d) * dg;
+            const T* g = gb + (size_t)(t - 1) * dg;
+            for (int c = 0; c < dg; ++c) acc = fmaf(to_f(wrow[c]), to_f(g[c]), acc);
+        }
+        from_f(acc, &X[o]);
+    }
+}
+
+// ------------------------------------------------------------------ fp32 grouped GEMM (CUDA cores)
+// Same tile space (128-row tiles, groups, buckets) and epilogues as the tcgen05 kernel, 32 output
+// columns per block; used for fp32 tensors, where bf16 tensor cores would lose precision.
+template <int EPI>
+__global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtGemmArgs a) {
+    const GemmParams& p = a.p;
+    const int t = blockIdx.x;
+    if (t >= total_tiles(p)) return;
+    const TileInfo ti = decode_tile(p, t);
+    constexpr bool SW = EPI == EPI_SWIGLU;
+    __shared__ float As[32][129];
+    __shared__ float Bs[SW ? 2 : 1][32][33];
+    __shared__ int rowb[128];
+    const int tid = threadIdx.x;
+    const int bank = p.sched == 0 ? ti.g : ti.g / p.E;
+    if (tid < 128) {
+        int b = -1;
+        if (tid < ti.nrows) b = p.sched == 0 ? ti.m * 128 + tid : p.bucket_rows[ti.row0 + tid];
+        if (b >= p.rows || ti.row0 + tid >= p.pos_limit) {
+            if (tid < ti.nrows) record_error(ERR_BOUNDS, 0x600);
+            b = -1;
+        }
+        rowb[tid] = b;
+    }
+    __syncthreads();
+    const int tx = tid & 7, ty = tid >> 3;   // 4 columns x 4 rows per thread
+    const int Nrows = SW ? (p.N >> 1) : p.N; // weight rows per group
+    const int col0 = ti.n * 32;
+    float acc0[4][4] = {}, acc1[4][4] = {};
+    for (int k0 = 0; k0 < p.K; k0 += 32) {
+        {
+            const int kk = tid & 31;
+            const int kq = k0 + kk;
+            for (int i = 0; i < 16; ++i) {
+                const int r = (tid >> 5) + 8 * i;
+                float v = 0.f;
+                const int b = rowb[r];
+                if (b >= 0 && kq < p.K)
+                    v = SW ? a.a[row_elem(p.amap, b, bank, kq)] : a.a[(size_t)(ti.row0 + r) * p.K + kq];
+                As[kk][r] = v;
+            }
+            for (int i = 0; i < 4; ++i) {
+                const int c = (tid >> 5) + 8 * i;
+                const size_t wrow = (size_t)ti.g * Nrows + col0 + c;
+                const bool ok = kq < p.K && col0 + c < Nrows;
+                Bs[0][kk][c] = ok ? a.w0[wrow * p.K + kq] : 0.f;
+                if (SW) Bs[SW ? 1 : 0][kk][c] = ok ? a.w1[wrow * p.K + kq] : 0.f;
+            }
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < 32; ++kk) {
+            float av[4], bv[4], uv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { av[i] = As[kk][ty * 4 + i]; bv[i] = Bs[0][kk][tx * 4 + i]; }
+            if (SW) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) uv[i] = Bs[SW ? 1 : 0][kk][tx * 4 + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc0[i][j] = fmaf(av[i], bv[j], acc0[i][j]);
+                    if (SW) acc1[i][j] = fmaf(av[i], uv[j], acc1[i][j]);
+                }
+        }
+        __syncthreads();
+    }
+    float* out = reinterpret_cast<float*>(p.out);
+    const float* resid = reinterpret_cast<const float*>(p.resid);
+    const float* extra = reinterpret_cast<const float*>(p.extra);
+    const float* slots = reinterpret_cast<const float*>(p.slots);
+    for (int i = 0; i < 4; ++i) {
+        const int r = ty * 4 + i;
+        const int b = rowb[r];
+        if (b < 0) continue;
+        const int pos = ti.row0 + r;
+        for (int j = 0; j < 4; ++j) {
+            const int col = col0 + tx * 4 + j;
+            if (col >= Nrows) continue;
+            if (SW) {
+                const float s = p.inv_rms[(size_t)b * p.banks + bank];
+                const float g = s * acc0[i][j], u = s * acc1[i][j];
+                out[(size_t)pos * p.out_ld + col] = g / (1.0f + expf(-g)) * u;
+            } else if (EPI == EPI_SLOT) {
+                out[(size_t)pos * p.out_ld + col] = acc0[i][j];
+            } else {
+                float v = acc0[i][j];
+                if (EPI == EPI_COMBINE) {
+                    const size_t e0 = ((size_t)b * p.banks + bank) * p.k;
+                    for (int q = 0; q < p.k; ++q) {
+                        const int sp = p.slot_of[e0 + q];
+                        if (sp < 0 || sp >= p.pos_limit) { record_error(ERR_BOUNDS, 0x601); continue; }
+                        v += p.gate[e0 + q] * slots[(size_t)sp * p.omap.W + col];
+                    }
+                }
+                const size_t off = row_elem(p.omap, b, bank, col);
+                if (resid) v += resid[off];
+                if (extra) v += extra[off];
+                out[off] = v;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ launchers
+static int grid_for(size_t n, int threads) {
+    size_t g = (n + threads - 1) / threads;
+    return (int)(g > 65535 * 8 ? 65535 * 8 : (g < 1 ? 1 : g));
+}
+
+cudaError_t launch_rms(int dtype, const void* x, RowMap m, int B, float eps, float* inv_rms, cudaStream_t st) {
+    ProfileScope ps_("rms", st);
+    const size_t rows = (size_t)B * m.banks;
+    const int grid = grid_for(rows * 32, 256);
+    if (dtype == 1)
+        rms_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, m, B, eps, inv_rms);
+    else
+        rms_kernel<float><<<grid, 256, 0, st>>>((const float*)x, m, B, eps, inv_rms);
+    return cudaGetLastError();
+}
+
+template <typename T, int EMAX, int R>
+static cudaError_t router_launch(const void* x, RowMap m, int B, float eps, const void* gain, const float* w_router,
+                                 int E, int k, float alpha, int32_t* idx, float* gate, float* inv_rms,
+                                 int32_t* counts, cudaStream_t st) {
+    const size_t smem = (size_t)E * m.W * sizeof(float);
+    auto kern = router_kernel<T, EMAX, R>;
+    static size_t configured = 0;   // largest dynamic size enabled so far for this instantiation
+    if (smem > configured) {
+        // dynamic + static shared memory may exceed the 48 KB default: always raise the limit
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = smem;
+    }
+    dim3 grid((B + kRouterChunk - 1) / kRouterChunk, m.banks);
+    kern<<<grid, 256, smem, st>>>((const T*)x, m, B, eps, (const T*)gain, w_router, E, k, alpha, idx, gate, inv_rms,
+                                  counts);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router(int dtype, const void* x, RowMap m, int B, float eps, const void* gain,
+                          const float* w_router, int E, int k, float alpha, int32_t* idx, float* gate, float* inv_rms,
+                          int32_t* counts, cudaStream_t st) {
+    ProfileScope ps_("router", st);
+#define TM_ROUTER(T)                                                                                              \
+    if (E <= 8) return router_launch<T, 8, 4>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st); \
+    if (E <= 16) return router_launch<T, 16, 4>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st); \
+    return router_launch<T, 32, 2>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st);
+    if (dtype == 1) { TM_ROUTER(__nv_bfloat16) }
+    TM_ROUTER(float)
+#undef TM_ROUTER
+}
+
+cudaError_t launch_offsets(const int32_t* counts_in, int32_t* chunk_prefix, int banks, int nchunks, int E,
+                           int32_t* bucket_offsets, int32_t* tile_start, cudaStream_t st) {
+    ProfileScope ps_("route_offsets", st);
+    if (counts_in != chunk_prefix) return cudaErrorInvalidValue;   // the scan runs in place
+    offsets_kernel<<<1, 1024, 0, st>>>(chunk_prefix, banks, nchunks, E, bucket_offsets, tile_start);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, const int32_t* bucket_offsets, int B,
+                           int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st) {
+    ProfileScope ps_("route_scatter", st);
+    dim3 grid((B + kRouterChunk - 1) / kRouterChunk, banks);
+    scatter_kernel<<<grid, kRouterChunk, 0, st>>>(idx, chunk_prefix, bucket_offsets, B, banks, E, k, bucket_rows,
+                                                  slot_of);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_permute(int dtype, const void* src, void* dst, int B, int T, int D, int H, bool to_mixed,
+                           cudaStream_t st) {
+    ProfileScope ps_(to_mixed ? "mix" : "revert", st);
+    const size_t n = (size_t)B * T * D;
+    const int grid = grid_for(n, 256);
+    if (dtype == 1)
+        permute_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)src, (__nv_bfloat16*)dst, B, T, D, H,
+                                                            to_mixed);
+    else
+        permute_kernel<float><<<grid, 256, 0, st>>>((const float*)src, (float*)dst, B, T, D, H, to_mixed);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fold_gain(int dtype, const void* w, const void* gain, void* out, size_t rows, int width,
+                             cudaStream_t st) {
+    ProfileScope ps_("fold_gain", st);
+    const size_t n = rows * width;
+    const int grid = grid_for(n, 256);
+    if (dtype == 1)
+        fold_gain_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)w, (const __nv_bfloat16*)gain,
+                                                              (__nv_bfloat16*)out, n, width);
+    else
+        fold_gain_kernel<float><<<grid, 256, 0, st>>>((const float*)w, (const float*)gain, (float*)out, n, width);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tokenize(int dtype, const void* groups, const void* w_group, const void* w_global, int dg, int B,
+                            int T, int D, void* X, cudaStream_t st) {
+    ProfileScope ps_("tokenize", st);
+    const size_t n = (size_t)B * T * D;
+    const int grid = grid_for(n, 256);
+    if (dtype == 1)
+        tokenize_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)groups, (const __nv_bfloat16*)w_group,
+                                                             (const __nv_bfloat16*)w_global, dg, B, T, D,
+                                                             (__nv_bfloat16*)X);
+    else
+        tokenize_kernel<float><<<grid, 256, 0, st>>>((const float*)groups, (const float*)w_group,
+                                                     (const float*)w_global, dg, B, T, D, (float*)X);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_simt_gemm(int epi, const SimtGemmArgs& a, int max_tiles, cudaStream_t st) {
+    if (max_tiles <= 0) return cudaSuccess;
+    ProfileScope ps_(epi == EPI_SWIGLU ? "simt_swiglu" : epi == EPI_RESID ? "simt_resid" : epi == EPI_SLOT ? "simt_slot" : "simt_combine", st);
+    switch (epi) {
+        case EPI_SWIGLU: simt_gemm_kernel<EPI_SWIGLU><<<max_tiles, 256, 0, st>>>(a); break;
+        case EPI_RESID: simt_gemm_kernel<EPI_RESID><<<max_tiles, 256, 0, st>>>(a); break;
+        case EPI_SLOT: simt_gemm_kernel<EPI_SLOT><<<max_tiles, 256, 0, st>>>(a); break;
+        default: simt_gemm_kernel<EPI_COMBINE><<<max_tiles, 256, 0, st>>>(a); break;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace tml
