@@ -160,7 +160,10 @@ def check_stack(cfg, y, samples=None, down_scale=None):
     """Stack output against the oracle with the model's storage rounding (X_revert and block
     outputs in the config dtype).  Samples without near ties: the stated tolerance; samples
     with one: counted and held to a loose bound only."""
-    res = oracle.run_stack(cfg, samples, down_scale=down_scale, storage=cfg.dtype)
+    big = cfg.L * sum(cfg.banks(s) * cfg.width(s) * (cfg.ffn(s).hidden + cfg.ffn(s).E * cfg.ffn(s).hidden_e
+                                                     + cfg.ffn(s).hidden_s) for s in (0, 1)) * 3 > 2e9
+    # weights of the largest workload are drawn bank by bank and dropped (16 GB in bf16)
+    res = oracle.run_stack(cfg, samples, down_scale=down_scale, storage=cfg.dtype, cache=not big)
     o = res["Y"]
     near = near_tie_samples(res, o.shape[0])
     keep = ~near

@@ -207,7 +207,8 @@ def test_fp32_stack_tiny_config_full():
     assert err_delta(y, o, S.to_f64(S.make_x(cfg)), "f32") <= 1e-3
 
 
-@pytest.mark.parametrize("name,n", [("dense_block_bf16", 256), ("nonsquare_dense_bf16", 128), ("moe_stack_bf16", 48)])
+@pytest.mark.parametrize("name,n", [("dense_block_bf16", 256), ("nonsquare_dense_bf16", 128), ("moe_stack_bf16", 48),
+                                    ("large_moe_stack_bf16", 12)])
 def test_full_size_config(name, n):
     cfg = S.CONFIGS[name]
     samples = S.subsample(cfg.B, n)
@@ -250,7 +251,9 @@ def test_tokenize_stub():
     wG = rng.standard_normal((D, G * dg)).astype(np.float32)
     X = api.tokenize_stub(dev(g), dev(wg), dev(wG), D, 8)
     ref = O.tokenize(g.astype(np.float64), wg.astype(np.float64), wG.astype(np.float64))
-    assert err_f32(to_np(X), ref) <= F32_TOL
+    # unit-scale random weights: outputs are sums of 120 terms that cancel near zero in places,
+    # so the fp32 accumulation error is measured against the output rms
+    assert err_bf16(to_np(X), ref) <= 1e-5, err_bf16(to_np(X), ref)
 
 
 def test_workspace_too_small_is_reported():
