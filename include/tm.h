@@ -151,6 +151,27 @@ TM_API tm_status tm_route_topk(const void *x, tm_layout layout, const tm_shape *
                         int32_t *bucket_offsets, int32_t *bucket_rows, int32_t *slot_of,
                         void *workspace, size_t workspace_bytes, void *stream);
 
+/* Fixed size of the routing scratch array that tm_route_topk_noalloc keeps in the library. */
+#define TM_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+/* tm_route_topk without a workspace argument, for callers that cannot allocate device memory
+ * (a host framework that passes this library only its inputs and outputs and owns no allocator
+ * it may call, or a serving loop that reserves all memory at start-up and allows no allocation
+ * later).  The pages have no counterpart: this is a library convenience, not part of the method.
+ * Same arguments, outputs and results as tm_route_topk.  Its scratch (per-chunk expert counts
+ * and the tile prefix: banks * ceil(B/128) * E + banks * E + 1 int32, 256-byte aligned) is a
+ * fixed TM_NOALLOC_SCRATCH_BYTES array inside the library's device image, held by every GPU that
+ * loads the library until the process exits; problems that need more return TM_ERR_WORKSPACE
+ * (message in tm_last_cuda_error) before any launch.  No device memory is allocated or freed.
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress), so
+ * make that first call before any stream capture.  All calls on a device share the array and it
+ * keeps the last call's contents (none of it needs to start at zero): calls that can overlap on
+ * the GPU (different streams without ordering) race on it and must not be issued. */
+TM_API tm_status tm_route_topk_noalloc(const void *x, tm_layout layout, const tm_shape *shape,
+                                       const void *norm_gain, const tm_moe_w *w, int32_t *topk_idx,
+                                       float *topk_gate, float *inv_rms, int32_t *bucket_offsets,
+                                       int32_t *bucket_rows, int32_t *slot_of, void *stream);
+
 /* Dense per-token SwiGLU sub-layer with pre-RMSNorm and residual
  * ([readme] block diagram; [digest] 2.3.2-2.3.3):
  *   y_row = SwiGLU_bank(RMSNorm(x_row) * gain) + residual_row

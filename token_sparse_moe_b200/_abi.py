@@ -14,7 +14,7 @@ TM_LAYOUT_ROWS, TM_LAYOUT_MIXED = 0, 1
 
 # Every entry point declared in include/tm.h (the CPU test checks the library exports each one).
 EXPORTS = ["tm_status_string", "tm_version", "tm_sublayer_workspace_bytes", "tm_route_workspace_bytes",
-           "tm_workspace_bytes", "tm_tokenize_stub", "tm_mix", "tm_revert", "tm_route_topk",
+           "tm_workspace_bytes", "tm_tokenize_stub", "tm_mix", "tm_revert", "tm_route_topk", "tm_route_topk_noalloc",
            "tm_pertoken_swiglu", "tm_sparse_pertoken_moe", "tm_block_forward", "tm_stack_forward",
            "tm_profile_start", "tm_profile_stop", "tm_last_cuda_error", "tm_launch_count",
            "tm_get_device_error"]
@@ -60,6 +60,8 @@ _SIGS = {
     "tm_revert": (c_int, [_P, _P, POINTER(tm_shape), _P]),
     "tm_route_topk": (c_int, [_P, c_int, POINTER(tm_shape), _P, POINTER(tm_moe_w), _P, _P, _P, _P, _P, _P, _P,
                               c_size_t, _P]),
+    "tm_route_topk_noalloc": (c_int, [_P, c_int, POINTER(tm_shape), _P, POINTER(tm_moe_w), _P, _P, _P, _P, _P, _P,
+                                      _P]),
     "tm_pertoken_swiglu": (c_int, [_P, _P, c_int, POINTER(tm_shape), _P, POINTER(tm_swiglu_w), _P, _P, c_size_t, _P]),
     "tm_sparse_pertoken_moe": (c_int, [_P, _P, c_int, POINTER(tm_shape), _P, POINTER(tm_moe_w), _P, _P, c_size_t, _P]),
     "tm_block_forward": (c_int, [_P, POINTER(tm_block), POINTER(tm_shape), _P, _P, _P, c_size_t, _P]),

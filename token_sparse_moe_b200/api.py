@@ -168,6 +168,29 @@ def route_topk(x: torch.Tensor, layout: int, sh: A.tm_shape, sub: SubLayer, work
     return out
 
 
+def route_topk_noalloc(x: torch.Tensor, layout: int, sh: A.tm_shape, sub: SubLayer, out: dict = None,
+                      stream=None) -> dict:
+    """tm_route_topk_noalloc: the same routing with the library's fixed scratch array instead of a
+    workspace.  `out` may hold preallocated output tensors (the keys route_topk returns), so a
+    caller that must not allocate can pass buffers it reserved earlier."""
+    w = sub.moe_c()
+    B, banks, k, E = sh.B, sub.banks, sub.k, sub.E
+    dev = x.device
+    if out is None:
+        out = {
+            "idx": torch.empty((B, banks, k), dtype=torch.int32, device=dev),
+            "gate": torch.empty((B, banks, k), dtype=torch.float32, device=dev),
+            "inv_rms": torch.empty((B, banks), dtype=torch.float32, device=dev),
+            "offsets": torch.empty(banks * E + 1, dtype=torch.int32, device=dev),
+            "rows": torch.empty(B * banks * k, dtype=torch.int32, device=dev),
+            "slot_of": torch.empty((B, banks, k), dtype=torch.int32, device=dev),
+        }
+    A.check(lib().tm_route_topk_noalloc(_p(x), layout, ctypes.byref(sh), _p(sub.gain), ctypes.byref(w),
+                                        _p(out["idx"]), _p(out["gate"]), _p(out["inv_rms"]), _p(out["offsets"]),
+                                        _p(out["rows"]), _p(out["slot_of"]), _s(stream)), "tm_route_topk_noalloc")
+    return out
+
+
 def sublayer_workspace_bytes(sh: A.tm_shape, layout: int, sub: SubLayer) -> int:
     c = sub.c()
     n = lib().tm_sublayer_workspace_bytes(ctypes.byref(sh), layout, ctypes.byref(c))

@@ -4,3 +4,4 @@
 #include "tm_gemm.cu"
 #include "tm_api.cu"
 #include "tm_profile.cu"
+#include "tm_noalloc.cu"

@@ -1,0 +1,98 @@
+// tm_noalloc.cu -- tm_route_topk_noalloc: the router and expert-first bucketing without a
+// caller workspace.
+//
+// Some callers cannot hand this library a scratch buffer: a host framework that owns no
+// allocator it may call, or a serving loop that reserves all device memory at start-up and
+// allows no allocation afterwards.  For them, the routing scratch (per-chunk expert counts
+// and the 128-row tile prefix) lives in a fixed array inside the library's device image.
+// Every GPU that loads the library holds that array until the process exits; nothing here
+// calls cudaMalloc, cudaFree or any allocating routine.
+#include <stdio.h>
+
+#include <mutex>
+
+#include "tm.h"
+#include "tm_internal.h"
+
+namespace tml {
+namespace {
+
+// The routing scratch shared by every call of tm_route_topk_noalloc on a device.
+static __device__ __align__(256) unsigned char g_route_scratch[TM_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_setup_mu;
+void* g_scratch_addr[64] = {nullptr};   // device address of g_route_scratch, per device
+
+// Once per device, with that device current: the array's device address.  In host code the
+// array's name is only a host-side stand-in, so kernels get this address, never the name.
+tm_status scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) { note_cuda_error("tm_route_topk_noalloc: cudaGetDevice", e); return TM_ERR_CUDA; }
+    if (dev < 0 || dev >= 64) return TM_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_setup_mu);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_route_scratch);
+        if (e != cudaSuccess || !p) {
+            note_cuda_error("tm_route_topk_noalloc: cudaGetSymbolAddress", e == cudaSuccess ? cudaErrorUnknown : e);
+            return TM_ERR_CUDA;
+        }
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return TM_OK;
+}
+
+size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
+
+}  // namespace
+}  // namespace tml
+
+using namespace tml;
+
+extern "C" tm_status tm_route_topk_noalloc(const void* x, tm_layout layout, const tm_shape* shape,
+                                          const void* norm_gain, const tm_moe_w* w, int32_t* topk_idx,
+                                          float* topk_gate, float* inv_rms, int32_t* bucket_offsets,
+                                          int32_t* bucket_rows, int32_t* slot_of, void* stream) {
+    // the same validation as tm_route_topk: shape, weights and layout through the size query
+    const size_t need = (shape && w) ? tm_route_workspace_bytes(shape, layout, w) : 0;
+    if (need == 0) return TM_ERR_INVALID_ARG;
+    auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (!x || !al16(x) || !topk_idx || !topk_gate || !bucket_offsets || !bucket_rows || !slot_of)
+        return TM_ERR_INVALID_ARG;
+    if (norm_gain && !al16(norm_gain)) return TM_ERR_INVALID_ARG;
+
+    const int B = shape->B, banks = w->banks, E = w->E;
+    const int nchunks = (B + kRouterChunk - 1) / kRouterChunk;
+    const size_t counts_bytes = (size_t)banks * nchunks * E * sizeof(int32_t);
+    const size_t tiles_bytes = ((size_t)banks * E + 1) * sizeof(int32_t);
+    if (up256(counts_bytes) + tiles_bytes > TM_NOALLOC_SCRATCH_BYTES) {
+        char msg[160];
+        snprintf(msg, sizeof(msg), "tm_route_topk_noalloc: needs %zu bytes of scratch, the fixed limit is %u",
+                 up256(counts_bytes) + tiles_bytes, (unsigned)TM_NOALLOC_SCRATCH_BYTES);
+        note_cuda_error(msg, cudaErrorInvalidValue);
+        return TM_ERR_WORKSPACE;
+    }
+    void* base = nullptr;
+    tm_status s = scratch_address(&base);
+    if (s != TM_OK) return s;
+    int32_t* counts = reinterpret_cast<int32_t*>(base);
+    int32_t* tiles = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(base) + up256(counts_bytes));
+
+    // Nothing in the scratch has to start at zero: the router writes every chunk count and the
+    // offsets kernel writes every tile-prefix entry before anything reads them.
+    const int dh = shape->D / shape->H;
+    const RowMap m{layout == TM_LAYOUT_MIXED ? 1 : 0, banks, w->width, shape->T, shape->D, dh};
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = launch_router(shape->dtype == TM_BF16 ? 1 : 0, x, m, B, shape->eps, norm_gain, w->w_router, E,
+                                  w->k, w->alpha, topk_idx, topk_gate, inv_rms, counts, st);
+    if (e == cudaSuccess) e = launch_offsets(counts, counts, banks, nchunks, E, bucket_offsets, tiles, st);
+    if (e == cudaSuccess)
+        e = launch_scatter(topk_idx, counts, bucket_offsets, B, banks, E, w->k, bucket_rows, slot_of, st);
+    if (e != cudaSuccess) {
+        note_cuda_error("tm_route_topk_noalloc: launch", e);
+        return TM_ERR_CUDA;
+    }
+    return TM_OK;
+}
