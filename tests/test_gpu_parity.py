@@ -40,6 +40,10 @@ DENSE_SMALL = [
     small("dense_ns", 200, 16, 384, 8, "bf16", FFNSpec("dense", hidden=192), FFNSpec("dense", hidden=320)),
     # fp32 CUDA-core path
     small("dense_f32", 150, 8, 64, 8, "f32", FFNSpec("dense", hidden=128), FFNSpec("dense", hidden=96)),
+    # one 128-row tile per bank: the single-CTA fused kernel (more rows run on CTA pairs); width 128
+    small("dense_one_tile", 100, 16, 128, 16, "bf16", FFNSpec("dense", hidden=192), FFNSpec("dense", hidden=128)),
+    # width 128 on CTA pairs with an odd tile count (the last pair's second tile is empty)
+    small("dense_w128", 600, 8, 128, 4, "bf16", FFNSpec("dense", hidden=128), FFNSpec("dense", hidden=256)),
 ]
 MOE_SMALL = [
     small("moe_sq", 300, 16, 256, 16, "bf16", moe(8, 2, 128, 128, 4.0), moe(4, 1, 64, 192, 4.0)),
@@ -214,6 +218,18 @@ def test_full_size_config(name, n):
     samples = S.subsample(cfg.B, n)
     y = _stack_gpu(cfg, samples=samples)
     check_stack(cfg, y, samples)
+
+
+@pytest.mark.parametrize("cfg", [DENSE_SMALL[0], DENSE_SMALL[4]], ids=lambda c: c.name)
+def test_fused_cta_pair_kernel(cfg, monkeypatch):
+    """The opt-in CTA-pair (2-SM MMA) version of the fused sub-layer gives the same results."""
+    monkeypatch.setenv("TM_FUSED_PAIRS", "1")
+    X, R = inputs(cfg)
+    for sub in (0, 1):
+        for ds in (None, 1.0):
+            y, _ = _run_sub(cfg, sub, X, R, ds)
+            o, _, _ = _oracle_sub(cfg, sub, X, R, ds)
+            check_outputs(cfg, y, o, S.to_f64(R), ds)
 
 
 def test_block_forward_matches_stack_and_returns_revert():

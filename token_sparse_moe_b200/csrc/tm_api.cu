@@ -2,6 +2,7 @@
 // carving, TMA tensor maps and the launch sequence of every call.  Nothing here
 // allocates device memory or synchronises (except tm_get_device_error).
 #include <math.h>
+#include <stdlib.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -255,6 +256,44 @@ tm_status gemm2_dense(const Geo& g, const void* hidden, const void* wd, int F, i
     return cuda_status(launch_grouped_gemm(bn, A_TMA_2D, epi, ma, mb, mb, p, dense_grid(p), st));
 }
 
+// ------------------------------------------------------------------ fused dense sub-layer
+// One launch for row widths 128 / 256: statistics, GEMM1, SwiGLU, GEMM2, residual.
+tm_status fused_dense(const Geo& g, const void* x, const void* wg, const void* wu, const void* wd, int F,
+                      const void* resid, const void* extra, void* y, cudaStream_t st) {
+    const int am = gemm1_amode(g);
+    // One CTA per 128-row tile by default.  TM_FUSED_PAIRS=1 selects the CTA-pair kernel (2-SM
+    // MMAs, half the weight bytes per SM); on B200 it measured slower on the dense block workload
+    // (0.189 ms against 0.149 ms per sub-layer): its per-chunk handoffs cross the CTA pair.
+    const char* env = getenv("TM_FUSED_PAIRS");
+    const bool pairs = g.B > 128 && env && env[0] == '1';
+    CUtensorMap ma, mg, mu, md;
+    if (!gemm1_amap(g, x, am, &ma)) return TM_ERR_CUDA;
+    if (!map_2d(&mg, wg, (uint64_t)g.banks * F, g.W, 64) || !map_2d(&mu, wu, (uint64_t)g.banks * F, g.W, 64) ||
+        !map_2d(&md, wd, (uint64_t)g.banks * g.W, F, pairs ? g.W / 2 : g.W))
+        return TM_ERR_CUDA;
+    FusedParams p;
+    memset(&p, 0, sizeof(p));
+    p.banks = g.banks;
+    p.rows = g.B;
+    p.F = F;
+    p.amap = g.map;
+    p.eps = g.eps;
+    p.out = (__nv_bfloat16*)y;
+    p.resid = (const __nv_bfloat16*)resid;
+    p.extra = (const __nv_bfloat16*)extra;
+    p.omap = g.map;
+    p.out_elems = (size_t)g.B * g.banks * g.W;
+    const long mt = (g.B + 127) / 128;
+    if (pairs) {
+        const long pair_tiles = (long)g.banks * ((mt + 1) / 2);
+        const long clusters = pair_tiles < num_sms() / 2 ? pair_tiles : num_sms() / 2;
+        return cuda_status(launch_fused2(g.W, am, ma, mg, mu, md, p, (int)(2 * clusters), st));
+    }
+    const long tiles = (long)g.banks * mt;
+    const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+    return cuda_status(launch_fused(g.W, am, ma, mg, mu, md, p, grid, st));
+}
+
 // ------------------------------------------------------------------ dense sub-layer
 struct DenseWs {
     float* inv_rms;
@@ -286,6 +325,8 @@ tm_status run_dense(const Geo& g, const void* x, const void* resid, const void* 
         wg = d.wg;
         wu = d.wu;
     }
+    if (g.dtype == TM_BF16 && fused_supported(g.W, gemm1_amode(g)) && w->hidden % 64 == 0)
+        return fused_dense(g, x, wg, wu, w->w_down, w->hidden, resid, extra, y, st);
     if ((s = cuda_status(launch_rms(g.dtype, x, g.map, g.B, g.eps, d.inv_rms, st))) != TM_OK) return s;
     if ((s = gemm1_dense(g, x, wg, wu, w->hidden, d.inv_rms, d.hidden, st)) != TM_OK) return s;
     return gemm2_dense(g, d.hidden, w->w_down, w->hidden, EPI_RESID, resid, extra, y, nullptr, nullptr, nullptr, 0, st);

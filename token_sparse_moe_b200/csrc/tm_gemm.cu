@@ -1,7 +1,75 @@
-// tm_gemm.cu -- instantiations and launcher of the tcgen05 grouped GEMM.
+// tm_gemm.cu -- instantiations and launchers of the tcgen05 kernels (grouped GEMM, fused sub-layer).
+#include <string.h>
+#include "tm_fused2.cuh"
 #include "tm_internal.h"
 
 namespace tml {
+
+template <int W, int AM>
+static cudaError_t launch_fused_one(const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
+                                    const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st) {
+    using C = FusedCfg<W, AM>;
+    auto kern = fused_swiglu_kernel<W, AM>;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    ProfileScope ps_("fused_swiglu", st);
+    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, g, u, d, p);
+    return cudaGetLastError();
+}
+
+template <int W, int AM>
+static cudaError_t launch_fused2_one(const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
+                                     const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st) {
+    using C = Fused2Cfg<W, AM>;
+    auto kern = fused2_swiglu_kernel<W, AM>;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(C::NTHREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    ProfileScope ps_("fused_swiglu", st);
+    return cudaLaunchKernelEx(&cfg, kern, a, g, u, d, p);
+}
+
+cudaError_t launch_fused2(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
+                          const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st) {
+    if (W == 256 && a_mode == A_TMA_MIX) return launch_fused2_one<256, A_TMA_MIX>(a, g, u, d, p, grid, st);
+    if (W == 256 && a_mode == A_TMA_3D) return launch_fused2_one<256, A_TMA_3D>(a, g, u, d, p, grid, st);
+    if (W == 128 && a_mode == A_TMA_MIX) return launch_fused2_one<128, A_TMA_MIX>(a, g, u, d, p, grid, st);
+    if (W == 128 && a_mode == A_TMA_3D) return launch_fused2_one<128, A_TMA_3D>(a, g, u, d, p, grid, st);
+    return cudaErrorInvalidValue;
+}
+
+bool fused_supported(int W, int a_mode) {
+    return (W == 128 || W == 256) && (a_mode == A_TMA_MIX || a_mode == A_TMA_3D);
+}
+
+cudaError_t launch_fused(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
+                         const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st) {
+    if (W == 256 && a_mode == A_TMA_MIX) return launch_fused_one<256, A_TMA_MIX>(a, g, u, d, p, grid, st);
+    if (W == 256 && a_mode == A_TMA_3D) return launch_fused_one<256, A_TMA_3D>(a, g, u, d, p, grid, st);
+    if (W == 128 && a_mode == A_TMA_MIX) return launch_fused_one<128, A_TMA_MIX>(a, g, u, d, p, grid, st);
+    if (W == 128 && a_mode == A_TMA_3D) return launch_fused_one<128, A_TMA_3D>(a, g, u, d, p, grid, st);
+    return cudaErrorInvalidValue;
+}
 
 template <int BN, int AM, int EPI>
 static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmParams& p,

@@ -299,8 +299,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
                         uint32_t pk[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const float h0 = silu_f(sc * gv[2 * i]) * (sc * uv[2 * i]);
-                            const float h1 = silu_f(sc * gv[2 * i + 1]) * (sc * uv[2 * i + 1]);
+                            const float h0 = silu_tanh(sc * gv[2 * i]) * (sc * uv[2 * i]);
+                            const float h1 = silu_tanh(sc * gv[2 * i + 1]) * (sc * uv[2 * i + 1]);
                             pk[i] = pack_bf16x2(h0, h1);
                         }
                         uint4* d4 = reinterpret_cast<uint4*>(dst + c);

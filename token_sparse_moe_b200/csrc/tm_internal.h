@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include "tm_gemm.cuh"
+#include "tm_fused2.cuh"
 
 namespace tml {
 
@@ -29,6 +30,14 @@ void note_cuda_error(const char* where, cudaError_t e);   // samples per router 
 cudaError_t launch_grouped_gemm(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                                 const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st);
 bool grouped_gemm_supported(int bn, int a_mode, int epi);
+
+// ---- fused dense sub-layer (row width 128 / 256) --------------------------------
+bool fused_supported(int W, int a_mode);
+cudaError_t launch_fused(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
+                         const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st);
+// CTA-pair version (2-SM MMAs, clusters of 2): grid = 2 x clusters; weight maps with half-size boxes
+cudaError_t launch_fused2(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
+                          const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st);
 int grouped_gemm_smem(int bn, int a_mode);
 
 // ---- CUDA-core kernels ------------------------------------------------------------
