@@ -140,7 +140,13 @@ tm_status check_moe(const Geo& g, const tm_moe_w* w) {
     if (!isfinite(w->alpha)) return TM_ERR_INVALID_ARG;
     if (w->E > 32 || w->k > 8) return TM_ERR_UNSUPPORTED;
     if ((size_t)w->banks * w->E > 4096) return TM_ERR_UNSUPPORTED;
-    if ((size_t)w->E * w->width * 4 > 200 * 1024) return TM_ERR_UNSUPPORTED;   // router weights staged in smem
+    // router weights (expert count rounded up to a power of two, rows padded by 4) and each
+    // warp's two staging buffers of rows, all in shared memory
+    {
+        const size_t ep = w->E <= 4 ? 4 : w->E <= 8 ? 8 : w->E <= 16 ? 16 : 32;
+        const size_t group = 32 / ep > 4 ? 32 / ep : 4;
+        if (ep * (w->width + 4) * 4 + 16 * group * (size_t)w->width * g.esz > 220 * 1024) return TM_ERR_UNSUPPORTED;
+    }
     if (!w->w_router || !w->we_gate || !w->we_up || !w->we_down) return TM_ERR_INVALID_ARG;
     if (!al16(w->w_router) || !al16(w->we_gate) || !al16(w->we_up) || !al16(w->we_down)) return TM_ERR_INVALID_ARG;
     if (w->hidden_s > 0) {

@@ -348,44 +348,56 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
                     tmem_ld32(taddr + c, v);
                     if (!valid) continue;
                     const int col0 = ti.n * BN + c;
+                    // all global reads of this 32-column slice are issued before any arithmetic:
+                    // residual and inter-residual first, then the slot rows two experts at a time
+                    size_t off[4];
+                    uint4 rv[4], ev[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        off[i] = row_elem(p.omap, b, bank, col0 + 8 * i);
+                        const bool in = off[i] + 8 <= p.out_elems;
+                        rv[i] = (p.resid && in) ? __ldg(reinterpret_cast<const uint4*>(p.resid + off[i])) : make_uint4(0, 0, 0, 0);
+                        ev[i] = (p.extra && in) ? __ldg(reinterpret_cast<const uint4*>(p.extra + off[i])) : make_uint4(0, 0, 0, 0);
+                    }
                     if (EPI == EPI_COMBINE) {
-                        for (int j = 0; j < p.k; ++j) {
-                            const uint4* s4 = reinterpret_cast<const uint4*>(p.slots + (size_t)spos[j] * p.omap.W + col0);
+                        for (int j = 0; j < p.k; j += 2) {
+                            const bool two = j + 1 < p.k;
+                            const uint4* s0 = reinterpret_cast<const uint4*>(p.slots + (size_t)spos[j] * p.omap.W + col0);
+                            const uint4* s1 = reinterpret_cast<const uint4*>(p.slots + (size_t)spos[two ? j + 1 : j] * p.omap.W + col0);
+                            uint4 a0[4], a1[4];
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
-                                const uint4 w = __ldg(s4 + i);
-                                const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                                a0[i] = __ldg(s0 + i);
+                                a1[i] = two ? __ldg(s1 + i) : make_uint4(0, 0, 0, 0);
+                            }
+                            const float g0 = sg[j], g1 = two ? sg[j + 1] : 0.f;
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const uint32_t w0[4] = {a0[i].x, a0[i].y, a0[i].z, a0[i].w};
+                                const uint32_t w1[4] = {a1[i].x, a1[i].y, a1[i].z, a1[i].w};
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
-                                    v[8 * i + 2 * e] += sg[j] * bf16_lo(wv[e]);
-                                    v[8 * i + 2 * e + 1] += sg[j] * bf16_hi(wv[e]);
+                                    v[8 * i + 2 * e] += g0 * bf16_lo(w0[e]) + g1 * bf16_lo(w1[e]);
+                                    v[8 * i + 2 * e + 1] += g0 * bf16_hi(w0[e]) + g1 * bf16_hi(w1[e]);
                                 }
                             }
                         }
                     }
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const size_t off = row_elem(p.omap, b, bank, col0 + 8 * i);
-                        if (off + 8 > p.out_elems) {
+                        if (off[i] + 8 > p.out_elems) {
                             record_error(ERR_BOUNDS, 0x313);
                             continue;
                         }
+                        const uint32_t rw[4] = {rv[i].x, rv[i].y, rv[i].z, rv[i].w};
+                        const uint32_t ew[4] = {ev[i].x, ev[i].y, ev[i].z, ev[i].w};
                         float o[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) o[e] = v[8 * i + e];
-                        if (p.resid) {
-                            const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.resid + off));
-                            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) { o[2 * e] += bf16_lo(wv[e]); o[2 * e + 1] += bf16_hi(wv[e]); }
+                        for (int e = 0; e < 4; ++e) {
+                            o[2 * e] = v[8 * i + 2 * e] + bf16_lo(rw[e]) + bf16_lo(ew[e]);
+                            o[2 * e + 1] = v[8 * i + 2 * e + 1] + bf16_hi(rw[e]) + bf16_hi(ew[e]);
                         }
-                        if (p.extra) {
-                            const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.extra + off));
-                            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) { o[2 * e] += bf16_lo(wv[e]); o[2 * e + 1] += bf16_hi(wv[e]); }
-                        }
-                        *reinterpret_cast<uint4*>(p.out + off) =
+                        *reinterpret_cast<uint4*>(p.out + off[i]) =
                             make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
                                        pack_bf16x2(o[6], o[7]));
                     }

@@ -19,11 +19,21 @@ template <> struct Vec<float> {
         const float4 v = __ldg(reinterpret_cast<const float4*>(p));
         o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
     }
+    __device__ static void load_shared(const float* p, float* o) {
+        const float4 v = *reinterpret_cast<const float4*>(p);
+        o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+    }
 };
 template <> struct Vec<__nv_bfloat16> {
     static constexpr int N = 8;
     __device__ static void load(const __nv_bfloat16* p, float* o) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { o[2 * i] = bf16_lo(w[i]); o[2 * i + 1] = bf16_hi(w[i]); }
+    }
+    __device__ static void load_shared(const __nv_bfloat16* p, float* o) {
+        const uint4 v = *reinterpret_cast<const uint4*>(p);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) { o[2 * i] = bf16_lo(w[i]); o[2 * i + 1] = bf16_hi(w[i]); }
@@ -63,112 +73,120 @@ __global__ void rms_kernel(const T* __restrict__ x, RowMap m, int B, float eps, 
 }
 
 // ------------------------------------------------------------------ router
-// Block (bank = blockIdx.y, chunk = blockIdx.x) routes samples [chunk*128, chunk*128 + 128) of
-// one bank.  Each warp handles R rows at a time; every lane accumulates partial dot products
-// for all experts, then a butterfly reduction gives every lane the totals.
-template <typename T, int EMAX, int R>
+// Block (bank = blockIdx.y, chunk = blockIdx.x) routes samples [chunk*128, chunk*128 + 128) of one
+// bank; warp w owns 16 of them.  Lane l works on the pair (row l / EP, expert l % EP) with EP the
+// expert count rounded up to a power of two: it walks the whole row in shared memory (x reads are
+// broadcasts among the row's lanes; router-weight rows are padded by 4 floats, so the float4 reads
+// of the EP lanes hit distinct banks) and accumulates its logit and the row's sum of squares.
+// Softmax and top-k then reduce over the EP lanes of a row only.  Each warp stages its own rows
+// with cp.async, double-buffered, so no block-wide barrier is needed after the weights load.
+template <typename T, int EP>
 __global__ void __launch_bounds__(256) router_kernel(const T* __restrict__ x, RowMap m, int B, float eps,
                                                      const T* __restrict__ gain, const float* __restrict__ w_router,
                                                      int E, int k, float alpha, int32_t* __restrict__ idx,
                                                      float* __restrict__ gate, float* __restrict__ inv_rms,
                                                      int32_t* __restrict__ counts) {
     constexpr int V = Vec<T>::N;
-    extern __shared__ float wr[];   // [E][W], gain folded in
-    __shared__ int cnt[EMAX];
-    const int bank = blockIdx.y, chunk = blockIdx.x, W = m.W;
-    for (int i = threadIdx.x; i < E * W; i += blockDim.x) {
-        const int c = i % W;
-        const float g = gain ? to_f(gain[c]) : 1.0f;
-        wr[i] = w_router[(size_t)bank * E * W + i] * g;
+    constexpr int ROWS = 32 / EP;                 // rows per warp pass
+    constexpr int GROUP = ROWS > 4 ? ROWS : 4;    // rows per staging buffer
+    constexpr int WARP_ROWS = kRouterChunk / 8;   // 16
+    static_assert(WARP_ROWS % GROUP == 0, "router row groups");
+    extern __shared__ __align__(16) float wr[];   // [EP][W + 4], then per warp 2 x [GROUP][W] rows
+    __shared__ int cnt[32];
+    const int bank = blockIdx.y, chunk = blockIdx.x, W = m.W, WP = W + 4;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < EP * WP; i += blockDim.x) {
+        const int e = i / WP, c = i - e * WP;
+        float v = 0.f;
+        if (e < E && c < W) v = w_router[((size_t)bank * E + e) * W + c] * (gain ? to_f(gain[c]) : 1.0f);
+        wr[i] = v;
     }
-    if (threadIdx.x < EMAX) cnt[threadIdx.x] = 0;
+    if (threadIdx.x < 32) cnt[threadIdx.x] = 0;
     __syncthreads();
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int ROWS_PER_WARP = kRouterChunk / 8;
-    for (int g0 = 0; g0 < ROWS_PER_WARP; g0 += R) {
-        int bs[R];
-#pragma unroll
-        for (int r = 0; r < R; ++r) bs[r] = chunk * kRouterChunk + warp * ROWS_PER_WARP + g0 + r;
-        float acc[R][EMAX];
-        float ss[R];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            ss[r] = 0.f;
-#pragma unroll
-            for (int e = 0; e < EMAX; ++e) acc[r][e] = 0.f;
-        }
+    T* xb = reinterpret_cast<T*>(wr + EP * WP) + (size_t)warp * 2 * GROUP * W;
+    const size_t row_stride = m.layout == 0 ? (size_t)m.banks * W : (size_t)m.T * m.D;   // sample b -> b+1
+    const int b_first = chunk * kRouterChunk + warp * WARP_ROWS;
+    auto stage = [&](int grp, int buf) {
+        T* dst = xb + (size_t)buf * GROUP * W;
         for (int c = lane * V; c < W; c += 32 * V) {
-            float xv[R][V];
+            const size_t base = row_elem(m, 0, bank, c);
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                if (bs[r] < B) {
-                    Vec<T>::load(x + row_elem(m, bs[r], bank, c), xv[r]);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < V; ++i) xv[r][i] = 0.f;
-                }
-#pragma unroll
-                for (int i = 0; i < V; ++i) ss[r] = fmaf(xv[r][i], xv[r][i], ss[r]);
-            }
-#pragma unroll
-            for (int e = 0; e < EMAX; ++e) {
-                if (e < E) {
-                    const float* wp = wr + e * W + c;
-#pragma unroll
-                    for (int i = 0; i < V; ++i) {
-                        const float w = wp[i];
-#pragma unroll
-                        for (int r = 0; r < R; ++r) acc[r][e] = fmaf(w, xv[r][i], acc[r][e]);
-                    }
-                }
+            for (int r = 0; r < GROUP; ++r) {
+                const int b = b_first + grp * GROUP + r;
+                const uint32_t d = smem_u32(dst + (size_t)r * W + c);
+                if (b < B) cp_async_16(d, x + base + (size_t)b * row_stride, 16u);
+                else cp_async_16(d, x, 0u);
             }
         }
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            ss[r] = warp_sum(ss[r]);
-#pragma unroll
-            for (int e = 0; e < EMAX; ++e)
-                if (e < E) acc[r][e] = warp_sum(acc[r][e]);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    constexpr int NG = WARP_ROWS / GROUP;
+    stage(0, 0);
+    const int rl = lane / EP, e = lane % EP;
+#pragma unroll 1
+    for (int gi = 0; gi < NG; ++gi) {
+        if (gi + 1 < NG) {
+            stage(gi + 1, (gi + 1) & 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
+        __syncwarp();
+        const T* xr0 = xb + (size_t)(gi & 1) * GROUP * W;
+#pragma unroll 1
+        for (int pass = 0; pass < GROUP / ROWS; ++pass) {
+            const int r = pass * ROWS + rl;
+            const int b = b_first + gi * GROUP + r;
+            const T* xr = xr0 + (size_t)r * W;
+            const float* wrow = wr + e * WP;
+            float dot = 0.f, ss = 0.f;
+            for (int c = 0; c < W; c += V) {
+                float xv[V];
+                Vec<T>::load_shared(xr + c, xv);
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int b = bs[r];
-            if (b >= B) continue;
-            const float irs = 1.0f / sqrtf(ss[r] / (float)W + eps);
-            float z[EMAX];
-            float zmax = -INFINITY;
+                for (int q = 0; q < V; q += 4) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(wrow + c + q);
+                    dot = fmaf(w4.x, xv[q], dot);
+                    dot = fmaf(w4.y, xv[q + 1], dot);
+                    dot = fmaf(w4.z, xv[q + 2], dot);
+                    dot = fmaf(w4.w, xv[q + 3], dot);
+                }
 #pragma unroll
-            for (int e = 0; e < EMAX; ++e) {
-                z[e] = e < E ? acc[r][e] * irs : -INFINITY;
-                zmax = fmaxf(zmax, z[e]);
+                for (int q = 0; q < V; ++q) ss = fmaf(xv[q], xv[q], ss);
             }
-            float sum = 0.f;
-            float pe[EMAX];
+            const float irs = 1.0f / sqrtf(ss / (float)W + eps);
+            float z = e < E ? dot * irs : -INFINITY;
+            float zmax = z;
 #pragma unroll
-            for (int e = 0; e < EMAX; ++e) {
-                pe[e] = e < E ? expf(z[e] - zmax) : 0.f;
-                sum += pe[e];
-            }
-            const float inv_sum = 1.0f / sum;
-            uint32_t taken = 0;
+            for (int o = 1; o < EP; o <<= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
+            const float pe = e < E ? expf(z - zmax) : 0.f;
+            float sum = pe;
+#pragma unroll
+            for (int o = 1; o < EP; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            const float p = pe / sum;
             const size_t rowi = (size_t)b * m.banks + bank;
+            float zc = z;                       // candidate logit; -inf once taken
             for (int j = 0; j < k; ++j) {
-                int best = -1;
-                float bz = -INFINITY, bp = 0.f;
+                float bz = zc;
+                int be = zc == -INFINITY ? 1 << 30 : e;   // ties and exhausted lanes: lower index wins
 #pragma unroll
-                for (int e = 0; e < EMAX; ++e) {
-                    if (e < E && !((taken >> e) & 1u) && (best < 0 || z[e] > bz)) { best = e; bz = z[e]; bp = pe[e]; }
+                for (int o = 1; o < EP; o <<= 1) {
+                    const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
+                    const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                    if (oz > bz || (oz == bz && oe < be)) { bz = oz; be = oe; }
                 }
-                taken |= 1u << best;
-                if (lane == 0) {
-                    idx[rowi * k + j] = best;
-                    gate[rowi * k + j] = alpha * (bp * inv_sum);
-                    atomicAdd(&cnt[best], 1);
+                const float pb = __shfl_sync(0xffffffffu, p, (lane & ~(EP - 1)) + (be < EP ? be : 0));
+                if (e == be) zc = -INFINITY;
+                if (e == 0 && b < B && be < E) {
+                    idx[rowi * k + j] = be;
+                    gate[rowi * k + j] = alpha * pb;
+                    atomicAdd(&cnt[be], 1);
                 }
             }
-            if (lane == 0 && inv_rms) inv_rms[rowi] = irs;
+            if (e == 0 && b < B && inv_rms) inv_rms[rowi] = irs;
         }
+        __syncwarp();                          // buffer (gi & 1) is refilled two groups later
     }
     __syncthreads();
     if (threadIdx.x < E) counts[((size_t)bank * gridDim.x + chunk) * E + threadIdx.x] = cnt[threadIdx.x];
@@ -433,12 +451,13 @@ cudaError_t launch_rms(int dtype, const void* x, RowMap m, int B, float eps, flo
     return cudaGetLastError();
 }
 
-template <typename T, int EMAX, int R>
+template <typename T, int EP>
 static cudaError_t router_launch(const void* x, RowMap m, int B, float eps, const void* gain, const float* w_router,
                                  int E, int k, float alpha, int32_t* idx, float* gate, float* inv_rms,
                                  int32_t* counts, cudaStream_t st) {
-    const size_t smem = (size_t)E * m.W * sizeof(float);
-    auto kern = router_kernel<T, EMAX, R>;
+    constexpr int GROUP = 32 / EP > 4 ? 32 / EP : 4;
+    const size_t smem = (size_t)EP * (m.W + 4) * sizeof(float) + (size_t)8 * 2 * GROUP * m.W * sizeof(T);
+    auto kern = router_kernel<T, EP>;
     static size_t configured = 0;   // largest dynamic size enabled so far for this instantiation
     if (smem > configured) {
         // dynamic + static shared memory may exceed the 48 KB default: always raise the limit
@@ -456,10 +475,11 @@ cudaError_t launch_router(int dtype, const void* x, RowMap m, int B, float eps, 
                           const float* w_router, int E, int k, float alpha, int32_t* idx, float* gate, float* inv_rms,
                           int32_t* counts, cudaStream_t st) {
     ProfileScope ps_("router", st);
-#define TM_ROUTER(T)                                                                                              \
-    if (E <= 8) return router_launch<T, 8, 4>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st); \
-    if (E <= 16) return router_launch<T, 16, 4>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st); \
-    return router_launch<T, 32, 2>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st);
+#define TM_ROUTER(T)                                                                                                  \
+    if (E <= 4) return router_launch<T, 4>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st);  \
+    if (E <= 8) return router_launch<T, 8>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st);  \
+    if (E <= 16) return router_launch<T, 16>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st); \
+    return router_launch<T, 32>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st);
     if (dtype == 1) { TM_ROUTER(__nv_bfloat16) }
     TM_ROUTER(float)
 #undef TM_ROUTER
