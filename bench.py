@@ -36,7 +36,7 @@ import tm_synth as S  # noqa: E402
 METRIC = "samples/sec & TFLOP/s of TokenMixer-Large fwd, % of B200 bf16 TC roofline"
 DEFAULT_WORKLOAD = "dense_block_bf16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["tm_gemm.cuh", "tm_fused.cuh", "tm_fused2.cuh", "tm_device.cuh", "tm_gemm.cu", "tm_kernels.cu", "tm_api.cu"]
+KERNEL_SOURCES = ["tm_gemm.cuh", "tm_fused.cuh", "tm_fused2.cuh", "tm_fused128.cuh", "tm_device.cuh", "tm_gemm.cu", "tm_kernels.cu", "tm_api.cu"]
 
 
 def describe(cfg) -> str:
@@ -237,7 +237,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.Stream(device=dev)
-    blocks = api.blocks_from_synth(cfg, dev)
+    blocks = api.blocks_from_synth(cfg, dev, workers=min(16, os.cpu_count() or 1))
     sh = api.config_shape(cfg)
     run = api.StackRunner(blocks, sh, cfg.gap, dev)
     X = api.to_device(S.make_x(cfg.with_(seed=cfg.seed + rank)), dev)

@@ -40,9 +40,9 @@ DENSE_SMALL = [
     small("dense_ns", 200, 16, 384, 8, "bf16", FFNSpec("dense", hidden=192), FFNSpec("dense", hidden=320)),
     # fp32 CUDA-core path
     small("dense_f32", 150, 8, 64, 8, "f32", FFNSpec("dense", hidden=128), FFNSpec("dense", hidden=96)),
-    # one 128-row tile per bank: the single-CTA fused kernel (more rows run on CTA pairs); width 128
+    # one 128-row tile per bank, width 128; mixing hidden 192 takes the 64-wide-chunk fused kernel
     small("dense_one_tile", 100, 16, 128, 16, "bf16", FFNSpec("dense", hidden=192), FFNSpec("dense", hidden=128)),
-    # width 128 on CTA pairs with an odd tile count (the last pair's second tile is empty)
+    # width 128 and 256 with 5 row tiles (an odd count on CTA pairs: the last pair's second tile is empty)
     small("dense_w128", 600, 8, 128, 4, "bf16", FFNSpec("dense", hidden=128), FFNSpec("dense", hidden=256)),
 ]
 MOE_SMALL = [
@@ -184,7 +184,9 @@ def test_norm_gain(cfg):
 
 
 def _stack_gpu(cfg, down_scale=None, samples=None):
-    blocks = api.blocks_from_synth(cfg, DEV, down_scale)
+    import os
+    big = cfg.B * cfg.T * cfg.D > 1e8
+    blocks = api.blocks_from_synth(cfg, DEV, down_scale, workers=min(16, os.cpu_count() or 1) if big else 1)
     sh = api.config_shape(cfg)
     X = S.make_x(cfg)
     Y = api.stack_forward(dev(X), blocks, cfg.gap, sh)
@@ -224,6 +226,19 @@ def test_full_size_config(name, n):
 def test_fused_cta_pair_kernel(cfg, monkeypatch):
     """The opt-in CTA-pair (2-SM MMA) version of the fused sub-layer gives the same results."""
     monkeypatch.setenv("TM_FUSED_PAIRS", "1")
+    X, R = inputs(cfg)
+    for sub in (0, 1):
+        for ds in (None, 1.0):
+            y, _ = _run_sub(cfg, sub, X, R, ds)
+            o, _, _ = _oracle_sub(cfg, sub, X, R, ds)
+            check_outputs(cfg, y, o, S.to_f64(R), ds)
+
+
+@pytest.mark.parametrize("cfg", [DENSE_SMALL[0], DENSE_SMALL[4]], ids=lambda c: c.name)
+def test_fused_64_wide_chunk_kernel(cfg, monkeypatch):
+    """The fused sub-layer with 64-wide hidden chunks (the kernel for F % 128 == 64) forced on
+    hidden widths that would otherwise take 128-wide chunks gives the same results."""
+    monkeypatch.setenv("TM_FUSED64", "1")
     X, R = inputs(cfg)
     for sub in (0, 1):
         for ds in (None, 1.0):

@@ -204,14 +204,15 @@ def sublayer_weights(cfg: Config, layer: int, sub: int, down_scale: Optional[flo
                      workers: Optional[int] = None) -> Dict[str, np.ndarray]:
     """All banks of one sub-layer stacked on a leading bank axis.
 
-    Large workloads are drawn bank-parallel in a spawn-started process pool
-    (spawn, so that it is safe after a CUDA context exists in the parent).
+    With workers > 1 the banks are drawn in a spawn-started process pool (spawn, so that it is
+    safe after a CUDA context exists in the parent; the caller's main module must be guarded).
     """
     banks = cfg.banks(sub)
-    spec, W = cfg.ffn(sub), cfg.width(sub)
-    per_bank = (3 * spec.hidden * W) if not spec.is_moe else (3 * spec.E * spec.hidden_e * W + 3 * spec.hidden_s * W)
     if workers is None:
-        workers = min(os.cpu_count() or 1, banks, 16) if per_bank * banks > 50_000_000 else 1
+        # a process pool only on request (TM_SYNTH_WORKERS or the argument): spawn-started workers
+        # re-import the caller's main module, which a script without a main guard cannot survive
+        workers = int(os.environ.get("TM_SYNTH_WORKERS", "1"))
+    workers = max(1, min(workers, banks))
     jobs = [(cfg, layer, sub, b, down_scale) for b in range(banks)]
     if workers <= 1:
         parts = [_bank_job(j) for j in jobs]

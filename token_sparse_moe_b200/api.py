@@ -91,10 +91,11 @@ class Block:
         return A.tm_block(self.mix.c(), self.rev.c())
 
 
-def sublayer_from_synth(cfg, layer: int, sub: int, device, down_scale=None, with_gain: bool = False) -> SubLayer:
+def sublayer_from_synth(cfg, layer: int, sub: int, device, down_scale=None, with_gain: bool = False,
+                        workers=None) -> SubLayer:
     import tm_synth
     spec = cfg.ffn(sub)
-    w = tm_synth.sublayer_weights(cfg, layer, sub, down_scale)
+    w = tm_synth.sublayer_weights(cfg, layer, sub, down_scale, workers)
     t = {k: to_device(v, device) for k, v in w.items()}
     g = to_device(tm_synth.gain(cfg, layer, sub), device) if with_gain else None
     if spec.is_moe:
@@ -103,8 +104,9 @@ def sublayer_from_synth(cfg, layer: int, sub: int, device, down_scale=None, with
     return SubLayer(False, cfg.banks(sub), cfg.width(sub), t, hidden=spec.hidden, gain=g)
 
 
-def blocks_from_synth(cfg, device, down_scale=None) -> List[Block]:
-    return [Block(sublayer_from_synth(cfg, l, 0, device, down_scale), sublayer_from_synth(cfg, l, 1, device, down_scale))
+def blocks_from_synth(cfg, device, down_scale=None, workers=None) -> List[Block]:
+    return [Block(sublayer_from_synth(cfg, l, 0, device, down_scale, workers=workers),
+                  sublayer_from_synth(cfg, l, 1, device, down_scale, workers=workers))
             for l in range(cfg.L)]
 
 

@@ -270,11 +270,15 @@ tm_status fused_dense(const Geo& g, const void* x, const void* wg, const void* w
     // One CTA per 128-row tile by default.  TM_FUSED_PAIRS=1 selects the CTA-pair kernel (2-SM
     // MMAs, half the weight bytes per SM); on B200 it measured slower on the dense block workload
     // (0.189 ms against 0.149 ms per sub-layer): its per-chunk handoffs cross the CTA pair.
+    // TM_FUSED64=1 keeps 64-wide hidden chunks where F % 128 == 0 (for comparison only).
     const char* env = getenv("TM_FUSED_PAIRS");
     const bool pairs = g.B > 128 && env && env[0] == '1';
+    const char* env64 = getenv("TM_FUSED64");
+    const bool wide = !pairs && F % 128 == 0 && !(env64 && env64[0] == '1');
+    const uint32_t gu_box = wide ? 128 : 64;
     CUtensorMap ma, mg, mu, md;
     if (!gemm1_amap(g, x, am, &ma)) return TM_ERR_CUDA;
-    if (!map_2d(&mg, wg, (uint64_t)g.banks * F, g.W, 64) || !map_2d(&mu, wu, (uint64_t)g.banks * F, g.W, 64) ||
+    if (!map_2d(&mg, wg, (uint64_t)g.banks * F, g.W, gu_box) || !map_2d(&mu, wu, (uint64_t)g.banks * F, g.W, gu_box) ||
         !map_2d(&md, wd, (uint64_t)g.banks * g.W, F, pairs ? g.W / 2 : g.W))
         return TM_ERR_CUDA;
     FusedParams p;
@@ -297,6 +301,7 @@ tm_status fused_dense(const Geo& g, const void* x, const void* wg, const void* w
     }
     const long tiles = (long)g.banks * mt;
     const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+    if (wide) return cuda_status(launch_fused128(g.W, am, ma, mg, mu, md, p, grid, st));
     return cuda_status(launch_fused(g.W, am, ma, mg, mu, md, p, grid, st));
 }
 

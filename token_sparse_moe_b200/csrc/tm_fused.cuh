@@ -220,70 +220,71 @@ __global__ void __launch_bounds__(FusedCfg<W, AMODE>::NTHREADS, 1)
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
+        // Buffer b (= chunk & 1) is used cnt_b = (NC + 1 - b) / 2 times per tile, so the use index of
+        // chunk c in the tile lt is lt * cnt_b + c / 2; barrier parities follow from it (no arrays).
         if (lane == 0) {
             constexpr uint32_t idesc1 = umma_idesc_bf16(128, 128);
             constexpr uint32_t idesc2 = umma_idesc_bf16(128, W);
+            const uint32_t cnt0 = (NC + 1) >> 1, cnt1 = NC >> 1;
             int s = 0;
             uint32_t ph = 0;
-            uint32_t u1[2] = {0, 0}, u2[2] = {0, 0};   // uses of g1 buffer / hidden buffer b
             int lt = 0;
             bool ok = true;
+            const uint32_t aS = smem_u32(sA);
             for (int t = blockIdx.x; t < ntile && ok; t += gridDim.x, ++lt) {
                 if (!wait_or_abort(a_full, lt & 1, abort_flag, 0x1200)) break;
                 tc_fence_after();
-                const uint32_t aS = smem_u32(sA);
-                auto gemm1 = [&](int c) -> bool {
-                    const int b = c & 1;
-                    if (!wait_or_abort(&g1_empty[b], (u1[b] & 1) ^ 1, abort_flag, 0x1201)) return false;
-                    tc_fence_after();
-                    const uint32_t d = tmem + C::G1COL + b * 128;
-                    for (int q = 0; q < 2; ++q) {
-                        if (!wait_or_abort(&full[s], ph, abort_flag, 0x1202)) return false;
+                // chunk order: G1(0), then for c: G1(c+1), G2(c)
+#pragma unroll 1
+                for (int step = -1; step < NC && ok; ++step) {
+                    // ---- GEMM1 of chunk c1 = step + 1
+                    const int c1 = step + 1;
+                    if (c1 < NC) {
+                        const int b = c1 & 1;
+                        const uint32_t use = lt * (b ? cnt1 : cnt0) + (c1 >> 1);
+                        if (!wait_or_abort(&g1_empty[b], (use & 1) ^ 1, abort_flag, 0x1201)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t d = tmem + C::G1COL + b * 128;
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            if (!wait_or_abort(&full[s], ph, abort_flag, 0x1202)) { ok = false; break; }
+                            tc_fence_after();
+                            const uint32_t st = smem_u32(sR + s * C::SB);
+#pragma unroll
+                            for (int kk = 0; kk < W / 32; ++kk) {
+                                const int k16 = q * (W / 32) + kk;
+                                const uint64_t ad = AMODE == A_TMA_MIX ? umma_sdesc_sw32(aS + k16 * 4096)
+                                                                       : umma_sdesc_sw128(aS + (k16 >> 2) * 16384) + 2 * (k16 & 3);
+                                const uint64_t bd = umma_sdesc_sw128(st + (kk >> 2) * 16384) + 2 * (kk & 3);
+                                umma_bf16(d, ad, bd, idesc1, (q | kk) != 0);
+                            }
+                            umma_commit(&empty[s]);
+                            if (++s == STAGES) { s = 0; ph ^= 1; }
+                        }
+                        if (!ok) break;
+                        umma_commit(&g1_full[b]);
+                        if (c1 == NC - 1) umma_commit(a_empty);       // last read of the A tile issued
+                    }
+                    // ---- GEMM2 of chunk c2 = step
+                    const int c2 = step;
+                    if (c2 >= 0) {
+                        const int b = c2 & 1;
+                        const uint32_t use = lt * (b ? cnt1 : cnt0) + (c2 >> 1);
+                        if (!wait_or_abort(&hid_full[b], use & 1, abort_flag, 0x1203)) { ok = false; break; }
+                        if (c2 == 0 && !wait_or_abort(y_empty, (lt & 1) ^ 1, abort_flag, 0x1204)) { ok = false; break; }
+                        if (!wait_or_abort(&full[s], ph, abort_flag, 0x1205)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t st = smem_u32(sR + s * C::SB);
+                        const uint64_t hd = umma_sdesc_sw128(smem_u32(sH + b * C::HID_BYTES));
+                        const uint64_t bd = umma_sdesc_sw128(st);
 #pragma unroll
-                        for (int kk = 0; kk < W / 32; ++kk) {       // 16-wide K steps inside this stage
-                            const int k16 = q * (W / 32) + kk;
-                            const uint64_t ad = AMODE == A_TMA_MIX ? umma_sdesc_sw32(aS + k16 * 4096)
-                                                                   : umma_sdesc_sw128(aS + (k16 >> 2) * 16384) + 2 * (k16 & 3);
-                            const uint64_t bd = umma_sdesc_sw128(st + (kk >> 2) * 16384) + 2 * (kk & 3);
-                            umma_bf16(d, ad, bd, idesc1, (q | kk) != 0);
-                        }
+                        for (int kk = 0; kk < 4; ++kk) umma_bf16(tmem, hd + 2 * kk, bd + 2 * kk, idesc2, (c2 | kk) != 0);
                         umma_commit(&empty[s]);
+                        umma_commit(&hid_empty[b]);
                         if (++s == STAGES) { s = 0; ph ^= 1; }
+                        if (c2 == NC - 1) umma_commit(y_full);
                     }
-                    umma_commit(&g1_full[b]);
-                    ++u1[b];
-                    return true;
-                };
-                auto gemm2 = [&](int c) -> bool {
-                    const int b = c & 1;
-                    if (!wait_or_abort(&hid_full[b], u2[b] & 1, abort_flag, 0x1203)) return false;
-                    if (c == 0 && !wait_or_abort(y_empty, (lt & 1) ^ 1, abort_flag, 0x1204)) return false;
-                    if (!wait_or_abort(&full[s], ph, abort_flag, 0x1205)) return false;
-                    tc_fence_after();
-                    const uint32_t st = smem_u32(sR + s * C::SB);
-                    const uint64_t hd = umma_sdesc_sw128(smem_u32(sH + b * C::HID_BYTES));
-                    const uint64_t bd = umma_sdesc_sw128(st);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) umma_bf16(tmem, hd + 2 * kk, bd + 2 * kk, idesc2, (c | kk) != 0);
-                    umma_commit(&empty[s]);
-                    umma_commit(&hid_empty[b]);
-                    ++u2[b];
-                    if (++s == STAGES) { s = 0; ph ^= 1; }
-                    return true;
-                };
-                // A is free once the last GEMM1 of the tile has completed
-                ok = gemm1(0);
-                if (ok && NC == 1) umma_commit(a_empty);
-                for (int c = 0; c < NC && ok; ++c) {
-                    if (c + 1 < NC) {
-                        ok = gemm1(c + 1);
-                        if (ok && c + 1 == NC - 1) umma_commit(a_empty);
-                    }
-                    if (ok) ok = gemm2(c);
                 }
-                if (ok) umma_commit(y_full);
             }
             umma_commit(drain);
             wait_or_abort(drain, 0, abort_flag, 0x1206);
@@ -293,7 +294,7 @@ __global__ void __launch_bounds__(FusedCfg<W, AMODE>::NTHREADS, 1)
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
         const int r = q * 32 + lane;
-        uint32_t u1[2] = {0, 0}, u2[2] = {0, 0};
+        const uint32_t cnt0 = (NC + 1) >> 1, cnt1 = NC >> 1;
         int lt = 0;
         for (int t = blockIdx.x; t < ntile; t += gridDim.x, ++lt) {
             const int g = t / mt, m = t - g * mt;
@@ -341,8 +342,8 @@ __global__ void __launch_bounds__(FusedCfg<W, AMODE>::NTHREADS, 1)
 #pragma unroll 1
             for (int c = 0; c < NC; ++c) {
                 const int bb = c & 1;
-                if (!wait_or_abort(&g1_full[bb], u1[bb] & 1, abort_flag, 0x1301)) { ok = false; break; }
-                ++u1[bb];
+                const uint32_t use = lt * (bb ? cnt1 : cnt0) + (c >> 1);
+                if (!wait_or_abort(&g1_full[bb], use & 1, abort_flag, 0x1301)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t ta = tmem + (uint32_t(q * 32) << 16) + C::G1COL + bb * 128 + half * 32;
                 float gv[32], uv[32];
@@ -356,8 +357,7 @@ __global__ void __launch_bounds__(FusedCfg<W, AMODE>::NTHREADS, 1)
                 for (int i = 0; i < 16; ++i)
                     pk[i] = pack_bf16x2(silu_tanh(sc * gv[2 * i]) * (sc * uv[2 * i]),
                                         silu_tanh(sc * gv[2 * i + 1]) * (sc * uv[2 * i + 1]));
-                if (!wait_or_abort(&hid_empty[bb], (u2[bb] & 1) ^ 1, abort_flag, 0x1302)) { ok = false; break; }
-                ++u2[bb];
+                if (!wait_or_abort(&hid_empty[bb], (use & 1) ^ 1, abort_flag, 0x1302)) { ok = false; break; }
                 uint8_t* hrow = sH + bb * C::HID_BYTES + r * 128;
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {

@@ -1,6 +1,7 @@
 // tm_gemm.cu -- instantiations and launchers of the tcgen05 kernels (grouped GEMM, fused sub-layer).
 #include <string.h>
 #include "tm_fused2.cuh"
+#include "tm_fused128.cuh"
 #include "tm_internal.h"
 
 namespace tml {
@@ -19,6 +20,31 @@ static cudaError_t launch_fused_one(const CUtensorMap& a, const CUtensorMap& g, 
     ProfileScope ps_("fused_swiglu", st);
     kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, g, u, d, p);
     return cudaGetLastError();
+}
+
+template <int W, int AM>
+static cudaError_t launch_fused128_one(const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
+                                       const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st) {
+    using C = Fused128Cfg<W, AM>;
+    auto kern = fused128_swiglu_kernel<W, AM>;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    ProfileScope ps_("fused_swiglu", st);
+    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, g, u, d, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fused128(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
+                            const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st) {
+    if (W == 256 && a_mode == A_TMA_MIX) return launch_fused128_one<256, A_TMA_MIX>(a, g, u, d, p, grid, st);
+    if (W == 256 && a_mode == A_TMA_3D) return launch_fused128_one<256, A_TMA_3D>(a, g, u, d, p, grid, st);
+    if (W == 128 && a_mode == A_TMA_MIX) return launch_fused128_one<128, A_TMA_MIX>(a, g, u, d, p, grid, st);
+    if (W == 128 && a_mode == A_TMA_3D) return launch_fused128_one<128, A_TMA_3D>(a, g, u, d, p, grid, st);
+    return cudaErrorInvalidValue;
 }
 
 template <int W, int AM>

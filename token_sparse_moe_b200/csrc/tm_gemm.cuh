@@ -360,7 +360,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
                         ev[i] = (p.extra && in) ? __ldg(reinterpret_cast<const uint4*>(p.extra + off[i])) : make_uint4(0, 0, 0, 0);
                     }
                     if (EPI == EPI_COMBINE) {
-                        for (int j = 0; j < p.k; j += 2) {
+#pragma unroll
+                        for (int j = 0; j < 8; j += 2) {
+                            if (j >= p.k) break;
                             const bool two = j + 1 < p.k;
                             const uint4* s0 = reinterpret_cast<const uint4*>(p.slots + (size_t)spos[j] * p.omap.W + col0);
                             const uint4* s1 = reinterpret_cast<const uint4*>(p.slots + (size_t)spos[two ? j + 1 : j] * p.omap.W + col0);

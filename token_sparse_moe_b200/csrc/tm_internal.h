@@ -36,6 +36,9 @@ bool fused_supported(int W, int a_mode);
 cudaError_t launch_fused(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
                          const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st);
 // CTA-pair version (2-SM MMAs, clusters of 2): grid = 2 x clusters; weight maps with half-size boxes
+// 128-wide hidden chunks (F % 128 == 0); gate/up maps with 128-row boxes
+cudaError_t launch_fused128(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
+                            const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st);
 cudaError_t launch_fused2(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
                           const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st);
 int grouped_gemm_smem(int bn, int a_mode);
