@@ -117,6 +117,29 @@ def test_dense_sublayer(cfg, sub, down_scale):
     check_outputs(cfg, y, o, R64, down_scale)
 
 
+@pytest.mark.parametrize("resid", ["input", "none"])
+@pytest.mark.parametrize("sub", [0, 1])
+@pytest.mark.parametrize("cfg", [DENSE_SMALL[0], DENSE_SMALL[4]], ids=lambda c: c.name)
+def test_dense_sublayer_residual_forms(cfg, sub, resid):
+    """The residual is the sub-layer input itself (the tensor core adds it from the resident input
+    tile) or absent; both against the oracle with R = X and R = 0."""
+    X, _ = inputs(cfg)
+    sw = api.sublayer_from_synth(cfg, 0, sub, DEV)
+    sh = api.config_shape(cfg)
+    layout = A.TM_LAYOUT_MIXED if sub == 0 else A.TM_LAYOUT_ROWS
+    Xd = dev(X)
+    y = api.pertoken_swiglu(Xd, Xd if resid == "input" else None, layout, sh, sw)
+    api.get_device_error()
+    R = X if resid == "input" else np.zeros_like(X)
+    o, _, _ = _oracle_sub(cfg, sub, X, R)
+    if resid == "input":
+        check_outputs(cfg, to_np(y), o, S.to_f64(R), None)
+    else:
+        # no residual: y is the FFN term alone, whose bf16 storage rounding reaches 2^-9 |y| at the
+        # tails (|y| ~ 10 rms), so one ulp of the stored value is allowed first
+        assert err_delta(to_np(y), o, 0.0, cfg.dtype) <= tol(cfg.dtype)
+
+
 @pytest.mark.parametrize("sub", [0, 1])
 @pytest.mark.parametrize("cfg", MOE_SMALL, ids=lambda c: c.name)
 def test_route_topk(cfg, sub):

@@ -274,7 +274,7 @@ tm_status fused_dense(const Geo& g, const void* x, const void* wg, const void* w
     const char* env = getenv("TM_FUSED_PAIRS");
     const bool pairs = g.B > 128 && env && env[0] == '1';
     const char* env64 = getenv("TM_FUSED64");
-    const bool wide = !pairs && F % 128 == 0 && !(env64 && env64[0] == '1');
+    const bool wide = !pairs && F % 128 == 0 && !(env64 && env64[0] == '1') && (uintptr_t)y % 32 == 0;
     const uint32_t gu_box = wide ? 128 : 64;
     CUtensorMap ma, mg, mu, md;
     if (!gemm1_amap(g, x, am, &ma)) return TM_ERR_CUDA;
@@ -301,7 +301,18 @@ tm_status fused_dense(const Geo& g, const void* x, const void* wg, const void* w
     }
     const long tiles = (long)g.banks * mt;
     const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-    if (wide) return cuda_status(launch_fused128(g.W, am, ma, mg, mu, md, p, grid, st));
+    if (wide) {
+        // residual: the A tile itself when it is the sub-layer input (same tensor, same row map),
+        // else streamed with the A geometry; the inter-residual likewise
+        CUtensorMap mr, me;
+        memset(&mr, 0, sizeof(mr));
+        memset(&me, 0, sizeof(me));
+        p.res_mode = resid == nullptr ? RES_NONE : resid == x ? RES_FROM_A : RES_STREAM;
+        p.has_extra = extra != nullptr;
+        if (p.res_mode == RES_STREAM && !gemm1_amap(g, resid, am, &mr)) return TM_ERR_CUDA;
+        if (p.has_extra && !gemm1_amap(g, extra, am, &me)) return TM_ERR_CUDA;
+        return cuda_status(launch_fused128(g.W, am, ma, mg, mu, md, mr, me, p, grid, st));
+    }
     return cuda_status(launch_fused(g.W, am, ma, mg, mu, md, p, grid, st));
 }
 

@@ -28,6 +28,8 @@ struct FusedParams {
     const __nv_bfloat16* extra;
     RowMap omap;
     size_t out_elems;
+    int res_mode;              // 128-wide-chunk kernel: residual none / from the A tile / streamed (FusedResid)
+    int has_extra;             // 128-wide-chunk kernel: inter-residual streamed
 };
 
 // Output epilogue of a fused tile for one thread: row b of bank g, columns [c_begin, c_begin + W/2).

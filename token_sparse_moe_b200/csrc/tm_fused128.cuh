@@ -6,13 +6,18 @@
 //   epilogue: h = silu(s*g) * (s*u)  -> bf16 chunk in shared memory (s = 1/rms of the row)
 //   GEMM2(c): TMEM Y += h . Wd[:, chunk c]^T       (N = W, K = 128)
 // issued in the order G1(0), G1(1), G2(0), G1(2), G2(1), ...: the epilogue copies g1 out of TMEM
-// while the tensor pipe runs G2(c-1) (so GEMM1 needs only one TMEM buffer) and computes the
-// SwiGLU while it runs G1(c+1).  TMEM: Y in columns [0, W), the GEMM1 buffer in [256, 512).
+// and releases it at once, so G1(c+1) queues behind G2(c-1) while the SwiGLU of chunk c runs.
+// TMEM: Y in columns [0, W), the GEMM1 buffer in [256, 512).
 //
-// The output epilogue is coalesced: residual slices are read 8 rows per warp instruction (4 lanes
-// per 64-byte row piece), prefetched before the accumulator is ready, transposed to one row per
-// thread through the warp's own rows of the (then idle) hidden buffer, added to the accumulator
-// in fp32 with a single rounding, and written back the same way.
+// The residual is added by the tensor core: before GEMM2(0) the accumulator Y is initialised with
+// the residual tile times a 16 x 16 identity (one N = 16 MMA per 16 columns; bf16 times one summed
+// in fp32 is exact).  When the residual is the sub-layer input itself (the mixing sub-layer) the
+// resident A tile is that operand; otherwise the residual tile, and the inter-residual of a gap
+// layer, stream through the weight ring with the same tensor-map geometry as A.  The output
+// epilogue is then only TMEM -> bf16 -> global, with 32-byte stores (one full sector per lane).
+//
+// The row statistics of the next tile are computed while this tile's last GEMM2 runs, so the
+// epilogue warps go from the output of tile t straight to the SwiGLU of tile t+1.
 //
 // Warp roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner, warps 2-9 epilogue
 // (TMEM lane quarter = warp % 4; warps 2-5 / 6-9 take the two column halves).
@@ -20,6 +25,8 @@
 #include "tm_fused.cuh"
 
 namespace tml {
+
+enum FusedResid : int { RES_NONE = 0, RES_FROM_A = 1, RES_STREAM = 2 };
 
 template <int W, int AMODE>
 struct Fused128Cfg {
@@ -29,21 +36,30 @@ struct Fused128Cfg {
     static constexpr int SB = 32768;                              // ring stage
     static constexpr int G1_STAGES = W / 64;                      // 256 rows x 64 K per stage
     static constexpr int G2_STAGES = W == 256 ? 2 : 1;            // W rows x 128 K per chunk
+    static constexpr int R_STAGES = W / 128;                      // residual tile: 128 rows x 128 columns per stage
     static constexpr int STAGES = W == 256 ? 4 : 5;
     static constexpr int NTHREADS = 10 * 32;
     static constexpr int OFF_HID = A_BYTES;
     static constexpr int OFF_RING = A_BYTES + HID_BYTES;
-    static constexpr int OFF_BAR = OFF_RING + STAGES * SB;
+    static constexpr int OFF_ID = OFF_RING + STAGES * SB;         // 16 x 16 identity, 32-byte swizzled K-major
+    static constexpr int OFF_BAR = OFF_ID + 1024;
     static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
     static constexpr int G1COL = 256;
-    static_assert(2 * 32 * 64 <= 4096, "output staging (residual + inter-residual) fits in a warp's hidden rows");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
+
+// 16 consecutive bf16 (32 bytes, one sector) from 8 packed words; p must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                 "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
 
 template <int W, int AMODE>
 __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
     fused128_swiglu_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
                            const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmD,
+                           const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmE,
                            const FusedParams p) {
     using C = Fused128Cfg<W, AMODE>;
     constexpr int STAGES = C::STAGES;
@@ -51,12 +67,15 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
     const int ntile = p.banks * mt;
     if ((int)blockIdx.x >= ntile) return;
     const int NC = p.F / 128;
+    const int res_stages = p.res_mode == RES_STREAM ? C::R_STAGES : 0;
+    const int ext_stages = p.has_extra ? C::R_STAGES : 0;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sH = smem + C::OFF_HID;
     uint8_t* sR = smem + C::OFF_RING;
+    uint8_t* sI = smem + C::OFF_ID;
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* full = bar;                  // [STAGES]
     uint64_t* empty = full + STAGES;       // [STAGES]
@@ -80,7 +99,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(a_full, 1);
-        mbar_init(a_empty, 1 + 8);             // MMA (last GEMM1 done) + each epilogue warp (statistics read)
+        mbar_init(a_empty, 1 + 8);             // MMA (last read of A issued) + each epilogue warp (statistics)
         mbar_init(g1_full, 1);
         mbar_init(g1_empty, 8);
         mbar_init(hid_full, 8);
@@ -90,6 +109,16 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
+    }
+    if (warp == 2) {
+        // identity B operand: 16 rows n x 16 columns k, 32-byte rows, 32-byte swizzle (the 16-byte
+        // half of row n that holds column k sits at half (k / 8) ^ ((n / 4) % 2))
+        const int n = lane & 15, hf = lane >> 4;
+        const uint32_t one = (n >> 3) == hf ? ((n & 1) ? 0x3F800000u : 0x00003F80u) : 0u;
+        const int wi = (n & 7) >> 1;
+        *reinterpret_cast<uint4*>(sI + n * 32 + ((hf ^ ((n >> 2) & 1)) << 4)) =
+            make_uint4(wi == 0 ? one : 0u, wi == 1 ? one : 0u, wi == 2 ? one : 0u, wi == 3 ? one : 0u);
+        fence_proxy_async_smem();
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -111,22 +140,27 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             uint32_t ph = 0;
             int lt = 0;
             bool ok = true;
+            // 128 rows x (16 * n16) columns from column 16 * col16 of a row tensor, in the A geometry
+            auto load_rows = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* b, int g, int m0, int col16, int n16) {
+                if (AMODE == A_TMA_MIX) {
+                    const int per = p.amap.dh >> 4;
+#pragma unroll 1
+                    for (int i = 0; i < n16; ++i) {
+                        const int ci = col16 + i, tok = ci / per, jj = ci - tok * per;
+                        tma_load_4d(dst + i * 4096, map, b, 0, g * per + jj, tok, m0);
+                    }
+                } else {
+#pragma unroll 1
+                    for (int i = 0; i < n16 / 4; ++i) tma_load_3d(dst + i * 16384, map, b, col16 * 16 + i * 64, g, m0);
+                }
+            };
             for (int t = blockIdx.x; t < ntile && ok; t += gridDim.x, ++lt) {
                 const int g = t / mt, m = t - g * mt;
                 if (!wait_or_abort(a_empty, (lt & 1) ^ 1, abort_flag, 0x3100)) break;
                 mbar_arrive_expect_tx(a_full, C::A_BYTES);
-                if (AMODE == A_TMA_MIX) {
-                    const int per = p.amap.dh >> 4;
-#pragma unroll 1
-                    for (int i = 0; i < W / 16; ++i) {
-                        const int tok = i / per, jj = i - tok * per;
-                        tma_load_4d(sA + i * 4096, &tmA, a_full, 0, g * per + jj, tok, m * 128);
-                    }
-                } else {
-#pragma unroll 1
-                    for (int i = 0; i < W / 64; ++i) tma_load_3d(sA + i * 16384, &tmA, a_full, i * 64, g, m * 128);
-                }
-                // weights in MMA order: G1(0); then for c >= 1: G1(c), G2(c-1); finally G2(NC-1)
+                load_rows(&tmA, sA, a_full, g, m * 128, 0, W / 16);
+                // ring order: G1(0); then for step >= 1: G1(step) (step < NC), the residual and
+                // inter-residual tiles (step 1 only), G2(step - 1)
 #pragma unroll 1
                 for (int step = 0; step <= NC && ok; ++step) {
                     if (step < NC) {
@@ -138,6 +172,17 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             mbar_arrive_expect_tx(&full[s], C::SB);
                             tma_load_2d(st, &tmG, &full[s], q * 64, g * p.F + c * 128);
                             tma_load_2d(st + 16384, &tmU, &full[s], q * 64, g * p.F + c * 128);
+                            if (++s == STAGES) { s = 0; ph ^= 1; }
+                        }
+                    }
+                    if (step == 1 && ok) {
+#pragma unroll 1
+                        for (int i = 0; i < res_stages + ext_stages; ++i) {    // 128 columns per stage
+                            if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x3103)) { ok = false; break; }
+                            uint8_t* st = sR + s * C::SB;
+                            mbar_arrive_expect_tx(&full[s], C::SB);
+                            const int q = i < res_stages ? i : i - res_stages;
+                            load_rows(i < res_stages ? &tmR : &tmE, st, &full[s], g, m * 128, q * 8, 8);
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                     }
@@ -165,6 +210,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         if (lane == 0) {
             constexpr uint32_t idesc1 = umma_idesc_bf16(128, 256);
             constexpr uint32_t idesc2 = umma_idesc_bf16(128, W);
+            constexpr uint32_t idescI = umma_idesc_bf16(128, 16);
             const uint32_t aS = smem_u32(sA), hS = smem_u32(sH), rS = smem_u32(sR);
             uint64_t adesc[W / 16];
 #pragma unroll
@@ -173,7 +219,13 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                                                 : umma_sdesc_sw128(aS + (k16 >> 2) * 16384) + 2 * (k16 & 3);
             const uint64_t hdesc0 = umma_sdesc_sw128(hS), hdesc1 = umma_sdesc_sw128(hS + 16384);
             const uint64_t rdesc0 = umma_sdesc_sw128(rS);
+            const uint64_t rdesc32 = umma_sdesc_sw32(rS);
+            const uint64_t idB = umma_sdesc_sw32(smem_u32(sI));
             constexpr uint64_t kStageDesc = C::SB >> 4;               // descriptor start-address step per stage
+            const bool y_init = p.res_mode != RES_NONE || p.has_extra;
+            // the A tile is released after the last step that reads it: GEMM1(NC-1), and the
+            // identity pass of step 1 when the residual comes from A
+            const int a_last = (p.res_mode == RES_FROM_A && NC < 2) ? 1 : NC - 1;
             int s = 0;
             uint32_t ph = 0;
             int lt = 0;
@@ -200,13 +252,38 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                         }
                         if (!ok) break;
                         umma_commit(g1_full);
-                        if (step == NC - 1) umma_commit(a_empty);
                     }
                     if (step >= 1) {                                   // ---- GEMM2(step - 1)
                         const int c = step - 1;
                         const uint32_t use = lt * NC + c;
+                        if (c == 0) {
+                            // Y free (previous tile read out), then Y = residual (+ inter-residual)
+                            if (!wait_or_abort(y_empty, (lt & 1) ^ 1, abort_flag, 0x3204)) { ok = false; break; }
+                            tc_fence_after();
+                            if (p.res_mode == RES_FROM_A) {
+#pragma unroll
+                                for (int k16 = 0; k16 < W / 16; ++k16) umma_bf16(tmem + 16 * k16, adesc[k16], idB, idescI, 0);
+                            }
+#pragma unroll 1
+                            for (int i = 0; i < res_stages + ext_stages; ++i) {
+                                if (!wait_or_abort(&full[s], ph, abort_flag, 0x3207)) { ok = false; break; }
+                                tc_fence_after();
+                                const uint32_t acc = (i >= res_stages && p.res_mode != RES_NONE) ? 1u : 0u;
+                                const int q = i < res_stages ? i : i - res_stages;
+                                const uint32_t st = rS + s * C::SB;
+#pragma unroll
+                                for (int k16 = 0; k16 < 8; ++k16) {
+                                    const uint64_t rd = AMODE == A_TMA_MIX
+                                                            ? rdesc32 + (uint64_t)s * kStageDesc + k16 * (4096 >> 4)
+                                                            : umma_sdesc_sw128(st + (k16 >> 2) * 16384) + 2 * (k16 & 3);
+                                    umma_bf16(tmem + 16 * (q * 8 + k16), rd, idB, idescI, acc);
+                                }
+                                umma_commit(&empty[s]);
+                                if (++s == STAGES) { s = 0; ph ^= 1; }
+                            }
+                            if (!ok) break;
+                        }
                         if (!wait_or_abort(hid_full, use & 1, abort_flag, 0x3203)) { ok = false; break; }
-                        if (c == 0 && !wait_or_abort(y_empty, (lt & 1) ^ 1, abort_flag, 0x3204)) { ok = false; break; }
 #pragma unroll
                         for (int q = 0; q < C::G2_STAGES; ++q) {
                             if (!wait_or_abort(&full[s], ph, abort_flag, 0x3205)) { ok = false; break; }
@@ -218,7 +295,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
 #pragma unroll
                                 for (int kk = 0; kk < 4; ++kk)
                                     umma_bf16(tmem, hd + 2 * kk, bd + kq * (16384 >> 4) + 2 * kk, idesc2,
-                                              (c | q | kq | kk) != 0);
+                                              (y_init || (c | q | kq | kk) != 0) ? 1u : 0u);
                             }
                             umma_commit(&empty[s]);
                             if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -227,6 +304,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                         umma_commit(hid_empty);
                         if (c == NC - 1) umma_commit(y_full);
                     }
+                    if (step == a_last) umma_commit(a_empty);
                 }
             }
             umma_commit(drain);
@@ -238,16 +316,8 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         const int half = (warp - 2) >> 2;
         const int r = q * 32 + lane;
         const uint32_t trow = tmem + (uint32_t(q * 32) << 16);
-        // output staging: inside this warp's own 32 rows of the hidden buffer (4 KB per half and
-        // lane quarter), which no other warp writes and the MMA no longer reads after y_full
-        uint8_t* stg = sH + half * 16384 + q * 4096;
-        int lt = 0;
-        for (int t = blockIdx.x; t < ntile; t += gridDim.x, ++lt) {
-            const int g = t / mt, m = t - g * mt;
-            const int nrows = min(128, p.rows - m * 128);
-            const bool valid = r < nrows;
-            if (!wait_or_abort(a_full, lt & 1, abort_flag, 0x3300)) break;
-            // ---- row statistics from the resident A tile (each warp reads its rows in full)
+        // 1/rms of this thread's row of the tile in the A buffer (0 for rows past the end)
+        auto row_scale = [&](int m_tile) -> float {
             float ss = 0.f;
             if (AMODE == A_TMA_MIX) {
 #pragma unroll 4
@@ -279,30 +349,47 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                     }
                 }
             }
-            const float sc = valid ? 1.0f / sqrtf(ss / (float)W + p.eps) : 0.f;
+            return r < p.rows - m_tile * 128 ? 1.0f / sqrtf(ss / (float)W + p.eps) : 0.f;
+        };
+        int lt = 0;
+        float sc = 0.f;
+        bool ok = wait_or_abort(a_full, 0, abort_flag, 0x3300);
+        if (ok) {
+            sc = row_scale((int)blockIdx.x % mt);
             __syncwarp();
             if (lane == 0) mbar_arrive(a_empty);
+        }
+        for (int t = blockIdx.x; t < ntile && ok; t += gridDim.x, ++lt) {
+            const int g = t / mt, m = t - g * mt;
+            const int nrows = min(128, p.rows - m * 128);
             // ---- SwiGLU chunks: this thread owns hidden columns [half*64, half*64 + 64) of its row
-            bool ok = true;
 #pragma unroll 1
             for (int c = 0; c < NC; ++c) {
                 const uint32_t use = lt * NC + c;
                 if (!wait_or_abort(g1_full, use & 1, abort_flag, 0x3301)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t pk[32];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float gv[32], uv[32];
-                    tmem_ld32(trow + C::G1COL + half * 64 + hh * 32, gv);
-                    tmem_ld32(trow + C::G1COL + 128 + half * 64 + hh * 32, uv);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        pk[hh * 16 + i] = pack_bf16x2(silu_tanh(sc * gv[2 * i]) * (sc * uv[2 * i]),
-                                                      silu_tanh(sc * gv[2 * i + 1]) * (sc * uv[2 * i + 1]));
-                }
+                // all four loads in flight, one wait, then the GEMM1 buffer is released before the math
+                uint32_t g0[32], u0[32], g1[32], u1[32];
+                const uint32_t tg = trow + C::G1COL + half * 64;
+                tmem_ld32_async(tg, g0);
+                tmem_ld32_async(tg + 128, u0);
+                tmem_ld32_async(tg + 32, g1);
+                tmem_ld32_async(tg + 160, u1);
+                tmem_wait_ld_tie(g0);
+                tmem_wait_ld_tie(u0);
+                tmem_wait_ld_tie(g1);
+                tmem_wait_ld_tie(u1);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(g1_empty);
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    pk[i] = pack_bf16x2(silu_tanh(sc * __uint_as_float(g0[2 * i])) * (sc * __uint_as_float(u0[2 * i])),
+                                        silu_tanh(sc * __uint_as_float(g0[2 * i + 1])) * (sc * __uint_as_float(u0[2 * i + 1])));
+                    pk[16 + i] = pack_bf16x2(silu_tanh(sc * __uint_as_float(g1[2 * i])) * (sc * __uint_as_float(u1[2 * i])),
+                                             silu_tanh(sc * __uint_as_float(g1[2 * i + 1])) * (sc * __uint_as_float(u1[2 * i + 1])));
+                }
                 if (!wait_or_abort(hid_empty, (use & 1) ^ 1, abort_flag, 0x3302)) { ok = false; break; }
                 // hidden chunk: 2 K-slabs of 64 columns (128-byte swizzled rows); this half is slab `half`
                 uint8_t* hrow = sH + half * 16384 + r * 128;
@@ -315,74 +402,37 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                 if (lane == 0) mbar_arrive(hid_full);
             }
             if (!ok) break;
-            // ---- output tile, coalesced: lane l moves 16 bytes of row (i*8 + l/4) of a 32-column slice.
-            // Staging rows are 64 bytes with the 16-byte piece index XORed by (row / 2) % 4, so both the
-            // 8-rows-per-instruction phase and the row-per-thread phase are free of bank conflicts.
-            const int c_begin = half * (W / 2);
-            const int b_warp = m * 128 + q * 32;                      // first row of this warp
-            const int lr = lane >> 2, lp = lane & 3;
-            uint8_t* stg_e = stg + 32 * 64;                            // inter-residual slice
-            uint4 rv[W / 16];                                          // W/64 slices x 4 row groups
-#pragma unroll
-            for (int j = 0; j < W / 64; ++j)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int rr = i * 8 + lr;
-                    rv[j * 4 + i] = make_uint4(0, 0, 0, 0);
-                    if (p.resid && q * 32 + rr < nrows) {
-                        const size_t off = row_elem(p.omap, b_warp + rr, g, c_begin + j * 32 + lp * 8);
-                        if (off + 8 <= p.out_elems) rv[j * 4 + i] = __ldg(reinterpret_cast<const uint4*>(p.resid + off));
-                    }
-                }
+            // ---- statistics of the next tile (its A tile is loaded once this tile's last read of A is issued)
+            if (t + (int)gridDim.x < ntile) {
+                if (!wait_or_abort(a_full, (lt + 1) & 1, abort_flag, 0x3304)) break;
+                sc = row_scale((t + (int)gridDim.x) % mt);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(a_empty);
+            }
+            // ---- output tile: Y (residual already accumulated) -> bf16, 32 bytes per store
             if (!wait_or_abort(y_full, lt & 1, abort_flag, 0x3303)) break;
             tc_fence_after();
+            const int b = m * 128 + r;
+            const bool valid = r < nrows;
 #pragma unroll
             for (int j = 0; j < W / 64; ++j) {
-                float v[32];
-                tmem_ld32(trow + c_begin + j * 32, v);
+                uint32_t v[32];
+                tmem_ld32_async(trow + half * (W / 2) + j * 32, v);
+                tmem_wait_ld_tie(v);
+                if (!valid) continue;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int rr = i * 8 + lr;
-                    const int so = rr * 64 + ((lp ^ ((rr >> 1) & 3)) << 4);
-                    *reinterpret_cast<uint4*>(stg + so) = rv[j * 4 + i];
-                    if (p.extra) {
-                        uint4 e4 = make_uint4(0, 0, 0, 0);
-                        if (q * 32 + rr < nrows) {
-                            const size_t off = row_elem(p.omap, b_warp + rr, g, c_begin + j * 32 + lp * 8);
-                            if (off + 8 <= p.out_elems) e4 = __ldg(reinterpret_cast<const uint4*>(p.extra + off));
-                        }
-                        *reinterpret_cast<uint4*>(stg_e + so) = e4;
-                    }
-                }
-                __syncwarp();
-                // one row per thread: Y + residual (+ inter-residual) in fp32, one rounding, back in place
-#pragma unroll
-                for (int pp = 0; pp < 4; ++pp) {
-                    const int so = lane * 64 + ((pp ^ ((lane >> 1) & 3)) << 4);
-                    const uint4 x4 = *reinterpret_cast<const uint4*>(stg + so);
-                    const uint4 e4 = p.extra ? *reinterpret_cast<const uint4*>(stg_e + so) : make_uint4(0, 0, 0, 0);
-                    const uint32_t a[4] = {x4.x, x4.y, x4.z, x4.w}, e[4] = {e4.x, e4.y, e4.z, e4.w};
-                    uint32_t o[4];
-#pragma unroll
-                    for (int z = 0; z < 4; ++z)
-                        o[z] = pack_bf16x2(v[pp * 8 + 2 * z] + bf16_lo(a[z]) + bf16_lo(e[z]),
-                                           v[pp * 8 + 2 * z + 1] + bf16_hi(a[z]) + bf16_hi(e[z]));
-                    *reinterpret_cast<uint4*>(stg + so) = make_uint4(o[0], o[1], o[2], o[3]);
-                }
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int rr = i * 8 + lr;
-                    if (q * 32 + rr >= nrows) continue;
-                    const size_t off = row_elem(p.omap, b_warp + rr, g, c_begin + j * 32 + lp * 8);
-                    if (off + 8 > p.out_elems) {
+                for (int h = 0; h < 2; ++h) {
+                    const size_t off = row_elem(p.omap, b, g, half * (W / 2) + j * 32 + h * 16);
+                    if (off + 16 > p.out_elems) {
                         record_error(ERR_BOUNDS, 0x3310);
                         continue;
                     }
-                    *reinterpret_cast<uint4*>(p.out + off) =
-                        *reinterpret_cast<const uint4*>(stg + rr * 64 + ((lp ^ ((rr >> 1) & 3)) << 4));
+                    uint32_t w[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(v[h * 16 + 2 * e]), __uint_as_float(v[h * 16 + 2 * e + 1]));
+                    st_global_v8(p.out + off, w);
                 }
-                __syncwarp();
             }
             tc_fence_before();
             __syncwarp();
