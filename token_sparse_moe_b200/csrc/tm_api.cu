@@ -169,18 +169,18 @@ int gemm1_amode(const Geo& g) {
     if (g.map.layout == 0) return A_TMA_3D;
     return (g.map.dh % 16 == 0) ? A_TMA_MIX : A_GATHER;
 }
-bool gemm1_amap(const Geo& g, const void* x, int amode, CUtensorMap* m) {
+bool gemm1_amap(const Geo& g, const void* x, int amode, CUtensorMap* m, uint32_t box_rows = 128) {
     if (amode == A_TMA_3D) {
         uint64_t dims[3] = {(uint64_t)g.W, (uint64_t)g.banks, (uint64_t)g.B};
         uint64_t strides[2] = {(uint64_t)g.W * 2, (uint64_t)g.banks * g.W * 2};
-        uint32_t box[3] = {64, 1, 128};
+        uint32_t box[3] = {64, 1, box_rows};
         return make_map(m, x, 3, dims, strides, box);
     }
     if (amode == A_TMA_MIX) {
         const RowMap& r = g.map;
         uint64_t dims[4] = {16, (uint64_t)r.D / 16, (uint64_t)r.T, (uint64_t)g.B};
         uint64_t strides[3] = {32, (uint64_t)r.D * 2, (uint64_t)r.T * r.D * 2};
-        uint32_t box[4] = {16, 1, 1, 128};
+        uint32_t box[4] = {16, 1, 1, box_rows};
         return make_map(m, x, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B);
     }
     memset(m, 0, sizeof(*m));
@@ -311,7 +311,10 @@ tm_status fused_dense(const Geo& g, const void* x, const void* wg, const void* w
         p.has_extra = extra != nullptr;
         if (p.res_mode == RES_STREAM && !gemm1_amap(g, resid, am, &mr)) return TM_ERR_CUDA;
         if (p.has_extra && !gemm1_amap(g, extra, am, &me)) return TM_ERR_CUDA;
-        return cuda_status(launch_fused128(g.W, am, ma, mg, mu, md, mr, me, p, grid, st));
+        // output: the same row geometry, 32-row boxes (one per epilogue warp)
+        CUtensorMap mo;
+        if (!gemm1_amap(g, y, am, &mo, 32)) return TM_ERR_CUDA;
+        return cuda_status(launch_fused128(g.W, am, ma, mg, mu, md, mr, me, mo, p, grid, st));
     }
     return cuda_status(launch_fused(g.W, am, ma, mg, mu, md, p, grid, st));
 }

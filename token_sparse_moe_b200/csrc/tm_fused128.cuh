@@ -16,11 +16,14 @@
 // layer, stream through the weight ring with the same tensor-map geometry as A.  The output
 // epilogue is then only TMEM -> bf16 -> global, with 32-byte stores (one full sector per lane).
 //
-// The row statistics of the next tile are computed while this tile's last GEMM2 runs, so the
-// epilogue warps go from the output of tile t straight to the SwiGLU of tile t+1.
+// The epilogue warps are software-pipelined across tiles: after the last hidden chunk of tile t
+// they compute the row statistics of tile t+1 (its A tile is already loaded), run the SwiGLU of
+// chunk 0 of t+1 (which releases the GEMM1 buffer for GEMM1(1) of t+1), and only then read Y of
+// tile t out, so the tensor pipe has GEMM1 work for t+1 while Y of t drains.
 //
-// Warp roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner, warps 2-9 epilogue
-// (TMEM lane quarter = warp % 4; warps 2-5 / 6-9 take the two column halves).
+// Warp roles: warp 0 TMA producer (and builds the identity tile), warp 1 MMA issuer and TMEM
+// owner, warps 2-9 epilogue (TMEM lane quarter = warp % 4; warps 2-5 / 6-9 take the two column
+// halves).
 #pragma once
 #include "tm_fused.cuh"
 
@@ -42,7 +45,8 @@ struct Fused128Cfg {
     static constexpr int OFF_HID = A_BYTES;
     static constexpr int OFF_RING = A_BYTES + HID_BYTES;
     static constexpr int OFF_ID = OFF_RING + STAGES * SB;         // 16 x 16 identity, 32-byte swizzled K-major
-    static constexpr int OFF_BAR = OFF_ID + 1024;
+    static constexpr int OFF_XCH = OFF_ID + 512;                  // row statistics exchange, 2 x 128 floats
+    static constexpr int OFF_BAR = OFF_XCH + 1024;
     static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
     static constexpr int G1COL = 256;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -60,7 +64,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
     fused128_swiglu_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
                            const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmD,
                            const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmE,
-                           const FusedParams p) {
+                           const __grid_constant__ CUtensorMap tmO, const FusedParams p) {
     using C = Fused128Cfg<W, AMODE>;
     constexpr int STAGES = C::STAGES;
     const int mt = (p.rows + 127) / 128;
@@ -88,7 +92,9 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
     uint64_t* y_full = hid_empty + 1;
     uint64_t* y_empty = y_full + 1;
     uint64_t* drain = y_empty + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* stats_bar = drain + 1;       // both halves' partial row sums written
+    uint64_t* stats_done = stats_bar + 1;  // both halves' partial row sums read
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stats_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -107,10 +113,12 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         mbar_init(y_full, 1);
         mbar_init(y_empty, 8);
         mbar_init(drain, 1);
+        mbar_init(stats_bar, 8);
+        mbar_init(stats_done, 8);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 2) {
+    if (warp == 0) {
         // identity B operand: 16 rows n x 16 columns k, 32-byte rows, 32-byte swizzle (the 16-byte
         // half of row n that holds column k sits at half (k / 8) ^ ((n / 4) % 2))
         const int n = lane & 15, hf = lane >> 4;
@@ -207,6 +215,9 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
+        // Barrier checks are batched: the GEMM1 buffer barrier and all stages of a GEMM1 (or the
+        // hidden barrier and the stages of a GEMM2) are tested together without blocking, so their
+        // latencies overlap; only a stage that is not ready yet is waited for on its own.
         if (lane == 0) {
             constexpr uint32_t idesc1 = umma_idesc_bf16(128, 256);
             constexpr uint32_t idesc2 = umma_idesc_bf16(128, W);
@@ -237,12 +248,25 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                 for (int step = 0; step <= NC && ok; ++step) {
                     if (step < NC) {                                   // ---- GEMM1(step)
                         const uint32_t use = lt * NC + step;
-                        if (!wait_or_abort(g1_empty, (use & 1) ^ 1, abort_flag, 0x3201)) { ok = false; break; }
+                        bool rdy[C::G1_STAGES];
+                        const bool e_rdy = mbar_test(g1_empty, (use & 1) ^ 1);
+                        {
+                            int ss = s;
+                            uint32_t pp = ph;
+#pragma unroll
+                            for (int q = 0; q < C::G1_STAGES; ++q) {
+                                rdy[q] = mbar_test(&full[ss], pp);
+                                if (++ss == STAGES) { ss = 0; pp ^= 1; }
+                            }
+                        }
+                        if (!e_rdy && !wait_or_abort(g1_empty, (use & 1) ^ 1, abort_flag, 0x3201)) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
                         for (int q = 0; q < C::G1_STAGES; ++q) {
-                            if (!wait_or_abort(&full[s], ph, abort_flag, 0x3202)) { ok = false; break; }
-                            tc_fence_after();
+                            if (!rdy[q]) {
+                                if (!wait_or_abort(&full[s], ph, abort_flag, 0x3202)) { ok = false; break; }
+                                tc_fence_after();
+                            }
                             const uint64_t bd = rdesc0 + (uint64_t)s * kStageDesc;
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
@@ -283,11 +307,25 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             }
                             if (!ok) break;
                         }
-                        if (!wait_or_abort(hid_full, use & 1, abort_flag, 0x3203)) { ok = false; break; }
+                        bool rdy[C::G2_STAGES];
+                        const bool h_rdy = mbar_test(hid_full, use & 1);
+                        {
+                            int ss = s;
+                            uint32_t pp = ph;
+#pragma unroll
+                            for (int q = 0; q < C::G2_STAGES; ++q) {
+                                rdy[q] = mbar_test(&full[ss], pp);
+                                if (++ss == STAGES) { ss = 0; pp ^= 1; }
+                            }
+                        }
+                        if (!h_rdy && !wait_or_abort(hid_full, use & 1, abort_flag, 0x3203)) { ok = false; break; }
+                        tc_fence_after();
 #pragma unroll
                         for (int q = 0; q < C::G2_STAGES; ++q) {
-                            if (!wait_or_abort(&full[s], ph, abort_flag, 0x3205)) { ok = false; break; }
-                            tc_fence_after();
+                            if (!rdy[q]) {
+                                if (!wait_or_abort(&full[s], ph, abort_flag, 0x3205)) { ok = false; break; }
+                                tc_fence_after();
+                            }
                             const uint64_t bd = rdesc0 + (uint64_t)s * kStageDesc;
 #pragma unroll
                             for (int kq = 0; kq < (W == 256 ? 1 : 2); ++kq) {   // 64-wide K slabs in this stage
@@ -316,16 +354,21 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         const int half = (warp - 2) >> 2;
         const int r = q * 32 + lane;
         const uint32_t trow = tmem + (uint32_t(q * 32) << 16);
-        // 1/rms of this thread's row of the tile in the A buffer (0 for rows past the end)
-        auto row_scale = [&](int m_tile) -> float {
+        float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);      // [half][row] partial sums of squares
+        uint8_t* stg = sH + half * 16384 + q * 4096;                  // this warp's 32 rows of the hidden buffer
+        int n_stats = 0;
+        // 1/rms of this thread's row of the tile in the A buffer (0 for rows past the end).  Each half
+        // sums the squares of its half of the row; the two partials meet in shared memory and are
+        // added in the same order by both threads of the row.
+        auto row_scale = [&](int m_tile, float& out) -> bool {
             float ss = 0.f;
             if (AMODE == A_TMA_MIX) {
 #pragma unroll 4
-                for (int i = 0; i < W / 16; ++i) {
-                    const uint4* rp = reinterpret_cast<const uint4*>(sA + i * 4096 + r * 32);
+                for (int i = 0; i < W / 32; ++i) {
+                    const uint4* rp = reinterpret_cast<const uint4*>(sA + (half * (W / 32) + i) * 4096 + r * 32);
 #pragma unroll
                     for (int v = 0; v < 2; ++v) {
-                        const uint4 w4 = rp[v ^ half];
+                        const uint4 w4 = rp[v];
                         const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -336,10 +379,11 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                 }
             } else {
 #pragma unroll 1
-                for (int i = 0; i < W / 64; ++i) {
+                for (int i = 0; i < W / 128; ++i) {
 #pragma unroll
                     for (int v = 0; v < 8; ++v) {
-                        const uint4 w4 = *reinterpret_cast<const uint4*>(sA + i * 16384 + r * 128 + (((v ^ r) & 7) << 4));
+                        const uint4 w4 = *reinterpret_cast<const uint4*>(sA + (half * (W / 128) + i) * 16384 + r * 128 +
+                                                                         (((v ^ r) & 7) << 4));
                         const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -349,19 +393,28 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                     }
                 }
             }
-            return r < p.rows - m_tile * 128 ? 1.0f / sqrtf(ss / (float)W + p.eps) : 0.f;
+            // the other half has read the previous round's partial before this one overwrites it
+            if (n_stats > 0 && !wait_or_abort(stats_done, (n_stats - 1) & 1, abort_flag, 0x3305)) return false;
+            xch[half * 128 + r] = ss;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(stats_bar);
+            if (!wait_or_abort(stats_bar, n_stats & 1, abort_flag, 0x3306)) return false;
+            const float tot = xch[r] + xch[128 + r];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(stats_done);
+            ++n_stats;
+            out = r < p.rows - m_tile * 128 ? 1.0f / sqrtf(tot / (float)W + p.eps) : 0.f;
+            return true;
         };
         int lt = 0;
         float sc = 0.f;
-        bool ok = wait_or_abort(a_full, 0, abort_flag, 0x3300);
+        bool ok = wait_or_abort(a_full, 0, abort_flag, 0x3300) && row_scale((int)blockIdx.x % mt, sc);
         if (ok) {
-            sc = row_scale((int)blockIdx.x % mt);
             __syncwarp();
             if (lane == 0) mbar_arrive(a_empty);
         }
         for (int t = blockIdx.x; t < ntile && ok; t += gridDim.x, ++lt) {
             const int g = t / mt, m = t - g * mt;
-            const int nrows = min(128, p.rows - m * 128);
             // ---- SwiGLU chunks: this thread owns hidden columns [half*64, half*64 + 64) of its row
 #pragma unroll 1
             for (int c = 0; c < NC; ++c) {
@@ -391,6 +444,11 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                                              silu_tanh(sc * __uint_as_float(g1[2 * i + 1])) * (sc * __uint_as_float(u1[2 * i + 1])));
                 }
                 if (!wait_or_abort(hid_empty, (use & 1) ^ 1, abort_flag, 0x3302)) { ok = false; break; }
+                // the previous tile's output stores have finished reading this warp's rows
+                if (c == 0 && lt > 0) {
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+                }
                 // hidden chunk: 2 K-slabs of 64 columns (128-byte swizzled rows); this half is slab `half`
                 uint8_t* hrow = sH + half * 16384 + r * 128;
 #pragma unroll
@@ -404,40 +462,66 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             if (!ok) break;
             // ---- statistics of the next tile (its A tile is loaded once this tile's last read of A is issued)
             if (t + (int)gridDim.x < ntile) {
-                if (!wait_or_abort(a_full, (lt + 1) & 1, abort_flag, 0x3304)) break;
-                sc = row_scale((t + (int)gridDim.x) % mt);
+                if (!wait_or_abort(a_full, (lt + 1) & 1, abort_flag, 0x3304) || !row_scale((t + (int)gridDim.x) % mt, sc))
+                    break;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(a_empty);
             }
-            // ---- output tile: Y (residual already accumulated) -> bf16, 32 bytes per store
+            // ---- output tile: Y (residual already accumulated) -> bf16 -> this warp's rows of the idle
+            // hidden buffer (the output box layout) -> bulk tensor store, 64 columns per round
             if (!wait_or_abort(y_full, lt & 1, abort_flag, 0x3303)) break;
             tc_fence_after();
-            const int b = m * 128 + r;
-            const bool valid = r < nrows;
+            const int b0 = m * 128 + q * 32;                          // first row of this warp's box
 #pragma unroll
-            for (int j = 0; j < W / 64; ++j) {
-                uint32_t v[32];
-                tmem_ld32_async(trow + half * (W / 2) + j * 32, v);
-                tmem_wait_ld_tie(v);
-                if (!valid) continue;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const size_t off = row_elem(p.omap, b, g, half * (W / 2) + j * 32 + h * 16);
-                    if (off + 16 > p.out_elems) {
-                        record_error(ERR_BOUNDS, 0x3310);
-                        continue;
-                    }
-                    uint32_t w[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        w[e] = pack_bf16x2(__uint_as_float(v[h * 16 + 2 * e]), __uint_as_float(v[h * 16 + 2 * e + 1]));
-                    st_global_v8(p.out + off, w);
+            for (int j = 0; j < W / 128; ++j) {
+                const int col0 = half * (W / 2) + j * 64;
+                uint32_t v0[32], v1[32];
+                tmem_ld32_async(trow + col0, v0);
+                tmem_ld32_async(trow + col0 + 32, v1);
+                tmem_wait_ld_tie(v0);
+                tmem_wait_ld_tie(v1);
+                if (j == W / 128 - 1) {                                // Y fully read: release it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(y_empty);
                 }
+                if (j > 0) {                                           // the previous round's store has read the rows
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {                       // 8 columns per 16-byte piece
+                    const uint32_t* vv = c8 < 4 ? v0 : v1;
+                    const int o = (c8 & 3) * 8;
+                    const uint4 w4 = make_uint4(pack_bf16x2(__uint_as_float(vv[o + 0]), __uint_as_float(vv[o + 1])),
+                                                pack_bf16x2(__uint_as_float(vv[o + 2]), __uint_as_float(vv[o + 3])),
+                                                pack_bf16x2(__uint_as_float(vv[o + 4]), __uint_as_float(vv[o + 5])),
+                                                pack_bf16x2(__uint_as_float(vv[o + 6]), __uint_as_float(vv[o + 7])));
+                    uint8_t* dst = AMODE == A_TMA_MIX
+                                       ? stg + (c8 >> 1) * 1024 + lane * 32 + (((c8 & 1) ^ ((lane >> 2) & 1)) << 4)
+                                       : stg + lane * 128 + ((c8 ^ (lane & 7)) << 4);
+                    *reinterpret_cast<uint4*>(dst) = w4;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && b0 < p.rows) {
+                    if (AMODE == A_TMA_MIX) {
+                        const int per = p.omap.dh >> 4;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int ci = (col0 >> 4) + k, tok = ci / per, jj = ci - tok * per;
+                            tma_store_4d(&tmO, stg + k * 1024, 0, g * per + jj, tok, b0);
+                        }
+                    } else {
+                        tma_store_3d(&tmO, stg, col0, g, b0);
+                    }
+                    bulk_commit_group();
+                }
+                __syncwarp();
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(y_empty);
         }
+        if (lane == 0) bulk_wait_all();                                // stores complete before exit
+        __syncwarp();
     }
 
     tc_fence_before();

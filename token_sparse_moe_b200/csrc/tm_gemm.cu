@@ -25,7 +25,7 @@ static cudaError_t launch_fused_one(const CUtensorMap& a, const CUtensorMap& g, 
 template <int W, int AM>
 static cudaError_t launch_fused128_one(const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
                                        const CUtensorMap& d, const CUtensorMap& r, const CUtensorMap& e,
-                                       const FusedParams& p, int grid, cudaStream_t st) {
+                                       const CUtensorMap& o, const FusedParams& p, int grid, cudaStream_t st) {
     using C = Fused128Cfg<W, AM>;
     auto kern = fused128_swiglu_kernel<W, AM>;
     static bool configured = false;
@@ -35,17 +35,17 @@ static cudaError_t launch_fused128_one(const CUtensorMap& a, const CUtensorMap& 
         configured = true;
     }
     ProfileScope ps_("fused_swiglu", st);
-    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, g, u, d, r, e, p);
+    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, g, u, d, r, e, o, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_fused128(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
-                            const CUtensorMap& d, const CUtensorMap& r, const CUtensorMap& e, const FusedParams& p,
-                            int grid, cudaStream_t st) {
-    if (W == 256 && a_mode == A_TMA_MIX) return launch_fused128_one<256, A_TMA_MIX>(a, g, u, d, r, e, p, grid, st);
-    if (W == 256 && a_mode == A_TMA_3D) return launch_fused128_one<256, A_TMA_3D>(a, g, u, d, r, e, p, grid, st);
-    if (W == 128 && a_mode == A_TMA_MIX) return launch_fused128_one<128, A_TMA_MIX>(a, g, u, d, r, e, p, grid, st);
-    if (W == 128 && a_mode == A_TMA_3D) return launch_fused128_one<128, A_TMA_3D>(a, g, u, d, r, e, p, grid, st);
+                            const CUtensorMap& d, const CUtensorMap& r, const CUtensorMap& e, const CUtensorMap& o,
+                            const FusedParams& p, int grid, cudaStream_t st) {
+    if (W == 256 && a_mode == A_TMA_MIX) return launch_fused128_one<256, A_TMA_MIX>(a, g, u, d, r, e, o, p, grid, st);
+    if (W == 256 && a_mode == A_TMA_3D) return launch_fused128_one<256, A_TMA_3D>(a, g, u, d, r, e, o, p, grid, st);
+    if (W == 128 && a_mode == A_TMA_MIX) return launch_fused128_one<128, A_TMA_MIX>(a, g, u, d, r, e, o, p, grid, st);
+    if (W == 128 && a_mode == A_TMA_3D) return launch_fused128_one<128, A_TMA_3D>(a, g, u, d, r, e, o, p, grid, st);
     return cudaErrorInvalidValue;
 }
 

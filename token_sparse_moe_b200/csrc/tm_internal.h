@@ -38,10 +38,11 @@ cudaError_t launch_fused(int W, int a_mode, const CUtensorMap& a, const CUtensor
                          const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st);
 // CTA-pair version (2-SM MMAs, clusters of 2): grid = 2 x clusters; weight maps with half-size boxes
 // 128-wide hidden chunks (F % 128 == 0); gate/up maps with 128-row boxes; r / e: residual and
-// inter-residual maps in the geometry of a (read when p.res_mode == RES_STREAM / p.has_extra)
+// inter-residual maps in the geometry of a (read when p.res_mode == RES_STREAM / p.has_extra);
+// o: the output in the geometry of a with 32-row boxes
 cudaError_t launch_fused128(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
-                            const CUtensorMap& d, const CUtensorMap& r, const CUtensorMap& e, const FusedParams& p,
-                            int grid, cudaStream_t st);
+                            const CUtensorMap& d, const CUtensorMap& r, const CUtensorMap& e, const CUtensorMap& o,
+                            const FusedParams& p, int grid, cudaStream_t st);
 cudaError_t launch_fused2(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
                           const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st);
 int grouped_gemm_smem(int bn, int a_mode);
