@@ -9,12 +9,14 @@
 // and releases it at once, so G1(c+1) queues behind G2(c-1) while the SwiGLU of chunk c runs.
 // TMEM: Y in columns [0, W), the GEMM1 buffer in [256, 512).
 //
-// The residual is added by the tensor core: before GEMM2(0) the accumulator Y is initialised with
-// the residual tile times a 16 x 16 identity (one N = 16 MMA per 16 columns; bf16 times one summed
-// in fp32 is exact).  When the residual is the sub-layer input itself (the mixing sub-layer) the
-// resident A tile is that operand; otherwise the residual tile, and the inter-residual of a gap
-// layer, stream through the weight ring with the same tensor-map geometry as A.  The output
-// epilogue is then only TMEM -> bf16 -> global, with 32-byte stores (one full sector per lane).
+// The residual is added by the tensor core: GEMM2(0) initialises the accumulator Y, and after
+// GEMM2(1) the residual tile times a 16 x 16 identity is accumulated into it (one N = 16 MMA per 16
+// columns; bf16 times one summed in fp32 is exact).  When the residual is the sub-layer input
+// itself (the mixing sub-layer) the resident A tile is that operand; otherwise the residual tile,
+// and the inter-residual of a gap layer, stream through the weight ring with the same tensor-map
+// geometry as A, prefetched like any weight stage.  The output epilogue is then only
+// TMEM -> bf16 -> shared memory -> bulk tensor store.  A is loaded and released slab by slab
+// (64 columns), so the next tile's A streams in while the last GEMM1 of this one still runs.
 //
 // The epilogue warps are software-pipelined across tiles: after the last hidden chunk of tile t
 // they compute the row statistics of tile t+1 (its A tile is already loaded), run the SwiGLU of
@@ -73,6 +75,9 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
     const int NC = p.F / 128;
     const int res_stages = p.res_mode == RES_STREAM ? C::R_STAGES : 0;
     const int ext_stages = p.has_extra ? C::R_STAGES : 0;
+    // the residual / inter-residual identity pass runs after GEMM2(s_r - 1) (Y is initialised by
+    // GEMM2(0)), where its streamed tiles come through the ring like any weight stage
+    const int s_r = NC < 2 ? NC : 2;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -84,8 +89,8 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
     uint64_t* full = bar;                  // [STAGES]
     uint64_t* empty = full + STAGES;       // [STAGES]
     uint64_t* a_full = empty + STAGES;
-    uint64_t* a_empty = a_full + 1;
-    uint64_t* g1_full = a_empty + 1;
+    uint64_t* a_empty = a_full + 1;        // [G1_STAGES]: one per 64-column slab of A
+    uint64_t* g1_full = a_empty + C::G1_STAGES;
     uint64_t* g1_empty = g1_full + 1;
     uint64_t* hid_full = g1_empty + 1;
     uint64_t* hid_empty = hid_full + 1;
@@ -105,7 +110,8 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(a_full, 1);
-        mbar_init(a_empty, 1 + 8);             // MMA (last read of A issued) + each epilogue warp (statistics)
+        // per slab of A: the MMA (last read issued) + the 4 epilogue warps of the half that reads it
+        for (int q = 0; q < C::G1_STAGES; ++q) mbar_init(&a_empty[q], 1 + 4);
         mbar_init(g1_full, 1);
         mbar_init(g1_empty, 8);
         mbar_init(hid_full, 8);
@@ -164,11 +170,16 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             };
             for (int t = blockIdx.x; t < ntile && ok; t += gridDim.x, ++lt) {
                 const int g = t / mt, m = t - g * mt;
-                if (!wait_or_abort(a_empty, (lt & 1) ^ 1, abort_flag, 0x3100)) break;
-                mbar_arrive_expect_tx(a_full, C::A_BYTES);
-                load_rows(&tmA, sA, a_full, g, m * 128, 0, W / 16);
-                // ring order: G1(0); then for step >= 1: G1(step) (step < NC), the residual and
-                // inter-residual tiles (step 1 only), G2(step - 1)
+                // A slab by slab, each as soon as the previous tile has released it
+#pragma unroll 1
+                for (int qa = 0; qa < C::G1_STAGES && ok; ++qa) {
+                    if (!wait_or_abort(&a_empty[qa], (lt & 1) ^ 1, abort_flag, 0x3100)) { ok = false; break; }
+                    if (qa == 0) mbar_arrive_expect_tx(a_full, C::A_BYTES);
+                    load_rows(&tmA, sA + qa * 16384, a_full, g, m * 128, qa * 4, 4);
+                }
+                if (!ok) break;
+                // ring order: G1(0); then for step >= 1: G1(step) (step < NC), G2(step - 1), and at
+                // step s_r the residual and inter-residual tiles
 #pragma unroll 1
                 for (int step = 0; step <= NC && ok; ++step) {
                     if (step < NC) {
@@ -180,17 +191,6 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             mbar_arrive_expect_tx(&full[s], C::SB);
                             tma_load_2d(st, &tmG, &full[s], q * 64, g * p.F + c * 128);
                             tma_load_2d(st + 16384, &tmU, &full[s], q * 64, g * p.F + c * 128);
-                            if (++s == STAGES) { s = 0; ph ^= 1; }
-                        }
-                    }
-                    if (step == 1 && ok) {
-#pragma unroll 1
-                        for (int i = 0; i < res_stages + ext_stages; ++i) {    // 128 columns per stage
-                            if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x3103)) { ok = false; break; }
-                            uint8_t* st = sR + s * C::SB;
-                            mbar_arrive_expect_tx(&full[s], C::SB);
-                            const int q = i < res_stages ? i : i - res_stages;
-                            load_rows(i < res_stages ? &tmR : &tmE, st, &full[s], g, m * 128, q * 8, 8);
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                     }
@@ -210,6 +210,18 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                     }
+                    if (step == s_r && ok) {
+#pragma unroll 1
+                        for (int i = 0; i < res_stages + ext_stages; ++i) {    // 128 columns per stage
+                            if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x3103)) { ok = false; break; }
+                            uint8_t* st = sR + s * C::SB;
+                            mbar_arrive_expect_tx(&full[s], C::SB);
+                            const int q = i < res_stages ? i : i - res_stages;
+                            load_rows(i < res_stages ? &tmR : &tmE, st, &full[s], g, m * 128, q * 8, 8);
+                            if (++s == STAGES) { s = 0; ph ^= 1; }
+                        }
+                    }
+
                 }
             }
         }
@@ -233,10 +245,9 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             const uint64_t rdesc32 = umma_sdesc_sw32(rS);
             const uint64_t idB = umma_sdesc_sw32(smem_u32(sI));
             constexpr uint64_t kStageDesc = C::SB >> 4;               // descriptor start-address step per stage
-            const bool y_init = p.res_mode != RES_NONE || p.has_extra;
-            // the A tile is released after the last step that reads it: GEMM1(NC-1), and the
-            // identity pass of step 1 when the residual comes from A
-            const int a_last = (p.res_mode == RES_FROM_A && NC < 2) ? 1 : NC - 1;
+            // A is released slab by slab after GEMM1(NC-1), or after the identity pass when that
+            // reads A and comes later
+            const bool a_after_id = p.res_mode == RES_FROM_A && s_r >= NC - 1;
             int s = 0;
             uint32_t ph = 0;
             int lt = 0;
@@ -272,6 +283,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             for (int kk = 0; kk < 4; ++kk)
                                 umma_bf16(tmem + C::G1COL, adesc[q * 4 + kk], bd + 2 * kk, idesc1, (q | kk) != 0);
                             umma_commit(&empty[s]);
+                            if (step == NC - 1 && !a_after_id) umma_commit(&a_empty[q]);
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                         if (!ok) break;
@@ -280,32 +292,9 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                     if (step >= 1) {                                   // ---- GEMM2(step - 1)
                         const int c = step - 1;
                         const uint32_t use = lt * NC + c;
-                        if (c == 0) {
-                            // Y free (previous tile read out), then Y = residual (+ inter-residual)
+                        if (c == 0) {                                  // GEMM2(0) initialises Y: wait until it is free
                             if (!wait_or_abort(y_empty, (lt & 1) ^ 1, abort_flag, 0x3204)) { ok = false; break; }
                             tc_fence_after();
-                            if (p.res_mode == RES_FROM_A) {
-#pragma unroll
-                                for (int k16 = 0; k16 < W / 16; ++k16) umma_bf16(tmem + 16 * k16, adesc[k16], idB, idescI, 0);
-                            }
-#pragma unroll 1
-                            for (int i = 0; i < res_stages + ext_stages; ++i) {
-                                if (!wait_or_abort(&full[s], ph, abort_flag, 0x3207)) { ok = false; break; }
-                                tc_fence_after();
-                                const uint32_t acc = (i >= res_stages && p.res_mode != RES_NONE) ? 1u : 0u;
-                                const int q = i < res_stages ? i : i - res_stages;
-                                const uint32_t st = rS + s * C::SB;
-#pragma unroll
-                                for (int k16 = 0; k16 < 8; ++k16) {
-                                    const uint64_t rd = AMODE == A_TMA_MIX
-                                                            ? rdesc32 + (uint64_t)s * kStageDesc + k16 * (4096 >> 4)
-                                                            : umma_sdesc_sw128(st + (k16 >> 2) * 16384) + 2 * (k16 & 3);
-                                    umma_bf16(tmem + 16 * (q * 8 + k16), rd, idB, idescI, acc);
-                                }
-                                umma_commit(&empty[s]);
-                                if (++s == STAGES) { s = 0; ph ^= 1; }
-                            }
-                            if (!ok) break;
                         }
                         bool rdy[C::G2_STAGES];
                         const bool h_rdy = mbar_test(hid_full, use & 1);
@@ -333,16 +322,42 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
 #pragma unroll
                                 for (int kk = 0; kk < 4; ++kk)
                                     umma_bf16(tmem, hd + 2 * kk, bd + kq * (16384 >> 4) + 2 * kk, idesc2,
-                                              (y_init || (c | q | kq | kk) != 0) ? 1u : 0u);
+                                              (c | q | kq | kk) != 0 ? 1u : 0u);
                             }
                             umma_commit(&empty[s]);
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                         if (!ok) break;
                         umma_commit(hid_empty);
-                        if (c == NC - 1) umma_commit(y_full);
                     }
-                    if (step == a_last) umma_commit(a_empty);
+                    if (step == s_r) {                                 // ---- Y += residual (+ inter-residual)
+                        if (p.res_mode == RES_FROM_A) {
+#pragma unroll
+                            for (int k16 = 0; k16 < W / 16; ++k16) umma_bf16(tmem + 16 * k16, adesc[k16], idB, idescI, 1);
+                            if (a_after_id) {
+#pragma unroll
+                                for (int q = 0; q < C::G1_STAGES; ++q) umma_commit(&a_empty[q]);
+                            }
+                        }
+#pragma unroll 1
+                        for (int i = 0; i < res_stages + ext_stages; ++i) {
+                            if (!wait_or_abort(&full[s], ph, abort_flag, 0x3207)) { ok = false; break; }
+                            tc_fence_after();
+                            const int q = i < res_stages ? i : i - res_stages;
+                            const uint32_t st = rS + s * C::SB;
+#pragma unroll
+                            for (int k16 = 0; k16 < 8; ++k16) {
+                                const uint64_t rd = AMODE == A_TMA_MIX
+                                                        ? rdesc32 + (uint64_t)s * kStageDesc + k16 * (4096 >> 4)
+                                                        : umma_sdesc_sw128(st + (k16 >> 2) * 16384) + 2 * (k16 & 3);
+                                umma_bf16(tmem + 16 * (q * 8 + k16), rd, idB, idescI, 1);
+                            }
+                            umma_commit(&empty[s]);
+                            if (++s == STAGES) { s = 0; ph ^= 1; }
+                        }
+                        if (!ok) break;
+                    }
+                    if (step == NC) umma_commit(y_full);
                 }
             }
             umma_commit(drain);
@@ -408,11 +423,16 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         };
         int lt = 0;
         float sc = 0.f;
-        bool ok = wait_or_abort(a_full, 0, abort_flag, 0x3300) && row_scale((int)blockIdx.x % mt, sc);
-        if (ok) {
+        // the statistics of a tile read the A slabs of this thread's half; release them afterwards
+        auto release_a = [&]() {
             __syncwarp();
-            if (lane == 0) mbar_arrive(a_empty);
-        }
+            if (lane == 0) {
+#pragma unroll
+                for (int qa = 0; qa < C::G1_STAGES / 2; ++qa) mbar_arrive(&a_empty[half * (C::G1_STAGES / 2) + qa]);
+            }
+        };
+        bool ok = wait_or_abort(a_full, 0, abort_flag, 0x3300) && row_scale((int)blockIdx.x % mt, sc);
+        if (ok) release_a();
         for (int t = blockIdx.x; t < ntile && ok; t += gridDim.x, ++lt) {
             const int g = t / mt, m = t - g * mt;
             // ---- SwiGLU chunks: this thread owns hidden columns [half*64, half*64 + 64) of its row
@@ -464,8 +484,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             if (t + (int)gridDim.x < ntile) {
                 if (!wait_or_abort(a_full, (lt + 1) & 1, abort_flag, 0x3304) || !row_scale((t + (int)gridDim.x) % mt, sc))
                     break;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(a_empty);
+                release_a();
             }
             // ---- output tile: Y (residual already accumulated) -> bf16 -> this warp's rows of the idle
             // hidden buffer (the output box layout) -> bulk tensor store, 64 columns per round
