@@ -256,6 +256,17 @@ __device__ __forceinline__ float silu_tanh(float z) {
     return fmaf(hz, t, hz);
 }
 
+// Two SwiGLU outputs with paired fp32 instructions: h = silu(s g) * (s u) for (g.x, u.x), (g.y, u.y),
+// with hs = s / 2 (so that hs g = (s g) / 2 exactly) and the same rounding steps as silu_tanh.
+__device__ __forceinline__ float2 swiglu2(float hs, float s, float2 g, float2 u) {
+    const float2 hz = __fmul2_rn(make_float2(hs, hs), g);
+    float2 t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t.x) : "f"(hz.x));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t.y) : "f"(hz.y));
+    const float2 sl = __ffma2_rn(hz, t, hz);
+    return __fmul2_rn(sl, __fmul2_rn(make_float2(s, s), u));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);

@@ -75,9 +75,14 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
     const int NC = p.F / 128;
     const int res_stages = p.res_mode == RES_STREAM ? C::R_STAGES : 0;
     const int ext_stages = p.has_extra ? C::R_STAGES : 0;
-    // the residual / inter-residual identity pass runs after GEMM2(s_r - 1) (Y is initialised by
+    // GEMM2(c) is issued in step c + LAG, after GEMM1(c + LAG).  LAG = 1: the SwiGLU of chunk c
+    // overlaps GEMM1(c+1) and its hidden write waits only for GEMM2(c-1).  (A lag of 2 measured
+    // 16% slower on the dense block workload: each hidden write then waits behind a whole GEMM1.)
+    constexpr int LAG = 1;
+    const int n_steps = NC + LAG;
+    // the residual / inter-residual identity pass runs after GEMM2(min(1, NC-1)) (Y is initialised by
     // GEMM2(0)), where its streamed tiles come through the ring like any weight stage
-    const int s_r = NC < 2 ? NC : 2;
+    const int s_r = (NC < 2 ? 0 : 1) + LAG;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -178,10 +183,10 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                     load_rows(&tmA, sA + qa * 16384, a_full, g, m * 128, qa * 4, 4);
                 }
                 if (!ok) break;
-                // ring order: G1(0); then for step >= 1: G1(step) (step < NC), G2(step - 1), and at
-                // step s_r the residual and inter-residual tiles
+                // ring order per step: G1(step) (step < NC), G2(step - LAG) (step >= LAG), and at step
+                // s_r the residual and inter-residual tiles
 #pragma unroll 1
-                for (int step = 0; step <= NC && ok; ++step) {
+                for (int step = 0; step < n_steps && ok; ++step) {
                     if (step < NC) {
                         const int c = step;
 #pragma unroll 1
@@ -194,8 +199,8 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                     }
-                    if (step >= 1 && ok) {
-                        const int c = step - 1;
+                    if (step >= LAG && ok) {
+                        const int c = step - LAG;
 #pragma unroll 1
                         for (int q = 0; q < C::G2_STAGES; ++q) {
                             if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x3102)) { ok = false; break; }
@@ -256,7 +261,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                 if (!wait_or_abort(a_full, lt & 1, abort_flag, 0x3200)) break;
                 tc_fence_after();
 #pragma unroll 1
-                for (int step = 0; step <= NC && ok; ++step) {
+                for (int step = 0; step < n_steps && ok; ++step) {
                     if (step < NC) {                                   // ---- GEMM1(step)
                         const uint32_t use = lt * NC + step;
                         bool rdy[C::G1_STAGES];
@@ -289,8 +294,8 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                         if (!ok) break;
                         umma_commit(g1_full);
                     }
-                    if (step >= 1) {                                   // ---- GEMM2(step - 1)
-                        const int c = step - 1;
+                    if (step >= LAG) {                                 // ---- GEMM2(step - LAG)
+                        const int c = step - LAG;
                         const uint32_t use = lt * NC + c;
                         if (c == 0) {                                  // GEMM2(0) initialises Y: wait until it is free
                             if (!wait_or_abort(y_empty, (lt & 1) ^ 1, abort_flag, 0x3204)) { ok = false; break; }
@@ -357,7 +362,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                         }
                         if (!ok) break;
                     }
-                    if (step == NC) umma_commit(y_full);
+                    if (step == n_steps - 1) umma_commit(y_full);
                 }
             }
             umma_commit(drain);
@@ -421,74 +426,10 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             out = r < p.rows - m_tile * 128 ? 1.0f / sqrtf(tot / (float)W + p.eps) : 0.f;
             return true;
         };
-        int lt = 0;
-        float sc = 0.f;
-        // the statistics of a tile read the A slabs of this thread's half; release them afterwards
-        auto release_a = [&]() {
-            __syncwarp();
-            if (lane == 0) {
-#pragma unroll
-                for (int qa = 0; qa < C::G1_STAGES / 2; ++qa) mbar_arrive(&a_empty[half * (C::G1_STAGES / 2) + qa]);
-            }
-        };
-        bool ok = wait_or_abort(a_full, 0, abort_flag, 0x3300) && row_scale((int)blockIdx.x % mt, sc);
-        if (ok) release_a();
-        for (int t = blockIdx.x; t < ntile && ok; t += gridDim.x, ++lt) {
-            const int g = t / mt, m = t - g * mt;
-            // ---- SwiGLU chunks: this thread owns hidden columns [half*64, half*64 + 64) of its row
-#pragma unroll 1
-            for (int c = 0; c < NC; ++c) {
-                const uint32_t use = lt * NC + c;
-                if (!wait_or_abort(g1_full, use & 1, abort_flag, 0x3301)) { ok = false; break; }
-                tc_fence_after();
-                // all four loads in flight, one wait, then the GEMM1 buffer is released before the math
-                uint32_t g0[32], u0[32], g1[32], u1[32];
-                const uint32_t tg = trow + C::G1COL + half * 64;
-                tmem_ld32_async(tg, g0);
-                tmem_ld32_async(tg + 128, u0);
-                tmem_ld32_async(tg + 32, g1);
-                tmem_ld32_async(tg + 160, u1);
-                tmem_wait_ld_tie(g0);
-                tmem_wait_ld_tie(u0);
-                tmem_wait_ld_tie(g1);
-                tmem_wait_ld_tie(u1);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(g1_empty);
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    pk[i] = pack_bf16x2(silu_tanh(sc * __uint_as_float(g0[2 * i])) * (sc * __uint_as_float(u0[2 * i])),
-                                        silu_tanh(sc * __uint_as_float(g0[2 * i + 1])) * (sc * __uint_as_float(u0[2 * i + 1])));
-                    pk[16 + i] = pack_bf16x2(silu_tanh(sc * __uint_as_float(g1[2 * i])) * (sc * __uint_as_float(u1[2 * i])),
-                                             silu_tanh(sc * __uint_as_float(g1[2 * i + 1])) * (sc * __uint_as_float(u1[2 * i + 1])));
-                }
-                if (!wait_or_abort(hid_empty, (use & 1) ^ 1, abort_flag, 0x3302)) { ok = false; break; }
-                // the previous tile's output stores have finished reading this warp's rows
-                if (c == 0 && lt > 0) {
-                    if (lane == 0) bulk_wait_read_all();
-                    __syncwarp();
-                }
-                // hidden chunk: 2 K-slabs of 64 columns (128-byte swizzled rows); this half is slab `half`
-                uint8_t* hrow = sH + half * 16384 + r * 128;
-#pragma unroll
-                for (int v = 0; v < 8; ++v)
-                    *reinterpret_cast<uint4*>(hrow + ((v ^ (r & 7)) << 4)) =
-                        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(hid_full);
-            }
-            if (!ok) break;
-            // ---- statistics of the next tile (its A tile is loaded once this tile's last read of A is issued)
-            if (t + (int)gridDim.x < ntile) {
-                if (!wait_or_abort(a_full, (lt + 1) & 1, abort_flag, 0x3304) || !row_scale((t + (int)gridDim.x) % mt, sc))
-                    break;
-                release_a();
-            }
-            // ---- output tile: Y (residual already accumulated) -> bf16 -> this warp's rows of the idle
-            // hidden buffer (the output box layout) -> bulk tensor store, 64 columns per round
-            if (!wait_or_abort(y_full, lt & 1, abort_flag, 0x3303)) break;
+        // Y of tile (g, m) (residual already accumulated) -> bf16 -> this warp's rows of the idle hidden
+        // buffer in the output box layout -> bulk tensor store, 64 columns per round; releases Y
+        auto output_tile = [&](int g, int m, int ylt) -> bool {
+            if (!wait_or_abort(y_full, ylt & 1, abort_flag, 0x3303)) return false;
             tc_fence_after();
             const int b0 = m * 128 + q * 32;                          // first row of this warp's box
 #pragma unroll
@@ -538,7 +479,84 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                 }
                 __syncwarp();
             }
+            return true;
+        };
+        int lt = 0;
+        float sc = 0.f;
+        // the statistics of a tile read the A slabs of this thread's half; release them afterwards
+        auto release_a = [&]() {
+            __syncwarp();
+            if (lane == 0) {
+#pragma unroll
+                for (int qa = 0; qa < C::G1_STAGES / 2; ++qa) mbar_arrive(&a_empty[half * (C::G1_STAGES / 2) + qa]);
+            }
+        };
+        bool ok = wait_or_abort(a_full, 0, abort_flag, 0x3300) && row_scale((int)blockIdx.x % mt, sc);
+        if (ok) release_a();
+        int prev_g = 0, prev_m = 0;
+        for (int t = blockIdx.x; t < ntile && ok; t += gridDim.x, ++lt) {
+            const int g = t / mt, m = t - g * mt;
+            // ---- SwiGLU chunks: this thread owns hidden columns [half*64, half*64 + 64) of its row
+#pragma unroll 1
+            for (int c = 0; c < NC; ++c) {
+                const uint32_t use = lt * NC + c;
+                if (!wait_or_abort(g1_full, use & 1, abort_flag, 0x3301)) { ok = false; break; }
+                tc_fence_after();
+                // all four loads in flight, one wait, then the GEMM1 buffer is released before the math
+                uint32_t g0[32], u0[32], g1[32], u1[32];
+                const uint32_t tg = trow + C::G1COL + half * 64;
+                tmem_ld32_async(tg, g0);
+                tmem_ld32_async(tg + 128, u0);
+                tmem_ld32_async(tg + 32, g1);
+                tmem_ld32_async(tg + 160, u1);
+                tmem_wait_ld_tie(g0);
+                tmem_wait_ld_tie(u0);
+                tmem_wait_ld_tie(g1);
+                tmem_wait_ld_tie(u1);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(g1_empty);
+                uint32_t pk[32];
+                const float hsc = 0.5f * sc;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 h0 = swiglu2(hsc, sc, make_float2(__uint_as_float(g0[2 * i]), __uint_as_float(g0[2 * i + 1])),
+                                              make_float2(__uint_as_float(u0[2 * i]), __uint_as_float(u0[2 * i + 1])));
+                    const float2 h1 = swiglu2(hsc, sc, make_float2(__uint_as_float(g1[2 * i]), __uint_as_float(g1[2 * i + 1])),
+                                              make_float2(__uint_as_float(u1[2 * i]), __uint_as_float(u1[2 * i + 1])));
+                    pk[i] = pack_bf16x2(h0.x, h0.y);
+                    pk[16 + i] = pack_bf16x2(h1.x, h1.y);
+                }
+                if (c == 0 && lt > 0) {
+                    // the previous tile's output, now that GEMM1(1) of this tile can run (its buffer is
+                    // released above); the hidden rows are its staging, so this chunk's hidden write
+                    // waits until the bulk stores have read them
+                    if (!output_tile(prev_g, prev_m, lt - 1)) { ok = false; break; }
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+                }
+                if (!wait_or_abort(hid_empty, (use & 1) ^ 1, abort_flag, 0x3302)) { ok = false; break; }
+                // hidden chunk: 2 K-slabs of 64 columns (128-byte swizzled rows); this half is slab `half`
+                uint8_t* hrow = sH + half * 16384 + r * 128;
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                    *reinterpret_cast<uint4*>(hrow + ((v ^ (r & 7)) << 4)) =
+                        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(hid_full);
+            }
+            if (!ok) break;
+            // ---- statistics of the next tile (its A tile is loaded once this tile's last read of A is issued)
+            if (t + (int)gridDim.x < ntile) {
+                if (!wait_or_abort(a_full, (lt + 1) & 1, abort_flag, 0x3304) || !row_scale((t + (int)gridDim.x) % mt, sc))
+                    break;
+                release_a();
+            }
+            prev_g = g;
+            prev_m = m;
         }
+        if (ok && lt > 0) ok = output_tile(prev_g, prev_m, lt - 1);
         if (lane == 0) bulk_wait_all();                                // stores complete before exit
         __syncwarp();
     }
