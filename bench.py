@@ -228,6 +228,28 @@ def run_reference(args, cfg, rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ multi-rank bookkeeping
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest of every rank's value (the job is as slow as its slowest rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(samples_per_rank: int, world: int, step_ms: float) -> float:
+    """Samples all ranks processed per second: each rank runs its own batch (weak scaling)."""
+    return samples_per_rank * world / (step_ms / 1e3)
+
+
+def rank_config(cfg, rank: int):
+    """Each rank draws its own input batch (seed offset by the rank); weights are shared."""
+    return cfg.with_(seed=cfg.seed + rank)
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_ours(args, cfg, rank, world, local_rank):
     import torch
@@ -240,7 +262,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     blocks = api.blocks_from_synth(cfg, dev, workers=min(16, os.cpu_count() or 1))
     sh = api.config_shape(cfg)
     run = api.StackRunner(blocks, sh, cfg.gap, dev)
-    X = api.to_device(S.make_x(cfg.with_(seed=cfg.seed + rank)), dev)
+    X = api.to_device(S.make_x(rank_config(cfg, rank)), dev)
     Y = torch.empty_like(X)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     K, W = args.steps, args.warmup
@@ -274,11 +296,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         api.get_device_error(stream)
         step_ms = [a.elapsed_time(b) for a, b in ev]
 
-    mean_ms = sum(step_ms) / K
-    if world > 1:
-        t = torch.tensor([mean_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        mean_ms = float(t.item())
+    mean_ms = max_over_ranks(sum(step_ms) / K, world, dev)
 
     # end to end through the public API: pinned host X -> device -> forward -> pinned host Y
     Ke = min(K, args.e2e_steps)
@@ -296,18 +314,14 @@ def run_ours(args, cfg, rank, world, local_rank):
             run.run_host(Xh, Yh, Xd, Y, stream)
             eve[i][1].record(stream)
         stream.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in eve) / Ke
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eve) / Ke, world, dev)
     io_bytes = X.numel() * X.element_size()
 
     if rank != 0:
         return
     pk, pk_src = peaks()
     total_samples = cfg.B * world
-    value = total_samples / (mean_ms / 1e3)
+    value = job_throughput(cfg.B, world, mean_ms)
     tflops = flops_per_sample(cfg) * value / 1e12
     # dominant kernel: largest share of device time in the timed region
     dom = max(kern.items(), key=lambda kv: kv[1]["total_ms"]) if kern else (None, None)
@@ -339,7 +353,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         "tflops": tflops, "tc_roofline_frac": tflops / pk["bf16_tflops"],
         "roofline": roof,
         "cpu_baseline": cpu,
-        "e2e": {"value": total_samples / (e2e_ms / 1e3), "unit": "samples/s", "h2d_bytes_per_step": io_bytes,
+        "e2e": {"value": job_throughput(cfg.B, world, e2e_ms), "unit": "samples/s", "h2d_bytes_per_step": io_bytes,
                 "d2h_bytes_per_step": io_bytes, "ms_per_step": e2e_ms, "steps": Ke},
         "gpu_launches": int(launches),
         "launches_per_step": launches / K,
