@@ -44,6 +44,11 @@ DENSE_SMALL = [
     small("dense_one_tile", 100, 16, 128, 16, "bf16", FFNSpec("dense", hidden=192), FFNSpec("dense", hidden=128)),
     # width 128 and 256 with 5 row tiles (an odd count on CTA pairs: the last pair's second tile is empty)
     small("dense_w128", 600, 8, 128, 4, "bf16", FFNSpec("dense", hidden=128), FFNSpec("dense", hidden=256)),
+    # 160 tiles on 148 SMs: with TM_FUSED_SPLIT=1 the 12 tiles of the last wave are split between CTA
+    # pairs by hidden chunks (mixing F=384: halves of 1 and 2 chunks; reverting F=256: 1 and 1)
+    small("dense_split", 1280, 16, 256, 16, "bf16", FFNSpec("dense", hidden=384), FFNSpec("dense", hidden=256)),
+    # width 128: 8 banks x 19 tiles (the last one ragged) = 152 tiles, 4 of them split under TM_FUSED_SPLIT=1
+    small("dense_split_w128", 2400, 8, 128, 4, "bf16", FFNSpec("dense", hidden=256), FFNSpec("dense", hidden=512)),
 ]
 MOE_SMALL = [
     small("moe_sq", 300, 16, 256, 16, "bf16", moe(8, 2, 128, 128, 4.0), moe(4, 1, 64, 192, 4.0)),
@@ -255,6 +260,28 @@ def test_fused_cta_pair_kernel(cfg, monkeypatch):
             y, _ = _run_sub(cfg, sub, X, R, ds)
             o, _, _ = _oracle_sub(cfg, sub, X, R, ds)
             check_outputs(cfg, y, o, S.to_f64(R), ds)
+
+
+@pytest.mark.parametrize("cfg", [DENSE_SMALL[5], DENSE_SMALL[6]], ids=lambda c: c.name)
+def test_fused_split_tiles_match_unsplit(cfg, monkeypatch):
+    """Tiles of the last wave split between two CTAs give the outputs of the unsplit kernel up to
+    the fp32 summation order of Y (two partial sums added once): within one bf16 ulp of the output
+    or, where the output is a near-cancellation of residual and FFN term, within the fp32 rounding
+    of those terms (2^-20 of the output's rms); bit-identical from one run to the next."""
+    X, R = inputs(cfg)
+    for sub in (0, 1):
+        monkeypatch.setenv("TM_FUSED_SPLIT", "1")
+        y_split, _ = _run_sub(cfg, sub, X, R)
+        y_split2, _ = _run_sub(cfg, sub, X, R)
+        assert np.array_equal(y_split, y_split2)
+        o, _, _ = _oracle_sub(cfg, sub, X, R)
+        check_outputs(cfg, y_split, o, S.to_f64(R), None)
+        monkeypatch.setenv("TM_FUSED_SPLIT", "0")
+        y_whole, _ = _run_sub(cfg, sub, X, R)
+        monkeypatch.delenv("TM_FUSED_SPLIT")
+        from parity_util import ulp
+        bound = np.maximum(ulp(y_whole, "bf16"), 2.0 ** -20 * rms(y_whole))
+        assert np.all(np.abs(y_split - y_whole) <= bound)
 
 
 @pytest.mark.parametrize("cfg", [DENSE_SMALL[0], DENSE_SMALL[4]], ids=lambda c: c.name)

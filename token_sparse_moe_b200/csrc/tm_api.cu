@@ -265,7 +265,8 @@ tm_status gemm2_dense(const Geo& g, const void* hidden, const void* wd, int F, i
 // ------------------------------------------------------------------ fused dense sub-layer
 // One launch for row widths 128 / 256: statistics, GEMM1, SwiGLU, GEMM2, residual.
 tm_status fused_dense(const Geo& g, const void* x, const void* wg, const void* wu, const void* wd, int F,
-                      const void* resid, const void* extra, void* y, cudaStream_t st) {
+                      const void* resid, const void* extra, void* y, void* scratch, size_t scratch_bytes,
+                      cudaStream_t st) {
     const int am = gemm1_amode(g);
     // One CTA per 128-row tile by default.  TM_FUSED_PAIRS=1 selects the CTA-pair kernel (2-SM
     // MMAs, half the weight bytes per SM); on B200 it measured slower on the dense block workload
@@ -314,6 +315,24 @@ tm_status fused_dense(const Geo& g, const void* x, const void* wg, const void* w
         // output: the same row geometry, 32-row boxes (one per epilogue warp)
         CUtensorMap mo;
         if (!gemm1_amap(g, y, am, &mo, 32)) return TM_ERR_CUDA;
+        // Opt-in (TM_FUSED_SPLIT=1): when the last partial wave holds at most half a wave of tiles,
+        // split each of them between two CTAs by hidden chunks (fp32 partials in the scratch space,
+        // which the fused path does not otherwise use; counters zeroed here).  On the dense block
+        // workload it shortens the slowest CTA by ~6% but measured 1.5% slower per launch with the
+        // L2 flushed between steps (the 17 MB of partials push a working set that nearly fills the
+        // L2 over it) plus a memset per launch, so it is off by default.
+        const long n_rem = tiles % grid;
+        const size_t part_bytes = (size_t)2 * n_rem * 128 * g.W * sizeof(float);
+        const size_t cnt_off = (part_bytes + 255) & ~(size_t)255;
+        const char* env_split = getenv("TM_FUSED_SPLIT");
+        if (n_rem > 0 && 2 * n_rem <= grid && F / 128 >= 2 && scratch && cnt_off + n_rem * 8 * sizeof(int) <= scratch_bytes &&
+            env_split && env_split[0] == '1') {
+            p.split_tiles = 1;
+            p.part = (float*)scratch;
+            p.cnt = (int*)((uint8_t*)scratch + cnt_off);
+            tm_status s = cuda_status(cudaMemsetAsync(p.cnt, 0, n_rem * 8 * sizeof(int), st));
+            if (s != TM_OK) return s;
+        }
         return cuda_status(launch_fused128(g.W, am, ma, mg, mu, md, mr, me, mo, p, grid, st));
     }
     return cuda_status(launch_fused(g.W, am, ma, mg, mu, md, p, grid, st));
@@ -351,7 +370,8 @@ tm_status run_dense(const Geo& g, const void* x, const void* resid, const void* 
         wu = d.wu;
     }
     if (g.dtype == TM_BF16 && fused_supported(g.W, gemm1_amode(g)) && w->hidden % 64 == 0)
-        return fused_dense(g, x, wg, wu, w->w_down, w->hidden, resid, extra, y, st);
+        return fused_dense(g, x, wg, wu, w->w_down, w->hidden, resid, extra, y, d.hidden,
+                           (size_t)g.banks * g.B * w->hidden * g.esz, st);
     if ((s = cuda_status(launch_rms(g.dtype, x, g.map, g.B, g.eps, d.inv_rms, st))) != TM_OK) return s;
     if ((s = gemm1_dense(g, x, wg, wu, w->hidden, d.inv_rms, d.hidden, st)) != TM_OK) return s;
     return gemm2_dense(g, d.hidden, w->w_down, w->hidden, EPI_RESID, resid, extra, y, nullptr, nullptr, nullptr, 0, st);

@@ -61,6 +61,15 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
                  : "memory");
 }
 
+// 8 consecutive 32-bit words (32 bytes) from global memory, cached in L2 only (data written by
+// another CTA of the same launch); p must be 32-byte aligned.
+__device__ __forceinline__ void ld_global_cg_v8(const void* p, uint32_t (&w)[8]) {
+    asm volatile("ld.global.cg.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                 : "l"(p)
+                 : "memory");
+}
+
 template <int W, int AMODE>
 __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
     fused128_swiglu_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
@@ -79,10 +88,36 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
     // overlaps GEMM1(c+1) and its hidden write waits only for GEMM2(c-1).  (A lag of 2 measured
     // 16% slower on the dense block workload: each hidden write then waits behind a whole GEMM1.)
     constexpr int LAG = 1;
-    const int n_steps = NC + LAG;
-    // the residual / inter-residual identity pass runs after GEMM2(min(1, NC-1)) (Y is initialised by
-    // GEMM2(0)), where its streamed tiles come through the ring like any weight stage
-    const int s_r = (NC < 2 ? 0 : 1) + LAG;
+    // Work items of this CTA: tile t = blockIdx.x + k * gridDim.x for the full waves.  With
+    // p.split_tiles the tiles of the last, partial wave are each split between two CTAs by hidden
+    // chunks (half 0: [0, NC/2), half 1: [NC/2, NC)), so every CTA ends within half a tile of the
+    // others; the halves meet through p.part (see the split output below).
+    const int full_waves = ntile / (int)gridDim.x;
+    const int n_rem = ntile - full_waves * (int)gridDim.x;
+    auto item = [&](int k, int& t, int& c0, int& c1, int& sp) -> bool {
+        const int b = blockIdx.x;
+        sp = -1;
+        c0 = 0;
+        c1 = NC;
+        if (k < full_waves) { t = b + k * (int)gridDim.x; return true; }
+        if (k > full_waves) return false;
+        if (p.split_tiles) {
+            if (b >= 2 * n_rem) return false;
+            t = full_waves * (int)gridDim.x + (b >> 1);
+            sp = b & 1;
+            c0 = sp ? NC / 2 : 0;
+            c1 = sp ? NC : NC / 2;
+            return true;
+        }
+        if (b >= n_rem) return false;
+        t = full_waves * (int)gridDim.x + b;
+        return true;
+    };
+    // per item with nc chunks: steps 0 .. nc + LAG - 1; the residual / inter-residual identity pass
+    // (only in the item that starts at chunk 0) runs in step s_r, after GEMM2(min(1, nc-1)): Y is
+    // initialised by the item's first GEMM2, and the streamed tiles come through the ring like
+    // any weight stage
+    auto id_step = [&](int nc) { return (nc < 2 ? 0 : 1) + LAG; };
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -173,8 +208,10 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                     for (int i = 0; i < n16 / 4; ++i) tma_load_3d(dst + i * 16384, map, b, col16 * 16 + i * 64, g, m0);
                 }
             };
-            for (int t = blockIdx.x; t < ntile && ok; t += gridDim.x, ++lt) {
+            int t, c0, c1, sp;
+            for (; ok && item(lt, t, c0, c1, sp); ++lt) {
                 const int g = t / mt, m = t - g * mt;
+                const int nc = c1 - c0, n_steps = nc + LAG, s_r = c0 == 0 ? id_step(nc) : -1;
                 // A slab by slab, each as soon as the previous tile has released it
 #pragma unroll 1
                 for (int qa = 0; qa < C::G1_STAGES && ok; ++qa) {
@@ -187,8 +224,8 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                 // s_r the residual and inter-residual tiles
 #pragma unroll 1
                 for (int step = 0; step < n_steps && ok; ++step) {
-                    if (step < NC) {
-                        const int c = step;
+                    if (step < nc) {
+                        const int c = c0 + step;
 #pragma unroll 1
                         for (int q = 0; q < C::G1_STAGES; ++q) {             // K slab q: 128 gate + 128 up rows
                             if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x3101)) { ok = false; break; }
@@ -200,7 +237,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                         }
                     }
                     if (step >= LAG && ok) {
-                        const int c = step - LAG;
+                        const int c = c0 + step - LAG;
 #pragma unroll 1
                         for (int q = 0; q < C::G2_STAGES; ++q) {
                             if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x3102)) { ok = false; break; }
@@ -250,20 +287,23 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             const uint64_t rdesc32 = umma_sdesc_sw32(rS);
             const uint64_t idB = umma_sdesc_sw32(smem_u32(sI));
             constexpr uint64_t kStageDesc = C::SB >> 4;               // descriptor start-address step per stage
-            // A is released slab by slab after GEMM1(NC-1), or after the identity pass when that
-            // reads A and comes later
-            const bool a_after_id = p.res_mode == RES_FROM_A && s_r >= NC - 1;
+            uint32_t ubase = 0;                                        // chunks of the items before this one
             int s = 0;
             uint32_t ph = 0;
             int lt = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < ntile && ok; t += gridDim.x, ++lt) {
+            int t, c0, c1, sp;
+            for (; ok && item(lt, t, c0, c1, sp); ++lt) {
+                const int nc = c1 - c0, n_steps = nc + LAG, s_r = c0 == 0 ? id_step(nc) : -1;
+                // A is released slab by slab after the item's last GEMM1, or after the identity pass
+                // when that reads A and comes later
+                const bool a_after_id = p.res_mode == RES_FROM_A && s_r >= nc - 1;
                 if (!wait_or_abort(a_full, lt & 1, abort_flag, 0x3200)) break;
                 tc_fence_after();
 #pragma unroll 1
                 for (int step = 0; step < n_steps && ok; ++step) {
-                    if (step < NC) {                                   // ---- GEMM1(step)
-                        const uint32_t use = lt * NC + step;
+                    if (step < nc) {                                   // ---- GEMM1(c0 + step)
+                        const uint32_t use = ubase + step;
                         bool rdy[C::G1_STAGES];
                         const bool e_rdy = mbar_test(g1_empty, (use & 1) ^ 1);
                         {
@@ -288,15 +328,15 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             for (int kk = 0; kk < 4; ++kk)
                                 umma_bf16(tmem + C::G1COL, adesc[q * 4 + kk], bd + 2 * kk, idesc1, (q | kk) != 0);
                             umma_commit(&empty[s]);
-                            if (step == NC - 1 && !a_after_id) umma_commit(&a_empty[q]);
+                            if (step == nc - 1 && !a_after_id) umma_commit(&a_empty[q]);
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                         if (!ok) break;
                         umma_commit(g1_full);
                     }
-                    if (step >= LAG) {                                 // ---- GEMM2(step - LAG)
-                        const int c = step - LAG;
-                        const uint32_t use = lt * NC + c;
+                    if (step >= LAG) {                                 // ---- GEMM2(c0 + step - LAG)
+                        const int c = step - LAG;                      // relative to c0
+                        const uint32_t use = ubase + c;
                         if (c == 0) {                                  // GEMM2(0) initialises Y: wait until it is free
                             if (!wait_or_abort(y_empty, (lt & 1) ^ 1, abort_flag, 0x3204)) { ok = false; break; }
                             tc_fence_after();
@@ -364,6 +404,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                     }
                     if (step == n_steps - 1) umma_commit(y_full);
                 }
+                ubase += nc;
             }
             umma_commit(drain);
             wait_or_abort(drain, 0, abort_flag, 0x3206);
@@ -481,6 +522,93 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             }
             return true;
         };
+        // One half of a split tile: this half's partial Y (fp32, rows of W) goes to p.part; for each
+        // warp's slice an atomic counter names the half that finishes second, which adds the other
+        // half's partial and writes the output.  fp32 a + b is commutative, so the result does not
+        // depend on which half that is; no CTA waits for another.
+        auto output_split = [&](int g, int m, int ylt, int sp, int st) -> bool {
+            if (!wait_or_abort(y_full, ylt & 1, abort_flag, 0x3303)) return false;
+            tc_fence_after();
+            const size_t row = (size_t)(q * 32 + lane);
+            float* mine = p.part + (((size_t)sp * n_rem + st) * 128 + row) * W + half * (W / 2);
+            const float* other = p.part + (((size_t)(1 - sp) * n_rem + st) * 128 + row) * W + half * (W / 2);
+#pragma unroll 1
+            for (int j = 0; j < W / 64; ++j) {
+                uint32_t v[32];
+                tmem_ld32_async(trow + half * (W / 2) + j * 32, v);
+                tmem_wait_ld_tie(v);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t w8[8] = {v[e * 8 + 0], v[e * 8 + 1], v[e * 8 + 2], v[e * 8 + 3],
+                                            v[e * 8 + 4], v[e * 8 + 5], v[e * 8 + 6], v[e * 8 + 7]};
+                    st_global_v8(mine + j * 32 + e * 8, w8);
+                }
+            }
+            __threadfence();
+            __syncwarp();
+            int second = 0;
+            if (lane == 0) second = atomicAdd(&p.cnt[st * 8 + (warp - 2)], 1);
+            second = __shfl_sync(0xffffffffu, second, 0);
+            if (!second) {                                             // first: the other half finishes
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(y_empty);
+                return true;
+            }
+            __threadfence();
+            const int b0 = m * 128 + q * 32;
+#pragma unroll 1
+            for (int j2 = 0; j2 < W / 128; ++j2) {                     // 64 columns per round
+                const int col0 = half * (W / 2) + j2 * 64;
+                if (j2 > 0) {                                          // the previous round's store has read the rows
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t v[32];
+                    tmem_ld32_async(trow + col0 + hh * 32, v);
+                    tmem_wait_ld_tie(v);
+                    if (j2 == W / 128 - 1 && hh == 1) {                 // Y fully read: release it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(y_empty);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {                      // 8 columns per 16-byte piece
+                        uint32_t o8[8];
+                        ld_global_cg_v8(other + j2 * 64 + hh * 32 + e * 8, o8);
+                        float f[8];
+#pragma unroll
+                        for (int z = 0; z < 8; ++z) f[z] = __uint_as_float(v[e * 8 + z]) + __uint_as_float(o8[z]);
+                        const uint4 w4 = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                    pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+                        const int c8 = hh * 4 + e;
+                        uint8_t* dst = AMODE == A_TMA_MIX
+                                           ? stg + (c8 >> 1) * 1024 + lane * 32 + (((c8 & 1) ^ ((lane >> 2) & 1)) << 4)
+                                           : stg + lane * 128 + ((c8 ^ (lane & 7)) << 4);
+                        *reinterpret_cast<uint4*>(dst) = w4;
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && b0 < p.rows) {
+                    if (AMODE == A_TMA_MIX) {
+                        const int per = p.omap.dh >> 4;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int ci = (col0 >> 4) + k, tok = ci / per, jj = ci - tok * per;
+                            tma_store_4d(&tmO, stg + k * 1024, 0, g * per + jj, tok, b0);
+                        }
+                    } else {
+                        tma_store_3d(&tmO, stg, col0, g, b0);
+                    }
+                    bulk_commit_group();
+                }
+                __syncwarp();
+            }
+            return true;
+        };
         int lt = 0;
         float sc = 0.f;
         // the statistics of a tile read the A slabs of this thread's half; release them afterwards
@@ -491,15 +619,21 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                 for (int qa = 0; qa < C::G1_STAGES / 2; ++qa) mbar_arrive(&a_empty[half * (C::G1_STAGES / 2) + qa]);
             }
         };
-        bool ok = wait_or_abort(a_full, 0, abort_flag, 0x3300) && row_scale((int)blockIdx.x % mt, sc);
+        int t, c0, c1, sp;
+        bool have = item(0, t, c0, c1, sp);
+        bool ok = have && wait_or_abort(a_full, 0, abort_flag, 0x3300) && row_scale(t % mt, sc);
         if (ok) release_a();
-        int prev_g = 0, prev_m = 0;
-        for (int t = blockIdx.x; t < ntile && ok; t += gridDim.x, ++lt) {
+        int prev_g = 0, prev_m = 0, prev_sp = -1, prev_st = 0;
+        auto output_prev = [&](int ylt) -> bool {
+            return prev_sp < 0 ? output_tile(prev_g, prev_m, ylt) : output_split(prev_g, prev_m, ylt, prev_sp, prev_st);
+        };
+        uint32_t ubase = 0;                                            // chunks of the items before this one
+        for (; ok && have; ++lt) {
             const int g = t / mt, m = t - g * mt;
             // ---- SwiGLU chunks: this thread owns hidden columns [half*64, half*64 + 64) of its row
 #pragma unroll 1
-            for (int c = 0; c < NC; ++c) {
-                const uint32_t use = lt * NC + c;
+            for (int c = c0; c < c1; ++c) {
+                const uint32_t use = ubase + (c - c0);
                 if (!wait_or_abort(g1_full, use & 1, abort_flag, 0x3301)) { ok = false; break; }
                 tc_fence_after();
                 // all four loads in flight, one wait, then the GEMM1 buffer is released before the math
@@ -527,11 +661,11 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                     pk[i] = pack_bf16x2(h0.x, h0.y);
                     pk[16 + i] = pack_bf16x2(h1.x, h1.y);
                 }
-                if (c == 0 && lt > 0) {
-                    // the previous tile's output, now that GEMM1(1) of this tile can run (its buffer is
-                    // released above); the hidden rows are its staging, so this chunk's hidden write
-                    // waits until the bulk stores have read them
-                    if (!output_tile(prev_g, prev_m, lt - 1)) { ok = false; break; }
+                if (c == c0 && lt > 0) {
+                    // the previous item's output, now that this item's second GEMM1 can run (the
+                    // buffer is released above); the hidden rows are its staging, so this chunk's
+                    // hidden write waits until the bulk stores have read them
+                    if (!output_prev(lt - 1)) { ok = false; break; }
                     if (lane == 0) bulk_wait_read_all();
                     __syncwarp();
                 }
@@ -547,16 +681,22 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                 if (lane == 0) mbar_arrive(hid_full);
             }
             if (!ok) break;
-            // ---- statistics of the next tile (its A tile is loaded once this tile's last read of A is issued)
-            if (t + (int)gridDim.x < ntile) {
-                if (!wait_or_abort(a_full, (lt + 1) & 1, abort_flag, 0x3304) || !row_scale((t + (int)gridDim.x) % mt, sc))
-                    break;
-                release_a();
-            }
+            ubase += c1 - c0;
             prev_g = g;
             prev_m = m;
+            prev_sp = sp;
+            prev_st = t - full_waves * (int)gridDim.x;
+            // ---- statistics of the next item (its A tile is loaded once this item's last read of A is issued)
+            have = item(lt + 1, t, c0, c1, sp);
+            if (have) {
+                if (!wait_or_abort(a_full, (lt + 1) & 1, abort_flag, 0x3304) || !row_scale(t % mt, sc)) {
+                    ok = false;
+                    break;
+                }
+                release_a();
+            }
         }
-        if (ok && lt > 0) ok = output_tile(prev_g, prev_m, lt - 1);
+        if (ok && lt > 0) ok = output_prev(lt - 1);
         if (lane == 0) bulk_wait_all();                                // stores complete before exit
         __syncwarp();
     }
