@@ -472,13 +472,25 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
         SimtGemmArgs a{p, (const float*)x, (const float*)weg, (const float*)weu};
         if ((s = cuda_status(launch_simt_gemm(EPI_SWIGLU, a, (int)(max_mt * p.n_tiles), st))) != TM_OK) return s;
     } else {
+        // MoEPermute: copy the routed rows into bucket order (the slot buffer, [routed, W], is free
+        // until the routed GEMM2 writes it), then GEMM1 reads A as contiguous rows through a 2-D
+        // tensor map.  TM_MOE_GATHER=1 keeps the row gather inside GEMM1 (cp.async; comparison).
+        const char* env_g = getenv("TM_MOE_GATHER");
+        const bool gather_in_gemm = env_g && env_g[0] == '1';
         const int bn = pick_bn_swiglu(Fe);
         p.n_tiles = p.N / bn;
-        CUtensorMap none, mg, mu;
-        memset(&none, 0, sizeof(none));
+        CUtensorMap ma, mg, mu;
+        memset(&ma, 0, sizeof(ma));
         if (!map_2d(&mg, weg, G * Fe, g.W, bn / 2) || !map_2d(&mu, weu, G * Fe, g.W, bn / 2)) return TM_ERR_CUDA;
+        if (!gather_in_gemm) {
+            if ((s = cuda_status(launch_gather_rows(g.dtype, x, g.map, g.B, w->E, m.offsets, (int)G, m.bucket_rows, routed,
+                                                    m.slots, st))) != TM_OK)
+                return s;
+            if (!map_2d(&ma, m.slots, routed, g.W, 128)) return TM_ERR_CUDA;
+        }
         const long grid = max_mt * p.n_tiles < num_sms() ? max_mt * p.n_tiles : num_sms();
-        if ((s = cuda_status(launch_grouped_gemm(bn, A_GATHER, EPI_SWIGLU, none, mg, mu, p, (int)grid, st))) != TM_OK)
+        if ((s = cuda_status(launch_grouped_gemm(bn, gather_in_gemm ? A_GATHER : A_TMA_2D, EPI_SWIGLU, ma, mg, mu, p,
+                                                 (int)grid, st))) != TM_OK)
             return s;
     }
     // shared expert GEMM1 (dense rows)

@@ -122,6 +122,7 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
     X(256, A_TMA_3D, EPI_SWIGLU) X(128, A_TMA_3D, EPI_SWIGLU) \
     X(256, A_TMA_MIX, EPI_SWIGLU) X(128, A_TMA_MIX, EPI_SWIGLU) \
     X(256, A_GATHER, EPI_SWIGLU) X(128, A_GATHER, EPI_SWIGLU) \
+    X(256, A_TMA_2D, EPI_SWIGLU) X(128, A_TMA_2D, EPI_SWIGLU) \
     X(256, A_TMA_2D, EPI_RESID) X(192, A_TMA_2D, EPI_RESID) X(128, A_TMA_2D, EPI_RESID) \
     X(256, A_TMA_2D, EPI_SLOT) X(192, A_TMA_2D, EPI_SLOT) X(128, A_TMA_2D, EPI_SLOT) \
     X(256, A_TMA_2D, EPI_COMBINE) X(192, A_TMA_2D, EPI_COMBINE) X(128, A_TMA_2D, EPI_COMBINE)

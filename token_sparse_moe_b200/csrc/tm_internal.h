@@ -57,6 +57,9 @@ cudaError_t launch_offsets(const int32_t* counts_in, int32_t* chunk_prefix, int 
                            int32_t* bucket_offsets, int32_t* tile_start, cudaStream_t st);
 cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, const int32_t* bucket_offsets, int B,
                            int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st);
+// MoEPermute data copy: routed row positions receive their source rows (see gather_rows_kernel)
+cudaError_t launch_gather_rows(int dtype, const void* x, RowMap m, int B, int E, const int32_t* offsets, int groups,
+                               const int32_t* bucket_rows, size_t routed, void* out, cudaStream_t st);
 cudaError_t launch_permute(int dtype, const void* src, void* dst, int B, int T, int D, int H, bool to_mixed,
                            cudaStream_t st);
 cudaError_t launch_fold_gain(int dtype, const void* w, const void* gain, void* out, size_t rows, int width,

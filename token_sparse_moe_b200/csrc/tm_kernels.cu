@@ -434,6 +434,43 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtGemmArgs a) {
     }
 }
 
+// MoEPermute, data part: row position pos of the bucketed order (bank-major, then expert, then
+// ascending sample) receives a copy of its source row (sample bucket_rows[pos], bank of the
+// position's group) read through the row map, so that the routed GEMM1 reads its A operand as
+// plain contiguous rows.  One warp per position; 16-byte pieces when a head segment holds whole
+// pieces, element copies otherwise.
+template <typename T>
+__global__ void __launch_bounds__(256) gather_rows_kernel(const T* __restrict__ x, RowMap m, int B, int E,
+                                                          const int32_t* __restrict__ offsets, int groups,
+                                                          const int32_t* __restrict__ bucket_rows, int routed,
+                                                          T* __restrict__ out) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int W = m.W;
+    constexpr int V = 16 / sizeof(T);
+    const bool vec = (m.layout == 0 || m.dh % V == 0) && W % V == 0;
+    for (int pos = warp; pos < routed; pos += nwarps) {
+        int lo = 0, hi = groups;   // offsets[lo] <= pos < offsets[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(&offsets[mid]) <= pos) lo = mid; else hi = mid;
+        }
+        const int bank = lo / E;
+        const int b = __ldg(&bucket_rows[pos]);
+        if (b < 0 || b >= B) {
+            if (lane == 0) record_error(ERR_BOUNDS, 0x520);
+            continue;
+        }
+        T* dst = out + (size_t)pos * W;
+        if (vec) {
+            for (int c = lane * V; c < W; c += 32 * V)
+                *reinterpret_cast<uint4*>(dst + c) = __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c)));
+        } else {
+            for (int c = lane; c < W; c += 32) dst[c] = x[row_elem(m, b, bank, c)];
+        }
+    }
+}
+
 // ------------------------------------------------------------------ launchers
 static int grid_for(size_t n, int threads) {
     size_t g = (n + threads - 1) / threads;
@@ -499,6 +536,19 @@ cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, cons
     dim3 grid((B + kRouterChunk - 1) / kRouterChunk, banks);
     scatter_kernel<<<grid, kRouterChunk, 0, st>>>(idx, chunk_prefix, bucket_offsets, B, banks, E, k, bucket_rows,
                                                   slot_of);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(int dtype, const void* x, RowMap m, int B, int E, const int32_t* offsets, int groups,
+                               const int32_t* bucket_rows, size_t routed, void* out, cudaStream_t st) {
+    ProfileScope ps_("moe_permute", st);
+    const int grid = grid_for(routed * 32, 256);
+    if (dtype == 1)
+        gather_rows_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, m, B, E, offsets, groups,
+                                                                bucket_rows, (int)routed, (__nv_bfloat16*)out);
+    else
+        gather_rows_kernel<float><<<grid, 256, 0, st>>>((const float*)x, m, B, E, offsets, groups, bucket_rows,
+                                                        (int)routed, (float*)out);
     return cudaGetLastError();
 }
 
