@@ -380,7 +380,7 @@ tm_status run_dense(const Geo& g, const void* x, const void* resid, const void* 
 // ------------------------------------------------------------------ MoE sub-layer
 struct MoeWs {
     float* inv_rms;
-    int32_t *idx, *slot_of, *bucket_rows, *offsets, *tile_start, *counts;
+    int32_t *idx, *slot_of, *bucket_rows, *offsets, *tile_start, *counts, *perm;
     float* gate;
     void *hidden_r, *slots, *hidden_s;
     void *weg, *weu, *wsg, *wsu;
@@ -396,6 +396,7 @@ MoeWs carve_moe(Carve& c, const Geo& g, const tm_moe_w* w, bool gain) {
     m.gate = c.take<float>(routed);
     m.slot_of = c.take<int32_t>(routed);
     m.bucket_rows = c.take<int32_t>(routed);
+    m.perm = c.take<int32_t>(routed);
     m.offsets = c.take<int32_t>(G + 1);
     m.tile_start = c.take<int32_t>(G + 1);
     m.counts = c.take<int32_t>((size_t)g.banks * nchunks * w->E);
@@ -412,6 +413,7 @@ MoeWs carve_moe(Carve& c, const Geo& g, const tm_moe_w* w, bool gain) {
 struct RouteOut {
     int32_t *idx, *offsets, *tile_start, *bucket_rows, *slot_of, *counts;
     float *gate, *inv_rms;
+    int32_t* perm = nullptr;   // optional: sample-order row of each bucket position
 };
 
 tm_status run_route(const Geo& g, const void* x, const void* gain, const tm_moe_w* w, const RouteOut& r,
@@ -424,7 +426,44 @@ tm_status run_route(const Geo& g, const void* x, const void* gain, const tm_moe_
     if ((s = cuda_status(launch_offsets(r.counts, r.counts, g.banks, nchunks, w->E, r.offsets, r.tile_start, st))) !=
         TM_OK)
         return s;
-    return cuda_status(launch_scatter(r.idx, r.counts, r.offsets, g.B, g.banks, w->E, w->k, r.bucket_rows, r.slot_of, st));
+    return cuda_status(launch_scatter(r.idx, r.counts, r.offsets, g.B, g.banks, w->E, w->k, r.bucket_rows, r.slot_of, st,
+                                      r.perm));
+}
+
+// MoE combine on the tensor core: Y = residual (+ inter-residual) + sum_j (gate-scaled expert row j
+// of the sample) + Shared(n), one grouped-GEMM launch: the sources enter the accumulator through
+// identity MMAs (tensor maps in the output's row geometry and over the sample-order expert rows
+// [B, banks, k, W]), then the shared expert's GEMM2 accumulates onto them.
+tm_status combine_sum(const Geo& g, const void* hidden_s, const void* wd, int Fs, const void* resid, const void* extra,
+                      void* y, const void* slots, int k, cudaStream_t st) {
+    GemmParams p = base_params(g);
+    p.sched = 0;
+    p.K = Fs;
+    p.N = g.W;
+    p.out = (__nv_bfloat16*)y;
+    p.out_elems = (size_t)g.B * g.banks * g.W;
+    p.k = k;
+    p.src_resid = resid != nullptr;
+    p.src_extra = extra != nullptr;
+    const int am = gemm1_amode(g);                  // the residual's geometry is that of x's rows
+    p.src_mix = am == A_TMA_MIX;
+    if (am != A_TMA_MIX && am != A_TMA_3D) return TM_ERR_UNSUPPORTED;
+    const int bn = pick_bn_out(g.W);
+    p.n_tiles = g.W / bn;
+    CUtensorMap ma, mb, m0, m1, m2;
+    memset(&m0, 0, sizeof(m0));
+    memset(&m1, 0, sizeof(m1));
+    if (!map_2d(&ma, hidden_s, (uint64_t)g.banks * g.B, Fs, 128) || !map_2d(&mb, wd, (uint64_t)g.banks * g.W, Fs, bn))
+        return TM_ERR_CUDA;
+    if (resid && !gemm1_amap(g, resid, am, &m0)) return TM_ERR_CUDA;
+    if (extra && !gemm1_amap(g, extra, am, &m1)) return TM_ERR_CUDA;
+    {
+        uint64_t dims[4] = {(uint64_t)g.W, (uint64_t)k, (uint64_t)g.banks, (uint64_t)g.B};
+        uint64_t strides[3] = {(uint64_t)g.W * 2, (uint64_t)k * g.W * 2, (uint64_t)g.banks * k * g.W * 2};
+        uint32_t box[4] = {64, 1, 1, 128};
+        if (!make_map(&m2, slots, 4, dims, strides, box)) return TM_ERR_CUDA;
+    }
+    return cuda_status(launch_grouped_gemm_src(bn, A_TMA_2D, EPI_SUM, ma, mb, mb, m0, m1, m2, p, dense_grid(p), st));
 }
 
 tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* extra, const void* gain,
@@ -446,6 +485,8 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
         weg = m.weg; weu = m.weu; wsg = m.wsg; wsu = m.wsu;
     }
     RouteOut r{m.idx, m.offsets, m.tile_start, m.bucket_rows, m.slot_of, m.counts, m.gate, m.inv_rms};
+    const bool bf16_path = g.dtype == TM_BF16;
+    if (bf16_path) r.perm = m.perm;
     if ((s = run_route(g, x, gain, w, r, st)) != TM_OK) return s;
 
     const size_t routed = (size_t)g.B * g.banks * w->k;
@@ -506,13 +547,18 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
         SimtGemmArgs a{p, (const float*)m.hidden_r, (const float*)w->we_down, nullptr};
         if ((s = cuda_status(launch_simt_gemm(EPI_SLOT, a, (int)(max_mt * p.n_tiles), st))) != TM_OK) return s;
     } else {
+        // rows written in sample order ((b * banks + bank) * k + j) and scaled by their gate, so that
+        // the combine reads each tile's expert rows as one tensor-map box per choice
         const int bn = pick_bn_out(g.W);
         p.n_tiles = g.W / bn;
+        p.perm = m.perm;
+        p.gate = m.gate;
         CUtensorMap ma, mb;
         if (!map_2d(&ma, m.hidden_r, routed, Fe, 128) || !map_2d(&mb, w->we_down, G * g.W, Fe, bn)) return TM_ERR_CUDA;
         const long grid = max_mt * p.n_tiles < num_sms() ? max_mt * p.n_tiles : num_sms();
-        if ((s = cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SLOT, ma, mb, mb, p, (int)grid, st))) != TM_OK)
+        if ((s = cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SLOT_PERM, ma, mb, mb, p, (int)grid, st))) != TM_OK)
             return s;
+        return combine_sum(g, m.hidden_s, w->ws_down, w->hidden_s, resid, extra, y, m.slots, w->k, st);
     }
     // shared expert GEMM2 + deterministic combine + residual(s), stored through the row map
     return gemm2_dense(g, m.hidden_s, w->ws_down, w->hidden_s, EPI_COMBINE, resid, extra, y, m.gate, m.slot_of,

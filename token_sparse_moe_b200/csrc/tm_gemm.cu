@@ -100,8 +100,8 @@ cudaError_t launch_fused(int W, int a_mode, const CUtensorMap& a, const CUtensor
 }
 
 template <int BN, int AM, int EPI>
-static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmParams& p,
-                              int grid, cudaStream_t st) {
+static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& s0,
+                              const CUtensorMap& s1, const CUtensorMap& s2, const GemmParams& p, int grid, cudaStream_t st) {
     using C = GemmCfg<BN, AM>;
     auto kern = grouped_gemm_kernel<BN, AM, EPI>;
     static bool configured = false;   // attribute set once per instantiation (per process)
@@ -110,8 +110,12 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    ProfileScope ps_(EPI == EPI_SWIGLU ? "gemm_swiglu" : EPI == EPI_RESID ? "gemm_resid" : EPI == EPI_SLOT ? "gemm_slot" : "gemm_combine", st);
-    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, b0, b1, p);
+    ProfileScope ps_(EPI == EPI_SWIGLU                          ? "gemm_swiglu"
+                     : EPI == EPI_RESID                         ? "gemm_resid"
+                     : (EPI == EPI_SLOT || EPI == EPI_SLOT_PERM) ? "gemm_slot"
+                                                                 : "gemm_combine",
+                     st);
+    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, b0, b1, s0, s1, s2, p);
     return cudaGetLastError();
 }
 
@@ -125,7 +129,9 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
     X(256, A_TMA_2D, EPI_SWIGLU) X(128, A_TMA_2D, EPI_SWIGLU) \
     X(256, A_TMA_2D, EPI_RESID) X(192, A_TMA_2D, EPI_RESID) X(128, A_TMA_2D, EPI_RESID) \
     X(256, A_TMA_2D, EPI_SLOT) X(192, A_TMA_2D, EPI_SLOT) X(128, A_TMA_2D, EPI_SLOT) \
-    X(256, A_TMA_2D, EPI_COMBINE) X(192, A_TMA_2D, EPI_COMBINE) X(128, A_TMA_2D, EPI_COMBINE)
+    X(256, A_TMA_2D, EPI_COMBINE) X(192, A_TMA_2D, EPI_COMBINE) X(128, A_TMA_2D, EPI_COMBINE) \
+    X(256, A_TMA_2D, EPI_SLOT_PERM) X(192, A_TMA_2D, EPI_SLOT_PERM) X(128, A_TMA_2D, EPI_SLOT_PERM) \
+    X(256, A_TMA_2D, EPI_SUM) X(192, A_TMA_2D, EPI_SUM) X(128, A_TMA_2D, EPI_SUM)
 
 bool grouped_gemm_supported(int bn, int a_mode, int epi) {
 #define X(BN, AM, EP) if (bn == BN && a_mode == AM && epi == EP) return true;
@@ -143,13 +149,22 @@ int grouped_gemm_smem(int bn, int a_mode) {
     }
 }
 
-cudaError_t launch_grouped_gemm(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
-                                const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st) {
-#define X(BN, AM, EP) \
-    if (bn == BN && a_mode == AM && epi == EP) return launch_one<BN, AM, EP>(tmA, tmB0, tmB1, p, grid, st);
+cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
+                                    const CUtensorMap& tmB1, const CUtensorMap& tmS0, const CUtensorMap& tmS1,
+                                    const CUtensorMap& tmS2, const GemmParams& p, int grid, cudaStream_t st) {
+#define X(BN, AM, EP)                                  \
+    if (bn == BN && a_mode == AM && epi == EP)         \
+        return launch_one<BN, AM, EP>(tmA, tmB0, tmB1, tmS0, tmS1, tmS2, p, grid, st);
     TM_GEMM_TABLE(X)
 #undef X
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_grouped_gemm(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
+                                const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st) {
+    CUtensorMap none;
+    memset(&none, 0, sizeof(none));
+    return launch_grouped_gemm_src(bn, a_mode, epi, tmA, tmB0, tmB1, none, none, none, p, grid, st);
 }
 
 }  // namespace tml

@@ -25,7 +25,10 @@
 namespace tml {
 
 enum AMode : int { A_TMA_2D = 0, A_TMA_3D = 1, A_TMA_MIX = 2, A_GATHER = 3 };
-enum Epi : int { EPI_SWIGLU = 0, EPI_RESID = 1, EPI_SLOT = 2, EPI_COMBINE = 3 };
+// EPI_SLOT_PERM: routed GEMM2 rows written in sample order (row perm[pos]) and scaled by their gate.
+// EPI_SUM: the combine with its sources (residual, inter-residual, the k gate-scaled expert rows of
+// each sample) added on the tensor core before the shared expert's GEMM2; plain output epilogue.
+enum Epi : int { EPI_SWIGLU = 0, EPI_RESID = 1, EPI_SLOT = 2, EPI_COMBINE = 3, EPI_SLOT_PERM = 4, EPI_SUM = 5 };
 
 // Where element c of the row (sample b, bank) of a sub-layer lives in a tensor.
 //   layout 0 (rows):  [B, banks, W]
@@ -67,6 +70,9 @@ struct GemmParams {
     const int* slot_of;        // combine: [B, banks, k]
     const __nv_bfloat16* slots;// combine: [row positions, W]
     int k;
+    const int* perm;           // EPI_SLOT_PERM: sample-order row (b * banks + bank) * k + j of each position
+    int src_resid, src_extra;  // EPI_SUM: residual / inter-residual present (maps tmS0 / tmS1)
+    int src_mix;               // EPI_SUM: residual maps use the 4-D mixed geometry (16-column boxes)
 };
 
 template <int BN, int AMODE>
@@ -79,7 +85,8 @@ struct GemmCfg {
     static constexpr int NWARPS = AMODE == A_GATHER ? 10 : 6;
     static constexpr int NTHREADS = NWARPS * 32;
     static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+    static constexpr int OFF_ID = STAGES * STAGE_BYTES;           // 16 x 16 identity (EPI_SUM), 1 KB
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024 + 256;
 };
 
 struct TileInfo {
@@ -134,15 +141,21 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 template <int BN, int AMODE, int EPI>
 __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                        const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
+                        const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmS0,
+                        const __grid_constant__ CUtensorMap tmS1, const __grid_constant__ CUtensorMap tmS2,
+                        const GemmParams p) {
     using C = GemmCfg<BN, AMODE>;
     constexpr int STAGES = C::STAGES;
     const int ntile = total_tiles(p);
     if ((int)blockIdx.x >= ntile) return;
+    // EPI_SUM source stages per tile: residual, inter-residual, then expert choice j = 0..k-1, each
+    // as BN / 64 slabs of 128 rows x 64 columns (one ring stage each, A part only)
+    const int n_src = EPI == EPI_SUM ? (p.src_resid + p.src_extra + p.k) : 0;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+    uint8_t* sI = smem + C::OFF_ID;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_ID + 1024);
     uint64_t* empty = full + STAGES;
     uint64_t* acc_full = empty + STAGES;
     uint64_t* acc_empty = acc_full + 2;
@@ -167,6 +180,16 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
+    if (EPI == EPI_SUM && warp == 0) {
+        // identity B operand: 16 rows n x 16 columns k, 32-byte rows, 32-byte swizzle (the 16-byte
+        // half of row n that holds column k sits at half (k / 8) ^ ((n / 4) % 2))
+        const int n = lane & 15, hf = lane >> 4;
+        const uint32_t one = (n >> 3) == hf ? ((n & 1) ? 0x3F800000u : 0x00003F80u) : 0u;
+        const int wi = (n & 7) >> 1;
+        *reinterpret_cast<uint4*>(sI + n * 32 + ((hf ^ ((n >> 2) & 1)) << 4)) =
+            make_uint4(wi == 0 ? one : 0u, wi == 1 ? one : 0u, wi == 2 ? one : 0u, wi == 3 ? one : 0u);
+        fence_proxy_async_smem();
+    }
     if (warp == 1) {
         tmem_alloc(tmem_base_smem, C::TMEM_COLS);
         tmem_relinquish();
@@ -186,6 +209,35 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
             uint32_t ph = 0;
             for (int t = blockIdx.x; t < ntile; t += gridDim.x) {
                 const TileInfo ti = decode_tile(p, t);
+                if (EPI == EPI_SUM) {
+                    // source slabs: rows of this tile's samples, output columns n*BN .. +BN
+#pragma unroll 1
+                    for (int src = 0; src < n_src; ++src) {
+                        const int kind = src < p.src_resid ? 0 : (src < p.src_resid + p.src_extra ? 1 : 2);
+                        const int j = src - p.src_resid - p.src_extra;
+#pragma unroll 1
+                        for (int sl = 0; sl < BN / 64; ++sl) {
+                            if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x103)) goto producer_done;
+                            uint8_t* sa = smem + s * C::STAGE_BYTES;
+                            mbar_arrive_expect_tx(&full[s], C::A_BYTES);
+                            const int col = ti.n * BN + sl * 64;
+                            if (kind == 2) {
+                                tma_load_4d(sa, &tmS2, &full[s], col, j, ti.g, ti.m * 128);
+                            } else if (p.src_mix) {
+                                const int per = p.omap.dh >> 4;
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    const int c16 = (col >> 4) + i, tk = c16 / per, jj = c16 - tk * per;
+                                    tma_load_4d(sa + i * 4096, kind == 0 ? &tmS0 : &tmS1, &full[s], 0, ti.g * per + jj, tk,
+                                                ti.m * 128);
+                                }
+                            } else {
+                                tma_load_3d(sa, kind == 0 ? &tmS0 : &tmS1, &full[s], col, ti.g, ti.m * 128);
+                            }
+                            if (++s == STAGES) { s = 0; ph ^= 1; }
+                        }
+                    }
+                }
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x100)) goto producer_done;
                     uint8_t* sa = smem + s * C::STAGE_BYTES;
@@ -232,6 +284,30 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
                 tc_fence_after();
                 const uint32_t d = tmem_base + buf * BN;
                 bool ok = true;
+                if (EPI == EPI_SUM) {
+                    // Y = residual + inter-residual + sum_j gate_j expert_j: one N = 16 identity MMA per
+                    // 16 columns and source (bf16 times one summed in fp32 is exact)
+                    constexpr uint32_t idescI = umma_idesc_bf16(128, 16);
+                    const uint64_t idB = umma_sdesc_sw32(smem_u32(sI));
+#pragma unroll 1
+                    for (int src = 0; src < n_src && ok; ++src) {
+                        const bool mixed = src < p.src_resid + p.src_extra && p.src_mix;
+#pragma unroll 1
+                        for (int sl = 0; sl < BN / 64; ++sl) {
+                            if (!wait_or_abort(&full[s], ph, abort_flag, 0x203)) { ok = false; break; }
+                            tc_fence_after();
+                            const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint64_t a_k = mixed ? umma_sdesc_sw32(sa + kk * 4096) : umma_sdesc_sw128(sa) + 2 * kk;
+                                umma_bf16(d + sl * 64 + kk * 16, a_k, idB, idescI, src > 0 ? 1u : 0u);
+                            }
+                            umma_commit(&empty[s]);
+                            if (++s == STAGES) { s = 0; ph ^= 1; }
+                        }
+                    }
+                    if (!ok) break;
+                }
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!wait_or_abort(&full[s], ph, abort_flag, 0x201)) { ok = false; break; }
                     tc_fence_after();
@@ -244,7 +320,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
                         // A: one 32-byte-swizzled 4 KB sub-slab per K step (mixed rows) or the
                         // 128-byte-swizzled 64-wide slab advanced by 32 bytes per K step
                         const uint64_t a_k = AMODE == A_TMA_MIX ? umma_sdesc_sw32(sa + kk * 4096) : ad + 2 * kk;
-                        umma_bf16(d, a_k, bd + 2 * kk, idesc, (kb | kk) != 0);
+                        umma_bf16(d, a_k, bd + 2 * kk, idesc, (EPI == EPI_SUM && n_src > 0) || (kb | kk) != 0);
                     }
                     umma_commit(&empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -282,7 +358,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
                 record_error(ERR_BOUNDS, 0x310);
                 valid = false;
             }
-            if (valid && EPI != EPI_RESID && EPI != EPI_COMBINE &&
+            if (valid && EPI != EPI_RESID && EPI != EPI_COMBINE && EPI != EPI_SUM &&
                 (size_t)(pos + 1) * p.out_ld > p.out_elems) {
                 record_error(ERR_BOUNDS, 0x312);
                 valid = false;
@@ -306,6 +382,49 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
                         uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+            } else if (EPI == EPI_SLOT_PERM) {
+                // the row of choice j of sample b (bank of the group), scaled by its gate
+                const int e = valid ? __ldg(&p.perm[pos]) : 0;
+                if (valid && (e < 0 || e >= p.pos_limit)) {
+                    record_error(ERR_BOUNDS, 0x314);
+                    valid = false;
+                }
+                const float gsc = valid ? __ldg(&p.gate[e]) : 0.f;
+                __nv_bfloat16* dst = p.out + (size_t)e * p.out_ld + ti.n * BN;
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    float v[32];
+                    tmem_ld32(taddr + c, v);
+                    if (valid) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            d4[i] = make_uint4(pack_bf16x2(gsc * v[8 * i], gsc * v[8 * i + 1]),
+                                               pack_bf16x2(gsc * v[8 * i + 2], gsc * v[8 * i + 3]),
+                                               pack_bf16x2(gsc * v[8 * i + 4], gsc * v[8 * i + 5]),
+                                               pack_bf16x2(gsc * v[8 * i + 6], gsc * v[8 * i + 7]));
+                    }
+                }
+            } else if (EPI == EPI_SUM) {
+                // Y already holds every term: bf16 through the row map
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    float v[32];
+                    tmem_ld32(taddr + c, v);
+                    if (!valid) continue;
+                    const int col0 = ti.n * BN + c;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const size_t off = row_elem(p.omap, b, bank, col0 + 8 * i);
+                        if (off + 8 > p.out_elems) {
+                            record_error(ERR_BOUNDS, 0x315);
+                            continue;
+                        }
+                        *reinterpret_cast<uint4*>(p.out + off) =
+                            make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                                       pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
                     }
                 }
             } else if (EPI == EPI_SLOT) {

@@ -28,6 +28,11 @@ void note_cuda_error(const char* where, cudaError_t e);   // samples per router 
 
 // ---- tcgen05 grouped GEMM (bf16) ------------------------------------------------
 // a_mode: AMode; epi: Epi; bn: tile width.  maps are passed by value into the kernel.
+// with the EPI_SUM source maps: s0 residual, s1 inter-residual (row geometry of the output),
+// s2 the sample-order expert rows [B, banks, k, W]
+cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
+                                    const CUtensorMap& tmB1, const CUtensorMap& tmS0, const CUtensorMap& tmS1,
+                                    const CUtensorMap& tmS2, const GemmParams& p, int grid, cudaStream_t st);
 cudaError_t launch_grouped_gemm(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                                 const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st);
 bool grouped_gemm_supported(int bn, int a_mode, int epi);
@@ -56,7 +61,8 @@ cudaError_t launch_router(int dtype, const void* x, RowMap m, int B, float eps, 
 cudaError_t launch_offsets(const int32_t* counts_in, int32_t* chunk_prefix, int banks, int nchunks, int E,
                            int32_t* bucket_offsets, int32_t* tile_start, cudaStream_t st);
 cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, const int32_t* bucket_offsets, int B,
-                           int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st);
+                           int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st,
+                           int32_t* perm = nullptr);
 // MoEPermute data copy: routed row positions receive their source rows (see gather_rows_kernel)
 cudaError_t launch_gather_rows(int dtype, const void* x, RowMap m, int B, int E, const int32_t* offsets, int groups,
                                const int32_t* bucket_rows, size_t routed, void* out, cudaStream_t st);

@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kRouterChunk) scatter_kernel(const int32_t* __
                                                                const int32_t* __restrict__ chunk_prefix,
                                                                const int32_t* __restrict__ bucket_offsets, int B,
                                                                int banks, int E, int k, int32_t* __restrict__ bucket_rows,
-                                                               int32_t* __restrict__ slot_of) {
+                                                               int32_t* __restrict__ slot_of, int32_t* __restrict__ perm) {
     __shared__ int wcount[kRouterChunk / 32][64];
     const int bank = blockIdx.y, chunk = blockIdx.x, nchunks = gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -279,6 +279,7 @@ __global__ void __launch_bounds__(kRouterChunk) scatter_kernel(const int32_t* __
         }
         slot_of[rowi * k + j] = pos;
         bucket_rows[pos] = b;
+        if (perm) perm[pos] = (int32_t)(rowi * k + j);   // inverse of slot_of (optional)
     }
 }
 
@@ -531,11 +532,11 @@ cudaError_t launch_offsets(const int32_t* counts_in, int32_t* chunk_prefix, int 
 }
 
 cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, const int32_t* bucket_offsets, int B,
-                           int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st) {
+                           int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st, int32_t* perm) {
     ProfileScope ps_("route_scatter", st);
     dim3 grid((B + kRouterChunk - 1) / kRouterChunk, banks);
     scatter_kernel<<<grid, kRouterChunk, 0, st>>>(idx, chunk_prefix, bucket_offsets, B, banks, E, k, bucket_rows,
-                                                  slot_of);
+                                                  slot_of, perm);
     return cudaGetLastError();
 }
 
