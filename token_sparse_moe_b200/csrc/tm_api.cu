@@ -169,6 +169,14 @@ int gemm1_amode(const Geo& g) {
     if (g.map.layout == 0) return A_TMA_3D;
     return (g.map.dh % 16 == 0) ? A_TMA_MIX : A_GATHER;
 }
+// bytes of the split router weights when the tensor-core router applies (bf16 rows read through a
+// 3-D or mixed tensor map, E <= kRouteMaxE), else 0
+size_t route_split_bytes(const Geo& g, const tm_moe_w* w) {
+    const int am = gemm1_amode(g);
+    if (g.dtype != TM_BF16 || (am != A_TMA_3D && am != A_TMA_MIX) || w->E > kRouteMaxE) return 0;
+    return (size_t)g.banks * 64 * g.W * 2;
+}
+
 bool gemm1_amap(const Geo& g, const void* x, int amode, CUtensorMap* m, uint32_t box_rows = 128) {
     if (amode == A_TMA_3D) {
         uint64_t dims[3] = {(uint64_t)g.W, (uint64_t)g.banks, (uint64_t)g.B};
@@ -384,6 +392,7 @@ struct MoeWs {
     float* gate;
     void *hidden_r, *slots, *hidden_s;
     void *weg, *weu, *wsg, *wsu;
+    void* wsplit;
 };
 MoeWs carve_moe(Carve& c, const Geo& g, const tm_moe_w* w, bool gain) {
     MoeWs m;
@@ -403,6 +412,8 @@ MoeWs carve_moe(Carve& c, const Geo& g, const tm_moe_w* w, bool gain) {
     m.hidden_r = c.take<uint8_t>(routed * w->hidden_e * g.esz);
     m.slots = c.take<uint8_t>(routed * g.W * g.esz);
     m.hidden_s = w->hidden_s > 0 ? c.take<uint8_t>(rows * w->hidden_s * g.esz) : nullptr;
+    const size_t split = route_split_bytes(g, w);
+    m.wsplit = split ? c.take<uint8_t>(split) : nullptr;
     m.weg = gain ? c.take<uint8_t>(G * w->hidden_e * g.W * g.esz) : nullptr;
     m.weu = gain ? c.take<uint8_t>(G * w->hidden_e * g.W * g.esz) : nullptr;
     m.wsg = gain && w->hidden_s ? c.take<uint8_t>((size_t)g.banks * w->hidden_s * g.W * g.esz) : nullptr;
@@ -414,15 +425,45 @@ struct RouteOut {
     int32_t *idx, *offsets, *tile_start, *bucket_rows, *slot_of, *counts;
     float *gate, *inv_rms;
     int32_t* perm = nullptr;   // optional: sample-order row of each bucket position
+    void* wsplit = nullptr;    // optional: [banks][64][W] bf16 split router weights (tensor-core router)
 };
+
 
 tm_status run_route(const Geo& g, const void* x, const void* gain, const tm_moe_w* w, const RouteOut& r,
                     cudaStream_t st) {
     tm_status s;
-    if ((s = cuda_status(launch_router(g.dtype, x, g.map, g.B, g.eps, gain, w->w_router, w->E, w->k, w->alpha, r.idx,
-                                       r.gate, r.inv_rms, r.counts, st))) != TM_OK)
-        return s;
     const int nchunks = (g.B + kRouterChunk - 1) / kRouterChunk;
+    const char* env_r = getenv("TM_ROUTER_SIMT");
+    if (r.wsplit && route_split_bytes(g, w) > 0 && !(env_r && env_r[0] == '1')) {
+        // router on the tensor core: split weights, then one grouped-GEMM launch (N = 64) whose
+        // epilogue writes top-k, gates, 1/rms and the per-chunk expert counts (zeroed first)
+        const int am = gemm1_amode(g);
+        if ((s = cuda_status(cudaMemsetAsync(r.counts, 0, (size_t)g.banks * nchunks * w->E * sizeof(int32_t), st))) !=
+            TM_OK)
+            return s;
+        if ((s = cuda_status(launch_router_split(g.dtype, w->w_router, gain, g.banks, w->E, g.W, r.wsplit, st))) != TM_OK)
+            return s;
+        GemmParams p = base_params(g);
+        p.sched = 0;
+        p.K = g.W;
+        p.N = 64;
+        p.n_tiles = 1;
+        p.E = w->E;
+        p.k = w->k;
+        p.r_idx = r.idx;
+        p.r_gate = r.gate;
+        p.r_inv_rms = r.inv_rms;
+        p.r_counts = r.counts;
+        p.r_nchunks = nchunks;
+        p.r_alpha = w->alpha;
+        p.r_eps = g.eps;
+        CUtensorMap ma, mb;
+        if (!gemm1_amap(g, x, am, &ma) || !map_2d(&mb, r.wsplit, (uint64_t)g.banks * 64, g.W, 64)) return TM_ERR_CUDA;
+        if ((s = cuda_status(launch_grouped_gemm(64, am, EPI_ROUTE, ma, mb, mb, p, dense_grid(p), st))) != TM_OK) return s;
+    } else if ((s = cuda_status(launch_router(g.dtype, x, g.map, g.B, g.eps, gain, w->w_router, w->E, w->k, w->alpha,
+                                              r.idx, r.gate, r.inv_rms, r.counts, st))) != TM_OK) {
+        return s;
+    }
     if ((s = cuda_status(launch_offsets(r.counts, r.counts, g.banks, nchunks, w->E, r.offsets, r.tile_start, st))) !=
         TM_OK)
         return s;
@@ -487,6 +528,7 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
     RouteOut r{m.idx, m.offsets, m.tile_start, m.bucket_rows, m.slot_of, m.counts, m.gate, m.inv_rms};
     const bool bf16_path = g.dtype == TM_BF16;
     if (bf16_path) r.perm = m.perm;
+    r.wsplit = m.wsplit;
     if ((s = run_route(g, x, gain, w, r, st)) != TM_OK) return s;
 
     const size_t routed = (size_t)g.B * g.banks * w->k;
@@ -664,7 +706,8 @@ size_t tm_route_workspace_bytes(const tm_shape* shape, tm_layout layout, const t
     Geo g;
     if (!w || make_geo(shape, layout, w->banks, w->width, &g) != TM_OK || check_moe(g, w) != TM_OK) return 0;
     const int nchunks = (g.B + kRouterChunk - 1) / kRouterChunk;
-    return align256((size_t)g.banks * nchunks * w->E * sizeof(int32_t)) + align256(((size_t)g.banks * w->E + 1) * 4);
+    return align256((size_t)g.banks * nchunks * w->E * sizeof(int32_t)) + align256(((size_t)g.banks * w->E + 1) * 4) +
+           align256(route_split_bytes(g, w));
 }
 
 size_t tm_workspace_bytes(const tm_shape* shape, const tm_block* blocks, int L, int gap) {
@@ -719,6 +762,8 @@ tm_status tm_route_topk(const void* x, tm_layout layout, const tm_shape* shape, 
     int32_t* counts = c.take<int32_t>((size_t)g.banks * nchunks * w->E);
     int32_t* tiles = c.take<int32_t>((size_t)g.banks * w->E + 1);
     RouteOut r{topk_idx, bucket_offsets, tiles, bucket_rows, slot_of, counts, topk_gate, inv_rms};
+    const size_t split = route_split_bytes(g, w);
+    r.wsplit = split ? c.take<uint8_t>(split) : nullptr;
     return run_route(g, x, norm_gain, w, r, (cudaStream_t)stream);
 }
 

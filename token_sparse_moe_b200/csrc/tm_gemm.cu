@@ -102,7 +102,7 @@ cudaError_t launch_fused(int W, int a_mode, const CUtensorMap& a, const CUtensor
 template <int BN, int AM, int EPI>
 static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& s0,
                               const CUtensorMap& s1, const CUtensorMap& s2, const GemmParams& p, int grid, cudaStream_t st) {
-    using C = GemmCfg<BN, AM>;
+    using C = GemmCfg<BN, AM, EPI>;
     auto kern = grouped_gemm_kernel<BN, AM, EPI>;
     static bool configured = false;   // attribute set once per instantiation (per process)
     if (!configured) {
@@ -110,7 +110,8 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    ProfileScope ps_(EPI == EPI_SWIGLU                          ? "gemm_swiglu"
+    ProfileScope ps_(EPI == EPI_ROUTE                           ? "router"
+                     : EPI == EPI_SWIGLU                        ? "gemm_swiglu"
                      : EPI == EPI_RESID                         ? "gemm_resid"
                      : (EPI == EPI_SLOT || EPI == EPI_SLOT_PERM) ? "gemm_slot"
                                                                  : "gemm_combine",
@@ -131,7 +132,8 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
     X(256, A_TMA_2D, EPI_SLOT) X(192, A_TMA_2D, EPI_SLOT) X(128, A_TMA_2D, EPI_SLOT) \
     X(256, A_TMA_2D, EPI_COMBINE) X(192, A_TMA_2D, EPI_COMBINE) X(128, A_TMA_2D, EPI_COMBINE) \
     X(256, A_TMA_2D, EPI_SLOT_PERM) X(192, A_TMA_2D, EPI_SLOT_PERM) X(128, A_TMA_2D, EPI_SLOT_PERM) \
-    X(256, A_TMA_2D, EPI_SUM) X(192, A_TMA_2D, EPI_SUM) X(128, A_TMA_2D, EPI_SUM)
+    X(256, A_TMA_2D, EPI_SUM) X(192, A_TMA_2D, EPI_SUM) X(128, A_TMA_2D, EPI_SUM) \
+    X(64, A_TMA_3D, EPI_ROUTE) X(64, A_TMA_MIX, EPI_ROUTE)
 
 bool grouped_gemm_supported(int bn, int a_mode, int epi) {
 #define X(BN, AM, EP) if (bn == BN && a_mode == AM && epi == EP) return true;

@@ -28,7 +28,13 @@ enum AMode : int { A_TMA_2D = 0, A_TMA_3D = 1, A_TMA_MIX = 2, A_GATHER = 3 };
 // EPI_SLOT_PERM: routed GEMM2 rows written in sample order (row perm[pos]) and scaled by their gate.
 // EPI_SUM: the combine with its sources (residual, inter-residual, the k gate-scaled expert rows of
 // each sample) added on the tensor core before the shared expert's GEMM2; plain output epilogue.
-enum Epi : int { EPI_SWIGLU = 0, EPI_RESID = 1, EPI_SLOT = 2, EPI_COMBINE = 3, EPI_SLOT_PERM = 4, EPI_SUM = 5 };
+// EPI_ROUTE: the router on the tensor core; B holds each fp32 router row split exactly into three
+// bf16 rows (hi, mid, lo), the accumulator's columns e, E+e, 2E+e add up to the fp32 logit; four
+// extra warps take each row's sum of squares from the A stages as they pass; the epilogue does
+// the scale, softmax, top-k, gates and the per-chunk expert counts.
+enum Epi : int { EPI_SWIGLU = 0, EPI_RESID = 1, EPI_SLOT = 2, EPI_COMBINE = 3, EPI_SLOT_PERM = 4, EPI_SUM = 5,
+                 EPI_ROUTE = 6 };
+constexpr int kRouteMaxE = 21;   // 3 * E <= 64 accumulator columns
 
 // Where element c of the row (sample b, bank) of a sub-layer lives in a tensor.
 //   layout 0 (rows):  [B, banks, W]
@@ -73,16 +79,23 @@ struct GemmParams {
     const int* perm;           // EPI_SLOT_PERM: sample-order row (b * banks + bank) * k + j of each position
     int src_resid, src_extra;  // EPI_SUM: residual / inter-residual present (maps tmS0 / tmS1)
     int src_mix;               // EPI_SUM: residual maps use the 4-D mixed geometry (16-column boxes)
+    // EPI_ROUTE outputs ([B, banks, k] rows of top-k, [B, banks] 1/rms, [banks][chunks][E] counts)
+    int32_t* r_idx;
+    float* r_gate;
+    float* r_inv_rms;
+    int32_t* r_counts;
+    int r_nchunks;
+    float r_alpha, r_eps;
 };
 
-template <int BN, int AMODE>
+template <int BN, int AMODE, int EPI = EPI_SWIGLU>
 struct GemmCfg {
     static constexpr int BM = 128, BK = 64;
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 192 ? 5 : 6);
-    static constexpr int NWARPS = AMODE == A_GATHER ? 10 : 6;
+    static constexpr int NWARPS = (AMODE == A_GATHER || EPI == EPI_ROUTE) ? 10 : 6;
     static constexpr int NTHREADS = NWARPS * 32;
     static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
     static constexpr int OFF_ID = STAGES * STAGE_BYTES;           // 16 x 16 identity (EPI_SUM), 1 KB
@@ -139,12 +152,12 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 }
 
 template <int BN, int AMODE, int EPI>
-__global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
+__global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmS0,
                         const __grid_constant__ CUtensorMap tmS1, const __grid_constant__ CUtensorMap tmS2,
                         const GemmParams p) {
-    using C = GemmCfg<BN, AMODE>;
+    using C = GemmCfg<BN, AMODE, EPI>;
     constexpr int STAGES = C::STAGES;
     const int ntile = total_tiles(p);
     if ((int)blockIdx.x >= ntile) return;
@@ -160,7 +173,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
     uint64_t* acc_full = empty + STAGES;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
-    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* st_full = drain + 1;         // [2] EPI_ROUTE: row sums of squares of a tile written
+    uint64_t* st_empty = st_full + 2;      // [2] EPI_ROUTE: ... and read by the epilogue
+    float* ssbuf = reinterpret_cast<float*>(sI);   // EPI_ROUTE: [2][128] (the identity slot is unused)
+    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(st_empty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -170,13 +186,17 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], AMODE == A_GATHER ? 1 + 128 : 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], EPI == EPI_ROUTE ? 1 + 4 : 1);   // + the four statistics warps
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], 4);
         }
         mbar_init(drain, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&st_full[b], 4);
+            mbar_init(&st_empty[b], 4);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -358,12 +378,70 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
                 record_error(ERR_BOUNDS, 0x310);
                 valid = false;
             }
-            if (valid && EPI != EPI_RESID && EPI != EPI_COMBINE && EPI != EPI_SUM &&
+            if (valid && EPI != EPI_RESID && EPI != EPI_COMBINE && EPI != EPI_SUM && EPI != EPI_ROUTE &&
                 (size_t)(pos + 1) * p.out_ld > p.out_elems) {
                 record_error(ERR_BOUNDS, 0x312);
                 valid = false;
             }
-            if (EPI == EPI_SWIGLU) {
+            if (EPI == EPI_ROUTE) {
+                // row statistics of this tile from the statistics warps
+                if (!wait_or_abort(&st_full[buf], aph, abort_flag, 0x330)) break;
+                const float ssq = ssbuf[buf * 128 + r];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&st_empty[buf]);
+                const int E = p.E;
+                const float irs = 1.0f / sqrtf(ssq / (float)p.K + p.r_eps);
+                // the three parts of logit e sit in columns e, E + e and 2E + e: one load from each
+                // base (columns past the accumulator's 3E are read and ignored)
+                float vh[32], vm[32], vl[32];
+                tmem_ld32(taddr, vh);
+                tmem_ld32(taddr + E, vm);
+                tmem_ld32(taddr + 2 * E, vl);
+                // logit e = (hi + mid) + lo, scaled by 1/rms; softmax; top-k with ties to the lower index
+                float z[kRouteMaxE];
+                float zmax = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < kRouteMaxE; ++e) {
+                    z[e] = -INFINITY;
+                    if (e < E) {
+                        z[e] = ((vh[e] + vm[e]) + vl[e]) * irs;
+                        zmax = fmaxf(zmax, z[e]);
+                    }
+                }
+                float pe[kRouteMaxE];
+                float sum = 0.f;
+#pragma unroll
+                for (int e = 0; e < kRouteMaxE; ++e) {
+                    pe[e] = e < E ? expf(z[e] - zmax) : 0.f;
+                    sum += pe[e];
+                }
+                const size_t rowi = (size_t)b * p.banks + bank;
+                uint32_t chosen = 0;
+#pragma unroll 1
+                for (int j = 0; j < p.k; ++j) {
+                    int be = -1;
+                    float bz = -INFINITY;
+#pragma unroll
+                    for (int e = 0; e < kRouteMaxE; ++e)
+                        if (e < E && !((chosen >> e) & 1u) && (be < 0 || z[e] > bz)) { bz = z[e]; be = e; }
+                    chosen |= 1u << be;
+                    float pb = 0.f;
+#pragma unroll
+                    for (int e = 0; e < kRouteMaxE; ++e)
+                        if (e == be) pb = pe[e] / sum;
+                    if (valid) {
+                        p.r_idx[rowi * p.k + j] = be;
+                        p.r_gate[rowi * p.k + j] = p.r_alpha * pb;
+                    }
+                }
+                if (valid && p.r_inv_rms) p.r_inv_rms[rowi] = irs;
+                // per 128-row chunk: rows of this bank that chose expert e
+                for (int e = 0; e < E; ++e) {
+                    const unsigned bal = __ballot_sync(0xffffffffu, valid && ((chosen >> e) & 1u));
+                    if (lane == 0 && bal)
+                        atomicAdd(&p.r_counts[((size_t)bank * p.r_nchunks + ti.m) * E + e], __popc(bal));
+                }
+            } else if (EPI == EPI_SWIGLU) {
                 const float sc = valid ? __ldg(&p.inv_rms[(size_t)b * p.banks + bank]) : 0.f;
                 __nv_bfloat16* dst = p.out + (size_t)pos * p.out_ld + ti.n * (BN / 2);
 #pragma unroll 1
@@ -527,6 +605,43 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE>::NTHREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+    } else if (EPI == EPI_ROUTE) {
+        // ---------------------------------------------------------------- row statistics (warps 6-9)
+        // Each lane sums the squares of its row of every A stage (a second consumer of the stage:
+        // the empty barrier also waits for these four warps), then hands the tile's sums over.
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        int s = 0, lt = 0;
+        uint32_t ph = 0;
+        for (int t = blockIdx.x; t < ntile; t += gridDim.x, ++lt) {
+            const int buf = lt & 1;
+            float ss = 0.f;
+            bool ok = true;
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!wait_or_abort(&full[s], ph, abort_flag, 0x420)) { ok = false; break; }
+                const uint8_t* sa = smem + s * C::STAGE_BYTES;
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const uint4 w4 = AMODE == A_TMA_MIX
+                                         ? *reinterpret_cast<const uint4*>(sa + (v >> 1) * 4096 + r * 32 + ((v & 1) << 4))
+                                         : *reinterpret_cast<const uint4*>(sa + r * 128 + (((v ^ r) & 7) << 4));
+                    const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float a = bf16_lo(wv[e]), c = bf16_hi(wv[e]);
+                        ss = fmaf(a, a, fmaf(c, c, ss));
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                if (++s == STAGES) { s = 0; ph ^= 1; }
+            }
+            if (!ok) break;
+            if (!wait_or_abort(&st_empty[buf], ((lt >> 1) & 1) ^ 1, abort_flag, 0x421)) break;
+            ssbuf[buf * 128 + r] = ss;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&st_full[buf]);
         }
     } else if (AMODE == A_GATHER) {
         // ---------------------------------------------------------------- row gatherers (warps 6-9)

@@ -63,6 +63,9 @@ cudaError_t launch_offsets(const int32_t* counts_in, int32_t* chunk_prefix, int 
 cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, const int32_t* bucket_offsets, int B,
                            int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st,
                            int32_t* perm = nullptr);
+// tensor-core router weights: [banks][64][W] bf16, rows e / E+e / 2E+e = hi / mid / lo of w * gain
+cudaError_t launch_router_split(int dtype, const float* w_router, const void* gain, int banks, int E, int W,
+                                void* out, cudaStream_t st);
 // MoEPermute data copy: routed row positions receive their source rows (see gather_rows_kernel)
 cudaError_t launch_gather_rows(int dtype, const void* x, RowMap m, int B, int E, const int32_t* offsets, int groups,
                                const int32_t* bucket_rows, size_t routed, void* out, cudaStream_t st);

@@ -472,6 +472,32 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const T* __restrict__ 
     }
 }
 
+// Router weights for the tensor-core router: each fp32 weight (times the RMSNorm gain) split
+// exactly into three bf16 parts, hi = bf16(v), mid = bf16(v - hi), lo = bf16(v - hi - mid) (each
+// difference is exact in fp32; hi + mid + lo matches v to about 2^-24 relative), stored as rows
+// e, E + e, 2E + e of a [banks][64][W] bf16 matrix (rows 3E .. 63 zero).
+template <typename T>
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ w, const T* __restrict__ gain,
+                                                           int banks, int E, int W, __nv_bfloat16* __restrict__ out) {
+    const size_t n = (size_t)banks * 64 * W;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const int c = (int)(i % W);
+        const int row = (int)((i / W) % 64);
+        const int bank = (int)(i / ((size_t)64 * W));
+        __nv_bfloat16 o = __float2bfloat16_rn(0.f);
+        if (row < 3 * E) {
+            const int part = row / E, e = row - part * E;
+            const float v = w[((size_t)bank * E + e) * W + c] * (gain ? to_f(gain[c]) : 1.0f);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+            const float r1 = v - __bfloat162float(hi);
+            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+            const float r2 = r1 - __bfloat162float(mid);
+            o = part == 0 ? hi : (part == 1 ? mid : __float2bfloat16_rn(r2));
+        }
+        out[i] = o;
+    }
+}
+
 // ------------------------------------------------------------------ launchers
 static int grid_for(size_t n, int threads) {
     size_t g = (n + threads - 1) / threads;
@@ -537,6 +563,18 @@ cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, cons
     dim3 grid((B + kRouterChunk - 1) / kRouterChunk, banks);
     scatter_kernel<<<grid, kRouterChunk, 0, st>>>(idx, chunk_prefix, bucket_offsets, B, banks, E, k, bucket_rows,
                                                   slot_of, perm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_split(int dtype, const float* w_router, const void* gain, int banks, int E, int W,
+                                void* out, cudaStream_t st) {
+    ProfileScope ps_("router_split", st);
+    const int grid = grid_for((size_t)banks * 64 * W, 256);
+    if (dtype == 1)
+        router_split_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(w_router, (const __nv_bfloat16*)gain, banks, E, W,
+                                                                 (__nv_bfloat16*)out);
+    else
+        router_split_kernel<float><<<grid, 256, 0, st>>>(w_router, (const float*)gain, banks, E, W, (__nv_bfloat16*)out);
     return cudaGetLastError();
 }
 
