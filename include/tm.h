@@ -152,17 +152,17 @@ TM_API tm_status tm_route_topk(const void *x, tm_layout layout, const tm_shape *
                         void *workspace, size_t workspace_bytes, void *stream);
 
 /* Fixed size of the routing scratch array that tm_route_topk_noalloc keeps in the library. */
-#define TM_NOALLOC_SCRATCH_BYTES (1u << 20)
+#define TM_NOALLOC_SCRATCH_BYTES (8u << 20)
 
 /* tm_route_topk without a workspace argument, for callers that cannot allocate device memory
  * (a host framework that passes this library only its inputs and outputs and owns no allocator
  * it may call, or a serving loop that reserves all memory at start-up and allows no allocation
  * later).  The pages have no counterpart: this is a library convenience, not part of the method.
- * Same arguments, outputs and results as tm_route_topk.  Its scratch (per-chunk expert counts
- * and the tile prefix: banks * ceil(B/128) * E + banks * E + 1 int32, 256-byte aligned) is a
- * fixed TM_NOALLOC_SCRATCH_BYTES array inside the library's device image, held by every GPU that
- * loads the library until the process exits; problems that need more return TM_ERR_WORKSPACE
- * (message in tm_last_cuda_error) before any launch.  No device memory is allocated or freed.
+ * Same arguments, outputs and results as tm_route_topk: it calls tm_route_topk with a fixed
+ * TM_NOALLOC_SCRATCH_BYTES array inside the library's device image as the workspace, held by
+ * every GPU that loads the library until the process exits; problems whose
+ * tm_route_workspace_bytes exceeds it return TM_ERR_WORKSPACE (message in tm_last_cuda_error)
+ * before any launch.  No device memory is allocated or freed.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress), so
  * make that first call before any stream capture.  All calls on a device share the array and it
  * keeps the last call's contents (none of it needs to start at zero): calls that can overlap on

@@ -312,6 +312,66 @@ def test_block_forward_matches_stack_and_returns_revert():
     assert np.array_equal(to_np(api.stack_forward(Xd, blocks, 0, sh)), to_np(Y))
 
 
+BLOCK_FUSED = [
+    # 3 row tiles x 16 banks: all 96 tiles in one wave, reverting tiles wait on mixing tiles beside them
+    DENSE_SMALL[0],
+    # 9 row tiles x 16 banks = 144 mixing tiles on 148 SMs: the second item of CTA c is a reverting tile of
+    # the row block of its own first (mixing) tile, whose output and count go out before that A load waits
+    small("block_selfdep", 1100, 16, 256, 16, "bf16", FFNSpec("dense", hidden=256), FFNSpec("dense", hidden=384)),
+    # width 128 (T = H = 8, dh = 16): 20 row tiles x 8 banks = 160 + 160 tiles, waves straddle the sub-layers
+    small("block_w128", 2500, 8, 128, 8, "bf16", FFNSpec("dense", hidden=256), FFNSpec("dense", hidden=128)),
+]
+
+
+def _fused_launches(fn):
+    api.profile_start()
+    out = fn()
+    api.get_device_error()
+    return out, api.profile_stop().get("fused_swiglu", {}).get("launches", 0)
+
+
+@pytest.mark.parametrize("cfg", BLOCK_FUSED, ids=lambda c: c.name)
+@pytest.mark.parametrize("with_gain", [False, True], ids=["gain1", "gain"])
+def test_fused_block_one_launch(cfg, with_gain, monkeypatch):
+    """Both dense sub-layers of a block in one launch (mixing tiles, then reverting tiles that wait
+    for their row block): the same bits as one launch per sub-layer, since every tile does the same
+    arithmetic, X_revert included; within tolerance of the oracle."""
+    X, _ = inputs(cfg)
+    blk = api.Block(api.sublayer_from_synth(cfg, 0, 0, DEV, None, with_gain),
+                    api.sublayer_from_synth(cfg, 0, 1, DEV, None, with_gain))
+    sh = api.config_shape(cfg)
+    Xd = dev(X)
+
+    def run():
+        Xr = torch.empty_like(Xd)
+        return api.block_forward(Xd, blk, sh, X_revert=Xr), Xr
+    (Y1, Xr1), n1 = _fused_launches(run)
+    monkeypatch.setenv("TM_FUSED_BLOCK", "0")
+    (Y0, Xr0), n0 = _fused_launches(run)
+    monkeypatch.delenv("TM_FUSED_BLOCK")
+    assert (n1, n0) == (1, 2)
+    assert torch.equal(Y1.view(torch.int16), Y0.view(torch.int16))
+    assert torch.equal(Xr1.view(torch.int16), Xr0.view(torch.int16))
+    gains = tuple(S.to_f64(S.gain(cfg, 0, sub)) for sub in (0, 1)) if with_gain else (None, None)
+    b = O.block_forward(S.to_f64(X), cfg, 0, oracle.synth_banks(cfg), gains=gains, storage="bf16")
+    assert err_bf16(to_np(Y1), b["Y"]) <= BF16_TOL
+    assert err_bf16(to_np(Xr1), b["Xr"]) <= BF16_TOL
+
+
+def test_fused_block_stack_with_inter_residual(monkeypatch):
+    """A dense stack with the inter-residual (gap 2) through one launch per block: the same bits as
+    one launch per sub-layer, and the oracle's stack within tolerance."""
+    cfg = small("stack_blk", 700, 16, 256, 16, "bf16", FFNSpec("dense", hidden=256), FFNSpec("dense", hidden=512),
+                L=3, gap=2)
+    y1, n1 = _fused_launches(lambda: _stack_gpu(cfg))
+    monkeypatch.setenv("TM_FUSED_BLOCK", "0")
+    y0, n0 = _fused_launches(lambda: _stack_gpu(cfg))
+    monkeypatch.delenv("TM_FUSED_BLOCK")
+    assert (n1, n0) == (3, 6)
+    assert np.array_equal(y1, y0)       # float64 copies of the bf16 outputs
+    check_stack(cfg, y1)
+
+
 def test_deterministic_bits():
     cfg = MOE_SMALL[0].with_(L=2, gap=2)
     blocks = api.blocks_from_synth(cfg, DEV)

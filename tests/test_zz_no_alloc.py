@@ -48,8 +48,8 @@ def test_noalloc_routing_matches_workspace_routing_on_two_calls():
 
 def test_noalloc_routing_refuses_problems_beyond_its_scratch():
     # host-side check: refused before any launch, so this runs without a GPU too
-    # 48 banks x 16 experts x ceil(48000/128) chunks of int32 counts is 1.15 MB > 1 MiB
-    B, T, D, H, E = 48000, 48, 768, 48, 16
+    # 48 banks x 16 experts x ceil(400000/128) chunks of int32 counts is 9.6 MB > 8 MiB
+    B, T, D, H, E = 400000, 48, 768, 48, 16
     spec = FFNSpec("moe", E=E, k=4, hidden_e=64, hidden_s=64, alpha=4.0)
     cfg = S.Config("too_big", B=B, T=T, D=D, H=H, L=1, dtype="bf16", mix=spec, rev=spec)
     sh = api.config_shape(cfg)

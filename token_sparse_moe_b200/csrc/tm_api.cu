@@ -648,14 +648,123 @@ tm_status check_block(const tm_shape* s, const tm_block* b, Geo* gm, Geo* gr) {
     return TM_OK;
 }
 
+// ------------------------------------------------------------------ fused dense block
+// Both sub-layers of a block in one launch (launch_fused128_block): dense bf16 sub-layers of the
+// same row width 128 or 256 (T == H), head width a multiple of 16, hidden widths multiples of 128.
+// TM_FUSED_BLOCK=0 keeps one launch per sub-layer (for comparison), as do the opt-in variants of
+// the sub-layer kernel.
+bool env_is(const char* name, char v) {
+    const char* e = getenv(name);
+    return e && e[0] == v;
+}
+
+bool block_fusable(const tm_shape* s, const tm_block* b, const Geo& gm, const Geo& gr, const void* Y, const void* Xr) {
+    if (s->dtype != TM_BF16 || b->mix.is_moe || b->rev.is_moe) return false;
+    if (gm.W != gr.W || (gm.W != 128 && gm.W != 256) || gm.banks != gr.banks) return false;
+    if (gemm1_amode(gm) != A_TMA_MIX) return false;
+    if (b->mix.dense.hidden % 128 || b->rev.dense.hidden % 128) return false;
+    if ((uintptr_t)Y % 32 || (uintptr_t)Xr % 32) return false;
+    if (env_is("TM_FUSED_BLOCK", '0') || env_is("TM_FUSED_PAIRS", '1') || env_is("TM_FUSED64", '1') ||
+        env_is("TM_FUSED_SPLIT", '1'))
+        return false;
+    return true;
+}
+
+struct BlockWs {
+    unsigned* dep;
+    void *wg1, *wu1, *wg2, *wu2;
+};
+BlockWs carve_block(Carve& c, const Geo& gm, const Geo& gr, const tm_block* b) {
+    BlockWs w;
+    w.dep = c.take<unsigned>((size_t)(gm.B + 127) / 128);
+    const size_t n1 = (size_t)gm.banks * b->mix.dense.hidden * gm.W * gm.esz;
+    const size_t n2 = (size_t)gr.banks * b->rev.dense.hidden * gr.W * gr.esz;
+    w.wg1 = b->mix.norm_gain ? c.take<uint8_t>(n1) : nullptr;
+    w.wu1 = b->mix.norm_gain ? c.take<uint8_t>(n1) : nullptr;
+    w.wg2 = b->rev.norm_gain ? c.take<uint8_t>(n2) : nullptr;
+    w.wu2 = b->rev.norm_gain ? c.take<uint8_t>(n2) : nullptr;
+    return w;
+}
+
+size_t block_ws(const Geo& gm, const Geo& gr, const tm_block* b) {
+    if (b->mix.is_moe || b->rev.is_moe) return 0;
+    Carve c{nullptr};
+    carve_block(c, gm, gr, b);
+    return align256(c.off);
+}
+
+// The gate and up weights of a dense sub-layer with its norm gain folded in (into ws), or as given.
+tm_status dense_gate_up(const Geo& g, const tm_sublayer* sub, void* wg_ws, void* wu_ws, const void** wg, const void** wu,
+                        cudaStream_t st) {
+    *wg = sub->dense.w_gate;
+    *wu = sub->dense.w_up;
+    if (!sub->norm_gain) return TM_OK;
+    const size_t rows = (size_t)g.banks * sub->dense.hidden;
+    tm_status s;
+    if ((s = cuda_status(launch_fold_gain(g.dtype, *wg, sub->norm_gain, wg_ws, rows, g.W, st))) != TM_OK) return s;
+    if ((s = cuda_status(launch_fold_gain(g.dtype, *wu, sub->norm_gain, wu_ws, rows, g.W, st))) != TM_OK) return s;
+    *wg = wg_ws;
+    *wu = wu_ws;
+    return TM_OK;
+}
+
+tm_status fused_block(const tm_block* b, const Geo& gm, const Geo& gr, const void* X, const void* extra, void* Y,
+                      void* Xr, void* ws, size_t wsb, cudaStream_t st) {
+    Carve c{(uint8_t*)ws};
+    BlockWs w = carve_block(c, gm, gr, b);
+    if (!ws || wsb < c.off || !al16(ws)) return TM_ERR_WORKSPACE;
+    const int W = gm.W, F1 = b->mix.dense.hidden, F2 = b->rev.dense.hidden;
+    const void *wg1, *wu1, *wg2, *wu2;
+    tm_status s;
+    if ((s = dense_gate_up(gm, &b->mix, w.wg1, w.wu1, &wg1, &wu1, st)) != TM_OK) return s;
+    if ((s = dense_gate_up(gr, &b->rev, w.wg2, w.wu2, &wg2, &wu2, st)) != TM_OK) return s;
+    const int mt = (gm.B + 127) / 128;
+    if ((s = cuda_status(cudaMemsetAsync(w.dep, 0, (size_t)mt * sizeof(unsigned), st))) != TM_OK) return s;
+    FusedMaps mm, mr;
+    CUtensorMap mres, mext;
+    memset(&mext, 0, sizeof(mext));
+    // mixing: A through the Mix map over X, output through the Revert map into X_revert
+    if (!gemm1_amap(gm, X, A_TMA_MIX, &mm.a) || !gemm1_amap(gm, Xr, A_TMA_MIX, &mm.o, 32) ||
+        !map_2d(&mm.g, wg1, (uint64_t)gm.banks * F1, W, 128) || !map_2d(&mm.u, wu1, (uint64_t)gm.banks * F1, W, 128) ||
+        !map_2d(&mm.d, b->mix.dense.w_down, (uint64_t)gm.banks * W, F1, W))
+        return TM_ERR_CUDA;
+    // reverting: A = rows of X_revert, residual X (and the inter-residual) streamed, output Y
+    if (!gemm1_amap(gr, Xr, A_TMA_3D, &mr.a) || !gemm1_amap(gr, Y, A_TMA_3D, &mr.o, 32) ||
+        !map_2d(&mr.g, wg2, (uint64_t)gr.banks * F2, W, 128) || !map_2d(&mr.u, wu2, (uint64_t)gr.banks * F2, W, 128) ||
+        !map_2d(&mr.d, b->rev.dense.w_down, (uint64_t)gr.banks * W, F2, W) || !gemm1_amap(gr, X, A_TMA_3D, &mres) ||
+        (extra && !gemm1_amap(gr, extra, A_TMA_3D, &mext)))
+        return TM_ERR_CUDA;
+    FusedParams p;
+    memset(&p, 0, sizeof(p));
+    p.banks = gm.banks;
+    p.rows = gm.B;
+    p.F = F1;
+    p.F2 = F2;
+    p.amap = gm.map;
+    p.omap = gm.map;
+    p.eps = gm.eps;
+    p.out = (__nv_bfloat16*)Y;
+    p.out_elems = (size_t)gm.B * gm.banks * W;
+    p.res_mode = RES_FROM_A;
+    p.has_extra = 0;
+    p.res_mode2 = RES_STREAM;
+    p.has_extra2 = extra != nullptr;
+    p.dep = w.dep;
+    const long tiles = 2L * gm.banks * mt;
+    const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+    return cuda_status(launch_fused128_block(W, mm, mr, mres, mext, p, grid, st));
+}
+
 size_t stack_ws(const tm_shape* s, const tm_block* blocks, int L, int gap, bool* ok) {
     size_t sub = 0;
     for (int l = 0; l < L; ++l) {
         Geo gm, gr;
         if (check_block(s, &blocks[l], &gm, &gr) != TM_OK) { *ok = false; return 0; }
         const size_t a = sublayer_ws(gm, &blocks[l].mix), b = sublayer_ws(gr, &blocks[l].rev);
+        const size_t f = block_ws(gm, gr, &blocks[l]);
         sub = a > sub ? a : sub;
         sub = b > sub ? b : sub;
+        sub = f > sub ? f : sub;
     }
     *ok = true;
     const size_t tok = align256((size_t)s->B * s->T * s->D * (s->dtype == TM_BF16 ? 2 : 4));
@@ -668,6 +777,7 @@ tm_status run_block(const tm_shape* s, const tm_block* b, const void* X, const v
     Geo gm, gr;
     tm_status r = check_block(s, b, &gm, &gr);
     if (r != TM_OK) return r;
+    if (block_fusable(s, b, gm, gr, Y, Xr)) return fused_block(b, gm, gr, X, extra, Y, Xr, sub_ws, sub_wsb, st);
     // H_next = FFN_mix(Norm(Mix(X))) + Mix(X), written through Revert straight into X_rev
     if ((r = run_sublayer(gm, X, X, nullptr, &b->mix, Xr, sub_ws, sub_wsb, st)) != TM_OK) return r;
     // Y = FFN_rev(Norm(X_rev)) + X (+ inter-residual)

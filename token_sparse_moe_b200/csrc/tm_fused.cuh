@@ -33,6 +33,11 @@ struct FusedParams {
     int split_tiles;           // 128-wide-chunk kernel: split the last wave's tiles between CTA pairs
     float* part;               // split tiles: partial Y, [2][tiles of the last wave][128][W] fp32
     int* cnt;                  // split tiles: [tiles of the last wave][8] counters, zero at launch
+    // Whole dense block in one launch (128-wide-chunk kernel, block mode): the fields above describe
+    // the mixing sub-layer, these the reverting one (same banks and row width).
+    int F2;                    // reverting hidden width
+    int res_mode2, has_extra2; // reverting residual (streamed) and inter-residual
+    unsigned* dep;             // [row tiles] finished-mixing-tile counters, zero at launch
 };
 
 // Output epilogue of a fused tile for one thread: row b of bank g, columns [c_begin, c_begin + W/2).

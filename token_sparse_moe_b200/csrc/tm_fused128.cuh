@@ -26,12 +26,25 @@
 // Warp roles: warp 0 TMA producer (and builds the identity tile), warp 1 MMA issuer and TMEM
 // owner, warps 2-9 epilogue (TMEM lane quarter = warp % 4; warps 2-5 / 6-9 take the two column
 // halves).
+//
+// Block mode (AMODE = A_BLOCK, when both sub-layers of a block are dense with the same row width,
+// i.e. T == H): one launch runs the whole block.  The tiles of the mixing sub-layer (A through the
+// Mix map, residual = A, output stored through the Revert map into X_revert) come first, then
+// those of the reverting sub-layer (A = rows of X_revert, residual X streamed), both ordered by
+// 128-sample row block.  A reverting tile of row block m reads X_revert rows that every mixing
+// tile of block m writes, so its A load waits for a per-block counter: each epilogue warp of a
+// mixing tile adds one with release semantics once its bulk stores are complete in global
+// memory.  No SM idles between the two sub-layers: the partial last wave of the mixing tiles is
+// filled with reverting tiles whose row blocks finished long before.  The launch is cooperative
+// (all CTAs resident), and a mixing tile's count never waits on a reverting tile (see the
+// epilogue), so every wait ends.
 #pragma once
 #include "tm_fused.cuh"
 
 namespace tml {
 
 enum FusedResid : int { RES_NONE = 0, RES_FROM_A = 1, RES_STREAM = 2 };
+constexpr int A_BLOCK = 4;   // fused128 kernel: a whole dense block (mixing tiles, then reverting tiles)
 
 template <int W, int AMODE>
 struct Fused128Cfg {
@@ -70,20 +83,34 @@ __device__ __forceinline__ void ld_global_cg_v8(const void* p, uint32_t (&w)[8])
                  : "memory");
 }
 
+// One work item of a CTA: tile t (bank g, row tile m), hidden chunks [c0, c1), split half sp
+// (-1: whole tile); sec: a tile of the second (reverting) sub-layer in block mode; mx: A, the
+// residual stream and the output use the Mix geometry.
+struct F128Item {
+    int t, g, m, c0, c1, sp;
+    bool sec, mx;
+};
+
 template <int W, int AMODE>
 __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
     fused128_swiglu_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
                            const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmD,
                            const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmE,
-                           const __grid_constant__ CUtensorMap tmO, const FusedParams p) {
+                           const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmA2,
+                           const __grid_constant__ CUtensorMap tmG2, const __grid_constant__ CUtensorMap tmU2,
+                           const __grid_constant__ CUtensorMap tmD2, const __grid_constant__ CUtensorMap tmO2,
+                           const FusedParams p) {
+    // Maps: A, G, U, D, O of the (first) sub-layer; R / E the streamed residual and inter-residual
+    // (in block mode those of the reverting sub-layer); A2, G2, U2, D2, O2 the reverting
+    // sub-layer's in block mode (unused otherwise).
     using C = Fused128Cfg<W, AMODE>;
+    constexpr bool BLK = AMODE == A_BLOCK;
     constexpr int STAGES = C::STAGES;
     const int mt = (p.rows + 127) / 128;
-    const int ntile = p.banks * mt;
+    const int ntile1 = p.banks * mt;                 // tiles of one sub-layer
+    const int ntile = BLK ? 2 * ntile1 : ntile1;
     if ((int)blockIdx.x >= ntile) return;
     const int NC = p.F / 128;
-    const int res_stages = p.res_mode == RES_STREAM ? C::R_STAGES : 0;
-    const int ext_stages = p.has_extra ? C::R_STAGES : 0;
     // GEMM2(c) is issued in step c + LAG, after GEMM1(c + LAG).  LAG = 1: the SwiGLU of chunk c
     // overlaps GEMM1(c+1) and its hidden write waits only for GEMM2(c-1).  (A lag of 2 measured
     // 16% slower on the dense block workload: each hidden write then waits behind a whole GEMM1.)
@@ -91,28 +118,51 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
     // Work items of this CTA: tile t = blockIdx.x + k * gridDim.x for the full waves.  With
     // p.split_tiles the tiles of the last, partial wave are each split between two CTAs by hidden
     // chunks (half 0: [0, NC/2), half 1: [NC/2, NC)), so every CTA ends within half a tile of the
-    // others; the halves meet through p.part (see the split output below).
+    // others; the halves meet through p.part (see the split output below).  Block mode: tiles
+    // [0, ntile1) mixing, [ntile1, 2 ntile1) reverting, each numbered m * banks + g; no splits.
     const int full_waves = ntile / (int)gridDim.x;
     const int n_rem = ntile - full_waves * (int)gridDim.x;
-    auto item = [&](int k, int& t, int& c0, int& c1, int& sp) -> bool {
+    auto item = [&](int k, F128Item& it) -> bool {
         const int b = blockIdx.x;
-        sp = -1;
-        c0 = 0;
-        c1 = NC;
-        if (k < full_waves) { t = b + k * (int)gridDim.x; return true; }
-        if (k > full_waves) return false;
-        if (p.split_tiles) {
-            if (b >= 2 * n_rem) return false;
-            t = full_waves * (int)gridDim.x + (b >> 1);
-            sp = b & 1;
-            c0 = sp ? NC / 2 : 0;
-            c1 = sp ? NC : NC / 2;
+        it.sp = -1;
+        it.c0 = 0;
+        if (BLK) {
+            it.t = b + k * (int)gridDim.x;
+            if (it.t >= ntile) return false;
+            it.sec = it.t >= ntile1;
+            it.mx = !it.sec;
+            const int tt = it.sec ? it.t - ntile1 : it.t;
+            it.m = tt / p.banks;
+            it.g = tt - it.m * p.banks;
+            it.c1 = (it.sec ? p.F2 : p.F) / 128;
             return true;
         }
-        if (b >= n_rem) return false;
-        t = full_waves * (int)gridDim.x + b;
+        it.sec = false;
+        it.mx = AMODE == A_TMA_MIX;
+        it.c1 = NC;
+        if (k < full_waves) {
+            it.t = b + k * (int)gridDim.x;
+        } else if (k > full_waves) {
+            return false;
+        } else if (p.split_tiles) {
+            if (b >= 2 * n_rem) return false;
+            it.t = full_waves * (int)gridDim.x + (b >> 1);
+            it.sp = b & 1;
+            it.c0 = it.sp ? NC / 2 : 0;
+            it.c1 = it.sp ? NC : NC / 2;
+        } else {
+            if (b >= n_rem) return false;
+            it.t = full_waves * (int)gridDim.x + b;
+        }
+        it.g = it.t / mt;
+        it.m = it.t - it.g * mt;
         return true;
     };
+    // per-item choices (compile-time constants outside block mode)
+    auto amix = [&](const F128Item& it) { return BLK ? it.mx : AMODE == A_TMA_MIX; };
+    auto rmode = [&](const F128Item& it) { return BLK && it.sec ? p.res_mode2 : p.res_mode; };
+    auto n_res = [&](const F128Item& it) { return rmode(it) == RES_STREAM ? C::R_STAGES : 0; };
+    auto n_ext = [&](const F128Item& it) { return (BLK && it.sec ? p.has_extra2 : p.has_extra) ? C::R_STAGES : 0; };
     // per item with nc chunks: steps 0 .. nc + LAG - 1; the residual / inter-residual identity pass
     // (only in the item that starts at chunk 0) runs in step s_r, after GEMM2(min(1, nc-1)): Y is
     // initialised by the item's first GEMM2, and the streamed tiles come through the ring like
@@ -190,13 +240,20 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             tma_prefetch_desc(&tmG);
             tma_prefetch_desc(&tmU);
             tma_prefetch_desc(&tmD);
+            if (BLK) {
+                tma_prefetch_desc(&tmA2);
+                tma_prefetch_desc(&tmG2);
+                tma_prefetch_desc(&tmU2);
+                tma_prefetch_desc(&tmD2);
+            }
             int s = 0;
             uint32_t ph = 0;
             int lt = 0;
             bool ok = true;
             // 128 rows x (16 * n16) columns from column 16 * col16 of a row tensor, in the A geometry
-            auto load_rows = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* b, int g, int m0, int col16, int n16) {
-                if (AMODE == A_TMA_MIX) {
+            auto load_rows = [&](const CUtensorMap* map, bool mx, uint8_t* dst, uint64_t* b, int g, int m0, int col16,
+                                 int n16) {
+                if (mx) {
                     const int per = p.amap.dh >> 4;
 #pragma unroll 1
                     for (int i = 0; i < n16; ++i) {
@@ -208,16 +265,44 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                     for (int i = 0; i < n16 / 4; ++i) tma_load_3d(dst + i * 16384, map, b, col16 * 16 + i * 64, g, m0);
                 }
             };
-            int t, c0, c1, sp;
-            for (; ok && item(lt, t, c0, c1, sp); ++lt) {
-                const int g = t / mt, m = t - g * mt;
-                const int nc = c1 - c0, n_steps = nc + LAG, s_r = c0 == 0 ? id_step(nc) : -1;
+            // block mode: every mixing tile of row block m has stored its X_revert rows (8 epilogue
+            // warps per tile count once each)
+            auto wait_block = [&](int m) -> bool {
+                const unsigned* ctr = p.dep + m;
+                const unsigned target = 8u * (unsigned)p.banks;
+                if (ld_acquire(ctr) < target) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire(ctr) < target) {
+                        if (*abort_flag) return false;
+                        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                            record_error(ERR_TIMEOUT, 0x3108);
+                            *abort_flag = 1;
+                            return false;
+                        }
+                        __nanosleep(64);
+                    }
+                }
+                fence_proxy_async_global();   // the bulk tensor loads below come after the acquire
+                return true;
+            };
+            F128Item it;
+            for (; ok && item(lt, it); ++lt) {
+                const int g = it.g, m = it.m, c0 = it.c0;
+                const int nc = it.c1 - it.c0, n_steps = nc + LAG, s_r = c0 == 0 ? id_step(nc) : -1;
+                const bool mx = amix(it);
+                const int F = BLK && it.sec ? p.F2 : p.F;
+                const int res_stages = n_res(it), ext_stages = n_ext(it);
+                const CUtensorMap* mA = BLK && it.sec ? &tmA2 : &tmA;
+                const CUtensorMap* mG = BLK && it.sec ? &tmG2 : &tmG;
+                const CUtensorMap* mU = BLK && it.sec ? &tmU2 : &tmU;
+                const CUtensorMap* mD = BLK && it.sec ? &tmD2 : &tmD;
+                if (BLK && it.sec && !wait_block(m)) break;
                 // A slab by slab, each as soon as the previous tile has released it
 #pragma unroll 1
                 for (int qa = 0; qa < C::G1_STAGES && ok; ++qa) {
                     if (!wait_or_abort(&a_empty[qa], (lt & 1) ^ 1, abort_flag, 0x3100)) { ok = false; break; }
                     if (qa == 0) mbar_arrive_expect_tx(a_full, C::A_BYTES);
-                    load_rows(&tmA, sA + qa * 16384, a_full, g, m * 128, qa * 4, 4);
+                    load_rows(mA, mx, sA + qa * 16384, a_full, g, m * 128, qa * 4, 4);
                 }
                 if (!ok) break;
                 // ring order per step: G1(step) (step < NC), G2(step - LAG) (step >= LAG), and at step
@@ -231,8 +316,8 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x3101)) { ok = false; break; }
                             uint8_t* st = sR + s * C::SB;
                             mbar_arrive_expect_tx(&full[s], C::SB);
-                            tma_load_2d(st, &tmG, &full[s], q * 64, g * p.F + c * 128);
-                            tma_load_2d(st + 16384, &tmU, &full[s], q * 64, g * p.F + c * 128);
+                            tma_load_2d(st, mG, &full[s], q * 64, g * F + c * 128);
+                            tma_load_2d(st + 16384, mU, &full[s], q * 64, g * F + c * 128);
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                     }
@@ -244,10 +329,10 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             uint8_t* st = sR + s * C::SB;
                             mbar_arrive_expect_tx(&full[s], C::SB);
                             if (W == 256) {
-                                tma_load_2d(st, &tmD, &full[s], c * 128 + q * 64, g * W);          // 256 rows x 64 K
+                                tma_load_2d(st, mD, &full[s], c * 128 + q * 64, g * W);          // 256 rows x 64 K
                             } else {
-                                tma_load_2d(st, &tmD, &full[s], c * 128, g * W);                   // 128 rows x 64 K
-                                tma_load_2d(st + 16384, &tmD, &full[s], c * 128 + 64, g * W);      // next 64 K
+                                tma_load_2d(st, mD, &full[s], c * 128, g * W);                   // 128 rows x 64 K
+                                tma_load_2d(st + 16384, mD, &full[s], c * 128 + 64, g * W);      // next 64 K
                             }
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
@@ -259,7 +344,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             uint8_t* st = sR + s * C::SB;
                             mbar_arrive_expect_tx(&full[s], C::SB);
                             const int q = i < res_stages ? i : i - res_stages;
-                            load_rows(i < res_stages ? &tmR : &tmE, st, &full[s], g, m * 128, q * 8, 8);
+                            load_rows(i < res_stages ? &tmR : &tmE, mx, st, &full[s], g, m * 128, q * 8, 8);
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                     }
@@ -278,10 +363,13 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             constexpr uint32_t idescI = umma_idesc_bf16(128, 16);
             const uint32_t aS = smem_u32(sA), hS = smem_u32(sH), rS = smem_u32(sR);
             uint64_t adesc[W / 16];
+            auto set_adesc = [&](bool mx) {
 #pragma unroll
-            for (int k16 = 0; k16 < W / 16; ++k16)
-                adesc[k16] = AMODE == A_TMA_MIX ? umma_sdesc_sw32(aS + k16 * 4096)
-                                                : umma_sdesc_sw128(aS + (k16 >> 2) * 16384) + 2 * (k16 & 3);
+                for (int k16 = 0; k16 < W / 16; ++k16)
+                    adesc[k16] = mx ? umma_sdesc_sw32(aS + k16 * 4096)
+                                    : umma_sdesc_sw128(aS + (k16 >> 2) * 16384) + 2 * (k16 & 3);
+            };
+            set_adesc(AMODE == A_TMA_MIX);
             const uint64_t hdesc0 = umma_sdesc_sw128(hS), hdesc1 = umma_sdesc_sw128(hS + 16384);
             const uint64_t rdesc0 = umma_sdesc_sw128(rS);
             const uint64_t rdesc32 = umma_sdesc_sw32(rS);
@@ -292,12 +380,15 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             uint32_t ph = 0;
             int lt = 0;
             bool ok = true;
-            int t, c0, c1, sp;
-            for (; ok && item(lt, t, c0, c1, sp); ++lt) {
-                const int nc = c1 - c0, n_steps = nc + LAG, s_r = c0 == 0 ? id_step(nc) : -1;
+            F128Item it;
+            for (; ok && item(lt, it); ++lt) {
+                const int nc = it.c1 - it.c0, n_steps = nc + LAG, s_r = it.c0 == 0 ? id_step(nc) : -1;
+                const bool mx = amix(it);
+                const int rm = rmode(it), res_stages = n_res(it), ext_stages = n_ext(it);
+                if (BLK) set_adesc(mx);
                 // A is released slab by slab after the item's last GEMM1, or after the identity pass
                 // when that reads A and comes later
-                const bool a_after_id = p.res_mode == RES_FROM_A && s_r >= nc - 1;
+                const bool a_after_id = rm == RES_FROM_A && s_r >= nc - 1;
                 if (!wait_or_abort(a_full, lt & 1, abort_flag, 0x3200)) break;
                 tc_fence_after();
 #pragma unroll 1
@@ -376,7 +467,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                         umma_commit(hid_empty);
                     }
                     if (step == s_r) {                                 // ---- Y += residual (+ inter-residual)
-                        if (p.res_mode == RES_FROM_A) {
+                        if (rm == RES_FROM_A) {
 #pragma unroll
                             for (int k16 = 0; k16 < W / 16; ++k16) umma_bf16(tmem + 16 * k16, adesc[k16], idB, idescI, 1);
                             if (a_after_id) {
@@ -392,7 +483,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             const uint32_t st = rS + s * C::SB;
 #pragma unroll
                             for (int k16 = 0; k16 < 8; ++k16) {
-                                const uint64_t rd = AMODE == A_TMA_MIX
+                                const uint64_t rd = mx
                                                         ? rdesc32 + (uint64_t)s * kStageDesc + k16 * (4096 >> 4)
                                                         : umma_sdesc_sw128(st + (k16 >> 2) * 16384) + 2 * (k16 & 3);
                                 umma_bf16(tmem + 16 * (q * 8 + k16), rd, idB, idescI, 1);
@@ -418,12 +509,28 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);      // [half][row] partial sums of squares
         uint8_t* stg = sH + half * 16384 + q * 4096;                  // this warp's 32 rows of the hidden buffer
         int n_stats = 0;
+        // Block mode: the row block of the last mixing tile whose bulk stores this warp issued and has
+        // not counted yet (-1: none).  Its count is added at this warp's next output, by which time
+        // the stores are long complete, or at once when the next item is a reverting tile or there
+        // is none (so a mixing tile's count never waits on a reverting tile).
+        int pend_m = -1;
+        auto flush_block = [&]() {
+            if (BLK && pend_m >= 0) {
+                if (lane == 0) {
+                    bulk_wait_all();                                   // this warp's stores are in global memory
+                    fence_proxy_async_global();
+                    red_release_add(p.dep + pend_m, 1u);
+                }
+                __syncwarp();
+                pend_m = -1;
+            }
+        };
         // 1/rms of this thread's row of the tile in the A buffer (0 for rows past the end).  Each half
         // sums the squares of its half of the row; the two partials meet in shared memory and are
         // added in the same order by both threads of the row.
-        auto row_scale = [&](int m_tile, float& out) -> bool {
+        auto row_scale = [&](int m_tile, bool mx, float& out) -> bool {
             float ss = 0.f;
-            if (AMODE == A_TMA_MIX) {
+            if (mx) {
 #pragma unroll 4
                 for (int i = 0; i < W / 32; ++i) {
                     const uint4* rp = reinterpret_cast<const uint4*>(sA + (half * (W / 32) + i) * 4096 + r * 32);
@@ -469,9 +576,11 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         };
         // Y of tile (g, m) (residual already accumulated) -> bf16 -> this warp's rows of the idle hidden
         // buffer in the output box layout -> bulk tensor store, 64 columns per round; releases Y
-        auto output_tile = [&](int g, int m, int ylt) -> bool {
+        auto output_tile = [&](int g, int m, int ylt, bool mx, bool sec) -> bool {
             if (!wait_or_abort(y_full, ylt & 1, abort_flag, 0x3303)) return false;
             tc_fence_after();
+            flush_block();                                            // the previous mixing tile's stores are done
+            const CUtensorMap* mo = BLK && sec ? &tmO2 : &tmO;
             const int b0 = m * 128 + q * 32;                          // first row of this warp's box
 #pragma unroll
             for (int j = 0; j < W / 128; ++j) {
@@ -498,28 +607,28 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                                                 pack_bf16x2(__uint_as_float(vv[o + 2]), __uint_as_float(vv[o + 3])),
                                                 pack_bf16x2(__uint_as_float(vv[o + 4]), __uint_as_float(vv[o + 5])),
                                                 pack_bf16x2(__uint_as_float(vv[o + 6]), __uint_as_float(vv[o + 7])));
-                    uint8_t* dst = AMODE == A_TMA_MIX
-                                       ? stg + (c8 >> 1) * 1024 + lane * 32 + (((c8 & 1) ^ ((lane >> 2) & 1)) << 4)
-                                       : stg + lane * 128 + ((c8 ^ (lane & 7)) << 4);
+                    uint8_t* dst = mx ? stg + (c8 >> 1) * 1024 + lane * 32 + (((c8 & 1) ^ ((lane >> 2) & 1)) << 4)
+                                      : stg + lane * 128 + ((c8 ^ (lane & 7)) << 4);
                     *reinterpret_cast<uint4*>(dst) = w4;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0 && b0 < p.rows) {
-                    if (AMODE == A_TMA_MIX) {
+                    if (mx) {
                         const int per = p.omap.dh >> 4;
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const int ci = (col0 >> 4) + k, tok = ci / per, jj = ci - tok * per;
-                            tma_store_4d(&tmO, stg + k * 1024, 0, g * per + jj, tok, b0);
+                            tma_store_4d(mo, stg + k * 1024, 0, g * per + jj, tok, b0);
                         }
                     } else {
-                        tma_store_3d(&tmO, stg, col0, g, b0);
+                        tma_store_3d(mo, stg, col0, g, b0);
                     }
                     bulk_commit_group();
                 }
                 __syncwarp();
             }
+            if (BLK && !sec) pend_m = m;                              // counted once the stores complete
             return true;
         };
         // One half of a split tile: this half's partial Y (fp32, rows of W) goes to p.part; for each
@@ -619,17 +728,19 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                 for (int qa = 0; qa < C::G1_STAGES / 2; ++qa) mbar_arrive(&a_empty[half * (C::G1_STAGES / 2) + qa]);
             }
         };
-        int t, c0, c1, sp;
-        bool have = item(0, t, c0, c1, sp);
-        bool ok = have && wait_or_abort(a_full, 0, abort_flag, 0x3300) && row_scale(t % mt, sc);
+        F128Item it;
+        bool have = item(0, it);
+        bool ok = have && wait_or_abort(a_full, 0, abort_flag, 0x3300) && row_scale(it.m, amix(it), sc);
         if (ok) release_a();
-        int prev_g = 0, prev_m = 0, prev_sp = -1, prev_st = 0;
+        F128Item prev = it;
+        bool prev_pending = false;                                     // prev's output is still to be written
         auto output_prev = [&](int ylt) -> bool {
-            return prev_sp < 0 ? output_tile(prev_g, prev_m, ylt) : output_split(prev_g, prev_m, ylt, prev_sp, prev_st);
+            return prev.sp < 0 ? output_tile(prev.g, prev.m, ylt, amix(prev), prev.sec)
+                               : output_split(prev.g, prev.m, ylt, prev.sp, prev.t - full_waves * (int)gridDim.x);
         };
         uint32_t ubase = 0;                                            // chunks of the items before this one
         for (; ok && have; ++lt) {
-            const int g = t / mt, m = t - g * mt;
+            const int c0 = it.c0, c1 = it.c1;
             // ---- SwiGLU chunks: this thread owns hidden columns [half*64, half*64 + 64) of its row
 #pragma unroll 1
             for (int c = c0; c < c1; ++c) {
@@ -661,11 +772,12 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                     pk[i] = pack_bf16x2(h0.x, h0.y);
                     pk[16 + i] = pack_bf16x2(h1.x, h1.y);
                 }
-                if (c == c0 && lt > 0) {
+                if (c == c0 && prev_pending) {
                     // the previous item's output, now that this item's second GEMM1 can run (the
                     // buffer is released above); the hidden rows are its staging, so this chunk's
                     // hidden write waits until the bulk stores have read them
                     if (!output_prev(lt - 1)) { ok = false; break; }
+                    prev_pending = false;
                     if (lane == 0) bulk_wait_read_all();
                     __syncwarp();
                 }
@@ -682,21 +794,27 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             }
             if (!ok) break;
             ubase += c1 - c0;
-            prev_g = g;
-            prev_m = m;
-            prev_sp = sp;
-            prev_st = t - full_waves * (int)gridDim.x;
+            prev = it;
+            prev_pending = true;
+            have = item(lt + 1, it);
+            // Block mode, last mixing tile of this CTA: its output and count go out now, before this
+            // warp waits for anything of the next item (a reverting tile's A load may wait for it).
+            if (BLK && !prev.sec && (!have || it.sec)) {
+                if (!output_prev(lt)) { ok = false; break; }
+                prev_pending = false;
+                flush_block();
+            }
             // ---- statistics of the next item (its A tile is loaded once this item's last read of A is issued)
-            have = item(lt + 1, t, c0, c1, sp);
             if (have) {
-                if (!wait_or_abort(a_full, (lt + 1) & 1, abort_flag, 0x3304) || !row_scale(t % mt, sc)) {
+                if (!wait_or_abort(a_full, (lt + 1) & 1, abort_flag, 0x3304) || !row_scale(it.m, amix(it), sc)) {
                     ok = false;
                     break;
                 }
                 release_a();
             }
         }
-        if (ok && lt > 0) ok = output_prev(lt - 1);
+        if (ok && prev_pending) ok = output_prev(lt - 1);
+        flush_block();
         if (lane == 0) bulk_wait_all();                                // stores complete before exit
         __syncwarp();
     }

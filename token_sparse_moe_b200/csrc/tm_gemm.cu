@@ -35,8 +35,43 @@ static cudaError_t launch_fused128_one(const CUtensorMap& a, const CUtensorMap& 
         configured = true;
     }
     ProfileScope ps_("fused_swiglu", st);
-    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, g, u, d, r, e, o, p);
+    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, g, u, d, r, e, o, a, g, u, d, o, p);
     return cudaGetLastError();
+}
+
+// A whole dense block in one launch.  Cooperative, so that all CTAs are resident together: a
+// reverting tile waits for mixing tiles that other CTAs run.
+template <int W>
+static cudaError_t launch_fused128_block_one(const FusedMaps& mix, const FusedMaps& rev, const CUtensorMap& r,
+                                             const CUtensorMap& e, const FusedParams& p, int grid, cudaStream_t st) {
+    using C = Fused128Cfg<W, A_BLOCK>;
+    auto kern = fused128_swiglu_kernel<W, A_BLOCK>;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (err != cudaSuccess) return err;
+        configured = true;
+    }
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(C::NTHREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    ProfileScope ps_("fused_swiglu", st);
+    return cudaLaunchKernelEx(&cfg, kern, mix.a, mix.g, mix.u, mix.d, r, e, mix.o, rev.a, rev.g, rev.u, rev.d, rev.o, p);
+}
+
+cudaError_t launch_fused128_block(int W, const FusedMaps& mix, const FusedMaps& rev, const CUtensorMap& r,
+                                  const CUtensorMap& e, const FusedParams& p, int grid, cudaStream_t st) {
+    if (W == 256) return launch_fused128_block_one<256>(mix, rev, r, e, p, grid, st);
+    if (W == 128) return launch_fused128_block_one<128>(mix, rev, r, e, p, grid, st);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_fused128(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,

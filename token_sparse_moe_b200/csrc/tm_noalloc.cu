@@ -6,7 +6,8 @@
 // allows no allocation afterwards.  For them, the routing scratch (per-chunk expert counts
 // and the 128-row tile prefix) lives in a fixed array inside the library's device image.
 // Every GPU that loads the library holds that array until the process exits; nothing here
-// calls cudaMalloc, cudaFree or any allocating routine.
+// calls cudaMalloc, cudaFree or any allocating routine.  The array serves as the workspace of
+// tm_route_topk, so the two entry points run the same kernels.
 #include <stdio.h>
 
 #include <mutex>
@@ -17,7 +18,8 @@
 namespace tml {
 namespace {
 
-// The routing scratch shared by every call of tm_route_topk_noalloc on a device.
+// The routing scratch shared by every call of tm_route_topk_noalloc on a device (per-chunk expert
+// counts, tile prefix and, for the tensor-core router, the split router weights).
 static __device__ __align__(256) unsigned char g_route_scratch[TM_NOALLOC_SCRATCH_BYTES];
 
 std::mutex g_setup_mu;
@@ -44,8 +46,6 @@ tm_status scratch_address(void** out) {
     return TM_OK;
 }
 
-size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
-
 }  // namespace
 }  // namespace tml
 
@@ -63,36 +63,18 @@ extern "C" tm_status tm_route_topk_noalloc(const void* x, tm_layout layout, cons
         return TM_ERR_INVALID_ARG;
     if (norm_gain && !al16(norm_gain)) return TM_ERR_INVALID_ARG;
 
-    const int B = shape->B, banks = w->banks, E = w->E;
-    const int nchunks = (B + kRouterChunk - 1) / kRouterChunk;
-    const size_t counts_bytes = (size_t)banks * nchunks * E * sizeof(int32_t);
-    const size_t tiles_bytes = ((size_t)banks * E + 1) * sizeof(int32_t);
-    if (up256(counts_bytes) + tiles_bytes > TM_NOALLOC_SCRATCH_BYTES) {
+    if (need > TM_NOALLOC_SCRATCH_BYTES) {
         char msg[160];
-        snprintf(msg, sizeof(msg), "tm_route_topk_noalloc: needs %zu bytes of scratch, the fixed limit is %u",
-                 up256(counts_bytes) + tiles_bytes, (unsigned)TM_NOALLOC_SCRATCH_BYTES);
+        snprintf(msg, sizeof(msg), "tm_route_topk_noalloc: needs %zu bytes of scratch, the fixed limit is %u", need,
+                 (unsigned)TM_NOALLOC_SCRATCH_BYTES);
         note_cuda_error(msg, cudaErrorInvalidValue);
         return TM_ERR_WORKSPACE;
     }
     void* base = nullptr;
     tm_status s = scratch_address(&base);
     if (s != TM_OK) return s;
-    int32_t* counts = reinterpret_cast<int32_t*>(base);
-    int32_t* tiles = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(base) + up256(counts_bytes));
-
-    // Nothing in the scratch has to start at zero: the router writes every chunk count and the
-    // offsets kernel writes every tile-prefix entry before anything reads them.
-    const int dh = shape->D / shape->H;
-    const RowMap m{layout == TM_LAYOUT_MIXED ? 1 : 0, banks, w->width, shape->T, shape->D, dh};
-    cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = launch_router(shape->dtype == TM_BF16 ? 1 : 0, x, m, B, shape->eps, norm_gain, w->w_router, E,
-                                  w->k, w->alpha, topk_idx, topk_gate, inv_rms, counts, st);
-    if (e == cudaSuccess) e = launch_offsets(counts, counts, banks, nchunks, E, bucket_offsets, tiles, st);
-    if (e == cudaSuccess)
-        e = launch_scatter(topk_idx, counts, bucket_offsets, B, banks, E, w->k, bucket_rows, slot_of, st);
-    if (e != cudaSuccess) {
-        note_cuda_error("tm_route_topk_noalloc: launch", e);
-        return TM_ERR_CUDA;
-    }
-    return TM_OK;
+    // The fixed array is the workspace of the ordinary entry point, so both take the same kernels
+    // in the same order and give the same bits.  Nothing in it has to start at zero.
+    return tm_route_topk(x, layout, shape, norm_gain, w, topk_idx, topk_gate, inv_rms, bucket_offsets, bucket_rows,
+                         slot_of, base, TM_NOALLOC_SCRATCH_BYTES, stream);
 }
