@@ -94,9 +94,16 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_hash() -> str:
+# The sources each profiled kernel family is compiled from (its own code and the device helpers it
+# uses); a DRAM figure in profiles/traffic.json counts only while these are unchanged.
+KERNEL_SOURCES_OF = {
+    "fused_swiglu": ["tm_fused128.cuh", "tm_fused.cuh", "tm_device.cuh"],
+}
+
+
+def kernel_hash(kernel: str = None) -> str:
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_SOURCES_OF.get(kernel, KERNEL_SOURCES):
         with open(os.path.join(ROOT, "token_sparse_moe_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -110,7 +117,7 @@ def traffic_for(kernel: str, workload: str):
     with open(path) as f:
         d = json.load(f)
     e = d.get(workload, {}).get(kernel)
-    if not e or e.get("kernel_hash") != kernel_hash():
+    if not e or e.get("kernel_hash") != kernel_hash(kernel):
         return None
     return float(e["dram_bytes_per_launch"])
 

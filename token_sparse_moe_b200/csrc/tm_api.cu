@@ -233,11 +233,12 @@ tm_status gemm1_dense(const Geo& g, const void* x, const void* wg, const void* w
     const int bn = pick_bn_swiglu(F);
     p.n_tiles = p.N / bn;
     const int am = gemm1_amode(g);
-    CUtensorMap ma, mg, mu;
+    CUtensorMap ma, mg, mu, mo;
     if (!gemm1_amap(g, x, am, &ma)) return TM_ERR_CUDA;
-    if (!map_2d(&mg, wg, (uint64_t)g.banks * F, g.W, bn / 2) || !map_2d(&mu, wu, (uint64_t)g.banks * F, g.W, bn / 2))
+    if (!map_2d(&mg, wg, (uint64_t)g.banks * F, g.W, bn / 2) || !map_2d(&mu, wu, (uint64_t)g.banks * F, g.W, bn / 2) ||
+        !map_2d(&mo, hidden, (uint64_t)g.banks * g.B, F, 32))
         return TM_ERR_CUDA;
-    return cuda_status(launch_grouped_gemm(bn, am, EPI_SWIGLU, ma, mg, mu, p, dense_grid(p), st));
+    return cuda_status(launch_grouped_gemm(bn, am, EPI_SWIGLU, ma, mg, mu, p, dense_grid(p), st, &mo));
 }
 
 // GEMM2 over dense hidden rows [banks*B, F] with the residual / combine epilogue into y (omap).
@@ -491,10 +492,11 @@ tm_status combine_sum(const Geo& g, const void* hidden_s, const void* wd, int Fs
     if (am != A_TMA_MIX && am != A_TMA_3D) return TM_ERR_UNSUPPORTED;
     const int bn = pick_bn_out(g.W);
     p.n_tiles = g.W / bn;
-    CUtensorMap ma, mb, m0, m1, m2;
+    CUtensorMap ma, mb, m0, m1, m2, mo;
     memset(&m0, 0, sizeof(m0));
     memset(&m1, 0, sizeof(m1));
-    if (!map_2d(&ma, hidden_s, (uint64_t)g.banks * g.B, Fs, 128) || !map_2d(&mb, wd, (uint64_t)g.banks * g.W, Fs, bn))
+    if (!map_2d(&ma, hidden_s, (uint64_t)g.banks * g.B, Fs, 128) || !map_2d(&mb, wd, (uint64_t)g.banks * g.W, Fs, bn) ||
+        !gemm1_amap(g, y, am, &mo, 32))
         return TM_ERR_CUDA;
     if (resid && !gemm1_amap(g, resid, am, &m0)) return TM_ERR_CUDA;
     if (extra && !gemm1_amap(g, extra, am, &m1)) return TM_ERR_CUDA;
@@ -504,7 +506,7 @@ tm_status combine_sum(const Geo& g, const void* hidden_s, const void* wd, int Fs
         uint32_t box[4] = {64, 1, 1, 128};
         if (!make_map(&m2, slots, 4, dims, strides, box)) return TM_ERR_CUDA;
     }
-    return cuda_status(launch_grouped_gemm_src(bn, A_TMA_2D, EPI_SUM, ma, mb, mb, m0, m1, m2, p, dense_grid(p), st));
+    return cuda_status(launch_grouped_gemm_src(bn, A_TMA_2D, EPI_SUM, ma, mb, mb, m0, m1, m2, p, dense_grid(p), st, &mo));
 }
 
 tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* extra, const void* gain,
@@ -562,18 +564,20 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
         const bool gather_in_gemm = env_g && env_g[0] == '1';
         const int bn = pick_bn_swiglu(Fe);
         p.n_tiles = p.N / bn;
-        CUtensorMap ma, mg, mu;
+        CUtensorMap ma, mg, mu, mo;
         memset(&ma, 0, sizeof(ma));
-        if (!map_2d(&mg, weg, G * Fe, g.W, bn / 2) || !map_2d(&mu, weu, G * Fe, g.W, bn / 2)) return TM_ERR_CUDA;
+        if (!map_2d(&mg, weg, G * Fe, g.W, bn / 2) || !map_2d(&mu, weu, G * Fe, g.W, bn / 2) ||
+            !map_2d(&mo, m.hidden_r, routed, Fe, 32))
+            return TM_ERR_CUDA;
         if (!gather_in_gemm) {
-            if ((s = cuda_status(launch_gather_rows(g.dtype, x, g.map, g.B, w->E, m.offsets, (int)G, m.bucket_rows, routed,
-                                                    m.slots, st))) != TM_OK)
+            if ((s = cuda_status(launch_scatter_rows(g.dtype, x, g.map, g.B, w->k, m.slot_of, routed, m.slots, st))) !=
+                TM_OK)
                 return s;
             if (!map_2d(&ma, m.slots, routed, g.W, 128)) return TM_ERR_CUDA;
         }
         const long grid = max_mt * p.n_tiles < num_sms() ? max_mt * p.n_tiles : num_sms();
         if ((s = cuda_status(launch_grouped_gemm(bn, gather_in_gemm ? A_GATHER : A_TMA_2D, EPI_SWIGLU, ma, mg, mu, p,
-                                                 (int)grid, st))) != TM_OK)
+                                                 (int)grid, st, &mo))) != TM_OK)
             return s;
     }
     // shared expert GEMM1 (dense rows)

@@ -136,7 +136,8 @@ cudaError_t launch_fused(int W, int a_mode, const CUtensorMap& a, const CUtensor
 
 template <int BN, int AM, int EPI>
 static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& s0,
-                              const CUtensorMap& s1, const CUtensorMap& s2, const GemmParams& p, int grid, cudaStream_t st) {
+                              const CUtensorMap& s1, const CUtensorMap& s2, const CUtensorMap& o, const GemmParams& p,
+                              int grid, cudaStream_t st) {
     using C = GemmCfg<BN, AM, EPI>;
     auto kern = grouped_gemm_kernel<BN, AM, EPI>;
     static bool configured = false;   // attribute set once per instantiation (per process)
@@ -151,7 +152,7 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
                      : (EPI == EPI_SLOT || EPI == EPI_SLOT_PERM) ? "gemm_slot"
                                                                  : "gemm_combine",
                      st);
-    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, b0, b1, s0, s1, s2, p);
+    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, b0, b1, s0, s1, s2, o, p);
     return cudaGetLastError();
 }
 
@@ -188,20 +189,27 @@ int grouped_gemm_smem(int bn, int a_mode) {
 
 cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                                     const CUtensorMap& tmB1, const CUtensorMap& tmS0, const CUtensorMap& tmS1,
-                                    const CUtensorMap& tmS2, const GemmParams& p, int grid, cudaStream_t st) {
+                                    const CUtensorMap& tmS2, const GemmParams& p, int grid, cudaStream_t st,
+                                    const CUtensorMap* tmO) {
+    // the SwiGLU and combine epilogues store through the output map
+    if ((epi == EPI_SWIGLU || epi == EPI_SUM) && !tmO) return cudaErrorInvalidValue;
+    CUtensorMap none;
+    memset(&none, 0, sizeof(none));
+    const CUtensorMap& o = tmO ? *tmO : none;
 #define X(BN, AM, EP)                                  \
     if (bn == BN && a_mode == AM && epi == EP)         \
-        return launch_one<BN, AM, EP>(tmA, tmB0, tmB1, tmS0, tmS1, tmS2, p, grid, st);
+        return launch_one<BN, AM, EP>(tmA, tmB0, tmB1, tmS0, tmS1, tmS2, o, p, grid, st);
     TM_GEMM_TABLE(X)
 #undef X
     return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_grouped_gemm(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
-                                const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st) {
+                                const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st,
+                                const CUtensorMap* tmO) {
     CUtensorMap none;
     memset(&none, 0, sizeof(none));
-    return launch_grouped_gemm_src(bn, a_mode, epi, tmA, tmB0, tmB1, none, none, none, p, grid, st);
+    return launch_grouped_gemm_src(bn, a_mode, epi, tmA, tmB0, tmB1, none, none, none, p, grid, st, tmO);
 }
 
 }  // namespace tml

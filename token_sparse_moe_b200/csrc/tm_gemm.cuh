@@ -15,6 +15,11 @@
 // 32-byte run of one token, fetched as a 128-row box with 32-byte swizzle), or a
 // cp.async row gather (routed rows).
 //
+// Output: GEMM1 hidden rows and the combine's rows go out through bulk tensor stores (tmO: the
+// hidden rows with 32 x 64 boxes, or the row / Revert geometry of y), one 4 KB box per epilogue
+// warp staged in shared memory; the routed GEMM2's sample-order rows are scattered, so they are
+// staged the same way and written by the warp four whole 128-byte row pieces per instruction.
+//
 // Tile: 128 rows x BN columns, K in 64-wide slabs with 128-byte swizzle.  Warp roles:
 // warp 0 TMA producer, warp 1 MMA issuer (one thread) and TMEM owner, warps 2-5
 // epilogue (TMEM lane quarter = warp % 4), warps 6-9 row gatherers (gather mode).
@@ -98,8 +103,13 @@ struct GemmCfg {
     static constexpr int NWARPS = (AMODE == A_GATHER || EPI == EPI_ROUTE) ? 10 : 6;
     static constexpr int NTHREADS = NWARPS * 32;
     static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
-    static constexpr int OFF_ID = STAGES * STAGE_BYTES;           // 16 x 16 identity (EPI_SUM), 1 KB
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024 + 256;
+    // output staging: one 32-row x 64-column bf16 box (4 KB) per epilogue warp
+    static constexpr bool STAGED = EPI == EPI_SWIGLU || EPI == EPI_SLOT_PERM || EPI == EPI_SUM;
+    static constexpr int OFF_STG = STAGES * STAGE_BYTES;
+    static constexpr int STG_BYTES = STAGED ? 4 * 4096 : 0;
+    static constexpr int OFF_ID = OFF_STG + STG_BYTES;             // 16 x 16 identity (EPI_SUM), 1 KB
+    static constexpr int SMEM_BYTES = OFF_ID + 1024 + 1024 + 256;
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 struct TileInfo {
@@ -116,9 +126,10 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int t) {
     const int gm = t / p.n_tiles;
     ti.n = t - gm * p.n_tiles;
     if (p.sched == 0) {
-        const int mt = (p.rows + 127) / 128;
-        ti.g = gm / mt;
-        ti.m = gm - ti.g * mt;
+        // row block major, banks innermost: the CTAs running side by side read the same samples'
+        // token rows (whole sectors when a bank's segment of a row is short, as with the Mix map)
+        ti.m = gm / p.groups;
+        ti.g = gm - ti.m * p.groups;
         ti.row0 = ti.g * p.rows + ti.m * 128;
         ti.nrows = min(128, p.rows - ti.m * 128);
     } else {
@@ -156,7 +167,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmS0,
                         const __grid_constant__ CUtensorMap tmS1, const __grid_constant__ CUtensorMap tmS2,
-                        const GemmParams p) {
+                        const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
     using C = GemmCfg<BN, AMODE, EPI>;
     constexpr int STAGES = C::STAGES;
     const int ntile = total_tiles(p);
@@ -356,6 +367,30 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
         // ---------------------------------------------------------------- epilogue
         const int q = warp & 3;
         const int r = q * 32 + lane;
+        uint8_t* stg = smem + C::OFF_STG + q * 4096;                  // this warp's 32 x 64 staging box
+        // this thread's row (lane) of a 64-column bf16 chunk into the box, 128-byte swizzled rows,
+        // once the warp's previous bulk store has read it
+        auto stage_row = [&](const uint32_t(&pk)[32]) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8)
+                *reinterpret_cast<uint4*>(stg + lane * 128 + ((c8 ^ (lane & 7)) << 4)) =
+                    make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+        };
+        // the staged box to global rows: row rr (lane rr's my_off: element offset of its chunk
+        // start, < 0 skips the row) gets columns col .. col + 63; four rows per store instruction
+        auto copy_rows = [&](long long my_off, int col) {
+            __syncwarp();
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+                const int rr = it * 4 + (lane >> 3), cc = lane & 7;
+                const long long off = __shfl_sync(0xffffffffu, my_off, rr);
+                const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((cc ^ (rr & 7)) << 4));
+                if (off >= 0) *reinterpret_cast<uint4*>(p.out + off + col + cc * 8) = v;
+            }
+            __syncwarp();
+        };
         int lt = 0;
         for (int t = blockIdx.x; t < ntile; t += gridDim.x, ++lt) {
             const TileInfo ti = decode_tile(p, t);
@@ -443,66 +478,98 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
                 }
             } else if (EPI == EPI_SWIGLU) {
                 const float sc = valid ? __ldg(&p.inv_rms[(size_t)b * p.banks + bank]) : 0.f;
-                __nv_bfloat16* dst = p.out + (size_t)pos * p.out_ld + ti.n * (BN / 2);
+                // a bulk tensor store per 32 x 64 box when all 32 rows of this warp belong to the
+                // tile's group; else the valid rows through coalesced stores
+                const bool box = __all_sync(0xffffffffu, valid);
+                const long long my_off = valid ? (long long)pos * p.out_ld + ti.n * (BN / 2) : -1ll;
 #pragma unroll 1
-                for (int c = 0; c < BN / 2; c += 32) {
-                    float gv[32], uv[32];
-                    tmem_ld32(taddr + c, gv);
-                    tmem_ld32(taddr + BN / 2 + c, uv);
-                    if (valid) {
-                        uint32_t pk[16];
+                for (int c = 0; c < BN / 2; c += 64) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float gv[32], uv[32];
+                        tmem_ld32(taddr + c + 32 * h, gv);
+                        tmem_ld32(taddr + BN / 2 + c + 32 * h, uv);
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const float h0 = silu_tanh(sc * gv[2 * i]) * (sc * uv[2 * i]);
                             const float h1 = silu_tanh(sc * gv[2 * i + 1]) * (sc * uv[2 * i + 1]);
-                            pk[i] = pack_bf16x2(h0, h1);
+                            pk[16 * h + i] = pack_bf16x2(h0, h1);
                         }
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                    stage_row(pk);
+                    if (box) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmO, stg, ti.n * (BN / 2) + c, ti.row0 + q * 32);
+                            bulk_commit_group();
+                        }
+                    } else {
+                        copy_rows(my_off, c);
                     }
                 }
             } else if (EPI == EPI_SLOT_PERM) {
-                // the row of choice j of sample b (bank of the group), scaled by its gate
+                // the row of choice j of sample b (bank of the group), scaled by its gate: rows are
+                // scattered, so each 64-column chunk is staged and written four whole rows at a time
                 const int e = valid ? __ldg(&p.perm[pos]) : 0;
                 if (valid && (e < 0 || e >= p.pos_limit)) {
                     record_error(ERR_BOUNDS, 0x314);
                     valid = false;
                 }
                 const float gsc = valid ? __ldg(&p.gate[e]) : 0.f;
-                __nv_bfloat16* dst = p.out + (size_t)e * p.out_ld + ti.n * BN;
+                const long long my_off = valid ? (long long)e * p.out_ld + ti.n * BN : -1ll;
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    float v[32];
-                    tmem_ld32(taddr + c, v);
-                    if (valid) {
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+                for (int c = 0; c < BN; c += 64) {
+                    uint32_t pk[32];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            d4[i] = make_uint4(pack_bf16x2(gsc * v[8 * i], gsc * v[8 * i + 1]),
-                                               pack_bf16x2(gsc * v[8 * i + 2], gsc * v[8 * i + 3]),
-                                               pack_bf16x2(gsc * v[8 * i + 4], gsc * v[8 * i + 5]),
-                                               pack_bf16x2(gsc * v[8 * i + 6], gsc * v[8 * i + 7]));
+                    for (int h = 0; h < 2; ++h) {
+                        float v[32];
+                        tmem_ld32(taddr + c + 32 * h, v);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) pk[16 * h + i] = pack_bf16x2(gsc * v[2 * i], gsc * v[2 * i + 1]);
                     }
+                    stage_row(pk);
+                    copy_rows(my_off, c);
                 }
             } else if (EPI == EPI_SUM) {
-                // Y already holds every term: bf16 through the row map
+                // Y already holds every term: bf16 through the output's row or Revert geometry, one
+                // bulk tensor store per 32 x 64 box (rows past B are clipped by the map)
+                const int b0 = ti.m * 128 + q * 32;
+                const bool mixed = p.omap.layout == 1;
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    float v[32];
-                    tmem_ld32(taddr + c, v);
-                    if (!valid) continue;
-                    const int col0 = ti.n * BN + c;
+                for (int c = 0; c < BN; c += 64) {
+                    uint32_t pk[32];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const size_t off = row_elem(p.omap, b, bank, col0 + 8 * i);
-                        if (off + 8 > p.out_elems) {
-                            record_error(ERR_BOUNDS, 0x315);
-                            continue;
+                    for (int h = 0; h < 2; ++h) {
+                        float v[32];
+                        tmem_ld32(taddr + c + 32 * h, v);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) pk[16 * h + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                    }
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+#pragma unroll
+                    for (int c8 = 0; c8 < 8; ++c8) {
+                        uint8_t* dst = mixed ? stg + (c8 >> 1) * 1024 + lane * 32 + (((c8 & 1) ^ ((lane >> 2) & 1)) << 4)
+                                             : stg + lane * 128 + ((c8 ^ (lane & 7)) << 4);
+                        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && b0 < p.rows) {
+                        const int col = ti.n * BN + c;
+                        if (mixed) {
+                            const int per = p.omap.dh >> 4;
+#pragma unroll
+                            for (int k4 = 0; k4 < 4; ++k4) {
+                                const int ci = (col >> 4) + k4, tok = ci / per, jj = ci - tok * per;
+                                tma_store_4d(&tmO, stg + k4 * 1024, 0, bank * per + jj, tok, b0);
+                            }
+                        } else {
+                            tma_store_3d(&tmO, stg, col, bank, b0);
                         }
-                        *reinterpret_cast<uint4*>(p.out + off) =
-                            make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                                       pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+                        bulk_commit_group();
                     }
                 }
             } else if (EPI == EPI_SLOT) {
@@ -606,6 +673,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
+        if (C::STAGED && lane == 0) bulk_wait_all();                  // stores complete before exit
+        __syncwarp();
     } else if (EPI == EPI_ROUTE) {
         // ---------------------------------------------------------------- row statistics (warps 6-9)
         // Each lane sums the squares of its row of every A stage (a second consumer of the stage:

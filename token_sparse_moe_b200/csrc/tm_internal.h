@@ -30,11 +30,15 @@ void note_cuda_error(const char* where, cudaError_t e);   // samples per router 
 // a_mode: AMode; epi: Epi; bn: tile width.  maps are passed by value into the kernel.
 // with the EPI_SUM source maps: s0 residual, s1 inter-residual (row geometry of the output),
 // s2 the sample-order expert rows [B, banks, k, W]
+// tmO: the output map, required by EPI_SWIGLU (the hidden rows, 64-column x 32-row boxes) and
+// EPI_SUM (y in its row geometry: 3-D rows or the 4-D Revert map, 32-row boxes)
 cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                                     const CUtensorMap& tmB1, const CUtensorMap& tmS0, const CUtensorMap& tmS1,
-                                    const CUtensorMap& tmS2, const GemmParams& p, int grid, cudaStream_t st);
+                                    const CUtensorMap& tmS2, const GemmParams& p, int grid, cudaStream_t st,
+                                    const CUtensorMap* tmO = nullptr);
 cudaError_t launch_grouped_gemm(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
-                                const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st);
+                                const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st,
+                                const CUtensorMap* tmO = nullptr);
 bool grouped_gemm_supported(int bn, int a_mode, int epi);
 
 // ---- fused dense sub-layer (row width 128 / 256) --------------------------------
@@ -76,9 +80,10 @@ cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, cons
 // tensor-core router weights: [banks][64][W] bf16, rows e / E+e / 2E+e = hi / mid / lo of w * gain
 cudaError_t launch_router_split(int dtype, const float* w_router, const void* gain, int banks, int E, int W,
                                 void* out, cudaStream_t st);
-// MoEPermute data copy: routed row positions receive their source rows (see gather_rows_kernel)
-cudaError_t launch_gather_rows(int dtype, const void* x, RowMap m, int B, int E, const int32_t* offsets, int groups,
-                               const int32_t* bucket_rows, size_t routed, void* out, cudaStream_t st);
+// MoEPermute data copy: each source row to the k bucketed row positions of its choices (slot_of
+// [B * banks * k], k <= 8), out [routed, W] (see scatter_rows_kernel)
+cudaError_t launch_scatter_rows(int dtype, const void* x, RowMap m, int B, int k, const int32_t* slot_of, size_t routed,
+                                void* out, cudaStream_t st);
 cudaError_t launch_permute(int dtype, const void* src, void* dst, int B, int T, int D, int H, bool to_mixed,
                            cudaStream_t st);
 cudaError_t launch_fold_gain(int dtype, const void* w, const void* gain, void* out, size_t rows, int width,

@@ -435,39 +435,61 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtGemmArgs a) {
     }
 }
 
-// MoEPermute, data part: row position pos of the bucketed order (bank-major, then expert, then
-// ascending sample) receives a copy of its source row (sample bucket_rows[pos], bank of the
-// position's group) read through the row map, so that the routed GEMM1 reads its A operand as
-// plain contiguous rows.  One warp per position; 16-byte pieces when a head segment holds whole
-// pieces, element copies otherwise.
+// MoEPermute, data part: each source row (sample b, bank), read once through the row map, is
+// copied to the k bucketed row positions of its choices (slot_of[(b * banks + bank) * k + j]), so
+// that the routed GEMM1 reads its A operand as plain contiguous rows.  Rows are visited in sample
+// order with the bank innermost: neighbouring warps read neighbouring head segments of the same
+// token rows (for the mixing sub-layer, 16 columns of every token of a sample per bank), so the
+// token rows' sectors are used whole.  One warp per source row; 16-byte pieces when a head
+// segment holds whole pieces, element copies otherwise.
 template <typename T>
-__global__ void __launch_bounds__(256) gather_rows_kernel(const T* __restrict__ x, RowMap m, int B, int E,
-                                                          const int32_t* __restrict__ offsets, int groups,
-                                                          const int32_t* __restrict__ bucket_rows, int routed,
-                                                          T* __restrict__ out) {
+__global__ void __launch_bounds__(256) scatter_rows_kernel(const T* __restrict__ x, RowMap m, int B, int k,
+                                                           const int32_t* __restrict__ slot_of, int routed,
+                                                           T* __restrict__ out) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
-    const int W = m.W;
+    const int W = m.W, banks = m.banks;
     constexpr int V = 16 / sizeof(T);
     const bool vec = (m.layout == 0 || m.dh % V == 0) && W % V == 0;
-    for (int pos = warp; pos < routed; pos += nwarps) {
-        int lo = 0, hi = groups;   // offsets[lo] <= pos < offsets[hi]
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (__ldg(&offsets[mid]) <= pos) lo = mid; else hi = mid;
+    const int rows = B * banks;
+    for (int row = warp; row < rows; row += nwarps) {
+        const int b = row / banks, bank = row - b * banks;
+        int pos[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            pos[j] = j < k ? __ldg(&slot_of[(size_t)row * k + j]) : -1;
+            if (j < k && (pos[j] < 0 || pos[j] >= routed)) {
+                if (lane == 0) record_error(ERR_BOUNDS, 0x520);
+                pos[j] = -1;
+            }
         }
-        const int bank = lo / E;
-        const int b = __ldg(&bucket_rows[pos]);
-        if (b < 0 || b >= B) {
-            if (lane == 0) record_error(ERR_BOUNDS, 0x520);
-            continue;
-        }
-        T* dst = out + (size_t)pos * W;
         if (vec) {
-            for (int c = lane * V; c < W; c += 32 * V)
-                *reinterpret_cast<uint4*>(dst + c) = __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c)));
+            // up to four 16-byte pieces per lane loaded before any store, so a row's reads are all
+            // in flight together
+            for (int c0 = lane * V; c0 < W; c0 += 4 * 32 * V) {
+                uint4 v[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int c = c0 + i * 32 * V;
+                    if (c < W) v[i] = __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c)));
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (pos[j] < 0) continue;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int c = c0 + i * 32 * V;
+                        if (c < W) *reinterpret_cast<uint4*>(out + (size_t)pos[j] * W + c) = v[i];
+                    }
+                }
+            }
         } else {
-            for (int c = lane; c < W; c += 32) dst[c] = x[row_elem(m, b, bank, c)];
+            for (int c = lane; c < W; c += 32) {
+                const T v = x[row_elem(m, b, bank, c)];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if (pos[j] >= 0) out[(size_t)pos[j] * W + c] = v;
+            }
         }
     }
 }
@@ -578,16 +600,15 @@ cudaError_t launch_router_split(int dtype, const float* w_router, const void* ga
     return cudaGetLastError();
 }
 
-cudaError_t launch_gather_rows(int dtype, const void* x, RowMap m, int B, int E, const int32_t* offsets, int groups,
-                               const int32_t* bucket_rows, size_t routed, void* out, cudaStream_t st) {
+cudaError_t launch_scatter_rows(int dtype, const void* x, RowMap m, int B, int k, const int32_t* slot_of, size_t routed,
+                                void* out, cudaStream_t st) {
     ProfileScope ps_("moe_permute", st);
-    const int grid = grid_for(routed * 32, 256);
+    const int grid = grid_for((size_t)B * m.banks * 32, 256);
     if (dtype == 1)
-        gather_rows_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, m, B, E, offsets, groups,
-                                                                bucket_rows, (int)routed, (__nv_bfloat16*)out);
+        scatter_rows_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, m, B, k, slot_of, (int)routed,
+                                                                 (__nv_bfloat16*)out);
     else
-        gather_rows_kernel<float><<<grid, 256, 0, st>>>((const float*)x, m, B, E, offsets, groups, bucket_rows,
-                                                        (int)routed, (float*)out);
+        scatter_rows_kernel<float><<<grid, 256, 0, st>>>((const float*)x, m, B, k, slot_of, (int)routed, (float*)out);
     return cudaGetLastError();
 }
 
