@@ -81,7 +81,10 @@ def kernel_flops(cfg, B) -> dict:
                 add("fused_swiglu", B * banks * 6.0 * W * s.hidden)
             else:
                 add("gemm_swiglu", B * banks * 4.0 * W * s.hidden)
-                add("gemm_resid", B * banks * 2.0 * W * s.hidden)
+                # bf16 rows readable through a tensor map (row layout, or mixed with 16-column head
+                # pieces) take the combine kernel (residual by identity MMAs); others the residual epilogue
+                tmap = cfg.dtype == "bf16" and (sub == 1 or (cfg.D // cfg.H) % 16 == 0)
+                add("gemm_combine" if tmap else "gemm_resid", B * banks * 2.0 * W * s.hidden)
     return out
 
 

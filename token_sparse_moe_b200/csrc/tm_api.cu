@@ -363,6 +363,9 @@ DenseWs carve_dense(Carve& c, const Geo& g, int F, bool gain) {
     return w;
 }
 
+tm_status combine_sum(const Geo& g, const void* hidden_s, const void* wd, int Fs, const void* resid, const void* extra,
+                      void* y, const void* slots, int k, cudaStream_t st);
+
 tm_status run_dense(const Geo& g, const void* x, const void* resid, const void* extra, const void* gain,
                     const tm_swiglu_w* w, void* y, void* ws, size_t wsb, cudaStream_t st) {
     Carve c{(uint8_t*)ws};
@@ -383,6 +386,11 @@ tm_status run_dense(const Geo& g, const void* x, const void* resid, const void* 
                            (size_t)g.banks * g.B * w->hidden * g.esz, st);
     if ((s = cuda_status(launch_rms(g.dtype, x, g.map, g.B, g.eps, d.inv_rms, st))) != TM_OK) return s;
     if ((s = gemm1_dense(g, x, wg, wu, w->hidden, d.inv_rms, d.hidden, st)) != TM_OK) return s;
+    // bf16 with a tensor-map row geometry: GEMM2 with the residual and inter-residual entering the
+    // accumulator through identity MMAs and bulk tensor stores out (the combine kernel, no expert rows)
+    const int am = gemm1_amode(g);
+    if (g.dtype == TM_BF16 && (am == A_TMA_3D || am == A_TMA_MIX))
+        return combine_sum(g, d.hidden, w->w_down, w->hidden, resid, extra, y, nullptr, 0, st);
     return gemm2_dense(g, d.hidden, w->w_down, w->hidden, EPI_RESID, resid, extra, y, nullptr, nullptr, nullptr, 0, st);
 }
 
@@ -390,7 +398,8 @@ tm_status run_dense(const Geo& g, const void* x, const void* resid, const void* 
 struct MoeWs {
     float* inv_rms;
     int32_t *idx, *slot_of, *bucket_rows, *offsets, *tile_start, *counts, *perm;
-    float* gate;
+    int4* tile_info;
+    float *gate, *inv_pos, *gate_pos;
     void *hidden_r, *slots, *hidden_s;
     void *weg, *weu, *wsg, *wsu;
     void* wsplit;
@@ -407,8 +416,11 @@ MoeWs carve_moe(Carve& c, const Geo& g, const tm_moe_w* w, bool gain) {
     m.slot_of = c.take<int32_t>(routed);
     m.bucket_rows = c.take<int32_t>(routed);
     m.perm = c.take<int32_t>(routed);
+    m.inv_pos = c.take<float>(routed);
+    m.gate_pos = c.take<float>(routed);
     m.offsets = c.take<int32_t>(G + 1);
     m.tile_start = c.take<int32_t>(G + 1);
+    m.tile_info = c.take<int4>(routed / 128 + G);   // at most this many 128-row tiles
     m.counts = c.take<int32_t>((size_t)g.banks * nchunks * w->E);
     m.hidden_r = c.take<uint8_t>(routed * w->hidden_e * g.esz);
     m.slots = c.take<uint8_t>(routed * g.W * g.esz);
@@ -427,6 +439,9 @@ struct RouteOut {
     float *gate, *inv_rms;
     int32_t* perm = nullptr;   // optional: sample-order row of each bucket position
     void* wsplit = nullptr;    // optional: [banks][64][W] bf16 split router weights (tensor-core router)
+    int4* tile_info = nullptr; // optional: per 128-row tile descriptors of the buckets
+    float* inv_pos = nullptr;  // optional: 1/rms of each bucket position's row
+    float* gate_pos = nullptr; // optional: gate of each bucket position's choice
 };
 
 
@@ -465,11 +480,11 @@ tm_status run_route(const Geo& g, const void* x, const void* gain, const tm_moe_
                                               r.idx, r.gate, r.inv_rms, r.counts, st))) != TM_OK) {
         return s;
     }
-    if ((s = cuda_status(launch_offsets(r.counts, r.counts, g.banks, nchunks, w->E, r.offsets, r.tile_start, st))) !=
-        TM_OK)
+    if ((s = cuda_status(launch_offsets(r.counts, r.counts, g.banks, nchunks, w->E, r.offsets, r.tile_start, st,
+                                        r.tile_info))) != TM_OK)
         return s;
     return cuda_status(launch_scatter(r.idx, r.counts, r.offsets, g.B, g.banks, w->E, w->k, r.bucket_rows, r.slot_of, st,
-                                      r.perm));
+                                      r.perm, r.inv_rms, r.gate, r.inv_pos, r.gate_pos));
 }
 
 // MoE combine on the tensor core: Y = residual (+ inter-residual) + sum_j (gate-scaled expert row j
@@ -500,7 +515,8 @@ tm_status combine_sum(const Geo& g, const void* hidden_s, const void* wd, int Fs
         return TM_ERR_CUDA;
     if (resid && !gemm1_amap(g, resid, am, &m0)) return TM_ERR_CUDA;
     if (extra && !gemm1_amap(g, extra, am, &m1)) return TM_ERR_CUDA;
-    {
+    memset(&m2, 0, sizeof(m2));
+    if (k > 0) {
         uint64_t dims[4] = {(uint64_t)g.W, (uint64_t)k, (uint64_t)g.banks, (uint64_t)g.B};
         uint64_t strides[3] = {(uint64_t)g.W * 2, (uint64_t)k * g.W * 2, (uint64_t)g.banks * k * g.W * 2};
         uint32_t box[4] = {64, 1, 1, 128};
@@ -529,8 +545,13 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
     }
     RouteOut r{m.idx, m.offsets, m.tile_start, m.bucket_rows, m.slot_of, m.counts, m.gate, m.inv_rms};
     const bool bf16_path = g.dtype == TM_BF16;
-    if (bf16_path) r.perm = m.perm;
+    if (bf16_path) {
+        r.perm = m.perm;
+        r.inv_pos = m.inv_pos;
+        r.gate_pos = m.gate_pos;
+    }
     r.wsplit = m.wsplit;
+    r.tile_info = m.tile_info;
     if ((s = run_route(g, x, gain, w, r, st)) != TM_OK) return s;
 
     const size_t routed = (size_t)g.B * g.banks * w->k;
@@ -542,7 +563,9 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
     p.E = w->E;
     p.row_start = m.offsets;
     p.tile_start = m.tile_start;
+    p.tile_info = m.tile_info;
     p.bucket_rows = m.bucket_rows;
+    p.pos_scale = bf16_path ? m.inv_pos : nullptr;
     p.pos_limit = (int)routed;
     p.K = g.W;
     p.N = 2 * Fe;
@@ -599,6 +622,7 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
         p.n_tiles = g.W / bn;
         p.perm = m.perm;
         p.gate = m.gate;
+        p.pos_scale = m.gate_pos;
         CUtensorMap ma, mb;
         if (!map_2d(&ma, m.hidden_r, routed, Fe, 128) || !map_2d(&mb, w->we_down, G * g.W, Fe, bn)) return TM_ERR_CUDA;
         const long grid = max_mt * p.n_tiles < num_sms() ? max_mt * p.n_tiles : num_sms();

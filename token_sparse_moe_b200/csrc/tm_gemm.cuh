@@ -63,7 +63,9 @@ struct GemmParams {
     int E;                     // sched 1: experts per bank (bank = g / E)
     const int* row_start;      // sched 1: [groups+1] first row position of each group
     const int* tile_start;     // sched 1: [groups+1] prefix of 128-row tiles per group
+    const int4* tile_info;     // sched 1: per 128-row tile {group, first row position, rows, tile in group}
     const int* bucket_rows;    // sched 1: sample index of each row position
+    const float* pos_scale;    // sched 1 (optional): per row position, 1/rms (EPI_SWIGLU) or gate (EPI_SLOT_PERM)
     int pos_limit;             // row positions in hidden / slot buffers (bounds check)
     size_t out_elems;          // elements of `out` (and of resid / extra for the row-map epilogues)
     int K, N, n_tiles;         // reduction length, output columns per group, N / BN
@@ -132,6 +134,12 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int t) {
         ti.g = gm - ti.m * p.groups;
         ti.row0 = ti.g * p.rows + ti.m * 128;
         ti.nrows = min(128, p.rows - ti.m * 128);
+    } else if (p.tile_info) {
+        const int4 d = __ldg(&p.tile_info[gm]);
+        ti.g = d.x;
+        ti.row0 = d.y;
+        ti.nrows = d.z;
+        ti.m = d.w;
     } else {
         int lo = 0, hi = p.groups;   // invariant: tile_start[lo] <= gm < tile_start[hi]
         while (hi - lo > 1) {
@@ -238,8 +246,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
             if (EPI == EPI_SWIGLU) tma_prefetch_desc(&tmB1);
             int s = 0;
             uint32_t ph = 0;
+            TileInfo tn = decode_tile(p, blockIdx.x);
             for (int t = blockIdx.x; t < ntile; t += gridDim.x) {
-                const TileInfo ti = decode_tile(p, t);
+                const TileInfo ti = tn;
+                if (t + (int)gridDim.x < ntile) tn = decode_tile(p, t + gridDim.x);   // in flight meanwhile
                 if (EPI == EPI_SUM) {
                     // source slabs: rows of this tile's samples, output columns n*BN .. +BN
 #pragma unroll 1
@@ -391,9 +401,41 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
             }
             __syncwarp();
         };
+        // This thread's row of a tile: sample b, sample-order slot e (EPI_SLOT_PERM), scale s (1/rms
+        // for EPI_SWIGLU, the gate for EPI_SLOT_PERM).  The loads are issued a tile ahead (and the
+        // tile descriptor two tiles ahead) and only waited for when the tile is processed.
+        struct RowMeta {
+            int b, e;
+            float s;
+        };
+        const bool by_pos = p.sched == 1 && p.pos_scale != nullptr;
+        auto row_meta = [&](const TileInfo& ti) -> RowMeta {
+            RowMeta m{0, 0, 0.f};
+            const int pos = ti.row0 + r;
+            if (r >= ti.nrows || pos < 0 || pos >= p.pos_limit) return m;
+            const bool need_b = p.sched == 1 && !(EPI == EPI_SLOT_PERM || (EPI == EPI_SWIGLU && by_pos));
+            m.b = p.sched == 0 ? ti.m * 128 + r : (need_b ? __ldg(&p.bucket_rows[pos]) : 0);
+            if (EPI == EPI_SWIGLU) {
+                const int bank = p.sched == 0 ? ti.g : ti.g / p.E;
+                m.s = by_pos ? __ldg(&p.pos_scale[pos]) : __ldg(&p.inv_rms[(size_t)m.b * p.banks + bank]);
+            } else if (EPI == EPI_SLOT_PERM) {
+                m.e = __ldg(&p.perm[pos]);
+                m.s = by_pos ? __ldg(&p.pos_scale[pos]) : 0.f;
+            }
+            return m;
+        };
+        TileInfo ti_n1 = decode_tile(p, blockIdx.x), ti_n2 = ti_n1;
+        RowMeta rm_n1 = row_meta(ti_n1);
+        if ((int)blockIdx.x + (int)gridDim.x < ntile) ti_n2 = decode_tile(p, blockIdx.x + gridDim.x);
         int lt = 0;
         for (int t = blockIdx.x; t < ntile; t += gridDim.x, ++lt) {
-            const TileInfo ti = decode_tile(p, t);
+            const TileInfo ti = ti_n1;
+            const RowMeta rm = rm_n1;
+            if (t + (int)gridDim.x < ntile) {
+                ti_n1 = ti_n2;
+                rm_n1 = row_meta(ti_n1);
+                if (t + 2 * (int)gridDim.x < ntile) ti_n2 = decode_tile(p, t + 2 * gridDim.x);
+            }
             const int buf = lt & 1;
             const uint32_t aph = (lt >> 1) & 1;
             if (!wait_or_abort(&acc_full[buf], aph, abort_flag, 0x300)) break;
@@ -401,14 +443,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
             const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + buf * BN;
             bool valid = r < ti.nrows;
             const int pos = ti.row0 + r;                      // row position (hidden / slot index)
-            int b, bank;
-            if (p.sched == 0) {
-                b = ti.m * 128 + r;
-                bank = ti.g;
-            } else {
-                b = valid ? __ldg(&p.bucket_rows[pos]) : 0;
-                bank = ti.g / p.E;
-            }
+            const int b = rm.b;
+            const int bank = p.sched == 0 ? ti.g : ti.g / p.E;
             if (valid && (b < 0 || b >= p.rows || pos < 0 || pos >= p.pos_limit)) {
                 record_error(ERR_BOUNDS, 0x310);
                 valid = false;
@@ -477,7 +513,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
                         atomicAdd(&p.r_counts[((size_t)bank * p.r_nchunks + ti.m) * E + e], __popc(bal));
                 }
             } else if (EPI == EPI_SWIGLU) {
-                const float sc = valid ? __ldg(&p.inv_rms[(size_t)b * p.banks + bank]) : 0.f;
+                const float sc = valid ? rm.s : 0.f;
                 // a bulk tensor store per 32 x 64 box when all 32 rows of this warp belong to the
                 // tile's group; else the valid rows through coalesced stores
                 const bool box = __all_sync(0xffffffffu, valid);
@@ -512,12 +548,12 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
             } else if (EPI == EPI_SLOT_PERM) {
                 // the row of choice j of sample b (bank of the group), scaled by its gate: rows are
                 // scattered, so each 64-column chunk is staged and written four whole rows at a time
-                const int e = valid ? __ldg(&p.perm[pos]) : 0;
+                const int e = valid ? rm.e : 0;
                 if (valid && (e < 0 || e >= p.pos_limit)) {
                     record_error(ERR_BOUNDS, 0x314);
                     valid = false;
                 }
-                const float gsc = valid ? __ldg(&p.gate[e]) : 0.f;
+                const float gsc = valid ? (by_pos ? rm.s : __ldg(&p.gate[e])) : 0.f;
                 const long long my_off = valid ? (long long)e * p.out_ld + ti.n * BN : -1ll;
 #pragma unroll 1
                 for (int c = 0; c < BN; c += 64) {

@@ -72,11 +72,15 @@ cudaError_t launch_rms(int dtype, const void* x, RowMap m, int B, float eps, flo
 cudaError_t launch_router(int dtype, const void* x, RowMap m, int B, float eps, const void* gain, const float* w_router,
                           int E, int k, float alpha, int32_t* idx, float* gate, float* inv_rms, int32_t* counts,
                           cudaStream_t st);
+// tile_info (optional): one {group, first row position, rows, tile within the group} per 128-row tile
 cudaError_t launch_offsets(const int32_t* counts_in, int32_t* chunk_prefix, int banks, int nchunks, int E,
-                           int32_t* bucket_offsets, int32_t* tile_start, cudaStream_t st);
+                           int32_t* bucket_offsets, int32_t* tile_start, cudaStream_t st, int4* tile_info = nullptr);
+// perm, inv_pos, gate_pos (optional, by bucket position): the sample-order row (b * banks + bank) * k + j,
+// the row's 1/rms (from inv_rms [B * banks]) and the choice's gate (from gate [B * banks * k])
 cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, const int32_t* bucket_offsets, int B,
                            int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st,
-                           int32_t* perm = nullptr);
+                           int32_t* perm = nullptr, const float* inv_rms = nullptr, const float* gate = nullptr,
+                           float* inv_pos = nullptr, float* gate_pos = nullptr);
 // tensor-core router weights: [banks][64][W] bf16, rows e / E+e / 2E+e = hi / mid / lo of w * gain
 cudaError_t launch_router_split(int dtype, const float* w_router, const void* gain, int banks, int E, int W,
                                 void* out, cudaStream_t st);

@@ -193,9 +193,10 @@ __global__ void __launch_bounds__(256) router_kernel(const T* __restrict__ x, Ro
 }
 
 // counts [banks][nchunks][E] -> (in place) exclusive prefix over chunks, plus the group
-// offsets and the 128-row tile prefix over groups g = bank*E + e.  One block.
+// offsets and the 128-row tile prefix over groups g = bank*E + e, and (optional) one descriptor
+// per 128-row tile {group, first row position, rows, tile within the group}.  One block.
 __global__ void __launch_bounds__(1024) offsets_kernel(int32_t* counts, int banks, int nchunks, int E,
-                                                       int32_t* bucket_offsets, int32_t* tile_start) {
+                                                       int32_t* bucket_offsets, int32_t* tile_start, int4* tile_info) {
     __shared__ int tot[4096];
     const int G = banks * E;
     for (int g = threadIdx.x; g < G; g += blockDim.x) {
@@ -231,6 +232,12 @@ __global__ void __launch_bounds__(1024) offsets_kernel(int32_t* counts, int bank
         }
         if (lane == 31) { bucket_offsets[G] = e1; tile_start[G] = e2; }
     }
+    if (!tile_info) return;
+    __syncthreads();                         // offsets and tile prefix written by warp 0
+    for (int g = threadIdx.x; g < G; g += blockDim.x) {
+        const int n = tot[g], r0 = bucket_offsets[g], t0 = tile_start[g];
+        for (int m = 0; m * 128 < n; ++m) tile_info[t0 + m] = make_int4(g, r0 + m * 128, min(128, n - m * 128), m);
+    }
 }
 
 // Stable scatter: position of (b, bank, j) = group offset + earlier chunks + earlier rows of
@@ -239,7 +246,10 @@ __global__ void __launch_bounds__(kRouterChunk) scatter_kernel(const int32_t* __
                                                                const int32_t* __restrict__ chunk_prefix,
                                                                const int32_t* __restrict__ bucket_offsets, int B,
                                                                int banks, int E, int k, int32_t* __restrict__ bucket_rows,
-                                                               int32_t* __restrict__ slot_of, int32_t* __restrict__ perm) {
+                                                               int32_t* __restrict__ slot_of, int32_t* __restrict__ perm,
+                                                               const float* __restrict__ inv_rms,
+                                                               const float* __restrict__ gate, float* __restrict__ inv_pos,
+                                                               float* __restrict__ gate_pos) {
     __shared__ int wcount[kRouterChunk / 32][64];
     const int bank = blockIdx.y, chunk = blockIdx.x, nchunks = gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -280,6 +290,10 @@ __global__ void __launch_bounds__(kRouterChunk) scatter_kernel(const int32_t* __
         slot_of[rowi * k + j] = pos;
         bucket_rows[pos] = b;
         if (perm) perm[pos] = (int32_t)(rowi * k + j);   // inverse of slot_of (optional)
+        // (optional) the row's 1/rms and the choice's gate by bucket position, so that the routed
+        // GEMMs read them as contiguous per-row values
+        if (inv_pos) inv_pos[pos] = inv_rms[rowi];
+        if (gate_pos) gate_pos[pos] = gate[rowi * k + j];
     }
 }
 
@@ -572,19 +586,21 @@ cudaError_t launch_router(int dtype, const void* x, RowMap m, int B, float eps, 
 }
 
 cudaError_t launch_offsets(const int32_t* counts_in, int32_t* chunk_prefix, int banks, int nchunks, int E,
-                           int32_t* bucket_offsets, int32_t* tile_start, cudaStream_t st) {
+                           int32_t* bucket_offsets, int32_t* tile_start, cudaStream_t st, int4* tile_info) {
     ProfileScope ps_("route_offsets", st);
     if (counts_in != chunk_prefix) return cudaErrorInvalidValue;   // the scan runs in place
-    offsets_kernel<<<1, 1024, 0, st>>>(chunk_prefix, banks, nchunks, E, bucket_offsets, tile_start);
+    offsets_kernel<<<1, 1024, 0, st>>>(chunk_prefix, banks, nchunks, E, bucket_offsets, tile_start, tile_info);
     return cudaGetLastError();
 }
 
 cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, const int32_t* bucket_offsets, int B,
-                           int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st, int32_t* perm) {
+                           int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st, int32_t* perm,
+                           const float* inv_rms, const float* gate, float* inv_pos, float* gate_pos) {
+    if ((inv_pos && !inv_rms) || (gate_pos && !gate)) return cudaErrorInvalidValue;
     ProfileScope ps_("route_scatter", st);
     dim3 grid((B + kRouterChunk - 1) / kRouterChunk, banks);
     scatter_kernel<<<grid, kRouterChunk, 0, st>>>(idx, chunk_prefix, bucket_offsets, B, banks, E, k, bucket_rows,
-                                                  slot_of, perm);
+                                                  slot_of, perm, inv_rms, gate, inv_pos, gate_pos);
     return cudaGetLastError();
 }
 
