@@ -101,14 +101,17 @@ struct GemmCfg {
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 192 ? 5 : 6);
-    static constexpr int NWARPS = (AMODE == A_GATHER || EPI == EPI_ROUTE) ? 10 : 6;
+    // the scattered-row epilogue is latency-bound per warp: two warps per TMEM lane quarter, each
+    // taking half of the tile's columns
+    static constexpr int EPI_WARPS = (EPI == EPI_SLOT_PERM && BN % 128 == 0) ? 8 : 4;
+    static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 192 ? (EPI_WARPS == 8 ? 4 : 5) : 6);
+    static constexpr int NWARPS = (AMODE == A_GATHER || EPI == EPI_ROUTE) ? 10 : 2 + EPI_WARPS;
     static constexpr int NTHREADS = NWARPS * 32;
     static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
     // output staging: one 32-row x 64-column bf16 box (4 KB) per epilogue warp
     static constexpr bool STAGED = EPI == EPI_SWIGLU || EPI == EPI_SLOT_PERM || EPI == EPI_SUM;
     static constexpr int OFF_STG = STAGES * STAGE_BYTES;
-    static constexpr int STG_BYTES = STAGED ? 4 * 4096 : 0;
+    static constexpr int STG_BYTES = STAGED ? EPI_WARPS * 4096 : 0;
     static constexpr int OFF_ID = OFF_STG + STG_BYTES;             // 16 x 16 identity (EPI_SUM), 1 KB
     static constexpr int SMEM_BYTES = OFF_ID + 1024 + 1024 + 256;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -209,7 +212,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 4);
+            mbar_init(&acc_empty[b], C::EPI_WARPS);
         }
         mbar_init(drain, 1);
         for (int b = 0; b < 2; ++b) {
@@ -373,11 +376,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
             umma_commit(drain);
             wait_or_abort(drain, 0, abort_flag, 0x202);
         }
-    } else if (warp >= 2 && warp < 6) {
+    } else if (warp >= 2 && warp < 2 + C::EPI_WARPS) {
         // ---------------------------------------------------------------- epilogue
         const int q = warp & 3;
         const int r = q * 32 + lane;
-        uint8_t* stg = smem + C::OFF_STG + q * 4096;                  // this warp's 32 x 64 staging box
+        // with 8 epilogue warps, warps 2-5 take columns [0, BN/2) and warps 6-9 [BN/2, BN)
+        const int c_lo = C::EPI_WARPS == 8 ? ((warp - 2) >> 2) * (BN / 2) : 0;
+        const int c_hi = C::EPI_WARPS == 8 ? c_lo + BN / 2 : BN;
+        uint8_t* stg = smem + C::OFF_STG + (warp - 2) * 4096;         // this warp's 32 x 64 staging box
         // this thread's row (lane) of a 64-column bf16 chunk into the box, 128-byte swizzled rows,
         // once the warp's previous bulk store has read it
         auto stage_row = [&](const uint32_t(&pk)[32]) {
@@ -556,7 +562,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
                 const float gsc = valid ? (by_pos ? rm.s : __ldg(&p.gate[e])) : 0.f;
                 const long long my_off = valid ? (long long)e * p.out_ld + ti.n * BN : -1ll;
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 64) {
+                for (int c = c_lo; c < c_hi; c += 64) {
                     uint32_t pk[32];
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
