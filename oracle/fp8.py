@@ -1,0 +1,139 @@
+"""FP8 E4M3 serving path of the dense per-token SwiGLU FFN: the float64 oracle.
+
+TEST INFRASTRUCTURE ONLY, like the rest of this package: imported by the tests, the smoke
+check and the benchmark's CPU leg, never by the library, and sharing no code or table with it.
+
+Source: [digest] "TokenMixer-Large: Scaling Up Large Ranking Models in Industrial
+Recommenders", section 2.5.2 (FP8 quantization): serving uses FP8 E4M3 post-training
+quantization of a model trained in bf16.  The page names the format only; the readings here
+(each one also listed in the repository's design notes):
+  * E4M3 is the 8-bit format with 1 sign bit, 4 exponent bits of bias 7 and 3 mantissa bits:
+    normal values 2^(e-7) * (1 + m/8) for exponent fields e = 1..15, subnormals m * 2^-9 for
+    e = 0, largest finite 448 (the all-ones pattern S.1111.111 is NaN; there are no
+    infinities).  Conversion rounds to nearest with ties to even and saturates at +-448.
+  * Weights: the gate and up projections (with the RMSNorm gain folded in and rounded to bf16
+    first, as the bf16 path stores them) are quantized per output channel:
+    s = max|w_row| / 448 in fp32 (1 for an all-zero row), q = E4M3(fp32(w / s)).
+  * Activations: every sub-layer row x (width W, the input of the RMSNorm) is quantized on its
+    own: s_a = max|x| / 448 in fp32 (1 for an all-zero row), q_a = E4M3(fp32(x / s_a)).
+  * GEMM1 runs on the quantized operands: gate_n = (q_a . q_gate_n) * s_a * s_gate_n / rms(x),
+    up_n likewise, with rms taken over the unquantized row exactly as in the bf16 path.  The
+    SwiGLU, the down projection and the residual are those of the bf16 path (the down
+    projection keeps its bf16 weights): GEMM1 carries two thirds of the FFN's flops.
+"""
+from __future__ import annotations
+
+from typing import Callable, Dict, Optional, Tuple
+
+import numpy as np
+
+from .tokenmixer import mix, revert, round_bf16, silu, storage_round
+
+E4M3_MAX = 448.0
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """fp32 values -> E4M3 codes (uint8), nearest with ties to even, saturating at +-448.
+
+    Rounding is done on |v| against the step of its binade: 2^(e-3) for normal values with
+    2^e <= |v| < 2^(e+1), e >= -6, and 2^-9 below 2^-6 (the subnormal spacing, which equals
+    the step of the lowest normal binade).  Codes are monotonic in |v|, so a magnitude that
+    rounds up to the next binade gets the right code from the same formula.
+    """
+    v = np.asarray(v, dtype=np.float32).astype(np.float64)
+    if np.isnan(v).any():
+        raise ValueError("NaN has no place in the quantized operands")
+    sign = np.signbit(v)
+    a = np.minimum(np.abs(v), E4M3_MAX)
+    _, ex = np.frexp(a)                                   # a = f * 2^ex, f in [0.5, 1)
+    e = np.maximum(ex - 1, -6)                            # binade exponent, floored at the lowest normal
+    step = np.ldexp(1.0, e - 3)
+    q = np.rint(a / step) * step                          # round half to even on the step grid
+    q = np.minimum(q, E4M3_MAX)
+    # encode the (exactly representable) magnitude q
+    _, qex = np.frexp(q)
+    qe = qex - 1
+    normal = q >= 2.0 ** -6
+    exp_field = np.where(normal, qe + 7, 0)
+    mant = np.where(normal, q / np.ldexp(1.0, qe) - 1.0, q / 2.0 ** -9) * np.where(normal, 8.0, 1.0)
+    code = (exp_field.astype(np.int64) << 3) | np.rint(mant).astype(np.int64)
+    code = np.where(q == 0, 0, code)
+    return (code | (sign.astype(np.int64) << 7)).astype(np.uint8)
+
+
+def e4m3_decode(code: np.ndarray) -> np.ndarray:
+    """E4M3 codes -> float64 values (NaN for the two NaN patterns)."""
+    c = np.asarray(code, dtype=np.uint8).astype(np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.ldexp(1.0, e - 7))
+    val = np.where((c & 0x7F) == 0x7F, np.nan, val)
+    return s * val
+
+
+def quantize_rows(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-row E4M3 quantization of a [R, K] array whose values are fp32-representable.
+
+    Returns (codes [R, K] uint8, scales [R] float32) with scale = max|row| / 448 in fp32
+    (1 for an all-zero row) and codes = E4M3(fp32(row / scale)).
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.max(np.abs(x32), axis=1)
+    s = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    s = np.where(amax > 0, s, np.float32(1.0)).astype(np.float32)
+    return e4m3_encode((x32 / s[:, None]).astype(np.float32)), s
+
+
+def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    return e4m3_decode(codes) * np.asarray(scales, dtype=np.float64)[:, None]
+
+
+def fold_gain(w: np.ndarray, gain: Optional[np.ndarray]) -> np.ndarray:
+    """The stored gate / up weights of a sub-layer with a norm gain: bf16(w * gain) per input column."""
+    return w if gain is None else round_bf16(w * gain[None, :])
+
+
+def quantize_bank(bw: Dict[str, np.ndarray], gain: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+    """E4M3 gate / up weights of one dense bank (per output channel), bf16 down weights kept."""
+    qg, sg = quantize_rows(fold_gain(bw["w_gate"], gain))
+    qu, su = quantize_rows(fold_gain(bw["w_up"], gain))
+    return {"q_gate": qg, "s_gate": sg, "q_up": qu, "s_up": su, "w_down": bw["w_down"]}
+
+
+def swiglu_fp8(rows: np.ndarray, qb: Dict[str, np.ndarray], eps: float) -> np.ndarray:
+    """FFN of one bank on the FP8 path, without the residual: rows [R, W] -> [R, W].
+
+    gate = (q_a . q_gate) * s_a * s_gate / rms(x), up likewise; silu(gate) * up; then the bf16
+    down projection.
+    """
+    ca, sa = quantize_rows(rows)
+    a = e4m3_decode(ca)                                   # [R, W] quantized row values / s_a
+    inv = 1.0 / np.sqrt(np.mean(rows * rows, axis=1) + eps)
+    rs = sa.astype(np.float64) * inv                      # per-row factor
+    g = (a @ e4m3_decode(qb["q_gate"]).T) * rs[:, None] * qb["s_gate"].astype(np.float64)[None, :]
+    u = (a @ e4m3_decode(qb["q_up"]).T) * rs[:, None] * qb["s_up"].astype(np.float64)[None, :]
+    return (silu(g) * u) @ qb["w_down"].T
+
+
+def sublayer_fp8(rows: np.ndarray, qbank: Callable[[int], Dict[str, np.ndarray]], eps: float) -> np.ndarray:
+    """rows [R, banks, W] -> FFN output [R, banks, W] (no residual), bank j with its own weights."""
+    out = np.empty_like(rows)
+    for j in range(rows.shape[1]):
+        out[:, j, :] = swiglu_fp8(rows[:, j, :], qbank(j), eps)
+    return out
+
+
+def block_forward_fp8(X: np.ndarray, cfg, qbank: Callable[[int, int], Dict[str, np.ndarray]],
+                      storage=None) -> Dict[str, np.ndarray]:
+    """A dense block on the FP8 path: the bf16 block with each sub-layer's GEMM1 quantized.
+
+    qbank(sub, j) gives the quantized weights of bank j of sub-layer sub (0 mixing, 1 reverting).
+    X_rev and the output are the stored tensors `storage` rounds, as in the bf16 block.
+    """
+    rnd = storage_round(storage)
+    Hm = mix(X, cfg.H)
+    Hn = sublayer_fp8(Hm, lambda j: qbank(0, j), cfg.eps) + Hm
+    Xr = rnd(revert(Hn, cfg.T))
+    Xn = sublayer_fp8(Xr, lambda j: qbank(1, j), cfg.eps) + X
+    return {"Hm": Hm, "Xr": Xr, "Y": rnd(Xn)}

@@ -1,0 +1,102 @@
+"""Pins of the FP8 E4M3 serving oracle (oracle/fp8.py) against things other than itself:
+PyTorch's float8_e4m3fn conversion (a library routine), the code table's closed forms, the
+rounding bound of a 3-bit mantissa, and the special case in which quantization is exact, where
+the FP8 FFN must equal the bf16 oracle's FFN.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import fp8 as F
+from oracle import tokenmixer as O
+
+
+def torch_codes(x):
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_codec_matches_torch_float8_conversion():
+    rng = np.random.default_rng(0)
+    parts = [
+        rng.standard_normal(20000).astype(np.float32) * 30,          # the normal range
+        rng.uniform(-2.0 ** -6, 2.0 ** -6, 20000).astype(np.float32),  # subnormals
+        rng.uniform(-448, 448, 20000).astype(np.float32),
+    ]
+    # exact ties between neighbouring codes in every binade (and the subnormal spacing)
+    vals = F.e4m3_decode(np.arange(0, 0x7E, dtype=np.uint8))
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    parts += [mids, -mids, np.float32([0.0, -0.0, 448.0, -448.0, 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -11])]
+    x = np.concatenate(parts)
+    assert np.array_equal(F.e4m3_encode(x), torch_codes(x))
+
+
+def test_code_table_closed_forms():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    assert np.array_equal(F.e4m3_encode(F.e4m3_decode(codes).astype(np.float32)), codes)
+    e = F.e4m3_encode(np.float32([448.0, 2.0 ** -9, 2.0 ** -6, 1.0, 1.0 + 1 / 16, 1.0 + 3 / 16, 1000.0, -1000.0,
+                                  2.0 ** -10, 1.5 * 2.0 ** -9]))
+    # 448 = 1.75*2^8 -> exponent field 15, mantissa 6; the smallest subnormal; the smallest normal;
+    # 1.0; ties go to the even mantissa (1.0 and 1.25); saturation; half the smallest subnormal is a
+    # tie that rounds to zero (even), 1.5 of it rounds up to 2 subnormal steps
+    assert list(e) == [0x7E, 0x01, 0x08, 0x38, 0x38, 0x3A, 0x7E, 0xFE, 0x00, 0x02]
+    assert F.e4m3_decode(np.uint8([0x7E]))[0] == 448.0
+    assert np.isnan(F.e4m3_decode(np.uint8([0x7F, 0xFF]))).all()
+
+
+def test_row_quantization_bounds():
+    rng = np.random.default_rng(1)
+    x = (rng.standard_normal((64, 256)) * rng.uniform(0.01, 100, (64, 1))).astype(np.float32)
+    x[3] = 0.0
+    codes, s = F.quantize_rows(x)
+    assert s.dtype == np.float32 and s[3] == 1.0
+    q = F.e4m3_decode(codes)
+    nz = np.arange(64) != 3
+    assert np.all(np.max(np.abs(q[nz]), axis=1) == 448.0)     # the largest element lands on the top code
+    err = np.abs(q * s[:, None].astype(np.float64) - x)
+    # half a step of a 3-bit mantissa (2^-4 relative) in the normal range, half the subnormal
+    # spacing (2^-10 * s) below it
+    bound = np.maximum(2.0 ** -4 * np.abs(x), 2.0 ** -10 * s[:, None])
+    assert np.all(err <= bound * (1 + 1e-6))
+
+
+def test_fp8_ffn_equals_bf16_ffn_when_quantization_is_exact():
+    # rows and weights already on the E4M3 grid, each row's largest magnitude exactly 448 * 2^k:
+    # the per-row scale is a power of two, x / s is exact and every code reproduces its value
+    rng = np.random.default_rng(2)
+    W, Fh, R = 64, 96, 24
+
+    def grid_rows(n, k, scale_pow):
+        c = rng.integers(0, 0x7E, (n, k)).astype(np.uint8) | (rng.integers(0, 2, (n, k)).astype(np.uint8) << 7)
+        c[:, 0] = 0x7E                                      # +448 in every row
+        return F.e4m3_decode(c) * 2.0 ** scale_pow
+    x = grid_rows(R, W, -6)
+    bw = {"w_gate": grid_rows(Fh, W, -12), "w_up": grid_rows(Fh, W, -12),
+          "w_down": O.round_bf16(rng.standard_normal((W, Fh)) * 0.05)}
+    qb = F.quantize_bank(bw)
+    assert np.array_equal(F.dequantize_rows(qb["q_gate"], qb["s_gate"]), bw["w_gate"])
+    eps = 1e-6
+    got = F.swiglu_fp8(x, qb, eps)
+    want = O.swiglu(O.rmsnorm(x, eps), bw["w_gate"], bw["w_up"], bw["w_down"])
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+
+
+def test_fp8_ffn_tracks_bf16_ffn_within_the_quantization_error():
+    # generic inputs: the FP8 FFN is the bf16 FFN up to the E4M3 rounding of both GEMM1 operands
+    rng = np.random.default_rng(3)
+    W, Fh, R = 128, 256, 64
+    x = O.round_bf16(rng.standard_normal((R, W)))
+    bw = {k: O.round_bf16(rng.standard_normal(shape) / np.sqrt(shape[1]))
+          for k, shape in (("w_gate", (Fh, W)), ("w_up", (Fh, W)), ("w_down", (W, Fh)))}
+    got = F.swiglu_fp8(x, F.quantize_bank(bw), 1e-6)
+    want = O.swiglu(O.rmsnorm(x, 1e-6), bw["w_gate"], bw["w_up"], bw["w_down"])
+    rel = np.sqrt(np.mean((got - want) ** 2) / np.mean(want ** 2))
+    assert 1e-3 < rel < 0.08, rel
+
+
+def test_gain_is_folded_then_quantized():
+    rng = np.random.default_rng(4)
+    w = O.round_bf16(rng.standard_normal((8, 32)))
+    g = O.round_bf16(1 + 0.1 * rng.standard_normal(32))
+    qb = F.quantize_bank({"w_gate": w, "w_up": w, "w_down": w.T}, g)
+    c, s = F.quantize_rows(O.round_bf16(w * g[None, :]))
+    assert np.array_equal(qb["q_gate"], c) and np.array_equal(qb["s_gate"], s)
