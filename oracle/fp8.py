@@ -11,12 +11,15 @@ quantization of a model trained in bf16.  The page names the format only; the re
     normal values 2^(e-7) * (1 + m/8) for exponent fields e = 1..15, subnormals m * 2^-9 for
     e = 0, largest finite 448 (the all-ones pattern S.1111.111 is NaN; there are no
     infinities).  Conversion rounds to nearest with ties to even and saturates at +-448.
-  * Weights: the gate and up projections (with the RMSNorm gain folded in and rounded to bf16
-    first, as the bf16 path stores them) are quantized per output channel:
-    s = max|w_row| / 448 in fp32 (1 for an all-zero row), q = E4M3(fp32(w / s)).
+  * Weights: the gate and up projections of each bank (with the RMSNorm gain folded in and
+    rounded to bf16 first, as the bf16 path stores them) are quantized per matrix, one scale per
+    bank: s = max|W| / 448 in fp32 (1 for an all-zero matrix), q = E4M3(fp32(w / s)).  E4M3 is a
+    floating-point format: every value inside its normal range (2^-6 .. 448 times s) keeps a 3-bit
+    mantissa whatever the scale, so per-row scales would change nothing for rows whose magnitudes
+    sit within that 2^15 range of the matrix maximum, as these projections' rows do.
   * Activations: every sub-layer row x (width W, the input of the RMSNorm) is quantized on its
     own: s_a = max|x| / 448 in fp32 (1 for an all-zero row), q_a = E4M3(fp32(x / s_a)).
-  * GEMM1 runs on the quantized operands: gate_n = (q_a . q_gate_n) * s_a * s_gate_n / rms(x),
+  * GEMM1 runs on the quantized operands: gate_n = (q_a . q_gate_n) * s_a * s_gate / rms(x),
     up_n likewise, with rms taken over the unquantized row exactly as in the bf16 path.  The
     SwiGLU, the down projection and the residual are those of the bf16 path (the down
     projection keeps its bf16 weights): GEMM1 carries two thirds of the FFN's flops.
@@ -89,15 +92,23 @@ def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     return e4m3_decode(codes) * np.asarray(scales, dtype=np.float64)[:, None]
 
 
+def quantize_matrix(w: np.ndarray) -> Tuple[np.ndarray, np.float32]:
+    """E4M3 quantization of a whole matrix with one scale: max|w| / 448 in fp32 (1 if all zero)."""
+    w32 = np.asarray(w, dtype=np.float32)
+    amax = np.float32(np.max(np.abs(w32))) if w32.size else np.float32(0)
+    s = np.float32(amax / np.float32(E4M3_MAX)) if amax > 0 else np.float32(1.0)
+    return e4m3_encode((w32 / s).astype(np.float32)), s
+
+
 def fold_gain(w: np.ndarray, gain: Optional[np.ndarray]) -> np.ndarray:
     """The stored gate / up weights of a sub-layer with a norm gain: bf16(w * gain) per input column."""
     return w if gain is None else round_bf16(w * gain[None, :])
 
 
 def quantize_bank(bw: Dict[str, np.ndarray], gain: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
-    """E4M3 gate / up weights of one dense bank (per output channel), bf16 down weights kept."""
-    qg, sg = quantize_rows(fold_gain(bw["w_gate"], gain))
-    qu, su = quantize_rows(fold_gain(bw["w_up"], gain))
+    """E4M3 gate / up weights of one dense bank (one scale per matrix), bf16 down weights kept."""
+    qg, sg = quantize_matrix(fold_gain(bw["w_gate"], gain))
+    qu, su = quantize_matrix(fold_gain(bw["w_up"], gain))
     return {"q_gate": qg, "s_gate": sg, "q_up": qu, "s_up": su, "w_down": bw["w_down"]}
 
 
@@ -105,14 +116,14 @@ def swiglu_fp8(rows: np.ndarray, qb: Dict[str, np.ndarray], eps: float) -> np.nd
     """FFN of one bank on the FP8 path, without the residual: rows [R, W] -> [R, W].
 
     gate = (q_a . q_gate) * s_a * s_gate / rms(x), up likewise; silu(gate) * up; then the bf16
-    down projection.
+    down projection.  s_gate, s_up: the bank's matrix scales.
     """
     ca, sa = quantize_rows(rows)
     a = e4m3_decode(ca)                                   # [R, W] quantized row values / s_a
     inv = 1.0 / np.sqrt(np.mean(rows * rows, axis=1) + eps)
     rs = sa.astype(np.float64) * inv                      # per-row factor
-    g = (a @ e4m3_decode(qb["q_gate"]).T) * rs[:, None] * qb["s_gate"].astype(np.float64)[None, :]
-    u = (a @ e4m3_decode(qb["q_up"]).T) * rs[:, None] * qb["s_up"].astype(np.float64)[None, :]
+    g = (a @ e4m3_decode(qb["q_gate"]).T) * (rs * np.float64(qb["s_gate"]))[:, None]
+    u = (a @ e4m3_decode(qb["q_up"]).T) * (rs * np.float64(qb["s_up"]))[:, None]
     return (silu(g) * u) @ qb["w_down"].T
 
 

@@ -60,8 +60,9 @@ def test_row_quantization_bounds():
 
 
 def test_fp8_ffn_equals_bf16_ffn_when_quantization_is_exact():
-    # rows and weights already on the E4M3 grid, each row's largest magnitude exactly 448 * 2^k:
-    # the per-row scale is a power of two, x / s is exact and every code reproduces its value
+    # rows and weights already on the E4M3 grid, each row's (and each weight matrix's) largest
+    # magnitude exactly 448 * 2^k: the scales are powers of two, x / s is exact and every code
+    # reproduces its value
     rng = np.random.default_rng(2)
     W, Fh, R = 64, 96, 24
 
@@ -73,7 +74,8 @@ def test_fp8_ffn_equals_bf16_ffn_when_quantization_is_exact():
     bw = {"w_gate": grid_rows(Fh, W, -12), "w_up": grid_rows(Fh, W, -12),
           "w_down": O.round_bf16(rng.standard_normal((W, Fh)) * 0.05)}
     qb = F.quantize_bank(bw)
-    assert np.array_equal(F.dequantize_rows(qb["q_gate"], qb["s_gate"]), bw["w_gate"])
+    assert qb["s_gate"] == np.float32(2.0 ** -12)
+    assert np.array_equal(F.e4m3_decode(qb["q_gate"]) * np.float64(qb["s_gate"]), bw["w_gate"])
     eps = 1e-6
     got = F.swiglu_fp8(x, qb, eps)
     want = O.swiglu(O.rmsnorm(x, eps), bw["w_gate"], bw["w_up"], bw["w_down"])
@@ -98,5 +100,19 @@ def test_gain_is_folded_then_quantized():
     w = O.round_bf16(rng.standard_normal((8, 32)))
     g = O.round_bf16(1 + 0.1 * rng.standard_normal(32))
     qb = F.quantize_bank({"w_gate": w, "w_up": w, "w_down": w.T}, g)
-    c, s = F.quantize_rows(O.round_bf16(w * g[None, :]))
-    assert np.array_equal(qb["q_gate"], c) and np.array_equal(qb["s_gate"], s)
+    c, s = F.quantize_matrix(O.round_bf16(w * g[None, :]))
+    assert np.array_equal(qb["q_gate"], c) and qb["s_gate"] == s
+
+
+def test_matrix_scale_is_the_matrix_maximum():
+    rng = np.random.default_rng(5)
+    w = (rng.standard_normal((16, 40)) * rng.uniform(0.1, 10, (16, 1))).astype(np.float32)
+    codes, s = F.quantize_matrix(w)
+    assert s == np.float32(np.max(np.abs(w)) / np.float32(448))
+    q = F.e4m3_decode(codes)
+    assert np.max(np.abs(q)) == 448.0
+    # every value above the subnormal range keeps the 2^-4 relative rounding bound, whatever its row
+    big = np.abs(w) >= 2.0 ** -6 * s
+    assert np.all(np.abs(q * np.float64(s) - w)[big] <= 2.0 ** -4 * np.abs(w)[big] * (1 + 1e-6))
+    assert np.array_equal(F.quantize_matrix(np.zeros((3, 4)))[0], np.zeros((3, 4), np.uint8))
+    assert F.quantize_matrix(np.zeros((3, 4)))[1] == 1.0
