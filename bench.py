@@ -88,6 +88,22 @@ def kernel_flops(cfg, B) -> dict:
     return out
 
 
+def kernel_flops_fp8(cfg, B) -> dict:
+    """The FP8 path: both sub-layers of every block run the fused kernel in its FP8 mode."""
+    f = 0.0
+    for _ in range(cfg.L):
+        for sub in (0, 1):
+            f += B * cfg.banks(sub) * 6.0 * cfg.width(sub) * cfg.ffn(sub).hidden
+    return {"fused_swiglu_fp8": f}
+
+
+def fp8_effective_peak(bf16_peak: float) -> float:
+    """Tensor peak of the FP8 kernel's mix of work: GEMM1 (4 W F flops per row) at the E4M3 rate,
+    taken as the measured bf16 peak x 2 (the nominal 4.5 / 2.25 PFLOP/s ratio), GEMM2 (2 W F) at
+    the bf16 rate: 6 / (4 / 2P + 2 / P) = 1.5 P."""
+    return 6.0 / (4.0 / (2.0 * bf16_peak) + 2.0 / bf16_peak)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -201,6 +217,29 @@ def time_oracle(cfg, budget_s: float, max_samples: int):
     return done / dt, {"cores": int(threads), "samples": done, "seconds": dt, "per_call": n}
 
 
+def time_oracle_fp8(cfg, budget_s: float, max_samples: int):
+    """The FP8 oracle's samples/s on the host cores (weights quantized beforehand, as served)."""
+    import oracle
+    from oracle import fp8 as F
+    from threadpoolctl import threadpool_info
+    get = oracle.synth_banks(cfg)
+    q = {(l, sub, j): F.quantize_bank(get(l, sub, j)) for l in range(cfg.L) for sub in (0, 1)
+         for j in range(cfg.banks(sub))}
+    n = min(max_samples, cfg.B)
+    X = S.to_f64(S.make_x(cfg, np.arange(n)))
+    done, t0 = 0, time.perf_counter()
+    while True:
+        Y = X
+        for l in range(cfg.L):
+            Y = F.block_forward_fp8(Y, cfg, lambda sub, j: q[(l, sub, j)])["Y"]
+        done += n
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return done / dt, {"cores": int(threads), "samples": done, "seconds": dt, "per_call": n}
+
+
 def run_reference(args, cfg, rank):
     if rank != 0:
         return
@@ -271,7 +310,12 @@ def run_ours(args, cfg, rank, world, local_rank):
     stream = torch.cuda.Stream(device=dev)
     blocks = api.blocks_from_synth(cfg, dev, workers=min(16, os.cpu_count() or 1))
     sh = api.config_shape(cfg)
-    run = api.StackRunner(blocks, sh, cfg.gap, dev)
+    if args.fp8:
+        if cfg.gap or cfg.dtype != "bf16" or any(cfg.ffn(sub).is_moe for sub in (0, 1)):
+            raise SystemExit("--fp8 covers bf16 dense blocks without the inter-residual")
+        run = api.Fp8BlockRunner([api.Block8.from_bf16(b) for b in blocks], sh, dev)
+    else:
+        run = api.StackRunner(blocks, sh, cfg.gap, dev)
     X = api.to_device(S.make_x(rank_config(cfg, rank)), dev)
     Y = torch.empty_like(X)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -336,31 +380,40 @@ def run_ours(args, cfg, rank, world, local_rank):
     # dominant kernel: largest share of device time in the timed region
     dom = max(kern.items(), key=lambda kv: kv[1]["total_ms"]) if kern else (None, None)
     roof = None
-    kf = kernel_flops(cfg, cfg.B)
+    kf = kernel_flops_fp8(cfg, cfg.B) if args.fp8 else kernel_flops(cfg, cfg.B)
     if dom[0] in kf:
         per_launch = kf[dom[0]] / (dom[1]["launches"] / K)
         avg_ms = dom[1]["total_ms"] / dom[1]["launches"]
         ach = per_launch / (avg_ms / 1e3) / 1e12
         tr = traffic_for(dom[0], cfg.name)
-        roof = {"kernel": dom[0], "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"], "traffic": tr,
-                "peak_source": ("measured bf16 burst (MEASURED_PEAKS.json bf16_tflops)" if pk_src == "measured"
-                                else "fallback 1.59 PFLOP/s"),
+        src = ("measured bf16 burst (MEASURED_PEAKS.json bf16_tflops)" if pk_src == "measured"
+               else "fallback 1.59 PFLOP/s")
+        peak = pk["bf16_tflops"]
+        if args.fp8:
+            peak = fp8_effective_peak(pk["bf16_tflops"])
+            src = ("GEMM1 at 2 x, GEMM2 at 1 x the " + src + ": 1.5 x the bf16 peak for the kernel's "
+                   "2:1 split of flops")
+        roof = {"kernel": dom[0], "bound": "tensor", "achieved": ach, "peak": peak,
+                "unit": "TFLOP/s", "frac": ach / peak, "traffic": tr, "peak_source": src,
                 "flops_per_launch": per_launch, "avg_launch_ms": avg_ms}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        v, info = time_oracle(cfg, args.cpu_seconds, args.cpu_samples)
+        v, info = (time_oracle_fp8 if args.fp8 else time_oracle)(cfg, args.cpu_seconds, args.cpu_samples)
         cpu = {"value": v, "unit": "samples/s", "cores": info["cores"], "kind": "oracle",
                "sample": f"{info['samples']} samples ({info['per_call']} per oracle call) of {cfg.name}, "
                          f"{info['seconds']:.1f} s of host time"}
     line = {
         "metric": METRIC, "value": value, "unit": "samples/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded normal inputs, random-init weights of the workload's shapes)",
+        "dtype": "e4m3+bf16" if args.fp8 else "bf16",
+        "data": "synthetic (seeded normal inputs, random-init weights of the workload's shapes)",
         "config": {"workload": describe(cfg), "global_batch": total_samples, "seq_len": cfg.T,
                    "parallelism": f"dp{world} (independent batches, no data-path collective)",
-                   "l2": "flushed by a 256 MB write between timed steps (outside the step events)"},
-        "tflops": tflops, "tc_roofline_frac": tflops / pk["bf16_tflops"],
+                   "l2": "flushed by a 256 MB write between timed steps (outside the step events)",
+                   **({"precision": "FP8 serving path: GEMM1 (gate, up) on E4M3 operands, per-channel weight and "
+                                    "per-row activation scales; GEMM2 and residual bf16"} if args.fp8 else {})},
+        "tflops": tflops,
+        "tc_roofline_frac": tflops / (fp8_effective_peak(pk["bf16_tflops"]) if args.fp8 else pk["bf16_tflops"]),
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(cfg.B, world, e2e_ms), "unit": "samples/s", "h2d_bytes_per_step": io_bytes,
@@ -389,6 +442,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-samples", type=int, default=128)
     ap.add_argument("--steps-ref", type=int, default=None)
+    ap.add_argument("--fp8", action="store_true",
+                    help="the FP8 E4M3 serving path (dense blocks): its own line, not the bf16 metric's")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -201,6 +201,65 @@ TM_API tm_status tm_stack_forward(const void *X, const tm_block *blocks, int L, 
                            const tm_shape *shape, void *Y, void *workspace, size_t workspace_bytes,
                            void *stream);
 
+/* ---- FP8 E4M3 serving path of the dense per-token FFN ----------------------------------
+ * [digest] 2.5.2 (FP8 quantization): serving runs on FP8 E4M3 post-training quantization of a
+ * model trained in bf16.  The page names the format only; this library's reading: GEMM1 (the
+ * gate and up projections, two thirds of the FFN's flops) runs on E4M3 operands on the tensor
+ * cores (kind::f8f6f4) with each bank's gate/up matrix quantized with one scale and every
+ * activation row quantized on its own; the SwiGLU, GEMM2 (down, bf16 weights) and the residual
+ * stay as in the bf16 path (fp32 accumulation, bf16 storage).  E4M3: 1 sign bit, 4 exponent
+ * bits of bias 7, 3 mantissa bits, largest finite 448; conversions round to nearest-even and
+ * saturate.  bf16 activations only; row widths 128 and 256 (the fused sub-layer kernel);
+ * hidden widths multiples of 128; mixed rows need a head width that is a multiple of 16.
+ * Unsupported shapes return TM_ERR_UNSUPPORTED before any launch. */
+
+/* E4M3 quantization of `groups` bf16 weight matrices w [groups, rows, cols] with one scale per
+ * matrix (a bank's gate or up projection), optionally times a per-column gain [cols]
+ * (multiplied and rounded to bf16 first, as the bf16 path folds the RMSNorm gain):
+ * scale[g] = max|matrix g| / 448 (1 for an all-zero matrix); q [groups, rows, cols] =
+ * E4M3(w / scale[g]) with IEEE fp32 division.  rows * cols even.  q (1-byte codes) and scale are
+ * device memory.  E4M3 keeps a 3-bit mantissa for every value inside its normal range
+ * (2^-6 .. 448 times the scale), so one scale serves all rows of a projection. */
+TM_API tm_status tm_quantize_fp8_weights(const void *w, const void *gain, int groups, size_t rows, int cols,
+                                         uint8_t *q, float *scale, void *stream);
+
+/* Per-row E4M3 quantization of a sub-layer's bf16 activation rows (banks, width as for the
+ * sub-layer, read through `layout`): q [B*banks, width] (row b*banks + bank) = E4M3(row / s)
+ * with s = max|row| / 448 (1 for an all-zero row), and rowscale [B*banks] = s / rms(row),
+ * rms = sqrt(mean(row^2) + eps) over the unquantized row. */
+TM_API tm_status tm_quantize_fp8_act(const void *x, tm_layout layout, const tm_shape *shape, int banks, int width,
+                                     uint8_t *q, float *rowscale, void *stream);
+
+/* A dense bank on the FP8 path: q_gate, q_up [banks, hidden, width] E4M3 codes with s_gate,
+ * s_up [banks] fp32 scales (one per bank matrix, the RMSNorm gain already folded in, as
+ * tm_quantize_fp8_weights makes them); w_down bf16 [banks, width, hidden]. */
+typedef struct {
+    int banks, width, hidden;
+    const uint8_t *q_gate, *q_up;
+    const float *s_gate, *s_up;
+    const void *w_down;
+} tm_swiglu_w8;
+
+/* A dense block on the FP8 path: mixing (banks = H, width = T*D/H) and reverting (banks = T,
+ * width = D) sub-layers. */
+typedef struct { tm_swiglu_w8 mix, rev; } tm_block_fp8;
+
+TM_API size_t tm_pertoken_swiglu_fp8_workspace_bytes(const tm_shape *shape, tm_layout layout, const tm_swiglu_w8 *w);
+
+/* Dense sub-layer on the FP8 path:  y_row = SwiGLU_bank(RMSNorm(x_row)) + residual_row, GEMM1 on
+ * E4M3 operands: gate_n = (q_row . q_gate_n) * rowscale * s_gate, up likewise (the activation
+ * rows are quantized into the workspace first).  residual may be NULL; y must not alias x. */
+TM_API tm_status tm_pertoken_swiglu_fp8(const void *x, const void *residual, tm_layout layout, const tm_shape *shape,
+                                        const tm_swiglu_w8 *w, void *y, void *workspace, size_t workspace_bytes,
+                                        void *stream);
+
+TM_API size_t tm_block_fp8_workspace_bytes(const tm_shape *shape, const tm_block_fp8 *block);
+
+/* One dense block as tm_block_forward, both sub-layers on the FP8 path.  X, Y [B,T,D];
+ * X_revert_opt [B,T,D] receives X_rev when not NULL. */
+TM_API tm_status tm_block_forward_fp8(const void *X, const tm_block_fp8 *block, const tm_shape *shape, void *Y,
+                                      void *X_revert_opt, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Per-kernel timing of the library's own launches (tracing). */
 typedef struct {
     char name[48];       /* kernel family, e.g. "gemm_swiglu" */

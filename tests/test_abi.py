@@ -47,6 +47,8 @@ int main(void) {
          sizeof(tm_shape), sizeof(tm_swiglu_w), sizeof(tm_moe_w), sizeof(tm_sublayer), sizeof(tm_block));
   P(tm_shape, eps) P(tm_swiglu_w, w_gate) P(tm_swiglu_w, w_down) P(tm_moe_w, alpha) P(tm_moe_w, w_router)
   P(tm_moe_w, ws_down) P(tm_sublayer, dense) P(tm_sublayer, moe) P(tm_block, rev)
+  printf("tm_swiglu_w8 %zu\ntm_block_fp8 %zu\n", sizeof(tm_swiglu_w8), sizeof(tm_block_fp8));
+  P(tm_swiglu_w8, q_gate) P(tm_swiglu_w8, s_up) P(tm_swiglu_w8, w_down) P(tm_block_fp8, rev)
   return 0;
 }
 ''')
@@ -62,6 +64,9 @@ int main(void) {
         "tm_moe_w.w_router": A.tm_moe_w.w_router.offset, "tm_moe_w.ws_down": A.tm_moe_w.ws_down.offset,
         "tm_sublayer.dense": A.tm_sublayer.dense.offset, "tm_sublayer.moe": A.tm_sublayer.moe.offset,
         "tm_block.rev": A.tm_block.rev.offset,
+        "tm_swiglu_w8": ctypes.sizeof(A.tm_swiglu_w8), "tm_block_fp8": ctypes.sizeof(A.tm_block_fp8),
+        "tm_swiglu_w8.q_gate": A.tm_swiglu_w8.q_gate.offset, "tm_swiglu_w8.s_up": A.tm_swiglu_w8.s_up.offset,
+        "tm_swiglu_w8.w_down": A.tm_swiglu_w8.w_down.offset, "tm_block_fp8.rev": A.tm_block_fp8.rev.offset,
     }
     assert {k: int(v) for k, v in got.items()} == want
 

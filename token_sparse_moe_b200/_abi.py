@@ -17,7 +17,9 @@ EXPORTS = ["tm_status_string", "tm_version", "tm_sublayer_workspace_bytes", "tm_
            "tm_workspace_bytes", "tm_tokenize_stub", "tm_mix", "tm_revert", "tm_route_topk", "tm_route_topk_noalloc",
            "tm_pertoken_swiglu", "tm_sparse_pertoken_moe", "tm_block_forward", "tm_stack_forward",
            "tm_profile_start", "tm_profile_stop", "tm_last_cuda_error", "tm_launch_count",
-           "tm_get_device_error"]
+           "tm_get_device_error", "tm_quantize_fp8_weights", "tm_quantize_fp8_act",
+           "tm_pertoken_swiglu_fp8_workspace_bytes", "tm_pertoken_swiglu_fp8", "tm_block_fp8_workspace_bytes",
+           "tm_block_forward_fp8"]
 
 
 class tm_shape(ctypes.Structure):
@@ -42,6 +44,15 @@ class tm_sublayer(ctypes.Structure):
 
 class tm_block(ctypes.Structure):
     _fields_ = [("mix", tm_sublayer), ("rev", tm_sublayer)]
+
+
+class tm_swiglu_w8(ctypes.Structure):
+    _fields_ = [("banks", c_int), ("width", c_int), ("hidden", c_int), ("q_gate", c_void_p), ("q_up", c_void_p),
+                ("s_gate", c_void_p), ("s_up", c_void_p), ("w_down", c_void_p)]
+
+
+class tm_block_fp8(ctypes.Structure):
+    _fields_ = [("mix", tm_swiglu_w8), ("rev", tm_swiglu_w8)]
 
 
 class tm_kernel_time(ctypes.Structure):
@@ -71,6 +82,12 @@ _SIGS = {
     "tm_last_cuda_error": (ctypes.c_char_p, []),
     "tm_launch_count": (ctypes.c_ulonglong, []),
     "tm_get_device_error": (c_int, [_P]),
+    "tm_quantize_fp8_weights": (c_int, [_P, _P, c_int, c_size_t, c_int, _P, _P, _P]),
+    "tm_quantize_fp8_act": (c_int, [_P, c_int, POINTER(tm_shape), c_int, c_int, _P, _P, _P]),
+    "tm_pertoken_swiglu_fp8_workspace_bytes": (c_size_t, [POINTER(tm_shape), c_int, POINTER(tm_swiglu_w8)]),
+    "tm_pertoken_swiglu_fp8": (c_int, [_P, _P, c_int, POINTER(tm_shape), POINTER(tm_swiglu_w8), _P, _P, c_size_t, _P]),
+    "tm_block_fp8_workspace_bytes": (c_size_t, [POINTER(tm_shape), POINTER(tm_block_fp8)]),
+    "tm_block_forward_fp8": (c_int, [_P, POINTER(tm_block_fp8), POINTER(tm_shape), _P, _P, _P, c_size_t, _P]),
 }
 
 _lib = None

@@ -275,6 +275,129 @@ def stack_forward(X, blocks: Sequence[Block], gap: int, sh: A.tm_shape, Y=None, 
     return StackRunner(blocks, sh, gap, X.device)(X, Y, stream)
 
 
+# ------------------------------------------------------------------ FP8 E4M3 serving path
+def quantize_fp8_weights(w: torch.Tensor, gain: Optional[torch.Tensor] = None, stream=None):
+    """tm_quantize_fp8_weights: bf16 [groups, rows, cols] matrices -> (E4M3 codes as uint8 of the
+    same shape, fp32 scales [groups], one per matrix)."""
+    groups, rows, cols = w.shape
+    q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    s = torch.empty((groups,), dtype=torch.float32, device=w.device)
+    A.check(lib().tm_quantize_fp8_weights(_p(w), _p(gain), groups, rows, cols, _p(q), _p(s), _s(stream)),
+            "tm_quantize_fp8_weights")
+    return q, s
+
+
+def quantize_fp8_act(x: torch.Tensor, layout: int, sh: A.tm_shape, banks: int, width: int, stream=None):
+    """tm_quantize_fp8_act: the sub-layer's activation rows -> (codes [B*banks, width] uint8,
+    rowscale [B*banks] fp32)."""
+    q = torch.empty((sh.B * banks, width), dtype=torch.uint8, device=x.device)
+    rs = torch.empty((sh.B * banks,), dtype=torch.float32, device=x.device)
+    A.check(lib().tm_quantize_fp8_act(_p(x), layout, ctypes.byref(sh), banks, width, _p(q), _p(rs), _s(stream)),
+            "tm_quantize_fp8_act")
+    return q, rs
+
+
+@dataclass
+class SubLayer8:
+    """A dense sub-layer on the FP8 path: E4M3 gate / up codes with one scale per bank matrix (gain
+    folded in) and the bf16 down weights.  Built from a bf16 SubLayer by the library's own quantizer."""
+    banks: int
+    width: int
+    hidden: int
+    tensors: Dict[str, torch.Tensor]
+
+    @staticmethod
+    def from_bf16(sub: "SubLayer", stream=None) -> "SubLayer8":
+        if sub.is_moe:
+            raise ValueError("the FP8 path covers dense sub-layers")
+        t = sub.tensors
+        qg, sg = quantize_fp8_weights(t["w_gate"], sub.gain, stream)
+        qu, su = quantize_fp8_weights(t["w_up"], sub.gain, stream)
+        return SubLayer8(sub.banks, sub.width, sub.hidden,
+                         {"q_gate": qg, "s_gate": sg, "q_up": qu, "s_up": su, "w_down": t["w_down"]})
+
+    def c(self) -> A.tm_swiglu_w8:
+        t = self.tensors
+        return A.tm_swiglu_w8(self.banks, self.width, self.hidden, _p(t["q_gate"]), _p(t["q_up"]), _p(t["s_gate"]),
+                              _p(t["s_up"]), _p(t["w_down"]))
+
+
+@dataclass
+class Block8:
+    mix: SubLayer8
+    rev: SubLayer8
+
+    @staticmethod
+    def from_bf16(block: "Block", stream=None) -> "Block8":
+        return Block8(SubLayer8.from_bf16(block.mix, stream), SubLayer8.from_bf16(block.rev, stream))
+
+    def c(self) -> A.tm_block_fp8:
+        return A.tm_block_fp8(self.mix.c(), self.rev.c())
+
+
+def pertoken_swiglu_fp8(x, residual, layout: int, sh: A.tm_shape, sub: SubLayer8, y=None, workspace=None, stream=None):
+    if layout == A.TM_LAYOUT_MIXED:
+        y = torch.empty((sh.B, sh.T, sh.D), dtype=x.dtype, device=x.device) if y is None else y
+    else:
+        y = torch.empty((sh.B, sub.banks, sub.width), dtype=x.dtype, device=x.device) if y is None else y
+    w = sub.c()
+    n = lib().tm_pertoken_swiglu_fp8_workspace_bytes(ctypes.byref(sh), layout, ctypes.byref(w))
+    if n == 0:
+        raise A.TMError(A.TM_ERR_UNSUPPORTED, "tm_pertoken_swiglu_fp8_workspace_bytes")
+    ws = _ws(n, x.device, workspace)
+    A.check(lib().tm_pertoken_swiglu_fp8(_p(x), _p(residual), layout, ctypes.byref(sh), ctypes.byref(w), _p(y), _p(ws),
+                                         ws.numel(), _s(stream)), "tm_pertoken_swiglu_fp8")
+    return y
+
+
+def block_fp8_workspace_bytes(sh: A.tm_shape, block: Block8) -> int:
+    c = block.c()
+    n = lib().tm_block_fp8_workspace_bytes(ctypes.byref(sh), ctypes.byref(c))
+    if n == 0:
+        raise A.TMError(A.TM_ERR_UNSUPPORTED, "tm_block_fp8_workspace_bytes")
+    return n
+
+
+def block_forward_fp8(X, block: Block8, sh: A.tm_shape, Y=None, X_revert=None, workspace=None, stream=None):
+    Y = torch.empty_like(X) if Y is None else Y
+    c = block.c()
+    ws = _ws(block_fp8_workspace_bytes(sh, block), X.device, workspace)
+    A.check(lib().tm_block_forward_fp8(_p(X), ctypes.byref(c), ctypes.byref(sh), _p(Y), _p(X_revert), _p(ws),
+                                       ws.numel(), _s(stream)), "tm_block_forward_fp8")
+    return Y
+
+
+class Fp8BlockRunner:
+    """Consecutive dense blocks on the FP8 path (no inter-residual), with a preallocated workspace
+    and ring of intermediate token tensors, so repeated forwards launch with no allocation."""
+
+    def __init__(self, blocks: Sequence[Block8], sh: A.tm_shape, device):
+        self.blocks = list(blocks)
+        self.sh = sh
+        self.cs = [b.c() for b in self.blocks]
+        self.ws = torch.empty(max(block_fp8_workspace_bytes(sh, b) for b in self.blocks), dtype=torch.uint8,
+                              device=device)
+        self.tmp = [torch.empty((sh.B, sh.T, sh.D), dtype=torch.bfloat16, device=device)
+                    for _ in range(min(2, len(self.blocks) - 1))]
+
+    def __call__(self, X: torch.Tensor, Y: torch.Tensor, stream=None) -> torch.Tensor:
+        cur = X
+        for i, c in enumerate(self.cs):
+            out = Y if i == len(self.cs) - 1 else self.tmp[i % 2]
+            A.check(lib().tm_block_forward_fp8(_p(cur), ctypes.byref(c), ctypes.byref(self.sh), _p(out), None,
+                                               _p(self.ws), self.ws.numel(), _s(stream)), "tm_block_forward_fp8")
+            cur = out
+        return Y
+
+    def run_host(self, X_host, Y_host, X_dev, Y_dev, stream=None):
+        s = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(s):
+            X_dev.copy_(X_host, non_blocking=True)
+            self(X_dev, Y_dev, s)
+            Y_host.copy_(Y_dev, non_blocking=True)
+        return Y_host
+
+
 def profile_start() -> None:
     A.check(lib().tm_profile_start(), "tm_profile_start")
 

@@ -63,6 +63,18 @@ bool map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint
     return make_map(m, base, 2, dims, strides, box);
 }
 
+// E4M3 codes (1-byte elements): dims / box innermost first in elements, strides in bytes;
+// 128-byte swizzle with a 128-element inner box.
+bool make_map_u8(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+                 const uint32_t* box) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int num_sms() {
     static int cache[64] = {0};
     int dev = 0;
@@ -635,6 +647,97 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
                        m.slots, w->k, st);
 }
 
+// ------------------------------------------------------------------ FP8 E4M3 dense sub-layer
+tm_status check_dense8(const Geo& g, const tm_swiglu_w8* w) {
+    if (!w || w->banks != g.banks || w->width != g.W || w->hidden <= 0) return TM_ERR_INVALID_ARG;
+    if (!w->q_gate || !w->q_up || !w->s_gate || !w->s_up || !w->w_down) return TM_ERR_INVALID_ARG;
+    if (!al16(w->q_gate) || !al16(w->q_up) || !al16(w->s_gate) || !al16(w->s_up) || !al16(w->w_down))
+        return TM_ERR_INVALID_ARG;
+    if (g.dtype != TM_BF16 || (g.W != 128 && g.W != 256) || w->hidden % 128) return TM_ERR_UNSUPPORTED;
+    const int am = gemm1_amode(g);
+    if (am != A_TMA_MIX && am != A_TMA_3D) return TM_ERR_UNSUPPORTED;
+    return TM_OK;
+}
+
+struct Dense8Ws {
+    uint8_t* q;
+    float* rowscale;
+};
+Dense8Ws carve_dense8(Carve& c, const Geo& g) {
+    Dense8Ws w;
+    w.q = c.take<uint8_t>((size_t)g.B * g.banks * g.W);
+    w.rowscale = c.take<float>((size_t)g.B * g.banks);
+    return w;
+}
+
+// Quantize the activation rows, then one launch of the fused kernel in its FP8 mode.
+tm_status run_dense8(const Geo& g, const void* x, const void* resid, const void* extra, const tm_swiglu_w8* w, void* y,
+                     void* ws, size_t wsb, cudaStream_t st) {
+    Carve c{(uint8_t*)ws};
+    Dense8Ws d = carve_dense8(c, g);
+    if (!ws || wsb < c.off || !al16(ws)) return TM_ERR_WORKSPACE;
+    if ((uintptr_t)y % 32) return TM_ERR_INVALID_ARG;
+    tm_status s;
+    if ((s = cuda_status(launch_quant_act_rows(x, g.map, g.B, g.eps, d.q, d.rowscale, st))) != TM_OK) return s;
+    const int am = gemm1_amode(g), F = w->hidden;
+    CUtensorMap ma, mg, mu, md, mr, me, mo;
+    memset(&mr, 0, sizeof(mr));
+    memset(&me, 0, sizeof(me));
+    {
+        uint64_t dims[3] = {(uint64_t)g.W, (uint64_t)g.banks, (uint64_t)g.B};
+        uint64_t strides[2] = {(uint64_t)g.W, (uint64_t)g.banks * g.W};
+        uint32_t box[3] = {128, 1, 128};
+        if (!make_map_u8(&ma, d.q, 3, dims, strides, box)) return TM_ERR_CUDA;
+    }
+    {
+        uint64_t dims[2] = {(uint64_t)g.W, (uint64_t)g.banks * F};
+        uint64_t strides[1] = {(uint64_t)g.W};
+        uint32_t box[2] = {128, 128};
+        if (!make_map_u8(&mg, w->q_gate, 2, dims, strides, box) || !make_map_u8(&mu, w->q_up, 2, dims, strides, box))
+            return TM_ERR_CUDA;
+    }
+    if (!map_2d(&md, w->w_down, (uint64_t)g.banks * g.W, F, g.W) || !gemm1_amap(g, y, am, &mo, 32)) return TM_ERR_CUDA;
+    if (resid && !gemm1_amap(g, resid, am, &mr)) return TM_ERR_CUDA;
+    if (extra && !gemm1_amap(g, extra, am, &me)) return TM_ERR_CUDA;
+    FusedParams p;
+    memset(&p, 0, sizeof(p));
+    p.banks = g.banks;
+    p.rows = g.B;
+    p.F = F;
+    p.amap = g.map;
+    p.omap = g.map;
+    p.eps = g.eps;
+    p.out = (__nv_bfloat16*)y;
+    p.out_elems = (size_t)g.B * g.banks * g.W;
+    p.res_mode = resid ? RES_STREAM : RES_NONE;
+    p.has_extra = extra != nullptr;
+    p.rowscale = d.rowscale;
+    p.s_gate = w->s_gate;
+    p.s_up = w->s_up;
+    const long tiles = (long)g.banks * ((g.B + 127) / 128);
+    const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+    return cuda_status(launch_fused128(g.W, am == A_TMA_MIX ? A_F8MIX : A_F8ROW, ma, mg, mu, md, mr, me, mo, p, grid, st));
+}
+
+// block geometry of the FP8 path
+tm_status check_block8(const tm_shape* s, const tm_block_fp8* b, Geo* gm, Geo* gr) {
+    if (!b) return TM_ERR_INVALID_ARG;
+    tm_status st = make_geo(s, TM_LAYOUT_MIXED, b->mix.banks, b->mix.width, gm);
+    if (st == TM_OK) st = check_dense8(*gm, &b->mix);
+    if (st == TM_OK) st = make_geo(s, TM_LAYOUT_ROWS, b->rev.banks, b->rev.width, gr);
+    if (st == TM_OK) st = check_dense8(*gr, &b->rev);
+    if (st == TM_OK && (gr->banks != s->T || gr->W != s->D)) st = TM_ERR_INVALID_ARG;
+    return st;
+}
+
+size_t block8_ws(const Geo& gm, const Geo& gr, const tm_shape* s) {
+    Carve a{nullptr}, b{nullptr};
+    carve_dense8(a, gm);
+    carve_dense8(b, gr);
+    const size_t sub = align256(a.off > b.off ? a.off : b.off);
+    return align256((size_t)s->B * s->T * s->D * 2) + sub;
+}
+
 // ------------------------------------------------------------------ sub-layer dispatch
 int sub_banks(const tm_sublayer* s) { return s->is_moe ? s->moe.banks : s->dense.banks; }
 int sub_width(const tm_sublayer* s) { return s->is_moe ? s->moe.width : s->dense.width; }
@@ -993,6 +1096,69 @@ tm_status tm_stack_forward(const void* X, const tm_block* blocks, int L, int gap
         if (s != TM_OK) return s;
     }
     return TM_OK;
+}
+
+tm_status tm_quantize_fp8_weights(const void* w, const void* gain, int groups, size_t rows, int cols, uint8_t* q,
+                                  float* scale, void* stream) {
+    if (!w || !q || !scale || groups <= 0 || rows == 0 || cols <= 0 || (rows * cols) % 2) return TM_ERR_INVALID_ARG;
+    if (!al16(w) || !al16(q) || (gain && !al16(gain)) || (reinterpret_cast<uintptr_t>(scale) & 3)) return TM_ERR_INVALID_ARG;
+    return cuda_status(launch_quant_matrices(w, gain, groups, rows * (size_t)cols, cols, q, scale, (cudaStream_t)stream));
+}
+
+tm_status tm_quantize_fp8_act(const void* x, tm_layout layout, const tm_shape* shape, int banks, int width, uint8_t* q,
+                              float* rowscale, void* stream) {
+    Geo g;
+    tm_status s = make_geo(shape, layout, banks, width, &g);
+    if (s != TM_OK) return s;
+    if (!x || !q || !rowscale || !al16(x) || !al16(q) || (reinterpret_cast<uintptr_t>(rowscale) & 3))
+        return TM_ERR_INVALID_ARG;
+    if (g.dtype != TM_BF16) return TM_ERR_UNSUPPORTED;
+    return cuda_status(launch_quant_act_rows(x, g.map, g.B, g.eps, q, rowscale, (cudaStream_t)stream));
+}
+
+size_t tm_pertoken_swiglu_fp8_workspace_bytes(const tm_shape* shape, tm_layout layout, const tm_swiglu_w8* w) {
+    Geo g;
+    if (!w || make_geo(shape, layout, w->banks, w->width, &g) != TM_OK || check_dense8(g, w) != TM_OK) return 0;
+    Carve c{nullptr};
+    carve_dense8(c, g);
+    return align256(c.off);
+}
+
+tm_status tm_pertoken_swiglu_fp8(const void* x, const void* residual, tm_layout layout, const tm_shape* shape,
+                                 const tm_swiglu_w8* w, void* y, void* workspace, size_t workspace_bytes, void* stream) {
+    Geo g;
+    if (!w) return TM_ERR_INVALID_ARG;
+    tm_status s = make_geo(shape, layout, w->banks, w->width, &g);
+    if (s != TM_OK) return s;
+    if ((s = check_dense8(g, w)) != TM_OK) return s;
+    if (!x || !y || x == y || !al16(x) || !al16(y) || (residual && !al16(residual))) return TM_ERR_INVALID_ARG;
+    return run_dense8(g, x, residual, nullptr, w, y, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+size_t tm_block_fp8_workspace_bytes(const tm_shape* shape, const tm_block_fp8* block) {
+    Geo gm, gr;
+    if (check_block8(shape, block, &gm, &gr) != TM_OK) return 0;
+    return block8_ws(gm, gr, shape);
+}
+
+tm_status tm_block_forward_fp8(const void* X, const tm_block_fp8* block, const tm_shape* shape, void* Y,
+                               void* X_revert_opt, void* workspace, size_t workspace_bytes, void* stream) {
+    Geo gm, gr;
+    tm_status s = check_block8(shape, block, &gm, &gr);
+    if (s != TM_OK) return s;
+    if (!X || !Y || X == Y || !al16(X) || !al16(Y) || (X_revert_opt && !al16(X_revert_opt))) return TM_ERR_INVALID_ARG;
+    const size_t need = block8_ws(gm, gr, shape);
+    if (!workspace || workspace_bytes < need || !al16(workspace)) return TM_ERR_WORKSPACE;
+    Carve c{(uint8_t*)workspace};
+    void* xr = c.take<uint8_t>((size_t)shape->B * shape->T * shape->D * 2);
+    if (X_revert_opt) xr = X_revert_opt;
+    c.off = align256(c.off);
+    void* sub_ws = (uint8_t*)workspace + c.off;
+    const size_t sub_wsb = workspace_bytes - c.off;
+    cudaStream_t st = (cudaStream_t)stream;
+    // H_next = FFN_mix(Norm(Mix(X))) + Mix(X) through Revert into X_rev; Y = FFN_rev(Norm(X_rev)) + X
+    if ((s = run_dense8(gm, X, X, nullptr, &block->mix, xr, sub_ws, sub_wsb, st)) != TM_OK) return s;
+    return run_dense8(gr, xr, X, nullptr, &block->rev, Y, sub_ws, sub_wsb, st);
 }
 
 tm_status tm_get_device_error(void* stream) {

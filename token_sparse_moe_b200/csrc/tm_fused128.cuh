@@ -45,14 +45,22 @@ namespace tml {
 
 enum FusedResid : int { RES_NONE = 0, RES_FROM_A = 1, RES_STREAM = 2 };
 constexpr int A_BLOCK = 4;   // fused128 kernel: a whole dense block (mixing tiles, then reverting tiles)
+// FP8 serving path of the fused sub-layer: A = E4M3 rows [B * banks, W] (quantized per row, read
+// through a 3-D map) and E4M3 gate / up weights, GEMM1 with kind::f8f6f4 MMAs; the SwiGLU takes
+// back the row factor and the bank's gate / up weight scales; GEMM2, the residual (always
+// streamed) and the output are those of the bf16 kernel, in the Mix geometry (A_F8MIX) or the
+// row one.
+constexpr int A_F8MIX = 5;
+constexpr int A_F8ROW = 6;
 
 template <int W, int AMODE>
 struct Fused128Cfg {
     static_assert(W == 128 || W == 256, "fused sub-layer supports row widths 128 and 256");
-    static constexpr int A_BYTES = 128 * W * 2;
+    static constexpr bool F8 = AMODE == A_F8MIX || AMODE == A_F8ROW;
+    static constexpr int A_BYTES = 128 * W * (F8 ? 1 : 2);
     static constexpr int HID_BYTES = 128 * 128 * 2;               // one 128-wide hidden chunk, 2 K-slabs
     static constexpr int SB = 32768;                              // ring stage
-    static constexpr int G1_STAGES = W / 64;                      // 256 rows x 64 K per stage
+    static constexpr int G1_STAGES = F8 ? W / 128 : W / 64;       // 256 rows x 64 K (bf16) or 128 K (E4M3) per stage
     static constexpr int G2_STAGES = W == 256 ? 2 : 1;            // W rows x 128 K per chunk
     static constexpr int R_STAGES = W / 128;                      // residual tile: 128 rows x 128 columns per stage
     static constexpr int STAGES = W == 256 ? 4 : 5;
@@ -91,20 +99,21 @@ struct F128Item {
     bool sec, mx;
 };
 
+// The kernel body; the tensor maps are the kernel's __grid_constant__ parameters, passed by
+// reference so that the bulk tensor instructions see their parameter-space addresses.
 template <int W, int AMODE>
-__global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
-    fused128_swiglu_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
-                           const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmD,
-                           const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmE,
-                           const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmA2,
-                           const __grid_constant__ CUtensorMap tmG2, const __grid_constant__ CUtensorMap tmU2,
-                           const __grid_constant__ CUtensorMap tmD2, const __grid_constant__ CUtensorMap tmO2,
-                           const FusedParams p) {
+__device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUtensorMap& tmG, const CUtensorMap& tmU,
+                                              const CUtensorMap& tmD, const CUtensorMap& tmR, const CUtensorMap& tmE,
+                                              const CUtensorMap& tmO, const CUtensorMap& tmA2, const CUtensorMap& tmG2,
+                                              const CUtensorMap& tmU2, const CUtensorMap& tmD2, const CUtensorMap& tmO2,
+                                              const FusedParams& p) {
     // Maps: A, G, U, D, O of the (first) sub-layer; R / E the streamed residual and inter-residual
     // (in block mode those of the reverting sub-layer); A2, G2, U2, D2, O2 the reverting
     // sub-layer's in block mode (unused otherwise).
     using C = Fused128Cfg<W, AMODE>;
     constexpr bool BLK = AMODE == A_BLOCK;
+    constexpr bool F8 = C::F8;
+    constexpr bool MIXG = AMODE == A_TMA_MIX || AMODE == A_F8MIX;   // Mix geometry outside block mode
     constexpr int STAGES = C::STAGES;
     const int mt = (p.rows + 127) / 128;
     const int ntile1 = p.banks * mt;                 // tiles of one sub-layer
@@ -138,7 +147,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             return true;
         }
         it.sec = false;
-        it.mx = AMODE == A_TMA_MIX;
+        it.mx = MIXG;
         it.c1 = NC;
         if (k < full_waves) {
             it.t = b + k * (int)gridDim.x;
@@ -159,7 +168,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         return true;
     };
     // per-item choices (compile-time constants outside block mode)
-    auto amix = [&](const F128Item& it) { return BLK ? it.mx : AMODE == A_TMA_MIX; };
+    auto amix = [&](const F128Item& it) { return BLK ? it.mx : MIXG; };
     auto rmode = [&](const F128Item& it) { return BLK && it.sec ? p.res_mode2 : p.res_mode; };
     auto n_res = [&](const F128Item& it) { return rmode(it) == RES_STREAM ? C::R_STAGES : 0; };
     auto n_ext = [&](const F128Item& it) { return (BLK && it.sec ? p.has_extra2 : p.has_extra) ? C::R_STAGES : 0; };
@@ -201,7 +210,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         }
         mbar_init(a_full, 1);
         // per slab of A: the MMA (last read issued) + the 4 epilogue warps of the half that reads it
-        for (int q = 0; q < C::G1_STAGES; ++q) mbar_init(&a_empty[q], 1 + 4);
+        for (int q = 0; q < C::G1_STAGES; ++q) mbar_init(&a_empty[q], F8 ? 1 : 1 + 4);
         mbar_init(g1_full, 1);
         mbar_init(g1_empty, 8);
         mbar_init(hid_full, 8);
@@ -302,7 +311,8 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                 for (int qa = 0; qa < C::G1_STAGES && ok; ++qa) {
                     if (!wait_or_abort(&a_empty[qa], (lt & 1) ^ 1, abort_flag, 0x3100)) { ok = false; break; }
                     if (qa == 0) mbar_arrive_expect_tx(a_full, C::A_BYTES);
-                    load_rows(mA, mx, sA + qa * 16384, a_full, g, m * 128, qa * 4, 4);
+                    if (F8) tma_load_3d(sA + qa * 16384, mA, a_full, qa * 128, g, m * 128);   // 128 E4M3 columns
+                    else load_rows(mA, mx, sA + qa * 16384, a_full, g, m * 128, qa * 4, 4);
                 }
                 if (!ok) break;
                 // ring order per step: G1(step) (step < NC), G2(step - LAG) (step >= LAG), and at step
@@ -316,8 +326,9 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x3101)) { ok = false; break; }
                             uint8_t* st = sR + s * C::SB;
                             mbar_arrive_expect_tx(&full[s], C::SB);
-                            tma_load_2d(st, mG, &full[s], q * 64, g * F + c * 128);
-                            tma_load_2d(st + 16384, mU, &full[s], q * 64, g * F + c * 128);
+                            const int kq = F8 ? q * 128 : q * 64;
+                            tma_load_2d(st, mG, &full[s], kq, g * F + c * 128);
+                            tma_load_2d(st + 16384, mU, &full[s], kq, g * F + c * 128);
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                     }
@@ -358,7 +369,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         // hidden barrier and the stages of a GEMM2) are tested together without blocking, so their
         // latencies overlap; only a stage that is not ready yet is waited for on its own.
         if (lane == 0) {
-            constexpr uint32_t idesc1 = umma_idesc_bf16(128, 256);
+            constexpr uint32_t idesc1 = F8 ? umma_idesc_e4m3(128, 256) : umma_idesc_bf16(128, 256);
             constexpr uint32_t idesc2 = umma_idesc_bf16(128, W);
             constexpr uint32_t idescI = umma_idesc_bf16(128, 16);
             const uint32_t aS = smem_u32(sA), hS = smem_u32(sH), rS = smem_u32(sR);
@@ -417,7 +428,8 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                             const uint64_t bd = rdesc0 + (uint64_t)s * kStageDesc;
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
-                                umma_bf16(tmem + C::G1COL, adesc[q * 4 + kk], bd + 2 * kk, idesc1, (q | kk) != 0);
+                                if (F8) umma_e4m3(tmem + C::G1COL, adesc[q * 4 + kk], bd + 2 * kk, idesc1, (q | kk) != 0);
+                                else umma_bf16(tmem + C::G1COL, adesc[q * 4 + kk], bd + 2 * kk, idesc1, (q | kk) != 0);
                             umma_commit(&empty[s]);
                             if (step == nc - 1 && !a_after_id) umma_commit(&a_empty[q]);
                             if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -693,7 +705,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                         const uint4 w4 = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
                                                     pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
                         const int c8 = hh * 4 + e;
-                        uint8_t* dst = AMODE == A_TMA_MIX
+                        uint8_t* dst = MIXG
                                            ? stg + (c8 >> 1) * 1024 + lane * 32 + (((c8 & 1) ^ ((lane >> 2) & 1)) << 4)
                                            : stg + lane * 128 + ((c8 ^ (lane & 7)) << 4);
                         *reinterpret_cast<uint4*>(dst) = w4;
@@ -702,7 +714,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0 && b0 < p.rows) {
-                    if (AMODE == A_TMA_MIX) {
+                    if (MIXG) {
                         const int per = p.omap.dh >> 4;
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
@@ -721,16 +733,27 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         int lt = 0;
         float sc = 0.f;
         // the statistics of a tile read the A slabs of this thread's half; release them afterwards
+        // (the FP8 path reads no A slab: its row factor comes with the quantized rows)
         auto release_a = [&]() {
+            if (F8) return;
             __syncwarp();
             if (lane == 0) {
 #pragma unroll
                 for (int qa = 0; qa < C::G1_STAGES / 2; ++qa) mbar_arrive(&a_empty[half * (C::G1_STAGES / 2) + qa]);
             }
         };
+        auto tile_scale = [&](const F128Item& t_it, float& out) -> bool {
+            if (F8) {
+                const int b = t_it.m * 128 + r;
+                out = b < p.rows ? __ldg(&p.rowscale[(size_t)b * p.banks + t_it.g]) : 0.f;
+                return true;
+            }
+            return row_scale(t_it.m, amix(t_it), out);
+        };
+
         F128Item it;
         bool have = item(0, it);
-        bool ok = have && wait_or_abort(a_full, 0, abort_flag, 0x3300) && row_scale(it.m, amix(it), sc);
+        bool ok = have && wait_or_abort(a_full, 0, abort_flag, 0x3300) && tile_scale(it, sc);
         if (ok) release_a();
         F128Item prev = it;
         bool prev_pending = false;                                     // prev's output is still to be written
@@ -741,6 +764,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         uint32_t ubase = 0;                                            // chunks of the items before this one
         for (; ok && have; ++lt) {
             const int c0 = it.c0, c1 = it.c1;
+            const float sgw = F8 ? __ldg(&p.s_gate[it.g]) : 1.f, suw = F8 ? __ldg(&p.s_up[it.g]) : 1.f;
             // ---- SwiGLU chunks: this thread owns hidden columns [half*64, half*64 + 64) of its row
 #pragma unroll 1
             for (int c = c0; c < c1; ++c) {
@@ -762,12 +786,14 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(g1_empty);
                 uint32_t pk[32];
-                const float hsc = 0.5f * sc;
+                // silu(sg * g) * (su * u): sg = su = 1/rms of the row; on the FP8 path the row factor
+                // times the bank's gate / up weight scale
+                const float hsc = 0.5f * (F8 ? sc * sgw : sc), scu = F8 ? sc * suw : sc;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float2 h0 = swiglu2(hsc, sc, make_float2(__uint_as_float(g0[2 * i]), __uint_as_float(g0[2 * i + 1])),
+                    const float2 h0 = swiglu2(hsc, scu, make_float2(__uint_as_float(g0[2 * i]), __uint_as_float(g0[2 * i + 1])),
                                               make_float2(__uint_as_float(u0[2 * i]), __uint_as_float(u0[2 * i + 1])));
-                    const float2 h1 = swiglu2(hsc, sc, make_float2(__uint_as_float(g1[2 * i]), __uint_as_float(g1[2 * i + 1])),
+                    const float2 h1 = swiglu2(hsc, scu, make_float2(__uint_as_float(g1[2 * i]), __uint_as_float(g1[2 * i + 1])),
                                               make_float2(__uint_as_float(u1[2 * i]), __uint_as_float(u1[2 * i + 1])));
                     pk[i] = pack_bf16x2(h0.x, h0.y);
                     pk[16 + i] = pack_bf16x2(h1.x, h1.y);
@@ -806,7 +832,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
             }
             // ---- statistics of the next item (its A tile is loaded once this item's last read of A is issued)
             if (have) {
-                if (!wait_or_abort(a_full, (lt + 1) & 1, abort_flag, 0x3304) || !row_scale(it.m, amix(it), sc)) {
+                if (!wait_or_abort(a_full, (lt + 1) & 1, abort_flag, 0x3304) || !tile_scale(it, sc)) {
                     ok = false;
                     break;
                 }
@@ -825,6 +851,18 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+}
+
+template <int W, int AMODE>
+__global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
+    fused128_swiglu_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
+                           const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmD,
+                           const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmE,
+                           const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmA2,
+                           const __grid_constant__ CUtensorMap tmG2, const __grid_constant__ CUtensorMap tmU2,
+                           const __grid_constant__ CUtensorMap tmD2, const __grid_constant__ CUtensorMap tmO2,
+                           const FusedParams p) {
+    fused128_body<W, AMODE>(tmA, tmG, tmU, tmD, tmR, tmE, tmO, tmA2, tmG2, tmU2, tmD2, tmO2, p);
 }
 
 }  // namespace tml

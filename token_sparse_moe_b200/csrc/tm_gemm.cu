@@ -34,7 +34,7 @@ static cudaError_t launch_fused128_one(const CUtensorMap& a, const CUtensorMap& 
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    ProfileScope ps_("fused_swiglu", st);
+    ProfileScope ps_(C::F8 ? "fused_swiglu_fp8" : "fused_swiglu", st);
     kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, g, u, d, r, e, o, a, g, u, d, o, p);
     return cudaGetLastError();
 }
@@ -81,6 +81,10 @@ cudaError_t launch_fused128(int W, int a_mode, const CUtensorMap& a, const CUten
     if (W == 256 && a_mode == A_TMA_3D) return launch_fused128_one<256, A_TMA_3D>(a, g, u, d, r, e, o, p, grid, st);
     if (W == 128 && a_mode == A_TMA_MIX) return launch_fused128_one<128, A_TMA_MIX>(a, g, u, d, r, e, o, p, grid, st);
     if (W == 128 && a_mode == A_TMA_3D) return launch_fused128_one<128, A_TMA_3D>(a, g, u, d, r, e, o, p, grid, st);
+    if (W == 256 && a_mode == A_F8MIX) return launch_fused128_one<256, A_F8MIX>(a, g, u, d, r, e, o, p, grid, st);
+    if (W == 256 && a_mode == A_F8ROW) return launch_fused128_one<256, A_F8ROW>(a, g, u, d, r, e, o, p, grid, st);
+    if (W == 128 && a_mode == A_F8MIX) return launch_fused128_one<128, A_F8MIX>(a, g, u, d, r, e, o, p, grid, st);
+    if (W == 128 && a_mode == A_F8ROW) return launch_fused128_one<128, A_F8ROW>(a, g, u, d, r, e, o, p, grid, st);
     return cudaErrorInvalidValue;
 }
 

@@ -88,6 +88,13 @@ cudaError_t launch_router_split(int dtype, const float* w_router, const void* ga
 // [B * banks * k], k <= 8), out [routed, W] (see scatter_rows_kernel)
 cudaError_t launch_scatter_rows(int dtype, const void* x, RowMap m, int B, int k, const int32_t* slot_of, size_t routed,
                                 void* out, cudaStream_t st);
+// FP8 E4M3 (bf16 inputs): the codes of `groups` weight matrices of n elements (rows of `cols`)
+// with one scale per matrix (gain optional, folded first), and the per-row activation codes
+// [B * banks, W] with rowscale = (max|x| / 448) / rms(x)
+cudaError_t launch_quant_matrices(const void* w, const void* gain, int groups, size_t n, int cols, uint8_t* q,
+                                  float* scale, cudaStream_t st);
+cudaError_t launch_quant_act_rows(const void* x, RowMap m, int B, float eps, uint8_t* q, float* rowscale,
+                                  cudaStream_t st);
 cudaError_t launch_permute(int dtype, const void* src, void* dst, int B, int T, int D, int H, bool to_mixed,
                            cudaStream_t st);
 cudaError_t launch_fold_gain(int dtype, const void* w, const void* gain, void* out, size_t rows, int width,

@@ -681,4 +681,126 @@ cudaError_t launch_simt_gemm(int epi, const SimtGemmArgs& a, int max_tiles, cuda
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ FP8 E4M3 serving path
+// Two fp32 values to two E4M3 codes (nearest, ties to even, saturating at +-448); the first
+// argument's code is the low byte.
+__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// E4M3 quantization of bf16 weight matrices, one scale per matrix ([digest] 2.5.2 FP8
+// quantization; the gate / up projections of each bank): `groups` matrices of n elements each,
+// the norm gain (optional, one per column of `cols`) multiplied in and rounded to bf16 first, as
+// the bf16 path folds it.  scale = max|matrix| / 448 (1 for an all-zero matrix), code =
+// E4M3(w / scale) with IEEE fp32 division.  Three passes: the matrix maxima (float bit patterns
+// of non-negative values order like the values, so an integer atomic max is exact), the codes,
+// and the scales written over the maxima.
+__device__ __forceinline__ float folded_weight(const __nv_bfloat16* w, const __nv_bfloat16* gain, size_t i, int cols) {
+    float v = __bfloat162float(w[i]);
+    if (gain) v = __bfloat162float(__float2bfloat16_rn(v * __bfloat162float(gain[i % cols])));
+    return v;
+}
+__device__ __forceinline__ float matrix_scale(unsigned amax_bits) {
+    const float amax = __uint_as_float(amax_bits);
+    return amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+}
+__global__ void __launch_bounds__(256) quant_matrix_amax_kernel(const __nv_bfloat16* __restrict__ w,
+                                                                const __nv_bfloat16* __restrict__ gain, size_t n,
+                                                                int cols, unsigned* __restrict__ amax_bits) {
+    const int g = blockIdx.y;
+    const __nv_bfloat16* wg = w + (size_t)g * n;
+    float m = 0.f;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        m = fmaxf(m, fabsf(folded_weight(wg, gain, i, cols)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) atomicMax(&amax_bits[g], __float_as_uint(m));
+}
+__global__ void __launch_bounds__(256) quant_matrix_codes_kernel(const __nv_bfloat16* __restrict__ w,
+                                                                 const __nv_bfloat16* __restrict__ gain, size_t n,
+                                                                 int cols, const unsigned* __restrict__ amax_bits,
+                                                                 uint8_t* __restrict__ q) {
+    const int g = blockIdx.y;
+    const float s = matrix_scale(amax_bits[g]);
+    const __nv_bfloat16* wg = w + (size_t)g * n;
+    uint8_t* qg = q + (size_t)g * n;
+    for (size_t i = 2 * (blockIdx.x * (size_t)blockDim.x + threadIdx.x); i < n; i += 2 * (size_t)gridDim.x * blockDim.x)
+        *reinterpret_cast<uint16_t*>(qg + i) =
+            e4m3x2(__fdiv_rn(folded_weight(wg, gain, i, cols), s), __fdiv_rn(folded_weight(wg, gain, i + 1, cols), s));
+}
+__global__ void quant_matrix_scales_kernel(unsigned* __restrict__ scale_bits, int groups) {
+    const int g = blockIdx.x * blockDim.x + threadIdx.x;
+    if (g < groups) scale_bits[g] = __float_as_uint(matrix_scale(scale_bits[g]));
+}
+
+// Per-row E4M3 quantization of the activation rows of a sub-layer, read through the row map
+// (the Mix permutation for the mixing sub-layer), written as plain rows [B * banks, W] (row
+// b * banks + bank).  One warp per row: sum of squares and max|x| by shuffles; rowscale =
+// (max|x| / 448) / rms(x), the factor the FP8 GEMM1 output takes back per row.
+__global__ void __launch_bounds__(256) quant_act_rows_kernel(const __nv_bfloat16* __restrict__ x, RowMap m, int B,
+                                                             float eps, uint8_t* __restrict__ q,
+                                                             float* __restrict__ rowscale) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int W = m.W, banks = m.banks;
+    for (int row = warp; row < B * banks; row += nwarps) {
+        const int b = row / banks, bank = row - b * banks;
+        float ss = 0.f, amax = 0.f;
+        for (int c = lane * 8; c < W; c += 256) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c)));
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(wv[e] << 16), hi = __uint_as_float(wv[e] & 0xFFFF0000u);
+                ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+                amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        }
+        const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+        for (int c = lane * 8; c < W; c += 256) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c)));
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+            uint16_t o4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                o4[e] = e4m3x2(__fdiv_rn(__uint_as_float(wv[e] << 16), s), __fdiv_rn(__uint_as_float(wv[e] & 0xFFFF0000u), s));
+            *reinterpret_cast<uint2*>(q + (size_t)row * W + c) =
+                make_uint2(o4[0] | (uint32_t(o4[1]) << 16), o4[2] | (uint32_t(o4[3]) << 16));
+        }
+        if (lane == 0) rowscale[row] = s * (1.0f / sqrtf(ss / (float)W + eps));
+    }
+}
+
+cudaError_t launch_quant_matrices(const void* w, const void* gain, int groups, size_t n, int cols, uint8_t* q,
+                                  float* scale, cudaStream_t st) {
+    ProfileScope ps_("fp8_quant_weights", st);
+    if (n % 2 || n % cols) return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(scale, 0, (size_t)groups * sizeof(float), st);
+    if (e != cudaSuccess) return e;
+    size_t bx = (n + 2047) / 2048;
+    dim3 grid((unsigned)(bx < 1024 ? bx : 1024), groups);
+    quant_matrix_amax_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)w, (const __nv_bfloat16*)gain, n, cols,
+                                                   (unsigned*)scale);
+    quant_matrix_codes_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)w, (const __nv_bfloat16*)gain, n, cols,
+                                                    (const unsigned*)scale, q);
+    quant_matrix_scales_kernel<<<(groups + 255) / 256, 256, 0, st>>>((unsigned*)scale, groups);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_act_rows(const void* x, RowMap m, int B, float eps, uint8_t* q, float* rowscale,
+                                  cudaStream_t st) {
+    ProfileScope ps_("fp8_quant_rows", st);
+    if (m.W % 8 || (m.layout == 1 && m.dh % 8)) return cudaErrorInvalidValue;
+    quant_act_rows_kernel<<<grid_for((size_t)B * m.banks * 32, 256), 256, 0, st>>>((const __nv_bfloat16*)x, m, B, eps,
+                                                                                  q, rowscale);
+    return cudaGetLastError();
+}
+
 }  // namespace tml
