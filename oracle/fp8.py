@@ -11,14 +11,20 @@ quantization of a model trained in bf16.  The page names the format only; the re
     normal values 2^(e-7) * (1 + m/8) for exponent fields e = 1..15, subnormals m * 2^-9 for
     e = 0, largest finite 448 (the all-ones pattern S.1111.111 is NaN; there are no
     infinities).  Conversion rounds to nearest with ties to even and saturates at +-448.
+  * Scales are powers of two: for values with largest magnitude m > 0 the scale is 2^e with e
+    the smallest integer such that m * 2^-e <= 448 (m = f * 2^x with f in [0.5, 1) gives
+    e = x - 9 when f <= 0.875, else x - 8); 1 when m = 0.  Then v * 2^-e is exact and the only
+    rounding is E4M3's own; the largest value lands in (224, 448].  E4M3 is a floating-point
+    format, so its 3-bit relative precision does not depend on the scale; a power-of-two scale
+    moves only the underflow threshold, by less than one binade.
   * Weights: the gate and up projections of each bank (with the RMSNorm gain folded in and
     rounded to bf16 first, as the bf16 path stores them) are quantized per matrix, one scale per
-    bank: s = max|W| / 448 in fp32 (1 for an all-zero matrix), q = E4M3(fp32(w / s)).  E4M3 is a
-    floating-point format: every value inside its normal range (2^-6 .. 448 times s) keeps a 3-bit
-    mantissa whatever the scale, so per-row scales would change nothing for rows whose magnitudes
-    sit within that 2^15 range of the matrix maximum, as these projections' rows do.
+    bank: q = E4M3(w * 2^-e).  Every value inside E4M3's normal range (2^-6 .. 448 times the
+    scale) keeps a 3-bit mantissa whatever the scale, so per-row scales would change nothing for
+    rows whose magnitudes sit within that 2^15 range of the matrix maximum, as these projections'
+    rows do.
   * Activations: every sub-layer row x (width W, the input of the RMSNorm) is quantized on its
-    own: s_a = max|x| / 448 in fp32 (1 for an all-zero row), q_a = E4M3(fp32(x / s_a)).
+    own: q_a = E4M3(x * 2^-e_a), s_a = 2^e_a.
   * GEMM1 runs on the quantized operands: gate_n = (q_a . q_gate_n) * s_a * s_gate / rms(x),
     up_n likewise, with rms taken over the unquantized row exactly as in the bf16 path.  The
     SwiGLU, the down projection and the residual are those of the bf16 path (the down
@@ -75,17 +81,25 @@ def e4m3_decode(code: np.ndarray) -> np.ndarray:
     return s * val
 
 
+def pow2_scale_exponent(amax: np.ndarray) -> np.ndarray:
+    """The smallest e with amax * 2^-e <= 448 (0 where amax == 0), from amax = f * 2^x, f in
+    [0.5, 1): 448 = 0.875 * 2^9, so e = x - 9 when f <= 0.875 and x - 8 otherwise."""
+    f, x = np.frexp(np.asarray(amax, dtype=np.float64))
+    e = np.where(f <= 0.875, x - 9, x - 8)
+    return np.where(np.asarray(amax) > 0, e, 0).astype(np.int64)
+
+
 def quantize_rows(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
     """Per-row E4M3 quantization of a [R, K] array whose values are fp32-representable.
 
-    Returns (codes [R, K] uint8, scales [R] float32) with scale = max|row| / 448 in fp32
-    (1 for an all-zero row) and codes = E4M3(fp32(row / scale)).
+    Returns (codes [R, K] uint8, scales [R] float32): scale = 2^e with e the smallest integer
+    such that max|row| * 2^-e <= 448 (1 for an all-zero row), codes = E4M3(row * 2^-e) (exact
+    scaling).
     """
     x32 = np.asarray(x, dtype=np.float32)
-    amax = np.max(np.abs(x32), axis=1)
-    s = (amax / np.float32(E4M3_MAX)).astype(np.float32)
-    s = np.where(amax > 0, s, np.float32(1.0)).astype(np.float32)
-    return e4m3_encode((x32 / s[:, None]).astype(np.float32)), s
+    e = pow2_scale_exponent(np.max(np.abs(x32), axis=1))
+    s = np.ldexp(np.float32(1.0), e).astype(np.float32)
+    return e4m3_encode(np.ldexp(x32.astype(np.float64), -e[:, None])), s
 
 
 def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
@@ -93,11 +107,10 @@ def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
 
 
 def quantize_matrix(w: np.ndarray) -> Tuple[np.ndarray, np.float32]:
-    """E4M3 quantization of a whole matrix with one scale: max|w| / 448 in fp32 (1 if all zero)."""
+    """E4M3 quantization of a whole matrix with one power-of-two scale (as quantize_rows)."""
     w32 = np.asarray(w, dtype=np.float32)
-    amax = np.float32(np.max(np.abs(w32))) if w32.size else np.float32(0)
-    s = np.float32(amax / np.float32(E4M3_MAX)) if amax > 0 else np.float32(1.0)
-    return e4m3_encode((w32 / s).astype(np.float32)), s
+    e = int(pow2_scale_exponent(np.max(np.abs(w32)) if w32.size else 0.0))
+    return e4m3_encode(np.ldexp(w32.astype(np.float64), -e)), np.float32(np.ldexp(1.0, e))
 
 
 def fold_gain(w: np.ndarray, gain: Optional[np.ndarray]) -> np.ndarray:

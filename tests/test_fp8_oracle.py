@@ -47,11 +47,20 @@ def test_row_quantization_bounds():
     rng = np.random.default_rng(1)
     x = (rng.standard_normal((64, 256)) * rng.uniform(0.01, 100, (64, 1))).astype(np.float32)
     x[3] = 0.0
+    x[5] = rng.uniform(-1, 1, 256).astype(np.float32)
+    x[5, 7] = 448.0 * 2.0 ** -4                                 # a row maximum exactly on the top code
     codes, s = F.quantize_rows(x)
-    assert s.dtype == np.float32 and s[3] == 1.0
+    assert s.dtype == np.float32 and s[3] == 1.0 and s[5] == 2.0 ** -4
+    assert np.all(np.frexp(s)[0] == 0.5)                        # powers of two
     q = F.e4m3_decode(codes)
     nz = np.arange(64) != 3
-    assert np.all(np.max(np.abs(q[nz]), axis=1) == 448.0)     # the largest element lands on the top code
+    # the smallest power-of-two scale that fits: the largest element scales into (224, 448] and
+    # rounds to a code in [224, 448]
+    m = np.max(np.abs(x[nz]), axis=1) / s[nz]
+    assert np.all((m > 224.0) & (m <= 448.0))
+    top = np.max(np.abs(q[nz]), axis=1)
+    assert np.all((top >= 224.0) & (top <= 448.0))
+    assert np.max(np.abs(q[5])) == 448.0
     err = np.abs(q * s[:, None].astype(np.float64) - x)
     # half a step of a 3-bit mantissa (2^-4 relative) in the normal range, half the subnormal
     # spacing (2^-10 * s) below it
@@ -61,8 +70,8 @@ def test_row_quantization_bounds():
 
 def test_fp8_ffn_equals_bf16_ffn_when_quantization_is_exact():
     # rows and weights already on the E4M3 grid, each row's (and each weight matrix's) largest
-    # magnitude exactly 448 * 2^k: the scales are powers of two, x / s is exact and every code
-    # reproduces its value
+    # magnitude exactly 448 * 2^k: the scale is 2^k, the scaling exact and every code reproduces
+    # its value
     rng = np.random.default_rng(2)
     W, Fh, R = 64, 96, 24
 
@@ -108,9 +117,10 @@ def test_matrix_scale_is_the_matrix_maximum():
     rng = np.random.default_rng(5)
     w = (rng.standard_normal((16, 40)) * rng.uniform(0.1, 10, (16, 1))).astype(np.float32)
     codes, s = F.quantize_matrix(w)
-    assert s == np.float32(np.max(np.abs(w)) / np.float32(448))
+    m = np.max(np.abs(w))
+    assert np.frexp(s)[0] == 0.5 and m / s <= 448.0 < 2 * m / s   # the smallest power of two that fits
     q = F.e4m3_decode(codes)
-    assert np.max(np.abs(q)) == 448.0
+    assert 224.0 <= np.max(np.abs(q)) <= 448.0
     # every value above the subnormal range keeps the 2^-4 relative rounding bound, whatever its row
     big = np.abs(w) >= 2.0 ** -6 * s
     assert np.all(np.abs(q * np.float64(s) - w)[big] <= 2.0 ** -4 * np.abs(w)[big] * (1 + 1e-6))
