@@ -410,8 +410,9 @@ def run_ours(args, cfg, rank, world, local_rank):
         "config": {"workload": describe(cfg), "global_batch": total_samples, "seq_len": cfg.T,
                    "parallelism": f"dp{world} (independent batches, no data-path collective)",
                    "l2": "flushed by a 256 MB write between timed steps (outside the step events)",
-                   **({"precision": "FP8 serving path: GEMM1 (gate, up) on E4M3 operands, per-channel weight and "
-                                    "per-row activation scales; GEMM2 and residual bf16"} if args.fp8 else {})},
+                   **({"precision": "FP8 serving path: GEMM1 (gate, up) on E4M3 operands, one power-of-two scale "
+                                    "per bank weight matrix and per activation row; GEMM2 and residual bf16"}
+                      if args.fp8 else {})},
         "tflops": tflops,
         "tc_roofline_frac": tflops / (fp8_effective_peak(pk["bf16_tflops"]) if args.fp8 else pk["bf16_tflops"]),
         "roofline": roof,

@@ -216,17 +216,19 @@ TM_API tm_status tm_stack_forward(const void *X, const tm_block *blocks, int L, 
 /* E4M3 quantization of `groups` bf16 weight matrices w [groups, rows, cols] with one scale per
  * matrix (a bank's gate or up projection), optionally times a per-column gain [cols]
  * (multiplied and rounded to bf16 first, as the bf16 path folds the RMSNorm gain):
- * scale[g] = max|matrix g| / 448 (1 for an all-zero matrix); q [groups, rows, cols] =
- * E4M3(w / scale[g]) with IEEE fp32 division.  rows * cols even.  q (1-byte codes) and scale are
- * device memory.  E4M3 keeps a 3-bit mantissa for every value inside its normal range
- * (2^-6 .. 448 times the scale), so one scale serves all rows of a projection. */
+ * scale[g] = 2^e with e the smallest integer such that max|matrix g| * 2^-e <= 448 (1 for an
+ * all-zero matrix); q [groups, rows, cols] = E4M3(w * 2^-e) (exact scaling).  rows * cols even.
+ * q (1-byte codes) and scale are device memory.  E4M3 keeps a 3-bit mantissa for every value
+ * inside its normal range (2^-6 .. 448 times the scale), so one scale serves all rows of a
+ * projection. */
 TM_API tm_status tm_quantize_fp8_weights(const void *w, const void *gain, int groups, size_t rows, int cols,
                                          uint8_t *q, float *scale, void *stream);
 
 /* Per-row E4M3 quantization of a sub-layer's bf16 activation rows (banks, width as for the
- * sub-layer, read through `layout`): q [B*banks, width] (row b*banks + bank) = E4M3(row / s)
- * with s = max|row| / 448 (1 for an all-zero row), and rowscale [B*banks] = s / rms(row),
- * rms = sqrt(mean(row^2) + eps) over the unquantized row. */
+ * sub-layer, read through `layout`): q [B*banks, width] (row b*banks + bank) = E4M3(row * 2^-e)
+ * with 2^e the row's power-of-two scale (as for the weights), and rowscale [B*banks] =
+ * 2^e / rms(row), rms = sqrt(mean(row^2) + eps) over the unquantized row.  bf16 rows of width
+ * <= 1024 (mixed rows: head width a multiple of 8); others return TM_ERR_UNSUPPORTED. */
 TM_API tm_status tm_quantize_fp8_act(const void *x, tm_layout layout, const tm_shape *shape, int banks, int width,
                                      uint8_t *q, float *rowscale, void *stream);
 

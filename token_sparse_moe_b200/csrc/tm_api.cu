@@ -1112,7 +1112,7 @@ tm_status tm_quantize_fp8_act(const void* x, tm_layout layout, const tm_shape* s
     if (s != TM_OK) return s;
     if (!x || !q || !rowscale || !al16(x) || !al16(q) || (reinterpret_cast<uintptr_t>(rowscale) & 3))
         return TM_ERR_INVALID_ARG;
-    if (g.dtype != TM_BF16) return TM_ERR_UNSUPPORTED;
+    if (g.dtype != TM_BF16 || g.W > 1024 || (g.map.layout == 1 && g.map.dh % 8)) return TM_ERR_UNSUPPORTED;
     return cuda_status(launch_quant_act_rows(x, g.map, g.B, g.eps, q, rowscale, (cudaStream_t)stream));
 }
 

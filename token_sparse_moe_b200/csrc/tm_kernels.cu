@@ -690,22 +690,31 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
     return r;
 }
 
+// Power-of-two E4M3 scales: for a largest magnitude m > 0 the scale is 2^e with e the smallest
+// integer such that m * 2^-e <= 448; with m = f * 2^x, f in [0.5, 1) and 448 = 0.875 * 2^9 that
+// is e = x - 9 when f <= 0.875, else x - 8 (0 when m == 0).  Scaling by 2^-e is exact.
+__device__ __forceinline__ int pow2_exponent(float m) {
+    if (!(m > 0.f)) return 0;
+    int x;
+    const float f = frexpf(m, &x);
+    return f <= 0.875f ? x - 9 : x - 8;
+}
+__device__ __forceinline__ float pow2f(int k) {
+    return (k >= -126 && k <= 127) ? __int_as_float((127 + k) << 23) : ldexpf(1.f, k);
+}
+
 // E4M3 quantization of bf16 weight matrices, one scale per matrix ([digest] 2.5.2 FP8
 // quantization; the gate / up projections of each bank): `groups` matrices of n elements each,
 // the norm gain (optional, one per column of `cols`) multiplied in and rounded to bf16 first, as
-// the bf16 path folds it.  scale = max|matrix| / 448 (1 for an all-zero matrix), code =
-// E4M3(w / scale) with IEEE fp32 division.  Three passes: the matrix maxima (float bit patterns
-// of non-negative values order like the values, so an integer atomic max is exact), the codes,
-// and the scales written over the maxima.
+// the bf16 path folds it.  scale = 2^e (above), code = E4M3(w * 2^-e).  Three passes: the matrix
+// maxima (float bit patterns of non-negative values order like the values, so an integer atomic
+// max is exact), the codes, and the scales written over the maxima.
 __device__ __forceinline__ float folded_weight(const __nv_bfloat16* w, const __nv_bfloat16* gain, size_t i, int cols) {
     float v = __bfloat162float(w[i]);
     if (gain) v = __bfloat162float(__float2bfloat16_rn(v * __bfloat162float(gain[i % cols])));
     return v;
 }
-__device__ __forceinline__ float matrix_scale(unsigned amax_bits) {
-    const float amax = __uint_as_float(amax_bits);
-    return amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-}
+
 __global__ void __launch_bounds__(256) quant_matrix_amax_kernel(const __nv_bfloat16* __restrict__ w,
                                                                 const __nv_bfloat16* __restrict__ gain, size_t n,
                                                                 int cols, unsigned* __restrict__ amax_bits) {
@@ -723,22 +732,23 @@ __global__ void __launch_bounds__(256) quant_matrix_codes_kernel(const __nv_bflo
                                                                  int cols, const unsigned* __restrict__ amax_bits,
                                                                  uint8_t* __restrict__ q) {
     const int g = blockIdx.y;
-    const float s = matrix_scale(amax_bits[g]);
+    const float inv = pow2f(-pow2_exponent(__uint_as_float(amax_bits[g])));
     const __nv_bfloat16* wg = w + (size_t)g * n;
     uint8_t* qg = q + (size_t)g * n;
     for (size_t i = 2 * (blockIdx.x * (size_t)blockDim.x + threadIdx.x); i < n; i += 2 * (size_t)gridDim.x * blockDim.x)
         *reinterpret_cast<uint16_t*>(qg + i) =
-            e4m3x2(__fdiv_rn(folded_weight(wg, gain, i, cols), s), __fdiv_rn(folded_weight(wg, gain, i + 1, cols), s));
+            e4m3x2(folded_weight(wg, gain, i, cols) * inv, folded_weight(wg, gain, i + 1, cols) * inv);
 }
 __global__ void quant_matrix_scales_kernel(unsigned* __restrict__ scale_bits, int groups) {
     const int g = blockIdx.x * blockDim.x + threadIdx.x;
-    if (g < groups) scale_bits[g] = __float_as_uint(matrix_scale(scale_bits[g]));
+    if (g < groups) scale_bits[g] = __float_as_uint(pow2f(pow2_exponent(__uint_as_float(scale_bits[g]))));
 }
 
 // Per-row E4M3 quantization of the activation rows of a sub-layer, read through the row map
 // (the Mix permutation for the mixing sub-layer), written as plain rows [B * banks, W] (row
-// b * banks + bank).  One warp per row: sum of squares and max|x| by shuffles; rowscale =
-// (max|x| / 448) / rms(x), the factor the FP8 GEMM1 output takes back per row.
+// b * banks + bank).  One warp per row: sum of squares and max|x| by shuffles; codes =
+// E4M3(x * 2^-e) with the row's power-of-two scale 2^e; rowscale = 2^e / rms(x), the factor the
+// FP8 GEMM1 output takes back per row.
 __global__ void __launch_bounds__(256) quant_act_rows_kernel(const __nv_bfloat16* __restrict__ x, RowMap m, int B,
                                                              float eps, uint8_t* __restrict__ q,
                                                              float* __restrict__ rowscale) {
@@ -747,10 +757,14 @@ __global__ void __launch_bounds__(256) quant_act_rows_kernel(const __nv_bfloat16
     const int W = m.W, banks = m.banks;
     for (int row = warp; row < B * banks; row += nwarps) {
         const int b = row / banks, bank = row - b * banks;
+        // the row stays in registers: up to four 8-element pieces per lane (W <= 1024)
+        uint4 v[4];
         float ss = 0.f, amax = 0.f;
-        for (int c = lane * 8; c < W; c += 256) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c)));
-            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int c = lane * 8 + 256 * k;
+            v[k] = c < W ? __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c))) : make_uint4(0, 0, 0, 0);
+            const uint32_t wv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float lo = __uint_as_float(wv[e] << 16), hi = __uint_as_float(wv[e] & 0xFFFF0000u);
@@ -763,14 +777,17 @@ __global__ void __launch_bounds__(256) quant_act_rows_kernel(const __nv_bfloat16
             ss += __shfl_xor_sync(0xffffffffu, ss, o);
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         }
-        const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-        for (int c = lane * 8; c < W; c += 256) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c)));
-            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        const int ex = pow2_exponent(amax);
+        const float s = pow2f(ex), inv = pow2f(-ex);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int c = lane * 8 + 256 * k;
+            if (c >= W) break;
+            const uint32_t wv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
             uint16_t o4[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-                o4[e] = e4m3x2(__fdiv_rn(__uint_as_float(wv[e] << 16), s), __fdiv_rn(__uint_as_float(wv[e] & 0xFFFF0000u), s));
+                o4[e] = e4m3x2(__uint_as_float(wv[e] << 16) * inv, __uint_as_float(wv[e] & 0xFFFF0000u) * inv);
             *reinterpret_cast<uint2*>(q + (size_t)row * W + c) =
                 make_uint2(o4[0] | (uint32_t(o4[1]) << 16), o4[2] | (uint32_t(o4[3]) << 16));
         }
@@ -797,7 +814,7 @@ cudaError_t launch_quant_matrices(const void* w, const void* gain, int groups, s
 cudaError_t launch_quant_act_rows(const void* x, RowMap m, int B, float eps, uint8_t* q, float* rowscale,
                                   cudaStream_t st) {
     ProfileScope ps_("fp8_quant_rows", st);
-    if (m.W % 8 || (m.layout == 1 && m.dh % 8)) return cudaErrorInvalidValue;
+    if (m.W % 8 || m.W > 1024 || (m.layout == 1 && m.dh % 8)) return cudaErrorInvalidValue;
     quant_act_rows_kernel<<<grid_for((size_t)B * m.banks * 32, 256), 256, 0, st>>>((const __nv_bfloat16*)x, m, B, eps,
                                                                                   q, rowscale);
     return cudaGetLastError();
