@@ -249,16 +249,18 @@ typedef struct { tm_swiglu_w8 mix, rev; } tm_block_fp8;
 TM_API size_t tm_pertoken_swiglu_fp8_workspace_bytes(const tm_shape *shape, tm_layout layout, const tm_swiglu_w8 *w);
 
 /* Dense sub-layer on the FP8 path:  y_row = SwiGLU_bank(RMSNorm(x_row)) + residual_row, GEMM1 on
- * E4M3 operands: gate_n = (q_row . q_gate_n) * rowscale * s_gate, up likewise (the activation
- * rows are quantized into the workspace first).  residual may be NULL; y must not alias x. */
+ * E4M3 operands: gate_n = (q_row . q_gate_n) * rowscale * s_gate, up likewise, q_row and rowscale
+ * as tm_quantize_fp8_act defines them (the kernel quantizes each row tile itself from the bf16
+ * rows it holds; the workspace, 256 bytes, is unused).  residual may be NULL; y must not alias x. */
 TM_API tm_status tm_pertoken_swiglu_fp8(const void *x, const void *residual, tm_layout layout, const tm_shape *shape,
                                         const tm_swiglu_w8 *w, void *y, void *workspace, size_t workspace_bytes,
                                         void *stream);
 
 TM_API size_t tm_block_fp8_workspace_bytes(const tm_shape *shape, const tm_block_fp8 *block);
 
-/* One dense block as tm_block_forward, both sub-layers on the FP8 path.  X, Y [B,T,D];
- * X_revert_opt [B,T,D] receives X_rev when not NULL. */
+/* One dense block as tm_block_forward, both sub-layers on the FP8 path (in one launch when both
+ * have the same row width, T == H, as the bf16 block).  X, Y [B,T,D]; X_revert_opt [B,T,D]
+ * receives X_rev when not NULL. */
 TM_API tm_status tm_block_forward_fp8(const void *X, const tm_block_fp8 *block, const tm_shape *shape, void *Y,
                                       void *X_revert_opt, void *workspace, size_t workspace_bytes, void *stream);
 

@@ -354,7 +354,7 @@ tm_status fused_dense(const Geo& g, const void* x, const void* wg, const void* w
             tm_status s = cuda_status(cudaMemsetAsync(p.cnt, 0, n_rem * 8 * sizeof(int), st));
             if (s != TM_OK) return s;
         }
-        return cuda_status(launch_fused128(g.W, am, ma, mg, mu, md, mr, me, mo, p, grid, st));
+        return cuda_status(launch_fused128(g.W, am, false, ma, mg, mu, md, mr, me, mo, p, grid, st));
     }
     return cuda_status(launch_fused(g.W, am, ma, mg, mu, md, p, grid, st));
 }
@@ -648,6 +648,8 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
 }
 
 // ------------------------------------------------------------------ FP8 E4M3 dense sub-layer
+bool env_is(const char* name, char v);
+
 tm_status check_dense8(const Geo& g, const tm_swiglu_w8* w) {
     if (!w || w->banks != g.banks || w->width != g.W || w->hidden <= 0) return TM_ERR_INVALID_ARG;
     if (!w->q_gate || !w->q_up || !w->s_gate || !w->s_up || !w->w_down) return TM_ERR_INVALID_ARG;
@@ -659,48 +661,33 @@ tm_status check_dense8(const Geo& g, const tm_swiglu_w8* w) {
     return TM_OK;
 }
 
-struct Dense8Ws {
-    uint8_t* q;
-    float* rowscale;
-};
-Dense8Ws carve_dense8(Carve& c, const Geo& g) {
-    Dense8Ws w;
-    w.q = c.take<uint8_t>((size_t)g.B * g.banks * g.W);
-    w.rowscale = c.take<float>((size_t)g.B * g.banks);
-    return w;
+// E4M3 gate / up maps of a bank set: [banks * F rows, W] codes, 128 x 128 boxes
+bool maps_e4m3(const Geo& g, const tm_swiglu_w8* w, CUtensorMap* mg, CUtensorMap* mu) {
+    uint64_t dims[2] = {(uint64_t)g.W, (uint64_t)g.banks * w->hidden};
+    uint64_t strides[1] = {(uint64_t)g.W};
+    uint32_t box[2] = {128, 128};
+    return make_map_u8(mg, w->q_gate, 2, dims, strides, box) && make_map_u8(mu, w->q_up, 2, dims, strides, box);
 }
 
-// Quantize the activation rows, then one launch of the fused kernel in its FP8 mode.
+// One launch of the fused kernel in its FP8 mode: the kernel quantizes each A tile itself (row
+// statistics and E4M3 codes from the resident bf16 tile), so no workspace is needed.
 tm_status run_dense8(const Geo& g, const void* x, const void* resid, const void* extra, const tm_swiglu_w8* w, void* y,
-                     void* ws, size_t wsb, cudaStream_t st) {
-    Carve c{(uint8_t*)ws};
-    Dense8Ws d = carve_dense8(c, g);
-    if (!ws || wsb < c.off || !al16(ws)) return TM_ERR_WORKSPACE;
+                     cudaStream_t st) {
     if ((uintptr_t)y % 32) return TM_ERR_INVALID_ARG;
-    tm_status s;
-    if ((s = cuda_status(launch_quant_act_rows(x, g.map, g.B, g.eps, d.q, d.rowscale, st))) != TM_OK) return s;
     const int am = gemm1_amode(g), F = w->hidden;
     CUtensorMap ma, mg, mu, md, mr, me, mo;
     memset(&mr, 0, sizeof(mr));
     memset(&me, 0, sizeof(me));
-    {
-        uint64_t dims[3] = {(uint64_t)g.W, (uint64_t)g.banks, (uint64_t)g.B};
-        uint64_t strides[2] = {(uint64_t)g.W, (uint64_t)g.banks * g.W};
-        uint32_t box[3] = {128, 1, 128};
-        if (!make_map_u8(&ma, d.q, 3, dims, strides, box)) return TM_ERR_CUDA;
-    }
-    {
-        uint64_t dims[2] = {(uint64_t)g.W, (uint64_t)g.banks * F};
-        uint64_t strides[1] = {(uint64_t)g.W};
-        uint32_t box[2] = {128, 128};
-        if (!make_map_u8(&mg, w->q_gate, 2, dims, strides, box) || !make_map_u8(&mu, w->q_up, 2, dims, strides, box))
-            return TM_ERR_CUDA;
-    }
-    if (!map_2d(&md, w->w_down, (uint64_t)g.banks * g.W, F, g.W) || !gemm1_amap(g, y, am, &mo, 32)) return TM_ERR_CUDA;
-    if (resid && !gemm1_amap(g, resid, am, &mr)) return TM_ERR_CUDA;
-    if (extra && !gemm1_amap(g, extra, am, &me)) return TM_ERR_CUDA;
+    if (!gemm1_amap(g, x, am, &ma) || !maps_e4m3(g, w, &mg, &mu) || !map_2d(&md, w->w_down, (uint64_t)g.banks * g.W, F, g.W) ||
+        !gemm1_amap(g, y, am, &mo, 32))
+        return TM_ERR_CUDA;
     FusedParams p;
     memset(&p, 0, sizeof(p));
+    // residual: the A tile itself when it is the sub-layer input, else streamed; the inter-residual likewise
+    p.res_mode = resid == nullptr ? RES_NONE : resid == x ? RES_FROM_A : RES_STREAM;
+    p.has_extra = extra != nullptr;
+    if (p.res_mode == RES_STREAM && !gemm1_amap(g, resid, am, &mr)) return TM_ERR_CUDA;
+    if (extra && !gemm1_amap(g, extra, am, &me)) return TM_ERR_CUDA;
     p.banks = g.banks;
     p.rows = g.B;
     p.F = F;
@@ -709,14 +696,57 @@ tm_status run_dense8(const Geo& g, const void* x, const void* resid, const void*
     p.eps = g.eps;
     p.out = (__nv_bfloat16*)y;
     p.out_elems = (size_t)g.B * g.banks * g.W;
-    p.res_mode = resid ? RES_STREAM : RES_NONE;
-    p.has_extra = extra != nullptr;
-    p.rowscale = d.rowscale;
     p.s_gate = w->s_gate;
     p.s_up = w->s_up;
     const long tiles = (long)g.banks * ((g.B + 127) / 128);
     const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-    return cuda_status(launch_fused128(g.W, am == A_TMA_MIX ? A_F8MIX : A_F8ROW, ma, mg, mu, md, mr, me, mo, p, grid, st));
+    return cuda_status(launch_fused128(g.W, am, true, ma, mg, mu, md, mr, me, mo, p, grid, st));
+}
+
+// Both sub-layers of an FP8 block in one launch (block mode, as fused_block): same row width
+// (T == H), head width a multiple of 16.  counters: ceil(B/128) uint32 of workspace.
+bool block8_fusable(const Geo& gm, const Geo& gr, const void* Y, const void* Xr) {
+    if (gm.W != gr.W || gm.banks != gr.banks || gemm1_amode(gm) != A_TMA_MIX) return false;
+    if ((uintptr_t)Y % 32 || (uintptr_t)Xr % 32 || env_is("TM_FUSED_BLOCK", '0')) return false;
+    return true;
+}
+
+tm_status fused_block8(const tm_block_fp8* b, const Geo& gm, const Geo& gr, const void* X, void* Y, void* Xr,
+                       unsigned* dep, cudaStream_t st) {
+    const int W = gm.W, mt = (gm.B + 127) / 128;
+    tm_status s;
+    if ((s = cuda_status(cudaMemsetAsync(dep, 0, (size_t)mt * sizeof(unsigned), st))) != TM_OK) return s;
+    FusedMaps mm, mr;
+    CUtensorMap mres, mext;
+    memset(&mext, 0, sizeof(mext));
+    if (!gemm1_amap(gm, X, A_TMA_MIX, &mm.a) || !gemm1_amap(gm, Xr, A_TMA_MIX, &mm.o, 32) ||
+        !maps_e4m3(gm, &b->mix, &mm.g, &mm.u) || !map_2d(&mm.d, b->mix.w_down, (uint64_t)gm.banks * W, b->mix.hidden, W))
+        return TM_ERR_CUDA;
+    if (!gemm1_amap(gr, Xr, A_TMA_3D, &mr.a) || !gemm1_amap(gr, Y, A_TMA_3D, &mr.o, 32) ||
+        !maps_e4m3(gr, &b->rev, &mr.g, &mr.u) || !map_2d(&mr.d, b->rev.w_down, (uint64_t)gr.banks * W, b->rev.hidden, W) ||
+        !gemm1_amap(gr, X, A_TMA_3D, &mres))
+        return TM_ERR_CUDA;
+    FusedParams p;
+    memset(&p, 0, sizeof(p));
+    p.banks = gm.banks;
+    p.rows = gm.B;
+    p.F = b->mix.hidden;
+    p.F2 = b->rev.hidden;
+    p.amap = gm.map;
+    p.omap = gm.map;
+    p.eps = gm.eps;
+    p.out = (__nv_bfloat16*)Y;
+    p.out_elems = (size_t)gm.B * gm.banks * W;
+    p.res_mode = RES_FROM_A;
+    p.res_mode2 = RES_STREAM;
+    p.dep = dep;
+    p.s_gate = b->mix.s_gate;
+    p.s_up = b->mix.s_up;
+    p.s_gate2 = b->rev.s_gate;
+    p.s_up2 = b->rev.s_up;
+    const long tiles = 2L * gm.banks * mt;
+    const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+    return cuda_status(launch_fused128_block(W, true, mm, mr, mres, mext, p, grid, st));
 }
 
 // block geometry of the FP8 path
@@ -730,12 +760,9 @@ tm_status check_block8(const tm_shape* s, const tm_block_fp8* b, Geo* gm, Geo* g
     return st;
 }
 
-size_t block8_ws(const Geo& gm, const Geo& gr, const tm_shape* s) {
-    Carve a{nullptr}, b{nullptr};
-    carve_dense8(a, gm);
-    carve_dense8(b, gr);
-    const size_t sub = align256(a.off > b.off ? a.off : b.off);
-    return align256((size_t)s->B * s->T * s->D * 2) + sub;
+// workspace of an FP8 block: X_revert and the row-block counters of block mode
+size_t block8_ws(const Geo& gm, const Geo&, const tm_shape* s) {
+    return align256((size_t)s->B * s->T * s->D * 2) + align256((size_t)(gm.B + 127) / 128 * sizeof(unsigned));
 }
 
 // ------------------------------------------------------------------ sub-layer dispatch
@@ -883,7 +910,7 @@ tm_status fused_block(const tm_block* b, const Geo& gm, const Geo& gr, const voi
     p.dep = w.dep;
     const long tiles = 2L * gm.banks * mt;
     const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-    return cuda_status(launch_fused128_block(W, mm, mr, mres, mext, p, grid, st));
+    return cuda_status(launch_fused128_block(W, false, mm, mr, mres, mext, p, grid, st));
 }
 
 size_t stack_ws(const tm_shape* s, const tm_block* blocks, int L, int gap, bool* ok) {
@@ -1119,9 +1146,7 @@ tm_status tm_quantize_fp8_act(const void* x, tm_layout layout, const tm_shape* s
 size_t tm_pertoken_swiglu_fp8_workspace_bytes(const tm_shape* shape, tm_layout layout, const tm_swiglu_w8* w) {
     Geo g;
     if (!w || make_geo(shape, layout, w->banks, w->width, &g) != TM_OK || check_dense8(g, w) != TM_OK) return 0;
-    Carve c{nullptr};
-    carve_dense8(c, g);
-    return align256(c.off);
+    return 256;   // nothing is needed; a minimal size keeps the workspace convention of the ABI
 }
 
 tm_status tm_pertoken_swiglu_fp8(const void* x, const void* residual, tm_layout layout, const tm_shape* shape,
@@ -1132,7 +1157,8 @@ tm_status tm_pertoken_swiglu_fp8(const void* x, const void* residual, tm_layout 
     if (s != TM_OK) return s;
     if ((s = check_dense8(g, w)) != TM_OK) return s;
     if (!x || !y || x == y || !al16(x) || !al16(y) || (residual && !al16(residual))) return TM_ERR_INVALID_ARG;
-    return run_dense8(g, x, residual, nullptr, w, y, workspace, workspace_bytes, (cudaStream_t)stream);
+    if (!workspace || workspace_bytes < 256 || !al16(workspace)) return TM_ERR_WORKSPACE;
+    return run_dense8(g, x, residual, nullptr, w, y, (cudaStream_t)stream);
 }
 
 size_t tm_block_fp8_workspace_bytes(const tm_shape* shape, const tm_block_fp8* block) {
@@ -1151,14 +1177,13 @@ tm_status tm_block_forward_fp8(const void* X, const tm_block_fp8* block, const t
     if (!workspace || workspace_bytes < need || !al16(workspace)) return TM_ERR_WORKSPACE;
     Carve c{(uint8_t*)workspace};
     void* xr = c.take<uint8_t>((size_t)shape->B * shape->T * shape->D * 2);
+    unsigned* dep = c.take<unsigned>((size_t)(gm.B + 127) / 128);
     if (X_revert_opt) xr = X_revert_opt;
-    c.off = align256(c.off);
-    void* sub_ws = (uint8_t*)workspace + c.off;
-    const size_t sub_wsb = workspace_bytes - c.off;
     cudaStream_t st = (cudaStream_t)stream;
+    if (block8_fusable(gm, gr, Y, xr)) return fused_block8(block, gm, gr, X, Y, xr, dep, st);
     // H_next = FFN_mix(Norm(Mix(X))) + Mix(X) through Revert into X_rev; Y = FFN_rev(Norm(X_rev)) + X
-    if ((s = run_dense8(gm, X, X, nullptr, &block->mix, xr, sub_ws, sub_wsb, st)) != TM_OK) return s;
-    return run_dense8(gr, xr, X, nullptr, &block->rev, Y, sub_ws, sub_wsb, st);
+    if ((s = run_dense8(gm, X, X, nullptr, &block->mix, xr, st)) != TM_OK) return s;
+    return run_dense8(gr, xr, X, nullptr, &block->rev, Y, st);
 }
 
 tm_status tm_get_device_error(void* stream) {

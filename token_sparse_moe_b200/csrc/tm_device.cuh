@@ -302,6 +302,27 @@ __device__ __forceinline__ float2 swiglu2(float hs, float s, float2 g, float2 u)
     return __fmul2_rn(sl, __fmul2_rn(make_float2(s, s), u));
 }
 
+// ------------------------------------------------------------------ E4M3 (FP8 serving path)
+// Two fp32 values to two E4M3 codes (nearest, ties to even, saturating at +-448); the first
+// argument's code is the low byte.
+__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+// Power-of-two E4M3 scales: for a largest magnitude m > 0 the scale is 2^e with e the smallest
+// integer such that m * 2^-e <= 448; with m = f * 2^x, f in [0.5, 1) and 448 = 0.875 * 2^9 that
+// is e = x - 9 when f <= 0.875, else x - 8 (0 when m == 0).  Scaling by 2^-e is exact.
+__device__ __forceinline__ int pow2_exponent(float m) {
+    if (!(m > 0.f)) return 0;
+    int x;
+    const float f = frexpf(m, &x);
+    return f <= 0.875f ? x - 9 : x - 8;
+}
+__device__ __forceinline__ float pow2f(int k) {
+    return (k >= -126 && k <= 127) ? __int_as_float((127 + k) << 23) : ldexpf(1.f, k);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);

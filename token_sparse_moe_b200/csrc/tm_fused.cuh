@@ -38,11 +38,12 @@ struct FusedParams {
     int F2;                    // reverting hidden width
     int res_mode2, has_extra2; // reverting residual (streamed) and inter-residual
     unsigned* dep;             // [row tiles] finished-mixing-tile counters, zero at launch
-    // FP8 GEMM1 (128-wide-chunk kernel, A_F8MIX / A_F8ROW): per row (b * banks + bank) the factor
-    // (max|x| / 448) / rms(x), per bank the gate / up weight matrix scales
-    const float* rowscale;
+    // FP8 GEMM1 (128-wide-chunk kernel, F8): per bank the gate / up weight matrix scales of the
+    // (first) sub-layer, and of the reverting one in block mode
     const float* s_gate;
     const float* s_up;
+    const float* s_gate2;
+    const float* s_up2;
 };
 
 // Output epilogue of a fused tile for one thread: row b of bank g, columns [c_begin, c_begin + W/2).

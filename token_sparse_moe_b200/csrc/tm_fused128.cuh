@@ -45,28 +45,28 @@ namespace tml {
 
 enum FusedResid : int { RES_NONE = 0, RES_FROM_A = 1, RES_STREAM = 2 };
 constexpr int A_BLOCK = 4;   // fused128 kernel: a whole dense block (mixing tiles, then reverting tiles)
-// FP8 serving path of the fused sub-layer: A = E4M3 rows [B * banks, W] (quantized per row, read
-// through a 3-D map) and E4M3 gate / up weights, GEMM1 with kind::f8f6f4 MMAs; the SwiGLU takes
-// back the row factor and the bank's gate / up weight scales; GEMM2, the residual (always
-// streamed) and the output are those of the bf16 kernel, in the Mix geometry (A_F8MIX) or the
-// row one.
-constexpr int A_F8MIX = 5;
-constexpr int A_F8ROW = 6;
-
-template <int W, int AMODE>
+// FP8 serving path (F8 = true, any A mode): the bf16 A tile arrives as in the bf16 kernel; the
+// epilogue warps' statistics pass also takes each row's max|x| and writes the row's E4M3 codes
+// (its power-of-two scale, exact scaling) into an E4M3 copy of the tile, which GEMM1 reads with
+// kind::f8f6f4 MMAs against E4M3 gate / up weights; the SwiGLU takes back the row factor
+// 2^e / rms and the bank's gate / up weight scales.  GEMM2, the residual and the output are
+// those of the bf16 kernel.
+template <int W, int AMODE, bool F8 = false>
 struct Fused128Cfg {
     static_assert(W == 128 || W == 256, "fused sub-layer supports row widths 128 and 256");
-    static constexpr bool F8 = AMODE == A_F8MIX || AMODE == A_F8ROW;
-    static constexpr int A_BYTES = 128 * W * (F8 ? 1 : 2);
+    static constexpr int A_BYTES = 128 * W * 2;                   // the bf16 A tile, W / 64 slabs
+    static constexpr int A_SLABS = W / 64;
+    static constexpr int A8_BYTES = F8 ? 128 * W : 0;             // FP8: its E4M3 copy, W / 128 slabs of 128 columns
     static constexpr int HID_BYTES = 128 * 128 * 2;               // one 128-wide hidden chunk, 2 K-slabs
     static constexpr int SB = 32768;                              // ring stage
     static constexpr int G1_STAGES = F8 ? W / 128 : W / 64;       // 256 rows x 64 K (bf16) or 128 K (E4M3) per stage
     static constexpr int G2_STAGES = W == 256 ? 2 : 1;            // W rows x 128 K per chunk
     static constexpr int R_STAGES = W / 128;                      // residual tile: 128 rows x 128 columns per stage
-    static constexpr int STAGES = W == 256 ? 4 : 5;
+    static constexpr int STAGES = F8 ? (W == 256 ? 3 : 4) : (W == 256 ? 4 : 5);
     static constexpr int NTHREADS = 10 * 32;
-    static constexpr int OFF_HID = A_BYTES;
-    static constexpr int OFF_RING = A_BYTES + HID_BYTES;
+    static constexpr int OFF_A8 = A_BYTES;
+    static constexpr int OFF_HID = A_BYTES + A8_BYTES;
+    static constexpr int OFF_RING = OFF_HID + HID_BYTES;
     static constexpr int OFF_ID = OFF_RING + STAGES * SB;         // 16 x 16 identity, 32-byte swizzled K-major
     static constexpr int OFF_XCH = OFF_ID + 512;                  // row statistics exchange, 2 x 128 floats
     static constexpr int OFF_BAR = OFF_XCH + 1024;
@@ -101,7 +101,7 @@ struct F128Item {
 
 // The kernel body; the tensor maps are the kernel's __grid_constant__ parameters, passed by
 // reference so that the bulk tensor instructions see their parameter-space addresses.
-template <int W, int AMODE>
+template <int W, int AMODE, bool F8>
 __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUtensorMap& tmG, const CUtensorMap& tmU,
                                               const CUtensorMap& tmD, const CUtensorMap& tmR, const CUtensorMap& tmE,
                                               const CUtensorMap& tmO, const CUtensorMap& tmA2, const CUtensorMap& tmG2,
@@ -110,10 +110,9 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
     // Maps: A, G, U, D, O of the (first) sub-layer; R / E the streamed residual and inter-residual
     // (in block mode those of the reverting sub-layer); A2, G2, U2, D2, O2 the reverting
     // sub-layer's in block mode (unused otherwise).
-    using C = Fused128Cfg<W, AMODE>;
+    using C = Fused128Cfg<W, AMODE, F8>;
     constexpr bool BLK = AMODE == A_BLOCK;
-    constexpr bool F8 = C::F8;
-    constexpr bool MIXG = AMODE == A_TMA_MIX || AMODE == A_F8MIX;   // Mix geometry outside block mode
+    constexpr bool MIXG = AMODE == A_TMA_MIX;                       // Mix geometry outside block mode
     constexpr int STAGES = C::STAGES;
     const int mt = (p.rows + 127) / 128;
     const int ntile1 = p.banks * mt;                 // tiles of one sub-layer
@@ -181,6 +180,7 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
+    uint8_t* sA8 = smem + C::OFF_A8;
     uint8_t* sH = smem + C::OFF_HID;
     uint8_t* sR = smem + C::OFF_RING;
     uint8_t* sI = smem + C::OFF_ID;
@@ -188,8 +188,8 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
     uint64_t* full = bar;                  // [STAGES]
     uint64_t* empty = full + STAGES;       // [STAGES]
     uint64_t* a_full = empty + STAGES;
-    uint64_t* a_empty = a_full + 1;        // [G1_STAGES]: one per 64-column slab of A
-    uint64_t* g1_full = a_empty + C::G1_STAGES;
+    uint64_t* a_empty = a_full + 1;        // [A_SLABS]: one per 64-column slab of A
+    uint64_t* g1_full = a_empty + C::A_SLABS;
     uint64_t* g1_empty = g1_full + 1;
     uint64_t* hid_full = g1_empty + 1;
     uint64_t* hid_empty = hid_full + 1;
@@ -198,7 +198,9 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
     uint64_t* drain = y_empty + 1;
     uint64_t* stats_bar = drain + 1;       // both halves' partial row sums written
     uint64_t* stats_done = stats_bar + 1;  // both halves' partial row sums read
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stats_done + 1);
+    uint64_t* a8_full = stats_done + 1;    // FP8: the tile's E4M3 codes written (8 epilogue warps)
+    uint64_t* a8_empty = a8_full + 1;      // FP8: the item's GEMM1s are done with them
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(a8_empty + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -209,8 +211,11 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
             mbar_init(&empty[s], 1);
         }
         mbar_init(a_full, 1);
-        // per slab of A: the MMA (last read issued) + the 4 epilogue warps of the half that reads it
-        for (int q = 0; q < C::G1_STAGES; ++q) mbar_init(&a_empty[q], F8 ? 1 : 1 + 4);
+        // per slab of A: the MMA (last read issued) + the epilogue warps that read it (the 4 of the
+        // half on the bf16 path; all 8 on the FP8 path, whose statistics read whole rows)
+        for (int q = 0; q < C::A_SLABS; ++q) mbar_init(&a_empty[q], F8 ? 1 + 8 : 1 + 4);
+        mbar_init(a8_full, 8);
+        mbar_init(a8_empty, 1);
         mbar_init(g1_full, 1);
         mbar_init(g1_empty, 8);
         mbar_init(hid_full, 8);
@@ -308,11 +313,10 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
                 if (BLK && it.sec && !wait_block(m)) break;
                 // A slab by slab, each as soon as the previous tile has released it
 #pragma unroll 1
-                for (int qa = 0; qa < C::G1_STAGES && ok; ++qa) {
+                for (int qa = 0; qa < C::A_SLABS && ok; ++qa) {
                     if (!wait_or_abort(&a_empty[qa], (lt & 1) ^ 1, abort_flag, 0x3100)) { ok = false; break; }
                     if (qa == 0) mbar_arrive_expect_tx(a_full, C::A_BYTES);
-                    if (F8) tma_load_3d(sA + qa * 16384, mA, a_full, qa * 128, g, m * 128);   // 128 E4M3 columns
-                    else load_rows(mA, mx, sA + qa * 16384, a_full, g, m * 128, qa * 4, 4);
+                    load_rows(mA, mx, sA + qa * 16384, a_full, g, m * 128, qa * 4, 4);
                 }
                 if (!ok) break;
                 // ring order per step: G1(step) (step < NC), G2(step - LAG) (step >= LAG), and at step
@@ -382,6 +386,11 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
             };
             set_adesc(AMODE == A_TMA_MIX);
             const uint64_t hdesc0 = umma_sdesc_sw128(hS), hdesc1 = umma_sdesc_sw128(hS + 16384);
+            // FP8: the E4M3 copy of A, 128-column slabs with 128-byte swizzle, 32 columns per MMA
+            uint64_t a8desc[F8 ? W / 32 : 1];
+#pragma unroll
+            for (int k = 0; k < (F8 ? W / 32 : 1); ++k)
+                a8desc[k] = umma_sdesc_sw128(smem_u32(sA8) + (k >> 2) * 16384) + 2 * (k & 3);
             const uint64_t rdesc0 = umma_sdesc_sw128(rS);
             const uint64_t rdesc32 = umma_sdesc_sw32(rS);
             const uint64_t idB = umma_sdesc_sw32(smem_u32(sI));
@@ -398,9 +407,17 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
                 const int rm = rmode(it), res_stages = n_res(it), ext_stages = n_ext(it);
                 if (BLK) set_adesc(mx);
                 // A is released slab by slab after the item's last GEMM1, or after the identity pass
-                // when that reads A and comes later
-                const bool a_after_id = rm == RES_FROM_A && s_r >= nc - 1;
+                // when that reads A and comes later.  FP8: GEMM1 reads the E4M3 copy, so the bf16 tile
+                // is released after the identity pass when that reads it, else at once.
+                const bool a_after_id = rm == RES_FROM_A && (F8 || s_r >= nc - 1);
                 if (!wait_or_abort(a_full, lt & 1, abort_flag, 0x3200)) break;
+                if (F8) {
+                    if (!a_after_id) {
+#pragma unroll
+                        for (int q = 0; q < C::A_SLABS; ++q) umma_commit(&a_empty[q]);
+                    }
+                    if (!wait_or_abort(a8_full, lt & 1, abort_flag, 0x3208)) break;   // the item's E4M3 codes
+                }
                 tc_fence_after();
 #pragma unroll 1
                 for (int step = 0; step < n_steps && ok; ++step) {
@@ -428,14 +445,15 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
                             const uint64_t bd = rdesc0 + (uint64_t)s * kStageDesc;
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
-                                if (F8) umma_e4m3(tmem + C::G1COL, adesc[q * 4 + kk], bd + 2 * kk, idesc1, (q | kk) != 0);
+                                if (F8) umma_e4m3(tmem + C::G1COL, a8desc[q * 4 + kk], bd + 2 * kk, idesc1, (q | kk) != 0);
                                 else umma_bf16(tmem + C::G1COL, adesc[q * 4 + kk], bd + 2 * kk, idesc1, (q | kk) != 0);
                             umma_commit(&empty[s]);
-                            if (step == nc - 1 && !a_after_id) umma_commit(&a_empty[q]);
+                            if (!F8 && step == nc - 1 && !a_after_id) umma_commit(&a_empty[q]);
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                         if (!ok) break;
                         umma_commit(g1_full);
+                        if (F8 && step == nc - 1) umma_commit(a8_empty);   // the E4M3 copy is free
                     }
                     if (step >= LAG) {                                 // ---- GEMM2(c0 + step - LAG)
                         const int c = step - LAG;                      // relative to c0
@@ -484,7 +502,7 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
                             for (int k16 = 0; k16 < W / 16; ++k16) umma_bf16(tmem + 16 * k16, adesc[k16], idB, idescI, 1);
                             if (a_after_id) {
 #pragma unroll
-                                for (int q = 0; q < C::G1_STAGES; ++q) umma_commit(&a_empty[q]);
+                                for (int q = 0; q < C::A_SLABS; ++q) umma_commit(&a_empty[q]);
                             }
                         }
 #pragma unroll 1
@@ -584,6 +602,56 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
             if (lane == 0) mbar_arrive(stats_done);
             ++n_stats;
             out = r < p.rows - m_tile * 128 ? 1.0f / sqrtf(tot / (float)W + p.eps) : 0.f;
+            return true;
+        };
+        // FP8: 8 bf16 of row r at column col (a multiple of 8) of the A tile, in either geometry
+        auto a_chunk = [&](bool mx, int col) -> uint4 {
+            if (mx)   // 16-column boxes of 128 rows x 32 bytes, 32-byte swizzle
+                return *reinterpret_cast<const uint4*>(sA + (col >> 4) * 4096 + r * 32 +
+                                                       ((((col >> 3) & 1) ^ ((r >> 2) & 1)) << 4));
+            return *reinterpret_cast<const uint4*>(sA + (col >> 6) * 16384 + r * 128 +   // 64-column slabs, 128-byte swizzle
+                                                   ((((col >> 3) & 7) ^ (r & 7)) << 4));
+        };
+        // FP8: the row's statistics over the whole row (both threads of a row sum in the same order,
+        // so they agree without an exchange), then this thread's half of the row as E4M3 codes in
+        // the tile's E4M3 copy (128-column slabs, 128-byte swizzle) with the row's power-of-two
+        // scale 2^e (the smallest with max|x| * 2^-e <= 448); out = 2^e / rms(x)
+        int n_q = 0;
+        auto row_scale8 = [&](int m_tile, bool mx, float& out) -> bool {
+            float ss = 0.f, amax = 0.f;
+#pragma unroll 4
+            for (int col = 0; col < W; col += 8) {
+                const uint4 w4 = a_chunk(mx, col);
+                const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float lo = bf16_lo(wv[e]), hi = bf16_hi(wv[e]);
+                    ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+                    amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+                }
+            }
+            const int ex = pow2_exponent(amax);
+            const float inv = pow2f(-ex);
+            // the previous item's GEMM1s are done with the E4M3 copy
+            if (n_q > 0 && !wait_or_abort(a8_empty, (n_q - 1) & 1, abort_flag, 0x3307)) return false;
+#pragma unroll 2
+            for (int col = half * (W / 2); col < (half + 1) * (W / 2); col += 16) {
+                const uint4 lo4 = a_chunk(mx, col), hi4 = a_chunk(mx, col + 8);
+                const uint32_t av[8] = {lo4.x, lo4.y, lo4.z, lo4.w, hi4.x, hi4.y, hi4.z, hi4.w};
+                uint32_t q4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    q4[e] = uint32_t(e4m3x2(bf16_lo(av[2 * e]) * inv, bf16_hi(av[2 * e]) * inv)) |
+                            (uint32_t(e4m3x2(bf16_lo(av[2 * e + 1]) * inv, bf16_hi(av[2 * e + 1]) * inv)) << 16);
+                const int k = (col & 127) >> 4;
+                *reinterpret_cast<uint4*>(sA8 + (col >> 7) * 16384 + r * 128 + ((k ^ (r & 7)) << 4)) =
+                    make_uint4(q4[0], q4[1], q4[2], q4[3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(a8_full);
+            ++n_q;
+            out = r < p.rows - m_tile * 128 ? pow2f(ex) * (1.0f / sqrtf(ss / (float)W + p.eps)) : 0.f;
             return true;
         };
         // Y of tile (g, m) (residual already accumulated) -> bf16 -> this warp's rows of the idle hidden
@@ -732,23 +800,22 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
         };
         int lt = 0;
         float sc = 0.f;
-        // the statistics of a tile read the A slabs of this thread's half; release them afterwards
-        // (the FP8 path reads no A slab: its row factor comes with the quantized rows)
+        // the statistics of a tile read the A slabs of this thread's half (FP8: of its whole row);
+        // release them afterwards
         auto release_a = [&]() {
-            if (F8) return;
             __syncwarp();
             if (lane == 0) {
+                if (F8) {
 #pragma unroll
-                for (int qa = 0; qa < C::G1_STAGES / 2; ++qa) mbar_arrive(&a_empty[half * (C::G1_STAGES / 2) + qa]);
+                    for (int qa = 0; qa < C::A_SLABS; ++qa) mbar_arrive(&a_empty[qa]);
+                } else {
+#pragma unroll
+                    for (int qa = 0; qa < C::A_SLABS / 2; ++qa) mbar_arrive(&a_empty[half * (C::A_SLABS / 2) + qa]);
+                }
             }
         };
         auto tile_scale = [&](const F128Item& t_it, float& out) -> bool {
-            if (F8) {
-                const int b = t_it.m * 128 + r;
-                out = b < p.rows ? __ldg(&p.rowscale[(size_t)b * p.banks + t_it.g]) : 0.f;
-                return true;
-            }
-            return row_scale(t_it.m, amix(t_it), out);
+            return F8 ? row_scale8(t_it.m, amix(t_it), out) : row_scale(t_it.m, amix(t_it), out);
         };
 
         F128Item it;
@@ -764,7 +831,8 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
         uint32_t ubase = 0;                                            // chunks of the items before this one
         for (; ok && have; ++lt) {
             const int c0 = it.c0, c1 = it.c1;
-            const float sgw = F8 ? __ldg(&p.s_gate[it.g]) : 1.f, suw = F8 ? __ldg(&p.s_up[it.g]) : 1.f;
+            const float sgw = F8 ? __ldg(&(BLK && it.sec ? p.s_gate2 : p.s_gate)[it.g]) : 1.f;
+            const float suw = F8 ? __ldg(&(BLK && it.sec ? p.s_up2 : p.s_up)[it.g]) : 1.f;
             // ---- SwiGLU chunks: this thread owns hidden columns [half*64, half*64 + 64) of its row
 #pragma unroll 1
             for (int c = c0; c < c1; ++c) {
@@ -853,8 +921,8 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
     }
 }
 
-template <int W, int AMODE>
-__global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
+template <int W, int AMODE, bool F8 = false>
+__global__ void __launch_bounds__(Fused128Cfg<W, AMODE, F8>::NTHREADS, 1)
     fused128_swiglu_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
                            const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmD,
                            const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmE,
@@ -862,7 +930,7 @@ __global__ void __launch_bounds__(Fused128Cfg<W, AMODE>::NTHREADS, 1)
                            const __grid_constant__ CUtensorMap tmG2, const __grid_constant__ CUtensorMap tmU2,
                            const __grid_constant__ CUtensorMap tmD2, const __grid_constant__ CUtensorMap tmO2,
                            const FusedParams p) {
-    fused128_body<W, AMODE>(tmA, tmG, tmU, tmD, tmR, tmE, tmO, tmA2, tmG2, tmU2, tmD2, tmO2, p);
+    fused128_body<W, AMODE, F8>(tmA, tmG, tmU, tmD, tmR, tmE, tmO, tmA2, tmG2, tmU2, tmD2, tmO2, p);
 }
 
 }  // namespace tml

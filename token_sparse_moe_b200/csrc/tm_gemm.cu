@@ -22,30 +22,30 @@ static cudaError_t launch_fused_one(const CUtensorMap& a, const CUtensorMap& g, 
     return cudaGetLastError();
 }
 
-template <int W, int AM>
+template <int W, int AM, bool F8>
 static cudaError_t launch_fused128_one(const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
                                        const CUtensorMap& d, const CUtensorMap& r, const CUtensorMap& e,
                                        const CUtensorMap& o, const FusedParams& p, int grid, cudaStream_t st) {
-    using C = Fused128Cfg<W, AM>;
-    auto kern = fused128_swiglu_kernel<W, AM>;
+    using C = Fused128Cfg<W, AM, F8>;
+    auto kern = fused128_swiglu_kernel<W, AM, F8>;
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    ProfileScope ps_(C::F8 ? "fused_swiglu_fp8" : "fused_swiglu", st);
+    ProfileScope ps_(F8 ? "fused_swiglu_fp8" : "fused_swiglu", st);
     kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, g, u, d, r, e, o, a, g, u, d, o, p);
     return cudaGetLastError();
 }
 
 // A whole dense block in one launch.  Cooperative, so that all CTAs are resident together: a
 // reverting tile waits for mixing tiles that other CTAs run.
-template <int W>
+template <int W, bool F8>
 static cudaError_t launch_fused128_block_one(const FusedMaps& mix, const FusedMaps& rev, const CUtensorMap& r,
                                              const CUtensorMap& e, const FusedParams& p, int grid, cudaStream_t st) {
-    using C = Fused128Cfg<W, A_BLOCK>;
-    auto kern = fused128_swiglu_kernel<W, A_BLOCK>;
+    using C = Fused128Cfg<W, A_BLOCK, F8>;
+    auto kern = fused128_swiglu_kernel<W, A_BLOCK, F8>;
     static bool configured = false;
     if (!configured) {
         cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -63,28 +63,28 @@ static cudaError_t launch_fused128_block_one(const FusedMaps& mix, const FusedMa
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    ProfileScope ps_("fused_swiglu", st);
+    ProfileScope ps_(F8 ? "fused_swiglu_fp8" : "fused_swiglu", st);
     return cudaLaunchKernelEx(&cfg, kern, mix.a, mix.g, mix.u, mix.d, r, e, mix.o, rev.a, rev.g, rev.u, rev.d, rev.o, p);
 }
 
-cudaError_t launch_fused128_block(int W, const FusedMaps& mix, const FusedMaps& rev, const CUtensorMap& r,
+cudaError_t launch_fused128_block(int W, bool f8, const FusedMaps& mix, const FusedMaps& rev, const CUtensorMap& r,
                                   const CUtensorMap& e, const FusedParams& p, int grid, cudaStream_t st) {
-    if (W == 256) return launch_fused128_block_one<256>(mix, rev, r, e, p, grid, st);
-    if (W == 128) return launch_fused128_block_one<128>(mix, rev, r, e, p, grid, st);
+    if (W == 256) return f8 ? launch_fused128_block_one<256, true>(mix, rev, r, e, p, grid, st)
+                            : launch_fused128_block_one<256, false>(mix, rev, r, e, p, grid, st);
+    if (W == 128) return f8 ? launch_fused128_block_one<128, true>(mix, rev, r, e, p, grid, st)
+                            : launch_fused128_block_one<128, false>(mix, rev, r, e, p, grid, st);
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_fused128(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
-                            const CUtensorMap& d, const CUtensorMap& r, const CUtensorMap& e, const CUtensorMap& o,
-                            const FusedParams& p, int grid, cudaStream_t st) {
-    if (W == 256 && a_mode == A_TMA_MIX) return launch_fused128_one<256, A_TMA_MIX>(a, g, u, d, r, e, o, p, grid, st);
-    if (W == 256 && a_mode == A_TMA_3D) return launch_fused128_one<256, A_TMA_3D>(a, g, u, d, r, e, o, p, grid, st);
-    if (W == 128 && a_mode == A_TMA_MIX) return launch_fused128_one<128, A_TMA_MIX>(a, g, u, d, r, e, o, p, grid, st);
-    if (W == 128 && a_mode == A_TMA_3D) return launch_fused128_one<128, A_TMA_3D>(a, g, u, d, r, e, o, p, grid, st);
-    if (W == 256 && a_mode == A_F8MIX) return launch_fused128_one<256, A_F8MIX>(a, g, u, d, r, e, o, p, grid, st);
-    if (W == 256 && a_mode == A_F8ROW) return launch_fused128_one<256, A_F8ROW>(a, g, u, d, r, e, o, p, grid, st);
-    if (W == 128 && a_mode == A_F8MIX) return launch_fused128_one<128, A_F8MIX>(a, g, u, d, r, e, o, p, grid, st);
-    if (W == 128 && a_mode == A_F8ROW) return launch_fused128_one<128, A_F8ROW>(a, g, u, d, r, e, o, p, grid, st);
+cudaError_t launch_fused128(int W, int a_mode, bool f8, const CUtensorMap& a, const CUtensorMap& g,
+                            const CUtensorMap& u, const CUtensorMap& d, const CUtensorMap& r, const CUtensorMap& e,
+                            const CUtensorMap& o, const FusedParams& p, int grid, cudaStream_t st) {
+#define TM_F128(WW, AMM)                                                                                      \
+    if (W == WW && a_mode == AMM)                                                                             \
+        return f8 ? launch_fused128_one<WW, AMM, true>(a, g, u, d, r, e, o, p, grid, st)                      \
+                  : launch_fused128_one<WW, AMM, false>(a, g, u, d, r, e, o, p, grid, st);
+    TM_F128(256, A_TMA_MIX) TM_F128(256, A_TMA_3D) TM_F128(128, A_TMA_MIX) TM_F128(128, A_TMA_3D)
+#undef TM_F128
     return cudaErrorInvalidValue;
 }
 

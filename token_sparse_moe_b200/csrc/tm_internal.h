@@ -48,9 +48,10 @@ cudaError_t launch_fused(int W, int a_mode, const CUtensorMap& a, const CUtensor
 // 128-wide hidden chunks (F % 128 == 0); gate/up maps with 128-row boxes; r / e: residual and
 // inter-residual maps in the geometry of a (read when p.res_mode == RES_STREAM / p.has_extra);
 // o: the output in the geometry of a with 32-row boxes
-cudaError_t launch_fused128(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
-                            const CUtensorMap& d, const CUtensorMap& r, const CUtensorMap& e, const CUtensorMap& o,
-                            const FusedParams& p, int grid, cudaStream_t st);
+// f8: the FP8 serving path (E4M3 gate / up maps, scales in p.s_gate / p.s_up)
+cudaError_t launch_fused128(int W, int a_mode, bool f8, const CUtensorMap& a, const CUtensorMap& g,
+                            const CUtensorMap& u, const CUtensorMap& d, const CUtensorMap& r, const CUtensorMap& e,
+                            const CUtensorMap& o, const FusedParams& p, int grid, cudaStream_t st);
 // The maps of one sub-layer of a fused block: A (input rows), gate, up, down, output.
 struct FusedMaps {
     CUtensorMap a, g, u, d, o;
@@ -59,7 +60,7 @@ struct FusedMaps {
 // geometry (output through the Revert map into X_revert), rev in the row geometry over X_revert;
 // r / e: the reverting sub-layer's residual (X) and inter-residual; p.dep: [ceil(B/128)] zeroed
 // counters; grid <= the number of SMs.
-cudaError_t launch_fused128_block(int W, const FusedMaps& mix, const FusedMaps& rev, const CUtensorMap& r,
+cudaError_t launch_fused128_block(int W, bool f8, const FusedMaps& mix, const FusedMaps& rev, const CUtensorMap& r,
                                   const CUtensorMap& e, const FusedParams& p, int grid, cudaStream_t st);
 // CTA-pair version (2-SM MMAs, clusters of 2): grid = 2 x clusters; weight maps with half-size boxes
 cudaError_t launch_fused2(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
