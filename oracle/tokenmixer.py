@@ -264,3 +264,22 @@ def tokenize(groups: np.ndarray, w_group: np.ndarray, w_global: np.ndarray) -> n
     for i in range(G):
         X[:, i + 1, :] = groups[:, i, :] @ w_group[i].T            # Eq. 2
     return X
+
+
+# ------------------------------------------------------------------ model head and end-to-end scoring
+def head(X: np.ndarray, w_head: np.ndarray) -> np.ndarray:
+    """Scoring head of the model.  [readme] block diagram: mean-pool over tokens, then a
+    projection head to one logit per sample (bias off, as the reproduction's default).
+    X [B, T, D], w_head [D]  ->  logits [B]."""
+    return X.mean(axis=1) @ w_head
+
+
+def model_forward(groups: np.ndarray, w_group: np.ndarray, w_global: np.ndarray, cfg,
+                  bank_w: Callable[[int, int, int], Weights], w_head: np.ndarray, storage=None) -> Dict[str, np.ndarray]:
+    """End-to-end scoring of a batch: tokenizer (Eq. 2-4) -> blocks with the inter-residual ->
+    head.  With `storage` the token tensor is stored once in the model dtype before the stack,
+    as the blocks' stored tensors are."""
+    rnd = storage_round(storage)
+    X = rnd(tokenize(groups, w_group, w_global))
+    st = stack_forward(X, cfg, bank_w, storage=storage)
+    return {"X": X, "Y": st["Y"], "logits": head(st["Y"], w_head)}
