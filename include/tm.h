@@ -130,6 +130,24 @@ TM_API tm_status tm_tokenize_stub(const void *groups, const void *w_group, const
  * X [B,T,D] -> Hm [B, H, T*D/H].  A test/API utility: the fused path never calls it. */
 TM_API tm_status tm_mix(const void *X, void *Hm, const tm_shape *shape, void *stream);
 
+/* Scoring head ([readme] block diagram: "mean-pool over tokens -> projection head -> logit",
+ * bias off as the reproduction's default): logits[b] = (1/T) sum_t sum_d X[b,t,d] * w_head[d],
+ * fp32 accumulation.  X [B,T,D] and w_head [D] in the shape's dtype; logits [B] fp32.
+ * An HBM-bound reduction kernel (one warp per sample). */
+TM_API tm_status tm_head_forward(const void *X, const tm_shape *shape, const void *w_head, float *logits,
+                                 void *stream);
+
+/* Workspace bytes needed by tm_model_forward. */
+TM_API size_t tm_model_workspace_bytes(const tm_shape *shape, const tm_block *blocks, int L, int inter_residual_gap);
+
+/* End-to-end scoring of a batch: tm_tokenize_stub -> tm_stack_forward -> tm_head_forward
+ * (groups [B,T-1,dg], w_group, w_global as tm_tokenize_stub; blocks, L, gap as
+ * tm_stack_forward; w_head [D]); logits [B] fp32.  The token tensors live in the workspace. */
+TM_API tm_status tm_model_forward(const void *groups, const void *w_group, const void *w_global, int dg,
+                                  const tm_block *blocks, int L, int inter_residual_gap, const void *w_head,
+                                  const tm_shape *shape, float *logits, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
 /* Revert ([digest] 2.3.1, Eq. 13-15), the inverse of Mix: Hm [B,H,T*D/H] -> X [B,T,D]. */
 TM_API tm_status tm_revert(const void *Hm, void *X, const tm_shape *shape, void *stream);
 

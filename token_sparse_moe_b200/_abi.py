@@ -19,7 +19,7 @@ EXPORTS = ["tm_status_string", "tm_version", "tm_sublayer_workspace_bytes", "tm_
            "tm_profile_start", "tm_profile_stop", "tm_last_cuda_error", "tm_launch_count",
            "tm_get_device_error", "tm_quantize_fp8_weights", "tm_quantize_fp8_act",
            "tm_pertoken_swiglu_fp8_workspace_bytes", "tm_pertoken_swiglu_fp8", "tm_block_fp8_workspace_bytes",
-           "tm_block_forward_fp8"]
+           "tm_block_forward_fp8", "tm_head_forward", "tm_model_workspace_bytes", "tm_model_forward"]
 
 
 class tm_shape(ctypes.Structure):
@@ -88,6 +88,10 @@ _SIGS = {
     "tm_pertoken_swiglu_fp8": (c_int, [_P, _P, c_int, POINTER(tm_shape), POINTER(tm_swiglu_w8), _P, _P, c_size_t, _P]),
     "tm_block_fp8_workspace_bytes": (c_size_t, [POINTER(tm_shape), POINTER(tm_block_fp8)]),
     "tm_block_forward_fp8": (c_int, [_P, POINTER(tm_block_fp8), POINTER(tm_shape), _P, _P, _P, c_size_t, _P]),
+    "tm_head_forward": (c_int, [_P, POINTER(tm_shape), _P, _P, _P]),
+    "tm_model_workspace_bytes": (c_size_t, [POINTER(tm_shape), POINTER(tm_block), c_int, c_int]),
+    "tm_model_forward": (c_int, [_P, _P, _P, c_int, POINTER(tm_block), c_int, c_int, _P, POINTER(tm_shape), _P, _P,
+                                 c_size_t, _P]),
 }
 
 _lib = None

@@ -275,6 +275,29 @@ def stack_forward(X, blocks: Sequence[Block], gap: int, sh: A.tm_shape, Y=None, 
     return StackRunner(blocks, sh, gap, X.device)(X, Y, stream)
 
 
+# ------------------------------------------------------------------ scoring head and end-to-end model
+def head_forward(X: torch.Tensor, sh: A.tm_shape, w_head: torch.Tensor, stream=None) -> torch.Tensor:
+    """tm_head_forward: X [B,T,D] -> logits [B] fp32 (mean over tokens, then w_head [D])."""
+    logits = torch.empty((sh.B,), dtype=torch.float32, device=X.device)
+    A.check(lib().tm_head_forward(_p(X), ctypes.byref(sh), _p(w_head), _p(logits), _s(stream)), "tm_head_forward")
+    return logits
+
+
+def model_forward(groups, w_group, w_global, blocks: Sequence[Block], gap: int, w_head, sh: A.tm_shape,
+                  stream=None) -> torch.Tensor:
+    """tm_model_forward: tokenizer -> stack -> head; returns logits [B] fp32."""
+    arr = (A.tm_block * len(blocks))(*[b.c() for b in blocks])
+    n = lib().tm_model_workspace_bytes(ctypes.byref(sh), arr, len(blocks), gap)
+    if n == 0:
+        raise A.TMError(A.TM_ERR_INVALID_ARG, "tm_model_workspace_bytes")
+    ws = torch.empty(n, dtype=torch.uint8, device=groups.device)
+    logits = torch.empty((sh.B,), dtype=torch.float32, device=groups.device)
+    A.check(lib().tm_model_forward(_p(groups), _p(w_group), _p(w_global), groups.shape[-1], arr, len(blocks), gap,
+                                   _p(w_head), ctypes.byref(sh), _p(logits), _p(ws), ws.numel(), _s(stream)),
+            "tm_model_forward")
+    return logits
+
+
 # ------------------------------------------------------------------ FP8 E4M3 serving path
 def quantize_fp8_weights(w: torch.Tensor, gain: Optional[torch.Tensor] = None, stream=None):
     """tm_quantize_fp8_weights: bf16 [groups, rows, cols] matrices -> (E4M3 codes as uint8 of the

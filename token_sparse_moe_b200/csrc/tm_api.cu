@@ -995,6 +995,37 @@ tm_status tm_tokenize_stub(const void* groups, const void* w_group, const void* 
                                        (cudaStream_t)stream));
 }
 
+tm_status tm_head_forward(const void* X, const tm_shape* shape, const void* w_head, float* logits, void* stream) {
+    tm_status s = check_shape(shape);
+    if (s != TM_OK) return s;
+    if (!X || !w_head || !logits || !al16(X) || !al16(w_head) || (reinterpret_cast<uintptr_t>(logits) & 3))
+        return TM_ERR_INVALID_ARG;
+    return cuda_status(launch_head(shape->dtype, X, w_head, shape->B, shape->T, shape->D, logits, (cudaStream_t)stream));
+}
+
+size_t tm_model_workspace_bytes(const tm_shape* shape, const tm_block* blocks, int L, int gap) {
+    const size_t st = tm_workspace_bytes(shape, blocks, L, gap);
+    if (st == 0) return 0;
+    const size_t tok = align256((size_t)shape->B * shape->T * shape->D * (shape->dtype == TM_BF16 ? 2 : 4));
+    return 2 * tok + st;
+}
+
+tm_status tm_model_forward(const void* groups, const void* w_group, const void* w_global, int dg, const tm_block* blocks,
+                           int L, int gap, const void* w_head, const tm_shape* shape, float* logits, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    const size_t need = tm_model_workspace_bytes(shape, blocks, L, gap);
+    if (need == 0) return TM_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < need || !al16(workspace)) return TM_ERR_WORKSPACE;
+    const size_t tok = align256((size_t)shape->B * shape->T * shape->D * (shape->dtype == TM_BF16 ? 2 : 4));
+    uint8_t* X = (uint8_t*)workspace;
+    uint8_t* Y = X + tok;
+    tm_status s;
+    if ((s = tm_tokenize_stub(groups, w_group, w_global, dg, shape, X, stream)) != TM_OK) return s;
+    if ((s = tm_stack_forward(X, blocks, L, gap, shape, Y, Y + tok, workspace_bytes - 2 * tok, stream)) != TM_OK)
+        return s;
+    return tm_head_forward(Y, shape, w_head, logits, stream);
+}
+
 tm_status tm_mix(const void* X, void* Hm, const tm_shape* shape, void* stream) {
     tm_status s = check_shape(shape);
     if (s != TM_OK) return s;

@@ -100,6 +100,8 @@ cudaError_t launch_permute(int dtype, const void* src, void* dst, int B, int T, 
                            cudaStream_t st);
 cudaError_t launch_fold_gain(int dtype, const void* w, const void* gain, void* out, size_t rows, int width,
                              cudaStream_t st);
+// scoring head: logits [B] fp32 = mean over tokens of X [B,T,D] projected on w [D]
+cudaError_t launch_head(int dtype, const void* X, const void* w, int B, int T, int D, float* logits, cudaStream_t st);
 cudaError_t launch_tokenize(int dtype, const void* groups, const void* w_group, const void* w_global, int dg, int B,
                             int T, int D, void* X, cudaStream_t st);
 

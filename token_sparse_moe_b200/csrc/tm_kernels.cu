@@ -654,6 +654,35 @@ cudaError_t launch_fold_gain(int dtype, const void* w, const void* gain, void* o
     return cudaGetLastError();
 }
 
+// Scoring head ([readme] block diagram: mean-pool over tokens, projection head to one logit, no
+// bias): logit[b] = (1/T) sum_t sum_d X[b,t,d] w[d], fp32 accumulation.  One warp per sample,
+// each lane a strided slice of the sample's T*D elements, then a shuffle sum.
+template <typename T>
+__global__ void __launch_bounds__(256) head_kernel(const T* __restrict__ X, const T* __restrict__ w, int B, int T_,
+                                                   int D, float* __restrict__ logits) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const size_t n = (size_t)T_ * D;
+    for (int b = warp; b < B; b += nwarps) {
+        const T* xb = X + (size_t)b * n;
+        float acc = 0.f;
+        for (size_t i = lane; i < n; i += 32) acc = fmaf(to_f(xb[i]), to_f(w[i % D]), acc);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) logits[b] = acc / (float)T_;
+    }
+}
+
+cudaError_t launch_head(int dtype, const void* X, const void* w, int B, int T, int D, float* logits, cudaStream_t st) {
+    ProfileScope ps_("head", st);
+    const int grid = grid_for((size_t)B * 32, 256);
+    if (dtype == 1)
+        head_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)X, (const __nv_bfloat16*)w, B, T, D, logits);
+    else
+        head_kernel<float><<<grid, 256, 0, st>>>((const float*)X, (const float*)w, B, T, D, logits);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_tokenize(int dtype, const void* groups, const void* w_group, const void* w_global, int dg, int B,
                             int T, int D, void* X, cudaStream_t st) {
     ProfileScope ps_("tokenize", st);
