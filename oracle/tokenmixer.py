@@ -122,14 +122,26 @@ def route(n: np.ndarray, w_router: np.ndarray, k: int) -> Dict[str, np.ndarray]:
     return {"logits": z, "p": p, "idx": idx, "gap": gap}
 
 
-def sp_moe(n: np.ndarray, bw: Weights, k: int, alpha: float) -> Dict[str, np.ndarray]:
+def sp_moe(n: np.ndarray, bw: Weights, k: int, alpha: float,
+           forced_idx: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
     """Sparse-Pertoken MoE of one bank on rows n [R, W].  [digest] 2.4, Eq. 19-21.
 
     out = alpha * sum_{e in topk} p_e * Expert_e(n) + SharedExpert(n), every
     expert a SwiGLU of its own (Eq. 19), the shared expert always on (Eq. 20),
     alpha the gate-value scale (Eq. 21).  Only the chosen experts are evaluated.
+
+    Teacher-forced routing: with forced_idx [R, k] the experts of each row are those given
+    (for instance another implementation's choices) instead of the top-k; the gates are still
+    alpha * p_e of the oracle's own softmax, so a row whose top-k is a near tie is compared
+    on the same experts everywhere else in the computation.
     """
     r = route(n, bw["w_router"], k)
+    if forced_idx is not None:
+        forced_idx = np.asarray(forced_idx)
+        assert forced_idx.shape == r["idx"].shape, (forced_idx.shape, r["idx"].shape)
+        assert np.all((forced_idx >= 0) & (forced_idx < r["p"].shape[1]))
+        assert all(len(set(row)) == k for row in forced_idx.tolist()), "forced experts repeat within a row"
+        r["idx"] = forced_idx
     idx = r["idx"]
     R, E = r["p"].shape
     out = np.zeros_like(n)
@@ -183,12 +195,13 @@ def storage_round(storage):
 
 # ------------------------------------------------------------------ sub-layer / block / stack
 def sublayer(rows: np.ndarray, bank_w: Callable[[int], Weights], spec, eps: float,
-             gain: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+             gain: Optional[np.ndarray] = None, forced_idx: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
     """FFN(RMSNorm(row)) for every row of every bank, without the residual.
 
     rows: [R, banks, W].  Bank j owns its own weights (parameter isolation,
     [digest] 2.3.2 and 2.4.2 "per-token").  Returns out [R, banks, W] and, for
-    MoE, the routing of each bank.
+    MoE, the routing of each bank.  forced_idx [R, banks, k] (MoE only): teacher-forced
+    routing, see sp_moe.
     """
     R, banks, W = rows.shape
     out = np.empty_like(rows)
@@ -197,7 +210,7 @@ def sublayer(rows: np.ndarray, bank_w: Callable[[int], Weights], spec, eps: floa
         n = rmsnorm(rows[:, j, :], eps, gain)
         bw = bank_w(j)
         if spec.is_moe:
-            r = sp_moe(n, bw, spec.k, spec.alpha)
+            r = sp_moe(n, bw, spec.k, spec.alpha, None if forced_idx is None else forced_idx[:, j, :])
             out[:, j, :] = r["out"]
             for key in info:
                 info[key].append(r[key])
@@ -211,7 +224,8 @@ def sublayer(rows: np.ndarray, bank_w: Callable[[int], Weights], spec, eps: floa
 
 
 def block_forward(X: np.ndarray, cfg, layer: int, bank_w: Callable[[int, int, int], Weights],
-                  gains=(None, None), extra: Optional[np.ndarray] = None, storage=None) -> Dict[str, np.ndarray]:
+                  gains=(None, None), extra: Optional[np.ndarray] = None, storage=None,
+                  forced=(None, None)) -> Dict[str, np.ndarray]:
     """One TokenMixer-Large block on X [R, T, D].  [readme] block diagram; [digest] Eq. 9-16.
 
         H      = Mix(X)
@@ -219,14 +233,15 @@ def block_forward(X: np.ndarray, cfg, layer: int, bank_w: Callable[[int, int, in
         X_rev  = Revert(H_next)
         X_next = FFN_rev(Norm(X_rev)) + X  (+ extra)   (residual to the block input; extra is
                                                          the inter-residual term of the stack)
-    X_rev and X_next are the stored tensors that `storage` rounds.
+    X_rev and X_next are the stored tensors that `storage` rounds.  forced: teacher-forced
+    routing [R, banks, k] per sub-layer (MoE sub-layers; see sp_moe), or None.
     """
     rnd = storage_round(storage)
     Hm = mix(X, cfg.H)
-    s_mix = sublayer(Hm, lambda j: bank_w(layer, 0, j), cfg.mix, cfg.eps, gains[0])
+    s_mix = sublayer(Hm, lambda j: bank_w(layer, 0, j), cfg.mix, cfg.eps, gains[0], forced[0])
     Hn = s_mix["out"] + Hm
     Xr = rnd(revert(Hn, cfg.T))
-    s_rev = sublayer(Xr, lambda j: bank_w(layer, 1, j), cfg.rev, cfg.eps, gains[1])
+    s_rev = sublayer(Xr, lambda j: bank_w(layer, 1, j), cfg.rev, cfg.eps, gains[1], forced[1])
     Xn = s_rev["out"] + X
     if extra is not None:
         Xn = Xn + extra

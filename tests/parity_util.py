@@ -47,13 +47,16 @@ def err_delta(y, o, x, dtype="bf16"):
     return float(np.max(excess) / rms(o - x))
 
 
-def routed_abs_contrib(cfg, layer, sub, rows, down_scale=None, gain=None, include_shared=False):
+def routed_abs_contrib(cfg, layer, sub, rows, down_scale=None, gain=None, include_shared=False, forced_idx=None,
+                       get=None):
     """Per element of each row: sum over the row's chosen experts of |alpha * p_e * Expert_e(n)|
     (plus |Shared(n)| when include_shared).
 
     The GPU stores each routed expert's output row in bf16 before the combine weights it by
-    alpha * p_e, so its rounding error there is at most 2^-8 of this sum."""
-    get = oracle.synth_banks(cfg, down_scale)
+    alpha * p_e, so its rounding error there is at most 2^-8 of this sum.  forced_idx
+    [R, banks, k]: the chosen experts, instead of the oracle's own top-k; get: a (layer, sub,
+    bank) weight getter in place of the synthetic weights."""
+    get = get or oracle.synth_banks(cfg, down_scale)
     spec = cfg.ffn(sub)
     R, banks, W = rows.shape
     out = np.zeros_like(rows)
@@ -61,8 +64,9 @@ def routed_abs_contrib(cfg, layer, sub, rows, down_scale=None, gain=None, includ
         bw = get(layer, sub, j)
         n = O.rmsnorm(rows[:, j, :], cfg.eps, gain)
         r = O.route(n, bw["w_router"], spec.k)
+        chosen = r["idx"] if forced_idx is None else forced_idx[:, j, :]
         for e in range(spec.E):
-            sel = np.nonzero(np.any(r["idx"] == e, axis=1))[0]
+            sel = np.nonzero(np.any(chosen == e, axis=1))[0]
             if sel.size:
                 ye = O.swiglu(n[sel], bw["we_gate"][e], bw["we_up"][e], bw["we_down"][e])
                 out[sel, j, :] += np.abs(spec.alpha * r["p"][sel, e][:, None] * ye)
@@ -96,10 +100,11 @@ def to_np(t):
     return t.cpu().numpy().astype(np.float64)
 
 
-def oracle_sublayer(cfg, layer, sub, rows, down_scale=None, gain=None):
-    """Oracle FFN(Norm(rows)) for one sub-layer of a synthetic workload (no residual)."""
-    get = oracle.synth_banks(cfg, down_scale)
-    return O.sublayer(rows, lambda j: get(layer, sub, j), cfg.ffn(sub), cfg.eps, gain)
+def oracle_sublayer(cfg, layer, sub, rows, down_scale=None, gain=None, forced_idx=None, get=None):
+    """Oracle FFN(Norm(rows)) for one sub-layer of a synthetic workload (no residual); MoE
+    sub-layers routed by forced_idx [R, banks, k] when given (teacher forcing)."""
+    get = get or oracle.synth_banks(cfg, down_scale)
+    return O.sublayer(rows, lambda j: get(layer, sub, j), cfg.ffn(sub), cfg.eps, gain, forced_idx)
 
 
 def check_routing(gpu_idx, gpu_gate, info, alpha, E):

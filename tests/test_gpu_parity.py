@@ -191,6 +191,47 @@ def test_moe_sublayer(cfg, sub, down_scale):
     assert e <= tol(cfg.dtype), e
 
 
+@pytest.mark.parametrize("tied", [False, True], ids=["generic", "tied_router"])
+@pytest.mark.parametrize("sub", [0, 1])
+@pytest.mark.parametrize("cfg", MOE_SMALL, ids=lambda c: c.name)
+def test_moe_sublayer_teacher_forced(cfg, sub, tied):
+    """Every row of an MoE sub-layer against the oracle routed by the GPU's own expert choices
+    (the oracle's teacher-forced mode), near ties included.  With tied routers, experts 0 and 1
+    of every bank share one router row, so their logits are equal for every row and the top-k
+    at the tie is decided by each side's own tie-breaking: the forced oracle follows the GPU."""
+    X, R = inputs(cfg)
+    sw = api.sublayer_from_synth(cfg, 0, sub, DEV, 1.0)
+    base = oracle.synth_banks(cfg, 1.0)
+    get = base
+    if tied:
+        sw.tensors["w_router"][:, 1].copy_(sw.tensors["w_router"][:, 0])
+
+        def get(layer, s, j):
+            w = dict(base(layer, s, j))
+            w["w_router"] = w["w_router"].copy()
+            w["w_router"][1] = w["w_router"][0]
+            return w
+    sh = api.config_shape(cfg)
+    layout = A.TM_LAYOUT_MIXED if sub == 0 else A.TM_LAYOUT_ROWS
+    gi = api.route_topk(dev(X), layout, sh, sw)["idx"].cpu().numpy().astype(np.int64)
+    y = to_np(api.sparse_pertoken_moe(dev(X), dev(R), layout, sh, sw))
+    api.get_device_error()
+    X64, R64 = S.to_f64(X), S.to_f64(R)
+    rows = O.mix(X64, cfg.H) if sub == 0 else X64
+    res = R64 if sub == 1 else O.mix(R64, cfg.H)
+    r = oracle_sublayer(cfg, 0, sub, rows, forced_idx=gi, get=get)
+    o = r["out"] + res
+    c = routed_abs_contrib(cfg, 0, sub, rows, forced_idx=gi, get=get)
+    if sub == 0:
+        o, c = O.revert(o, cfg.T), O.revert(c, cfg.T)
+    e = err_moe_delta(y, o, R64, c, cfg.dtype)
+    assert e <= tol(cfg.dtype), e
+    # the GPU's choices differ from the oracle's own only inside near ties (exact ones included)
+    own = oracle_sublayer(cfg, 0, sub, rows, get=get)
+    flip = np.any(np.sort(gi, -1) != np.sort(own["idx"], -1), axis=-1)
+    assert np.all(own["gap"][flip] < GAP_TOL)
+
+
 @pytest.mark.parametrize("cfg", [DENSE_SMALL[0], MOE_SMALL[0], DENSE_SMALL[2]], ids=lambda c: c.name)
 def test_norm_gain(cfg):
     X, R = inputs(cfg)

@@ -390,3 +390,33 @@ def test_storage_rounding_keeps_zero_down_identity():
     hist = O.stack_forward(X, cfg, lambda l, s, j: w[(l, s, j)], storage="bf16")["hist"]
     for l, c in enumerate([1, 1, 2, 2, 2]):
         assert np.array_equal(hist[l], c * X), l
+
+
+def test_teacher_forced_routing():
+    """The oracle's teacher-forced routing: forcing its own choices (in any order) reproduces its
+    output; forcing another expert set on one row changes that row alone, to alpha * sum over the
+    forced experts of p_e * Expert_e plus the shared expert, written out here row by row."""
+    rng = np.random.default_rng(21)
+    R, W, E, k, Fe = 12, 16, 5, 2, 8
+    n = rng.standard_normal((R, W))
+    bw = {"w_router": rng.standard_normal((E, W)) / 4,
+          "we_gate": rng.standard_normal((E, Fe, W)) / 4, "we_up": rng.standard_normal((E, Fe, W)) / 4,
+          "we_down": rng.standard_normal((E, W, Fe)) / 4,
+          "ws_gate": rng.standard_normal((Fe, W)) / 4, "ws_up": rng.standard_normal((Fe, W)) / 4,
+          "ws_down": rng.standard_normal((W, Fe)) / 4}
+    base = O.sp_moe(n, bw, k, 2.5)
+    assert np.array_equal(O.sp_moe(n, bw, k, 2.5, base["idx"])["out"], base["out"])
+    assert np.allclose(O.sp_moe(n, bw, k, 2.5, base["idx"][:, ::-1])["out"], base["out"], rtol=1e-14, atol=1e-14)
+    forced = base["idx"].copy()
+    row = 3
+    other = [e for e in range(E) if e not in set(forced[row].tolist())][:k]
+    forced[row] = other
+    got = O.sp_moe(n, bw, k, 2.5, forced)["out"]
+    keep = np.arange(R) != row
+    assert np.array_equal(got[keep], base["out"][keep])
+    p = O.softmax(n[row] @ bw["w_router"].T)
+    want = sum(2.5 * p[e] * O.swiglu(n[row:row + 1], bw["we_gate"][e], bw["we_up"][e], bw["we_down"][e])[0]
+               for e in other) + O.swiglu(n[row:row + 1], bw["ws_gate"], bw["ws_up"], bw["ws_down"])[0]
+    assert np.allclose(got[row], want, rtol=1e-12, atol=1e-12)
+    with pytest.raises(AssertionError):
+        O.sp_moe(n, bw, k, 2.5, np.zeros_like(forced))       # an expert chosen twice in a row
