@@ -1,0 +1,145 @@
+"""Pins of the backward oracle (oracle/backward.py) against things other than its own formulas:
+central finite differences of the (separately pinned) forward oracle, the scale invariance of
+RMSNorm, and the special case of a zero down projection, where the block is the identity.
+"""
+import numpy as np
+import pytest
+
+from oracle import backward as BW
+from oracle import tokenmixer as O
+from tm_synth import Config, FFNSpec
+
+
+def fd_grad(f, a, h=1e-6):
+    """Central differences of the scalar f() with respect to every element of the array a
+    (perturbed in place and restored)."""
+    g = np.zeros_like(a)
+    it = np.nditer(a, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        v = a[i]
+        a[i] = v + h
+        fp = f()
+        a[i] = v - h
+        fm = f()
+        a[i] = v
+        g[i] = (fp - fm) / (2 * h)
+    return g
+
+
+def close(got, want, rel=1e-6):
+    scale = max(np.max(np.abs(want)), 1e-12)
+    return np.max(np.abs(got - want)) <= rel * scale
+
+
+@pytest.mark.parametrize("with_gain", [False, True])
+def test_ffn_backward_matches_finite_differences(with_gain):
+    rng = np.random.default_rng(0)
+    R, W, F = 5, 8, 6
+    x = rng.standard_normal((R, W))
+    dy = rng.standard_normal((R, W))
+    bw = {"w_gate": rng.standard_normal((F, W)), "w_up": rng.standard_normal((F, W)),
+          "w_down": rng.standard_normal((W, F))}
+    gain = 1 + 0.3 * rng.standard_normal(W) if with_gain else None
+    eps = 1e-3                              # large enough that the eps term is exercised
+
+    def loss():
+        return float(np.sum(dy * O.swiglu(O.rmsnorm(x, eps, gain), bw["w_gate"], bw["w_up"], bw["w_down"])))
+    g = BW.swiglu_ffn_backward(x, dy, bw, eps, gain)
+    assert close(g["dx"], fd_grad(loss, x))
+    for key in ("w_gate", "w_up", "w_down"):
+        assert close(g["d" + key], fd_grad(loss, bw[key])), key
+    if with_gain:
+        assert close(g["dgain"], fd_grad(loss, gain))
+    else:
+        assert g["dgain"] is None
+
+
+def test_rmsnorm_backward_is_orthogonal_to_the_input_without_eps():
+    # with eps = 0 the normalised row does not change under x -> c x, so the gradient has no
+    # component along x: sum_k x_k dx_k = 0 for every row
+    rng = np.random.default_rng(1)
+    R, W, F = 7, 16, 12
+    x = rng.standard_normal((R, W)) * rng.uniform(0.1, 10, (R, 1))
+    bw = {"w_gate": rng.standard_normal((F, W)), "w_up": rng.standard_normal((F, W)),
+          "w_down": rng.standard_normal((W, F))}
+    g = BW.swiglu_ffn_backward(x, rng.standard_normal((R, W)), bw, 0.0)
+    dots = np.sum(x * g["dx"], axis=1)
+    assert np.all(np.abs(dots) <= 1e-12 * np.linalg.norm(x, axis=1) * np.linalg.norm(g["dx"], axis=1))
+    # and dx scales as 1/c
+    g2 = BW.swiglu_ffn_backward(3.0 * x, np.ones((R, W)), bw, 0.0)
+    g1 = BW.swiglu_ffn_backward(x, np.ones((R, W)), bw, 0.0)
+    assert np.allclose(g2["dx"] * 3.0, g1["dx"], rtol=1e-12, atol=1e-12)
+
+
+def _cfg(T, D, H, L=1, gap=0, F1=5, F2=3):
+    return Config("tiny", B=2, T=T, D=D, H=H, L=L, dtype="f32", mix=FFNSpec("dense", hidden=F1),
+                  rev=FFNSpec("dense", hidden=F2), gap=gap, eps=1e-6)
+
+
+def _weights(cfg, rng, down=0.7):
+    w = {}
+    for l in range(cfg.L):
+        for sub in (0, 1):
+            F, W = cfg.ffn(sub).hidden, cfg.width(sub)
+            for j in range(cfg.banks(sub)):
+                w[(l, sub, j)] = {"w_gate": rng.standard_normal((F, W)), "w_up": rng.standard_normal((F, W)),
+                                  "w_down": down * rng.standard_normal((W, F))}
+    return w
+
+
+@pytest.mark.parametrize("T,D,H", [(2, 4, 2), (3, 4, 2), (2, 6, 1), (4, 4, 4)])
+def test_block_backward_matches_finite_differences(T, D, H):
+    cfg = _cfg(T, D, H)
+    rng = np.random.default_rng(T * 100 + D * 10 + H)
+    w = _weights(cfg, rng)
+    get = lambda l, s, j: w[(l, s, j)]
+    X = rng.standard_normal((cfg.B, T, D))
+    dY = rng.standard_normal((cfg.B, T, D))
+
+    def loss():
+        return float(np.sum(dY * O.block_forward(X, cfg, 0, get)["Y"]))
+    g = BW.block_backward(X, cfg, 0, get, dY)
+    assert close(g["dX"], fd_grad(loss, X))
+    for sub, key in ((0, "mix"), (1, "rev")):
+        j = cfg.banks(sub) - 1
+        for name in ("w_gate", "w_up", "w_down"):
+            assert close(g[key]["d" + name][j], fd_grad(loss, w[(0, sub, j)][name])), (key, name)
+
+
+def test_stack_backward_with_inter_residual_matches_finite_differences():
+    cfg = _cfg(2, 4, 2, L=3, gap=2)          # inter-residual after block 2 (block 3 is the last)
+    rng = np.random.default_rng(5)
+    w = _weights(cfg, rng)
+    get = lambda l, s, j: w[(l, s, j)]
+    X = rng.standard_normal((cfg.B, 2, 4))
+    dY = rng.standard_normal((cfg.B, 2, 4))
+
+    def loss():
+        return float(np.sum(dY * O.stack_forward(X, cfg, get)["Y"]))
+    g = BW.stack_backward(X, cfg, get, dY)
+    assert close(g["dX"], fd_grad(loss, X))
+    assert close(g["blocks"][0]["mix"]["dw_up"][0], fd_grad(loss, w[(0, 0, 0)]["w_up"]))
+    assert close(g["blocks"][2]["rev"]["dw_down"][1], fd_grad(loss, w[(2, 1, 1)]["w_down"]))
+    # without the inter-residual the gradient differs (the skip carries gradient to X_0)
+    cfg0 = _cfg(2, 4, 2, L=3, gap=0)
+    assert not np.allclose(BW.stack_backward(X, cfg0, get, dY)["dX"], g["dX"])
+
+
+def test_zero_down_projection_block_is_identity():
+    cfg = _cfg(2, 4, 2)
+    rng = np.random.default_rng(6)
+    w = _weights(cfg, rng, down=0.0)
+    get = lambda l, s, j: w[(l, s, j)]
+    X = rng.standard_normal((cfg.B, 2, 4))
+    dY = rng.standard_normal((cfg.B, 2, 4))
+    g = BW.block_backward(X, cfg, 0, get, dY)
+    assert np.array_equal(g["dX"], dY)
+    # the reverting sub-layer's residual is the block input, so with its FFN term zero nothing
+    # downstream reads the mixing sub-layer: every mixing gradient vanishes
+    for j in range(cfg.banks(0)):
+        for name in ("dw_gate", "dw_up", "dw_down"):
+            assert not np.any(g["mix"][name][j])
+    for j in range(cfg.banks(1)):
+        assert not np.any(g["rev"]["dw_gate"][j]) and not np.any(g["rev"]["dw_up"][j])
+        assert np.any(g["rev"]["dw_down"][j])
