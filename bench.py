@@ -34,6 +34,7 @@ import numpy as np  # noqa: E402
 import tm_synth as S  # noqa: E402
 
 METRIC = "samples/sec & TFLOP/s of TokenMixer-Large fwd, % of B200 bf16 TC roofline"
+METRIC_BWD = "samples/sec & TFLOP/s of TokenMixer-Large dense block backward, % of B200 bf16 TC roofline"
 DEFAULT_WORKLOAD = "dense_block_bf16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["tm_gemm.cuh", "tm_fused.cuh", "tm_fused2.cuh", "tm_fused128.cuh", "tm_device.cuh", "tm_gemm.cu", "tm_kernels.cu", "tm_api.cu"]
@@ -95,6 +96,29 @@ def kernel_flops_fp8(cfg, B) -> dict:
         for sub in (0, 1):
             f += B * cfg.banks(sub) * 6.0 * cfg.width(sub) * cfg.ffn(sub).hidden
     return {"fused_swiglu_fp8": f}
+
+
+def backward_flops_per_sample(cfg) -> float:
+    """Algorithmic flops of the dense block backward per sample: per row and bank of each sub-layer
+    the derivative's own contractions, dH (2 W F), dWd (2 W F), dWg and dWu (4 W F) and the gradient
+    at the normalised row (4 W F), i.e. twice the forward's 6 W F.  The recomputation the step also
+    performs (the gate / up projections, 4 W F, and the mixing sub-layer's forward) is not counted."""
+    return cfg.L * sum(cfg.banks(sub) * 12.0 * cfg.width(sub) * cfg.ffn(sub).hidden for sub in (0, 1))
+
+
+def kernel_flops_backward(cfg, B) -> dict:
+    """Flops of one backward step per kernel family: every contraction of the two sub-layer
+    backward passes (recomputed projections included, 16 W F per row and bank) runs on the grouped
+    GEMM's plain store epilogue ("gemm_slot"); the mixing sub-layer's forward (X_rev recomputed)
+    takes the forward's dispatch."""
+    out = {"gemm_slot": sum(B * cfg.banks(sub) * 16.0 * cfg.width(sub) * cfg.ffn(sub).hidden for sub in (0, 1))}
+    W, F, H = cfg.W, cfg.mix.hidden, cfg.H
+    if W in (128, 256) and F % 64 == 0:
+        out["fused_swiglu"] = B * H * 6.0 * W * F
+    else:
+        out["gemm_swiglu"] = B * H * 4.0 * W * F
+        out["gemm_combine" if (cfg.D // H) % 16 == 0 else "gemm_resid"] = B * H * 2.0 * W * F
+    return out
 
 
 def fp8_effective_peak(bf16_peak: float) -> float:
@@ -240,6 +264,29 @@ def time_oracle_fp8(cfg, budget_s: float, max_samples: int):
     return done / dt, {"cores": int(threads), "samples": done, "seconds": dt, "per_call": n}
 
 
+def time_oracle_backward(cfg, budget_s: float, max_samples: int):
+    """The backward oracle's samples/s on the host cores over a bounded sample (one dense block)."""
+    import oracle
+    from oracle import backward as BW
+    from threadpoolctl import threadpool_info
+    get = oracle.synth_banks(cfg)
+    for sub in (0, 1):
+        for j in range(cfg.banks(sub)):
+            get(0, sub, j)
+    n = min(max_samples, cfg.B)
+    X = S.to_f64(S.make_x(cfg, np.arange(n)))
+    dY = S.to_f64(S.make_x(cfg.with_(seed=cfg.seed + 17), np.arange(n)))
+    done, t0 = 0, time.perf_counter()
+    while True:
+        BW.block_backward(X, cfg, 0, get, dY, storage=cfg.dtype)
+        done += n
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return done / dt, {"cores": int(threads), "samples": done, "seconds": dt, "per_call": n}
+
+
 def run_reference(args, cfg, rank):
     if rank != 0:
         return
@@ -310,9 +357,16 @@ def run_ours(args, cfg, rank, world, local_rank):
     stream = torch.cuda.Stream(device=dev)
     blocks = api.blocks_from_synth(cfg, dev, workers=min(16, os.cpu_count() or 1))
     sh = api.config_shape(cfg)
-    if args.fp8:
+    dY = None
+    if args.fp8 or args.backward:
         if cfg.gap or cfg.dtype != "bf16" or any(cfg.ffn(sub).is_moe for sub in (0, 1)):
-            raise SystemExit("--fp8 covers bf16 dense blocks without the inter-residual")
+            raise SystemExit("--fp8 and --backward cover bf16 dense blocks without the inter-residual")
+    if args.backward:
+        if cfg.L != 1:
+            raise SystemExit("--backward times one dense block")
+        dY = api.to_device(S.make_x(rank_config(cfg, rank).with_(seed=cfg.seed + rank + 17)), dev)
+        run = api.BlockBackwardRunner(blocks[0], sh, dY, dev)
+    elif args.fp8:
         run = api.Fp8BlockRunner([api.Block8.from_bf16(b) for b in blocks], sh, dev)
     else:
         run = api.StackRunner(blocks, sh, cfg.gap, dev)
@@ -357,30 +411,36 @@ def run_ours(args, cfg, rank, world, local_rank):
     Xh = X.cpu().pin_memory()
     Yh = torch.empty_like(Xh).pin_memory()
     Xd = torch.empty_like(X)
+    # the backward step's inputs are X and dY (both copied in), its result dX (copied back)
+    dYh = dY.cpu().pin_memory() if args.backward else None
+    host = (lambda: run.run_host(Xh, Yh, Xd, Y, dYh, stream)) if args.backward else \
+        (lambda: run.run_host(Xh, Yh, Xd, Y, stream))
     with torch.cuda.stream(stream):
         for _ in range(3):
-            run.run_host(Xh, Yh, Xd, Y, stream)
+            host()
         stream.synchronize()
         eve = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
         for i in range(Ke):
             flush.zero_()
             eve[i][0].record(stream)
-            run.run_host(Xh, Yh, Xd, Y, stream)
+            host()
             eve[i][1].record(stream)
         stream.synchronize()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eve) / Ke, world, dev)
     io_bytes = X.numel() * X.element_size()
+    h2d_bytes = io_bytes * (2 if args.backward else 1)
 
     if rank != 0:
         return
     pk, pk_src = peaks()
     total_samples = cfg.B * world
     value = job_throughput(cfg.B, world, mean_ms)
-    tflops = flops_per_sample(cfg) * value / 1e12
+    tflops = (backward_flops_per_sample(cfg) if args.backward else flops_per_sample(cfg)) * value / 1e12
     # dominant kernel: largest share of device time in the timed region
     dom = max(kern.items(), key=lambda kv: kv[1]["total_ms"]) if kern else (None, None)
     roof = None
-    kf = kernel_flops_fp8(cfg, cfg.B) if args.fp8 else kernel_flops(cfg, cfg.B)
+    kf = (kernel_flops_fp8(cfg, cfg.B) if args.fp8 else
+          kernel_flops_backward(cfg, cfg.B) if args.backward else kernel_flops(cfg, cfg.B))
     if dom[0] in kf:
         per_launch = kf[dom[0]] / (dom[1]["launches"] / K)
         avg_ms = dom[1]["total_ms"] / dom[1]["launches"]
@@ -398,12 +458,13 @@ def run_ours(args, cfg, rank, world, local_rank):
                 "flops_per_launch": per_launch, "avg_launch_ms": avg_ms}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        v, info = (time_oracle_fp8 if args.fp8 else time_oracle)(cfg, args.cpu_seconds, args.cpu_samples)
+        timer = time_oracle_fp8 if args.fp8 else time_oracle_backward if args.backward else time_oracle
+        v, info = timer(cfg, args.cpu_seconds, args.cpu_samples)
         cpu = {"value": v, "unit": "samples/s", "cores": info["cores"], "kind": "oracle",
                "sample": f"{info['samples']} samples ({info['per_call']} per oracle call) of {cfg.name}, "
                          f"{info['seconds']:.1f} s of host time"}
     line = {
-        "metric": METRIC, "value": value, "unit": "samples/s", "n_gpus": world, "steps": K, "warmup": W,
+        "metric": METRIC_BWD if args.backward else METRIC, "value": value, "unit": "samples/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3+bf16" if args.fp8 else "bf16",
         "data": "synthetic (seeded normal inputs, random-init weights of the workload's shapes)",
@@ -412,12 +473,16 @@ def run_ours(args, cfg, rank, world, local_rank):
                    "l2": "flushed by a 256 MB write between timed steps (outside the step events)",
                    **({"precision": "FP8 serving path: GEMM1 (gate, up) on E4M3 operands, one power-of-two scale "
                                     "per bank weight matrix and per activation row; GEMM2 and residual bf16"}
-                      if args.fp8 else {})},
+                      if args.fp8 else {}),
+                   **({"step": "tm_block_backward: the mixing sub-layer's forward recomputed (X_rev), then the "
+                               "reverting and mixing sub-layer backward passes (dX and all six weight gradients); "
+                               "tflops counts the backward's own 12 W F per row and bank, not the recomputation"}
+                      if args.backward else {})},
         "tflops": tflops,
         "tc_roofline_frac": tflops / (fp8_effective_peak(pk["bf16_tflops"]) if args.fp8 else pk["bf16_tflops"]),
         "roofline": roof,
         "cpu_baseline": cpu,
-        "e2e": {"value": job_throughput(cfg.B, world, e2e_ms), "unit": "samples/s", "h2d_bytes_per_step": io_bytes,
+        "e2e": {"value": job_throughput(cfg.B, world, e2e_ms), "unit": "samples/s", "h2d_bytes_per_step": h2d_bytes,
                 "d2h_bytes_per_step": io_bytes, "ms_per_step": e2e_ms, "steps": Ke},
         "gpu_launches": int(launches),
         "launches_per_step": launches / K,
@@ -443,6 +508,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-samples", type=int, default=128)
     ap.add_argument("--steps-ref", type=int, default=None)
+    ap.add_argument("--backward", action="store_true",
+                    help="the dense block backward (training): its own line, not the forward metric's")
     ap.add_argument("--fp8", action="store_true",
                     help="the FP8 E4M3 serving path (dense blocks): its own line, not the bf16 metric's")
     args = ap.parse_args()

@@ -282,6 +282,54 @@ TM_API size_t tm_block_fp8_workspace_bytes(const tm_shape *shape, const tm_block
 TM_API tm_status tm_block_forward_fp8(const void *X, const tm_block_fp8 *block, const tm_shape *shape, void *Y,
                                       void *X_revert_opt, void *workspace, size_t workspace_bytes, void *stream);
 
+/* ---- Training: backward of the dense sub-layer and block ---------------------------------
+ * The pages train the model in bf16 ([digest] 2.5.2; [readme] training flags) and print no
+ * backward pass, so these calls compute the exact derivative of the forward above by the chain
+ * rule, for the FFN term of a dense sub-layer (n = x / rms(x), g = n Wg^T, u = n Wu^T,
+ * h = silu(g) * u, y = h Wd^T; [digest] Eq. 17-18 and 2.3.3):
+ *   dWd = dy^T h;  dh = dy Wd;  dg = dh * u * s * (1 + g * (1 - s)), s = sigmoid(g);  du = dh * silu(g)
+ *   dWg = dg^T n;  dWu = du^T n;  dn = dg Wg + du Wu;  dx = (dn - n * mean(dn * n)) / rms(x)
+ * bf16 tensors, fp32 accumulation on the tensor cores; intermediates are stored in bf16.
+ * Supported: bf16, RMSNorm gain 1 (norm_gain NULL; a gain returns TM_ERR_UNSUPPORTED), row and
+ * hidden widths multiples of 128.  MoE sub-layers have no backward here (TM_ERR_UNSUPPORTED).
+ * Weight gradients are written (not accumulated) in the weights' own layouts, bf16. */
+typedef struct {
+    void *dw_gate, *dw_up;   /* [banks, hidden, width] */
+    void *dw_down;           /* [banks, width, hidden] */
+} tm_swiglu_grads;
+
+/* Weight gradients of the two sub-layers of a dense block. */
+typedef struct { tm_swiglu_grads mix, rev; } tm_block_grads;
+
+/* Workspace of tm_pertoken_swiglu_backward (0: unsupported shape or weights). */
+TM_API size_t tm_pertoken_swiglu_backward_workspace_bytes(const tm_shape *shape, tm_layout layout,
+                                                          const tm_swiglu_w *w);
+
+/* Backward of the FFN term of a dense sub-layer: with y_row = SwiGLU_bank(RMSNorm(x_row)) and an
+ * upstream gradient dy (the layout of x), writes dx = (dy/dx)^T dy + dx_add (dx_add NULL: none;
+ * pass dy itself when the sub-layer adds its own input as the residual) and the bank weight
+ * gradients into `grads`.  x, dy, dx, dx_add share `layout` (rows or the Mix view of [B,T,D]);
+ * dx must not alias x or dy.  The GEMM-ready copies of the rows and the transposed operands
+ * live in the workspace (about (5 W + 9 F) * 2 bytes per row and bank). */
+TM_API tm_status tm_pertoken_swiglu_backward(const void *x, const void *dy, const void *dx_add, tm_layout layout,
+                                             const tm_shape *shape, const void *norm_gain, const tm_swiglu_w *w,
+                                             void *dx, const tm_swiglu_grads *grads, void *workspace,
+                                             size_t workspace_bytes, void *stream);
+
+/* Workspace of tm_block_backward (0: unsupported block). */
+TM_API size_t tm_block_backward_workspace_bytes(const tm_shape *shape, const tm_block *block);
+
+/* Backward of one dense block (tm_block_forward) for the gradient dY of its output:
+ *   X_rev is recomputed by the mixing sub-layer's forward;
+ *   dX_rev = (d FFN_rev(Norm(X_rev)) / d X_rev)^T dY;
+ *   dH_next = Mix(dX_rev);  dH = (d FFN_mix(Norm(H)) / dH)^T dH_next + dH_next;
+ *   dX = dY + Revert(dH)   (Mix and Revert are permutations, each the other's adjoint).
+ * X, dY, dX [B,T,D] bf16; dX must not alias X or dY; grads receives both sub-layers' weight
+ * gradients. */
+TM_API tm_status tm_block_backward(const void *X, const void *dY, const tm_block *block, const tm_shape *shape,
+                                   void *dX, const tm_block_grads *grads, void *workspace, size_t workspace_bytes,
+                                   void *stream);
+
 /* Per-kernel timing of the library's own launches (tracing). */
 typedef struct {
     char name[48];       /* kernel family, e.g. "gemm_swiglu" */

@@ -49,6 +49,8 @@ int main(void) {
   P(tm_moe_w, ws_down) P(tm_sublayer, dense) P(tm_sublayer, moe) P(tm_block, rev)
   printf("tm_swiglu_w8 %zu\ntm_block_fp8 %zu\n", sizeof(tm_swiglu_w8), sizeof(tm_block_fp8));
   P(tm_swiglu_w8, q_gate) P(tm_swiglu_w8, s_up) P(tm_swiglu_w8, w_down) P(tm_block_fp8, rev)
+  printf("tm_swiglu_grads %zu\ntm_block_grads %zu\n", sizeof(tm_swiglu_grads), sizeof(tm_block_grads));
+  P(tm_swiglu_grads, dw_up) P(tm_swiglu_grads, dw_down) P(tm_block_grads, rev)
   return 0;
 }
 ''')
@@ -67,6 +69,10 @@ int main(void) {
         "tm_swiglu_w8": ctypes.sizeof(A.tm_swiglu_w8), "tm_block_fp8": ctypes.sizeof(A.tm_block_fp8),
         "tm_swiglu_w8.q_gate": A.tm_swiglu_w8.q_gate.offset, "tm_swiglu_w8.s_up": A.tm_swiglu_w8.s_up.offset,
         "tm_swiglu_w8.w_down": A.tm_swiglu_w8.w_down.offset, "tm_block_fp8.rev": A.tm_block_fp8.rev.offset,
+        "tm_swiglu_grads": ctypes.sizeof(A.tm_swiglu_grads), "tm_block_grads": ctypes.sizeof(A.tm_block_grads),
+        "tm_swiglu_grads.dw_up": A.tm_swiglu_grads.dw_up.offset,
+        "tm_swiglu_grads.dw_down": A.tm_swiglu_grads.dw_down.offset,
+        "tm_block_grads.rev": A.tm_block_grads.rev.offset,
     }
     assert {k: int(v) for k, v in got.items()} == want
 
@@ -150,3 +156,40 @@ def test_host_validation_rejects_before_launch():
     blocks = (A.tm_block * 1)(api.Block(sub, _fake_sub(cfg, 1)).c())
     assert lib.tm_stack_forward(x, blocks, 0, 0, ctypes.byref(good), y, ws, 1 << 30, None) == A.TM_ERR_INVALID_ARG
     assert lib.tm_stack_forward(x, blocks, 1, 0, ctypes.byref(good), x, ws, 1 << 30, None) == A.TM_ERR_INVALID_ARG
+
+
+def test_backward_queries_and_validation():
+    lib = A.load()
+    cfg = S.CONFIGS["dense_block_bf16"]
+    sh = api.config_shape(cfg)
+    mix, rev = _fake_sub(cfg, 0), _fake_sub(cfg, 1)
+    w = mix.dense_c()
+    n = lib.tm_pertoken_swiglu_backward_workspace_bytes(ctypes.byref(sh), A.TM_LAYOUT_MIXED, ctypes.byref(w))
+    rows = cfg.B * cfg.H
+    assert n >= rows * (5 * cfg.W + 9 * 1024) * 2        # the bf16 copies and transposed operands
+    blk = api.Block(mix, rev).c()
+    nb = lib.tm_block_backward_workspace_bytes(ctypes.byref(sh), ctypes.byref(blk))
+    assert nb >= n + 2 * cfg.B * cfg.T * cfg.D * 2
+    x, dy, dx, ws = (ctypes.c_void_p(a) for a in (0x200000, 0x400000, 0x600000, 0x800000))
+    g = A.tm_swiglu_grads(0x1000000, 0x2000000, 0x3000000)
+    call = lambda **kw: lib.tm_pertoken_swiglu_backward(
+        kw.get("x", x), kw.get("dy", dy), None, kw.get("layout", A.TM_LAYOUT_MIXED), ctypes.byref(kw.get("sh", sh)),
+        kw.get("gain", None), ctypes.byref(kw.get("w", w)), kw.get("dx", dx), ctypes.byref(kw.get("g", g)), ws,
+        kw.get("wsb", 1 << 40), None)
+    assert call(wsb=16) == A.TM_ERR_WORKSPACE
+    assert call(gain=ctypes.c_void_p(0x900000)) == A.TM_ERR_UNSUPPORTED       # RMSNorm gain: forward only
+    assert call(sh=api.shape(cfg.B, cfg.T, cfg.D, cfg.H, "fp32")) == A.TM_ERR_UNSUPPORTED
+    assert call(w=A.tm_swiglu_w(cfg.H, cfg.W, 960, 0x100000, 0x200000, 0x300000)) == A.TM_ERR_UNSUPPORTED
+    assert call(dx=x) == A.TM_ERR_INVALID_ARG                                 # dx aliases x
+    assert call(dx=ctypes.c_void_p(0x600008)) == A.TM_ERR_INVALID_ARG         # misaligned
+    assert call(g=A.tm_swiglu_grads(0x1000000, None, 0x3000000)) == A.TM_ERR_INVALID_ARG
+    # MoE blocks have no backward here
+    mcfg = S.CONFIGS["moe_stack_bf16"]
+    mblk = api.Block(_fake_sub(mcfg, 0), _fake_sub(mcfg, 1)).c()
+    msh = api.config_shape(mcfg)
+    assert lib.tm_block_backward_workspace_bytes(ctypes.byref(msh), ctypes.byref(mblk)) == 0
+    bg = A.tm_block_grads(g, g)
+    assert lib.tm_block_backward(x, dy, ctypes.byref(mblk), ctypes.byref(msh), dx, ctypes.byref(bg), ws, 1 << 40,
+                                 None) == A.TM_ERR_UNSUPPORTED
+    assert lib.tm_block_backward(x, dy, ctypes.byref(blk), ctypes.byref(sh), dx, ctypes.byref(bg), ws, 16,
+                                 None) == A.TM_ERR_WORKSPACE

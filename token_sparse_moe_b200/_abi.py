@@ -19,7 +19,9 @@ EXPORTS = ["tm_status_string", "tm_version", "tm_sublayer_workspace_bytes", "tm_
            "tm_profile_start", "tm_profile_stop", "tm_last_cuda_error", "tm_launch_count",
            "tm_get_device_error", "tm_quantize_fp8_weights", "tm_quantize_fp8_act",
            "tm_pertoken_swiglu_fp8_workspace_bytes", "tm_pertoken_swiglu_fp8", "tm_block_fp8_workspace_bytes",
-           "tm_block_forward_fp8", "tm_head_forward", "tm_model_workspace_bytes", "tm_model_forward"]
+           "tm_block_forward_fp8", "tm_head_forward", "tm_model_workspace_bytes", "tm_model_forward",
+           "tm_pertoken_swiglu_backward_workspace_bytes", "tm_pertoken_swiglu_backward",
+           "tm_block_backward_workspace_bytes", "tm_block_backward"]
 
 
 class tm_shape(ctypes.Structure):
@@ -53,6 +55,14 @@ class tm_swiglu_w8(ctypes.Structure):
 
 class tm_block_fp8(ctypes.Structure):
     _fields_ = [("mix", tm_swiglu_w8), ("rev", tm_swiglu_w8)]
+
+
+class tm_swiglu_grads(ctypes.Structure):
+    _fields_ = [("dw_gate", c_void_p), ("dw_up", c_void_p), ("dw_down", c_void_p)]
+
+
+class tm_block_grads(ctypes.Structure):
+    _fields_ = [("mix", tm_swiglu_grads), ("rev", tm_swiglu_grads)]
 
 
 class tm_kernel_time(ctypes.Structure):
@@ -92,6 +102,12 @@ _SIGS = {
     "tm_model_workspace_bytes": (c_size_t, [POINTER(tm_shape), POINTER(tm_block), c_int, c_int]),
     "tm_model_forward": (c_int, [_P, _P, _P, c_int, POINTER(tm_block), c_int, c_int, _P, POINTER(tm_shape), _P, _P,
                                  c_size_t, _P]),
+    "tm_pertoken_swiglu_backward_workspace_bytes": (c_size_t, [POINTER(tm_shape), c_int, POINTER(tm_swiglu_w)]),
+    "tm_pertoken_swiglu_backward": (c_int, [_P, _P, _P, c_int, POINTER(tm_shape), _P, POINTER(tm_swiglu_w), _P,
+                                            POINTER(tm_swiglu_grads), _P, c_size_t, _P]),
+    "tm_block_backward_workspace_bytes": (c_size_t, [POINTER(tm_shape), POINTER(tm_block)]),
+    "tm_block_backward": (c_int, [_P, _P, POINTER(tm_block), POINTER(tm_shape), _P, POINTER(tm_block_grads), _P,
+                                  c_size_t, _P]),
 }
 
 _lib = None

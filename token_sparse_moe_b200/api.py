@@ -421,6 +421,88 @@ class Fp8BlockRunner:
         return Y_host
 
 
+def _grads_c(grads: Dict[str, torch.Tensor]) -> A.tm_swiglu_grads:
+    return A.tm_swiglu_grads(_p(grads["dw_gate"]), _p(grads["dw_up"]), _p(grads["dw_down"]))
+
+
+def _grads_like(sub: SubLayer, device) -> Dict[str, torch.Tensor]:
+    F, W, nb = sub.hidden, sub.width, sub.banks
+    return {"dw_gate": torch.empty((nb, F, W), dtype=torch.bfloat16, device=device),
+            "dw_up": torch.empty((nb, F, W), dtype=torch.bfloat16, device=device),
+            "dw_down": torch.empty((nb, W, F), dtype=torch.bfloat16, device=device)}
+
+
+def pertoken_swiglu_backward(x, dy, layout: int, sh: A.tm_shape, sub: SubLayer, dx_add=None, dx=None, grads=None,
+                             workspace=None, stream=None):
+    """dx and the weight gradients {dw_gate, dw_up, dw_down} of the FFN term of a dense sub-layer
+    for the upstream gradient dy (tm_pertoken_swiglu_backward)."""
+    dx = torch.empty_like(x) if dx is None else dx
+    grads = _grads_like(sub, x.device) if grads is None else grads
+    w = sub.dense_c()
+    n = lib().tm_pertoken_swiglu_backward_workspace_bytes(ctypes.byref(sh), layout, ctypes.byref(w))
+    if n == 0:
+        raise A.TMError(A.TM_ERR_UNSUPPORTED, "tm_pertoken_swiglu_backward_workspace_bytes")
+    ws = _ws(n, x.device, workspace)
+    g = _grads_c(grads)
+    A.check(lib().tm_pertoken_swiglu_backward(_p(x), _p(dy), _p(dx_add), layout, ctypes.byref(sh), _p(sub.gain),
+                                              ctypes.byref(w), _p(dx), ctypes.byref(g), _p(ws), ws.numel(),
+                                              _s(stream)), "tm_pertoken_swiglu_backward")
+    return dx, grads
+
+
+def block_backward_workspace_bytes(sh: A.tm_shape, block: Block) -> int:
+    c = block.c()
+    n = lib().tm_block_backward_workspace_bytes(ctypes.byref(sh), ctypes.byref(c))
+    if n == 0:
+        raise A.TMError(A.TM_ERR_UNSUPPORTED, "tm_block_backward_workspace_bytes")
+    return n
+
+
+def block_backward(X, dY, block: Block, sh: A.tm_shape, dX=None, grads=None, workspace=None, stream=None):
+    """dX and both sub-layers' weight gradients ({"mix": {...}, "rev": {...}}) of a dense block for
+    the gradient dY of its output (tm_block_backward)."""
+    dX = torch.empty_like(X) if dX is None else dX
+    if grads is None:
+        grads = {"mix": _grads_like(block.mix, X.device), "rev": _grads_like(block.rev, X.device)}
+    c = block.c()
+    ws = _ws(block_backward_workspace_bytes(sh, block), X.device, workspace)
+    g = A.tm_block_grads(_grads_c(grads["mix"]), _grads_c(grads["rev"]))
+    A.check(lib().tm_block_backward(_p(X), _p(dY), ctypes.byref(c), ctypes.byref(sh), _p(dX), ctypes.byref(g), _p(ws),
+                                    ws.numel(), _s(stream)), "tm_block_backward")
+    return dX, grads
+
+
+class BlockBackwardRunner:
+    """Repeated dense-block backward passes with a preallocated workspace and gradient buffers:
+    __call__(X, dX) writes dX and the weight gradients for the upstream gradient self.dY."""
+
+    def __init__(self, block: Block, sh: A.tm_shape, dY: torch.Tensor, device):
+        self.block = block
+        self.sh = sh
+        self.c = block.c()
+        self.dY = dY
+        self.ws = torch.empty(block_backward_workspace_bytes(sh, block), dtype=torch.uint8, device=device)
+        self.grads = {"mix": _grads_like(block.mix, device), "rev": _grads_like(block.rev, device)}
+        self.gc = A.tm_block_grads(_grads_c(self.grads["mix"]), _grads_c(self.grads["rev"]))
+
+    def __call__(self, X: torch.Tensor, dX: torch.Tensor, stream=None) -> torch.Tensor:
+        A.check(lib().tm_block_backward(_p(X), _p(self.dY), ctypes.byref(self.c), ctypes.byref(self.sh), _p(dX),
+                                        ctypes.byref(self.gc), _p(self.ws), self.ws.numel(), _s(stream)),
+                "tm_block_backward")
+        return dX
+
+    def run_host(self, X_host, dX_host, X_dev, dX_dev, dY_host=None, stream=None):
+        """End to end on one stream: pinned host X (and dY) -> device, backward, device -> pinned host dX."""
+        s = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(s):
+            X_dev.copy_(X_host, non_blocking=True)
+            if dY_host is not None:
+                self.dY.copy_(dY_host, non_blocking=True)
+            self(X_dev, dX_dev, s)
+            dX_host.copy_(dX_dev, non_blocking=True)
+        return dX_host
+
+
 def profile_start() -> None:
     A.check(lib().tm_profile_start(), "tm_profile_start")
 

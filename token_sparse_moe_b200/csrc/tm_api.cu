@@ -942,6 +942,144 @@ tm_status run_block(const tm_shape* s, const tm_block* b, const void* X, const v
     return run_sublayer(gr, Xr, X, extra, &b->rev, Y, sub_ws, sub_wsb, st);
 }
 
+// ------------------------------------------------------------------ dense sub-layer backward
+// Gradients of the FFN term y = SwiGLU_bank(RMSNorm(x)) of a dense bf16 sub-layer (gain 1) for an
+// upstream gradient dy.  Every contraction runs on the tcgen05 grouped GEMM with its plain bf16
+// store epilogue (both operands K-major, fp32 accumulation in TMEM):
+//   G = xh Wg^T, U = xh Wu^T                   recomputed, A = xh [banks][B][W]
+//   dH = dy Wd                                 B operand Wd^T [banks][F][W]
+//   dWd = dy^T H                               A = dy^T [banks][W][Bp], B operand H^T [banks][F][Bp]
+//   dWg = dG^T xh, dWu = dU^T xh               A = dG^T, dU^T [banks][F][Bp], B operand xh^T [banks][W][Bp]
+//   dN = dG Wg + dU Wu = (dG | dU) (Wg ; Wu)   B operand (Wg ; Wu)^T [banks][W][2F]
+// with Bp = B rounded up to the 64-wide K slab (the transposes write zeros into the padding).  The
+// CUDA-core kernels of tm_backward.cu do the row pass, the transposes, the SwiGLU derivative and
+// the RMSNorm derivative.
+struct DenseBwdWs {
+    float* inv_rms;
+    uint16_t *xh, *dyb, *G, *U, *dH, *dGU, *Hd, *dN, *WdT, *WguT, *dyT, *HT, *dgT, *duT, *xhT;
+};
+DenseBwdWs carve_dense_bwd(Carve& c, const Geo& g, int F) {
+    const size_t nb = g.banks, B = g.B, W = g.W, Bp = (B + 63) / 64 * 64;
+    DenseBwdWs w;
+    w.inv_rms = c.take<float>(nb * B);
+    w.xh = c.take<uint16_t>(nb * B * W);
+    w.dyb = c.take<uint16_t>(nb * B * W);
+    w.G = c.take<uint16_t>(nb * B * F);
+    w.U = c.take<uint16_t>(nb * B * F);
+    w.dH = c.take<uint16_t>(nb * B * F);
+    w.dGU = c.take<uint16_t>(nb * B * 2 * F);
+    w.Hd = c.take<uint16_t>(nb * B * F);
+    w.dN = c.take<uint16_t>(nb * B * W);
+    w.WdT = c.take<uint16_t>(nb * F * W);
+    w.WguT = c.take<uint16_t>(nb * W * 2 * F);
+    w.dyT = c.take<uint16_t>(nb * W * Bp);
+    w.HT = c.take<uint16_t>(nb * F * Bp);
+    w.dgT = c.take<uint16_t>(nb * F * Bp);
+    w.duT = c.take<uint16_t>(nb * F * Bp);
+    w.xhT = c.take<uint16_t>(nb * W * Bp);
+    return w;
+}
+size_t dense_bwd_ws(const Geo& g, int F) {
+    Carve c{nullptr};
+    carve_dense_bwd(c, g, F);
+    return align256(c.off);
+}
+
+// bf16 only, gain 1 (NULL), row and hidden widths multiples of 128 (64-wide K slabs, N tiles of
+// 128 / 192 / 256 columns)
+tm_status check_dense_bwd(const Geo& g, const tm_swiglu_w* w, const void* gain) {
+    tm_status s = check_dense(g, w);
+    if (s != TM_OK) return s;
+    if (g.dtype != TM_BF16 || gain) return TM_ERR_UNSUPPORTED;
+    if (g.W % 128 || w->hidden % 128) return TM_ERR_UNSUPPORTED;
+    return TM_OK;
+}
+
+// out[g*rows + r][n] = sum_k A[g*rows + r][k] * Bm[g*N + n][k] for every group g (bf16 out, fp32
+// accumulation): the grouped GEMM with its plain store epilogue.  K % 64 == 0, N % 128 == 0.
+tm_status gemm_plain(const void* A, int groups, int rows, int K, const void* Bm, int N, void* out, cudaStream_t st) {
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.sched = 0;
+    p.groups = groups;
+    p.rows = rows;
+    p.banks = groups;
+    p.E = 1;
+    p.K = K;
+    p.N = N;
+    const int bn = pick_bn_out(N);
+    p.n_tiles = N / bn;
+    p.out = (__nv_bfloat16*)out;
+    p.out_ld = N;
+    p.out_elems = (size_t)groups * rows * N;
+    p.pos_limit = groups * rows;
+    CUtensorMap ma, mb;
+    if (!map_2d(&ma, A, (uint64_t)groups * rows, K, 128) || !map_2d(&mb, Bm, (uint64_t)groups * N, K, bn))
+        return TM_ERR_CUDA;
+    return cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SLOT, ma, mb, mb, p, dense_grid(p), st));
+}
+
+// dx = d(FFN term)/dx applied to dy, plus add0 and add1 (NULL: none; both in dx's row layout);
+// the weight gradients dwg, dwu [banks, F, W] and dwd [banks, W, F].
+tm_status run_dense_bwd(const Geo& g, const void* x, const void* dy, const void* add0, const void* add1,
+                        const tm_swiglu_w* w, void* dx, void* dwg, void* dwu, void* dwd, void* ws, size_t wsb,
+                        cudaStream_t st) {
+    const int B = g.B, W = g.W, F = w->hidden, nb = g.banks;
+    const int Bp = (B + 63) / 64 * 64;
+    Carve c{(uint8_t*)ws};
+    DenseBwdWs d = carve_dense_bwd(c, g, F);
+    if (!ws || wsb < c.off || !al16(ws)) return TM_ERR_WORKSPACE;
+    const size_t BW = (size_t)B * W, BF = (size_t)B * F, FW = (size_t)F * W;
+    tm_status s;
+#define TM_TRY(expr)                         \
+    do {                                     \
+        if ((s = (expr)) != TM_OK) return s; \
+    } while (0)
+    TM_TRY(cuda_status(launch_bwd_rows(x, dy, g.map, B, g.eps, d.xh, d.dyb, d.inv_rms, st)));
+    // the recomputed projections and the gradient at the down projection's input
+    TM_TRY(gemm_plain(d.xh, nb, B, W, w->w_gate, F, d.G, st));
+    TM_TRY(gemm_plain(d.xh, nb, B, W, w->w_up, F, d.U, st));
+    TM_TRY(cuda_status(launch_transpose(w->w_down, FW, F, W, F, d.WdT, FW, W, W, nb, st)));
+    TM_TRY(gemm_plain(d.dyb, nb, B, W, d.WdT, F, d.dH, st));
+    TM_TRY(cuda_status(launch_swiglu_bwd(d.G, d.U, d.dH, (size_t)nb * B, F, d.dGU, d.Hd, st)));
+    // weight gradients: contractions over the samples
+    TM_TRY(cuda_status(launch_transpose(d.dyb, BW, W, B, W, d.dyT, (size_t)W * Bp, Bp, Bp, nb, st)));
+    TM_TRY(cuda_status(launch_transpose(d.Hd, BF, F, B, F, d.HT, (size_t)F * Bp, Bp, Bp, nb, st)));
+    TM_TRY(gemm_plain(d.dyT, nb, W, Bp, d.HT, F, dwd, st));
+    TM_TRY(cuda_status(launch_transpose(d.dGU, 2 * BF, 2 * F, B, F, d.dgT, (size_t)F * Bp, Bp, Bp, nb, st)));
+    TM_TRY(cuda_status(launch_transpose(d.dGU + F, 2 * BF, 2 * F, B, F, d.duT, (size_t)F * Bp, Bp, Bp, nb, st)));
+    TM_TRY(cuda_status(launch_transpose(d.xh, BW, W, B, W, d.xhT, (size_t)W * Bp, Bp, Bp, nb, st)));
+    TM_TRY(gemm_plain(d.dgT, nb, F, Bp, d.xhT, W, dwg, st));
+    TM_TRY(gemm_plain(d.duT, nb, F, Bp, d.xhT, W, dwu, st));
+    // the gradient at the normalised row, then through the RMSNorm
+    TM_TRY(cuda_status(launch_transpose(w->w_gate, FW, W, F, W, d.WguT, (size_t)W * 2 * F, 2 * F, F, nb, st)));
+    TM_TRY(cuda_status(launch_transpose(w->w_up, FW, W, F, W, d.WguT + F, (size_t)W * 2 * F, 2 * F, F, nb, st)));
+    TM_TRY(gemm_plain(d.dGU, nb, B, 2 * F, d.WguT, W, d.dN, st));
+    TM_TRY(cuda_status(launch_rms_bwd(x, d.dN, d.inv_rms, add0, add1, g.map, B, dx, st)));
+#undef TM_TRY
+    return TM_OK;
+}
+
+bool grads_ok(const tm_swiglu_grads* gr) {
+    return gr && gr->dw_gate && gr->dw_up && gr->dw_down && al16(gr->dw_gate) && al16(gr->dw_up) && al16(gr->dw_down);
+}
+
+// Block backward: both sub-layers dense bf16 with gain 1.  Workspace: X_rev, dX_rev, then one
+// region shared by the mixing sub-layer's forward (X_rev recomputed) and the two backward passes.
+tm_status check_block_bwd(const tm_shape* s, const tm_block* b, Geo* gm, Geo* gr) {
+    tm_status st = check_block(s, b, gm, gr);
+    if (st != TM_OK) return st;
+    if (b->mix.is_moe || b->rev.is_moe) return TM_ERR_UNSUPPORTED;
+    if ((st = check_dense_bwd(*gm, &b->mix.dense, b->mix.norm_gain)) != TM_OK) return st;
+    return check_dense_bwd(*gr, &b->rev.dense, b->rev.norm_gain);
+}
+size_t block_bwd_sub_ws(const Geo& gm, const Geo& gr, const tm_block* b) {
+    size_t n = sublayer_ws(gm, &b->mix);
+    const size_t m = dense_bwd_ws(gm, b->mix.dense.hidden), r = dense_bwd_ws(gr, b->rev.dense.hidden);
+    n = m > n ? m : n;
+    return r > n ? r : n;
+}
+
 }  // namespace
 }  // namespace tml
 
@@ -1215,6 +1353,66 @@ tm_status tm_block_forward_fp8(const void* X, const tm_block_fp8* block, const t
     // H_next = FFN_mix(Norm(Mix(X))) + Mix(X) through Revert into X_rev; Y = FFN_rev(Norm(X_rev)) + X
     if ((s = run_dense8(gm, X, X, nullptr, &block->mix, xr, st)) != TM_OK) return s;
     return run_dense8(gr, xr, X, nullptr, &block->rev, Y, st);
+}
+
+size_t tm_pertoken_swiglu_backward_workspace_bytes(const tm_shape* shape, tm_layout layout, const tm_swiglu_w* w) {
+    Geo g;
+    if (!w || make_geo(shape, layout, w->banks, w->width, &g) != TM_OK || check_dense_bwd(g, w, nullptr) != TM_OK)
+        return 0;
+    return dense_bwd_ws(g, w->hidden);
+}
+
+tm_status tm_pertoken_swiglu_backward(const void* x, const void* dy, const void* dx_add, tm_layout layout,
+                                      const tm_shape* shape, const void* norm_gain, const tm_swiglu_w* w, void* dx,
+                                      const tm_swiglu_grads* grads, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+    if (!w) return TM_ERR_INVALID_ARG;
+    Geo g;
+    tm_status s = make_geo(shape, layout, w->banks, w->width, &g);
+    if (s != TM_OK) return s;
+    if (norm_gain && !al16(norm_gain)) return TM_ERR_INVALID_ARG;
+    if ((s = check_dense_bwd(g, w, norm_gain)) != TM_OK) return s;
+    if (!x || !dy || !dx || !al16(x) || !al16(dy) || !al16(dx) || (dx_add && !al16(dx_add)) || dx == x || dx == dy ||
+        !grads_ok(grads))
+        return TM_ERR_INVALID_ARG;
+    return run_dense_bwd(g, x, dy, dx_add, nullptr, w, dx, grads->dw_gate, grads->dw_up, grads->dw_down, workspace,
+                         workspace_bytes, (cudaStream_t)stream);
+}
+
+size_t tm_block_backward_workspace_bytes(const tm_shape* shape, const tm_block* block) {
+    Geo gm, gr;
+    if (!block || check_block_bwd(shape, block, &gm, &gr) != TM_OK) return 0;
+    const size_t tok = align256((size_t)shape->B * shape->T * shape->D * 2);
+    return 2 * tok + block_bwd_sub_ws(gm, gr, block);
+}
+
+tm_status tm_block_backward(const void* X, const void* dY, const tm_block* block, const tm_shape* shape, void* dX,
+                            const tm_block_grads* grads, void* workspace, size_t workspace_bytes, void* stream) {
+    Geo gm, gr;
+    if (!block) return TM_ERR_INVALID_ARG;
+    tm_status s = check_block_bwd(shape, block, &gm, &gr);
+    if (s != TM_OK) return s;
+    if (!X || !dY || !dX || !al16(X) || !al16(dY) || !al16(dX) || dX == X || dX == dY || !grads ||
+        !grads_ok(&grads->mix) || !grads_ok(&grads->rev))
+        return TM_ERR_INVALID_ARG;
+    const size_t tok = align256((size_t)shape->B * shape->T * shape->D * 2);
+    const size_t sub = block_bwd_sub_ws(gm, gr, block);
+    if (!workspace || workspace_bytes < 2 * tok + sub || !al16(workspace)) return TM_ERR_WORKSPACE;
+    uint8_t* base = (uint8_t*)workspace;
+    void* Xr = base;
+    void* dXr = base + tok;
+    void* ws = base + 2 * tok;
+    cudaStream_t st = (cudaStream_t)stream;
+    // X_rev = Revert(FFN_mix(Norm(Mix(X))) + Mix(X)), as the forward stored it
+    if ((s = run_sublayer(gm, X, X, nullptr, &block->mix, Xr, ws, sub, st)) != TM_OK) return s;
+    // reverting sub-layer: dX_rev = d FFN_rev(Norm(X_rev)) / d X_rev applied to dY
+    if ((s = run_dense_bwd(gr, Xr, dY, nullptr, nullptr, &block->rev.dense, dXr, grads->rev.dw_gate,
+                           grads->rev.dw_up, grads->rev.dw_down, ws, sub, st)) != TM_OK)
+        return s;
+    // mixing sub-layer on mixed rows: dH_next = Mix(dX_rev); dX = dY + Revert(d FFN_mix applied to
+    // dH_next + dH_next), written through the same row map
+    return run_dense_bwd(gm, X, dXr, dXr, dY, &block->mix.dense, dX, grads->mix.dw_gate, grads->mix.dw_up,
+                         grads->mix.dw_down, ws, sub, st);
 }
 
 tm_status tm_get_device_error(void* stream) {
