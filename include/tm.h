@@ -330,6 +330,20 @@ TM_API tm_status tm_block_backward(const void *X, const void *dY, const tm_block
                                    void *dX, const tm_block_grads *grads, void *workspace, size_t workspace_bytes,
                                    void *stream);
 
+/* Workspace of tm_stack_backward (0: unsupported blocks). */
+TM_API size_t tm_stack_backward_workspace_bytes(const tm_shape *shape, const tm_block *blocks, int L,
+                                                int inter_residual_gap);
+
+/* Backward of L dense blocks with the inter-residual of tm_stack_forward ([digest] 2.3.4), for the
+ * gradient dY of the stack's output: every block input X_1 .. X_{L-1} is recomputed by the forward
+ * (kept in the workspace), then, last block first, the gradient of X_{l-1} is block l's input
+ * gradient (tm_block_backward) plus, when X_{l-1+gap} = Block(...) + X_{l-1}, the gradient of
+ * X_{l-1+gap}.  grads[l] receives block l's weight gradients.  X, dY, dX [B,T,D] bf16; dX must not
+ * alias X or dY. */
+TM_API tm_status tm_stack_backward(const void *X, const void *dY, const tm_block *blocks, int L, int inter_residual_gap,
+                                   const tm_shape *shape, void *dX, const tm_block_grads *grads, void *workspace,
+                                   size_t workspace_bytes, void *stream);
+
 /* Per-kernel timing of the library's own launches (tracing). */
 typedef struct {
     char name[48];       /* kernel family, e.g. "gemm_swiglu" */

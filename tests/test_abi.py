@@ -193,3 +193,25 @@ def test_backward_queries_and_validation():
                                  None) == A.TM_ERR_UNSUPPORTED
     assert lib.tm_block_backward(x, dy, ctypes.byref(blk), ctypes.byref(sh), dx, ctypes.byref(bg), ws, 16,
                                  None) == A.TM_ERR_WORKSPACE
+
+
+def test_stack_backward_queries():
+    lib = A.load()
+    cfg = S.CONFIGS["dense_block_bf16"]
+    sh = api.config_shape(cfg)
+    blk = api.Block(_fake_sub(cfg, 0), _fake_sub(cfg, 1)).c()
+    one = lib.tm_block_backward_workspace_bytes(ctypes.byref(sh), ctypes.byref(blk))
+    arr = (A.tm_block * 4)(*[blk] * 4)
+    four = lib.tm_stack_backward_workspace_bytes(ctypes.byref(sh), arr, 4, 2)
+    tok = cfg.B * cfg.T * cfg.D * 2
+    assert four >= one + 6 * tok                       # X_1..X_3 and their gradients
+    assert lib.tm_stack_backward_workspace_bytes(ctypes.byref(sh), arr, 0, 2) == 0
+    mcfg = S.CONFIGS["moe_stack_bf16"]
+    marr = (A.tm_block * 1)(api.Block(_fake_sub(mcfg, 0), _fake_sub(mcfg, 1)).c())
+    msh = api.config_shape(mcfg)
+    assert lib.tm_stack_backward_workspace_bytes(ctypes.byref(msh), marr, 1, 0) == 0
+    g = A.tm_swiglu_grads(0x1000000, 0x2000000, 0x3000000)
+    garr = (A.tm_block_grads * 4)(*[A.tm_block_grads(g, g)] * 4)
+    x, dy, dx, ws = (ctypes.c_void_p(a) for a in (0x200000, 0x400000, 0x600000, 0x800000))
+    assert lib.tm_stack_backward(x, dy, arr, 4, 2, ctypes.byref(sh), dx, garr, ws, 16, None) == A.TM_ERR_WORKSPACE
+    assert lib.tm_stack_backward(x, dy, arr, 4, 2, ctypes.byref(sh), x, garr, ws, 1 << 40, None) == A.TM_ERR_INVALID_ARG

@@ -38,9 +38,9 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def small(name, B, T, D, H, mix, rev):
-    return S.Config(name, B=B, T=T, D=D, H=H, L=1, dtype="bf16", mix=FFNSpec("dense", hidden=mix),
-                    rev=FFNSpec("dense", hidden=rev))
+def small(name, B, T, D, H, mix, rev, L=1, gap=0):
+    return S.Config(name, B=B, T=T, D=D, H=H, L=L, dtype="bf16", mix=FFNSpec("dense", hidden=mix),
+                    rev=FFNSpec("dense", hidden=rev), gap=gap)
 
 
 CASES = [
@@ -168,3 +168,42 @@ def test_backward_rejects_gain_and_moe():
     sw = api.sublayer_from_synth(cfg, 0, 1, DEV, with_gain=True)
     with pytest.raises(TMError):
         api.pertoken_swiglu_backward(dev(X), dev(dY), A.TM_LAYOUT_ROWS, api.config_shape(cfg), sw)
+
+
+STACKS = [
+    # four blocks, inter-residual after block 2 (X_2 += X_0; none after the last block)
+    small("bwd_stack_gap2", 300, 16, 256, 16, 256, 384, L=4, gap=2),
+    # three blocks with gap 1 (X_1 += X_0, X_2 += X_1) on the width-128 geometry
+    small("bwd_stack_gap1", 200, 8, 128, 4, 128, 256, L=3, gap=1),
+]
+
+
+@pytest.mark.parametrize("cfg", STACKS, ids=lambda c: c.name)
+def test_stack_backward(cfg):
+    """tm_stack_backward against the oracle's stack backward (the forward recomputed with the bf16
+    storage of X_rev and of every block output, the inter-residual's gradient handed back)."""
+    X, dY = seeded(cfg)
+    blocks = api.blocks_from_synth(cfg, DEV)
+    sh = api.config_shape(cfg)
+    dX, grads = api.stack_backward(dev(X), dev(dY), blocks, cfg.gap, sh)
+    api.get_device_error()
+    o = BW.stack_backward(S.to_f64(X), cfg, oracle.synth_banks(cfg), S.to_f64(dY), storage="bf16")
+    check("dX", to_np(dX), o["dX"])
+    for l in range(cfg.L):
+        check_bank_grads(grads_np(grads[l]["mix"]), o["blocks"][l]["mix"], f"block{l}.mix")
+        check_bank_grads(grads_np(grads[l]["rev"]), o["blocks"][l]["rev"], f"block{l}.rev")
+
+
+def test_stack_backward_one_block_is_block_backward():
+    """L = 1: the stack backward is the block backward, bit for bit."""
+    cfg = CASES[0]
+    X, dY = seeded(cfg)
+    blk = api.Block(api.sublayer_from_synth(cfg, 0, 0, DEV), api.sublayer_from_synth(cfg, 0, 1, DEV))
+    sh = api.config_shape(cfg)
+    a, ga = api.block_backward(dev(X), dev(dY), blk, sh)
+    b, gb = api.stack_backward(dev(X), dev(dY), [blk], 0, sh)
+    api.get_device_error()
+    assert torch.equal(a, b)
+    for s in ("mix", "rev"):
+        for k in ga[s]:
+            assert torch.equal(ga[s][k], gb[0][s][k]), (s, k)

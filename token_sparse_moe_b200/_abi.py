@@ -21,7 +21,8 @@ EXPORTS = ["tm_status_string", "tm_version", "tm_sublayer_workspace_bytes", "tm_
            "tm_pertoken_swiglu_fp8_workspace_bytes", "tm_pertoken_swiglu_fp8", "tm_block_fp8_workspace_bytes",
            "tm_block_forward_fp8", "tm_head_forward", "tm_model_workspace_bytes", "tm_model_forward",
            "tm_pertoken_swiglu_backward_workspace_bytes", "tm_pertoken_swiglu_backward",
-           "tm_block_backward_workspace_bytes", "tm_block_backward"]
+           "tm_block_backward_workspace_bytes", "tm_block_backward", "tm_stack_backward_workspace_bytes",
+           "tm_stack_backward"]
 
 
 class tm_shape(ctypes.Structure):
@@ -108,6 +109,9 @@ _SIGS = {
     "tm_block_backward_workspace_bytes": (c_size_t, [POINTER(tm_shape), POINTER(tm_block)]),
     "tm_block_backward": (c_int, [_P, _P, POINTER(tm_block), POINTER(tm_shape), _P, POINTER(tm_block_grads), _P,
                                   c_size_t, _P]),
+    "tm_stack_backward_workspace_bytes": (c_size_t, [POINTER(tm_shape), POINTER(tm_block), c_int, c_int]),
+    "tm_stack_backward": (c_int, [_P, _P, POINTER(tm_block), c_int, c_int, POINTER(tm_shape), _P,
+                                  POINTER(tm_block_grads), _P, c_size_t, _P]),
 }
 
 _lib = None

@@ -472,6 +472,25 @@ def block_backward(X, dY, block: Block, sh: A.tm_shape, dX=None, grads=None, wor
     return dX, grads
 
 
+def stack_backward(X, dY, blocks: Sequence[Block], gap: int, sh: A.tm_shape, dX=None, grads=None, workspace=None,
+                   stream=None):
+    """dX and every block's weight gradients (a list of {"mix": {...}, "rev": {...}}) of a dense
+    stack with the inter-residual every `gap` blocks (tm_stack_backward)."""
+    blocks = list(blocks)
+    dX = torch.empty_like(X) if dX is None else dX
+    if grads is None:
+        grads = [{"mix": _grads_like(b.mix, X.device), "rev": _grads_like(b.rev, X.device)} for b in blocks]
+    arr = (A.tm_block * len(blocks))(*[b.c() for b in blocks])
+    n = lib().tm_stack_backward_workspace_bytes(ctypes.byref(sh), arr, len(blocks), gap)
+    if n == 0:
+        raise A.TMError(A.TM_ERR_UNSUPPORTED, "tm_stack_backward_workspace_bytes")
+    ws = _ws(n, X.device, workspace)
+    garr = (A.tm_block_grads * len(blocks))(*[A.tm_block_grads(_grads_c(g["mix"]), _grads_c(g["rev"])) for g in grads])
+    A.check(lib().tm_stack_backward(_p(X), _p(dY), arr, len(blocks), gap, ctypes.byref(sh), _p(dX), garr, _p(ws),
+                                    ws.numel(), _s(stream)), "tm_stack_backward")
+    return dX, grads
+
+
 class BlockBackwardRunner:
     """Repeated dense-block backward passes with a preallocated workspace and gradient buffers:
     __call__(X, dX) writes dX and the weight gradients for the upstream gradient self.dY."""

@@ -1013,17 +1013,18 @@ tm_status gemm_plain(const void* A, int groups, int rows, int K, const void* Bm,
     p.out_ld = N;
     p.out_elems = (size_t)groups * rows * N;
     p.pos_limit = groups * rows;
-    CUtensorMap ma, mb;
-    if (!map_2d(&ma, A, (uint64_t)groups * rows, K, 128) || !map_2d(&mb, Bm, (uint64_t)groups * N, K, bn))
+    CUtensorMap ma, mb, mo;
+    if (!map_2d(&ma, A, (uint64_t)groups * rows, K, 128) || !map_2d(&mb, Bm, (uint64_t)groups * N, K, bn) ||
+        !map_2d(&mo, out, (uint64_t)groups * rows, N, 32))
         return TM_ERR_CUDA;
-    return cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SLOT, ma, mb, mb, p, dense_grid(p), st));
+    return cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SLOT, ma, mb, mb, p, dense_grid(p), st, &mo));
 }
 
-// dx = d(FFN term)/dx applied to dy, plus add0 and add1 (NULL: none; both in dx's row layout);
+// dx = d(FFN term)/dx applied to dy, plus add0, add1 and add2 (NULL: none; all in dx's row layout);
 // the weight gradients dwg, dwu [banks, F, W] and dwd [banks, W, F].
 tm_status run_dense_bwd(const Geo& g, const void* x, const void* dy, const void* add0, const void* add1,
-                        const tm_swiglu_w* w, void* dx, void* dwg, void* dwu, void* dwd, void* ws, size_t wsb,
-                        cudaStream_t st) {
+                        const void* add2, const tm_swiglu_w* w, void* dx, void* dwg, void* dwu, void* dwd, void* ws,
+                        size_t wsb, cudaStream_t st) {
     const int B = g.B, W = g.W, F = w->hidden, nb = g.banks;
     const int Bp = (B + 63) / 64 * 64;
     Carve c{(uint8_t*)ws};
@@ -1055,7 +1056,7 @@ tm_status run_dense_bwd(const Geo& g, const void* x, const void* dy, const void*
     TM_TRY(cuda_status(launch_transpose(w->w_gate, FW, W, F, W, d.WguT, (size_t)W * 2 * F, 2 * F, F, nb, st)));
     TM_TRY(cuda_status(launch_transpose(w->w_up, FW, W, F, W, d.WguT + F, (size_t)W * 2 * F, 2 * F, F, nb, st)));
     TM_TRY(gemm_plain(d.dGU, nb, B, 2 * F, d.WguT, W, d.dN, st));
-    TM_TRY(cuda_status(launch_rms_bwd(x, d.dN, d.inv_rms, add0, add1, g.map, B, dx, st)));
+    TM_TRY(cuda_status(launch_rms_bwd(x, d.dN, d.inv_rms, add0, add1, add2, g.map, B, dx, st)));
 #undef TM_TRY
     return TM_OK;
 }
@@ -1078,6 +1079,24 @@ size_t block_bwd_sub_ws(const Geo& gm, const Geo& gr, const tm_block* b) {
     const size_t m = dense_bwd_ws(gm, b->mix.dense.hidden), r = dense_bwd_ws(gr, b->rev.dense.hidden);
     n = m > n ? m : n;
     return r > n ? r : n;
+}
+
+// One block's backward: X_rev recomputed into Xr, dX_rev into dXr (both [B,T,D] scratch), then
+// dX = dY + Revert(dH) + extra (extra: NULL or a further gradient of X, e.g. an inter-residual's).
+tm_status run_block_bwd(const Geo& gm, const Geo& gr, const tm_block* b, const void* X, const void* dY,
+                        const void* extra, void* dX, const tm_block_grads* grads, void* Xr, void* dXr, void* ws,
+                        size_t wsb, cudaStream_t st) {
+    tm_status s;
+    // X_rev = Revert(FFN_mix(Norm(Mix(X))) + Mix(X)), as the forward stored it
+    if ((s = run_sublayer(gm, X, X, nullptr, &b->mix, Xr, ws, wsb, st)) != TM_OK) return s;
+    // reverting sub-layer: dX_rev = d FFN_rev(Norm(X_rev)) / d X_rev applied to dY
+    if ((s = run_dense_bwd(gr, Xr, dY, nullptr, nullptr, nullptr, &b->rev.dense, dXr, grads->rev.dw_gate,
+                           grads->rev.dw_up, grads->rev.dw_down, ws, wsb, st)) != TM_OK)
+        return s;
+    // mixing sub-layer on mixed rows: dH_next = Mix(dX_rev); dX = dY + Revert(d FFN_mix applied to
+    // dH_next + dH_next) (+ extra), written through the same row map
+    return run_dense_bwd(gm, X, dXr, dXr, dY, extra, &b->mix.dense, dX, grads->mix.dw_gate, grads->mix.dw_up,
+                         grads->mix.dw_down, ws, wsb, st);
 }
 
 }  // namespace
@@ -1375,7 +1394,7 @@ tm_status tm_pertoken_swiglu_backward(const void* x, const void* dy, const void*
     if (!x || !dy || !dx || !al16(x) || !al16(dy) || !al16(dx) || (dx_add && !al16(dx_add)) || dx == x || dx == dy ||
         !grads_ok(grads))
         return TM_ERR_INVALID_ARG;
-    return run_dense_bwd(g, x, dy, dx_add, nullptr, w, dx, grads->dw_gate, grads->dw_up, grads->dw_down, workspace,
+    return run_dense_bwd(g, x, dy, dx_add, nullptr, nullptr, w, dx, grads->dw_gate, grads->dw_up, grads->dw_down, workspace,
                          workspace_bytes, (cudaStream_t)stream);
 }
 
@@ -1399,20 +1418,69 @@ tm_status tm_block_backward(const void* X, const void* dY, const tm_block* block
     const size_t sub = block_bwd_sub_ws(gm, gr, block);
     if (!workspace || workspace_bytes < 2 * tok + sub || !al16(workspace)) return TM_ERR_WORKSPACE;
     uint8_t* base = (uint8_t*)workspace;
+    return run_block_bwd(gm, gr, block, X, dY, nullptr, dX, grads, base, base + tok, base + 2 * tok, sub,
+                         (cudaStream_t)stream);
+}
+
+size_t tm_stack_backward_workspace_bytes(const tm_shape* shape, const tm_block* blocks, int L, int gap) {
+    if (!blocks || L < 1 || gap < 0) return 0;
+    size_t sub = 0;
+    for (int l = 0; l < L; ++l) {
+        Geo gm, gr;
+        if (check_block_bwd(shape, &blocks[l], &gm, &gr) != TM_OK) return 0;
+        // the block backward's region, and the one a block forward (run_block) needs
+        const size_t n[4] = {block_bwd_sub_ws(gm, gr, &blocks[l]), sublayer_ws(gm, &blocks[l].mix),
+                             sublayer_ws(gr, &blocks[l].rev), block_ws(gm, gr, &blocks[l])};
+        for (size_t v : n) sub = v > sub ? v : sub;
+    }
+    const size_t tok = align256((size_t)shape->B * shape->T * shape->D * 2);
+    return tok * (2 + 2 * (size_t)(L - 1)) + sub;
+}
+
+tm_status tm_stack_backward(const void* X, const void* dY, const tm_block* blocks, int L, int gap,
+                            const tm_shape* shape, void* dX, const tm_block_grads* grads, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    if (!blocks || L < 1 || gap < 0 || !grads) return TM_ERR_INVALID_ARG;
+    Geo gm[64], gr[64];
+    if (L > 64) return TM_ERR_UNSUPPORTED;
+    for (int l = 0; l < L; ++l) {
+        tm_status s = check_block_bwd(shape, &blocks[l], &gm[l], &gr[l]);
+        if (s != TM_OK) return s;
+        if (!grads_ok(&grads[l].mix) || !grads_ok(&grads[l].rev)) return TM_ERR_INVALID_ARG;
+    }
+    if (!X || !dY || !dX || !al16(X) || !al16(dY) || !al16(dX) || dX == X || dX == dY) return TM_ERR_INVALID_ARG;
+    const size_t need = tm_stack_backward_workspace_bytes(shape, blocks, L, gap);
+    if (need == 0) return TM_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < need || !al16(workspace)) return TM_ERR_WORKSPACE;
+    const size_t tok = align256((size_t)shape->B * shape->T * shape->D * 2);
+    uint8_t* base = (uint8_t*)workspace;
     void* Xr = base;
     void* dXr = base + tok;
-    void* ws = base + 2 * tok;
+    // xs[l] = X_l (l = 1 .. L-1), gs[l] = the gradient of X_l (l = 1 .. L-1)
+    uint8_t* xs = base + 2 * tok;
+    uint8_t* gs = xs + (size_t)(L - 1) * tok;
+    void* ws = gs + (size_t)(L - 1) * tok;
+    const size_t wsb = workspace_bytes - (size_t)((uint8_t*)ws - base);
+    auto xl = [&](int l) -> const void* { return l == 0 ? X : (const void*)(xs + (size_t)(l - 1) * tok); };
+    auto gl = [&](int l) -> void* { return l == 0 ? dX : (l == L ? const_cast<void*>(dY) : (void*)(gs + (size_t)(l - 1) * tok)); };
     cudaStream_t st = (cudaStream_t)stream;
-    // X_rev = Revert(FFN_mix(Norm(Mix(X))) + Mix(X)), as the forward stored it
-    if ((s = run_sublayer(gm, X, X, nullptr, &block->mix, Xr, ws, sub, st)) != TM_OK) return s;
-    // reverting sub-layer: dX_rev = d FFN_rev(Norm(X_rev)) / d X_rev applied to dY
-    if ((s = run_dense_bwd(gr, Xr, dY, nullptr, nullptr, &block->rev.dense, dXr, grads->rev.dw_gate,
-                           grads->rev.dw_up, grads->rev.dw_down, ws, sub, st)) != TM_OK)
-        return s;
-    // mixing sub-layer on mixed rows: dH_next = Mix(dX_rev); dX = dY + Revert(d FFN_mix applied to
-    // dH_next + dH_next), written through the same row map
-    return run_dense_bwd(gm, X, dXr, dXr, dY, &block->mix.dense, dX, grads->mix.dw_gate, grads->mix.dw_up,
-                         grads->mix.dw_down, ws, sub, st);
+    tm_status s;
+    // the forward again, keeping every block input: X_l = Block_l(X_{l-1}) (+ X_{l-gap}), as
+    // tm_stack_forward computes it
+    for (int l = 1; l < L; ++l) {
+        const void* extra = (gap > 0 && l % gap == 0 && l < L) ? xl(l - gap) : nullptr;
+        if ((s = run_block(shape, &blocks[l - 1], xl(l - 1), extra, (void*)xl(l), Xr, ws, wsb, st)) != TM_OK) return s;
+    }
+    // backward, last block first: the gradient of X_{l-1} is block l's input gradient plus, when
+    // X_{l-1+gap} = Block(...) + X_{l-1} (an inter-residual), the gradient of X_{l-1+gap}
+    for (int l = L; l >= 1; --l) {
+        const int j = l - 1 + gap;
+        const void* extra = (gap > 0 && j % gap == 0 && j < L) ? gl(j) : nullptr;
+        if ((s = run_block_bwd(gm[l - 1], gr[l - 1], &blocks[l - 1], xl(l - 1), gl(l), extra, gl(l - 1), &grads[l - 1],
+                               Xr, dXr, ws, wsb, st)) != TM_OK)
+            return s;
+    }
+    return TM_OK;
 }
 
 tm_status tm_get_device_error(void* stream) {

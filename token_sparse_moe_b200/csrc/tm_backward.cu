@@ -50,29 +50,41 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const __nv_bfloat16* __re
     }
 }
 
-// out[g][c][r] = in[g][r][c] for r < R and 0 for R <= r < Rp (c < C): 32 x 32 tiles staged in
-// shared memory, so that reads run along c and writes along r.  Grid (Rp / 32, C / 32, groups),
-// 256 threads.  The tile rows are 34 elements (17 words) apart, so the column reads of a warp
-// hit 32 different banks.
+// out[g][c][r] = in[g][r][c] for r < R and 0 for R <= r < Rp (c < C): 64 x 64 tiles staged in
+// shared memory, read with 16-byte loads along c and written with 16-byte stores along r (eight
+// threads cover 128 contiguous bytes on both sides).  Grid (Rp / 64, C / 64, groups), 256 threads.
+// In shared memory element (r, c) of the tile sits in row r at 8-element piece (c / 8) ^ (r / 8 % 8),
+// so the column reads of a warp (eight row pieces, four columns) fall in distinct banks.  C, Rp,
+// the leading dimensions and group strides are multiples of 8 elements and both bases 16-byte
+// aligned (checked by the launcher), so every 8-element piece is whole and aligned.
 __global__ void __launch_bounds__(256) transpose_kernel(const __nv_bfloat16* __restrict__ in, size_t in_gs, int in_ld,
                                                         int R, int C, __nv_bfloat16* __restrict__ out, size_t out_gs,
                                                         int out_ld, int Rp) {
-    __shared__ __nv_bfloat16 tile[32][34];
+    __shared__ __align__(16) uint16_t tile[64 * 64];
     const int g = blockIdx.z;
-    const int r0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    const int r0 = blockIdx.x * 64, c0 = blockIdx.y * 64;
     const __nv_bfloat16* src = in + (size_t)g * in_gs;
 #pragma unroll
-    for (int j = ty; j < 32; j += 8) {
-        const int r = r0 + j, c = c0 + tx;
-        tile[j][tx] = (r < R && c < C) ? src[(size_t)r * in_ld + c] : __float2bfloat16_rn(0.f);
+    for (int i = threadIdx.x; i < 512; i += 256) {
+        const int rr = i >> 3, q = i & 7;
+        const int r = r0 + rr, c = c0 + q * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r < R && c < C) v = __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * in_ld + c));
+        *reinterpret_cast<uint4*>(&tile[rr * 64 + ((q ^ ((rr >> 3) & 7)) << 3)]) = v;
     }
     __syncthreads();
     __nv_bfloat16* dst = out + (size_t)g * out_gs;
 #pragma unroll
-    for (int j = ty; j < 32; j += 8) {
-        const int c = c0 + j, r = r0 + tx;
-        if (c < C && r < Rp) dst[(size_t)c * out_ld + r] = tile[tx][j];
+    for (int i = threadIdx.x; i < 512; i += 256) {
+        const int cc = i >> 3, q = i & 7;
+        const int c = c0 + cc, r = r0 + q * 8;
+        if (c >= C || r >= Rp) continue;
+        const int col = (((cc >> 3) ^ q) << 3) + (cc & 7);   // rows q*8 .. q*8+7 share the piece swizzle q
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w[k] = (uint32_t)tile[(q * 8 + 2 * k) * 64 + col] | ((uint32_t)tile[(q * 8 + 2 * k + 1) * 64 + col] << 16);
+        *reinterpret_cast<uint4*>(dst + (size_t)c * out_ld + r) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -110,14 +122,15 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const __nv_bfloat16* __
     }
 }
 
-// One warp per (b, bank) row: dx = r (dn - xh mean(dn xh)) + add0 + add1, with xh = x r (x
+// One warp per (b, bank) row: dx = r (dn - xh mean(dn xh)) + add0 + add1 + add2, with xh = x r (x
 // re-read through the row map, r from the row pass), dn bank-major [banks][B][W]; dx and the
 // optional addends go through the row map.
 __global__ void __launch_bounds__(256) rms_bwd_kernel(const __nv_bfloat16* __restrict__ x,
                                                       const __nv_bfloat16* __restrict__ dN,
                                                       const float* __restrict__ inv_rms,
                                                       const __nv_bfloat16* __restrict__ add0,
-                                                      const __nv_bfloat16* __restrict__ add1, RowMap m, int B,
+                                                      const __nv_bfloat16* __restrict__ add1,
+                                                      const __nv_bfloat16* __restrict__ add2, RowMap m, int B,
                                                       __nv_bfloat16* __restrict__ dx) {
     const int lane = threadIdx.x & 31;
     const int nrows = B * m.banks;
@@ -137,16 +150,17 @@ __global__ void __launch_bounds__(256) rms_bwd_kernel(const __nv_bfloat16* __res
         const float mean = warp_sum(dot) / (float)m.W;
         for (int c = lane * 8; c < m.W; c += 256) {
             const size_t e = row_elem(m, b, bank, c);
-            float v[8], d[8], a0[8], a1[8];
+            float v[8], d[8], a0[8], a1[8], a2[8];
             Vec<__nv_bfloat16>::load(x + e, v);
             Vec<__nv_bfloat16>::load(dn + c, d);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) a0[i] = a1[i] = 0.f;
+            for (int i = 0; i < 8; ++i) a0[i] = a1[i] = a2[i] = 0.f;
             if (add0) Vec<__nv_bfloat16>::load(add0 + e, a0);
             if (add1) Vec<__nv_bfloat16>::load(add1 + e, a1);
+            if (add2) Vec<__nv_bfloat16>::load(add2 + e, a2);
             float o[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = r * (d[i] - v[i] * r * mean) + a0[i] + a1[i];
+            for (int i = 0; i < 8; ++i) o[i] = r * (d[i] - v[i] * r * mean) + a0[i] + a1[i] + a2[i];
             *reinterpret_cast<uint4*>(dx + e) = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
                                                            pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
         }
@@ -169,9 +183,12 @@ cudaError_t launch_bwd_rows(const void* x, const void* dy, RowMap m, int B, floa
 cudaError_t launch_transpose(const void* in, size_t in_gs, int in_ld, int R, int C, void* out, size_t out_gs,
                              int out_ld, int Rp, int groups, cudaStream_t st) {
     if (groups <= 0 || R <= 0 || C <= 0 || Rp < R) return cudaErrorInvalidValue;
-    if ((C + 31) / 32 > 65535 || groups > 65535) return cudaErrorInvalidValue;
+    if ((C + 63) / 64 > 65535 || groups > 65535) return cudaErrorInvalidValue;
+    if (C % 8 || Rp % 8 || in_ld % 8 || out_ld % 8 || in_gs % 8 || out_gs % 8 || in_ld < C || out_ld < Rp ||
+        ((uintptr_t)in & 15) || ((uintptr_t)out & 15))
+        return cudaErrorInvalidValue;
     ProfileScope ps_("transpose", st);
-    dim3 grid((Rp + 31) / 32, (C + 31) / 32, groups);
+    dim3 grid((Rp + 63) / 64, (C + 63) / 64, groups);
     transpose_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)in, in_gs, in_ld, R, C, (__nv_bfloat16*)out, out_gs,
                                            out_ld, Rp);
     return cudaGetLastError();
@@ -190,11 +207,11 @@ cudaError_t launch_swiglu_bwd(const void* Gp, const void* Up, const void* dH, si
 }
 
 cudaError_t launch_rms_bwd(const void* x, const void* dN, const float* inv_rms, const void* add0, const void* add1,
-                           RowMap m, int B, void* dx, cudaStream_t st) {
+                           const void* add2, RowMap m, int B, void* dx, cudaStream_t st) {
     ProfileScope ps_("rms_bwd", st);
     rms_bwd_kernel<<<rows_grid((long)B * m.banks), 256, 0, st>>>(
         (const __nv_bfloat16*)x, (const __nv_bfloat16*)dN, inv_rms, (const __nv_bfloat16*)add0,
-        (const __nv_bfloat16*)add1, m, B, (__nv_bfloat16*)dx);
+        (const __nv_bfloat16*)add1, (const __nv_bfloat16*)add2, m, B, (__nv_bfloat16*)dx);
     return cudaGetLastError();
 }
 

@@ -6,7 +6,7 @@
 //                s = per-row 1/rms, i.e. the pre-RMSNorm folded into the epilogue)
 //   EPI_RESID  : y = A Wd^T + residual (+ inter-residual), stored through the row map
 //                (for mixed rows this store IS the Revert permutation)
-//   EPI_SLOT   : slot row = A Wd^T (a routed expert's output, bf16)
+//   EPI_SLOT   : plain rows out = A B^T (bf16), staged and bulk-stored (the backward's contractions)
 //   EPI_COMBINE: y = A Ws^T + sum_j gate_j * slot_j + residual (+ inter-residual):
 //                shared expert GEMM2 plus the MoE combine, in fixed order
 // A operand sources: a plain 2-D TMA map (hidden rows), a 3-D TMA map over
@@ -109,7 +109,7 @@ struct GemmCfg {
     static constexpr int NTHREADS = NWARPS * 32;
     static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
     // output staging: one 32-row x 64-column bf16 box (4 KB) per epilogue warp
-    static constexpr bool STAGED = EPI == EPI_SWIGLU || EPI == EPI_SLOT_PERM || EPI == EPI_SUM;
+    static constexpr bool STAGED = EPI == EPI_SWIGLU || EPI == EPI_SLOT_PERM || EPI == EPI_SUM || EPI == EPI_SLOT;
     static constexpr int OFF_STG = STAGES * STAGE_BYTES;
     static constexpr int STG_BYTES = STAGED ? EPI_WARPS * 4096 : 0;
     static constexpr int OFF_ID = OFF_STG + STG_BYTES;             // 16 x 16 identity (EPI_SUM), 1 KB
@@ -615,17 +615,31 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
                     }
                 }
             } else if (EPI == EPI_SLOT) {
-                __nv_bfloat16* dst = p.out + (size_t)pos * p.out_ld + ti.n * BN;
+                // plain rows out[pos, n*BN + c]: a bulk tensor store per 32 x 64 box when all 32 rows of
+                // this warp belong to the tile's group (tmO: the output rows, 32-row boxes); else the
+                // valid rows through coalesced stores from the same staged box
+                const bool box = __all_sync(0xffffffffu, valid);
+                const long long my_off = valid ? (long long)pos * p.out_ld + ti.n * BN : -1ll;
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    float v[32];
-                    tmem_ld32(taddr + c, v);
-                    if (valid) {
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+                for (int c = 0; c < BN; c += 64) {
+                    uint32_t pk[32];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            d4[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                                               pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+                    for (int h = 0; h < 2; ++h) {
+                        float v[32];
+                        tmem_ld32(taddr + c + 32 * h, v);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) pk[16 * h + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                    }
+                    stage_row(pk);
+                    if (box) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmO, stg, ti.n * BN + c, ti.row0 + q * 32);
+                            bulk_commit_group();
+                        }
+                    } else {
+                        copy_rows(my_off, c);
                     }
                 }
             } else {   // EPI_RESID / EPI_COMBINE

@@ -109,15 +109,16 @@ cudaError_t launch_tokenize(int dtype, const void* groups, const void* w_group, 
 // row pass: inv_rms [banks][B], xh = x * inv_rms and a copy of dy, both bank-major [banks][B][W]
 cudaError_t launch_bwd_rows(const void* x, const void* dy, RowMap m, int B, float eps, void* xh, void* dyb,
                             float* inv_rms, cudaStream_t st);
-// out[g][c][r] = in[g][r][c] (r < R, c < C), zero for R <= r < Rp; element strides per group / row
+// out[g][c][r] = in[g][r][c] (r < R, c < C), zero for R <= r < Rp; element strides per group / row;
+// C, Rp, strides multiples of 8 elements, bases 16-byte aligned (else cudaErrorInvalidValue)
 cudaError_t launch_transpose(const void* in, size_t in_gs, int in_ld, int R, int C, void* out, size_t out_gs,
                              int out_ld, int Rp, int groups, cudaStream_t st);
 // SwiGLU derivative over [rows, F]: dGU [rows, 2F] = (dg | du), Hd [rows, F] = silu(g) * u
 cudaError_t launch_swiglu_bwd(const void* Gp, const void* Up, const void* dH, size_t rows, int F, void* dGU, void* Hd,
                               cudaStream_t st);
-// RMSNorm derivative: dx = inv_rms (dn - xh mean(dn xh)) + add0 + add1 through the row map
+// RMSNorm derivative: dx = inv_rms (dn - xh mean(dn xh)) + add0 + add1 + add2 through the row map
 cudaError_t launch_rms_bwd(const void* x, const void* dN, const float* inv_rms, const void* add0, const void* add1,
-                           RowMap m, int B, void* dx, cudaStream_t st);
+                           const void* add2, RowMap m, int B, void* dx, cudaStream_t st);
 
 // fp32 CUDA-core grouped GEMM with the same tile space and epilogues as the tcgen05 one.
 // A is x (gathered through amap) when epi == EPI_SWIGLU, else hidden rows [positions, K].
