@@ -126,6 +126,25 @@ def test_stack_backward_with_inter_residual_matches_finite_differences():
     assert not np.allclose(BW.stack_backward(X, cfg0, get, dY)["dX"], g["dX"])
 
 
+@pytest.mark.parametrize("L,gap", [(3, 1), (4, 2)])
+def test_stack_backward_gap_forms_match_finite_differences(L, gap):
+    """gap 1 (every block but the last adds its input back) and two blocks after an
+    inter-residual (L = 4, gap = 2: X_2 += X_0, nothing after the last block)."""
+    cfg = _cfg(2, 4, 2, L=L, gap=gap)
+    rng = np.random.default_rng(10 + L + gap)
+    w = _weights(cfg, rng)
+    get = lambda l, s, j: w[(l, s, j)]
+    X = rng.standard_normal((cfg.B, 2, 4))
+    dY = rng.standard_normal((cfg.B, 2, 4))
+
+    def loss():
+        return float(np.sum(dY * O.stack_forward(X, cfg, get)["Y"]))
+    g = BW.stack_backward(X, cfg, get, dY)
+    assert close(g["dX"], fd_grad(loss, X))
+    assert close(g["blocks"][0]["rev"]["dw_gate"][1], fd_grad(loss, w[(0, 1, 1)]["w_gate"]))
+    assert close(g["blocks"][L - 2]["mix"]["dw_down"][0], fd_grad(loss, w[(L - 2, 0, 0)]["w_down"]))
+
+
 def test_zero_down_projection_block_is_identity():
     cfg = _cfg(2, 4, 2)
     rng = np.random.default_rng(6)
