@@ -413,8 +413,18 @@ def run_ours(args, cfg, rank, world, local_rank):
     Xd = torch.empty_like(X)
     # the backward step's inputs are X and dY (both copied in), its result dX (copied back)
     dYh = dY.cpu().pin_memory() if args.backward else None
-    host = (lambda: run.run_host(Xh, Yh, Xd, Y, dYh, stream)) if args.backward else \
-        (lambda: run.run_host(Xh, Yh, Xd, Y, stream))
+    chunks = args.e2e_chunks if not (args.backward or args.fp8) else 1
+    if args.backward:
+        host = lambda: run.run_host(Xh, Yh, Xd, Y, dYh, stream)
+    elif chunks > 1:
+        host = lambda: run.run_host(Xh, Yh, Xd, Y, stream, chunks=chunks)
+    else:
+        host = lambda: run.run_host(Xh, Yh, Xd, Y, stream)
+    # the whole batch on the device once more, for the bit-exact check of the end-to-end result
+    Yref = torch.empty_like(Y)
+    with torch.cuda.stream(stream):
+        run(X, Yref, stream)
+    stream.synchronize()
     with torch.cuda.stream(stream):
         for _ in range(3):
             host()
@@ -427,6 +437,7 @@ def run_ours(args, cfg, rank, world, local_rank):
             eve[i][1].record(stream)
         stream.synchronize()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eve) / Ke, world, dev)
+    e2e_exact = bool(torch.equal(Yh, Yref.cpu()))
     io_bytes = X.numel() * X.element_size()
     h2d_bytes = io_bytes * (2 if args.backward else 1)
 
@@ -483,7 +494,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(cfg.B, world, e2e_ms), "unit": "samples/s", "h2d_bytes_per_step": h2d_bytes,
-                "d2h_bytes_per_step": io_bytes, "ms_per_step": e2e_ms, "steps": Ke},
+                "d2h_bytes_per_step": io_bytes, "ms_per_step": e2e_ms, "steps": Ke, "chunks": chunks,
+                "matches_device_result": e2e_exact},
         "gpu_launches": int(launches),
         "launches_per_step": launches / K,
         "kernels": {k: {"launches": v["launches"], "avg_ms": v["total_ms"] / v["launches"],
@@ -508,6 +520,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-samples", type=int, default=128)
     ap.add_argument("--steps-ref", type=int, default=None)
+    ap.add_argument("--e2e-chunks", type=int, default=8,
+                    help="end-to-end leg: split the batch into this many chunks whose host copies overlap "
+                         "the compute (forward only)")
     ap.add_argument("--backward", action="store_true",
                     help="the dense block backward (training): its own line, not the forward metric's")
     ap.add_argument("--fp8", action="store_true",

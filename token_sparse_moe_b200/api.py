@@ -260,13 +260,53 @@ class StackRunner:
 
 
     def run_host(self, X_host: torch.Tensor, Y_host: torch.Tensor, X_dev: torch.Tensor, Y_dev: torch.Tensor,
-                 stream=None) -> torch.Tensor:
-        """End to end on one stream: pinned host X -> device, stack forward, device -> pinned host Y."""
+                 stream=None, chunks: int = 1) -> torch.Tensor:
+        """End to end: pinned host X -> device, stack forward, device -> pinned host Y.
+
+        chunks == 1: all on `stream`.  chunks > 1: the batch is split along the samples (which are
+        independent, so every output is the same bits) and pipelined over three streams: the
+        host-to-device copy of chunk i+1 and the device-to-host copy of chunk i-1 run while chunk i
+        computes on `stream`.  All work of the call lies between an event recorded on `stream` at
+        entry and `stream`'s wait for the last copy, so events on `stream` around the call time
+        all of it; the next call's work on the same buffers starts only after that."""
         s = torch.cuda.current_stream() if stream is None else stream
-        with torch.cuda.stream(s):
-            X_dev.copy_(X_host, non_blocking=True)
-            self(X_dev, Y_dev, s)
-            Y_host.copy_(Y_dev, non_blocking=True)
+        B = X_host.shape[0]
+        if chunks <= 1 or B < 2 * chunks:
+            with torch.cuda.stream(s):
+                X_dev.copy_(X_host, non_blocking=True)
+                self(X_dev, Y_dev, s)
+                Y_host.copy_(Y_dev, non_blocking=True)
+            return Y_host
+        if not hasattr(self, "_pipe"):
+            self._pipe = (torch.cuda.Stream(device=X_dev.device), torch.cuda.Stream(device=X_dev.device))
+        h2d, d2h = self._pipe
+        bounds = [B * i // chunks for i in range(chunks + 1)]
+        start = torch.cuda.Event()
+        start.record(s)
+        h2d.wait_event(start)
+        done_in, done_out = [], []
+        for i in range(chunks):
+            a, b = bounds[i], bounds[i + 1]
+            with torch.cuda.stream(h2d):
+                X_dev[a:b].copy_(X_host[a:b], non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(h2d)
+                done_in.append(e)
+        for i in range(chunks):
+            a, b = bounds[i], bounds[i + 1]
+            s.wait_event(done_in[i])
+            sh = A.tm_shape(b - a, self.sh.T, self.sh.D, self.sh.H, self.sh.dtype, self.sh.eps)
+            A.check(lib().tm_stack_forward(_p(X_dev[a:b]), self.arr, len(self.blocks), self.gap, ctypes.byref(sh),
+                                           _p(Y_dev[a:b]), _p(self.ws), self.ws.numel(), _s(s)), "tm_stack_forward")
+            e = torch.cuda.Event()
+            e.record(s)
+            d2h.wait_event(e)
+            with torch.cuda.stream(d2h):
+                Y_host[a:b].copy_(Y_dev[a:b], non_blocking=True)
+                e2 = torch.cuda.Event()
+                e2.record(d2h)
+                done_out.append(e2)
+        s.wait_event(done_out[-1])
         return Y_host
 
 
