@@ -162,3 +162,112 @@ def test_zero_down_projection_block_is_identity():
     for j in range(cfg.banks(1)):
         assert not np.any(g["rev"]["dw_gate"][j]) and not np.any(g["rev"]["dw_up"][j])
         assert np.any(g["rev"]["dw_down"][j])
+
+
+# ------------------------------------------------------------------ Sparse-Pertoken MoE
+def _moe_bank(rng, W, E, Fe, Fs, down=0.7):
+    bw = {"w_router": rng.standard_normal((E, W)),
+          "we_gate": rng.standard_normal((E, Fe, W)), "we_up": rng.standard_normal((E, Fe, W)),
+          "we_down": down * rng.standard_normal((E, W, Fe))}
+    if Fs:
+        bw.update({"ws_gate": rng.standard_normal((Fs, W)), "ws_up": rng.standard_normal((Fs, W)),
+                   "ws_down": down * rng.standard_normal((W, Fs))})
+    return bw
+
+
+def _clear_of_ties(x, bw, k, eps, gain=None, min_gap=1e-3):
+    """Finite differences of a top-k MoE are valid only away from routing ties (the chosen set
+    must not change under the 1e-6 perturbations)."""
+    return O.route(O.rmsnorm(x, eps, gain), bw["w_router"], k)["gap"].min() > min_gap
+
+
+@pytest.mark.parametrize("E,k,Fs,with_gain", [(4, 2, 3, False), (4, 2, 0, True), (3, 3, 2, False), (5, 1, 4, True)])
+def test_moe_backward_matches_finite_differences(E, k, Fs, with_gain):
+    rng = np.random.default_rng(20 + E * 10 + k + Fs)
+    R, W, Fe = 6, 8, 5
+    alpha = E / k
+    bw = _moe_bank(rng, W, E, Fe, Fs)
+    gain = 1 + 0.3 * rng.standard_normal(W) if with_gain else None
+    x = rng.standard_normal((R, W))
+    dy = rng.standard_normal((R, W))
+    eps = 1e-3
+    assert _clear_of_ties(x, bw, k, eps, gain)
+
+    def loss():
+        return float(np.sum(dy * O.sp_moe(O.rmsnorm(x, eps, gain), bw, k, alpha)["out"]))
+    g = BW.moe_ffn_backward(x, dy, bw, k, alpha, eps, gain)
+    assert close(g["dx"], fd_grad(loss, x))
+    assert close(g["dw_router"], fd_grad(loss, bw["w_router"]))
+    chosen = sorted(set(g["idx"].ravel().tolist()))
+    for e in (chosen[0], chosen[-1]):
+        for name in ("we_gate", "we_up", "we_down"):
+            assert close(g["d" + name][e], fd_grad(loss, bw[name][e])), (name, e)
+    if Fs:
+        for name in ("ws_gate", "ws_up", "ws_down"):
+            assert close(g["d" + name], fd_grad(loss, bw[name])), name
+    else:
+        assert "dws_gate" not in g
+    if with_gain:
+        assert close(g["dgain"], fd_grad(loss, gain))
+
+
+def test_moe_backward_special_cases():
+    rng = np.random.default_rng(31)
+    R, W, Fe = 9, 8, 4
+    x = rng.standard_normal((R, W))
+    dy = rng.standard_normal((R, W))
+    # E = k = 1: p = 1 whatever the logit, so the router gets no gradient, exactly
+    b1 = _moe_bank(rng, W, 1, Fe, 3)
+    g1 = BW.moe_ffn_backward(x, dy, b1, 1, 1.0, 1e-6)
+    assert not np.any(g1["dw_router"])
+    # ... and the expert then acts as a second shared expert: its gradients are the dense ones
+    dense = BW.swiglu_ffn_backward(x, dy, {"w_gate": b1["we_gate"][0], "w_up": b1["we_up"][0],
+                                           "w_down": b1["we_down"][0]}, 1e-6)
+    assert np.allclose(g1["dwe_down"][0], dense["dw_down"], rtol=1e-12, atol=1e-12)
+    # an expert that no row chose gets exactly zero gradients (choices forced to experts 0..4)
+    b = _moe_bank(rng, W, 6, Fe, 0)
+    forced = np.array([[i % 5, (i + 1) % 5] for i in range(R)])
+    g = BW.moe_ffn_backward(x, dy, b, 2, 3.0, 1e-6, forced_idx=forced)
+    assert 5 not in g["idx"]
+    assert not np.any(g["dwe_gate"][5]) and not np.any(g["dwe_up"][5]) and not np.any(g["dwe_down"][5])
+    # the router gradient of every row sums to zero over the experts (softmax shift invariance):
+    # sum_e dz_e = 0, hence sum_e dWr_e = 0
+    assert np.allclose(g["dw_router"].sum(axis=0), 0.0, atol=1e-10 * np.abs(g["dw_router"]).max())
+
+
+def test_moe_backward_scales_with_alpha():
+    """Without a shared expert the output is linear in alpha, so every gradient is too."""
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((7, 8))
+    dy = rng.standard_normal((7, 8))
+    b = _moe_bank(rng, 8, 4, 5, 0)
+    g1 = BW.moe_ffn_backward(x, dy, b, 2, 1.0, 1e-6)
+    g3 = BW.moe_ffn_backward(x, dy, b, 2, 3.0, 1e-6)
+    for key in ("dx", "dw_router", "dwe_gate", "dwe_down"):
+        assert np.allclose(g3[key], 3.0 * g1[key], rtol=1e-12, atol=1e-12), key
+
+
+def test_moe_block_backward_matches_finite_differences():
+    cfg = Config("tiny_moe", B=3, T=2, D=4, H=2, L=1, dtype="f32",
+                 mix=FFNSpec("moe", E=3, k=2, hidden_e=3, hidden_s=2, alpha=1.5),
+                 rev=FFNSpec("moe", E=4, k=1, hidden_e=2, hidden_s=3, alpha=4.0), gap=0, eps=1e-6)
+    rng = np.random.default_rng(33)
+    w = {}
+    for sub in (0, 1):
+        s = cfg.ffn(sub)
+        for j in range(cfg.banks(sub)):
+            w[(0, sub, j)] = _moe_bank(rng, cfg.width(sub), s.E, s.hidden_e, s.hidden_s)
+    get = lambda l, s, j: w[(l, s, j)]
+    X = rng.standard_normal((cfg.B, cfg.T, cfg.D))
+    dY = rng.standard_normal((cfg.B, cfg.T, cfg.D))
+    # every routed row of both sub-layers clear of ties
+    fwd = O.block_forward(X, cfg, 0, get)
+    for key in ("mix", "rev"):
+        assert np.min(fwd[key]["gap"]) > 1e-3, key
+
+    def loss():
+        return float(np.sum(dY * O.block_forward(X, cfg, 0, get)["Y"]))
+    g = BW.block_backward(X, cfg, 0, get, dY)
+    assert close(g["dX"], fd_grad(loss, X))
+    assert close(g["mix"]["dw_router"][1], fd_grad(loss, w[(0, 0, 1)]["w_router"]))
+    assert close(g["rev"]["dws_up"][0], fd_grad(loss, w[(0, 1, 0)]["ws_up"]))
