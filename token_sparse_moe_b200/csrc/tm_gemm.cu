@@ -175,22 +175,6 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
     X(256, A_TMA_2D, EPI_SUM) X(192, A_TMA_2D, EPI_SUM) X(128, A_TMA_2D, EPI_SUM) \
     X(64, A_TMA_3D, EPI_ROUTE) X(64, A_TMA_MIX, EPI_ROUTE)
 
-bool grouped_gemm_supported(int bn, int a_mode, int epi) {
-#define X(BN, AM, EP) if (bn == BN && a_mode == AM && epi == EP) return true;
-    TM_GEMM_TABLE(X)
-#undef X
-    return false;
-}
-
-int grouped_gemm_smem(int bn, int a_mode) {
-    if (a_mode == A_GATHER) return bn == 256 ? GemmCfg<256, A_GATHER>::SMEM_BYTES : GemmCfg<128, A_GATHER>::SMEM_BYTES;
-    switch (bn) {
-        case 256: return GemmCfg<256, A_TMA_2D>::SMEM_BYTES;
-        case 192: return GemmCfg<192, A_TMA_2D>::SMEM_BYTES;
-        default: return GemmCfg<128, A_TMA_2D>::SMEM_BYTES;
-    }
-}
-
 cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                                     const CUtensorMap& tmB1, const CUtensorMap& tmS0, const CUtensorMap& tmS1,
                                     const CUtensorMap& tmS2, const GemmParams& p, int grid, cudaStream_t st,

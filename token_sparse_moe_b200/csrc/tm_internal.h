@@ -39,7 +39,6 @@ cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorM
 cudaError_t launch_grouped_gemm(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                                 const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st,
                                 const CUtensorMap* tmO = nullptr);
-bool grouped_gemm_supported(int bn, int a_mode, int epi);
 
 // ---- fused dense sub-layer (row width 128 / 256) --------------------------------
 bool fused_supported(int W, int a_mode);
@@ -65,7 +64,6 @@ cudaError_t launch_fused128_block(int W, bool f8, const FusedMaps& mix, const Fu
 // CTA-pair version (2-SM MMAs, clusters of 2): grid = 2 x clusters; weight maps with half-size boxes
 cudaError_t launch_fused2(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
                           const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st);
-int grouped_gemm_smem(int bn, int a_mode);
 
 // ---- CUDA-core kernels ------------------------------------------------------------
 // dtype: 0 fp32, 1 bf16.
