@@ -215,3 +215,34 @@ def test_stack_backward_queries():
     x, dy, dx, ws = (ctypes.c_void_p(a) for a in (0x200000, 0x400000, 0x600000, 0x800000))
     assert lib.tm_stack_backward(x, dy, arr, 4, 2, ctypes.byref(sh), dx, garr, ws, 16, None) == A.TM_ERR_WORKSPACE
     assert lib.tm_stack_backward(x, dy, arr, 4, 2, ctypes.byref(sh), x, garr, ws, 1 << 40, None) == A.TM_ERR_INVALID_ARG
+
+
+def test_plain_c_client_links_and_calls(tmp_path):
+    """A C program (no Python, no torch) includes tm.h, links libtm.so and gets answers from the
+    host-side calls: version, status strings, workspace sizes and argument validation."""
+    src = tmp_path / "client.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "tm.h"
+int main(void) {
+  tm_shape s = {4096, 16, 256, 16, TM_BF16, 1e-6f};
+  tm_swiglu_w mix = {16, 256, 1024, (void*)0x100000, (void*)0x200000, (void*)0x300000};
+  tm_swiglu_w rev = {16, 256, 1024, (void*)0x400000, (void*)0x500000, (void*)0x600000};
+  tm_block b = {{0, 0, mix}, {0, 0, rev}};
+  size_t ws = tm_workspace_bytes(&s, &b, 1, 0);
+  size_t bw = tm_block_backward_workspace_bytes(&s, &b);
+  tm_shape bad = s; bad.D = 250;
+  tm_status st = tm_pertoken_swiglu((void*)0x700000, 0, TM_LAYOUT_MIXED, &bad, 0, &mix, (void*)0x800000,
+                                    (void*)0x900000, (size_t)1 << 30, 0);
+  printf("%d %zu %zu %d %s\n", tm_version(), ws, bw, (int)st, tm_status_string(st));
+  return 0;
+}
+''')
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(A.LIB_PATH)
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-ltm",
+                    "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert out[0] == "100"
+    assert int(out[1]) > 4096 * 16 * 256 * 2 and int(out[2]) > int(out[1])
+    assert int(out[3]) == A.TM_ERR_INVALID_ARG
