@@ -162,7 +162,9 @@ def test_backward_deterministic_bits():
             assert torch.equal(ga[s][k], gb[s][k]), (s, k)
 
 
-def test_backward_rejects_gain_and_moe():
+def test_backward_rejects_a_norm_gain():
+    """The GPU backward supports gain 1 only; a gain is refused before any launch (MoE blocks are
+    refused the same way, checked on the CPU in test_abi)."""
     cfg = CASES[0]
     X, dY = seeded(cfg)
     sw = api.sublayer_from_synth(cfg, 0, 1, DEV, with_gain=True)
