@@ -520,6 +520,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-samples", type=int, default=128)
     ap.add_argument("--steps-ref", type=int, default=None)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="run the workload with this many samples instead of its own B (small cases for "
+                         "profiler captures; the line's workload string carries the B used)")
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="end-to-end leg: split the batch into this many chunks whose host copies overlap "
                          "the compute (forward only)")
@@ -532,6 +535,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     cfg = S.CONFIGS[args.workload]
+    if args.batch is not None:
+        if args.batch < 1:
+            raise SystemExit("--batch must be positive")
+        cfg = cfg.with_(B=args.batch)
     if args.impl == "reference":
         args.steps_ref = args.steps_ref or min(args.steps, 20)
         run_reference(args, cfg, rank)
