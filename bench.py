@@ -8,10 +8,15 @@ HBM.  Each timed step is bracketed by CUDA events on the launching stream; a 256
 write between steps flushes the 126 MB L2, so every step starts cold.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+                  [--batch B] [--e2e-chunks C] [--fp8 | --backward]
 
 N > 1 (under torchrun): every rank runs its own batch (weak scaling, no data-path
 collective); the step time is the max over ranks.  --impl reference times the CPU
-float64 oracle on the host cores (rank 0 only) on a bounded sample of the workload.
+float64 oracle on the host cores (rank 0 only) on a bounded sample of the workload.  The
+end-to-end leg copies each step's batch from pinned host memory and the result back, in C
+sample chunks pipelined against the compute (the result is checked bit for bit against the
+full-batch device run).  --fp8 and --backward print their own lines (the FP8 serving path, the
+dense block backward).
 """
 from __future__ import annotations
 
