@@ -1,22 +1,26 @@
 #!/usr/bin/env python
 """Throughput of the TokenMixer-Large forward on B200 (one JSON line on rank 0).
 
-A step is one tm_stack_forward over one batch of the dense bf16 block workload
-(B=4096 samples, T=16 tokens, D=256, H=16 heads, per-token SwiGLU hidden 1024 in
-both sub-layers, L=1) with synthetic inputs and random weights already resident in
-HBM.  Each timed step is bracketed by CUDA events on the launching stream; a 256 MB
-write between steps flushes the 126 MB L2, so every step starts cold.
+A step is one tm_stack_forward over one batch of a workload with synthetic inputs and random
+weights already resident in HBM.  The default workload is the large Sparse-Pertoken MoE stack
+(B=16384 samples, T=48 tokens, D=768, H=48 heads, L=4 blocks with the inter-residual every 2,
+per token E=16 SwiGLU experts of hidden 512, top-4, alpha=4, a shared expert of hidden 768,
+~8e9 expert parameters resident): the largest workload that fits one GPU.  Each timed step is
+bracketed by CUDA events on the launching stream; a 256 MB write between steps flushes the
+126 MB L2 (the workload's inputs and weights are far larger than the L2 as well).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
-                  [--batch B] [--e2e-chunks C] [--fp8 | --backward]
+                  [--batch B] [--layers L] [--e2e-chunks C] [--fp8 | --backward]
 
-N > 1 (under torchrun): every rank runs its own batch (weak scaling, no data-path
-collective); the step time is the max over ranks.  --impl reference times the CPU
+Without --steps the step count is chosen from the warm-up steps' time so that the timed region
+lasts about two seconds.  N > 1 (under torchrun): every rank runs its own batch (weak scaling,
+no data-path collective); the step time is the max over ranks.  --impl reference times the CPU
 float64 oracle on the host cores (rank 0 only) on a bounded sample of the workload.  The
 end-to-end leg copies each step's batch from pinned host memory and the result back, in C
 sample chunks pipelined against the compute (the result is checked bit for bit against the
-full-batch device run).  --fp8 and --backward print their own lines (the FP8 serving path, the
-dense block backward).
+full-batch device run).  --batch and --layers run a smaller case of the same kernels (profiler
+captures).  --fp8 and --backward print their own lines (the FP8 serving path, the dense block
+backward) on a dense workload.
 """
 from __future__ import annotations
 
@@ -40,9 +44,9 @@ import tm_synth as S  # noqa: E402
 
 METRIC = "samples/sec & TFLOP/s of TokenMixer-Large fwd, % of B200 bf16 TC roofline"
 METRIC_BWD = "samples/sec & TFLOP/s of TokenMixer-Large dense block backward, % of B200 bf16 TC roofline"
-DEFAULT_WORKLOAD = "dense_block_bf16"
+DEFAULT_WORKLOAD = "large_moe_stack_bf16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["tm_gemm.cuh", "tm_fused.cuh", "tm_fused2.cuh", "tm_fused128.cuh", "tm_device.cuh", "tm_gemm.cu", "tm_kernels.cu", "tm_api.cu"]
+KERNEL_SOURCES = ["tm_gemm.cuh", "tm_fused.cuh", "tm_fused128.cuh", "tm_device.cuh", "tm_gemm.cu", "tm_kernels.cu", "tm_api.cu"]
 
 
 def describe(cfg) -> str:
@@ -146,6 +150,10 @@ def peaks():
 # uses); a DRAM figure in profiles/traffic.json counts only while these are unchanged.
 KERNEL_SOURCES_OF = {
     "fused_swiglu": ["tm_fused128.cuh", "tm_fused.cuh", "tm_device.cuh"],
+    "gemm_swiglu": ["tm_gemm.cuh", "tm_device.cuh"],
+    "gemm_slot": ["tm_gemm.cuh", "tm_device.cuh"],
+    "gemm_combine": ["tm_gemm.cuh", "tm_device.cuh"],
+    "router": ["tm_gemm.cuh", "tm_device.cuh"],
 }
 
 
@@ -224,26 +232,78 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle timing
+def oracle_param_bytes(cfg) -> float:
+    """float64 bytes of every weight of the workload (what the oracle would hold to run it whole)."""
+    n = 0
+    for sub in (0, 1):
+        s, W, banks = cfg.ffn(sub), cfg.width(sub), cfg.banks(sub)
+        per = 3 * W * s.hidden if not s.is_moe else s.E * (W + 3 * W * s.hidden_e) + 3 * W * s.hidden_s
+        n += banks * per
+    return 8.0 * cfg.L * n
+
+
+def oracle_probe(cfg, n: int, max_banks: int = 2):
+    """The oracle as it stands, on a bounded sample of the workload: a function that runs it once and
+    returns the host seconds that the whole stack would take on n samples, plus a description.
+
+    Workloads whose weights fit the host in float64 (up to 4 GB): stack_forward on samples
+    0..n-1, weights drawn beforehand.  Larger ones: the oracle's sub-layer (sublayer(): RMSNorm,
+    routing, experts) on samples 0..n-1 and the first nb banks of both sub-layers of block 1,
+    scaled by banks / nb and by the L blocks (every bank and block has the same shapes and the
+    routing is near uniform); the token rows stand in for the reverting sub-layer's input (the
+    same shape and distribution as X_revert)."""
+    import oracle
+    from oracle import tokenmixer as O
+    n = min(n, cfg.B)
+    X = S.to_f64(S.make_x(cfg, np.arange(n)))
+    if oracle_param_bytes(cfg) <= 4e9:
+        get = oracle.synth_banks(cfg)
+        for l in range(cfg.L):
+            for sub in (0, 1):
+                for j in range(cfg.banks(sub)):
+                    get(l, sub, j)
+
+        def step():
+            t0 = time.perf_counter()
+            oracle.stack_forward(X, cfg, get)
+            return time.perf_counter() - t0
+        return step, f"oracle stack_forward on samples 0..{n - 1} of {cfg.name}"
+    nb = min(max_banks, cfg.H, cfg.T)
+    get = oracle.synth_banks(cfg)
+    for sub in (0, 1):
+        for j in range(nb):
+            get(0, sub, j)
+    rows_mix = O.mix(X, cfg.H)[:, :nb]
+    rows_rev = X[:, :nb]
+
+    def step():
+        t0 = time.perf_counter()
+        O.sublayer(rows_mix, lambda j: get(0, 0, j), cfg.mix, cfg.eps)
+        t1 = time.perf_counter()
+        O.sublayer(rows_rev, lambda j: get(0, 1, j), cfg.rev, cfg.eps)
+        t2 = time.perf_counter()
+        return cfg.L * ((t1 - t0) * cfg.H / nb + (t2 - t1) * cfg.T / nb)
+    return step, (f"oracle sublayer() on samples 0..{n - 1} x banks 0..{nb - 1} of both sub-layers of block 1 "
+                  f"of {cfg.name}, scaled to all {cfg.H}+{cfg.T} banks and {cfg.L} blocks")
+
+
+def oracle_threads() -> int:
+    from threadpoolctl import threadpool_info
+    return int(max([i.get("num_threads", 1) for i in threadpool_info()] or [1]))
+
+
 def time_oracle(cfg, budget_s: float, max_samples: int):
     """Oracle samples/s on the host cores over a bounded sample (weights drawn beforehand)."""
-    import oracle
-    from threadpoolctl import threadpool_info
-    get = oracle.synth_banks(cfg)
-    for l in range(cfg.L):
-        for sub in (0, 1):
-            for j in range(cfg.banks(sub)):
-                get(l, sub, j)
+    step, desc = oracle_probe(cfg, max_samples)
     n = min(max_samples, cfg.B)
-    X = S.to_f64(S.make_x(cfg, np.arange(n)))
-    done, t0 = 0, time.perf_counter()
+    done, equiv, t0 = 0, 0.0, time.perf_counter()
     while True:
-        oracle.stack_forward(X, cfg, get)
+        equiv += step()
         done += n
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return done / dt, {"cores": int(threads), "samples": done, "seconds": dt, "per_call": n}
+    return done / equiv, {"cores": oracle_threads(), "samples": done, "seconds": dt, "per_call": n, "desc": desc}
 
 
 def time_oracle_fp8(cfg, budget_s: float, max_samples: int):
@@ -295,24 +355,12 @@ def time_oracle_backward(cfg, budget_s: float, max_samples: int):
 def run_reference(args, cfg, rank):
     if rank != 0:
         return
-    steps, warm = args.steps_ref, max(1, min(args.warmup, 1))
-    import oracle
-    get = oracle.synth_banks(cfg)
-    for l in range(cfg.L):
-        for sub in (0, 1):
-            for j in range(cfg.banks(sub)):
-                get(l, sub, j)
+    steps, warm = args.steps_ref, min(args.warmup, 3)
     n = min(args.ref_samples, cfg.B)
-    X = S.to_f64(S.make_x(cfg, np.arange(n)))
+    step, desc = oracle_probe(cfg, n)
     for _ in range(warm):
-        oracle.stack_forward(X, cfg, get)
-    t = []
-    for _ in range(steps):
-        t0 = time.perf_counter()
-        oracle.stack_forward(X, cfg, get)
-        t.append(time.perf_counter() - t0)
-    from threadpoolctl import threadpool_info
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        step()
+    t = [step() for _ in range(steps)]
     sec = sum(t)
     value = n * steps / sec
     line = {
@@ -320,10 +368,10 @@ def run_reference(args, cfg, rank):
         "steps": steps, "warmup": warm, "ms_per_step": 1e3 * sec / steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": describe(cfg), "global_batch": n, "parallelism": "host cores",
-                   "step": f"oracle stack forward on the first {n} samples of the batch"},
+                   "step": f"{desc}; ms_per_step is the whole stack's time on those {n} samples"},
         "tflops": flops_per_sample(cfg) * value / 1e12,
-        "cpu_baseline": {"value": value, "unit": "samples/s", "cores": int(threads), "kind": "oracle",
-                         "sample": f"{steps} steps x {n} samples of {cfg.name}"},
+        "cpu_baseline": {"value": value, "unit": "samples/s", "cores": oracle_threads(), "kind": "oracle",
+                         "sample": f"{steps} steps: {desc}"},
         "e2e": {"value": value, "unit": "samples/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -381,11 +429,18 @@ def run_ours(args, cfg, rank, world, local_rank):
     K, W = args.steps, args.warmup
 
     with torch.cuda.stream(stream):
+        t_warm = time.perf_counter()
         for _ in range(W):
             flush.zero_()
             run(X, Y, stream)
         stream.synchronize()
+        t_warm = (time.perf_counter() - t_warm) / max(W, 1)
         api.get_device_error(stream)
+        if K is None:
+            # about two seconds of timed steps (the same count on every rank)
+            K = int(min(5000, max(10, round(2.0 / max(t_warm, 1e-5)))))
+            if world > 1:
+                K = int(max_over_ranks(float(K), world, dev))
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
         if world > 1:
             dist.barrier()
@@ -462,22 +517,28 @@ def run_ours(args, cfg, rank, world, local_rank):
         avg_ms = dom[1]["total_ms"] / dom[1]["launches"]
         ach = per_launch / (avg_ms / 1e3) / 1e12
         tr = traffic_for(dom[0], cfg.name)
-        src = ("measured bf16 burst (MEASURED_PEAKS.json bf16_tflops)" if pk_src == "measured"
-               else "fallback 1.59 PFLOP/s")
-        peak = pk["bf16_tflops"]
+        # a step of 10 ms or more keeps the GPU at its power limit for the whole timed region: the
+        # sustained figure (a seconds-long cuBLAS loop); shorter steps: the burst figure
+        long_step = mean_ms >= 10.0
+        key = "bf16_tflops_sustained" if long_step else "bf16_tflops"
+        src = (f"measured bf16 {'sustained' if long_step else 'burst'} (MEASURED_PEAKS.json {key})"
+               if pk_src == "measured" else f"fallback {'1.40' if long_step else '1.59'} PFLOP/s")
+        peak = pk[key]
         if args.fp8:
             peak = fp8_effective_peak(pk["bf16_tflops"])
             src = ("GEMM1 at 2 x, GEMM2 at 1 x the " + src + ": 1.5 x the bf16 peak for the kernel's "
                    "2:1 split of flops")
         roof = {"kernel": dom[0], "bound": "tensor", "achieved": ach, "peak": peak,
                 "unit": "TFLOP/s", "frac": ach / peak, "traffic": tr, "peak_source": src,
+                "frac_of_burst": ach / (fp8_effective_peak(pk["bf16_tflops"]) if args.fp8 else pk["bf16_tflops"]),
                 "flops_per_launch": per_launch, "avg_launch_ms": avg_ms}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         timer = time_oracle_fp8 if args.fp8 else time_oracle_backward if args.backward else time_oracle
         v, info = timer(cfg, args.cpu_seconds, args.cpu_samples)
         cpu = {"value": v, "unit": "samples/s", "cores": info["cores"], "kind": "oracle",
-               "sample": f"{info['samples']} samples ({info['per_call']} per oracle call) of {cfg.name}, "
+               "sample": (f"{info['desc']}; " if "desc" in info else "") +
+                         f"{info['samples']} samples ({info['per_call']} per oracle call) of {cfg.name}, "
                          f"{info['seconds']:.1f} s of host time"}
     line = {
         "metric": METRIC_BWD if args.backward else METRIC, "value": value, "unit": "samples/s", "n_gpus": world, "steps": K, "warmup": W,
@@ -515,8 +576,9 @@ def run_ours(args, cfg, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: about two seconds' worth, from the warm-up steps' time)")
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(S.CONFIGS))
     ap.add_argument("--e2e-steps", type=int, default=200)
@@ -528,6 +590,8 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="run the workload with this many samples instead of its own B (small cases for "
                          "profiler captures; the line's workload string carries the B used)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="run the workload with this many blocks (small cases for profiler captures)")
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="end-to-end leg: split the batch into this many chunks whose host copies overlap "
                          "the compute (forward only)")
@@ -544,8 +608,14 @@ def main():
         if args.batch < 1:
             raise SystemExit("--batch must be positive")
         cfg = cfg.with_(B=args.batch)
+    if args.layers is not None:
+        if args.layers < 1:
+            raise SystemExit("--layers must be positive")
+        cfg = cfg.with_(L=args.layers)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":
-        args.steps_ref = args.steps_ref or min(args.steps, 20)
+        args.steps_ref = args.steps_ref or min(args.steps or 10, 10)
         run_reference(args, cfg, rank)
         return
     if world > 1:

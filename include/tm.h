@@ -158,6 +158,9 @@ TM_API tm_status tm_revert(const void *Hm, void *X, const tm_shape *shape, void 
  * descending order.  Outputs:
  *   topk_idx   [B, banks, k] int32  chosen experts
  *   topk_gate  [B, banks, k] fp32   alpha * p of each chosen expert (no renormalisation)
+ *   logit_gap_opt [B, banks] fp32   z_(k) - z_(k+1): the k-th largest logit minus the largest
+ *                                   logit left out (+inf when k == E), so a caller can tell the
+ *                                   rows whose choice is a near tie (may be NULL)
  *   inv_rms    [B, banks]    fp32   1/sqrt(mean(row^2) + eps)   (may be NULL)
  *   bucket_offsets [banks*E + 1] int32  start of group g = bank*E + e in bucket_rows
  *   bucket_rows    [B*banks*k]   int32  sample index b of every routed row, grouped by
@@ -165,8 +168,8 @@ TM_API tm_status tm_revert(const void *Hm, void *X, const tm_shape *shape, void 
  *   slot_of        [B, banks, k] int32  position in bucket_rows of (b, bank, j)
  * x and layout as in tm_layout. */
 TM_API tm_status tm_route_topk(const void *x, tm_layout layout, const tm_shape *shape, const void *norm_gain,
-                        const tm_moe_w *w, int32_t *topk_idx, float *topk_gate, float *inv_rms,
-                        int32_t *bucket_offsets, int32_t *bucket_rows, int32_t *slot_of,
+                        const tm_moe_w *w, int32_t *topk_idx, float *topk_gate, float *logit_gap_opt,
+                        float *inv_rms, int32_t *bucket_offsets, int32_t *bucket_rows, int32_t *slot_of,
                         void *workspace, size_t workspace_bytes, void *stream);
 
 /* Fixed size of the routing scratch array that tm_route_topk_noalloc keeps in the library. */
@@ -182,13 +185,15 @@ TM_API tm_status tm_route_topk(const void *x, tm_layout layout, const tm_shape *
  * tm_route_workspace_bytes exceeds it return TM_ERR_WORKSPACE (message in tm_last_cuda_error)
  * before any launch.  No device memory is allocated or freed.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress), so
- * make that first call before any stream capture.  All calls on a device share the array and it
+ * make that first call before any stream capture; the lookup is repeated when the device's
+ * context has changed (after a device reset).  All calls on a device share the array and it
  * keeps the last call's contents (none of it needs to start at zero): calls that can overlap on
  * the GPU (different streams without ordering) race on it and must not be issued. */
 TM_API tm_status tm_route_topk_noalloc(const void *x, tm_layout layout, const tm_shape *shape,
                                        const void *norm_gain, const tm_moe_w *w, int32_t *topk_idx,
-                                       float *topk_gate, float *inv_rms, int32_t *bucket_offsets,
-                                       int32_t *bucket_rows, int32_t *slot_of, void *stream);
+                                       float *topk_gate, float *logit_gap_opt, float *inv_rms,
+                                       int32_t *bucket_offsets, int32_t *bucket_rows, int32_t *slot_of,
+                                       void *stream);
 
 /* Dense per-token SwiGLU sub-layer with pre-RMSNorm and residual
  * ([readme] block diagram; [digest] 2.3.2-2.3.3):
@@ -211,6 +216,16 @@ TM_API tm_status tm_sparse_pertoken_moe(const void *x, const void *residual, tm_
  * X, Y [B,T,D]; X_revert_opt [B,T,D] receives X_rev when not NULL. */
 TM_API tm_status tm_block_forward(const void *X, const tm_block *block, const tm_shape *shape, void *Y,
                            void *X_revert_opt, void *workspace, size_t workspace_bytes, void *stream);
+
+/* One step of tm_stack_forward: Y = Block(X) + X_skip, where X_skip (NULL: none) is the skip term
+ * of the inter-residual ([digest] 2.3.4), added in the block's last epilogue before Y's single
+ * rounding to the storage dtype.  With X_skip NULL this is tm_block_forward.  tm_stack_forward is
+ * this call repeated (X_skip = X_{l-gap} where its rule applies), so a caller that runs a stack
+ * block by block -- to keep every X_l, or to interleave its own work -- gets the same bits.
+ * X, X_skip, Y, X_revert_opt [B,T,D]; X_skip must not alias Y or X_revert_opt.  Workspace: as
+ * tm_block_forward (tm_workspace_bytes with L = 1). */
+TM_API tm_status tm_stack_step(const void *X, const void *X_skip, const tm_block *block, const tm_shape *shape,
+                               void *Y, void *X_revert_opt, void *workspace, size_t workspace_bytes, void *stream);
 
 /* L blocks with the inter-residual of [digest] 2.3.4 ([readme]: "at gap 2, excluded
  * from the final layer"): X_l = Block_l(X_{l-1}); X_l += X_{l-gap} when gap > 0,
@@ -369,6 +384,37 @@ TM_API unsigned long long tm_launch_count(void);
 /* Synchronises `stream`, returns the first device-side error recorded since the
  * last call (TM_OK if none) and clears it. */
 TM_API tm_status tm_get_device_error(void *stream);
+
+/* Where the error that tm_get_device_error last returned was recorded (a site code of the
+ * kernel's wait or bounds check, also named in tm_last_cuda_error); 0 after TM_OK. */
+TM_API unsigned tm_last_device_error_site(void);
+
+/* Failure detection.  Every device wait of the library's kernels (a pipeline barrier, a tensor-memory
+ * handshake, the fused block's row-block counter) gives up after a wall-clock limit, records
+ * TM_ERR_DEVICE_TIMEOUT with its site and lets the kernel return; bounds checks on indices read from
+ * device data record TM_ERR_DEVICE_BOUNDS and skip the access.  No kernel traps.
+ *
+ * Sets that limit for the current device, in nanoseconds (1e3 .. 6e10; the default is 2 s, far
+ * above any legitimate wait).  Kernels already enqueued may run with either value.  The pages have
+ * no counterpart: this is a library facility, not part of the method. */
+TM_API tm_status tm_set_wait_limit_ns(uint64_t ns);
+
+/* Self-test of the bounded waits (one CTA, one thread): a wait on a barrier that nothing ever
+ * completes runs out after the limit above and records TM_ERR_DEVICE_TIMEOUT at site 0x7001; a
+ * second wait, made with the CTA's abort flag already raised, returns at once and records nothing.
+ * result_opt (device memory, 4 x uint64, may be NULL): the first wait's duration in ns, 1 (it
+ * failed), the second's duration in ns, 1 (it failed).  Read the outcome with tm_get_device_error. */
+TM_API tm_status tm_selftest_wait(uint64_t *result_opt, void *stream);
+
+/* The MoEPermute scatter of tm_route_topk run on caller-supplied tables, for tests of its bounds
+ * checks: topk_idx [B, banks, k]; chunk_prefix [banks][ceil(B/128)][E], the number of rows of each
+ * bank routed to each expert in the earlier 128-sample chunks; bucket_offsets [banks*E + 1];
+ * bucket_rows has `capacity` entries; slot_of [B, banks, k].  A position at or past `capacity`
+ * (a table that under-counts the choices) records TM_ERR_DEVICE_BOUNDS (site 0x501) and is not
+ * written; nothing outside the given arrays is read or written.  E <= 64, k <= 8. */
+TM_API tm_status tm_selftest_bucket_scatter(const int32_t *topk_idx, const int32_t *chunk_prefix,
+                                            const int32_t *bucket_offsets, int B, int banks, int E, int k,
+                                            int32_t *bucket_rows, int capacity, int32_t *slot_of, void *stream);
 
 #ifdef __cplusplus
 }

@@ -9,3 +9,13 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 and the built CUDA library")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+def pytest_terminal_summary(terminalreporter):
+    # near-tie counts and worst errors the parity tests recorded (tests/parity_util.py REPORT)
+    mod = sys.modules.get("parity_util")
+    lines = getattr(mod, "REPORT", None) if mod else None
+    if lines:
+        terminalreporter.write_sep("-", "parity report")
+        for line in lines:
+            terminalreporter.write_line(line)

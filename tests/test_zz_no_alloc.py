@@ -31,9 +31,13 @@ def _case(B, T, D, H, E, k, layout):
 
 @pytest.mark.gpu
 def test_noalloc_routing_matches_workspace_routing_on_two_calls():
-    cases = [_case(300, 16, 256, 16, 8, 2, A.TM_LAYOUT_MIXED),
-             _case(170, 8, 384, 4, 16, 4, A.TM_LAYOUT_ROWS)]
-    for (cfg, sw), layout in zip(cases, [A.TM_LAYOUT_MIXED, A.TM_LAYOUT_ROWS]):
+    # tensor-core router (E <= 21, bf16 rows through a tensor map) on two shapes in a row, then the
+    # CUDA-core router (E = 32), whose scratch holds only the counts and the tile prefix
+    layouts = [A.TM_LAYOUT_MIXED, A.TM_LAYOUT_ROWS, A.TM_LAYOUT_ROWS]
+    cases = [_case(300, 16, 256, 16, 8, 2, layouts[0]),
+             _case(170, 8, 384, 4, 16, 4, layouts[1]),
+             _case(210, 8, 256, 8, 32, 4, layouts[2])]
+    for (cfg, sw), layout in zip(cases, layouts):
         x = api.to_device(S.make_x(cfg), DEV)
         sh = api.config_shape(cfg)
         got = api.route_topk_noalloc(x, layout, sh, sw)
@@ -42,7 +46,7 @@ def test_noalloc_routing_matches_workspace_routing_on_two_calls():
         api.get_device_error()
         for key in ("idx", "offsets", "rows", "slot_of"):
             assert torch.equal(got[key], ref[key]), key
-        for key in ("gate", "inv_rms"):       # same kernels on the same input: the same bits
+        for key in ("gate", "gap", "inv_rms"):       # same kernels on the same input: the same bits
             assert torch.equal(got[key], ref[key]), key
 
 
@@ -58,7 +62,7 @@ def test_noalloc_routing_refuses_problems_beyond_its_scratch():
     w = A.tm_moe_w(H, T * D // H, E, 4, 64, 64, 4.0, fake["r"], fake["wg"], fake["wu"], fake["wd"], fake["sg"],
                    fake["su"], fake["sd"])
     st = api.lib().tm_route_topk_noalloc(fake["x"], A.TM_LAYOUT_MIXED, ctypes.byref(sh), None, ctypes.byref(w),
-                                         fake["idx"], fake["gate"], fake["inv"], fake["off"], fake["rows"],
+                                         fake["idx"], fake["gate"], None, fake["inv"], fake["off"], fake["rows"],
                                          fake["slot"], None)
     assert st == A.TM_ERR_WORKSPACE
     assert b"fixed limit" in api.lib().tm_last_cuda_error()

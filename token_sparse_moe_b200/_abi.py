@@ -15,14 +15,15 @@ TM_LAYOUT_ROWS, TM_LAYOUT_MIXED = 0, 1
 # Every entry point declared in include/tm.h (the CPU test checks the library exports each one).
 EXPORTS = ["tm_status_string", "tm_version", "tm_sublayer_workspace_bytes", "tm_route_workspace_bytes",
            "tm_workspace_bytes", "tm_tokenize_stub", "tm_mix", "tm_revert", "tm_route_topk", "tm_route_topk_noalloc",
-           "tm_pertoken_swiglu", "tm_sparse_pertoken_moe", "tm_block_forward", "tm_stack_forward",
+           "tm_pertoken_swiglu", "tm_sparse_pertoken_moe", "tm_block_forward", "tm_stack_step", "tm_stack_forward",
            "tm_profile_start", "tm_profile_stop", "tm_last_cuda_error", "tm_launch_count",
            "tm_get_device_error", "tm_quantize_fp8_weights", "tm_quantize_fp8_act",
            "tm_pertoken_swiglu_fp8_workspace_bytes", "tm_pertoken_swiglu_fp8", "tm_block_fp8_workspace_bytes",
            "tm_block_forward_fp8", "tm_head_forward", "tm_model_workspace_bytes", "tm_model_forward",
            "tm_pertoken_swiglu_backward_workspace_bytes", "tm_pertoken_swiglu_backward",
            "tm_block_backward_workspace_bytes", "tm_block_backward", "tm_stack_backward_workspace_bytes",
-           "tm_stack_backward"]
+           "tm_stack_backward", "tm_last_device_error_site", "tm_set_wait_limit_ns", "tm_selftest_wait",
+           "tm_selftest_bucket_scatter"]
 
 
 class tm_shape(ctypes.Structure):
@@ -80,19 +81,24 @@ _SIGS = {
     "tm_tokenize_stub": (c_int, [_P, _P, _P, c_int, POINTER(tm_shape), _P, _P]),
     "tm_mix": (c_int, [_P, _P, POINTER(tm_shape), _P]),
     "tm_revert": (c_int, [_P, _P, POINTER(tm_shape), _P]),
-    "tm_route_topk": (c_int, [_P, c_int, POINTER(tm_shape), _P, POINTER(tm_moe_w), _P, _P, _P, _P, _P, _P, _P,
+    "tm_route_topk": (c_int, [_P, c_int, POINTER(tm_shape), _P, POINTER(tm_moe_w), _P, _P, _P, _P, _P, _P, _P, _P,
                               c_size_t, _P]),
     "tm_route_topk_noalloc": (c_int, [_P, c_int, POINTER(tm_shape), _P, POINTER(tm_moe_w), _P, _P, _P, _P, _P, _P,
-                                      _P]),
+                                      _P, _P]),
     "tm_pertoken_swiglu": (c_int, [_P, _P, c_int, POINTER(tm_shape), _P, POINTER(tm_swiglu_w), _P, _P, c_size_t, _P]),
     "tm_sparse_pertoken_moe": (c_int, [_P, _P, c_int, POINTER(tm_shape), _P, POINTER(tm_moe_w), _P, _P, c_size_t, _P]),
     "tm_block_forward": (c_int, [_P, POINTER(tm_block), POINTER(tm_shape), _P, _P, _P, c_size_t, _P]),
+    "tm_stack_step": (c_int, [_P, _P, POINTER(tm_block), POINTER(tm_shape), _P, _P, _P, c_size_t, _P]),
     "tm_stack_forward": (c_int, [_P, POINTER(tm_block), c_int, c_int, POINTER(tm_shape), _P, _P, c_size_t, _P]),
     "tm_profile_start": (c_int, []),
     "tm_profile_stop": (c_int, [POINTER(tm_kernel_time), c_int, POINTER(c_int)]),
     "tm_last_cuda_error": (ctypes.c_char_p, []),
     "tm_launch_count": (ctypes.c_ulonglong, []),
     "tm_get_device_error": (c_int, [_P]),
+    "tm_last_device_error_site": (ctypes.c_uint, []),
+    "tm_set_wait_limit_ns": (c_int, [ctypes.c_uint64]),
+    "tm_selftest_wait": (c_int, [_P, _P]),
+    "tm_selftest_bucket_scatter": (c_int, [_P, _P, _P, c_int, c_int, c_int, c_int, _P, c_int, _P, _P]),
     "tm_quantize_fp8_weights": (c_int, [_P, _P, c_int, c_size_t, c_int, _P, _P, _P]),
     "tm_quantize_fp8_act": (c_int, [_P, c_int, POINTER(tm_shape), c_int, c_int, _P, _P, _P]),
     "tm_pertoken_swiglu_fp8_workspace_bytes": (c_size_t, [POINTER(tm_shape), c_int, POINTER(tm_swiglu_w8)]),

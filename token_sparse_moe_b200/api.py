@@ -155,6 +155,7 @@ def route_topk(x: torch.Tensor, layout: int, sh: A.tm_shape, sub: SubLayer, work
     out = {
         "idx": torch.empty((B, banks, k), dtype=torch.int32, device=dev),
         "gate": torch.empty((B, banks, k), dtype=torch.float32, device=dev),
+        "gap": torch.empty((B, banks), dtype=torch.float32, device=dev),
         "inv_rms": torch.empty((B, banks), dtype=torch.float32, device=dev),
         "offsets": torch.empty(banks * E + 1, dtype=torch.int32, device=dev),
         "rows": torch.empty(B * banks * k, dtype=torch.int32, device=dev),
@@ -165,8 +166,8 @@ def route_topk(x: torch.Tensor, layout: int, sh: A.tm_shape, sub: SubLayer, work
         raise A.TMError(A.TM_ERR_INVALID_ARG, "tm_route_workspace_bytes")
     ws = _ws(nb, dev, workspace)
     A.check(lib().tm_route_topk(_p(x), layout, ctypes.byref(sh), _p(sub.gain), ctypes.byref(w), _p(out["idx"]),
-                                _p(out["gate"]), _p(out["inv_rms"]), _p(out["offsets"]), _p(out["rows"]),
-                                _p(out["slot_of"]), _p(ws), ws.numel(), _s(stream)), "tm_route_topk")
+                                _p(out["gate"]), _p(out["gap"]), _p(out["inv_rms"]), _p(out["offsets"]),
+                                _p(out["rows"]), _p(out["slot_of"]), _p(ws), ws.numel(), _s(stream)), "tm_route_topk")
     return out
 
 
@@ -182,14 +183,16 @@ def route_topk_noalloc(x: torch.Tensor, layout: int, sh: A.tm_shape, sub: SubLay
         out = {
             "idx": torch.empty((B, banks, k), dtype=torch.int32, device=dev),
             "gate": torch.empty((B, banks, k), dtype=torch.float32, device=dev),
+            "gap": torch.empty((B, banks), dtype=torch.float32, device=dev),
             "inv_rms": torch.empty((B, banks), dtype=torch.float32, device=dev),
             "offsets": torch.empty(banks * E + 1, dtype=torch.int32, device=dev),
             "rows": torch.empty(B * banks * k, dtype=torch.int32, device=dev),
             "slot_of": torch.empty((B, banks, k), dtype=torch.int32, device=dev),
         }
     A.check(lib().tm_route_topk_noalloc(_p(x), layout, ctypes.byref(sh), _p(sub.gain), ctypes.byref(w),
-                                        _p(out["idx"]), _p(out["gate"]), _p(out["inv_rms"]), _p(out["offsets"]),
-                                        _p(out["rows"]), _p(out["slot_of"]), _s(stream)), "tm_route_topk_noalloc")
+                                        _p(out["idx"]), _p(out["gate"]), _p(out.get("gap")), _p(out["inv_rms"]),
+                                        _p(out["offsets"]), _p(out["rows"]), _p(out["slot_of"]), _s(stream)),
+            "tm_route_topk_noalloc")
     return out
 
 
@@ -240,6 +243,16 @@ def block_forward(X, block: Block, sh: A.tm_shape, Y=None, X_revert=None, worksp
     ws = _ws(workspace_bytes(sh, [block]), X.device, workspace)
     A.check(lib().tm_block_forward(_p(X), ctypes.byref(c), ctypes.byref(sh), _p(Y), _p(X_revert), _p(ws), ws.numel(),
                                    _s(stream)), "tm_block_forward")
+    return Y
+
+
+def stack_step(X, X_skip, block: Block, sh: A.tm_shape, Y=None, X_revert=None, workspace=None, stream=None):
+    """tm_stack_step: Y = Block(X) + X_skip (X_skip None: none), one step of the stack forward."""
+    Y = torch.empty_like(X) if Y is None else Y
+    c = block.c()
+    ws = _ws(workspace_bytes(sh, [block]), X.device, workspace)
+    A.check(lib().tm_stack_step(_p(X), _p(X_skip), ctypes.byref(c), ctypes.byref(sh), _p(Y), _p(X_revert), _p(ws),
+                                ws.numel(), _s(stream)), "tm_stack_step")
     return Y
 
 

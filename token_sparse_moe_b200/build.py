@@ -9,7 +9,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libtm.so")
-SOURCES = ["tm_lib.cu", "tm_kernels.cu", "tm_backward.cu", "tm_gemm.cu", "tm_api.cu", "tm_profile.cu", "tm_noalloc.cu", "tm_gemm.cuh", "tm_fused.cuh", "tm_fused2.cuh", "tm_fused128.cuh", "tm_device.cuh", "tm_internal.h"]
+SOURCES = ["tm_lib.cu", "tm_kernels.cu", "tm_backward.cu", "tm_gemm.cu", "tm_api.cu", "tm_profile.cu", "tm_noalloc.cu", "tm_gemm.cuh", "tm_fused.cuh", "tm_fused128.cuh", "tm_device.cuh", "tm_internal.h"]
 
 
 def nvcc() -> str:

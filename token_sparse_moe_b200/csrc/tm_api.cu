@@ -284,24 +284,18 @@ tm_status gemm2_dense(const Geo& g, const void* hidden, const void* wd, int F, i
 }
 
 // ------------------------------------------------------------------ fused dense sub-layer
-// One launch for row widths 128 / 256: statistics, GEMM1, SwiGLU, GEMM2, residual.
+// One launch for row widths 128 / 256: statistics, GEMM1, SwiGLU, GEMM2, residual.  Hidden widths
+// that are multiples of 128 take the 128-wide-chunk kernel (tm_fused128.cuh), the others (F % 128
+// == 64) the 64-wide-chunk kernel (tm_fused.cuh).
 tm_status fused_dense(const Geo& g, const void* x, const void* wg, const void* wu, const void* wd, int F,
-                      const void* resid, const void* extra, void* y, void* scratch, size_t scratch_bytes,
-                      cudaStream_t st) {
+                      const void* resid, const void* extra, void* y, cudaStream_t st) {
     const int am = gemm1_amode(g);
-    // One CTA per 128-row tile by default.  TM_FUSED_PAIRS=1 selects the CTA-pair kernel (2-SM
-    // MMAs, half the weight bytes per SM); on B200 it measured slower on the dense block workload
-    // (0.189 ms against 0.149 ms per sub-layer): its per-chunk handoffs cross the CTA pair.
-    // TM_FUSED64=1 keeps 64-wide hidden chunks where F % 128 == 0 (for comparison only).
-    const char* env = getenv("TM_FUSED_PAIRS");
-    const bool pairs = g.B > 128 && env && env[0] == '1';
-    const char* env64 = getenv("TM_FUSED64");
-    const bool wide = !pairs && F % 128 == 0 && !(env64 && env64[0] == '1') && (uintptr_t)y % 32 == 0;
+    const bool wide = F % 128 == 0 && (uintptr_t)y % 32 == 0;
     const uint32_t gu_box = wide ? 128 : 64;
     CUtensorMap ma, mg, mu, md;
     if (!gemm1_amap(g, x, am, &ma)) return TM_ERR_CUDA;
     if (!map_2d(&mg, wg, (uint64_t)g.banks * F, g.W, gu_box) || !map_2d(&mu, wu, (uint64_t)g.banks * F, g.W, gu_box) ||
-        !map_2d(&md, wd, (uint64_t)g.banks * g.W, F, pairs ? g.W / 2 : g.W))
+        !map_2d(&md, wd, (uint64_t)g.banks * g.W, F, g.W))
         return TM_ERR_CUDA;
     FusedParams p;
     memset(&p, 0, sizeof(p));
@@ -315,13 +309,7 @@ tm_status fused_dense(const Geo& g, const void* x, const void* wg, const void* w
     p.extra = (const __nv_bfloat16*)extra;
     p.omap = g.map;
     p.out_elems = (size_t)g.B * g.banks * g.W;
-    const long mt = (g.B + 127) / 128;
-    if (pairs) {
-        const long pair_tiles = (long)g.banks * ((mt + 1) / 2);
-        const long clusters = pair_tiles < num_sms() / 2 ? pair_tiles : num_sms() / 2;
-        return cuda_status(launch_fused2(g.W, am, ma, mg, mu, md, p, (int)(2 * clusters), st));
-    }
-    const long tiles = (long)g.banks * mt;
+    const long tiles = (long)g.banks * ((g.B + 127) / 128);
     const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
     if (wide) {
         // residual: the A tile itself when it is the sub-layer input (same tensor, same row map),
@@ -336,24 +324,6 @@ tm_status fused_dense(const Geo& g, const void* x, const void* wg, const void* w
         // output: the same row geometry, 32-row boxes (one per epilogue warp)
         CUtensorMap mo;
         if (!gemm1_amap(g, y, am, &mo, 32)) return TM_ERR_CUDA;
-        // Opt-in (TM_FUSED_SPLIT=1): when the last partial wave holds at most half a wave of tiles,
-        // split each of them between two CTAs by hidden chunks (fp32 partials in the scratch space,
-        // which the fused path does not otherwise use; counters zeroed here).  On the dense block
-        // workload it shortens the slowest CTA by ~6% but measured 1.5% slower per launch with the
-        // L2 flushed between steps (the 17 MB of partials push a working set that nearly fills the
-        // L2 over it) plus a memset per launch, so it is off by default.
-        const long n_rem = tiles % grid;
-        const size_t part_bytes = (size_t)2 * n_rem * 128 * g.W * sizeof(float);
-        const size_t cnt_off = (part_bytes + 255) & ~(size_t)255;
-        const char* env_split = getenv("TM_FUSED_SPLIT");
-        if (n_rem > 0 && 2 * n_rem <= grid && F / 128 >= 2 && scratch && cnt_off + n_rem * 8 * sizeof(int) <= scratch_bytes &&
-            env_split && env_split[0] == '1') {
-            p.split_tiles = 1;
-            p.part = (float*)scratch;
-            p.cnt = (int*)((uint8_t*)scratch + cnt_off);
-            tm_status s = cuda_status(cudaMemsetAsync(p.cnt, 0, n_rem * 8 * sizeof(int), st));
-            if (s != TM_OK) return s;
-        }
         return cuda_status(launch_fused128(g.W, am, false, ma, mg, mu, md, mr, me, mo, p, grid, st));
     }
     return cuda_status(launch_fused(g.W, am, ma, mg, mu, md, p, grid, st));
@@ -394,8 +364,7 @@ tm_status run_dense(const Geo& g, const void* x, const void* resid, const void* 
         wu = d.wu;
     }
     if (g.dtype == TM_BF16 && fused_supported(g.W, gemm1_amode(g)) && w->hidden % 64 == 0)
-        return fused_dense(g, x, wg, wu, w->w_down, w->hidden, resid, extra, y, d.hidden,
-                           (size_t)g.banks * g.B * w->hidden * g.esz, st);
+        return fused_dense(g, x, wg, wu, w->w_down, w->hidden, resid, extra, y, st);
     if ((s = cuda_status(launch_rms(g.dtype, x, g.map, g.B, g.eps, d.inv_rms, st))) != TM_OK) return s;
     if ((s = gemm1_dense(g, x, wg, wu, w->hidden, d.inv_rms, d.hidden, st)) != TM_OK) return s;
     // bf16 with a tensor-map row geometry: GEMM2 with the residual and inter-residual entering the
@@ -454,6 +423,7 @@ struct RouteOut {
     int4* tile_info = nullptr; // optional: per 128-row tile descriptors of the buckets
     float* inv_pos = nullptr;  // optional: 1/rms of each bucket position's row
     float* gate_pos = nullptr; // optional: gate of each bucket position's choice
+    float* gap = nullptr;      // optional: logit gap z_(k) - z_(k+1) of each row [B * banks]
 };
 
 
@@ -461,8 +431,7 @@ tm_status run_route(const Geo& g, const void* x, const void* gain, const tm_moe_
                     cudaStream_t st) {
     tm_status s;
     const int nchunks = (g.B + kRouterChunk - 1) / kRouterChunk;
-    const char* env_r = getenv("TM_ROUTER_SIMT");
-    if (r.wsplit && route_split_bytes(g, w) > 0 && !(env_r && env_r[0] == '1')) {
+    if (r.wsplit && route_split_bytes(g, w) > 0) {
         // router on the tensor core: split weights, then one grouped-GEMM launch (N = 64) whose
         // epilogue writes top-k, gates, 1/rms and the per-chunk expert counts (zeroed first)
         const int am = gemm1_amode(g);
@@ -481,6 +450,7 @@ tm_status run_route(const Geo& g, const void* x, const void* gain, const tm_moe_
         p.r_idx = r.idx;
         p.r_gate = r.gate;
         p.r_inv_rms = r.inv_rms;
+        p.r_gap = r.gap;
         p.r_counts = r.counts;
         p.r_nchunks = nchunks;
         p.r_alpha = w->alpha;
@@ -489,7 +459,7 @@ tm_status run_route(const Geo& g, const void* x, const void* gain, const tm_moe_
         if (!gemm1_amap(g, x, am, &ma) || !map_2d(&mb, r.wsplit, (uint64_t)g.banks * 64, g.W, 64)) return TM_ERR_CUDA;
         if ((s = cuda_status(launch_grouped_gemm(64, am, EPI_ROUTE, ma, mb, mb, p, dense_grid(p), st))) != TM_OK) return s;
     } else if ((s = cuda_status(launch_router(g.dtype, x, g.map, g.B, g.eps, gain, w->w_router, w->E, w->k, w->alpha,
-                                              r.idx, r.gate, r.inv_rms, r.counts, st))) != TM_OK) {
+                                              r.idx, r.gate, r.inv_rms, r.gap, r.counts, st))) != TM_OK) {
         return s;
     }
     if ((s = cuda_status(launch_offsets(r.counts, r.counts, g.banks, nchunks, w->E, r.offsets, r.tile_start, st,
@@ -594,25 +564,18 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
     } else {
         // MoEPermute: copy the routed rows into bucket order (the slot buffer, [routed, W], is free
         // until the routed GEMM2 writes it), then GEMM1 reads A as contiguous rows through a 2-D
-        // tensor map.  TM_MOE_GATHER=1 keeps the row gather inside GEMM1 (cp.async; comparison).
-        const char* env_g = getenv("TM_MOE_GATHER");
-        const bool gather_in_gemm = env_g && env_g[0] == '1';
+        // tensor map.
         const int bn = pick_bn_swiglu(Fe);
         p.n_tiles = p.N / bn;
         CUtensorMap ma, mg, mu, mo;
-        memset(&ma, 0, sizeof(ma));
         if (!map_2d(&mg, weg, G * Fe, g.W, bn / 2) || !map_2d(&mu, weu, G * Fe, g.W, bn / 2) ||
             !map_2d(&mo, m.hidden_r, routed, Fe, 32))
             return TM_ERR_CUDA;
-        if (!gather_in_gemm) {
-            if ((s = cuda_status(launch_scatter_rows(g.dtype, x, g.map, g.B, w->k, m.slot_of, routed, m.slots, st))) !=
-                TM_OK)
-                return s;
-            if (!map_2d(&ma, m.slots, routed, g.W, 128)) return TM_ERR_CUDA;
-        }
+        if ((s = cuda_status(launch_scatter_rows(g.dtype, x, g.map, g.B, w->k, m.slot_of, routed, m.slots, st))) != TM_OK)
+            return s;
+        if (!map_2d(&ma, m.slots, routed, g.W, 128)) return TM_ERR_CUDA;
         const long grid = max_mt * p.n_tiles < num_sms() ? max_mt * p.n_tiles : num_sms();
-        if ((s = cuda_status(launch_grouped_gemm(bn, gather_in_gemm ? A_GATHER : A_TMA_2D, EPI_SWIGLU, ma, mg, mu, p,
-                                                 (int)grid, st, &mo))) != TM_OK)
+        if ((s = cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SWIGLU, ma, mg, mu, p, (int)grid, st, &mo))) != TM_OK)
             return s;
     }
     // shared expert GEMM1 (dense rows)
@@ -809,8 +772,8 @@ tm_status check_block(const tm_shape* s, const tm_block* b, Geo* gm, Geo* gr) {
 // ------------------------------------------------------------------ fused dense block
 // Both sub-layers of a block in one launch (launch_fused128_block): dense bf16 sub-layers of the
 // same row width 128 or 256 (T == H), head width a multiple of 16, hidden widths multiples of 128.
-// TM_FUSED_BLOCK=0 keeps one launch per sub-layer (for comparison), as do the opt-in variants of
-// the sub-layer kernel.
+// TM_FUSED_BLOCK=0 in the environment keeps one launch per sub-layer: the tests use it to show
+// that the one-launch block gives the same bits as the per-sub-layer launches.
 bool env_is(const char* name, char v) {
     const char* e = getenv(name);
     return e && e[0] == v;
@@ -822,9 +785,7 @@ bool block_fusable(const tm_shape* s, const tm_block* b, const Geo& gm, const Ge
     if (gemm1_amode(gm) != A_TMA_MIX) return false;
     if (b->mix.dense.hidden % 128 || b->rev.dense.hidden % 128) return false;
     if ((uintptr_t)Y % 32 || (uintptr_t)Xr % 32) return false;
-    if (env_is("TM_FUSED_BLOCK", '0') || env_is("TM_FUSED_PAIRS", '1') || env_is("TM_FUSED64", '1') ||
-        env_is("TM_FUSED_SPLIT", '1'))
-        return false;
+    if (env_is("TM_FUSED_BLOCK", '0')) return false;
     return true;
 }
 
@@ -1200,7 +1161,7 @@ tm_status tm_revert(const void* Hm, void* X, const tm_shape* shape, void* stream
 }
 
 tm_status tm_route_topk(const void* x, tm_layout layout, const tm_shape* shape, const void* norm_gain,
-                        const tm_moe_w* w, int32_t* topk_idx, float* topk_gate, float* inv_rms,
+                        const tm_moe_w* w, int32_t* topk_idx, float* topk_gate, float* logit_gap_opt, float* inv_rms,
                         int32_t* bucket_offsets, int32_t* bucket_rows, int32_t* slot_of, void* workspace,
                         size_t workspace_bytes, void* stream) {
     Geo g;
@@ -1211,6 +1172,9 @@ tm_status tm_route_topk(const void* x, tm_layout layout, const tm_shape* shape, 
     if (!x || !al16(x) || !topk_idx || !topk_gate || !bucket_offsets || !bucket_rows || !slot_of)
         return TM_ERR_INVALID_ARG;
     if (norm_gain && !al16(norm_gain)) return TM_ERR_INVALID_ARG;
+    if ((logit_gap_opt && (reinterpret_cast<uintptr_t>(logit_gap_opt) & 3)) ||
+        (inv_rms && (reinterpret_cast<uintptr_t>(inv_rms) & 3)))
+        return TM_ERR_INVALID_ARG;
     const size_t need = tm_route_workspace_bytes(shape, layout, w);
     if (!workspace || workspace_bytes < need || !al16(workspace)) return TM_ERR_WORKSPACE;
     Carve c{(uint8_t*)workspace};
@@ -1218,6 +1182,7 @@ tm_status tm_route_topk(const void* x, tm_layout layout, const tm_shape* shape, 
     int32_t* counts = c.take<int32_t>((size_t)g.banks * nchunks * w->E);
     int32_t* tiles = c.take<int32_t>((size_t)g.banks * w->E + 1);
     RouteOut r{topk_idx, bucket_offsets, tiles, bucket_rows, slot_of, counts, topk_gate, inv_rms};
+    r.gap = logit_gap_opt;
     const size_t split = route_split_bytes(g, w);
     r.wsplit = split ? c.take<uint8_t>(split) : nullptr;
     return run_route(g, x, norm_gain, w, r, (cudaStream_t)stream);
@@ -1272,6 +1237,27 @@ tm_status tm_block_forward(const void* X, const tm_block* block, const tm_shape*
     if (X_revert_opt) xr = X_revert_opt;
     c.off = align256(c.off);
     return run_block(shape, block, X, nullptr, Y, xr, (uint8_t*)workspace + c.off, workspace_bytes - c.off,
+                     (cudaStream_t)stream);
+}
+
+tm_status tm_stack_step(const void* X, const void* X_skip, const tm_block* block, const tm_shape* shape, void* Y,
+                        void* X_revert_opt, void* workspace, size_t workspace_bytes, void* stream) {
+    bool ok = false;
+    const size_t need = block ? stack_ws(shape, block, 1, 0, &ok) : 0;
+    if (!ok) {
+        Geo a, b;
+        tm_status s = check_block(shape, block, &a, &b);
+        return s == TM_OK ? TM_ERR_INVALID_ARG : s;
+    }
+    if (!X || !Y || X == Y || !al16(X) || !al16(Y) || (X_revert_opt && !al16(X_revert_opt))) return TM_ERR_INVALID_ARG;
+    if (X_skip && (!al16(X_skip) || X_skip == Y || X_skip == X_revert_opt)) return TM_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < need || !al16(workspace)) return TM_ERR_WORKSPACE;
+    Carve c{(uint8_t*)workspace};
+    const size_t tok = (size_t)shape->B * shape->T * shape->D * (shape->dtype == TM_BF16 ? 2 : 4);
+    void* xr = c.take<uint8_t>(tok);
+    if (X_revert_opt) xr = X_revert_opt;
+    c.off = align256(c.off);
+    return run_block(shape, block, X, X_skip, Y, xr, (uint8_t*)workspace + c.off, workspace_bytes - c.off,
                      (cudaStream_t)stream);
 }
 
@@ -1483,12 +1469,17 @@ tm_status tm_stack_backward(const void* X, const void* dY, const tm_block* block
     return TM_OK;
 }
 
+static unsigned g_last_site = 0;   // site of the last device error tm_get_device_error returned
+
+unsigned tm_last_device_error_site(void) { return g_last_site; }
+
 tm_status tm_get_device_error(void* stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) { note_cuda_error("tm_get_device_error: stream synchronize", e); return TM_ERR_CUDA; }
     unsigned int h[2] = {0, 0};
     e = cudaMemcpyFromSymbol(h, g_error, sizeof(h));
     if (e != cudaSuccess) { note_cuda_error("tm_get_device_error: read error word", e); return TM_ERR_CUDA; }
+    g_last_site = h[0] ? h[1] : 0u;
     if (h[0] == 0) return TM_OK;
     char where[64];
     snprintf(where, sizeof(where), "device error %u at site 0x%x", h[0], h[1]);
@@ -1497,6 +1488,29 @@ tm_status tm_get_device_error(void* stream) {
     e = cudaMemcpyToSymbol(g_error, z, sizeof(z));
     if (e != cudaSuccess) { note_cuda_error("tm_get_device_error: clear error word", e); return TM_ERR_CUDA; }
     return h[0] == ERR_TIMEOUT ? TM_ERR_DEVICE_TIMEOUT : TM_ERR_DEVICE_BOUNDS;
+}
+
+tm_status tm_set_wait_limit_ns(uint64_t ns) {
+    if (ns < 1000ull || ns > 60000000000ull) return TM_ERR_INVALID_ARG;
+    const unsigned long long v = ns;
+    cudaError_t e = cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v));
+    if (e != cudaSuccess) { note_cuda_error("tm_set_wait_limit_ns", e); return TM_ERR_CUDA; }
+    return TM_OK;
+}
+
+tm_status tm_selftest_wait(uint64_t* result_opt, void* stream) {
+    if (result_opt && (reinterpret_cast<uintptr_t>(result_opt) & 7)) return TM_ERR_INVALID_ARG;
+    return cuda_status(launch_wait_selftest(reinterpret_cast<unsigned long long*>(result_opt), (cudaStream_t)stream));
+}
+
+tm_status tm_selftest_bucket_scatter(const int32_t* topk_idx, const int32_t* chunk_prefix, const int32_t* bucket_offsets,
+                                     int B, int banks, int E, int k, int32_t* bucket_rows, int capacity,
+                                     int32_t* slot_of, void* stream) {
+    if (!topk_idx || !chunk_prefix || !bucket_offsets || !bucket_rows || !slot_of) return TM_ERR_INVALID_ARG;
+    if (B <= 0 || banks <= 0 || E < 1 || k < 1 || k > E || capacity < 0) return TM_ERR_INVALID_ARG;
+    if (E > 64 || k > 8) return TM_ERR_UNSUPPORTED;
+    return cuda_status(launch_scatter(topk_idx, chunk_prefix, bucket_offsets, B, banks, E, k, bucket_rows, slot_of,
+                                      (cudaStream_t)stream, nullptr, nullptr, nullptr, nullptr, nullptr, capacity));
 }
 
 }  // extern "C"

@@ -29,7 +29,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: far above any legitimate wait
+// Limit of every bounded wait in nanoseconds: 2 s by default, far above any legitimate wait;
+// settable at run time per device (tm_set_wait_limit_ns).
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
+
+__device__ __forceinline__ uint64_t wait_limit_ns() {
+    return *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -75,10 +81,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned where) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = globaltimer_ns(), lim = wait_limit_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > lim) {
             record_error(ERR_TIMEOUT, where);
             return false;
         }

@@ -30,9 +30,6 @@ struct FusedParams {
     size_t out_elems;
     int res_mode;              // 128-wide-chunk kernel: residual none / from the A tile / streamed (FusedResid)
     int has_extra;             // 128-wide-chunk kernel: inter-residual streamed
-    int split_tiles;           // 128-wide-chunk kernel: split the last wave's tiles between CTA pairs
-    float* part;               // split tiles: partial Y, [2][tiles of the last wave][128][W] fp32
-    int* cnt;                  // split tiles: [tiles of the last wave][8] counters, zero at launch
     // Whole dense block in one launch (128-wide-chunk kernel, block mode): the fields above describe
     // the mixing sub-layer, these the reverting one (same banks and row width).
     int F2;                    // reverting hidden width

@@ -75,27 +75,12 @@ struct Fused128Cfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// 16 consecutive bf16 (32 bytes, one sector) from 8 packed words; p must be 32-byte aligned.
-__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
-    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
-                 "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
-                 : "memory");
-}
 
-// 8 consecutive 32-bit words (32 bytes) from global memory, cached in L2 only (data written by
-// another CTA of the same launch); p must be 32-byte aligned.
-__device__ __forceinline__ void ld_global_cg_v8(const void* p, uint32_t (&w)[8]) {
-    asm volatile("ld.global.cg.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
-                 : "l"(p)
-                 : "memory");
-}
-
-// One work item of a CTA: tile t (bank g, row tile m), hidden chunks [c0, c1), split half sp
-// (-1: whole tile); sec: a tile of the second (reverting) sub-layer in block mode; mx: A, the
-// residual stream and the output use the Mix geometry.
+// One work item of a CTA: tile t (bank g, row tile m), hidden chunks [c0, c1); sec: a tile of the
+// second (reverting) sub-layer in block mode; mx: A, the residual stream and the output use the
+// Mix geometry.
 struct F128Item {
-    int t, g, m, c0, c1, sp;
+    int t, g, m, c0, c1;
     bool sec, mx;
 };
 
@@ -123,16 +108,13 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
     // overlaps GEMM1(c+1) and its hidden write waits only for GEMM2(c-1).  (A lag of 2 measured
     // 16% slower on the dense block workload: each hidden write then waits behind a whole GEMM1.)
     constexpr int LAG = 1;
-    // Work items of this CTA: tile t = blockIdx.x + k * gridDim.x for the full waves.  With
-    // p.split_tiles the tiles of the last, partial wave are each split between two CTAs by hidden
-    // chunks (half 0: [0, NC/2), half 1: [NC/2, NC)), so every CTA ends within half a tile of the
-    // others; the halves meet through p.part (see the split output below).  Block mode: tiles
-    // [0, ntile1) mixing, [ntile1, 2 ntile1) reverting, each numbered m * banks + g; no splits.
+    // Work items of this CTA: tile t = blockIdx.x + k * gridDim.x, all hidden chunks of the tile.
+    // Block mode: tiles [0, ntile1) mixing, [ntile1, 2 ntile1) reverting, each numbered
+    // m * banks + g.
     const int full_waves = ntile / (int)gridDim.x;
     const int n_rem = ntile - full_waves * (int)gridDim.x;
     auto item = [&](int k, F128Item& it) -> bool {
         const int b = blockIdx.x;
-        it.sp = -1;
         it.c0 = 0;
         if (BLK) {
             it.t = b + k * (int)gridDim.x;
@@ -152,12 +134,6 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
             it.t = b + k * (int)gridDim.x;
         } else if (k > full_waves) {
             return false;
-        } else if (p.split_tiles) {
-            if (b >= 2 * n_rem) return false;
-            it.t = full_waves * (int)gridDim.x + (b >> 1);
-            it.sp = b & 1;
-            it.c0 = it.sp ? NC / 2 : 0;
-            it.c1 = it.sp ? NC : NC / 2;
         } else {
             if (b >= n_rem) return false;
             it.t = full_waves * (int)gridDim.x + b;
@@ -285,10 +261,10 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
                 const unsigned* ctr = p.dep + m;
                 const unsigned target = 8u * (unsigned)p.banks;
                 if (ld_acquire(ctr) < target) {
-                    const uint64_t t0 = globaltimer_ns();
+                    const uint64_t t0 = globaltimer_ns(), lim = wait_limit_ns();
                     while (ld_acquire(ctr) < target) {
                         if (*abort_flag) return false;
-                        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                        if (globaltimer_ns() - t0 > lim) {
                             record_error(ERR_TIMEOUT, 0x3108);
                             *abort_flag = 1;
                             return false;
@@ -711,93 +687,6 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
             if (BLK && !sec) pend_m = m;                              // counted once the stores complete
             return true;
         };
-        // One half of a split tile: this half's partial Y (fp32, rows of W) goes to p.part; for each
-        // warp's slice an atomic counter names the half that finishes second, which adds the other
-        // half's partial and writes the output.  fp32 a + b is commutative, so the result does not
-        // depend on which half that is; no CTA waits for another.
-        auto output_split = [&](int g, int m, int ylt, int sp, int st) -> bool {
-            if (!wait_or_abort(y_full, ylt & 1, abort_flag, 0x3303)) return false;
-            tc_fence_after();
-            const size_t row = (size_t)(q * 32 + lane);
-            float* mine = p.part + (((size_t)sp * n_rem + st) * 128 + row) * W + half * (W / 2);
-            const float* other = p.part + (((size_t)(1 - sp) * n_rem + st) * 128 + row) * W + half * (W / 2);
-#pragma unroll 1
-            for (int j = 0; j < W / 64; ++j) {
-                uint32_t v[32];
-                tmem_ld32_async(trow + half * (W / 2) + j * 32, v);
-                tmem_wait_ld_tie(v);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const uint32_t w8[8] = {v[e * 8 + 0], v[e * 8 + 1], v[e * 8 + 2], v[e * 8 + 3],
-                                            v[e * 8 + 4], v[e * 8 + 5], v[e * 8 + 6], v[e * 8 + 7]};
-                    st_global_v8(mine + j * 32 + e * 8, w8);
-                }
-            }
-            __threadfence();
-            __syncwarp();
-            int second = 0;
-            if (lane == 0) second = atomicAdd(&p.cnt[st * 8 + (warp - 2)], 1);
-            second = __shfl_sync(0xffffffffu, second, 0);
-            if (!second) {                                             // first: the other half finishes
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(y_empty);
-                return true;
-            }
-            __threadfence();
-            const int b0 = m * 128 + q * 32;
-#pragma unroll 1
-            for (int j2 = 0; j2 < W / 128; ++j2) {                     // 64 columns per round
-                const int col0 = half * (W / 2) + j2 * 64;
-                if (j2 > 0) {                                          // the previous round's store has read the rows
-                    if (lane == 0) bulk_wait_read_all();
-                    __syncwarp();
-                }
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t v[32];
-                    tmem_ld32_async(trow + col0 + hh * 32, v);
-                    tmem_wait_ld_tie(v);
-                    if (j2 == W / 128 - 1 && hh == 1) {                 // Y fully read: release it
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(y_empty);
-                    }
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {                      // 8 columns per 16-byte piece
-                        uint32_t o8[8];
-                        ld_global_cg_v8(other + j2 * 64 + hh * 32 + e * 8, o8);
-                        float f[8];
-#pragma unroll
-                        for (int z = 0; z < 8; ++z) f[z] = __uint_as_float(v[e * 8 + z]) + __uint_as_float(o8[z]);
-                        const uint4 w4 = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                                    pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-                        const int c8 = hh * 4 + e;
-                        uint8_t* dst = MIXG
-                                           ? stg + (c8 >> 1) * 1024 + lane * 32 + (((c8 & 1) ^ ((lane >> 2) & 1)) << 4)
-                                           : stg + lane * 128 + ((c8 ^ (lane & 7)) << 4);
-                        *reinterpret_cast<uint4*>(dst) = w4;
-                    }
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0 && b0 < p.rows) {
-                    if (MIXG) {
-                        const int per = p.omap.dh >> 4;
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const int ci = (col0 >> 4) + k, tok = ci / per, jj = ci - tok * per;
-                            tma_store_4d(&tmO, stg + k * 1024, 0, g * per + jj, tok, b0);
-                        }
-                    } else {
-                        tma_store_3d(&tmO, stg, col0, g, b0);
-                    }
-                    bulk_commit_group();
-                }
-                __syncwarp();
-            }
-            return true;
-        };
         int lt = 0;
         float sc = 0.f;
         // the statistics of a tile read the A slabs of this thread's half (FP8: of its whole row);
@@ -824,10 +713,7 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
         if (ok) release_a();
         F128Item prev = it;
         bool prev_pending = false;                                     // prev's output is still to be written
-        auto output_prev = [&](int ylt) -> bool {
-            return prev.sp < 0 ? output_tile(prev.g, prev.m, ylt, amix(prev), prev.sec)
-                               : output_split(prev.g, prev.m, ylt, prev.sp, prev.t - full_waves * (int)gridDim.x);
-        };
+        auto output_prev = [&](int ylt) -> bool { return output_tile(prev.g, prev.m, ylt, amix(prev), prev.sec); };
         uint32_t ubase = 0;                                            // chunks of the items before this one
         for (; ok && have; ++lt) {
             const int c0 = it.c0, c1 = it.c1;

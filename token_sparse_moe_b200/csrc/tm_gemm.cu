@@ -1,6 +1,5 @@
 // tm_gemm.cu -- instantiations and launchers of the tcgen05 kernels (grouped GEMM, fused sub-layer).
 #include <string.h>
-#include "tm_fused2.cuh"
 #include "tm_fused128.cuh"
 #include "tm_internal.h"
 
@@ -85,43 +84,6 @@ cudaError_t launch_fused128(int W, int a_mode, bool f8, const CUtensorMap& a, co
                   : launch_fused128_one<WW, AMM, false>(a, g, u, d, r, e, o, p, grid, st);
     TM_F128(256, A_TMA_MIX) TM_F128(256, A_TMA_3D) TM_F128(128, A_TMA_MIX) TM_F128(128, A_TMA_3D)
 #undef TM_F128
-    return cudaErrorInvalidValue;
-}
-
-template <int W, int AM>
-static cudaError_t launch_fused2_one(const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
-                                     const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st) {
-    using C = Fused2Cfg<W, AM>;
-    auto kern = fused2_swiglu_kernel<W, AM>;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(C::NTHREADS, 1, 1);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    ProfileScope ps_("fused_swiglu", st);
-    return cudaLaunchKernelEx(&cfg, kern, a, g, u, d, p);
-}
-
-cudaError_t launch_fused2(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
-                          const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st) {
-    if (W == 256 && a_mode == A_TMA_MIX) return launch_fused2_one<256, A_TMA_MIX>(a, g, u, d, p, grid, st);
-    if (W == 256 && a_mode == A_TMA_3D) return launch_fused2_one<256, A_TMA_3D>(a, g, u, d, p, grid, st);
-    if (W == 128 && a_mode == A_TMA_MIX) return launch_fused2_one<128, A_TMA_MIX>(a, g, u, d, p, grid, st);
-    if (W == 128 && a_mode == A_TMA_3D) return launch_fused2_one<128, A_TMA_3D>(a, g, u, d, p, grid, st);
     return cudaErrorInvalidValue;
 }
 

@@ -90,6 +90,7 @@ struct GemmParams {
     int32_t* r_idx;
     float* r_gate;
     float* r_inv_rms;
+    float* r_gap;              // optional [B, banks]: logit gap z_(k) - z_(k+1) (+inf when k == E)
     int32_t* r_counts;
     int r_nchunks;
     float r_alpha, r_eps;
@@ -161,11 +162,11 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int t) {
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               unsigned where) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = globaltimer_ns(), lim = wait_limit_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > lim) {
             record_error(ERR_TIMEOUT, where);
             *abort_flag = 1;
             return false;
@@ -494,6 +495,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
                 }
                 const size_t rowi = (size_t)b * p.banks + bank;
                 uint32_t chosen = 0;
+                float zk = INFINITY;   // logit of the k-th choice
 #pragma unroll 1
                 for (int j = 0; j < p.k; ++j) {
                     int be = -1;
@@ -502,6 +504,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
                     for (int e = 0; e < kRouteMaxE; ++e)
                         if (e < E && !((chosen >> e) & 1u) && (be < 0 || z[e] > bz)) { bz = z[e]; be = e; }
                     chosen |= 1u << be;
+                    zk = bz;
                     float pb = 0.f;
 #pragma unroll
                     for (int e = 0; e < kRouteMaxE; ++e)
@@ -512,6 +515,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
                     }
                 }
                 if (valid && p.r_inv_rms) p.r_inv_rms[rowi] = irs;
+                if (valid && p.r_gap) {
+                    // distance of the k-th choice to the best expert left out (none left: +inf)
+                    float zn = -INFINITY;
+#pragma unroll
+                    for (int e = 0; e < kRouteMaxE; ++e)
+                        if (e < E && !((chosen >> e) & 1u)) zn = fmaxf(zn, z[e]);
+                    p.r_gap[rowi] = zk - zn;
+                }
                 // per 128-row chunk: rows of this bank that chose expert e
                 for (int e = 0; e < E; ++e) {
                     const unsigned bal = __ballot_sync(0xffffffffu, valid && ((chosen >> e) & 1u));

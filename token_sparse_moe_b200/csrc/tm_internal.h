@@ -6,7 +6,6 @@
 #include <stdint.h>
 
 #include "tm_gemm.cuh"
-#include "tm_fused2.cuh"
 #include "tm_fused128.cuh"
 
 namespace tml {
@@ -61,25 +60,26 @@ struct FusedMaps {
 // counters; grid <= the number of SMs.
 cudaError_t launch_fused128_block(int W, bool f8, const FusedMaps& mix, const FusedMaps& rev, const CUtensorMap& r,
                                   const CUtensorMap& e, const FusedParams& p, int grid, cudaStream_t st);
-// CTA-pair version (2-SM MMAs, clusters of 2): grid = 2 x clusters; weight maps with half-size boxes
-cudaError_t launch_fused2(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
-                          const CUtensorMap& d, const FusedParams& p, int grid, cudaStream_t st);
 
 // ---- CUDA-core kernels ------------------------------------------------------------
 // dtype: 0 fp32, 1 bf16.
 cudaError_t launch_rms(int dtype, const void* x, RowMap m, int B, float eps, float* inv_rms, cudaStream_t st);
 cudaError_t launch_router(int dtype, const void* x, RowMap m, int B, float eps, const void* gain, const float* w_router,
-                          int E, int k, float alpha, int32_t* idx, float* gate, float* inv_rms, int32_t* counts,
-                          cudaStream_t st);
+                          int E, int k, float alpha, int32_t* idx, float* gate, float* inv_rms, float* logit_gap,
+                          int32_t* counts, cudaStream_t st);
 // tile_info (optional): one {group, first row position, rows, tile within the group} per 128-row tile
 cudaError_t launch_offsets(const int32_t* counts_in, int32_t* chunk_prefix, int banks, int nchunks, int E,
                            int32_t* bucket_offsets, int32_t* tile_start, cudaStream_t st, int4* tile_info = nullptr);
 // perm, inv_pos, gate_pos (optional, by bucket position): the sample-order row (b * banks + bank) * k + j,
 // the row's 1/rms (from inv_rms [B * banks]) and the choice's gate (from gate [B * banks * k])
+// limit: entries of bucket_rows (positions at or past it are reported as a bounds error and not
+// written); < 0: B * banks * k
 cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, const int32_t* bucket_offsets, int B,
                            int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st,
                            int32_t* perm = nullptr, const float* inv_rms = nullptr, const float* gate = nullptr,
-                           float* inv_pos = nullptr, float* gate_pos = nullptr);
+                           float* inv_pos = nullptr, float* gate_pos = nullptr, int limit = -1);
+// bounded-wait self-test (one CTA): res [4] device memory or NULL
+cudaError_t launch_wait_selftest(unsigned long long* res, cudaStream_t st);
 // tensor-core router weights: [banks][64][W] bf16, rows e / E+e / 2E+e = hi / mid / lo of w * gain
 cudaError_t launch_router_split(int dtype, const float* w_router, const void* gain, int banks, int E, int W,
                                 void* out, cudaStream_t st);

@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(256) router_kernel(const T* __restrict__ x, Ro
                                                      const T* __restrict__ gain, const float* __restrict__ w_router,
                                                      int E, int k, float alpha, int32_t* __restrict__ idx,
                                                      float* __restrict__ gate, float* __restrict__ inv_rms,
-                                                     int32_t* __restrict__ counts) {
+                                                     float* __restrict__ logit_gap, int32_t* __restrict__ counts) {
     constexpr int V = Vec<T>::N;
     constexpr int ROWS = 32 / EP;                 // rows per warp pass
     constexpr int GROUP = ROWS > 4 ? ROWS : 4;    // rows per staging buffer
@@ -167,6 +167,7 @@ __global__ void __launch_bounds__(256) router_kernel(const T* __restrict__ x, Ro
             const float p = pe / sum;
             const size_t rowi = (size_t)b * m.banks + bank;
             float zc = z;                       // candidate logit; -inf once taken
+            float zk = INFINITY;                // logit of the k-th choice
             for (int j = 0; j < k; ++j) {
                 float bz = zc;
                 int be = zc == -INFINITY ? 1 << 30 : e;   // ties and exhausted lanes: lower index wins
@@ -178,6 +179,7 @@ __global__ void __launch_bounds__(256) router_kernel(const T* __restrict__ x, Ro
                 }
                 const float pb = __shfl_sync(0xffffffffu, p, (lane & ~(EP - 1)) + (be < EP ? be : 0));
                 if (e == be) zc = -INFINITY;
+                zk = bz;
                 if (e == 0 && b < B && be < E) {
                     idx[rowi * k + j] = be;
                     gate[rowi * k + j] = alpha * pb;
@@ -185,6 +187,13 @@ __global__ void __launch_bounds__(256) router_kernel(const T* __restrict__ x, Ro
                 }
             }
             if (e == 0 && b < B && inv_rms) inv_rms[rowi] = irs;
+            if (logit_gap) {
+                // the best logit left after the k choices (lanes taken or past E hold -inf)
+                float zn = zc;
+#pragma unroll
+                for (int o = 1; o < EP; o <<= 1) zn = fmaxf(zn, __shfl_xor_sync(0xffffffffu, zn, o));
+                if (e == 0 && b < B) logit_gap[rowi] = zk - zn;
+            }
         }
         __syncwarp();                          // buffer (gi & 1) is refilled two groups later
     }
@@ -245,7 +254,8 @@ __global__ void __launch_bounds__(1024) offsets_kernel(int32_t* counts, int bank
 __global__ void __launch_bounds__(kRouterChunk) scatter_kernel(const int32_t* __restrict__ idx,
                                                                const int32_t* __restrict__ chunk_prefix,
                                                                const int32_t* __restrict__ bucket_offsets, int B,
-                                                               int banks, int E, int k, int32_t* __restrict__ bucket_rows,
+                                                               int banks, int E, int k, int limit,
+                                                               int32_t* __restrict__ bucket_rows,
                                                                int32_t* __restrict__ slot_of, int32_t* __restrict__ perm,
                                                                const float* __restrict__ inv_rms,
                                                                const float* __restrict__ gate, float* __restrict__ inv_pos,
@@ -274,7 +284,8 @@ __global__ void __launch_bounds__(kRouterChunk) scatter_kernel(const int32_t* __
     }
     __syncthreads();
     if (!valid) return;
-    const int limit = B * banks * k;
+    // positions must fall inside the caller's bucket_rows (limit entries): a table that does not
+    // match the choices is reported, never written out of range
     for (int j = 0; j < k; ++j) {
         const int e = my[j];
         if (e < 0 || e >= E) {
@@ -554,7 +565,7 @@ cudaError_t launch_rms(int dtype, const void* x, RowMap m, int B, float eps, flo
 template <typename T, int EP>
 static cudaError_t router_launch(const void* x, RowMap m, int B, float eps, const void* gain, const float* w_router,
                                  int E, int k, float alpha, int32_t* idx, float* gate, float* inv_rms,
-                                 int32_t* counts, cudaStream_t st) {
+                                 float* logit_gap, int32_t* counts, cudaStream_t st) {
     constexpr int GROUP = 32 / EP > 4 ? 32 / EP : 4;
     const size_t smem = (size_t)EP * (m.W + 4) * sizeof(float) + (size_t)8 * 2 * GROUP * m.W * sizeof(T);
     auto kern = router_kernel<T, EP>;
@@ -567,19 +578,19 @@ static cudaError_t router_launch(const void* x, RowMap m, int B, float eps, cons
     }
     dim3 grid((B + kRouterChunk - 1) / kRouterChunk, m.banks);
     kern<<<grid, 256, smem, st>>>((const T*)x, m, B, eps, (const T*)gain, w_router, E, k, alpha, idx, gate, inv_rms,
-                                  counts);
+                                  logit_gap, counts);
     return cudaGetLastError();
 }
 
 cudaError_t launch_router(int dtype, const void* x, RowMap m, int B, float eps, const void* gain,
                           const float* w_router, int E, int k, float alpha, int32_t* idx, float* gate, float* inv_rms,
-                          int32_t* counts, cudaStream_t st) {
+                          float* logit_gap, int32_t* counts, cudaStream_t st) {
     ProfileScope ps_("router", st);
 #define TM_ROUTER(T)                                                                                                  \
-    if (E <= 4) return router_launch<T, 4>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st);  \
-    if (E <= 8) return router_launch<T, 8>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st);  \
-    if (E <= 16) return router_launch<T, 16>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st); \
-    return router_launch<T, 32>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, counts, st);
+    if (E <= 4) return router_launch<T, 4>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, logit_gap, counts, st);  \
+    if (E <= 8) return router_launch<T, 8>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, logit_gap, counts, st);  \
+    if (E <= 16) return router_launch<T, 16>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, logit_gap, counts, st); \
+    return router_launch<T, 32>(x, m, B, eps, gain, w_router, E, k, alpha, idx, gate, inv_rms, logit_gap, counts, st);
     if (dtype == 1) { TM_ROUTER(__nv_bfloat16) }
     TM_ROUTER(float)
 #undef TM_ROUTER
@@ -595,12 +606,47 @@ cudaError_t launch_offsets(const int32_t* counts_in, int32_t* chunk_prefix, int 
 
 cudaError_t launch_scatter(const int32_t* idx, const int32_t* chunk_prefix, const int32_t* bucket_offsets, int B,
                            int banks, int E, int k, int32_t* bucket_rows, int32_t* slot_of, cudaStream_t st, int32_t* perm,
-                           const float* inv_rms, const float* gate, float* inv_pos, float* gate_pos) {
+                           const float* inv_rms, const float* gate, float* inv_pos, float* gate_pos, int limit) {
     if ((inv_pos && !inv_rms) || (gate_pos && !gate)) return cudaErrorInvalidValue;
+    if (E > 64 || k > 8) return cudaErrorInvalidValue;
     ProfileScope ps_("route_scatter", st);
     dim3 grid((B + kRouterChunk - 1) / kRouterChunk, banks);
-    scatter_kernel<<<grid, kRouterChunk, 0, st>>>(idx, chunk_prefix, bucket_offsets, B, banks, E, k, bucket_rows,
-                                                  slot_of, perm, inv_rms, gate, inv_pos, gate_pos);
+    scatter_kernel<<<grid, kRouterChunk, 0, st>>>(idx, chunk_prefix, bucket_offsets, B, banks, E, k,
+                                                  limit < 0 ? B * banks * k : limit, bucket_rows, slot_of, perm,
+                                                  inv_rms, gate, inv_pos, gate_pos);
+    return cudaGetLastError();
+}
+
+// Self-test of the bounded waits: no arrival ever comes, so each wait must give up, record where
+// and return (it never traps and never spins on).  Thread 0: first a plain bounded wait on barrier
+// 0 (site 0x7001), which runs out after the configured limit; then, with the CTA's abort flag set,
+// the role wait of the grouped GEMM on barrier 1, which must return at once without a record of its
+// own.  res[0], res[2]: nanoseconds each wait took; res[1], res[3]: 1 where the wait reported failure.
+__global__ void wait_selftest_kernel(unsigned long long* res) {
+    __shared__ uint64_t bars[2];
+    __shared__ int abort_flag;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    abort_flag = 0;
+    fence_barrier_init();
+    uint64_t t0 = globaltimer_ns();
+    const bool ok0 = mbar_wait(&bars[0], 0, 0x7001);
+    uint64_t t1 = globaltimer_ns();
+    if (!ok0) abort_flag = 1;
+    const bool ok1 = wait_or_abort(&bars[1], 0, reinterpret_cast<volatile int*>(&abort_flag), 0x7002);
+    uint64_t t2 = globaltimer_ns();
+    if (res) {
+        res[0] = t1 - t0;
+        res[1] = ok0 ? 0ull : 1ull;
+        res[2] = t2 - t1;
+        res[3] = ok1 ? 0ull : 1ull;
+    }
+}
+
+cudaError_t launch_wait_selftest(unsigned long long* res, cudaStream_t st) {
+    ProfileScope ps_("wait_selftest", st);
+    wait_selftest_kernel<<<1, 32, 0, st>>>(res);
     return cudaGetLastError();
 }
 

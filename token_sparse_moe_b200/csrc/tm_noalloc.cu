@@ -24,16 +24,39 @@ static __device__ __align__(256) unsigned char g_route_scratch[TM_NOALLOC_SCRATC
 
 std::mutex g_setup_mu;
 void* g_scratch_addr[64] = {nullptr};   // device address of g_route_scratch, per device
+void* g_scratch_ctx[64] = {nullptr};    // the context that address belongs to
 
-// Once per device, with that device current: the array's device address.  In host code the
-// array's name is only a host-side stand-in, so kernels get this address, never the name.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The calling thread's current driver context (NULL if it cannot be read).
+void* current_context() {
+    static CtxGetCurrentFn fn = nullptr;
+    static bool looked = false;
+    if (!looked) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+        looked = true;
+    }
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+// Once per device and context, with that device current: the array's device address.  In host
+// code the array's name is only a host-side stand-in, so kernels get this address, never the
+// name.  The address is looked up again when the device's context has changed (after a device
+// reset the module, and with it the array, is loaded anew).
 tm_status scratch_address(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) { note_cuda_error("tm_route_topk_noalloc: cudaGetDevice", e); return TM_ERR_CUDA; }
     if (dev < 0 || dev >= 64) return TM_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_setup_mu);
-    if (!g_scratch_addr[dev]) {
+    void* ctx = current_context();
+    if (!g_scratch_addr[dev] || ctx != g_scratch_ctx[dev]) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_route_scratch);
         if (e != cudaSuccess || !p) {
@@ -41,6 +64,7 @@ tm_status scratch_address(void** out) {
             return TM_ERR_CUDA;
         }
         g_scratch_addr[dev] = p;
+        g_scratch_ctx[dev] = current_context();
     }
     *out = g_scratch_addr[dev];
     return TM_OK;
@@ -53,8 +77,9 @@ using namespace tml;
 
 extern "C" tm_status tm_route_topk_noalloc(const void* x, tm_layout layout, const tm_shape* shape,
                                           const void* norm_gain, const tm_moe_w* w, int32_t* topk_idx,
-                                          float* topk_gate, float* inv_rms, int32_t* bucket_offsets,
-                                          int32_t* bucket_rows, int32_t* slot_of, void* stream) {
+                                          float* topk_gate, float* logit_gap_opt, float* inv_rms,
+                                          int32_t* bucket_offsets, int32_t* bucket_rows, int32_t* slot_of,
+                                          void* stream) {
     // the same validation as tm_route_topk: shape, weights and layout through the size query
     const size_t need = (shape && w) ? tm_route_workspace_bytes(shape, layout, w) : 0;
     if (need == 0) return TM_ERR_INVALID_ARG;
@@ -75,6 +100,6 @@ extern "C" tm_status tm_route_topk_noalloc(const void* x, tm_layout layout, cons
     if (s != TM_OK) return s;
     // The fixed array is the workspace of the ordinary entry point, so both take the same kernels
     // in the same order and give the same bits.  Nothing in it has to start at zero.
-    return tm_route_topk(x, layout, shape, norm_gain, w, topk_idx, topk_gate, inv_rms, bucket_offsets, bucket_rows,
-                         slot_of, base, TM_NOALLOC_SCRATCH_BYTES, stream);
+    return tm_route_topk(x, layout, shape, norm_gain, w, topk_idx, topk_gate, logit_gap_opt, inv_rms, bucket_offsets,
+                         bucket_rows, slot_of, base, TM_NOALLOC_SCRATCH_BYTES, stream);
 }
