@@ -85,6 +85,19 @@ def err_moe_delta(y, o, x, contrib, dtype="bf16", extra=None):
     return float(np.max(excess) / rms(o - x))
 
 
+def err_stored(dtype, y, o):
+    """The stated measure applied to a tensor the model stores in its dtype: for bf16, the error beyond
+    one unit in the last place of the stored value, max(0, |y - o| - ulp) / rms(o), ulp the larger of
+    the two values' spacings.  bf16 keeps 8 significant bits, so one ulp of an element with |v| >= 4
+    already exceeds 2e-2 of an output rms near 1; two correct evaluations (fp32 on the GPU, float64 in
+    the oracle) may round the same real value to neighbouring bf16 numbers, and deeper blocks carry
+    such a difference on through the residual.  fp32 tensors: the plain relative measure."""
+    if dtype == "f32":
+        return err_f32(y, o)
+    allow = np.maximum(ulp(o, dtype), ulp(y, dtype))
+    return float(np.max(np.maximum(np.abs(y - o) - allow, 0.0)) / rms(o))
+
+
 def tol(dtype):
     return F32_TOL if dtype == "f32" else BF16_TOL
 
@@ -246,8 +259,8 @@ def check_stack(cfg, blocks, y, samples=None, down_scale=None, device="cuda:0", 
     (gpu_stack_chain): samples are independent, so that batch must give y bit for bit, and it
     yields every block's output, X_revert and routing.  The oracle runs the same blocks from the
     same input (oracle_stack_forced), following the GPU only on near-tie rows.  Every sampled row
-    of every block (and X_revert) must meet the workload's tolerance; a routing difference outside
-    a near tie fails.  The counts go to REPORT."""
+    of every block (and X_revert) must meet the workload's tolerance beyond the storage rounding
+    (err_stored); a routing difference outside a near tie fails.  The counts go to REPORT."""
     import torch
     from token_sparse_moe_b200 import api
     n = cfg.B if samples is None else len(samples)
@@ -264,13 +277,17 @@ def check_stack(cfg, blocks, y, samples=None, down_scale=None, device="cuda:0", 
                              workers=min(16, os.cpu_count() or 1))
     gpu_idx = [{k: v["idx"].cpu().numpy() for k, v in r.items()} for r in routes]
     res = oracle_stack_forced(cfg, S.to_f64(X), get, gpu_idx)
-    worst = 0.0
+    assert res["bad"] == 0, f"{res['bad']} routing decisions differ outside near ties"
+    worst, worst_plain, n_ulp = 0.0, 0.0, 0
     for l in range(cfg.L):
         for name, g, o in (("Y", hist[l], res["Y"][l]), ("X_revert", Xr[l], res["Xr"][l])):
-            e = err(cfg.dtype, to_np(g), o)
+            gy = to_np(g)
+            e = err_stored(cfg.dtype, gy, o)
             assert e <= tol(cfg.dtype), (label or cfg.name, l + 1, name, e)
             worst = max(worst, e)
-    assert res["bad"] == 0, f"{res['bad']} routing decisions differ outside near ties"
+            worst_plain = max(worst_plain, err(cfg.dtype, gy, o))
+            if cfg.dtype == "bf16":
+                n_ulp += int(np.sum(np.abs(gy - o) > 0.75 * ulp(o, "bf16")))
     gpu_near = sum(int((r[k]["gap"] < GAP_TOL).sum().item()) for r in routes for k in r)
     if res["gap_mix0"] is not None:
         # block 1's mixing routers see the same input on both sides: the reported gaps agree
@@ -279,7 +296,8 @@ def check_stack(cfg, blocks, y, samples=None, down_scale=None, device="cuda:0", 
         fin = np.isfinite(og)
         assert np.array_equal(np.isfinite(gg), fin)
         assert np.max(np.abs(gg[fin] - og[fin]), initial=0.0) <= 1e-4
-    REPORT.append(f"{label or cfg.name}: {n} samples x {cfg.L} blocks, worst max|y-o|/scale {worst:.2e} "
-                  f"(tol {tol(cfg.dtype):g}); routing decisions {res['decisions']}, near-tie rows where the GPU "
-                  f"took the other valid set {res['near']}, GPU-reported gaps < {GAP_TOL:g}: {gpu_near}")
+    REPORT.append(f"{label or cfg.name}: {n} samples x {cfg.L} blocks (Y and X_revert of each), worst error beyond "
+                  f"storage rounding {worst:.2e} (tol {tol(cfg.dtype):g}), plain max|y-o|/rms {worst_plain:.2e}, "
+                  f"elements a whole ulp apart {n_ulp}; routing decisions {res['decisions']}, near-tie rows where "
+                  f"the GPU took the other valid set {res['near']}, GPU-reported gaps < {GAP_TOL:g}: {gpu_near}")
     return worst, res

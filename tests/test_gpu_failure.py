@@ -80,12 +80,15 @@ def _scatter_tables(B, banks, E, counted):
 
 
 def _run_scatter(idx, prefix, offsets, B, banks, E, capacity, guard=256):
-    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    # the device copies stay referenced until the kernel has run (the caching allocator would hand a
+    # freed temporary's memory to the next copy)
+    dev = [torch.from_numpy(np.ascontiguousarray(a)).to(DEV) for a in (idx, prefix, offsets)]
     rows = torch.full((capacity + guard,), -7, dtype=torch.int32, device=DEV)
     slot = torch.full((B, banks, 2), -5, dtype=torch.int32, device=DEV)
-    A.check(api.lib().tm_selftest_bucket_scatter(api._p(d(idx)), api._p(d(prefix)), api._p(d(offsets)), B, banks, E, 2,
+    A.check(api.lib().tm_selftest_bucket_scatter(api._p(dev[0]), api._p(dev[1]), api._p(dev[2]), B, banks, E, 2,
                                                  api._p(rows), capacity, api._p(slot), api._s(None)),
             "tm_selftest_bucket_scatter")
+    torch.cuda.synchronize()
     st = api.lib().tm_get_device_error(api._s(None))
     return st, rows.cpu().numpy(), slot.cpu().numpy()
 

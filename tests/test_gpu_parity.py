@@ -391,6 +391,24 @@ def test_deterministic_bits():
     assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
 
 
+@pytest.mark.parametrize("cfg", [DENSE_SMALL[0], DENSE_SMALL[3], MOE_SMALL[0], MOE_SMALL[1]], ids=lambda c: c.name)
+def test_rows_give_the_same_bits_wherever_they_sit(cfg):
+    """Samples are independent, so each sample's output bits must not depend on where it sits in
+    the batch (its row within a 128-row tile, its bucket position): the batch in reverse order and
+    a shuffled half of it give the same rows as the batch in order."""
+    c = cfg.with_(L=2, gap=0)
+    blocks = api.blocks_from_synth(c, DEV)
+    X = dev(S.make_x(c))
+    Y = api.stack_forward(X, blocks, 0, api.config_shape(c))
+    rev = torch.arange(c.B - 1, -1, -1, device=DEV)
+    Yr = api.stack_forward(X[rev].contiguous(), blocks, 0, api.config_shape(c))
+    assert torch.equal(Yr.view(torch.int16), Y[rev].view(torch.int16))
+    sub = torch.from_numpy(np.random.default_rng(5).permutation(c.B)[: c.B // 2].copy()).to(DEV)
+    Ys = api.stack_forward(X[sub].contiguous(), blocks, 0, api.config_shape(c.with_(B=c.B // 2)))
+    api.get_device_error()
+    assert torch.equal(Ys.view(torch.int16), Y[sub].view(torch.int16))
+
+
 def test_tokenize_stub():
     rng = np.random.default_rng(3)
     B, G, dg, D = 33, 5, 24, 64

@@ -7,7 +7,7 @@ import numpy as np
 import oracle
 import tm_synth as S
 from oracle import tokenmixer as O
-from parity_util import GAP_TOL, force_near_ties, oracle_stack_forced
+from parity_util import GAP_TOL, err_stored, force_near_ties, oracle_stack_forced, rms
 from tm_synth import FFNSpec
 
 
@@ -72,3 +72,18 @@ def test_layer_prefetch_getter_gives_the_same_weights():
                 wa, wb = plain(l, s, j), layer(l, s, j)
                 assert set(wa) == set(wb)
                 assert all(np.array_equal(wa[k], wb[k]) for k in wa)
+
+
+def test_stored_measure_allows_one_ulp_and_no_more():
+    """err_stored: a bf16 value one ulp away from the oracle's counts as no error (the two sides may
+    round one real number to neighbouring bf16 values); anything beyond that ulp counts in full."""
+    o = np.array([5.0, -0.25, 1.0, 3.0])          # rms 2.96
+    y = o.copy()
+    y[0] = 5.03125                                 # one ulp above 5 (bf16 spacing 2^-5 in [4, 8))
+    assert err_stored("bf16", y, o) == 0.0
+    y[0] = 5.0625                                  # two ulps
+    assert np.isclose(err_stored("bf16", y, o), 0.03125 / rms(o))
+    y = o.copy()
+    y[1] = -0.25 - 0.1                             # far beyond the ulp of a small value
+    assert np.isclose(err_stored("bf16", y, o), (0.1 - 2.0 ** -9) / rms(o))   # ulp in [0.25, 0.5): 2^-9
+    assert err_stored("f32", o * (1 + 1e-6), o) <= 1.01e-6

@@ -471,8 +471,8 @@ tm_status run_route(const Geo& g, const void* x, const void* gain, const tm_moe_
 
 // MoE combine on the tensor core: Y = residual (+ inter-residual) + sum_j (gate-scaled expert row j
 // of the sample) + Shared(n), one grouped-GEMM launch: the sources enter the accumulator through
-// identity MMAs (tensor maps in the output's row geometry and over the sample-order expert rows
-// [B, banks, k, W]), then the shared expert's GEMM2 accumulates onto them.
+// identity MMAs (tensor maps in the output's row geometry and over the bank-major expert rows
+// [banks][k][B][W]), then the shared expert's GEMM2 accumulates onto them.
 tm_status combine_sum(const Geo& g, const void* hidden_s, const void* wd, int Fs, const void* resid, const void* extra,
                       void* y, const void* slots, int k, cudaStream_t st) {
     GemmParams p = base_params(g);
@@ -499,10 +499,11 @@ tm_status combine_sum(const Geo& g, const void* hidden_s, const void* wd, int Fs
     if (extra && !gemm1_amap(g, extra, am, &m1)) return TM_ERR_CUDA;
     memset(&m2, 0, sizeof(m2));
     if (k > 0) {
-        uint64_t dims[4] = {(uint64_t)g.W, (uint64_t)k, (uint64_t)g.banks, (uint64_t)g.B};
-        uint64_t strides[3] = {(uint64_t)g.W * 2, (uint64_t)k * g.W * 2, (uint64_t)g.banks * k * g.W * 2};
-        uint32_t box[4] = {64, 1, 1, 128};
-        if (!make_map(&m2, slots, 4, dims, strides, box)) return TM_ERR_CUDA;
+        // the gate-scaled expert rows, bank-major [banks * k][B][W]: 128 consecutive samples per box
+        uint64_t dims[3] = {(uint64_t)g.W, (uint64_t)g.B, (uint64_t)g.banks * k};
+        uint64_t strides[2] = {(uint64_t)g.W * 2, (uint64_t)g.B * g.W * 2};
+        uint32_t box[3] = {64, 128, 1};
+        if (!make_map(&m2, slots, 3, dims, strides, box)) return TM_ERR_CUDA;
     }
     return cuda_status(launch_grouped_gemm_src(bn, A_TMA_2D, EPI_SUM, ma, mb, mb, m0, m1, m2, p, dense_grid(p), st, &mo));
 }
@@ -591,8 +592,8 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
         SimtGemmArgs a{p, (const float*)m.hidden_r, (const float*)w->we_down, nullptr};
         if ((s = cuda_status(launch_simt_gemm(EPI_SLOT, a, (int)(max_mt * p.n_tiles), st))) != TM_OK) return s;
     } else {
-        // rows written in sample order ((b * banks + bank) * k + j) and scaled by their gate, so that
-        // the combine reads each tile's expert rows as one tensor-map box per choice
+        // rows written in combine order ((bank * k + j) * B + b) and scaled by their gate, so that
+        // the combine reads each tile's expert rows as one contiguous tensor-map box per choice
         const int bn = pick_bn_out(g.W);
         p.n_tiles = g.W / bn;
         p.perm = m.perm;

@@ -323,7 +323,9 @@ __global__ void __launch_bounds__(FusedCfg<W, AMODE>::NTHREADS, 1)
                     const uint4* rp = reinterpret_cast<const uint4*>(sA + i * 4096 + r * 32);
 #pragma unroll
                     for (int v = 0; v < 2; ++v) {
-                        const uint4 w4 = rp[v ^ half];
+                        // logical half v (stored at v ^ ((r / 4) % 2) by the 32-byte swizzle): both
+                        // halves and every row position sum in column order
+                        const uint4 w4 = rp[v ^ ((r >> 2) & 1)];
                         const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {

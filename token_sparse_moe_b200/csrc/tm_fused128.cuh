@@ -542,7 +542,9 @@ __device__ __forceinline__ void fused128_body(const CUtensorMap& tmA, const CUte
                     const uint4* rp = reinterpret_cast<const uint4*>(sA + (half * (W / 32) + i) * 4096 + r * 32);
 #pragma unroll
                     for (int v = 0; v < 2; ++v) {
-                        const uint4 w4 = rp[v];
+                        // logical half v (the 32-byte swizzle stores it at v ^ ((r / 4) % 2)): every row
+                        // sums in column order wherever it sits in the tile
+                        const uint4 w4 = rp[v ^ ((r >> 2) & 1)];
                         const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {

@@ -30,7 +30,8 @@
 namespace tml {
 
 enum AMode : int { A_TMA_2D = 0, A_TMA_3D = 1, A_TMA_MIX = 2, A_GATHER = 3 };
-// EPI_SLOT_PERM: routed GEMM2 rows written in sample order (row perm[pos]) and scaled by their gate.
+// EPI_SLOT_PERM: routed GEMM2 rows written in combine order (row perm[pos] = (bank * k + j) * B + b)
+// and scaled by their gate.
 // EPI_SUM: the combine with its sources (residual, inter-residual, the k gate-scaled expert rows of
 // each sample) added on the tensor core before the shared expert's GEMM2; plain output epilogue.
 // EPI_ROUTE: the router on the tensor core; B holds each fp32 router row split exactly into three
@@ -83,7 +84,7 @@ struct GemmParams {
     const int* slot_of;        // combine: [B, banks, k]
     const __nv_bfloat16* slots;// combine: [row positions, W]
     int k;
-    const int* perm;           // EPI_SLOT_PERM: sample-order row (b * banks + bank) * k + j of each position
+    const int* perm;           // EPI_SLOT_PERM: combine-order row (bank * k + j) * B + b of each position
     int src_resid, src_extra;  // EPI_SUM: residual / inter-residual present (maps tmS0 / tmS1)
     int src_mix;               // EPI_SUM: residual maps use the 4-D mixed geometry (16-column boxes)
     // EPI_ROUTE outputs ([B, banks, k] rows of top-k, [B, banks] 1/rms, [banks][chunks][E] counts)
@@ -267,7 +268,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
                             mbar_arrive_expect_tx(&full[s], C::A_BYTES);
                             const int col = ti.n * BN + sl * 64;
                             if (kind == 2) {
-                                tma_load_4d(sa, &tmS2, &full[s], col, j, ti.g, ti.m * 128);
+                                // choice j's expert rows of the tile's 128 samples: rows m*128.. of
+                                // region (bank, j) of the bank-major expert rows
+                                tma_load_3d(sa, &tmS2, &full[s], col, ti.m * 128, ti.g * p.k + j);
                             } else if (p.src_mix) {
                                 const int per = p.omap.dh >> 4;
 #pragma unroll
@@ -759,8 +762,12 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
                 const uint8_t* sa = smem + s * C::STAGE_BYTES;
 #pragma unroll
                 for (int v = 0; v < 8; ++v) {
+                    // logical 16-byte piece v of the row (column order, wherever the row sits in the
+                    // tile): 32-byte swizzle stores half h at h ^ ((r / 4) % 2), 128-byte swizzle
+                    // stores piece v at v ^ (r % 8)
                     const uint4 w4 = AMODE == A_TMA_MIX
-                                         ? *reinterpret_cast<const uint4*>(sa + (v >> 1) * 4096 + r * 32 + ((v & 1) << 4))
+                                         ? *reinterpret_cast<const uint4*>(sa + (v >> 1) * 4096 + r * 32 +
+                                                                           (((v & 1) ^ ((r >> 2) & 1)) << 4))
                                          : *reinterpret_cast<const uint4*>(sa + r * 128 + (((v ^ r) & 7) << 4));
                     const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll

@@ -70,7 +70,7 @@ cudaError_t launch_router(int dtype, const void* x, RowMap m, int B, float eps, 
 // tile_info (optional): one {group, first row position, rows, tile within the group} per 128-row tile
 cudaError_t launch_offsets(const int32_t* counts_in, int32_t* chunk_prefix, int banks, int nchunks, int E,
                            int32_t* bucket_offsets, int32_t* tile_start, cudaStream_t st, int4* tile_info = nullptr);
-// perm, inv_pos, gate_pos (optional, by bucket position): the sample-order row (b * banks + bank) * k + j,
+// perm, inv_pos, gate_pos (optional, by bucket position): the combine-order row (bank * k + j) * B + b,
 // the row's 1/rms (from inv_rms [B * banks]) and the choice's gate (from gate [B * banks * k])
 // limit: entries of bucket_rows (positions at or past it are reported as a bounds error and not
 // written); < 0: B * banks * k

@@ -300,7 +300,9 @@ __global__ void __launch_bounds__(kRouterChunk) scatter_kernel(const int32_t* __
         }
         slot_of[rowi * k + j] = pos;
         bucket_rows[pos] = b;
-        if (perm) perm[pos] = (int32_t)(rowi * k + j);   // inverse of slot_of (optional)
+        // (optional) the combine-order row of this choice: bank-major, (bank * k + j) * B + b, so a
+        // tile of 128 samples of one bank reads each choice's expert rows as one contiguous box
+        if (perm) perm[pos] = (int32_t)(((size_t)bank * k + j) * B + b);
         // (optional) the row's 1/rms and the choice's gate by bucket position, so that the routed
         // GEMMs read them as contiguous per-row values
         if (inv_pos) inv_pos[pos] = inv_rms[rowi];
