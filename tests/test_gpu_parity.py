@@ -409,6 +409,23 @@ def test_rows_give_the_same_bits_wherever_they_sit(cfg):
     assert torch.equal(Ys.view(torch.int16), Y[sub].view(torch.int16))
 
 
+@pytest.mark.parametrize("cfg", [MOE_SMALL[0], MOE_SMALL[1], DENSE_SMALL[1]], ids=lambda c: c.name)
+def test_cta_pair_gemms_match_single_cta_gemms(cfg, monkeypatch):
+    """The grouped GEMMs on CTA pairs (M = 256 per tile, each SM streaming half of the weight rows)
+    against the one-CTA form (TM_PAIR=0): the same bits, a stack of two blocks with the gain."""
+    c = cfg.with_(L=2, gap=0)
+    blocks = [api.Block(api.sublayer_from_synth(c, l, 0, DEV, None, True), api.sublayer_from_synth(c, l, 1, DEV, None, True))
+              for l in range(c.L)]
+    X = dev(S.make_x(c))
+    sh = api.config_shape(c)
+    Y1 = api.stack_forward(X, blocks, 0, sh)
+    monkeypatch.setenv("TM_PAIR", "0")
+    Y0 = api.stack_forward(X, blocks, 0, sh)
+    monkeypatch.delenv("TM_PAIR")
+    api.get_device_error()
+    assert torch.equal(Y1.view(torch.int16), Y0.view(torch.int16))
+
+
 def test_tokenize_stub():
     rng = np.random.default_rng(3)
     B, G, dg, D = 33, 5, 24, 64

@@ -225,6 +225,28 @@ int dense_grid(const GemmParams& p) {
     return (int)(tiles < num_sms() ? tiles : num_sms());
 }
 
+bool env_is(const char* name, char v);
+
+// CTA pairs (M = 256 per tile, each SM streaming half of the weight rows) for the combine of bf16
+// rows: the kernel that streams the most weight rows per tile (the shared expert's down projection
+// beside its k + 1 source slabs) measured 7-10% faster so on the MoE stacks, while GEMM1 measured
+// the same and the routed GEMM2, whose epilogue bounds it, slower (a pair waits for the slower of
+// its two epilogues).  TM_PAIR=0 in the environment keeps one CTA per tile: the tests use it to show
+// that both forms give the same bits.
+bool use_pair(const Geo& g, int amode) {
+    return g.dtype == TM_BF16 && amode != A_GATHER && !env_is("TM_PAIR", '0');
+}
+// grid of a pair-mode launch: two CTAs per cluster, at most one cluster per two SMs
+int pair_grid(long pair_tiles) {
+    const long c = pair_tiles < num_sms() / 2 ? pair_tiles : num_sms() / 2;
+    return (int)(2 * (c > 0 ? c : 1));
+}
+// grid of a launch over dense groups (sched 0) in either form
+int sched0_grid(const GemmParams& p, bool pair) {
+    if (!pair) return dense_grid(p);
+    return pair_grid((long)p.groups * ((p.rows + 255) / 256) * p.n_tiles);
+}
+
 // SwiGLU GEMM1 over x (dense groups = banks, rows = B): hidden [banks*B, F]
 tm_status gemm1_dense(const Geo& g, const void* x, const void* wg, const void* wu, int F, const float* inv_rms,
                       void* hidden, cudaStream_t st) {
@@ -489,11 +511,12 @@ tm_status combine_sum(const Geo& g, const void* hidden_s, const void* wd, int Fs
     if (am != A_TMA_MIX && am != A_TMA_3D) return TM_ERR_UNSUPPORTED;
     const int bn = pick_bn_out(g.W);
     p.n_tiles = g.W / bn;
+    const bool pair = use_pair(g, A_TMA_2D);
     CUtensorMap ma, mb, m0, m1, m2, mo;
     memset(&m0, 0, sizeof(m0));
     memset(&m1, 0, sizeof(m1));
-    if (!map_2d(&ma, hidden_s, (uint64_t)g.banks * g.B, Fs, 128) || !map_2d(&mb, wd, (uint64_t)g.banks * g.W, Fs, bn) ||
-        !gemm1_amap(g, y, am, &mo, 32))
+    if (!map_2d(&ma, hidden_s, (uint64_t)g.banks * g.B, Fs, 128) ||
+        !map_2d(&mb, wd, (uint64_t)g.banks * g.W, Fs, pair ? bn / 2 : bn) || !gemm1_amap(g, y, am, &mo, 32))
         return TM_ERR_CUDA;
     if (resid && !gemm1_amap(g, resid, am, &m0)) return TM_ERR_CUDA;
     if (extra && !gemm1_amap(g, extra, am, &m1)) return TM_ERR_CUDA;
@@ -505,7 +528,8 @@ tm_status combine_sum(const Geo& g, const void* hidden_s, const void* wd, int Fs
         uint32_t box[3] = {64, 128, 1};
         if (!make_map(&m2, slots, 3, dims, strides, box)) return TM_ERR_CUDA;
     }
-    return cuda_status(launch_grouped_gemm_src(bn, A_TMA_2D, EPI_SUM, ma, mb, mb, m0, m1, m2, p, dense_grid(p), st, &mo));
+    return cuda_status(
+        launch_grouped_gemm_src(bn, A_TMA_2D, EPI_SUM, ma, mb, mb, m0, m1, m2, p, sched0_grid(p, pair), st, &mo, pair));
 }
 
 tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* extra, const void* gain,
@@ -557,7 +581,7 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
     p.out_ld = Fe;
     p.out_elems = routed * Fe;
     p.a_ptr = (const __nv_bfloat16*)x;
-    const long max_mt = (long)(routed / 128) + (long)G;
+    const long max_mt = (long)(routed / 128) + (long)G;   // 128-row tiles of the buckets, at most
     if (g.dtype == TM_F32) {
         p.n_tiles = Fe / 32;
         SimtGemmArgs a{p, (const float*)x, (const float*)weg, (const float*)weu};

@@ -100,12 +100,12 @@ cudaError_t launch_fused(int W, int a_mode, const CUtensorMap& a, const CUtensor
     return cudaErrorInvalidValue;
 }
 
-template <int BN, int AM, int EPI>
+template <int BN, int AM, int EPI, bool PAIR>
 static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& s0,
                               const CUtensorMap& s1, const CUtensorMap& s2, const CUtensorMap& o, const GemmParams& p,
                               int grid, cudaStream_t st) {
-    using C = GemmCfg<BN, AM, EPI>;
-    auto kern = grouped_gemm_kernel<BN, AM, EPI>;
+    using C = GemmCfg<BN, AM, EPI, PAIR>;
+    auto kern = grouped_gemm_kernel<BN, AM, EPI, PAIR>;
     static bool configured = false;   // attribute set once per instantiation (per process)
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -118,37 +118,57 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
                      : (EPI == EPI_SLOT || EPI == EPI_SLOT_PERM) ? "gemm_slot"
                                                                  : "gemm_combine",
                      st);
-    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, b0, b1, s0, s1, s2, o, p);
-    return cudaGetLastError();
+    if (!PAIR) {
+        kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(a, b0, b1, s0, s1, s2, o, p);
+        return cudaGetLastError();
+    }
+    // pair mode: clusters of two CTAs (grid even)
+    if (grid % 2) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(C::NTHREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, s0, s1, s2, o, p);
 }
 
-// Supported (BN, A mode, epilogue) combinations.
-//   GEMM1 (SwiGLU): A from x (3-D rows map, 4-D mixed map, or gather), BN 256 or 128
+// Supported (BN, A mode, epilogue, pair mode) combinations.
+//   GEMM1 (SwiGLU): A from x (3-D rows map, 4-D mixed map, or gather) or bucketed rows, BN 256 or 128
 //   GEMM2:          A = hidden rows (2-D map), BN 256, 192 or 128
+//   pair mode (CTA pairs, M = 256): the MoE GEMMs and the combine
 #define TM_GEMM_TABLE(X)                                  \
-    X(256, A_TMA_3D, EPI_SWIGLU) X(128, A_TMA_3D, EPI_SWIGLU) \
-    X(256, A_TMA_MIX, EPI_SWIGLU) X(128, A_TMA_MIX, EPI_SWIGLU) \
-    X(256, A_GATHER, EPI_SWIGLU) X(128, A_GATHER, EPI_SWIGLU) \
-    X(256, A_TMA_2D, EPI_SWIGLU) X(128, A_TMA_2D, EPI_SWIGLU) \
-    X(256, A_TMA_2D, EPI_RESID) X(192, A_TMA_2D, EPI_RESID) X(128, A_TMA_2D, EPI_RESID) \
-    X(256, A_TMA_2D, EPI_SLOT) X(192, A_TMA_2D, EPI_SLOT) X(128, A_TMA_2D, EPI_SLOT) \
-    X(256, A_TMA_2D, EPI_COMBINE) X(192, A_TMA_2D, EPI_COMBINE) X(128, A_TMA_2D, EPI_COMBINE) \
-    X(256, A_TMA_2D, EPI_SLOT_PERM) X(192, A_TMA_2D, EPI_SLOT_PERM) X(128, A_TMA_2D, EPI_SLOT_PERM) \
-    X(256, A_TMA_2D, EPI_SUM) X(192, A_TMA_2D, EPI_SUM) X(128, A_TMA_2D, EPI_SUM) \
-    X(64, A_TMA_3D, EPI_ROUTE) X(64, A_TMA_MIX, EPI_ROUTE)
+    X(256, A_TMA_3D, EPI_SWIGLU, 0) X(128, A_TMA_3D, EPI_SWIGLU, 0) \
+    X(256, A_TMA_MIX, EPI_SWIGLU, 0) X(128, A_TMA_MIX, EPI_SWIGLU, 0) \
+    X(256, A_GATHER, EPI_SWIGLU, 0) X(128, A_GATHER, EPI_SWIGLU, 0) \
+    X(256, A_TMA_2D, EPI_SWIGLU, 0) X(128, A_TMA_2D, EPI_SWIGLU, 0) \
+    X(256, A_TMA_2D, EPI_RESID, 0) X(192, A_TMA_2D, EPI_RESID, 0) X(128, A_TMA_2D, EPI_RESID, 0) \
+    X(256, A_TMA_2D, EPI_SLOT, 0) X(192, A_TMA_2D, EPI_SLOT, 0) X(128, A_TMA_2D, EPI_SLOT, 0) \
+    X(256, A_TMA_2D, EPI_COMBINE, 0) X(192, A_TMA_2D, EPI_COMBINE, 0) X(128, A_TMA_2D, EPI_COMBINE, 0) \
+    X(256, A_TMA_2D, EPI_SLOT_PERM, 0) X(192, A_TMA_2D, EPI_SLOT_PERM, 0) X(128, A_TMA_2D, EPI_SLOT_PERM, 0) \
+    X(256, A_TMA_2D, EPI_SUM, 0) X(192, A_TMA_2D, EPI_SUM, 0) X(128, A_TMA_2D, EPI_SUM, 0) \
+    X(64, A_TMA_3D, EPI_ROUTE, 0) X(64, A_TMA_MIX, EPI_ROUTE, 0) \
+    X(256, A_TMA_2D, EPI_SUM, 1) X(192, A_TMA_2D, EPI_SUM, 1) X(128, A_TMA_2D, EPI_SUM, 1)
 
 cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                                     const CUtensorMap& tmB1, const CUtensorMap& tmS0, const CUtensorMap& tmS1,
                                     const CUtensorMap& tmS2, const GemmParams& p, int grid, cudaStream_t st,
-                                    const CUtensorMap* tmO) {
+                                    const CUtensorMap* tmO, bool pair) {
     // the SwiGLU, combine and plain-row epilogues store through the output map
     if ((epi == EPI_SWIGLU || epi == EPI_SUM || epi == EPI_SLOT) && !tmO) return cudaErrorInvalidValue;
     CUtensorMap none;
     memset(&none, 0, sizeof(none));
     const CUtensorMap& o = tmO ? *tmO : none;
-#define X(BN, AM, EP)                                  \
-    if (bn == BN && a_mode == AM && epi == EP)         \
-        return launch_one<BN, AM, EP>(tmA, tmB0, tmB1, tmS0, tmS1, tmS2, o, p, grid, st);
+#define X(BN, AM, EP, PR)                                               \
+    if (bn == BN && a_mode == AM && epi == EP && pair == (PR != 0))     \
+        return launch_one<BN, AM, EP, PR != 0>(tmA, tmB0, tmB1, tmS0, tmS1, tmS2, o, p, grid, st);
     TM_GEMM_TABLE(X)
 #undef X
     return cudaErrorInvalidValue;
@@ -156,10 +176,10 @@ cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorM
 
 cudaError_t launch_grouped_gemm(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                                 const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st,
-                                const CUtensorMap* tmO) {
+                                const CUtensorMap* tmO, bool pair) {
     CUtensorMap none;
     memset(&none, 0, sizeof(none));
-    return launch_grouped_gemm_src(bn, a_mode, epi, tmA, tmB0, tmB1, none, none, none, p, grid, st, tmO);
+    return launch_grouped_gemm_src(bn, a_mode, epi, tmA, tmB0, tmB1, none, none, none, p, grid, st, tmO, pair);
 }
 
 }  // namespace tml

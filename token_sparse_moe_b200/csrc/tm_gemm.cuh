@@ -24,6 +24,14 @@
 // warp 0 TMA producer, warp 1 MMA issuer (one thread) and TMEM owner, warps 2-5
 // epilogue (TMEM lane quarter = warp % 4), warps 6-9 row gatherers (gather mode).
 // TMEM holds two accumulators so the epilogue of tile i overlaps the MMAs of i+1.
+//
+// Pair mode (PAIR, groups of equal rows): a cluster of two CTAs on two SMs works on 256 rows of one
+// group; each CTA loads its own 128 A rows and half of the BN weight rows (GEMM1: the leader the
+// gate rows, the peer the up rows; otherwise the two halves of the N tile), and the leader issues one
+// tcgen05.mma.cta_group::2 (M = 256) per K step, so each SM streams half the weight bytes of a
+// 128-row tile.  Both CTAs' loads complete on the leader's stage barriers; the leader's commits
+// arrive on the barriers of both CTAs; each CTA's epilogue reads its own accumulator rows and
+// arrives on the leader's accumulator-free barrier.  No load and no commit uses multicast.
 #pragma once
 #include "tm_device.cuh"
 
@@ -97,16 +105,23 @@ struct GemmParams {
     float r_alpha, r_eps;
 };
 
-template <int BN, int AMODE, int EPI = EPI_SWIGLU>
+template <int BN, int AMODE, int EPI = EPI_SWIGLU, bool PAIR = false>
 struct GemmCfg {
     static constexpr int BM = 128, BK = 64;
     static constexpr int A_BYTES = BM * BK * 2;
-    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * BK * 2;   // this CTA's weight rows of a stage
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     // the scattered-row epilogue is latency-bound per warp: two warps per TMEM lane quarter, each
     // taking half of the tile's columns
     static constexpr int EPI_WARPS = (EPI == EPI_SLOT_PERM && BN % 128 == 0) ? 8 : 4;
-    static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 192 ? (EPI_WARPS == 8 ? 4 : 5) : 6);
+    static constexpr int STG_BYTES_ = (EPI == EPI_SWIGLU || EPI == EPI_SLOT_PERM || EPI == EPI_SUM || EPI == EPI_SLOT)
+                                          ? EPI_WARPS * 4096 : 0;
+    // pair mode: as many stages as the shared memory holds, at most 8
+    static constexpr int PAIR_STAGES_ = (232448 - 2304 - STG_BYTES_) / STAGE_BYTES;
+    static constexpr int STAGES = PAIR ? (PAIR_STAGES_ > 8 ? 8 : PAIR_STAGES_)
+                                       : (BN >= 256 ? 4 : (BN >= 192 ? (EPI_WARPS == 8 ? 4 : 5) : 6));
+    static_assert(!PAIR || (AMODE != A_GATHER && EPI != EPI_ROUTE && EPI != EPI_RESID && EPI != EPI_COMBINE),
+                  "pair mode covers tensor-map A operands and the staged epilogues");
     static constexpr int NWARPS = (AMODE == A_GATHER || EPI == EPI_ROUTE) ? 10 : 2 + EPI_WARPS;
     static constexpr int NTHREADS = NWARPS * 32;
     static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
@@ -126,6 +141,26 @@ struct TileInfo {
 __device__ __forceinline__ int total_tiles(const GemmParams& p) {
     if (p.sched == 0) return p.groups * ((p.rows + 127) / 128) * p.n_tiles;
     return __ldg(&p.tile_start[p.groups]) * p.n_tiles;
+}
+
+// Pair mode (groups of equal rows, sched 0): tiles of 256 rows, two CTAs' 128-row halves.
+__device__ __forceinline__ int total_tiles_pair(const GemmParams& p) {
+    return p.groups * ((p.rows + 255) / 256) * p.n_tiles;
+}
+
+// This CTA's 128-row half (rank 0: the first) of 256-row tile t, row block major with the banks
+// innermost as decode_tile; a half past the group's end has nrows = 0 (its rows are loaded,
+// multiplied and never stored).
+__device__ __forceinline__ TileInfo decode_tile_pair(const GemmParams& p, int t, int rank) {
+    TileInfo ti;
+    const int gm = t / p.n_tiles;
+    ti.n = t - gm * p.n_tiles;
+    const int m2 = gm / p.groups;
+    ti.g = gm - m2 * p.groups;
+    ti.m = 2 * m2 + rank;
+    ti.row0 = ti.g * p.rows + ti.m * 128;
+    ti.nrows = max(0, min(128, p.rows - ti.m * 128));
+    return ti;
 }
 
 __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int t) {
@@ -159,6 +194,23 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int t) {
     return ti;
 }
 
+// The same wait with cluster-scope acquire: for barriers that the other CTA of a pair (its loads,
+// commits or arrivals) completes.
+__device__ __forceinline__ bool wait_or_abort_cl(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                 unsigned where) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns(), lim = wait_limit_ns();
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > lim) {
+            record_error(ERR_TIMEOUT, where);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
 // Bounded wait that also gives up as soon as another role of the CTA has given up.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               unsigned where) {
@@ -175,16 +227,23 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     }
 }
 
-template <int BN, int AMODE, int EPI>
-__global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
+template <int BN, int AMODE, int EPI, bool PAIR>
+__global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmS0,
                         const __grid_constant__ CUtensorMap tmS1, const __grid_constant__ CUtensorMap tmS2,
                         const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
-    using C = GemmCfg<BN, AMODE, EPI>;
+    using C = GemmCfg<BN, AMODE, EPI, PAIR>;
     constexpr int STAGES = C::STAGES;
-    const int ntile = total_tiles(p);
-    if ((int)blockIdx.x >= ntile) return;
+    // pair mode: the two CTAs of a cluster share the tile sequence (cluster index cid), each taking
+    // its 128-row half; both return here together, so both reach the closing cluster barrier
+    const int rank = PAIR ? (int)cluster_ctarank() : 0;
+    const bool leader = rank == 0;
+    const int cid = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int ncid = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    const int ntile = PAIR ? total_tiles_pair(p) : total_tiles(p);
+    if (cid >= ntile) return;
+    auto dec = [&](int t) -> TileInfo { return PAIR ? decode_tile_pair(p, t, rank) : decode_tile(p, t); };
     // EPI_SUM source stages per tile: residual, inter-residual, then expert choice j = 0..k-1, each
     // as BN / 64 slabs of 128 rows x 64 columns (one ring stage each, A part only)
     const int n_src = EPI == EPI_SUM ? (p.src_resid + p.src_extra + p.k) : 0;
@@ -206,6 +265,13 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int KB = p.K / 64;
+    // pair mode: the leader's copy (L) and the peer's copy (P) of a barrier of this CTA's layout
+    auto L = [&](uint64_t* b) { return mapa_shared(smem_u32(b), 0); };
+    auto P = [&](uint64_t* b) { return mapa_shared(smem_u32(b), 1); };
+    // waits on barriers that the other CTA of a pair completes take cluster-scope acquire
+    auto wait = [&](uint64_t* b, uint32_t par, unsigned where) -> bool {
+        return PAIR ? wait_or_abort_cl(b, par, abort_flag, where) : wait_or_abort(b, par, abort_flag, where);
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -214,7 +280,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], C::EPI_WARPS);
+            mbar_init(&acc_empty[b], C::EPI_WARPS * (PAIR ? 2 : 1));   // pair: both CTAs' epilogue warps
         }
         mbar_init(drain, 1);
         for (int b = 0; b < 2; ++b) {
@@ -226,20 +292,29 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
     }
     if (EPI == EPI_SUM && warp == 0) {
         // identity B operand: 16 rows n x 16 columns k, 32-byte rows, 32-byte swizzle (the 16-byte
-        // half of row n that holds column k sits at half (k / 8) ^ ((n / 4) % 2))
-        const int n = lane & 15, hf = lane >> 4;
-        const uint32_t one = (n >> 3) == hf ? ((n & 1) ? 0x3F800000u : 0x00003F80u) : 0u;
+        // half of row n that holds column k sits at half (k / 8) ^ ((n / 4) % 2)).  Pair mode: the N
+        // rows are split between the CTAs, so this CTA holds identity rows n = 8 rank + i as its
+        // local rows i = 0..7.
+        const int i = lane & 15, hf = lane >> 4;
+        const int n = PAIR ? 8 * rank + (i & 7) : i;
+        const uint32_t one = (PAIR && i >= 8) ? 0u : ((n >> 3) == hf ? ((n & 1) ? 0x3F800000u : 0x00003F80u) : 0u);
         const int wi = (n & 7) >> 1;
-        *reinterpret_cast<uint4*>(sI + n * 32 + ((hf ^ ((n >> 2) & 1)) << 4)) =
+        *reinterpret_cast<uint4*>(sI + i * 32 + ((hf ^ ((i >> 2) & 1)) << 4)) =
             make_uint4(wi == 0 ? one : 0u, wi == 1 ? one : 0u, wi == 2 ? one : 0u, wi == 3 ? one : 0u);
         fence_proxy_async_smem();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_base_smem, C::TMEM_COLS);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(tmem_base_smem, C::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_base_smem, C::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR) cluster_sync_all();            // both CTAs' barriers exist before any remote use
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_smem;
 
@@ -251,10 +326,30 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
             if (EPI == EPI_SWIGLU) tma_prefetch_desc(&tmB1);
             int s = 0;
             uint32_t ph = 0;
-            TileInfo tn = decode_tile(p, blockIdx.x);
-            for (int t = blockIdx.x; t < ntile; t += gridDim.x) {
+            // a stage's loads count their bytes on this CTA's full barrier, or in pair mode on the
+            // leader's, which expects both CTAs' bytes
+            const uint32_t bytes_src = (PAIR ? 2 : 1) * C::A_BYTES;
+            const uint32_t bytes_k = (PAIR ? 2 : 1) * ((AMODE == A_GATHER ? 0 : C::A_BYTES) + C::B_BYTES);
+            auto begin_stage = [&](uint32_t bytes) {
+                if (!PAIR) mbar_arrive_expect_tx(&full[s], bytes);
+                else if (leader) mbar_arrive_expect_tx(&full[s], bytes);
+            };
+            auto ld2 = [&](void* dst, const CUtensorMap* m, int c0, int c1) {
+                if (PAIR) tma_load_2d_pair(dst, m, L(&full[s]), c0, c1);
+                else tma_load_2d(dst, m, &full[s], c0, c1);
+            };
+            auto ld3 = [&](void* dst, const CUtensorMap* m, int c0, int c1, int c2) {
+                if (PAIR) tma_load_3d_pair(dst, m, L(&full[s]), c0, c1, c2);
+                else tma_load_3d(dst, m, &full[s], c0, c1, c2);
+            };
+            auto ld4 = [&](void* dst, const CUtensorMap* m, int c0, int c1, int c2, int c3) {
+                if (PAIR) tma_load_4d_pair(dst, m, L(&full[s]), c0, c1, c2, c3);
+                else tma_load_4d(dst, m, &full[s], c0, c1, c2, c3);
+            };
+            TileInfo tn = dec(cid);
+            for (int t = cid; t < ntile; t += ncid) {
                 const TileInfo ti = tn;
-                if (t + (int)gridDim.x < ntile) tn = decode_tile(p, t + gridDim.x);   // in flight meanwhile
+                if (t + ncid < ntile) tn = dec(t + ncid);   // in flight meanwhile
                 if (EPI == EPI_SUM) {
                     // source slabs: rows of this tile's samples, output columns n*BN .. +BN
 #pragma unroll 1
@@ -263,38 +358,37 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
                         const int j = src - p.src_resid - p.src_extra;
 #pragma unroll 1
                         for (int sl = 0; sl < BN / 64; ++sl) {
-                            if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x103)) goto producer_done;
+                            if (!wait(&empty[s], ph ^ 1, 0x103)) goto producer_done;
                             uint8_t* sa = smem + s * C::STAGE_BYTES;
-                            mbar_arrive_expect_tx(&full[s], C::A_BYTES);
+                            begin_stage(bytes_src);
                             const int col = ti.n * BN + sl * 64;
                             if (kind == 2) {
                                 // choice j's expert rows of the tile's 128 samples: rows m*128.. of
                                 // region (bank, j) of the bank-major expert rows
-                                tma_load_3d(sa, &tmS2, &full[s], col, ti.m * 128, ti.g * p.k + j);
+                                ld3(sa, &tmS2, col, ti.m * 128, ti.g * p.k + j);
                             } else if (p.src_mix) {
                                 const int per = p.omap.dh >> 4;
 #pragma unroll
                                 for (int i = 0; i < 4; ++i) {
                                     const int c16 = (col >> 4) + i, tk = c16 / per, jj = c16 - tk * per;
-                                    tma_load_4d(sa + i * 4096, kind == 0 ? &tmS0 : &tmS1, &full[s], 0, ti.g * per + jj, tk,
-                                                ti.m * 128);
+                                    ld4(sa + i * 4096, kind == 0 ? &tmS0 : &tmS1, 0, ti.g * per + jj, tk, ti.m * 128);
                                 }
                             } else {
-                                tma_load_3d(sa, kind == 0 ? &tmS0 : &tmS1, &full[s], col, ti.g, ti.m * 128);
+                                ld3(sa, kind == 0 ? &tmS0 : &tmS1, col, ti.g, ti.m * 128);
                             }
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                     }
                 }
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, 0x100)) goto producer_done;
+                    if (!wait(&empty[s], ph ^ 1, 0x100)) goto producer_done;
                     uint8_t* sa = smem + s * C::STAGE_BYTES;
                     uint8_t* sb = sa + C::A_BYTES;
-                    mbar_arrive_expect_tx(&full[s], (AMODE == A_GATHER ? 0 : C::A_BYTES) + C::B_BYTES);
+                    begin_stage(bytes_k);
                     if (AMODE == A_TMA_2D) {
-                        tma_load_2d(sa, &tmA, &full[s], kb * 64, ti.row0);
+                        ld2(sa, &tmA, kb * 64, ti.row0);
                     } else if (AMODE == A_TMA_3D) {
-                        tma_load_3d(sa, &tmA, &full[s], kb * 64, ti.g, ti.m * 128);
+                        ld3(sa, &tmA, kb * 64, ti.g, ti.m * 128);
                     } else if (AMODE == A_TMA_MIX) {
                         // mixed-row columns c16*16 .. +15 = token t, head piece jj of head ti.g
                         const int per = p.amap.dh >> 4;
@@ -302,16 +396,22 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
                         for (int i = 0; i < 4; ++i) {
                             const int c16 = kb * 4 + i;
                             const int t = c16 / per, jj = c16 - t * per;
-                            tma_load_4d(sa + i * 4096, &tmA, &full[s], 0, ti.g * per + jj, t, ti.m * 128);
+                            ld4(sa + i * 4096, &tmA, 0, ti.g * per + jj, t, ti.m * 128);
                         }
                     }
                     if (EPI == EPI_SWIGLU) {
                         const int F = p.N >> 1;
                         const int r0 = ti.g * F + ti.n * (BN / 2);
-                        tma_load_2d(sb, &tmB0, &full[s], kb * 64, r0);
-                        tma_load_2d(sb + (BN / 2) * 128, &tmB1, &full[s], kb * 64, r0);
+                        if (PAIR) {
+                            // the leader holds the BN/2 gate rows (N rows 0 .. BN/2-1), the peer the up rows
+                            ld2(sb, leader ? &tmB0 : &tmB1, kb * 64, r0);
+                        } else {
+                            ld2(sb, &tmB0, kb * 64, r0);
+                            ld2(sb + (BN / 2) * 128, &tmB1, kb * 64, r0);
+                        }
                     } else {
-                        tma_load_2d(sb, &tmB0, &full[s], kb * 64, ti.g * p.N + ti.n * BN);
+                        // pair mode: this CTA's half of the N tile's weight rows
+                        ld2(sb, &tmB0, kb * 64, ti.g * p.N + ti.n * BN + (PAIR ? rank * (BN / 2) : 0));
                     }
                     if (++s == STAGES) { s = 0; ph ^= 1; }
                 }
@@ -319,45 +419,59 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
         }
     producer_done:;
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = umma_idesc_bf16(128, BN);
+        // ---------------------------------------------------------------- MMA issuer (pair mode: leader)
+        if (lane == 0 && leader) {
+            constexpr uint32_t idesc = umma_idesc_bf16(PAIR ? 256 : 128, BN);
+            // an MMA of this CTA (M = 128) or of the pair (M = 256); commits arrive on this CTA's
+            // barrier, or on the same barrier of both CTAs
+            auto mma = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+                if (PAIR) umma_bf16_pair(d, a, b, id, acc);
+                else umma_bf16(d, a, b, id, acc);
+            };
+            auto commit = [&](uint64_t* b) {
+                if (PAIR) {
+                    umma_commit_pair(L(b));
+                    umma_commit_pair(P(b));
+                } else {
+                    umma_commit(b);
+                }
+            };
             int s = 0;
             uint32_t ph = 0;
             int lt = 0;
-            for (int t = blockIdx.x; t < ntile; t += gridDim.x, ++lt) {
+            for (int t = cid; t < ntile; t += ncid, ++lt) {
                 const int buf = lt & 1;
                 const uint32_t aph = (lt >> 1) & 1;
-                if (!wait_or_abort(&acc_empty[buf], aph ^ 1, abort_flag, 0x200)) break;
+                if (!wait(&acc_empty[buf], aph ^ 1, 0x200)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + buf * BN;
                 bool ok = true;
                 if (EPI == EPI_SUM) {
                     // Y = residual + inter-residual + sum_j gate_j expert_j: one N = 16 identity MMA per
                     // 16 columns and source (bf16 times one summed in fp32 is exact)
-                    constexpr uint32_t idescI = umma_idesc_bf16(128, 16);
+                    constexpr uint32_t idescI = umma_idesc_bf16(PAIR ? 256 : 128, 16);
                     const uint64_t idB = umma_sdesc_sw32(smem_u32(sI));
 #pragma unroll 1
                     for (int src = 0; src < n_src && ok; ++src) {
                         const bool mixed = src < p.src_resid + p.src_extra && p.src_mix;
 #pragma unroll 1
                         for (int sl = 0; sl < BN / 64; ++sl) {
-                            if (!wait_or_abort(&full[s], ph, abort_flag, 0x203)) { ok = false; break; }
+                            if (!wait(&full[s], ph, 0x203)) { ok = false; break; }
                             tc_fence_after();
                             const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
                                 const uint64_t a_k = mixed ? umma_sdesc_sw32(sa + kk * 4096) : umma_sdesc_sw128(sa) + 2 * kk;
-                                umma_bf16(d + sl * 64 + kk * 16, a_k, idB, idescI, src > 0 ? 1u : 0u);
+                                mma(d + sl * 64 + kk * 16, a_k, idB, idescI, src > 0 ? 1u : 0u);
                             }
-                            umma_commit(&empty[s]);
+                            commit(&empty[s]);
                             if (++s == STAGES) { s = 0; ph ^= 1; }
                         }
                     }
                     if (!ok) break;
                 }
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!wait_or_abort(&full[s], ph, abort_flag, 0x201)) { ok = false; break; }
+                    if (!wait(&full[s], ph, 0x201)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
                     const uint32_t sb = sa + C::A_BYTES;
@@ -368,16 +482,17 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
                         // A: one 32-byte-swizzled 4 KB sub-slab per K step (mixed rows) or the
                         // 128-byte-swizzled 64-wide slab advanced by 32 bytes per K step
                         const uint64_t a_k = AMODE == A_TMA_MIX ? umma_sdesc_sw32(sa + kk * 4096) : ad + 2 * kk;
-                        umma_bf16(d, a_k, bd + 2 * kk, idesc, (EPI == EPI_SUM && n_src > 0) || (kb | kk) != 0);
+                        mma(d, a_k, bd + 2 * kk, idesc, (EPI == EPI_SUM && n_src > 0) || (kb | kk) != 0);
                     }
-                    umma_commit(&empty[s]);
+                    commit(&empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1; }
                 }
                 if (!ok) break;
-                umma_commit(&acc_full[buf]);
+                commit(&acc_full[buf]);
             }
             // every MMA this thread issued must be complete before TMEM is released
-            umma_commit(drain);
+            if (PAIR) umma_commit_pair(L(drain));
+            else umma_commit(drain);
             wait_or_abort(drain, 0, abort_flag, 0x202);
         }
     } else if (warp >= 2 && warp < 2 + C::EPI_WARPS) {
@@ -434,21 +549,21 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
             }
             return m;
         };
-        TileInfo ti_n1 = decode_tile(p, blockIdx.x), ti_n2 = ti_n1;
+        TileInfo ti_n1 = dec(cid), ti_n2 = ti_n1;
         RowMeta rm_n1 = row_meta(ti_n1);
-        if ((int)blockIdx.x + (int)gridDim.x < ntile) ti_n2 = decode_tile(p, blockIdx.x + gridDim.x);
+        if (cid + ncid < ntile) ti_n2 = dec(cid + ncid);
         int lt = 0;
-        for (int t = blockIdx.x; t < ntile; t += gridDim.x, ++lt) {
+        for (int t = cid; t < ntile; t += ncid, ++lt) {
             const TileInfo ti = ti_n1;
             const RowMeta rm = rm_n1;
-            if (t + (int)gridDim.x < ntile) {
+            if (t + ncid < ntile) {
                 ti_n1 = ti_n2;
                 rm_n1 = row_meta(ti_n1);
-                if (t + 2 * (int)gridDim.x < ntile) ti_n2 = decode_tile(p, t + 2 * gridDim.x);
+                if (t + 2 * ncid < ntile) ti_n2 = dec(t + 2 * ncid);
             }
             const int buf = lt & 1;
             const uint32_t aph = (lt >> 1) & 1;
-            if (!wait_or_abort(&acc_full[buf], aph, abort_flag, 0x300)) break;
+            if (!wait(&acc_full[buf], aph, 0x300)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + buf * BN;
             bool valid = r < ti.nrows;
@@ -741,7 +856,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (lane == 0) {
+                if (PAIR) mbar_arrive_cluster(L(&acc_empty[buf]));     // the leader issues the next MMAs
+                else mbar_arrive(&acc_empty[buf]);
+            }
         }
         if (C::STAGED && lane == 0) bulk_wait_all();                  // stores complete before exit
         __syncwarp();
@@ -753,7 +871,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
         const int r = q * 32 + lane;
         int s = 0, lt = 0;
         uint32_t ph = 0;
-        for (int t = blockIdx.x; t < ntile; t += gridDim.x, ++lt) {
+        for (int t = cid; t < ntile; t += ncid, ++lt) {
             const int buf = lt & 1;
             float ss = 0.f;
             bool ok = true;
@@ -796,8 +914,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
         const int rsub = gt >> 3;
         int s = 0, pend_s = -1;
         uint32_t ph = 0;
-        for (int t = blockIdx.x; t < ntile; t += gridDim.x) {
-            const TileInfo ti = decode_tile(p, t);
+        for (int t = cid; t < ntile; t += ncid) {
+            const TileInfo ti = dec(t);
             int rb[8];
             int bank = p.sched == 0 ? ti.g : ti.g / p.E;
 #pragma unroll
@@ -840,10 +958,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI>::NTHREADS, 1)
     }
 
     tc_fence_before();
-    __syncthreads();
+    // pair mode: neither CTA releases its tensor memory or exits while the other may still arrive
+    // on its barriers or be the target of the pair's MMAs
+    if (PAIR) cluster_sync_all();
+    else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
+        if (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+        else tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
 }
 

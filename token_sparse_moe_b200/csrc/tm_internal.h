@@ -31,13 +31,15 @@ void note_cuda_error(const char* where, cudaError_t e);   // samples per router 
 // s2 the sample-order expert rows [B, banks, k, W]
 // tmO: the output map, required by EPI_SWIGLU (the hidden rows, 64-column x 32-row boxes) and
 // EPI_SUM (y in its row geometry: 3-D rows or the 4-D Revert map, 32-row boxes)
+// pair: CTA pairs (clusters of two, M = 256 per tile, grid even, weight maps with BN/2-row boxes;
+// groups of equal rows, sched 0)
 cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                                     const CUtensorMap& tmB1, const CUtensorMap& tmS0, const CUtensorMap& tmS1,
                                     const CUtensorMap& tmS2, const GemmParams& p, int grid, cudaStream_t st,
-                                    const CUtensorMap* tmO = nullptr);
+                                    const CUtensorMap* tmO = nullptr, bool pair = false);
 cudaError_t launch_grouped_gemm(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                                 const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st,
-                                const CUtensorMap* tmO = nullptr);
+                                const CUtensorMap* tmO = nullptr, bool pair = false);
 
 // ---- fused dense sub-layer (row width 128 / 256) --------------------------------
 bool fused_supported(int W, int a_mode);
