@@ -210,6 +210,16 @@ TM_API tm_status tm_sparse_pertoken_moe(const void *x, const void *residual, tm_
                                  const void *norm_gain, const tm_moe_w *w, void *y,
                                  void *workspace, size_t workspace_bytes, void *stream);
 
+/* One sub-layer of either kind (sub->is_moe: Sparse-Pertoken MoE, else per-token SwiGLU) with two
+ * residual terms: y_row = FFN_bank(RMSNorm(x_row) * gain) + residual_row + extra_row, both terms
+ * added in the output epilogue before y's single rounding (residual / extra NULL: none).  extra is
+ * the inter-residual of [digest] 2.3.4 when a stack runs sub-layer by sub-layer, e.g. with its
+ * banks sharded over GPUs (Token Parallel, [digest] 2.5.3).  x, residual, extra and y share `layout`;
+ * y must not alias x or extra.  Workspace: tm_sublayer_workspace_bytes. */
+TM_API tm_status tm_sublayer_forward(const void *x, const void *residual, const void *extra, tm_layout layout,
+                                     const tm_shape *shape, const tm_sublayer *sub, void *y, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
 /* One TokenMixer-Large block ([readme] block diagram; [digest] Eq. 9-16, pre-norm reading):
  *   H = Mix(X); H_next = FFN_mix(Norm(H)) + H; X_rev = Revert(H_next);
  *   Y = FFN_rev(Norm(X_rev)) + X.

@@ -1,0 +1,39 @@
+"""Token Parallel on one GPU: P ranks' shards run in one process on the library's kernels (the
+all-to-all becomes a transpose of the ranks' chunks).  Each rank computes its heads' mixing rows
+and its tokens' reverting rows with tm_sublayer_forward; reassembled, the result must be the same
+bits as tm_stack_forward over the whole model, since every row is computed by the same kernels on
+the same data."""
+import pytest
+import torch
+
+import tm_synth as S
+from tm_synth import FFNSpec
+from token_sparse_moe_b200 import api
+from token_sparse_moe_b200 import token_parallel as TP
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+CASES = [
+    S.Config("tp_moe", B=300, T=16, D=256, H=16, L=3, gap=2, dtype="bf16",
+             mix=FFNSpec("moe", E=8, k=2, hidden_e=128, hidden_s=128, alpha=4.0),
+             rev=FFNSpec("moe", E=8, k=2, hidden_e=128, hidden_s=128, alpha=4.0)),
+    S.Config("tp_dense", B=200, T=16, D=256, H=16, L=2, gap=1, dtype="bf16",
+             mix=FFNSpec("dense", hidden=256), rev=FFNSpec("dense", hidden=384)),
+]
+
+
+@pytest.mark.parametrize("P", [2, 4])
+@pytest.mark.parametrize("cfg", CASES, ids=lambda c: c.name)
+def test_token_parallel_shards_reproduce_the_stack(cfg, P):
+    blocks = api.blocks_from_synth(cfg, DEV)
+    sh = api.config_shape(cfg)
+    X = api.to_device(S.make_x(cfg), DEV)
+    Y = api.stack_forward(X, blocks, cfg.gap, sh)
+    plan = TP.ShardPlan(cfg.T, cfg.D, cfg.H, P)
+    stages = [TP.RankStage(blocks, plan, p, sh, DEV) for p in range(P)]
+    xs = [X[:, slice(*plan.tokens(p))].contiguous() for p in range(P)]
+    ys = TP.forward_all_ranks(stages, plan, xs, cfg.L, cfg.gap)
+    api.get_device_error()
+    Yp = torch.cat(ys, dim=1)
+    assert torch.equal(Yp.view(torch.int16), Y.view(torch.int16))

@@ -16,6 +16,7 @@ TM_LAYOUT_ROWS, TM_LAYOUT_MIXED = 0, 1
 EXPORTS = ["tm_status_string", "tm_version", "tm_sublayer_workspace_bytes", "tm_route_workspace_bytes",
            "tm_workspace_bytes", "tm_tokenize_stub", "tm_mix", "tm_revert", "tm_route_topk", "tm_route_topk_noalloc",
            "tm_pertoken_swiglu", "tm_sparse_pertoken_moe", "tm_block_forward", "tm_stack_step", "tm_stack_forward",
+           "tm_sublayer_forward",
            "tm_profile_start", "tm_profile_stop", "tm_last_cuda_error", "tm_launch_count",
            "tm_get_device_error", "tm_quantize_fp8_weights", "tm_quantize_fp8_act",
            "tm_pertoken_swiglu_fp8_workspace_bytes", "tm_pertoken_swiglu_fp8", "tm_block_fp8_workspace_bytes",
@@ -89,6 +90,7 @@ _SIGS = {
     "tm_sparse_pertoken_moe": (c_int, [_P, _P, c_int, POINTER(tm_shape), _P, POINTER(tm_moe_w), _P, _P, c_size_t, _P]),
     "tm_block_forward": (c_int, [_P, POINTER(tm_block), POINTER(tm_shape), _P, _P, _P, c_size_t, _P]),
     "tm_stack_step": (c_int, [_P, _P, POINTER(tm_block), POINTER(tm_shape), _P, _P, _P, c_size_t, _P]),
+    "tm_sublayer_forward": (c_int, [_P, _P, _P, c_int, POINTER(tm_shape), POINTER(tm_sublayer), _P, _P, c_size_t, _P]),
     "tm_stack_forward": (c_int, [_P, POINTER(tm_block), c_int, c_int, POINTER(tm_shape), _P, _P, c_size_t, _P]),
     "tm_profile_start": (c_int, []),
     "tm_profile_stop": (c_int, [POINTER(tm_kernel_time), c_int, POINTER(c_int)]),

@@ -229,6 +229,26 @@ def sparse_pertoken_moe(x, residual, layout: int, sh: A.tm_shape, sub: SubLayer,
     return y
 
 
+def sublayer_forward(x, residual, extra, layout: int, sh: A.tm_shape, sub: SubLayer, y=None, workspace=None,
+                     stream=None):
+    """tm_sublayer_forward: y = FFN(Norm(x)) + residual + extra for a dense or MoE sub-layer."""
+    y = _out_like(x, layout, sh, sub) if y is None else y
+    ws = _ws(sublayer_workspace_bytes(sh, layout, sub), x.device, workspace)
+    c = sub.c()
+    A.check(lib().tm_sublayer_forward(_p(x), _p(residual), _p(extra), layout, ctypes.byref(sh), ctypes.byref(c), _p(y),
+                                      _p(ws), ws.numel(), _s(stream)), "tm_sublayer_forward")
+    return y
+
+
+def slice_banks(sub: SubLayer, lo: int, hi: int) -> SubLayer:
+    """Banks lo .. hi-1 of a sub-layer (views of its weight tensors, whose leading axis is the bank)."""
+    if not (0 <= lo < hi <= sub.banks):
+        raise ValueError(f"bank range [{lo}, {hi}) outside [0, {sub.banks})")
+    t = {k: v.narrow(0, lo, hi - lo) for k, v in sub.tensors.items()}
+    return SubLayer(sub.is_moe, hi - lo, sub.width, t, hidden=sub.hidden, E=sub.E, k=sub.k, hidden_e=sub.hidden_e,
+                    hidden_s=sub.hidden_s, alpha=sub.alpha, gain=sub.gain)
+
+
 def workspace_bytes(sh: A.tm_shape, blocks: Sequence[Block], gap: int = 0) -> int:
     arr = (A.tm_block * len(blocks))(*[b.c() for b in blocks])
     n = lib().tm_workspace_bytes(ctypes.byref(sh), arr, len(blocks), gap)

@@ -589,7 +589,9 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
     } else {
         // MoEPermute: copy the routed rows into bucket order (the slot buffer, [routed, W], is free
         // until the routed GEMM2 writes it), then GEMM1 reads A as contiguous rows through a 2-D
-        // tensor map.
+        // tensor map.  (Gathering the rows inside GEMM1 instead, by tile::gather4 TMA loads of
+        // one-row boxes, measured 2.2x slower for GEMM1 than this copy plus one 16 KB box per K slab:
+        // every N tile gathers its A rows again, 32 four-row operations per slab.)
         const int bn = pick_bn_swiglu(Fe);
         p.n_tiles = p.N / bn;
         CUtensorMap ma, mg, mu, mo;
@@ -623,10 +625,13 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
         p.perm = m.perm;
         p.gate = m.gate;
         p.pos_scale = m.gate_pos;
-        CUtensorMap ma, mb;
-        if (!map_2d(&ma, m.hidden_r, routed, Fe, 128) || !map_2d(&mb, w->we_down, G * g.W, Fe, bn)) return TM_ERR_CUDA;
+        // the expert rows leave through scatter stores of one-row boxes into the slot rows
+        CUtensorMap ma, mb, mo;
+        if (!map_2d(&ma, m.hidden_r, routed, Fe, 128) || !map_2d(&mb, w->we_down, G * g.W, Fe, bn) ||
+            !map_2d(&mo, m.slots, routed, g.W, 1))
+            return TM_ERR_CUDA;
         const long grid = max_mt * p.n_tiles < num_sms() ? max_mt * p.n_tiles : num_sms();
-        if ((s = cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SLOT_PERM, ma, mb, mb, p, (int)grid, st))) != TM_OK)
+        if ((s = cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SLOT_PERM, ma, mb, mb, p, (int)grid, st, &mo))) != TM_OK)
             return s;
         return combine_sum(g, m.hidden_s, w->ws_down, w->hidden_s, resid, extra, y, m.slots, w->k, st);
     }
@@ -1243,6 +1248,17 @@ tm_status tm_sparse_pertoken_moe(const void* x, const void* residual, tm_layout 
     if (s != TM_OK) return s;
     if (!x || !y || !al16(x) || !al16(y) || x == y || (residual && !al16(residual))) return TM_ERR_INVALID_ARG;
     return run_sublayer(g, x, residual, nullptr, &sub, y, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+tm_status tm_sublayer_forward(const void* x, const void* residual, const void* extra, tm_layout layout,
+                              const tm_shape* shape, const tm_sublayer* sub, void* y, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    Geo g;
+    tm_status s = check_sublayer(shape, layout, sub, &g);
+    if (s != TM_OK) return s;
+    if (!x || !y || !al16(x) || !al16(y) || x == y || (residual && !al16(residual))) return TM_ERR_INVALID_ARG;
+    if (extra && (!al16(extra) || extra == y)) return TM_ERR_INVALID_ARG;
+    return run_sublayer(g, x, residual, extra, sub, y, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 tm_status tm_block_forward(const void* X, const tm_block* block, const tm_shape* shape, void* Y, void* X_revert_opt,

@@ -128,6 +128,16 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* m, const void* s
                  "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
                  : "memory");
 }
+// Four rows of a staged box (4 x the box bytes at src, one after another) to rows r0..r3 of a 2-D
+// tensor map whose box is one row high (tile::scatter4), from column c0.  Bulk-group completion.
+__device__ __forceinline__ void tma_scatter4(const CUtensorMap* m, const void* src, int c0, int r0, int r1, int r2,
+                                             int r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.tile::scatter4.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(m)),
+        "r"(smem_u32(src)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // this thread's bulk stores have finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

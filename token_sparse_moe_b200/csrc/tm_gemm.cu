@@ -161,8 +161,9 @@ cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorM
                                     const CUtensorMap& tmB1, const CUtensorMap& tmS0, const CUtensorMap& tmS1,
                                     const CUtensorMap& tmS2, const GemmParams& p, int grid, cudaStream_t st,
                                     const CUtensorMap* tmO, bool pair) {
-    // the SwiGLU, combine and plain-row epilogues store through the output map
-    if ((epi == EPI_SWIGLU || epi == EPI_SUM || epi == EPI_SLOT) && !tmO) return cudaErrorInvalidValue;
+    // the SwiGLU, combine, plain-row and expert-row epilogues store through the output map
+    if ((epi == EPI_SWIGLU || epi == EPI_SUM || epi == EPI_SLOT || epi == EPI_SLOT_PERM) && !tmO)
+        return cudaErrorInvalidValue;
     CUtensorMap none;
     memset(&none, 0, sizeof(none));
     const CUtensorMap& o = tmO ? *tmO : none;

@@ -593,22 +593,23 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
                 tmem_ld32(taddr, vh);
                 tmem_ld32(taddr + E, vm);
                 tmem_ld32(taddr + 2 * E, vl);
-                // logit e = (hi + mid) + lo, scaled by 1/rms; softmax; top-k with ties to the lower index
+                // logit e = (hi + mid) + lo, scaled by 1/rms; softmax; top-k with ties to the lower index.
+                // The loops are unrolled for register-resident arrays and leave at E (uniform across the
+                // warp), so only E experts' instructions issue.
                 float z[kRouteMaxE];
                 float zmax = -INFINITY;
 #pragma unroll
                 for (int e = 0; e < kRouteMaxE; ++e) {
-                    z[e] = -INFINITY;
-                    if (e < E) {
-                        z[e] = ((vh[e] + vm[e]) + vl[e]) * irs;
-                        zmax = fmaxf(zmax, z[e]);
-                    }
+                    if (e >= E) break;
+                    z[e] = ((vh[e] + vm[e]) + vl[e]) * irs;
+                    zmax = fmaxf(zmax, z[e]);
                 }
                 float pe[kRouteMaxE];
                 float sum = 0.f;
 #pragma unroll
                 for (int e = 0; e < kRouteMaxE; ++e) {
-                    pe[e] = e < E ? expf(z[e] - zmax) : 0.f;
+                    if (e >= E) break;
+                    pe[e] = expf(z[e] - zmax);
                     sum += pe[e];
                 }
                 const size_t rowi = (size_t)b * p.banks + bank;
@@ -617,19 +618,17 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
 #pragma unroll 1
                 for (int j = 0; j < p.k; ++j) {
                     int be = -1;
-                    float bz = -INFINITY;
+                    float bz = -INFINITY, bp = 0.f;
 #pragma unroll
-                    for (int e = 0; e < kRouteMaxE; ++e)
-                        if (e < E && !((chosen >> e) & 1u) && (be < 0 || z[e] > bz)) { bz = z[e]; be = e; }
+                    for (int e = 0; e < kRouteMaxE; ++e) {
+                        if (e >= E) break;
+                        if (!((chosen >> e) & 1u) && (be < 0 || z[e] > bz)) { bz = z[e]; be = e; bp = pe[e]; }
+                    }
                     chosen |= 1u << be;
                     zk = bz;
-                    float pb = 0.f;
-#pragma unroll
-                    for (int e = 0; e < kRouteMaxE; ++e)
-                        if (e == be) pb = pe[e] / sum;
                     if (valid) {
                         p.r_idx[rowi * p.k + j] = be;
-                        p.r_gate[rowi * p.k + j] = p.r_alpha * pb;
+                        p.r_gate[rowi * p.k + j] = p.r_alpha * (bp / sum);
                     }
                 }
                 if (valid && p.r_inv_rms) p.r_inv_rms[rowi] = irs;
@@ -637,8 +636,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
                     // distance of the k-th choice to the best expert left out (none left: +inf)
                     float zn = -INFINITY;
 #pragma unroll
-                    for (int e = 0; e < kRouteMaxE; ++e)
-                        if (e < E && !((chosen >> e) & 1u)) zn = fmaxf(zn, z[e]);
+                    for (int e = 0; e < kRouteMaxE; ++e) {
+                        if (e >= E) break;
+                        if (!((chosen >> e) & 1u)) zn = fmaxf(zn, z[e]);
+                    }
                     p.r_gap[rowi] = zk - zn;
                 }
                 // per 128-row chunk: rows of this bank that chose expert e
@@ -682,7 +683,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
                 }
             } else if (EPI == EPI_SLOT_PERM) {
                 // the row of choice j of sample b (bank of the group), scaled by its gate: rows are
-                // scattered, so each 64-column chunk is staged and written four whole rows at a time
+                // scattered, so each 64-column chunk is staged, then written by eight tile::scatter4 bulk
+                // stores of four rows each (lanes 0-7: rows 4l .. 4l+3 of the warp's 32) when all 32 rows
+                // are valid, else four whole rows per store instruction of the warp
                 const int e = valid ? rm.e : 0;
                 if (valid && (e < 0 || e >= p.pos_limit)) {
                     record_error(ERR_BOUNDS, 0x314);
@@ -690,6 +693,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
                 }
                 const float gsc = valid ? (by_pos ? rm.s : __ldg(&p.gate[e])) : 0.f;
                 const long long my_off = valid ? (long long)e * p.out_ld + ti.n * BN : -1ll;
+                const bool whole = __all_sync(0xffffffffu, valid);
+                int e4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) e4[i] = __shfl_sync(0xffffffffu, e, (4 * lane + i) & 31);
 #pragma unroll 1
                 for (int c = c_lo; c < c_hi; c += 64) {
                     uint32_t pk[32];
@@ -700,8 +707,22 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
 #pragma unroll
                         for (int i = 0; i < 16; ++i) pk[16 * h + i] = pack_bf16x2(gsc * v[2 * i], gsc * v[2 * i + 1]);
                     }
-                    stage_row(pk);
-                    copy_rows(my_off, c);
+                    if (lane < 8) bulk_wait_read_all();   // this lane's previous scatter stores have read the box
+                    __syncwarp();
+#pragma unroll
+                    for (int c8 = 0; c8 < 8; ++c8)
+                        *reinterpret_cast<uint4*>(stg + lane * 128 + ((c8 ^ (lane & 7)) << 4)) =
+                            make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+                    if (whole) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane < 8) {
+                            tma_scatter4(&tmO, stg + lane * 512, ti.n * BN + c, e4[0], e4[1], e4[2], e4[3]);
+                            bulk_commit_group();
+                        }
+                    } else {
+                        copy_rows(my_off, c);
+                    }
                 }
             } else if (EPI == EPI_SUM) {
                 // Y already holds every term: bf16 through the output's row or Revert geometry, one
@@ -861,7 +882,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
                 else mbar_arrive(&acc_empty[buf]);
             }
         }
-        if (C::STAGED && lane == 0) bulk_wait_all();                  // stores complete before exit
+        if (C::STAGED && lane < 8) bulk_wait_all();                   // stores complete before exit
         __syncwarp();
     } else if (EPI == EPI_ROUTE) {
         // ---------------------------------------------------------------- row statistics (warps 6-9)
