@@ -36,7 +36,7 @@ from typing import Callable, Dict, Optional, Tuple
 
 import numpy as np
 
-from .tokenmixer import mix, revert, round_bf16, silu, storage_round
+from .tokenmixer import mix, revert, rmsnorm, round_bf16, route, silu, storage_round
 
 E4M3_MAX = 448.0
 
@@ -146,6 +146,67 @@ def sublayer_fp8(rows: np.ndarray, qbank: Callable[[int], Dict[str, np.ndarray]]
     for j in range(rows.shape[1]):
         out[:, j, :] = swiglu_fp8(rows[:, j, :], qbank(j), eps)
     return out
+
+
+# ------------------------------------------------------------------ Sparse-Pertoken MoE on the FP8 path
+def quantize_moe_bank(bw: Dict[str, np.ndarray], gain: Optional[np.ndarray] = None) -> Dict[str, object]:
+    """E4M3 gate / up weights of one MoE bank: one scale per routed expert's matrix and per shared
+    matrix (the gain folded in first, as the bf16 path stores them); the fp32 router and the bf16
+    down projections kept."""
+    E = bw["we_gate"].shape[0]
+    q = {"w_router": bw["w_router"],
+         "experts": [quantize_bank({"w_gate": bw["we_gate"][e], "w_up": bw["we_up"][e], "w_down": bw["we_down"][e]},
+                                   gain) for e in range(E)]}
+    if "ws_gate" in bw:
+        q["shared"] = quantize_bank({"w_gate": bw["ws_gate"], "w_up": bw["ws_up"], "w_down": bw["ws_down"]}, gain)
+    return q
+
+
+def sp_moe_fp8(rows: np.ndarray, qb: Dict[str, object], k: int, alpha: float, eps: float,
+               gain: Optional[np.ndarray] = None, forced_idx: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+    """Sparse-Pertoken MoE of one bank ([digest] 2.4, Eq. 19-21) with every expert's GEMM1 on the FP8
+    path ([digest] 2.5.2): rows [R, W] (the sub-layer's rows, before the RMSNorm) -> [R, W].
+
+    The routing is the bf16 path's (RMSNorm with the gain, fp32 router, softmax, top-k, gates
+    alpha * p): quantization changes the experts, not which of them a row uses.  Each chosen expert
+    and the shared expert run swiglu_fp8 on the row (per-row E4M3 activations, per-matrix E4M3
+    weights, 1/rms of the unquantized row), combined as alpha * sum p_e * Expert_e + Shared.
+    forced_idx [R, k]: the experts of each row, as in the bf16 oracle's teacher forcing."""
+    n = rmsnorm(rows, eps, gain)
+    r = route(n, qb["w_router"], k)
+    if forced_idx is not None:
+        forced_idx = np.asarray(forced_idx)
+        assert forced_idx.shape == r["idx"].shape
+        assert all(len(set(row)) == k for row in forced_idx.tolist()), "forced experts repeat within a row"
+        r["idx"] = forced_idx
+    idx = r["idx"]
+    out = np.zeros_like(rows)
+    for e in range(r["p"].shape[1]):
+        sel = np.nonzero(np.any(idx == e, axis=1))[0]
+        if sel.size:
+            out[sel] += alpha * r["p"][sel, e][:, None] * swiglu_fp8(rows[sel], qb["experts"][e], eps)
+    if "shared" in qb:
+        out += swiglu_fp8(rows, qb["shared"], eps)
+    r["out"] = out
+    return r
+
+
+def sublayer_moe_fp8(rows: np.ndarray, qbank: Callable[[int], Dict[str, object]], spec, eps: float,
+                     gain: Optional[np.ndarray] = None, forced_idx: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+    """rows [R, banks, W] -> {"out": FFN output [R, banks, W] (no residual), routing per bank}."""
+    R, banks, W = rows.shape
+    out = np.empty_like(rows)
+    info = {"idx": [], "p": [], "logits": [], "gap": []}
+    for j in range(banks):
+        r = sp_moe_fp8(rows[:, j, :], qbank(j), spec.k, spec.alpha, eps, gain,
+                       None if forced_idx is None else forced_idx[:, j, :])
+        out[:, j, :] = r["out"]
+        for key in info:
+            info[key].append(r[key])
+    res = {"out": out}
+    for key in info:
+        res[key] = np.stack(info[key], axis=1)
+    return res
 
 
 def block_forward_fp8(X: np.ndarray, cfg, qbank: Callable[[int, int], Dict[str, np.ndarray]],

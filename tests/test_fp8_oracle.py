@@ -126,3 +126,67 @@ def test_matrix_scale_is_the_matrix_maximum():
     assert np.all(np.abs(q * np.float64(s) - w)[big] <= 2.0 ** -4 * np.abs(w)[big] * (1 + 1e-6))
     assert np.array_equal(F.quantize_matrix(np.zeros((3, 4)))[0], np.zeros((3, 4), np.uint8))
     assert F.quantize_matrix(np.zeros((3, 4)))[1] == 1.0
+
+
+def _grid(rng, n, k, scale_pow):
+    """[n, k] values on the E4M3 grid, each row's largest magnitude exactly 448 * 2^scale_pow."""
+    c = rng.integers(0, 0x7E, (n, k)).astype(np.uint8) | (rng.integers(0, 2, (n, k)).astype(np.uint8) << 7)
+    c[:, 0] = 0x7E
+    return F.e4m3_decode(c) * 2.0 ** scale_pow
+
+
+def _moe_bank(rng, W, E, Fe, Fs, on_grid):
+    if on_grid:
+        gu = lambda n: _grid(rng, n, W, -12)
+    else:
+        gu = lambda n: O.round_bf16(rng.standard_normal((n, W)) / np.sqrt(W))
+    return {"w_router": rng.standard_normal((E, W)) / np.sqrt(W),
+            "we_gate": np.stack([gu(Fe) for _ in range(E)]), "we_up": np.stack([gu(Fe) for _ in range(E)]),
+            "we_down": O.round_bf16(rng.standard_normal((E, W, Fe)) * 0.05),
+            "ws_gate": gu(Fs), "ws_up": gu(Fs), "ws_down": O.round_bf16(rng.standard_normal((W, Fs)) * 0.05)}
+
+
+def test_fp8_moe_equals_bf16_moe_when_quantization_is_exact():
+    # on-grid rows and expert weights: every expert's GEMM1 is exact, so the FP8 MoE is the bf16
+    # oracle's MoE (same routing, same gates alpha * p, same shared expert) up to float64 rounding
+    rng = np.random.default_rng(11)
+    W, E, k, Fe, Fs, R = 64, 6, 2, 32, 48, 40
+    bw = _moe_bank(rng, W, E, Fe, Fs, on_grid=True)
+    x = _grid(rng, R, W, -6)
+    qb = F.quantize_moe_bank(bw)
+    assert [q["s_gate"] for q in qb["experts"]] == [np.float32(2.0 ** -12)] * E
+    got = F.sp_moe_fp8(x, qb, k, 3.0, 1e-6)
+    want = O.sp_moe(O.rmsnorm(x, 1e-6), bw, k, 3.0)
+    assert np.array_equal(got["idx"], want["idx"])
+    assert np.allclose(got["out"], want["out"], rtol=1e-12, atol=1e-12 * np.abs(want["out"]).max())
+    # a dropped expert scale (a plausible mistake) shows
+    bad = dict(qb)
+    bad["experts"] = [dict(q, s_gate=np.float32(1.0)) for q in qb["experts"]]
+    assert not np.allclose(F.sp_moe_fp8(x, bad, k, 3.0, 1e-6)["out"], want["out"], rtol=1e-3)
+
+
+def test_fp8_moe_with_k_equal_E_is_the_dense_softmax_sum_of_fp8_experts():
+    rng = np.random.default_rng(12)
+    W, E, Fe, Fs, R = 32, 4, 16, 16, 20
+    bw = _moe_bank(rng, W, E, Fe, Fs, on_grid=False)
+    x = O.round_bf16(rng.standard_normal((R, W)))
+    qb = F.quantize_moe_bank(bw)
+    got = F.sp_moe_fp8(x, qb, E, 1.0, 1e-6)["out"]
+    p = O.softmax(O.rmsnorm(x, 1e-6) @ bw["w_router"].T)
+    want = sum(p[:, e:e + 1] * F.swiglu_fp8(x, qb["experts"][e], 1e-6) for e in range(E)) + F.swiglu_fp8(x, qb["shared"], 1e-6)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-13)
+
+
+def test_fp8_moe_tracks_bf16_moe_and_forcing_works():
+    rng = np.random.default_rng(13)
+    W, E, k, Fe, Fs, R = 64, 8, 2, 32, 32, 64
+    bw = _moe_bank(rng, W, E, Fe, Fs, on_grid=False)
+    x = O.round_bf16(rng.standard_normal((R, W)))
+    qb = F.quantize_moe_bank(bw)
+    got = F.sp_moe_fp8(x, qb, k, 4.0, 1e-6)
+    want = O.sp_moe(O.rmsnorm(x, 1e-6), bw, k, 4.0)
+    assert np.array_equal(got["idx"], want["idx"])              # quantization leaves the routing alone
+    rel = np.sqrt(np.mean((got["out"] - want["out"]) ** 2) / np.mean(want["out"] ** 2))
+    assert 1e-3 < rel < 0.08, rel
+    forced = got["idx"][:, ::-1].copy()                       # the same sets, other order: same output
+    assert np.allclose(F.sp_moe_fp8(x, qb, k, 4.0, 1e-6, forced_idx=forced)["out"], got["out"], rtol=1e-12, atol=1e-15)
