@@ -99,12 +99,23 @@ def kernel_flops(cfg, B) -> dict:
 
 
 def kernel_flops_fp8(cfg, B) -> dict:
-    """The FP8 path: both sub-layers of every block run the fused kernel in its FP8 mode."""
-    f = 0.0
+    """The FP8 path: dense sub-layers run the fused kernel in its FP8 mode; MoE sub-layers run every
+    expert's GEMM1 (routed and shared) as the E4M3 grouped GEMM and the rest as on the bf16 path."""
+    out = {}
+
+    def add(k, v):
+        out[k] = out.get(k, 0.0) + v
     for _ in range(cfg.L):
         for sub in (0, 1):
-            f += B * cfg.banks(sub) * 6.0 * cfg.width(sub) * cfg.ffn(sub).hidden
-    return {"fused_swiglu_fp8": f}
+            s, W, banks = cfg.ffn(sub), cfg.width(sub), cfg.banks(sub)
+            if s.is_moe:
+                add("gemm_swiglu_fp8", B * banks * 4.0 * W * (s.k * s.hidden_e + s.hidden_s))
+                add("gemm_slot", B * banks * s.k * 2.0 * W * s.hidden_e)
+                add("gemm_combine", B * banks * 2.0 * W * s.hidden_s)
+                add("router", B * banks * 2.0 * W * s.E)
+            else:
+                add("fused_swiglu_fp8", B * banks * 6.0 * W * s.hidden)
+    return out
 
 
 def backward_flops_per_sample(cfg) -> float:
@@ -135,6 +146,21 @@ def fp8_effective_peak(bf16_peak: float) -> float:
     taken as the measured bf16 peak x 2 (the nominal 4.5 / 2.25 PFLOP/s ratio), GEMM2 (2 W F) at
     the bf16 rate: 6 / (4 / 2P + 2 / P) = 1.5 P."""
     return 6.0 / (4.0 / (2.0 * bf16_peak) + 2.0 / bf16_peak)
+
+
+def kernel_peak_factor(kernel: str) -> float:
+    """The kernel's tensor peak in units of the measured bf16 peak: the fused FP8 sub-layer 1.5
+    (fp8_effective_peak), the E4M3 grouped GEMM1 2 (all of its flops at the E4M3 rate), bf16 kernels 1."""
+    return {"fused_swiglu_fp8": 1.5, "gemm_swiglu_fp8": 2.0}.get(kernel, 1.0)
+
+
+def step_peak_factor(cfg, fp8: bool) -> float:
+    """The whole step's tensor peak in units of the bf16 peak: its flops over the time they take at
+    each kernel's own peak."""
+    if not fp8:
+        return 1.0
+    kf = kernel_flops_fp8(cfg, 1)
+    return sum(kf.values()) / sum(v / kernel_peak_factor(k) for k, v in kf.items())
 
 
 def peaks():
@@ -307,10 +333,13 @@ def time_oracle(cfg, budget_s: float, max_samples: int):
 
 
 def time_oracle_fp8(cfg, budget_s: float, max_samples: int):
-    """The FP8 oracle's samples/s on the host cores (weights quantized beforehand, as served)."""
+    """The FP8 oracle's samples/s on the host cores (weights quantized beforehand, as served).  MoE
+    workloads: the FP8 MoE sub-layer on the first banks of block 1, scaled as oracle_probe scales."""
     import oracle
     from oracle import fp8 as F
     from threadpoolctl import threadpool_info
+    if any(cfg.ffn(s).is_moe for s in (0, 1)):
+        return time_oracle_fp8_moe(cfg, budget_s, max_samples)
     get = oracle.synth_banks(cfg)
     q = {(l, sub, j): F.quantize_bank(get(l, sub, j)) for l in range(cfg.L) for sub in (0, 1)
          for j in range(cfg.banks(sub))}
@@ -394,6 +423,31 @@ def job_throughput(samples_per_rank: int, world: int, step_ms: float) -> float:
     return samples_per_rank * world / (step_ms / 1e3)
 
 
+def time_oracle_fp8_moe(cfg, budget_s: float, max_samples: int, max_banks: int = 2):
+    import oracle
+    from oracle import fp8 as F
+    from oracle import tokenmixer as O
+    n = min(max_samples, cfg.B)
+    nb = min(max_banks, cfg.H, cfg.T)
+    get = oracle.synth_banks(cfg)
+    q = {(s, j): F.quantize_moe_bank(get(0, s, j)) for s in (0, 1) for j in range(nb)}
+    X = S.to_f64(S.make_x(cfg, np.arange(n)))
+    rows = {0: O.mix(X, cfg.H)[:, :nb], 1: X[:, :nb]}
+    done, equiv, t0 = 0, 0.0, time.perf_counter()
+    while True:
+        for s, banks in ((0, cfg.H), (1, cfg.T)):
+            t1 = time.perf_counter()
+            F.sublayer_moe_fp8(rows[s], lambda j: q[(s, j)], cfg.ffn(s), cfg.eps)
+            equiv += cfg.L * (time.perf_counter() - t1) * banks / nb
+        done += n
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done / equiv, {"cores": oracle_threads(), "samples": done, "seconds": dt, "per_call": n,
+                          "desc": f"oracle fp8.sublayer_moe_fp8 on samples 0..{n - 1} x banks 0..{nb - 1} of both "
+                                  f"sub-layers of block 1, scaled to all {cfg.H}+{cfg.T} banks and {cfg.L} blocks"}
+
+
 def rank_config(cfg, rank: int):
     """Each rank draws its own input batch (seed offset by the rank); weights are shared."""
     return cfg.with_(seed=cfg.seed + rank)
@@ -411,14 +465,21 @@ def run_ours(args, cfg, rank, world, local_rank):
     blocks = api.blocks_from_synth(cfg, dev, workers=min(16, os.cpu_count() or 1))
     sh = api.config_shape(cfg)
     dY = None
-    if args.fp8 or args.backward:
-        if cfg.gap or cfg.dtype != "bf16" or any(cfg.ffn(sub).is_moe for sub in (0, 1)):
-            raise SystemExit("--fp8 and --backward cover bf16 dense blocks without the inter-residual")
+    moe = any(cfg.ffn(sub).is_moe for sub in (0, 1))
+    if args.backward and (cfg.gap or cfg.dtype != "bf16" or moe):
+        raise SystemExit("--backward covers bf16 dense blocks without the inter-residual")
+    if args.fp8 and cfg.dtype != "bf16":
+        raise SystemExit("--fp8 covers bf16 workloads")
     if args.backward:
         if cfg.L != 1:
             raise SystemExit("--backward times one dense block")
         dY = api.to_device(S.make_x(rank_config(cfg, rank).with_(seed=cfg.seed + rank + 17)), dev)
         run = api.BlockBackwardRunner(blocks[0], sh, dY, dev)
+    elif args.fp8 and (moe or cfg.gap):
+        run = api.Fp8StackRunner([(api.sublayer8_from_bf16(b.mix), api.sublayer8_from_bf16(b.rev)) for b in blocks],
+                                 sh, cfg.gap, dev)
+        del blocks
+        torch.cuda.empty_cache()
     elif args.fp8:
         run = api.Fp8BlockRunner([api.Block8.from_bf16(b) for b in blocks], sh, dev)
     else:
@@ -523,14 +584,16 @@ def run_ours(args, cfg, rank, world, local_rank):
         key = "bf16_tflops_sustained" if long_step else "bf16_tflops"
         src = (f"measured bf16 {'sustained' if long_step else 'burst'} (MEASURED_PEAKS.json {key})"
                if pk_src == "measured" else f"fallback {'1.40' if long_step else '1.59'} PFLOP/s")
-        peak = pk[key]
-        if args.fp8:
-            peak = fp8_effective_peak(pk["bf16_tflops"])
+        fac = kernel_peak_factor(dom[0])
+        peak = pk[key] * fac
+        if fac == 1.5:
             src = ("GEMM1 at 2 x, GEMM2 at 1 x the " + src + ": 1.5 x the bf16 peak for the kernel's "
                    "2:1 split of flops")
+        elif fac == 2.0:
+            src = "2 x the " + src + " (E4M3 operands: the nominal 4.5 / 2.25 PFLOP/s ratio)"
         roof = {"kernel": dom[0], "bound": "tensor", "achieved": ach, "peak": peak,
                 "unit": "TFLOP/s", "frac": ach / peak, "traffic": tr, "peak_source": src,
-                "frac_of_burst": ach / (fp8_effective_peak(pk["bf16_tflops"]) if args.fp8 else pk["bf16_tflops"]),
+                "frac_of_burst": ach / (pk["bf16_tflops"] * fac),
                 "flops_per_launch": per_launch, "avg_launch_ms": avg_ms}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -550,13 +613,17 @@ def run_ours(args, cfg, rank, world, local_rank):
                    "l2": "flushed by a 256 MB write between timed steps (outside the step events)",
                    **({"precision": "FP8 serving path: GEMM1 (gate, up) on E4M3 operands, one power-of-two scale "
                                     "per bank weight matrix and per activation row; GEMM2 and residual bf16"}
-                      if args.fp8 else {}),
+                      if args.fp8 and not moe else {}),
+                   **({"precision": "FP8 serving path: every expert's GEMM1 (routed and shared gate, up) on E4M3 "
+                                    "operands, one power-of-two scale per (bank, expert) weight matrix and per "
+                                    "activation row; fp32 router, bf16 GEMM2, combine and residuals"}
+                      if args.fp8 and moe else {}),
                    **({"step": "tm_block_backward: the mixing sub-layer's forward recomputed (X_rev), then the "
                                "reverting and mixing sub-layer backward passes (dX and all six weight gradients); "
                                "tflops counts the backward's own 12 W F per row and bank, not the recomputation"}
                       if args.backward else {})},
         "tflops": tflops,
-        "tc_roofline_frac": tflops / (fp8_effective_peak(pk["bf16_tflops"]) if args.fp8 else pk["bf16_tflops"]),
+        "tc_roofline_frac": tflops / (pk["bf16_tflops"] * step_peak_factor(cfg, args.fp8)),
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(cfg.B, world, e2e_ms), "unit": "samples/s", "h2d_bytes_per_step": h2d_bytes,
@@ -598,7 +665,8 @@ def main():
     ap.add_argument("--backward", action="store_true",
                     help="the dense block backward (training): its own line, not the forward metric's")
     ap.add_argument("--fp8", action="store_true",
-                    help="the FP8 E4M3 serving path (dense blocks): its own line, not the bf16 metric's")
+                    help="the FP8 E4M3 serving path (GEMM1 of dense banks and of every MoE expert): its own "
+                         "line, not the bf16 metric's")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

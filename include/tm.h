@@ -307,6 +307,63 @@ TM_API size_t tm_block_fp8_workspace_bytes(const tm_shape *shape, const tm_block
 TM_API tm_status tm_block_forward_fp8(const void *X, const tm_block_fp8 *block, const tm_shape *shape, void *Y,
                                       void *X_revert_opt, void *workspace, size_t workspace_bytes, void *stream);
 
+/* A Sparse-Pertoken MoE bank on the FP8 path ([digest] 2.4, Eq. 19-21, with 2.5.2's E4M3
+ * serving quantization): the fp32 router w_router [banks, E, width] and the bf16 down projections
+ * we_down [banks, E, width, hidden_e], ws_down [banks, width, hidden_s] are those of tm_moe_w; the
+ * gate / up projections are E4M3 codes, the routed experts' qe_gate, qe_up [banks, E, hidden_e,
+ * width] with one fp32 scale per (bank, expert) matrix se_gate, se_up [banks * E], the shared
+ * expert's qs_gate, qs_up [banks, hidden_s, width] with ss_gate, ss_up [banks]
+ * (tm_quantize_fp8_weights makes them, the RMSNorm gain folded in; groups = banks * E, rows =
+ * hidden_e for the routed experts, groups = banks, rows = hidden_s for the shared one). */
+typedef struct {
+    int banks, width, E, k, hidden_e, hidden_s;
+    float alpha;
+    const float *w_router;
+    const uint8_t *qe_gate, *qe_up;
+    const float *se_gate, *se_up;
+    const void *we_down;
+    const uint8_t *qs_gate, *qs_up;
+    const float *ss_gate, *ss_up;
+    const void *ws_down;
+} tm_moe_w8;
+
+/* One sub-layer on the FP8 path: a dense bank (is_moe 0, .dense) or a Sparse-Pertoken MoE bank
+ * (is_moe 1, .moe).  norm_gain [width] (NULL = ones) is the RMSNorm gain that the MoE router
+ * applies to the normalized row before its logits; the E4M3 weights carry it already (for a
+ * dense bank it must be NULL). */
+typedef struct {
+    const void *norm_gain;
+    int is_moe;
+    tm_swiglu_w8 dense;
+    tm_moe_w8 moe;
+} tm_sublayer8;
+
+/* Workspace bytes of tm_sublayer_forward_fp8 / tm_sparse_pertoken_moe_fp8 (0: arguments invalid or
+ * unsupported). */
+TM_API size_t tm_sublayer_fp8_workspace_bytes(const tm_shape *shape, tm_layout layout, const tm_sublayer8 *sub);
+
+/* One sub-layer on the FP8 path with two residual terms, as tm_sublayer_forward:
+ *   y_row = FFN_bank(row) + residual_row + extra_row   (residual / extra NULL: none).
+ * MoE bank: the routing is the bf16 path's (fp32 logits of the normalized row, softmax, top-k,
+ * gates alpha * p; tm_route_topk); each row x is quantized once, q = E4M3(x * 2^-e) with 2^e the
+ * smallest power of two such that max|x| * 2^-e <= 448, and every expert that the row reaches --
+ * its k routed experts and the shared one -- runs GEMM1 on E4M3 operands:
+ *   gate_n = (q . q_gate_n) * 2^e / rms(x) * s_gate,  up_n likewise,  rms over the unquantized row,
+ * then the bf16 SwiGLU, down projection and fixed-order combine of tm_sparse_pertoken_moe.
+ * Supported: bf16, row widths multiples of 128 up to 1024 (mixed rows: head width a multiple of
+ * 8), expert hidden widths multiples of 128, a shared expert (hidden_s > 0), E <= 32, k <= 8; a
+ * dense bank as tm_pertoken_swiglu_fp8.  Others return TM_ERR_UNSUPPORTED before any launch.
+ * y must not alias x, residual or extra. */
+TM_API tm_status tm_sublayer_forward_fp8(const void *x, const void *residual, const void *extra, tm_layout layout,
+                                         const tm_shape *shape, const tm_sublayer8 *sub, void *y, void *workspace,
+                                         size_t workspace_bytes, void *stream);
+
+/* The MoE sub-layer on the FP8 path with one residual: tm_sublayer_forward_fp8 with is_moe 1 and
+ * extra NULL. */
+TM_API tm_status tm_sparse_pertoken_moe_fp8(const void *x, const void *residual, tm_layout layout, const tm_shape *shape,
+                                            const void *norm_gain, const tm_moe_w8 *w, void *y, void *workspace,
+                                            size_t workspace_bytes, void *stream);
+
 /* ---- Training: backward of the dense sub-layer and block ---------------------------------
  * The pages train the model in bf16 ([digest] 2.5.2; [readme] training flags) and print no
  * backward pass, so these calls compute the exact derivative of the forward above by the chain

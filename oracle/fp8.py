@@ -222,3 +222,31 @@ def block_forward_fp8(X: np.ndarray, cfg, qbank: Callable[[int, int], Dict[str, 
     Xr = rnd(revert(Hn, cfg.T))
     Xn = sublayer_fp8(Xr, lambda j: qbank(1, j), cfg.eps) + X
     return {"Hm": Hm, "Xr": Xr, "Y": rnd(Xn)}
+
+
+def block_forward_fp8_any(X: np.ndarray, cfg, qbank: Callable[[int, int], Dict[str, object]],
+                          extra: Optional[np.ndarray] = None, storage=None, forced=(None, None),
+                          gains=(None, None)) -> Dict[str, object]:
+    """A block on the FP8 path whose sub-layers may be dense or Sparse-Pertoken MoE banks: the bf16
+    block ([digest] 2.3, Eq. 9-16, residual to the block input, `extra` the stack's inter-residual
+    term of 2.3.4) with every sub-layer's GEMM1 quantized as 2.5.2 serves it.  qbank(sub, j) gives
+    bank j of sub-layer sub as quantize_bank (dense) or quantize_moe_bank (MoE) makes it; gains: the
+    RMSNorm gains the MoE routers apply (already folded into the quantized weights); forced: the
+    experts of each row per sub-layer, as sublayer_moe_fp8 takes them.  X_rev and the output are the
+    stored tensors `storage` rounds."""
+    rnd = storage_round(storage)
+    info = {}
+
+    def ffn(rows, sub):
+        spec = cfg.ffn(sub)
+        if spec.is_moe:
+            r = sublayer_moe_fp8(rows, lambda j: qbank(sub, j), spec, cfg.eps, gains[sub], forced[sub])
+            info[sub] = r
+            return r["out"]
+        return sublayer_fp8(rows, lambda j: qbank(sub, j), cfg.eps)
+    Hm = mix(X, cfg.H)
+    Xr = rnd(revert(ffn(Hm, 0) + Hm, cfg.T))
+    Y = ffn(Xr, 1) + X
+    if extra is not None:
+        Y = Y + extra
+    return {"Xr": Xr, "Y": rnd(Y), "mix": info.get(0), "rev": info.get(1)}

@@ -246,3 +246,36 @@ int main(void) {
     assert out[0] == "100"
     assert int(out[1]) > 4096 * 16 * 256 * 2 and int(out[2]) > int(out[1])
     assert int(out[3]) == A.TM_ERR_INVALID_ARG
+
+
+def _fake_moe8(cfg, sub, hidden_e=None):
+    spec = cfg.ffn(sub)
+    names = ["w_router", "qe_gate", "qe_up", "se_gate", "se_up", "we_down", "qs_gate", "qs_up", "ss_gate", "ss_up",
+             "ws_down"]
+    t = {n: _FakeTensor(0x100000 * (i + 1)) for i, n in enumerate(names)}
+    return api.MoeSubLayer8(cfg.banks(sub), cfg.width(sub), spec.E, spec.k, hidden_e or spec.hidden_e, spec.hidden_s,
+                            spec.alpha, t)
+
+
+@pytest.mark.parametrize("name", ["moe_stack_bf16", "large_moe_stack_bf16"])
+def test_fp8_moe_workspace_and_validation(name):
+    """The FP8 MoE sub-layer's workspace query and host checks (no launch): the bf16 MoE workspace
+    plus one fp32 row factor per row; unsupported hidden widths and misaligned pointers are refused."""
+    lib = A.load()
+    cfg = S.CONFIGS[name]
+    sh = api.config_shape(cfg)
+    for sub, layout in ((0, A.TM_LAYOUT_MIXED), (1, A.TM_LAYOUT_ROWS)):
+        s8 = _fake_moe8(cfg, sub)
+        n8 = api.sublayer_fp8_workspace_bytes(sh, layout, s8)
+        n16 = api.sublayer_workspace_bytes(sh, layout, _fake_sub(cfg, sub))
+        assert n16 < n8 <= n16 + cfg.B * cfg.banks(sub) * 4 + 512
+        c = s8.sub_c()
+        x, y, ws = ctypes.c_void_p(0x200000), ctypes.c_void_p(0x400000), ctypes.c_void_p(0x800000)
+        assert lib.tm_sublayer_forward_fp8(x, None, None, layout, ctypes.byref(sh), ctypes.byref(c), y, ws, 16,
+                                           None) == A.TM_ERR_WORKSPACE
+        assert lib.tm_sublayer_forward_fp8(x, None, None, layout, ctypes.byref(sh), ctypes.byref(c),
+                                           ctypes.c_void_p(0x400002), ws, n8, None) == A.TM_ERR_INVALID_ARG
+        bad = _fake_moe8(cfg, sub, hidden_e=64).sub_c()
+        assert lib.tm_sublayer_fp8_workspace_bytes(ctypes.byref(sh), layout, ctypes.byref(bad)) == 0
+        assert lib.tm_sublayer_forward_fp8(x, None, None, layout, ctypes.byref(sh), ctypes.byref(bad), y, ws, n8,
+                                           None) == A.TM_ERR_UNSUPPORTED

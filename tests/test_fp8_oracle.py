@@ -190,3 +190,42 @@ def test_fp8_moe_tracks_bf16_moe_and_forcing_works():
     assert 1e-3 < rel < 0.08, rel
     forced = got["idx"][:, ::-1].copy()                       # the same sets, other order: same output
     assert np.allclose(F.sp_moe_fp8(x, qb, k, 4.0, 1e-6, forced_idx=forced)["out"], got["out"], rtol=1e-12, atol=1e-15)
+
+
+def _moe_cfg():
+    import tm_synth as S
+    spec = S.FFNSpec("moe", E=4, k=2, hidden_e=16, hidden_s=16, alpha=2.0)
+    return S.Config("fp8_block_pin", B=12, T=4, D=64, H=4, L=1, dtype="bf16", mix=spec, rev=spec)
+
+
+def test_fp8_moe_block_reductions():
+    """block_forward_fp8_any against what fixes it: (1) zero down projections make the block the
+    identity, plus the inter-residual term; (2) on E4M3-grid rows and weights the mixing sub-layer's
+    GEMM1s are exact, so X_rev is the bf16 oracle block's; (3) with dense banks it is block_forward_fp8."""
+    import tm_synth as S
+    cfg = _moe_cfg()
+    rng = np.random.default_rng(21)
+    banks = {(s, j): _moe_bank(rng, cfg.width(s), 4, 16, 16, on_grid=True) for s in (0, 1) for j in range(4)}
+    X = _grid(rng, cfg.B * cfg.T, cfg.D, -6).reshape(cfg.B, cfg.T, cfg.D)
+    q = {key: F.quantize_moe_bank(bw) for key, bw in banks.items()}
+    got = F.block_forward_fp8_any(X, cfg, lambda s, j: q[(s, j)])
+    want = O.block_forward(X, cfg, 0, lambda l, s, j: banks[(s, j)])
+    assert np.allclose(got["Xr"], want["Xr"], rtol=1e-12, atol=1e-12)
+    assert np.array_equal(got["mix"]["idx"], want["mix"]["idx"])
+    # zero down projections: Y = X + extra exactly, X_rev = X
+    zq = {key: dict(v, experts=[dict(e, w_down=0 * e["w_down"]) for e in v["experts"]],
+                    shared=dict(v["shared"], w_down=0 * v["shared"]["w_down"])) for key, v in q.items()}
+    extra = O.round_bf16(rng.standard_normal(X.shape))
+    z = F.block_forward_fp8_any(X, cfg, lambda s, j: zq[(s, j)], extra=extra)
+    assert np.array_equal(z["Xr"], X) and np.array_equal(z["Y"], X + extra)
+    # dense banks: the dense FP8 block
+    dcfg = S.Config("fp8_block_pin_dense", B=12, T=4, D=64, H=4, L=1, dtype="bf16",
+                    mix=S.FFNSpec("dense", hidden=32), rev=S.FFNSpec("dense", hidden=32))
+    dq = {(s, j): F.quantize_bank({"w_gate": O.round_bf16(rng.standard_normal((32, 64)) / 8),
+                                   "w_up": O.round_bf16(rng.standard_normal((32, 64)) / 8),
+                                   "w_down": O.round_bf16(rng.standard_normal((64, 32)) / 8)})
+          for s in (0, 1) for j in range(4)}
+    Xd = O.round_bf16(rng.standard_normal(X.shape))
+    a = F.block_forward_fp8_any(Xd, dcfg, lambda s, j: dq[(s, j)], storage="bf16")
+    b = F.block_forward_fp8(Xd, dcfg, lambda s, j: dq[(s, j)], storage="bf16")
+    assert np.array_equal(a["Y"], b["Y"]) and np.array_equal(a["Xr"], b["Xr"])

@@ -50,8 +50,7 @@ DENSE_SMALL = [
     small("dense_split_w128", 2400, 8, 128, 4, "bf16", FFNSpec("dense", hidden=256), FFNSpec("dense", hidden=512)),
 ]
 MOE_SMALL = [
-    # tensor-core router; the mixing router also writes the mixed rows out in row layout, from which
-    # the routed GEMM1 gathers (tile::gather4), as it does from the reverting sub-layer's input
+    # tensor-core router; routed rows copied into bucket order, then read by GEMM1 through a 2-D map
     small("moe_sq", 300, 16, 256, 16, "bf16", moe(8, 2, 128, 128, 4.0), moe(4, 1, 64, 192, 4.0)),
     small("moe_ns", 260, 8, 384, 4, "bf16", moe(16, 4, 128, 256), moe(6, 3, 64, 64)),
     # 24 experts: the CUDA-core router; mixed rows then reach GEMM1 through the bucket-order copy

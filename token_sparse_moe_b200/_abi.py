@@ -24,7 +24,8 @@ EXPORTS = ["tm_status_string", "tm_version", "tm_sublayer_workspace_bytes", "tm_
            "tm_pertoken_swiglu_backward_workspace_bytes", "tm_pertoken_swiglu_backward",
            "tm_block_backward_workspace_bytes", "tm_block_backward", "tm_stack_backward_workspace_bytes",
            "tm_stack_backward", "tm_last_device_error_site", "tm_set_wait_limit_ns", "tm_selftest_wait",
-           "tm_selftest_bucket_scatter"]
+           "tm_selftest_bucket_scatter", "tm_sublayer_fp8_workspace_bytes", "tm_sublayer_forward_fp8",
+           "tm_sparse_pertoken_moe_fp8"]
 
 
 class tm_shape(ctypes.Structure):
@@ -58,6 +59,18 @@ class tm_swiglu_w8(ctypes.Structure):
 
 class tm_block_fp8(ctypes.Structure):
     _fields_ = [("mix", tm_swiglu_w8), ("rev", tm_swiglu_w8)]
+
+
+class tm_moe_w8(ctypes.Structure):
+    _fields_ = [("banks", c_int), ("width", c_int), ("E", c_int), ("k", c_int), ("hidden_e", c_int),
+                ("hidden_s", c_int), ("alpha", c_float), ("w_router", c_void_p),
+                ("qe_gate", c_void_p), ("qe_up", c_void_p), ("se_gate", c_void_p), ("se_up", c_void_p),
+                ("we_down", c_void_p), ("qs_gate", c_void_p), ("qs_up", c_void_p), ("ss_gate", c_void_p),
+                ("ss_up", c_void_p), ("ws_down", c_void_p)]
+
+
+class tm_sublayer8(ctypes.Structure):
+    _fields_ = [("norm_gain", c_void_p), ("is_moe", c_int), ("dense", tm_swiglu_w8), ("moe", tm_moe_w8)]
 
 
 class tm_swiglu_grads(ctypes.Structure):
@@ -107,6 +120,11 @@ _SIGS = {
     "tm_pertoken_swiglu_fp8": (c_int, [_P, _P, c_int, POINTER(tm_shape), POINTER(tm_swiglu_w8), _P, _P, c_size_t, _P]),
     "tm_block_fp8_workspace_bytes": (c_size_t, [POINTER(tm_shape), POINTER(tm_block_fp8)]),
     "tm_block_forward_fp8": (c_int, [_P, POINTER(tm_block_fp8), POINTER(tm_shape), _P, _P, _P, c_size_t, _P]),
+    "tm_sublayer_fp8_workspace_bytes": (c_size_t, [POINTER(tm_shape), c_int, POINTER(tm_sublayer8)]),
+    "tm_sublayer_forward_fp8": (c_int, [_P, _P, _P, c_int, POINTER(tm_shape), POINTER(tm_sublayer8), _P, _P, c_size_t,
+                                        _P]),
+    "tm_sparse_pertoken_moe_fp8": (c_int, [_P, _P, c_int, POINTER(tm_shape), _P, POINTER(tm_moe_w8), _P, _P, c_size_t,
+                                           _P]),
     "tm_head_forward": (c_int, [_P, POINTER(tm_shape), _P, _P, _P]),
     "tm_model_workspace_bytes": (c_size_t, [POINTER(tm_shape), POINTER(tm_block), c_int, c_int]),
     "tm_model_forward": (c_int, [_P, _P, _P, c_int, POINTER(tm_block), c_int, c_int, _P, POINTER(tm_shape), _P, _P,

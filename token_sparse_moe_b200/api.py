@@ -418,6 +418,98 @@ class SubLayer8:
                               _p(t["s_up"]), _p(t["w_down"]))
 
 
+    def sub_c(self) -> A.tm_sublayer8:
+        s = A.tm_sublayer8()
+        s.is_moe = 0
+        s.dense = self.c()
+        return s
+
+
+@dataclass
+class MoeSubLayer8:
+    """A Sparse-Pertoken MoE sub-layer on the FP8 path: E4M3 gate / up codes of every routed expert
+    (one scale per (bank, expert) matrix) and of the shared expert (one per bank), the RMSNorm gain
+    folded in by the library's quantizer; the fp32 router, the bf16 down projections and the gain
+    (applied by the router) are the bf16 sub-layer's own tensors."""
+    banks: int
+    width: int
+    E: int
+    k: int
+    hidden_e: int
+    hidden_s: int
+    alpha: float
+    tensors: Dict[str, torch.Tensor]
+    gain: Optional[torch.Tensor] = None
+
+    @staticmethod
+    def from_bf16(sub: "SubLayer", stream=None) -> "MoeSubLayer8":
+        if not sub.is_moe or sub.hidden_s == 0:
+            raise ValueError("the FP8 MoE path covers MoE sub-layers with a shared expert")
+        t = sub.tensors
+        G = sub.banks * sub.E
+        qeg, seg = quantize_fp8_weights(t["we_gate"].reshape(G, sub.hidden_e, sub.width), sub.gain, stream)
+        qeu, seu = quantize_fp8_weights(t["we_up"].reshape(G, sub.hidden_e, sub.width), sub.gain, stream)
+        qsg, ssg = quantize_fp8_weights(t["ws_gate"], sub.gain, stream)
+        qsu, ssu = quantize_fp8_weights(t["ws_up"], sub.gain, stream)
+        q = {"w_router": t["w_router"], "qe_gate": qeg, "se_gate": seg, "qe_up": qeu, "se_up": seu,
+             "we_down": t["we_down"], "qs_gate": qsg, "ss_gate": ssg, "qs_up": qsu, "ss_up": ssu,
+             "ws_down": t["ws_down"]}
+        return MoeSubLayer8(sub.banks, sub.width, sub.E, sub.k, sub.hidden_e, sub.hidden_s, sub.alpha, q, sub.gain)
+
+    def c(self) -> A.tm_moe_w8:
+        t = self.tensors
+        return A.tm_moe_w8(self.banks, self.width, self.E, self.k, self.hidden_e, self.hidden_s, self.alpha,
+                           _p(t["w_router"]), _p(t["qe_gate"]), _p(t["qe_up"]), _p(t["se_gate"]), _p(t["se_up"]),
+                           _p(t["we_down"]), _p(t["qs_gate"]), _p(t["qs_up"]), _p(t["ss_gate"]), _p(t["ss_up"]),
+                           _p(t["ws_down"]))
+
+    def sub_c(self) -> A.tm_sublayer8:
+        s = A.tm_sublayer8()
+        s.norm_gain = _p(self.gain)
+        s.is_moe = 1
+        s.moe = self.c()
+        return s
+
+
+def sublayer8_from_bf16(sub: "SubLayer", stream=None):
+    """The FP8 form of a bf16 sub-layer: MoeSubLayer8 for a MoE bank, SubLayer8 for a dense one."""
+    return MoeSubLayer8.from_bf16(sub, stream) if sub.is_moe else SubLayer8.from_bf16(sub, stream)
+
+
+def sublayer_fp8_workspace_bytes(sh: A.tm_shape, layout: int, sub) -> int:
+    c = sub.sub_c()
+    n = lib().tm_sublayer_fp8_workspace_bytes(ctypes.byref(sh), layout, ctypes.byref(c))
+    if n == 0:
+        raise A.TMError(A.TM_ERR_UNSUPPORTED, "tm_sublayer_fp8_workspace_bytes")
+    return n
+
+
+def sublayer_forward_fp8(x, residual, extra, layout: int, sh: A.tm_shape, sub, y=None, workspace=None, stream=None):
+    """tm_sublayer_forward_fp8: y = FFN_bank(row) + residual + extra on the FP8 path (sub: SubLayer8 or
+    MoeSubLayer8)."""
+    if y is None:
+        y = (torch.empty((sh.B, sh.T, sh.D), dtype=x.dtype, device=x.device) if layout == A.TM_LAYOUT_MIXED
+             else torch.empty((sh.B, sub.banks, sub.width), dtype=x.dtype, device=x.device))
+    c = sub.sub_c()
+    ws = _ws(sublayer_fp8_workspace_bytes(sh, layout, sub), x.device, workspace)
+    A.check(lib().tm_sublayer_forward_fp8(_p(x), _p(residual), _p(extra), layout, ctypes.byref(sh), ctypes.byref(c),
+                                          _p(y), _p(ws), ws.numel(), _s(stream)), "tm_sublayer_forward_fp8")
+    return y
+
+
+def sparse_pertoken_moe_fp8(x, residual, layout: int, sh: A.tm_shape, sub: MoeSubLayer8, y=None, workspace=None,
+                            stream=None):
+    if y is None:
+        y = (torch.empty((sh.B, sh.T, sh.D), dtype=x.dtype, device=x.device) if layout == A.TM_LAYOUT_MIXED
+             else torch.empty((sh.B, sub.banks, sub.width), dtype=x.dtype, device=x.device))
+    w = sub.c()
+    ws = _ws(sublayer_fp8_workspace_bytes(sh, layout, sub), x.device, workspace)
+    A.check(lib().tm_sparse_pertoken_moe_fp8(_p(x), _p(residual), layout, ctypes.byref(sh), _p(sub.gain),
+                                             ctypes.byref(w), _p(y), _p(ws), ws.numel(), _s(stream)),
+            "tm_sparse_pertoken_moe_fp8")
+    return y
+
+
 @dataclass
 class Block8:
     mix: SubLayer8
@@ -483,6 +575,51 @@ class Fp8BlockRunner:
             A.check(lib().tm_block_forward_fp8(_p(cur), ctypes.byref(c), ctypes.byref(self.sh), _p(out), None,
                                                _p(self.ws), self.ws.numel(), _s(stream)), "tm_block_forward_fp8")
             cur = out
+        return Y
+
+    def run_host(self, X_host, Y_host, X_dev, Y_dev, stream=None):
+        s = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(s):
+            X_dev.copy_(X_host, non_blocking=True)
+            self(X_dev, Y_dev, s)
+            Y_host.copy_(Y_dev, non_blocking=True)
+        return Y_host
+
+
+class Fp8StackRunner:
+    """A stack on the FP8 path, one tm_sublayer_forward_fp8 call per sub-layer, with the inter-residual
+    every `gap` blocks ([digest] 2.3.4: block l adds X_{l-gap} when l % gap == 0, except the last).
+    blocks: (mixing, reverting) pairs of SubLayer8 / MoeSubLayer8.  Block l runs
+      X_rev = FFN_mix(Mix(X_{l-1})) + Mix(X_{l-1}), stored through Revert (mixed layout, residual X_{l-1});
+      X_l   = FFN_rev(X_rev) + X_{l-1} (+ X_{l-gap})                       (row layout)
+    with a preallocated workspace and intermediate token tensors, so repeated forwards allocate nothing."""
+
+    def __init__(self, blocks: Sequence, sh: A.tm_shape, gap: int, device):
+        self.blocks = list(blocks)
+        self.sh = sh
+        self.gap = gap
+        L = len(self.blocks)
+        self.cs = [(m.sub_c(), r.sub_c()) for m, r in self.blocks]
+        n = max(max(sublayer_fp8_workspace_bytes(sh, A.TM_LAYOUT_MIXED, m),
+                    sublayer_fp8_workspace_bytes(sh, A.TM_LAYOUT_ROWS, r)) for m, r in self.blocks)
+        self.ws = torch.empty(n, dtype=torch.uint8, device=device)
+        tok = (sh.B, sh.T, sh.D)
+        self.xr = torch.empty(tok, dtype=torch.bfloat16, device=device)
+        self.hist = [torch.empty(tok, dtype=torch.bfloat16, device=device) for _ in range(L - 1)]
+
+    def _sub(self, x, resid, extra, layout, c, y, stream):
+        A.check(lib().tm_sublayer_forward_fp8(_p(x), _p(resid), _p(extra), layout, ctypes.byref(self.sh),
+                                              ctypes.byref(c), _p(y), _p(self.ws), self.ws.numel(), _s(stream)),
+                "tm_sublayer_forward_fp8")
+
+    def __call__(self, X: torch.Tensor, Y: torch.Tensor, stream=None) -> torch.Tensor:
+        L = len(self.cs)
+        xs = [X] + self.hist + [Y]
+        for l in range(1, L + 1):
+            cm, cr = self.cs[l - 1]
+            self._sub(xs[l - 1], xs[l - 1], None, A.TM_LAYOUT_MIXED, cm, self.xr, stream)
+            skip = xs[l - self.gap] if (self.gap > 0 and l % self.gap == 0 and l < L) else None
+            self._sub(self.xr, xs[l - 1], skip, A.TM_LAYOUT_ROWS, cr, xs[l], stream)
         return Y
 
     def run_host(self, X_host, Y_host, X_dev, Y_dev, stream=None):

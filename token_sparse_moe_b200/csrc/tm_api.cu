@@ -220,6 +220,18 @@ GemmParams base_params(const Geo& g) {
     return p;
 }
 
+// Banks per chunk of the sched-0 tile order (a power of two): as many as keep one row block's working
+// set of the chunk -- each bank's weight tiles (w_bytes) and the rows it streams for one row block
+// (row_bytes) -- within 24 MB of the 126 MB L2.  A bank's weights are then read from DRAM about once
+// per chunk instead of once per row block: with all 48 banks of the large MoE stack in one cycle
+// (113 MB of shared-expert gate / up weights) the shared GEMM1 read 12 GB for 1.3 GB of data.
+int bank_chunk(double w_bytes, double row_bytes) {
+    const double per = w_bytes + row_bytes;
+    int c = 1;
+    while (c < (1 << 20) && 2.0 * c * per <= 24.0 * (1 << 20)) c *= 2;
+    return c;
+}
+
 int dense_grid(const GemmParams& p) {
     const long tiles = (long)p.groups * ((p.rows + 127) / 128) * p.n_tiles;
     return (int)(tiles < num_sms() ? tiles : num_sms());
@@ -247,7 +259,8 @@ int sched0_grid(const GemmParams& p, bool pair) {
     return pair_grid((long)p.groups * ((p.rows + 255) / 256) * p.n_tiles);
 }
 
-// SwiGLU GEMM1 over x (dense groups = banks, rows = B): hidden [banks*B, F]
+// SwiGLU GEMM1 over x (dense groups = banks, rows = B): hidden [banks*B, F].  inv_rms NULL (bf16 rows
+// read through a 3-D or Mix map): the kernel takes the row statistics itself (EPI_SWIGLU_NORM).
 tm_status gemm1_dense(const Geo& g, const void* x, const void* wg, const void* wu, int F, const float* inv_rms,
                       void* hidden, cudaStream_t st) {
     GemmParams p = base_params(g);
@@ -266,13 +279,17 @@ tm_status gemm1_dense(const Geo& g, const void* x, const void* wg, const void* w
     }
     const int bn = pick_bn_swiglu(F);
     p.n_tiles = p.N / bn;
+    p.bank_chunk = bank_chunk(2.0 * 2 * F * g.W, 128.0 * 2 * (g.W + F));
     const int am = gemm1_amode(g);
+    const int epi = inv_rms ? EPI_SWIGLU : EPI_SWIGLU_NORM;
+    if (!inv_rms && am != A_TMA_3D && am != A_TMA_MIX) return TM_ERR_UNSUPPORTED;
+    p.r_eps = g.eps;
     CUtensorMap ma, mg, mu, mo;
     if (!gemm1_amap(g, x, am, &ma)) return TM_ERR_CUDA;
     if (!map_2d(&mg, wg, (uint64_t)g.banks * F, g.W, bn / 2) || !map_2d(&mu, wu, (uint64_t)g.banks * F, g.W, bn / 2) ||
         !map_2d(&mo, hidden, (uint64_t)g.banks * g.B, F, 32))
         return TM_ERR_CUDA;
-    return cuda_status(launch_grouped_gemm(bn, am, EPI_SWIGLU, ma, mg, mu, p, dense_grid(p), st, &mo));
+    return cuda_status(launch_grouped_gemm(bn, am, epi, ma, mg, mu, p, dense_grid(p), st, &mo));
 }
 
 // GEMM2 over dense hidden rows [banks*B, F] with the residual / combine epilogue into y (omap).
@@ -299,6 +316,7 @@ tm_status gemm2_dense(const Geo& g, const void* hidden, const void* wd, int F, i
     }
     const int bn = pick_bn_out(g.W);
     p.n_tiles = g.W / bn;
+    p.bank_chunk = bank_chunk(2.0 * F * g.W, 128.0 * 2 * (F + (3 + k) * g.W));
     CUtensorMap ma, mb;
     if (!map_2d(&ma, hidden, (uint64_t)g.banks * g.B, F, 128) || !map_2d(&mb, wd, (uint64_t)g.banks * g.W, F, bn))
         return TM_ERR_CUDA;
@@ -387,11 +405,14 @@ tm_status run_dense(const Geo& g, const void* x, const void* resid, const void* 
     }
     if (g.dtype == TM_BF16 && fused_supported(g.W, gemm1_amode(g)) && w->hidden % 64 == 0)
         return fused_dense(g, x, wg, wu, w->w_down, w->hidden, resid, extra, y, st);
-    if ((s = cuda_status(launch_rms(g.dtype, x, g.map, g.B, g.eps, d.inv_rms, st))) != TM_OK) return s;
-    if ((s = gemm1_dense(g, x, wg, wu, w->hidden, d.inv_rms, d.hidden, st)) != TM_OK) return s;
+    // bf16 rows read through a tensor map: GEMM1 takes the row statistics itself; otherwise they come
+    // from rms_kernel first
+    const int am = gemm1_amode(g);
+    const bool stats_in_gemm = g.dtype == TM_BF16 && (am == A_TMA_3D || am == A_TMA_MIX);
+    if (!stats_in_gemm && (s = cuda_status(launch_rms(g.dtype, x, g.map, g.B, g.eps, d.inv_rms, st))) != TM_OK) return s;
+    if ((s = gemm1_dense(g, x, wg, wu, w->hidden, stats_in_gemm ? nullptr : d.inv_rms, d.hidden, st)) != TM_OK) return s;
     // bf16 with a tensor-map row geometry: GEMM2 with the residual and inter-residual entering the
     // accumulator through identity MMAs and bulk tensor stores out (the combine kernel, no expert rows)
-    const int am = gemm1_amode(g);
     if (g.dtype == TM_BF16 && (am == A_TMA_3D || am == A_TMA_MIX))
         return combine_sum(g, d.hidden, w->w_down, w->hidden, resid, extra, y, nullptr, 0, st);
     return gemm2_dense(g, d.hidden, w->w_down, w->hidden, EPI_RESID, resid, extra, y, nullptr, nullptr, nullptr, 0, st);
@@ -512,6 +533,7 @@ tm_status combine_sum(const Geo& g, const void* hidden_s, const void* wd, int Fs
     const int bn = pick_bn_out(g.W);
     p.n_tiles = g.W / bn;
     const bool pair = use_pair(g, A_TMA_2D);
+    p.bank_chunk = bank_chunk(2.0 * Fs * g.W, (pair ? 256.0 : 128.0) * 2 * (Fs + (3 + k) * g.W));
     CUtensorMap ma, mb, m0, m1, m2, mo;
     memset(&m0, 0, sizeof(m0));
     memset(&m1, 0, sizeof(m1));
@@ -756,6 +778,184 @@ tm_status check_block8(const tm_shape* s, const tm_block_fp8* b, Geo* gm, Geo* g
 // workspace of an FP8 block: X_revert and the row-block counters of block mode
 size_t block8_ws(const Geo& gm, const Geo&, const tm_shape* s) {
     return align256((size_t)s->B * s->T * s->D * 2) + align256((size_t)(gm.B + 127) / 128 * sizeof(unsigned));
+}
+
+// ------------------------------------------------------------------ FP8 E4M3 MoE sub-layer
+// The routing view of an FP8 MoE bank (router, counts, k, alpha) with its code matrices standing in
+// for the bf16 gate / up weights, so that the bf16 path's checks and workspace carve apply.
+tm_moe_w moe_view(const tm_moe_w8* w) {
+    tm_moe_w v;
+    v.banks = w->banks;
+    v.width = w->width;
+    v.E = w->E;
+    v.k = w->k;
+    v.hidden_e = w->hidden_e;
+    v.hidden_s = w->hidden_s;
+    v.alpha = w->alpha;
+    v.w_router = w->w_router;
+    v.we_gate = w->qe_gate;
+    v.we_up = w->qe_up;
+    v.we_down = w->we_down;
+    v.ws_gate = w->qs_gate;
+    v.ws_up = w->qs_up;
+    v.ws_down = w->ws_down;
+    return v;
+}
+
+tm_status check_moe8(const Geo& g, const tm_moe_w8* w) {
+    if (!w) return TM_ERR_INVALID_ARG;
+    const tm_moe_w v = moe_view(w);
+    tm_status s = check_moe(g, &v);
+    if (s != TM_OK) return s;
+    if (!w->se_gate || !w->se_up || !al16(w->se_gate) || !al16(w->se_up)) return TM_ERR_INVALID_ARG;
+    if (w->hidden_s > 0 && (!w->ss_gate || !w->ss_up || !al16(w->ss_gate) || !al16(w->ss_up))) return TM_ERR_INVALID_ARG;
+    if (g.dtype != TM_BF16 || w->hidden_s == 0) return TM_ERR_UNSUPPORTED;
+    // E4M3 K slabs of 128 codes; the quantizer holds a row in one warp's registers
+    if (g.W % 128 || g.W > 1024 || w->hidden_e % 128 || w->hidden_s % 128) return TM_ERR_UNSUPPORTED;
+    if (g.map.layout == 1 && g.map.dh % 8) return TM_ERR_UNSUPPORTED;
+    const int am = gemm1_amode(g);
+    if (am != A_TMA_MIX && am != A_TMA_3D) return TM_ERR_UNSUPPORTED;   // the combine's residual maps
+    return TM_OK;
+}
+
+// The bf16 MoE workspace (routing tables, hidden rows, slot rows) plus the rows' E4M3 factors.  The
+// codes live in the slot buffer, which is free until the routed GEMM2 writes it: the bucket-order
+// codes [routed, W] first, then the row-order codes [B * banks, W] (routed * W * 2 bytes hold both).
+struct Moe8Ws {
+    MoeWs m;
+    float* rowscale;
+    uint8_t *qpos, *q;
+};
+Moe8Ws carve_moe8(Carve& c, const Geo& g, const tm_moe_w8* w) {
+    Moe8Ws r;
+    const tm_moe_w v = moe_view(w);
+    r.m = carve_moe(c, g, &v, false);
+    r.rowscale = c.take<float>((size_t)g.B * g.banks);
+    const size_t routed = (size_t)g.B * g.banks * w->k;
+    r.qpos = (uint8_t*)r.m.slots;
+    r.q = r.qpos + routed * g.W;
+    return r;
+}
+
+// E4M3 GEMM1 + SwiGLU over `groups` groups of code rows (tmA), weights q_gate / q_up [groups * F, W]
+tm_status gemm1_f8(GemmParams p, int a_mode, const CUtensorMap& ma, const uint8_t* qg, const uint8_t* qu, int F,
+                   const float* sg, const float* su, void* hidden, size_t rows_out, int grid, cudaStream_t st) {
+    const int bn = pick_bn_swiglu(F);
+    p.N = 2 * F;
+    p.n_tiles = p.N / bn;
+    p.out = (__nv_bfloat16*)hidden;
+    p.out_ld = F;
+    p.out_elems = rows_out * F;
+    p.w8_sgate = sg;
+    p.w8_sup = su;
+    uint64_t dims[2] = {(uint64_t)p.K, (uint64_t)p.groups * F};
+    uint64_t strides[1] = {(uint64_t)p.K};
+    uint32_t box[2] = {128, (uint32_t)bn / 2};
+    CUtensorMap mg, mu, mo;
+    if (!make_map_u8(&mg, qg, 2, dims, strides, box) || !make_map_u8(&mu, qu, 2, dims, strides, box) ||
+        !map_2d(&mo, hidden, rows_out, F, 32))
+        return TM_ERR_CUDA;
+    if (grid <= 0) grid = dense_grid(p);
+    return cuda_status(launch_grouped_gemm_f8(bn, a_mode, ma, mg, mu, p, grid, st, &mo));
+}
+
+// The MoE sub-layer with E4M3 GEMM1s: route (bf16 path's router) -> quantize every row once, writing
+// its codes in row order and at its k bucket positions -> routed GEMM1 over the buckets, shared GEMM1
+// over the rows (both kind::f8f6f4) -> the bf16 routed GEMM2 into combine order -> combine + shared
+// GEMM2 + residuals.
+tm_status run_moe8(const Geo& g, const void* x, const void* resid, const void* extra, const void* gain,
+                   const tm_moe_w8* w, void* y, void* ws, size_t wsb, cudaStream_t st) {
+    Carve c{(uint8_t*)ws};
+    Moe8Ws q = carve_moe8(c, g, w);
+    MoeWs& m = q.m;
+    if (!ws || wsb < c.off || !al16(ws)) return TM_ERR_WORKSPACE;
+    const tm_moe_w v = moe_view(w);
+    tm_status s;
+    RouteOut r{m.idx, m.offsets, m.tile_start, m.bucket_rows, m.slot_of, m.counts, m.gate, m.inv_rms};
+    r.perm = m.perm;
+    r.inv_pos = nullptr;        // the row factors by position come from the quantizer
+    r.gate_pos = m.gate_pos;
+    r.wsplit = m.wsplit;
+    r.tile_info = m.tile_info;
+    if ((s = run_route(g, x, gain, &v, r, st)) != TM_OK) return s;
+
+    const size_t rows = (size_t)g.B * g.banks, routed = rows * w->k;
+    if ((s = cuda_status(launch_quant_act_rows(x, g.map, g.B, g.eps, q.q, q.rowscale, st, m.slot_of, w->k, routed,
+                                               q.qpos, m.inv_pos))) != TM_OK)
+        return s;
+    const size_t G = (size_t)g.banks * w->E;
+    const int Fe = w->hidden_e;
+    const long max_mt = (long)(routed / 128) + (long)G;
+    // routed experts: bucket-order codes through a 2-D map, row factor by bucket position
+    GemmParams p = base_params(g);
+    p.sched = 1;
+    p.groups = (int)G;
+    p.E = w->E;
+    p.row_start = m.offsets;
+    p.tile_start = m.tile_start;
+    p.tile_info = m.tile_info;
+    p.bucket_rows = m.bucket_rows;
+    p.pos_scale = m.inv_pos;
+    p.pos_limit = (int)routed;
+    p.K = g.W;
+    {
+        uint64_t dims[2] = {(uint64_t)g.W, (uint64_t)routed};
+        uint64_t strides[1] = {(uint64_t)g.W};
+        uint32_t box[2] = {128, 128};
+        CUtensorMap ma;
+        if (!make_map_u8(&ma, q.qpos, 2, dims, strides, box)) return TM_ERR_CUDA;
+        const int nt = 2 * Fe / pick_bn_swiglu(Fe);
+        const long grid = max_mt * nt < num_sms() ? max_mt * nt : num_sms();
+        if ((s = gemm1_f8(p, A_TMA_2D, ma, w->qe_gate, w->qe_up, Fe, w->se_gate, w->se_up, m.hidden_r, routed, (int)grid,
+                          st)) != TM_OK)
+            return s;
+    }
+    // shared expert: row-order codes [B, banks, W] through a 3-D map, row factor by row
+    {
+        GemmParams ps = base_params(g);
+        ps.sched = 0;
+        ps.K = g.W;
+        ps.inv_rms = q.rowscale;
+        ps.bank_chunk = bank_chunk(2.0 * w->hidden_s * g.W, 128.0 * (g.W + 2.0 * w->hidden_s));
+        uint64_t dims[3] = {(uint64_t)g.W, (uint64_t)g.banks, (uint64_t)g.B};
+        uint64_t strides[2] = {(uint64_t)g.W, (uint64_t)g.banks * g.W};
+        uint32_t box[3] = {128, 1, 128};
+        CUtensorMap ma;
+        if (!make_map_u8(&ma, q.q, 3, dims, strides, box)) return TM_ERR_CUDA;
+        if ((s = gemm1_f8(ps, A_TMA_3D, ma, w->qs_gate, w->qs_up, w->hidden_s, w->ss_gate, w->ss_up, m.hidden_s, rows, 0,
+                          st)) != TM_OK)
+            return s;
+    }
+    // routed GEMM2 (bf16) into combine order, gate-scaled, then the combine with the shared GEMM2
+    p.pos_scale = m.gate_pos;
+    p.K = Fe;
+    p.N = g.W;
+    p.out = (__nv_bfloat16*)m.slots;
+    p.out_ld = g.W;
+    p.out_elems = routed * g.W;
+    const int bn = pick_bn_out(g.W);
+    p.n_tiles = g.W / bn;
+    p.perm = m.perm;
+    p.gate = m.gate;
+    CUtensorMap ma, mb, mo;
+    if (!map_2d(&ma, m.hidden_r, routed, Fe, 128) || !map_2d(&mb, w->we_down, G * g.W, Fe, bn) ||
+        !map_2d(&mo, m.slots, routed, g.W, 1))
+        return TM_ERR_CUDA;
+    const long grid = max_mt * p.n_tiles < num_sms() ? max_mt * p.n_tiles : num_sms();
+    if ((s = cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SLOT_PERM, ma, mb, mb, p, (int)grid, st, &mo))) != TM_OK)
+        return s;
+    return combine_sum(g, m.hidden_s, w->ws_down, w->hidden_s, resid, extra, y, m.slots, w->k, st);
+}
+
+tm_status check_sublayer8(const tm_shape* shape, int layout, const tm_sublayer8* sub, Geo* g) {
+    if (!sub) return TM_ERR_INVALID_ARG;
+    const int banks = sub->is_moe ? sub->moe.banks : sub->dense.banks;
+    const int width = sub->is_moe ? sub->moe.width : sub->dense.width;
+    tm_status s = make_geo(shape, layout, banks, width, g);
+    if (s != TM_OK) return s;
+    if (sub->norm_gain && !al16(sub->norm_gain)) return TM_ERR_INVALID_ARG;
+    if (!sub->is_moe && sub->norm_gain) return TM_ERR_INVALID_ARG;   // folded into the codes
+    return sub->is_moe ? check_moe8(*g, &sub->moe) : check_dense8(*g, &sub->dense);
 }
 
 // ------------------------------------------------------------------ sub-layer dispatch
@@ -1356,6 +1556,41 @@ tm_status tm_quantize_fp8_act(const void* x, tm_layout layout, const tm_shape* s
         return TM_ERR_INVALID_ARG;
     if (g.dtype != TM_BF16 || g.W > 1024 || (g.map.layout == 1 && g.map.dh % 8)) return TM_ERR_UNSUPPORTED;
     return cuda_status(launch_quant_act_rows(x, g.map, g.B, g.eps, q, rowscale, (cudaStream_t)stream));
+}
+
+size_t tm_sublayer_fp8_workspace_bytes(const tm_shape* shape, tm_layout layout, const tm_sublayer8* sub) {
+    Geo g;
+    if (check_sublayer8(shape, layout, sub, &g) != TM_OK) return 0;
+    if (!sub->is_moe) return 256;
+    Carve c{nullptr};
+    carve_moe8(c, g, &sub->moe);
+    return align256(c.off);
+}
+
+tm_status tm_sublayer_forward_fp8(const void* x, const void* residual, const void* extra, tm_layout layout,
+                                  const tm_shape* shape, const tm_sublayer8* sub, void* y, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    Geo g;
+    tm_status s = check_sublayer8(shape, layout, sub, &g);
+    if (s != TM_OK) return s;
+    if (!x || !y || !al16(x) || !al16(y) || x == y || (residual && (!al16(residual) || residual == y)))
+        return TM_ERR_INVALID_ARG;
+    if (extra && (!al16(extra) || extra == y)) return TM_ERR_INVALID_ARG;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (sub->is_moe) return run_moe8(g, x, residual, extra, sub->norm_gain, &sub->moe, y, workspace, workspace_bytes, st);
+    return run_dense8(g, x, residual, extra, &sub->dense, y, st);
+}
+
+tm_status tm_sparse_pertoken_moe_fp8(const void* x, const void* residual, tm_layout layout, const tm_shape* shape,
+                                     const void* norm_gain, const tm_moe_w8* w, void* y, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+    if (!w) return TM_ERR_INVALID_ARG;
+    tm_sublayer8 sub;
+    memset(&sub, 0, sizeof(sub));
+    sub.norm_gain = norm_gain;
+    sub.is_moe = 1;
+    sub.moe = *w;
+    return tm_sublayer_forward_fp8(x, residual, nullptr, layout, shape, &sub, y, workspace, workspace_bytes, stream);
 }
 
 size_t tm_pertoken_swiglu_fp8_workspace_bytes(const tm_shape* shape, tm_layout layout, const tm_swiglu_w8* w) {

@@ -100,12 +100,12 @@ cudaError_t launch_fused(int W, int a_mode, const CUtensorMap& a, const CUtensor
     return cudaErrorInvalidValue;
 }
 
-template <int BN, int AM, int EPI, bool PAIR>
+template <int BN, int AM, int EPI, bool PAIR, bool F8 = false>
 static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& s0,
                               const CUtensorMap& s1, const CUtensorMap& s2, const CUtensorMap& o, const GemmParams& p,
                               int grid, cudaStream_t st) {
-    using C = GemmCfg<BN, AM, EPI, PAIR>;
-    auto kern = grouped_gemm_kernel<BN, AM, EPI, PAIR>;
+    using C = GemmCfg<BN, AM, EPI, PAIR, F8>;
+    auto kern = grouped_gemm_kernel<BN, AM, EPI, PAIR, F8>;
     static bool configured = false;   // attribute set once per instantiation (per process)
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -113,7 +113,8 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
         configured = true;
     }
     ProfileScope ps_(EPI == EPI_ROUTE                           ? "router"
-                     : EPI == EPI_SWIGLU                        ? "gemm_swiglu"
+                     : F8 ? "gemm_swiglu_fp8"
+                     : (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_NORM) ? "gemm_swiglu"
                      : EPI == EPI_RESID                         ? "gemm_resid"
                      : (EPI == EPI_SLOT || EPI == EPI_SLOT_PERM) ? "gemm_slot"
                                                                  : "gemm_combine",
@@ -147,6 +148,8 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
 #define TM_GEMM_TABLE(X)                                  \
     X(256, A_TMA_3D, EPI_SWIGLU, 0) X(128, A_TMA_3D, EPI_SWIGLU, 0) \
     X(256, A_TMA_MIX, EPI_SWIGLU, 0) X(128, A_TMA_MIX, EPI_SWIGLU, 0) \
+    X(256, A_TMA_3D, EPI_SWIGLU_NORM, 0) X(128, A_TMA_3D, EPI_SWIGLU_NORM, 0) \
+    X(256, A_TMA_MIX, EPI_SWIGLU_NORM, 0) X(128, A_TMA_MIX, EPI_SWIGLU_NORM, 0) \
     X(256, A_GATHER, EPI_SWIGLU, 0) X(128, A_GATHER, EPI_SWIGLU, 0) \
     X(256, A_TMA_2D, EPI_SWIGLU, 0) X(128, A_TMA_2D, EPI_SWIGLU, 0) \
     X(256, A_TMA_2D, EPI_RESID, 0) X(192, A_TMA_2D, EPI_RESID, 0) X(128, A_TMA_2D, EPI_RESID, 0) \
@@ -162,7 +165,8 @@ cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorM
                                     const CUtensorMap& tmS2, const GemmParams& p, int grid, cudaStream_t st,
                                     const CUtensorMap* tmO, bool pair) {
     // the SwiGLU, combine, plain-row and expert-row epilogues store through the output map
-    if ((epi == EPI_SWIGLU || epi == EPI_SUM || epi == EPI_SLOT || epi == EPI_SLOT_PERM) && !tmO)
+    if ((epi == EPI_SWIGLU || epi == EPI_SWIGLU_NORM || epi == EPI_SUM || epi == EPI_SLOT || epi == EPI_SLOT_PERM) &&
+        !tmO)
         return cudaErrorInvalidValue;
     CUtensorMap none;
     memset(&none, 0, sizeof(none));
@@ -172,6 +176,25 @@ cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorM
         return launch_one<BN, AM, EP, PR != 0>(tmA, tmB0, tmB1, tmS0, tmS1, tmS2, o, p, grid, st);
     TM_GEMM_TABLE(X)
 #undef X
+    return cudaErrorInvalidValue;
+}
+
+// GEMM1 + SwiGLU on E4M3 operands (kind::f8f6f4): A through a 2-D map (bucket-order rows) or a
+// 3-D map ([B, banks, W] rows) of codes with 128-code boxes, B the E4M3 gate / up maps.
+cudaError_t launch_grouped_gemm_f8(int bn, int a_mode, const CUtensorMap& tmA, const CUtensorMap& tmB0,
+                                   const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st,
+                                   const CUtensorMap* tmO) {
+    if (!tmO || !p.w8_sgate || !p.w8_sup) return cudaErrorInvalidValue;
+    CUtensorMap none;
+    memset(&none, 0, sizeof(none));
+    if (bn == 256 && a_mode == A_TMA_2D)
+        return launch_one<256, A_TMA_2D, EPI_SWIGLU, false, true>(tmA, tmB0, tmB1, none, none, none, *tmO, p, grid, st);
+    if (bn == 128 && a_mode == A_TMA_2D)
+        return launch_one<128, A_TMA_2D, EPI_SWIGLU, false, true>(tmA, tmB0, tmB1, none, none, none, *tmO, p, grid, st);
+    if (bn == 256 && a_mode == A_TMA_3D)
+        return launch_one<256, A_TMA_3D, EPI_SWIGLU, false, true>(tmA, tmB0, tmB1, none, none, none, *tmO, p, grid, st);
+    if (bn == 128 && a_mode == A_TMA_3D)
+        return launch_one<128, A_TMA_3D, EPI_SWIGLU, false, true>(tmA, tmB0, tmB1, none, none, none, *tmO, p, grid, st);
     return cudaErrorInvalidValue;
 }
 

@@ -46,8 +46,11 @@ enum AMode : int { A_TMA_2D = 0, A_TMA_3D = 1, A_TMA_MIX = 2, A_GATHER = 3 };
 // bf16 rows (hi, mid, lo), the accumulator's columns e, E+e, 2E+e add up to the fp32 logit; four
 // extra warps take each row's sum of squares from the A stages as they pass; the epilogue does
 // the scale, softmax, top-k, gates and the per-chunk expert counts.
+// EPI_SWIGLU_NORM: EPI_SWIGLU with the pre-RMSNorm's row statistics taken in the kernel: four extra
+// warps sum each row's squares from the A stages as they pass (as for EPI_ROUTE), the epilogue
+// scales by 1/sqrt(sum / K + eps) (dense groups of rows read through a 3-D or Mix map).
 enum Epi : int { EPI_SWIGLU = 0, EPI_RESID = 1, EPI_SLOT = 2, EPI_COMBINE = 3, EPI_SLOT_PERM = 4, EPI_SUM = 5,
-                 EPI_ROUTE = 6 };
+                 EPI_ROUTE = 6, EPI_SWIGLU_NORM = 7 };
 constexpr int kRouteMaxE = 21;   // 3 * E <= 64 accumulator columns
 
 // Where element c of the row (sample b, bank) of a sub-layer lives in a tensor.
@@ -66,6 +69,7 @@ __host__ __device__ __forceinline__ size_t row_elem(const RowMap& m, int b, int 
 struct GemmParams {
     // tile space
     int sched;                 // 0: groups of `rows` rows (dense banks); 1: bucketed (routed experts)
+    int bank_chunk;            // sched 0: banks per chunk of the tile order (0: all); see decode_tile
     int groups;                // number of groups (sched 1: banks * E)
     int rows;                  // sched 0: rows per group (= B)
     int banks;                 // sub-layer banks
@@ -103,30 +107,43 @@ struct GemmParams {
     int32_t* r_counts;
     int r_nchunks;
     float r_alpha, r_eps;
+    // F8 (E4M3 GEMM1): the gate / up weight matrices' scales, one per group
+    const float* w8_sgate;
+    const float* w8_sup;
 };
 
-template <int BN, int AMODE, int EPI = EPI_SWIGLU, bool PAIR = false>
+template <int BN, int AMODE, int EPI = EPI_SWIGLU, bool PAIR = false, bool F8 = false>
 struct GemmCfg {
     static constexpr int BM = 128, BK = 64;
+    // K elements per 128-byte slab row: 64 bf16, or 128 E4M3 codes (F8: GEMM1 on kind::f8f6f4)
+    static constexpr int KSLAB = F8 ? 128 : 64;
+    static_assert(!F8 || (EPI == EPI_SWIGLU && !PAIR && (AMODE == A_TMA_2D || AMODE == A_TMA_3D)),
+                  "the E4M3 mode covers GEMM1 with plain row maps");
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * BK * 2;   // this CTA's weight rows of a stage
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     // the scattered-row epilogue is latency-bound per warp: two warps per TMEM lane quarter, each
     // taking half of the tile's columns
     static constexpr int EPI_WARPS = (EPI == EPI_SLOT_PERM && BN % 128 == 0) ? 8 : 4;
-    static constexpr int STG_BYTES_ = (EPI == EPI_SWIGLU || EPI == EPI_SLOT_PERM || EPI == EPI_SUM || EPI == EPI_SLOT)
+    static constexpr int STG_BYTES_ = (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_NORM || EPI == EPI_SLOT_PERM ||
+                                       EPI == EPI_SUM || EPI == EPI_SLOT)
                                           ? EPI_WARPS * 4096 : 0;
+    // the row-statistics warps (6-9) of the router and of GEMM1 with the norm in the kernel
+    static constexpr bool STATS = EPI == EPI_ROUTE || EPI == EPI_SWIGLU_NORM;
     // pair mode: as many stages as the shared memory holds, at most 8
     static constexpr int PAIR_STAGES_ = (232448 - 2304 - STG_BYTES_) / STAGE_BYTES;
     static constexpr int STAGES = PAIR ? (PAIR_STAGES_ > 8 ? 8 : PAIR_STAGES_)
                                        : (BN >= 256 ? 4 : (BN >= 192 ? (EPI_WARPS == 8 ? 4 : 5) : 6));
     static_assert(!PAIR || (AMODE != A_GATHER && EPI != EPI_ROUTE && EPI != EPI_RESID && EPI != EPI_COMBINE),
                   "pair mode covers tensor-map A operands and the staged epilogues");
-    static constexpr int NWARPS = (AMODE == A_GATHER || EPI == EPI_ROUTE) ? 10 : 2 + EPI_WARPS;
+    static constexpr int NWARPS = (AMODE == A_GATHER || STATS) ? 10 : 2 + EPI_WARPS;
+    static_assert(EPI != EPI_SWIGLU_NORM || AMODE == A_TMA_3D || AMODE == A_TMA_MIX,
+                  "in-kernel row statistics read rows through a 3-D or Mix map");
     static constexpr int NTHREADS = NWARPS * 32;
     static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
     // output staging: one 32-row x 64-column bf16 box (4 KB) per epilogue warp
-    static constexpr bool STAGED = EPI == EPI_SWIGLU || EPI == EPI_SLOT_PERM || EPI == EPI_SUM || EPI == EPI_SLOT;
+    static constexpr bool STAGED =
+        EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_NORM || EPI == EPI_SLOT_PERM || EPI == EPI_SUM || EPI == EPI_SLOT;
     static constexpr int OFF_STG = STAGES * STAGE_BYTES;
     static constexpr int STG_BYTES = STAGED ? EPI_WARPS * 4096 : 0;
     static constexpr int OFF_ID = OFF_STG + STG_BYTES;             // 16 x 16 identity (EPI_SUM), 1 KB
@@ -148,15 +165,20 @@ __device__ __forceinline__ int total_tiles_pair(const GemmParams& p) {
     return p.groups * ((p.rows + 255) / 256) * p.n_tiles;
 }
 
-// This CTA's 128-row half (rank 0: the first) of 256-row tile t, row block major with the banks
-// innermost as decode_tile; a half past the group's end has nrows = 0 (its rows are loaded,
+// This CTA's 128-row half (rank 0: the first) of 256-row tile t, in decode_tile's order (bank chunks,
+// row block major inside a chunk); a half past the group's end has nrows = 0 (its rows are loaded,
 // multiplied and never stored).
 __device__ __forceinline__ TileInfo decode_tile_pair(const GemmParams& p, int t, int rank) {
     TileInfo ti;
     const int gm = t / p.n_tiles;
     ti.n = t - gm * p.n_tiles;
-    const int m2 = gm / p.groups;
-    ti.g = gm - m2 * p.groups;
+    const int mt2 = (p.rows + 255) / 256;
+    const int cb = (p.bank_chunk > 0 && p.bank_chunk < p.groups) ? p.bank_chunk : p.groups;
+    const int c = gm / (cb * mt2);
+    const int rr = gm - c * cb * mt2;
+    const int g0 = c * cb, nb = min(cb, p.groups - g0);
+    const int m2 = rr / nb;
+    ti.g = g0 + (rr - m2 * nb);
     ti.m = 2 * m2 + rank;
     ti.row0 = ti.g * p.rows + ti.m * 128;
     ti.nrows = max(0, min(128, p.rows - ti.m * 128));
@@ -168,10 +190,17 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int t) {
     const int gm = t / p.n_tiles;
     ti.n = t - gm * p.n_tiles;
     if (p.sched == 0) {
-        // row block major, banks innermost: the CTAs running side by side read the same samples'
+        // chunks of banks whose weights fit in the L2 together, in turn; inside a chunk row block
+        // major with the banks innermost: the CTAs running side by side read the same samples'
         // token rows (whole sectors when a bank's segment of a row is short, as with the Mix map)
-        ti.m = gm / p.groups;
-        ti.g = gm - ti.m * p.groups;
+        // while the chunk's weights stay in the L2 from one row block to the next
+        const int mt = (p.rows + 127) / 128;
+        const int cb = (p.bank_chunk > 0 && p.bank_chunk < p.groups) ? p.bank_chunk : p.groups;
+        const int c = gm / (cb * mt);
+        const int rr = gm - c * cb * mt;
+        const int g0 = c * cb, nb = min(cb, p.groups - g0);
+        ti.m = rr / nb;
+        ti.g = g0 + (rr - ti.m * nb);
         ti.row0 = ti.g * p.rows + ti.m * 128;
         ti.nrows = min(128, p.rows - ti.m * 128);
     } else if (p.tile_info) {
@@ -227,14 +256,15 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     }
 }
 
-template <int BN, int AMODE, int EPI, bool PAIR>
-__global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
+template <int BN, int AMODE, int EPI, bool PAIR, bool F8>
+__global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR, F8>::NTHREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmS0,
                         const __grid_constant__ CUtensorMap tmS1, const __grid_constant__ CUtensorMap tmS2,
                         const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
-    using C = GemmCfg<BN, AMODE, EPI, PAIR>;
+    using C = GemmCfg<BN, AMODE, EPI, PAIR, F8>;
     constexpr int STAGES = C::STAGES;
+    constexpr int KSLAB = C::KSLAB;
     // pair mode: the two CTAs of a cluster share the tile sequence (cluster index cid), each taking
     // its 128-row half; both return here together, so both reach the closing cluster barrier
     const int rank = PAIR ? (int)cluster_ctarank() : 0;
@@ -256,15 +286,15 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
     uint64_t* acc_full = empty + STAGES;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
-    uint64_t* st_full = drain + 1;         // [2] EPI_ROUTE: row sums of squares of a tile written
-    uint64_t* st_empty = st_full + 2;      // [2] EPI_ROUTE: ... and read by the epilogue
-    float* ssbuf = reinterpret_cast<float*>(sI);   // EPI_ROUTE: [2][128] (the identity slot is unused)
+    uint64_t* st_full = drain + 1;         // [2] statistics warps: row sums of squares of a tile written
+    uint64_t* st_empty = st_full + 2;      // [2] ... and read by the epilogue
+    float* ssbuf = reinterpret_cast<float*>(sI);   // statistics: [2][128] (the identity slot is unused)
     uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(st_empty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int KB = p.K / 64;
+    const int KB = p.K / KSLAB;
     // pair mode: the leader's copy (L) and the peer's copy (P) of a barrier of this CTA's layout
     auto L = [&](uint64_t* b) { return mapa_shared(smem_u32(b), 0); };
     auto P = [&](uint64_t* b) { return mapa_shared(smem_u32(b), 1); };
@@ -276,7 +306,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], AMODE == A_GATHER ? 1 + 128 : 1);
-            mbar_init(&empty[s], EPI == EPI_ROUTE ? 1 + 4 : 1);   // + the four statistics warps
+            mbar_init(&empty[s], C::STATS ? 1 + 4 : 1);   // + the four statistics warps
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
@@ -323,7 +353,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
         if (lane == 0) {
             if (AMODE != A_GATHER) tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmB0);
-            if (EPI == EPI_SWIGLU) tma_prefetch_desc(&tmB1);
+            if (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_NORM) tma_prefetch_desc(&tmB1);
             int s = 0;
             uint32_t ph = 0;
             // a stage's loads count their bytes on this CTA's full barrier, or in pair mode on the
@@ -386,9 +416,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
                     uint8_t* sb = sa + C::A_BYTES;
                     begin_stage(bytes_k);
                     if (AMODE == A_TMA_2D) {
-                        ld2(sa, &tmA, kb * 64, ti.row0);
+                        ld2(sa, &tmA, kb * KSLAB, ti.row0);
                     } else if (AMODE == A_TMA_3D) {
-                        ld3(sa, &tmA, kb * 64, ti.g, ti.m * 128);
+                        ld3(sa, &tmA, kb * KSLAB, ti.g, ti.m * 128);
                     } else if (AMODE == A_TMA_MIX) {
                         // mixed-row columns c16*16 .. +15 = token t, head piece jj of head ti.g
                         const int per = p.amap.dh >> 4;
@@ -399,15 +429,15 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
                             ld4(sa + i * 4096, &tmA, 0, ti.g * per + jj, t, ti.m * 128);
                         }
                     }
-                    if (EPI == EPI_SWIGLU) {
+                    if (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_NORM) {
                         const int F = p.N >> 1;
                         const int r0 = ti.g * F + ti.n * (BN / 2);
                         if (PAIR) {
                             // the leader holds the BN/2 gate rows (N rows 0 .. BN/2-1), the peer the up rows
-                            ld2(sb, leader ? &tmB0 : &tmB1, kb * 64, r0);
+                            ld2(sb, leader ? &tmB0 : &tmB1, kb * KSLAB, r0);
                         } else {
-                            ld2(sb, &tmB0, kb * 64, r0);
-                            ld2(sb + (BN / 2) * 128, &tmB1, kb * 64, r0);
+                            ld2(sb, &tmB0, kb * KSLAB, r0);
+                            ld2(sb + (BN / 2) * 128, &tmB1, kb * KSLAB, r0);
                         }
                     } else {
                         // pair mode: this CTA's half of the N tile's weight rows
@@ -421,11 +451,12 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer (pair mode: leader)
         if (lane == 0 && leader) {
-            constexpr uint32_t idesc = umma_idesc_bf16(PAIR ? 256 : 128, BN);
+            constexpr uint32_t idesc = F8 ? umma_idesc_e4m3(128, BN) : umma_idesc_bf16(PAIR ? 256 : 128, BN);
             // an MMA of this CTA (M = 128) or of the pair (M = 256); commits arrive on this CTA's
             // barrier, or on the same barrier of both CTAs
             auto mma = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
                 if (PAIR) umma_bf16_pair(d, a, b, id, acc);
+                else if (F8) umma_e4m3(d, a, b, id, acc);    // K = 32 codes per instruction
                 else umma_bf16(d, a, b, id, acc);
             };
             auto commit = [&](uint64_t* b) {
@@ -648,8 +679,18 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
                     if (lane == 0 && bal)
                         atomicAdd(&p.r_counts[((size_t)bank * p.r_nchunks + ti.m) * E + e], __popc(bal));
                 }
-            } else if (EPI == EPI_SWIGLU) {
-                const float sc = valid ? rm.s : 0.f;
+            } else if (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_NORM) {
+                float sc = valid ? rm.s : 0.f;
+                // F8: the row factor (E4M3 row scale / rms) times each projection's matrix scale
+                const float sg8 = F8 ? __ldg(&p.w8_sgate[ti.g]) : 1.f, su8 = F8 ? __ldg(&p.w8_sup[ti.g]) : 1.f;
+                if (EPI == EPI_SWIGLU_NORM) {
+                    // 1/rms of this row from the statistics warps' sum of squares over the K columns
+                    if (!wait_or_abort(&st_full[buf], aph, abort_flag, 0x331)) break;
+                    const float ssq = ssbuf[buf * 128 + r];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&st_empty[buf]);
+                    sc = valid ? 1.0f / sqrtf(ssq / (float)p.K + p.r_eps) : 0.f;
+                }
                 // a bulk tensor store per 32 x 64 box when all 32 rows of this warp belong to the
                 // tile's group; else the valid rows through coalesced stores
                 const bool box = __all_sync(0xffffffffu, valid);
@@ -664,8 +705,15 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
                         tmem_ld32(taddr + BN / 2 + c + 32 * h, uv);
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const float h0 = silu_tanh(sc * gv[2 * i]) * (sc * uv[2 * i]);
-                            const float h1 = silu_tanh(sc * gv[2 * i + 1]) * (sc * uv[2 * i + 1]);
+                            float h0, h1;
+                            if (F8) {
+                                const float sg = sc * sg8, su = sc * su8;
+                                h0 = silu_tanh(sg * gv[2 * i]) * (su * uv[2 * i]);
+                                h1 = silu_tanh(sg * gv[2 * i + 1]) * (su * uv[2 * i + 1]);
+                            } else {
+                                h0 = silu_tanh(sc * gv[2 * i]) * (sc * uv[2 * i]);
+                                h1 = silu_tanh(sc * gv[2 * i + 1]) * (sc * uv[2 * i + 1]);
+                            }
                             pk[16 * h + i] = pack_bf16x2(h0, h1);
                         }
                     }
@@ -884,7 +932,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, AMODE, EPI, PAIR>::NTHREADS, 1)
         }
         if (C::STAGED && lane < 8) bulk_wait_all();                   // stores complete before exit
         __syncwarp();
-    } else if (EPI == EPI_ROUTE) {
+    } else if (C::STATS) {
         // ---------------------------------------------------------------- row statistics (warps 6-9)
         // Each lane sums the squares of its row of every A stage (a second consumer of the stage:
         // the empty barrier also waits for these four warps), then hands the tile's sums over.

@@ -41,6 +41,14 @@ cudaError_t launch_grouped_gemm(int bn, int a_mode, int epi, const CUtensorMap& 
                                 const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st,
                                 const CUtensorMap* tmO = nullptr, bool pair = false);
 
+// GEMM1 + SwiGLU on E4M3 operands: A codes through a 2-D (bucket-order rows) or 3-D ([B, banks, W])
+// map with 128-code boxes and 128-byte swizzle, tmB0 / tmB1 the E4M3 gate / up maps (BN/2-row boxes);
+// p.w8_sgate / p.w8_sup the matrices' scales per group; the row factor by position (p.pos_scale) or
+// by row (p.inv_rms)
+cudaError_t launch_grouped_gemm_f8(int bn, int a_mode, const CUtensorMap& tmA, const CUtensorMap& tmB0,
+                                   const CUtensorMap& tmB1, const GemmParams& p, int grid, cudaStream_t st,
+                                   const CUtensorMap* tmO);
+
 // ---- fused dense sub-layer (row width 128 / 256) --------------------------------
 bool fused_supported(int W, int a_mode);
 cudaError_t launch_fused(int W, int a_mode, const CUtensorMap& a, const CUtensorMap& g, const CUtensorMap& u,
@@ -91,11 +99,14 @@ cudaError_t launch_scatter_rows(int dtype, const void* x, RowMap m, int B, int k
                                 void* out, cudaStream_t st);
 // FP8 E4M3 (bf16 inputs): the codes of `groups` weight matrices of n elements (rows of `cols`)
 // with one scale per matrix (gain optional, folded first), and the per-row activation codes
-// [B * banks, W] with rowscale = (max|x| / 448) / rms(x)
+// [B * banks, W] with rowscale = 2^e / rms(x), 2^e the row's power-of-two E4M3 scale
 cudaError_t launch_quant_matrices(const void* w, const void* gain, int groups, size_t n, int cols, uint8_t* q,
                                   float* scale, cudaStream_t st);
+// slot_of (optional, [B * banks, k]): the codes and row factors also to the rows' k bucket positions
+// (qpos [routed, W], scale_pos [routed]); q / rowscale may then be NULL
 cudaError_t launch_quant_act_rows(const void* x, RowMap m, int B, float eps, uint8_t* q, float* rowscale,
-                                  cudaStream_t st);
+                                  cudaStream_t st, const int32_t* slot_of = nullptr, int k = 0, size_t routed = 0,
+                                  uint8_t* qpos = nullptr, float* scale_pos = nullptr);
 cudaError_t launch_permute(int dtype, const void* src, void* dst, int B, int T, int D, int H, bool to_mixed,
                            cudaStream_t st);
 cudaError_t launch_fold_gain(int dtype, const void* w, const void* gain, void* out, size_t rows, int width,

@@ -807,9 +807,14 @@ __global__ void quant_matrix_scales_kernel(unsigned* __restrict__ scale_bits, in
 // b * banks + bank).  One warp per row: sum of squares and max|x| by shuffles; codes =
 // E4M3(x * 2^-e) with the row's power-of-two scale 2^e; rowscale = 2^e / rms(x), the factor the
 // FP8 GEMM1 output takes back per row.
+// With slot_of (the bucketing of tm_route_topk, [B * banks, k]) the row's codes and row factor also
+// go to its k bucket positions (qpos [routed, W], scale_pos [routed]): the MoEPermute copy of the
+// FP8 path, one byte per element.
 __global__ void __launch_bounds__(256) quant_act_rows_kernel(const __nv_bfloat16* __restrict__ x, RowMap m, int B,
                                                              float eps, uint8_t* __restrict__ q,
-                                                             float* __restrict__ rowscale) {
+                                                             float* __restrict__ rowscale,
+                                                             const int32_t* __restrict__ slot_of, int k, int routed,
+                                                             uint8_t* __restrict__ qpos, float* __restrict__ scale_pos) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
     const int W = m.W, banks = m.banks;
@@ -819,10 +824,10 @@ __global__ void __launch_bounds__(256) quant_act_rows_kernel(const __nv_bfloat16
         uint4 v[4];
         float ss = 0.f, amax = 0.f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int c = lane * 8 + 256 * k;
-            v[k] = c < W ? __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c))) : make_uint4(0, 0, 0, 0);
-            const uint32_t wv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+        for (int kk = 0; kk < 4; ++kk) {
+            const int c = lane * 8 + 256 * kk;
+            v[kk] = c < W ? __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c))) : make_uint4(0, 0, 0, 0);
+            const uint32_t wv[4] = {v[kk].x, v[kk].y, v[kk].z, v[kk].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float lo = __uint_as_float(wv[e] << 16), hi = __uint_as_float(wv[e] & 0xFFFF0000u);
@@ -837,19 +842,41 @@ __global__ void __launch_bounds__(256) quant_act_rows_kernel(const __nv_bfloat16
         }
         const int ex = pow2_exponent(amax);
         const float s = pow2f(ex), inv = pow2f(-ex);
+        // the row's bucket positions (FP8 MoE path)
+        int pos[8];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int c = lane * 8 + 256 * k;
+        for (int j = 0; j < 8; ++j) {
+            pos[j] = -1;
+            if (slot_of && j < k) {
+                pos[j] = __ldg(&slot_of[(size_t)row * k + j]);
+                if (pos[j] < 0 || pos[j] >= routed) {
+                    if (lane == 0) record_error(ERR_BOUNDS, 0x530);
+                    pos[j] = -1;
+                }
+            }
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const int c = lane * 8 + 256 * kk;
             if (c >= W) break;
-            const uint32_t wv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+            const uint32_t wv[4] = {v[kk].x, v[kk].y, v[kk].z, v[kk].w};
             uint16_t o4[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 o4[e] = e4m3x2(__uint_as_float(wv[e] << 16) * inv, __uint_as_float(wv[e] & 0xFFFF0000u) * inv);
-            *reinterpret_cast<uint2*>(q + (size_t)row * W + c) =
-                make_uint2(o4[0] | (uint32_t(o4[1]) << 16), o4[2] | (uint32_t(o4[3]) << 16));
+            const uint2 w2 = make_uint2(o4[0] | (uint32_t(o4[1]) << 16), o4[2] | (uint32_t(o4[3]) << 16));
+            if (q) *reinterpret_cast<uint2*>(q + (size_t)row * W + c) = w2;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (pos[j] >= 0) *reinterpret_cast<uint2*>(qpos + (size_t)pos[j] * W + c) = w2;
         }
-        if (lane == 0) rowscale[row] = s * (1.0f / sqrtf(ss / (float)W + eps));
+        const float rs = s * (1.0f / sqrtf(ss / (float)W + eps));
+        if (lane == 0) {
+            if (rowscale) rowscale[row] = rs;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (pos[j] >= 0 && scale_pos) scale_pos[pos[j]] = rs;
+        }
     }
 }
 
@@ -870,11 +897,13 @@ cudaError_t launch_quant_matrices(const void* w, const void* gain, int groups, s
 }
 
 cudaError_t launch_quant_act_rows(const void* x, RowMap m, int B, float eps, uint8_t* q, float* rowscale,
-                                  cudaStream_t st) {
-    ProfileScope ps_("fp8_quant_rows", st);
+                                  cudaStream_t st, const int32_t* slot_of, int k, size_t routed, uint8_t* qpos,
+                                  float* scale_pos) {
+    ProfileScope ps_(slot_of ? "fp8_quant_permute" : "fp8_quant_rows", st);
     if (m.W % 8 || m.W > 1024 || (m.layout == 1 && m.dh % 8)) return cudaErrorInvalidValue;
-    quant_act_rows_kernel<<<grid_for((size_t)B * m.banks * 32, 256), 256, 0, st>>>((const __nv_bfloat16*)x, m, B, eps,
-                                                                                  q, rowscale);
+    if (slot_of && (k < 1 || k > 8 || !qpos)) return cudaErrorInvalidValue;
+    quant_act_rows_kernel<<<grid_for((size_t)B * m.banks * 32, 256), 256, 0, st>>>(
+        (const __nv_bfloat16*)x, m, B, eps, q, rowscale, slot_of, k, (int)routed, qpos, scale_pos);
     return cudaGetLastError();
 }
 
