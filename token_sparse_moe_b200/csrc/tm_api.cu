@@ -554,6 +554,25 @@ tm_status combine_sum(const Geo& g, const void* hidden_s, const void* wd, int Fs
         launch_grouped_gemm_src(bn, A_TMA_2D, EPI_SUM, ma, mb, mb, m0, m1, m2, p, sched0_grid(p, pair), st, &mo, pair));
 }
 
+// The routed GEMM2: expert rows scaled by their gates, written to their combine positions by scatter
+// stores of one-row boxes; p carries the bucket schedule.
+tm_status routed_gemm2(const Geo& g, GemmParams p, const void* hidden_r, const void* wd, int Fe, size_t routed, long max_mt,
+                       void* slots, cudaStream_t st) {
+    p.K = Fe;
+    p.N = g.W;
+    p.out = (__nv_bfloat16*)slots;
+    p.out_ld = g.W;
+    p.out_elems = routed * g.W;
+    const int bn = pick_bn_out(g.W);
+    p.n_tiles = g.W / bn;
+    CUtensorMap ma, mb, mo;
+    if (!map_2d(&ma, hidden_r, routed, Fe, 128) || !map_2d(&mb, wd, (uint64_t)p.groups * g.W, Fe, bn) ||
+        !map_2d(&mo, slots, routed, g.W, 1))
+        return TM_ERR_CUDA;
+    const long grid = max_mt * p.n_tiles < num_sms() ? max_mt * p.n_tiles : num_sms();
+    return cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SLOT_PERM, ma, mb, mb, p, (int)grid, st, &mo));
+}
+
 tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* extra, const void* gain,
                   const tm_moe_w* w, void* y, void* ws, size_t wsb, cudaStream_t st) {
     Carve c{(uint8_t*)ws};
@@ -641,20 +660,12 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
         if ((s = cuda_status(launch_simt_gemm(EPI_SLOT, a, (int)(max_mt * p.n_tiles), st))) != TM_OK) return s;
     } else {
         // rows written in combine order ((bank * k + j) * B + b) and scaled by their gate, so that
-        // the combine reads each tile's expert rows as one contiguous tensor-map box per choice
-        const int bn = pick_bn_out(g.W);
-        p.n_tiles = g.W / bn;
+        // the combine reads each tile's expert rows as one contiguous tensor-map box per choice; they
+        // leave through scatter stores of one-row boxes into the slot rows
         p.perm = m.perm;
         p.gate = m.gate;
         p.pos_scale = m.gate_pos;
-        // the expert rows leave through scatter stores of one-row boxes into the slot rows
-        CUtensorMap ma, mb, mo;
-        if (!map_2d(&ma, m.hidden_r, routed, Fe, 128) || !map_2d(&mb, w->we_down, G * g.W, Fe, bn) ||
-            !map_2d(&mo, m.slots, routed, g.W, 1))
-            return TM_ERR_CUDA;
-        const long grid = max_mt * p.n_tiles < num_sms() ? max_mt * p.n_tiles : num_sms();
-        if ((s = cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SLOT_PERM, ma, mb, mb, p, (int)grid, st, &mo))) != TM_OK)
-            return s;
+        if ((s = routed_gemm2(g, p, m.hidden_r, w->we_down, Fe, routed, max_mt, m.slots, st)) != TM_OK) return s;
         return combine_sum(g, m.hidden_s, w->ws_down, w->hidden_s, resid, extra, y, m.slots, w->k, st);
     }
     // shared expert GEMM2 + deterministic combine + residual(s), stored through the row map
@@ -928,22 +939,9 @@ tm_status run_moe8(const Geo& g, const void* x, const void* resid, const void* e
     }
     // routed GEMM2 (bf16) into combine order, gate-scaled, then the combine with the shared GEMM2
     p.pos_scale = m.gate_pos;
-    p.K = Fe;
-    p.N = g.W;
-    p.out = (__nv_bfloat16*)m.slots;
-    p.out_ld = g.W;
-    p.out_elems = routed * g.W;
-    const int bn = pick_bn_out(g.W);
-    p.n_tiles = g.W / bn;
     p.perm = m.perm;
     p.gate = m.gate;
-    CUtensorMap ma, mb, mo;
-    if (!map_2d(&ma, m.hidden_r, routed, Fe, 128) || !map_2d(&mb, w->we_down, G * g.W, Fe, bn) ||
-        !map_2d(&mo, m.slots, routed, g.W, 1))
-        return TM_ERR_CUDA;
-    const long grid = max_mt * p.n_tiles < num_sms() ? max_mt * p.n_tiles : num_sms();
-    if ((s = cuda_status(launch_grouped_gemm(bn, A_TMA_2D, EPI_SLOT_PERM, ma, mb, mb, p, (int)grid, st, &mo))) != TM_OK)
-        return s;
+    if ((s = routed_gemm2(g, p, m.hidden_r, w->we_down, Fe, routed, max_mt, m.slots, st)) != TM_OK) return s;
     return combine_sum(g, m.hidden_s, w->ws_down, w->hidden_s, resid, extra, y, m.slots, w->k, st);
 }
 

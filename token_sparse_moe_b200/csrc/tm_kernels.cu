@@ -810,6 +810,12 @@ __global__ void quant_matrix_scales_kernel(unsigned* __restrict__ scale_bits, in
 // With slot_of (the bucketing of tm_route_topk, [B * banks, k]) the row's codes and row factor also
 // go to its k bucket positions (qpos [routed, W], scale_pos [routed]): the MoEPermute copy of the
 // FP8 path, one byte per element.
+// Each warp takes QROWS rows at a time and issues all their loads (bucket positions and row pieces)
+// before any reduction or store, so that a warp keeps QROWS rows of reads in flight.  NP: 8-element
+// pieces per lane (W <= 256 * NP); KMAX: bucket positions per row held (k <= KMAX; 0: no scatter),
+// both compile-time so that the registers hold only what the row needs.
+constexpr int QROWS = 2;
+template <int NP, int KMAX>
 __global__ void __launch_bounds__(256) quant_act_rows_kernel(const __nv_bfloat16* __restrict__ x, RowMap m, int B,
                                                              float eps, uint8_t* __restrict__ q,
                                                              float* __restrict__ rowscale,
@@ -817,65 +823,94 @@ __global__ void __launch_bounds__(256) quant_act_rows_kernel(const __nv_bfloat16
                                                              uint8_t* __restrict__ qpos, float* __restrict__ scale_pos) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
-    const int W = m.W, banks = m.banks;
-    for (int row = warp; row < B * banks; row += nwarps) {
-        const int b = row / banks, bank = row - b * banks;
-        // the row stays in registers: up to four 8-element pieces per lane (W <= 1024)
-        uint4 v[4];
-        float ss = 0.f, amax = 0.f;
+    const int W = m.W, banks = m.banks, nrows = B * banks;
+    for (int row0 = warp * QROWS; row0 < nrows; row0 += nwarps * QROWS) {
+        // the rows' bucket positions (FP8 MoE path) and the rows themselves, all loads issued before
+        // they are used
+        int pos[QROWS][KMAX > 0 ? KMAX : 1];
+        uint4 v[QROWS][NP];
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            const int c = lane * 8 + 256 * kk;
-            v[kk] = c < W ? __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c))) : make_uint4(0, 0, 0, 0);
-            const uint32_t wv[4] = {v[kk].x, v[kk].y, v[kk].z, v[kk].w};
+        for (int rr = 0; rr < QROWS; ++rr) {
+            const int row = row0 + rr;
+            const bool ok = row < nrows;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float lo = __uint_as_float(wv[e] << 16), hi = __uint_as_float(wv[e] & 0xFFFF0000u);
-                ss = fmaf(lo, lo, fmaf(hi, hi, ss));
-                amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+            for (int j = 0; j < KMAX; ++j)
+                pos[rr][j] = (ok && j < k) ? __ldg(&slot_of[(size_t)row * k + j]) : -1;
+            const int b = ok ? row / banks : 0, bank = ok ? row - b * banks : 0;
+#pragma unroll
+            for (int kk = 0; kk < NP; ++kk) {
+                const int c = lane * 8 + 256 * kk;
+                v[rr][kk] = (ok && c < W) ? __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c)))
+                                          : make_uint4(0, 0, 0, 0);
             }
+        }
+        // sum of squares in fp32 on element pairs (paired FMA: the even and odd elements accumulate
+        // apart and are added at the end); max|x| on the packed bf16 magnitudes as 16-bit integers
+        // (non-negative floats order as their bit patterns), widened once per row
+        float ss[QROWS], amax[QROWS];
+#pragma unroll
+        for (int rr = 0; rr < QROWS; ++rr) {
+            float2 s2 = make_float2(0.f, 0.f);
+            uint32_t m2 = 0;
+#pragma unroll
+            for (int kk = 0; kk < NP; ++kk) {
+                const uint32_t wv[4] = {v[rr][kk].x, v[rr][kk].y, v[rr][kk].z, v[rr][kk].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 p2 = make_float2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
+                    s2 = __ffma2_rn(p2, p2, s2);
+                    m2 = __vmaxu2(m2, wv[e] & 0x7FFF7FFFu);
+                }
+            }
+            ss[rr] = s2.x + s2.y;
+            amax[rr] = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-            ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        }
-        const int ex = pow2_exponent(amax);
-        const float s = pow2f(ex), inv = pow2f(-ex);
-        // the row's bucket positions (FP8 MoE path)
-        int pos[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            pos[j] = -1;
-            if (slot_of && j < k) {
-                pos[j] = __ldg(&slot_of[(size_t)row * k + j]);
-                if (pos[j] < 0 || pos[j] >= routed) {
-                    if (lane == 0) record_error(ERR_BOUNDS, 0x530);
-                    pos[j] = -1;
-                }
+            for (int rr = 0; rr < QROWS; ++rr) {
+                ss[rr] += __shfl_xor_sync(0xffffffffu, ss[rr], o);
+                amax[rr] = fmaxf(amax[rr], __shfl_xor_sync(0xffffffffu, amax[rr], o));
             }
         }
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            const int c = lane * 8 + 256 * kk;
-            if (c >= W) break;
-            const uint32_t wv[4] = {v[kk].x, v[kk].y, v[kk].z, v[kk].w};
-            uint16_t o4[4];
+        for (int rr = 0; rr < QROWS; ++rr) {
+            const int row = row0 + rr;
+            if (row >= nrows) break;
+            const int ex = pow2_exponent(amax[rr]);
+            const float s = pow2f(ex), inv = pow2f(-ex);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                o4[e] = e4m3x2(__uint_as_float(wv[e] << 16) * inv, __uint_as_float(wv[e] & 0xFFFF0000u) * inv);
-            const uint2 w2 = make_uint2(o4[0] | (uint32_t(o4[1]) << 16), o4[2] | (uint32_t(o4[3]) << 16));
-            if (q) *reinterpret_cast<uint2*>(q + (size_t)row * W + c) = w2;
+            for (int j = 0; j < KMAX; ++j) {
+                if (j < k && (pos[rr][j] < 0 || pos[rr][j] >= routed)) {
+                    if (lane == 0) record_error(ERR_BOUNDS, 0x530);
+                    pos[rr][j] = -1;
+                }
+            }
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if (pos[j] >= 0) *reinterpret_cast<uint2*>(qpos + (size_t)pos[j] * W + c) = w2;
-        }
-        const float rs = s * (1.0f / sqrtf(ss / (float)W + eps));
-        if (lane == 0) {
-            if (rowscale) rowscale[row] = rs;
+            for (int kk = 0; kk < NP; ++kk) {
+                const int c = lane * 8 + 256 * kk;
+                if (c >= W) break;
+                const uint32_t wv[4] = {v[rr][kk].x, v[rr][kk].y, v[rr][kk].z, v[rr][kk].w};
+                uint16_t o4[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if (pos[j] >= 0 && scale_pos) scale_pos[pos[j]] = rs;
+                for (int e = 0; e < 4; ++e) {
+                    const float2 t = __fmul2_rn(make_float2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u)),
+                                                make_float2(inv, inv));
+                    o4[e] = e4m3x2(t.x, t.y);
+                }
+                const uint2 w2 = make_uint2(o4[0] | (uint32_t(o4[1]) << 16), o4[2] | (uint32_t(o4[3]) << 16));
+                if (q) *reinterpret_cast<uint2*>(q + (size_t)row * W + c) = w2;
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j)
+                    if (pos[rr][j] >= 0) *reinterpret_cast<uint2*>(qpos + (size_t)pos[rr][j] * W + c) = w2;
+            }
+            const float rs = s * (1.0f / sqrtf(ss[rr] / (float)W + eps));
+            if (lane == 0) {
+                if (rowscale) rowscale[row] = rs;
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j)
+                    if (pos[rr][j] >= 0 && scale_pos) scale_pos[pos[rr][j]] = rs;
+            }
         }
     }
 }
@@ -902,9 +937,19 @@ cudaError_t launch_quant_act_rows(const void* x, RowMap m, int B, float eps, uin
     ProfileScope ps_(slot_of ? "fp8_quant_permute" : "fp8_quant_rows", st);
     if (m.W % 8 || m.W > 1024 || (m.layout == 1 && m.dh % 8)) return cudaErrorInvalidValue;
     if (slot_of && (k < 1 || k > 8 || !qpos)) return cudaErrorInvalidValue;
-    quant_act_rows_kernel<<<grid_for((size_t)B * m.banks * 32, 256), 256, 0, st>>>(
-        (const __nv_bfloat16*)x, m, B, eps, q, rowscale, slot_of, k, (int)routed, qpos, scale_pos);
-    return cudaGetLastError();
+    const int grid = grid_for(((size_t)B * m.banks + QROWS - 1) / QROWS * 32, 256);
+    const int np = (m.W + 255) / 256, kmax = !slot_of ? 0 : k <= 2 ? 2 : k <= 4 ? 4 : 8;
+#define QLAUNCH(NP, KM)                                                                                              \
+    if (np == NP && kmax == KM) {                                                                                    \
+        quant_act_rows_kernel<NP, KM><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, m, B, eps, q, rowscale, slot_of, \
+                                                            k, (int)routed, qpos, scale_pos);                         \
+        return cudaGetLastError();                                                                                   \
+    }
+#define QLAUNCH_NP(NP) QLAUNCH(NP, 0) QLAUNCH(NP, 2) QLAUNCH(NP, 4) QLAUNCH(NP, 8)
+    QLAUNCH_NP(1) QLAUNCH_NP(2) QLAUNCH_NP(3) QLAUNCH_NP(4)
+#undef QLAUNCH_NP
+#undef QLAUNCH
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace tml
