@@ -20,7 +20,7 @@ end-to-end leg copies each step's batch from pinned host memory and the result b
 sample chunks pipelined against the compute (the result is checked bit for bit against the
 full-batch device run).  --batch and --layers run a smaller case of the same kernels (profiler
 captures).  --fp8 and --backward print their own lines (the FP8 serving path, the dense block
-backward) on a dense workload.
+backward).
 """
 from __future__ import annotations
 
@@ -534,10 +534,11 @@ def run_ours(args, cfg, rank, world, local_rank):
     Xd = torch.empty_like(X)
     # the backward step's inputs are X and dY (both copied in), its result dX (copied back)
     dYh = dY.cpu().pin_memory() if args.backward else None
-    chunks = args.e2e_chunks if not (args.backward or args.fp8) else 1
+    chunks = (api.RAMP_CHUNKS if args.e2e_chunks == "ramp" else int(args.e2e_chunks)) \
+        if not (args.backward or args.fp8) else 1
     if args.backward:
         host = lambda: run.run_host(Xh, Yh, Xd, Y, dYh, stream)
-    elif chunks > 1:
+    elif chunks != 1:
         host = lambda: run.run_host(Xh, Yh, Xd, Y, stream, chunks=chunks)
     else:
         host = lambda: run.run_host(Xh, Yh, Xd, Y, stream)
@@ -627,7 +628,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(cfg.B, world, e2e_ms), "unit": "samples/s", "h2d_bytes_per_step": h2d_bytes,
-                "d2h_bytes_per_step": io_bytes, "ms_per_step": e2e_ms, "steps": Ke, "chunks": chunks,
+                "d2h_bytes_per_step": io_bytes, "ms_per_step": e2e_ms, "steps": Ke,
+                "chunks": list(chunks) if not isinstance(chunks, int) else chunks,
                 "matches_device_result": e2e_exact},
         "gpu_launches": int(launches),
         "launches_per_step": launches / K,
@@ -659,9 +661,9 @@ def main():
                          "profiler captures; the line's workload string carries the B used)")
     ap.add_argument("--layers", type=int, default=None,
                     help="run the workload with this many blocks (small cases for profiler captures)")
-    ap.add_argument("--e2e-chunks", type=int, default=8,
-                    help="end-to-end leg: split the batch into this many chunks whose host copies overlap "
-                         "the compute (forward only)")
+    ap.add_argument("--e2e-chunks", default="ramp",
+                    help="end-to-end leg: split the batch into this many equal chunks whose host copies overlap "
+                         "the compute, or 'ramp' (chunk sizes 1:4:16:8:2:1, small at both ends; forward only)")
     ap.add_argument("--backward", action="store_true",
                     help="the dense block backward (training): its own line, not the forward metric's")
     ap.add_argument("--fp8", action="store_true",

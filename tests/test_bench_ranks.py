@@ -83,3 +83,16 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     args = argparse.Namespace(steps_ref=1, warmup=1, ref_samples=2, gpus=2)
     b.run_reference(args, S.CONFIGS["tiny_f32_dense"], rank=1)
     assert capsys.readouterr().out == ""
+
+
+def test_end_to_end_chunk_bounds():
+    """The pipelined end-to-end call's chunks: every sample in exactly one chunk, in order; the ramp
+    keeps the first and last chunks at 1/32 of the batch (the copy time left uncovered)."""
+    from token_sparse_moe_b200 import api
+    assert api.chunk_bounds(16384, api.RAMP_CHUNKS) == [0, 512, 2560, 10752, 14848, 15872, 16384]
+    assert api.chunk_bounds(8192, 8) == [1024 * i for i in range(9)]
+    assert api.chunk_bounds(10, api.RAMP_CHUNKS) == [0, 10]          # too small to split
+    assert api.chunk_bounds(4096, 1) == [0, 4096]
+    for B in (13, 100, 333, 4097):
+        b = api.chunk_bounds(B, api.RAMP_CHUNKS)
+        assert b[0] == 0 and b[-1] == B and all(x < y for x, y in zip(b, b[1:]))

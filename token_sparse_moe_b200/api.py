@@ -276,6 +276,27 @@ def stack_step(X, X_skip, block: Block, sh: A.tm_shape, Y=None, X_revert=None, w
     return Y
 
 
+# Relative chunk sizes of the pipelined end-to-end call: each chunk's host-to-device copy must end
+# before the previous chunk's compute does, and its device-to-host copy before the next chunk's
+# compute does; with a copy 4x faster than the compute per sample, chunks may grow 4x and then
+# shrink, leaving only the first copy-in and the last copy-out (1/32 of the batch each) uncovered.
+RAMP_CHUNKS = (1, 4, 16, 8, 2, 1)
+
+
+def chunk_bounds(B: int, chunks) -> List[int]:
+    """Sample boundaries [0, ..., B] of the end-to-end call's chunks: `chunks` equal ones (an int) or
+    sizes proportional to a sequence of weights; [0, B] (one chunk) when the batch is too small to
+    give every chunk two samples."""
+    weights = [1] * chunks if isinstance(chunks, int) else list(chunks)
+    if len(weights) <= 1 or B < 2 * len(weights):
+        return [0, B]
+    tot, acc, bounds = float(sum(weights)), 0.0, [0]
+    for w in weights:
+        acc += w
+        bounds.append(int(round(B * acc / tot)))
+    return sorted(set(bounds))
+
+
 class StackRunner:
     """Holds the C block array and a workspace so repeated stack forwards launch with no allocation."""
 
@@ -293,18 +314,22 @@ class StackRunner:
 
 
     def run_host(self, X_host: torch.Tensor, Y_host: torch.Tensor, X_dev: torch.Tensor, Y_dev: torch.Tensor,
-                 stream=None, chunks: int = 1) -> torch.Tensor:
+                 stream=None, chunks=1) -> torch.Tensor:
         """End to end: pinned host X -> device, stack forward, device -> pinned host Y.
 
-        chunks == 1: all on `stream`.  chunks > 1: the batch is split along the samples (which are
+        chunks == 1: all on `stream`.  Otherwise the batch is split along the samples (which are
         independent, so every output is the same bits) and pipelined over three streams: the
         host-to-device copy of chunk i+1 and the device-to-host copy of chunk i-1 run while chunk i
-        computes on `stream`.  All work of the call lies between an event recorded on `stream` at
-        entry and `stream`'s wait for the last copy, so events on `stream` around the call time
-        all of it; the next call's work on the same buffers starts only after that."""
+        computes on `stream`.  chunks: a count of equal chunks, or a sequence of relative chunk
+        sizes (RAMP_CHUNKS: small first and last chunks, so that little copy time is left
+        uncovered at either end, and large ones between, so that few launches run on small
+        batches).  All work of the call lies between an event recorded on `stream` at entry and
+        `stream`'s wait for the last copy, so events on `stream` around the call time all of it;
+        the next call's work on the same buffers starts only after that."""
         s = torch.cuda.current_stream() if stream is None else stream
         B = X_host.shape[0]
-        if chunks <= 1 or B < 2 * chunks:
+        bounds = chunk_bounds(B, chunks)
+        if len(bounds) <= 2:
             with torch.cuda.stream(s):
                 X_dev.copy_(X_host, non_blocking=True)
                 self(X_dev, Y_dev, s)
@@ -313,7 +338,7 @@ class StackRunner:
         if not hasattr(self, "_pipe"):
             self._pipe = (torch.cuda.Stream(device=X_dev.device), torch.cuda.Stream(device=X_dev.device))
         h2d, d2h = self._pipe
-        bounds = [B * i // chunks for i in range(chunks + 1)]
+        chunks = len(bounds) - 1
         start = torch.cuda.Event()
         start.record(s)
         h2d.wait_event(start)

@@ -521,6 +521,53 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const T* __restrict__
     }
 }
 
+// The same copy for bf16 rows of width <= 256 * NP whose head segments hold whole 16-byte pieces:
+// each warp takes two source rows at a time and issues all their loads (bucket positions, row
+// pieces) before any store, with NP and the bucket positions held (KMAX >= k) as template
+// constants so that the registers hold only what the rows need.
+template <int NP, int KMAX>
+__global__ void __launch_bounds__(256) scatter_rows_vec_kernel(const __nv_bfloat16* __restrict__ x, RowMap m, int B,
+                                                               int k, const int32_t* __restrict__ slot_of, int routed,
+                                                               __nv_bfloat16* __restrict__ out) {
+    constexpr int R = 2;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int W = m.W, banks = m.banks, rows = B * banks;
+    for (int row0 = warp * R; row0 < rows; row0 += nwarps * R) {
+        int pos[R][KMAX];
+        uint4 v[R][NP];
+#pragma unroll
+        for (int rr = 0; rr < R; ++rr) {
+            const int row = row0 + rr;
+            const bool ok = row < rows;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) pos[rr][j] = (ok && j < k) ? __ldg(&slot_of[(size_t)row * k + j]) : -1;
+            const int b = ok ? row / banks : 0, bank = ok ? row - b * banks : 0;
+#pragma unroll
+            for (int i = 0; i < NP; ++i) {
+                const int c = lane * 8 + 256 * i;
+                if (ok && c < W) v[rr][i] = __ldg(reinterpret_cast<const uint4*>(x + row_elem(m, b, bank, c)));
+            }
+        }
+#pragma unroll
+        for (int rr = 0; rr < R; ++rr) {
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                if (j < k && row0 + rr < rows && (pos[rr][j] < 0 || pos[rr][j] >= routed)) {
+                    if (lane == 0) record_error(ERR_BOUNDS, 0x521);
+                    pos[rr][j] = -1;
+                }
+                if (pos[rr][j] < 0) continue;
+#pragma unroll
+                for (int i = 0; i < NP; ++i) {
+                    const int c = lane * 8 + 256 * i;
+                    if (c < W) *reinterpret_cast<uint4*>(out + (size_t)pos[rr][j] * W + c) = v[rr][i];
+                }
+            }
+        }
+    }
+}
+
 // Router weights for the tensor-core router: each fp32 weight (times the RMSNorm gain) split
 // exactly into three bf16 parts, hi = bf16(v), mid = bf16(v - hi), lo = bf16(v - hi - mid) (each
 // difference is exact in fp32; hi + mid + lo matches v to about 2^-24 relative), stored as rows
@@ -667,6 +714,20 @@ cudaError_t launch_router_split(int dtype, const float* w_router, const void* ga
 cudaError_t launch_scatter_rows(int dtype, const void* x, RowMap m, int B, int k, const int32_t* slot_of, size_t routed,
                                 void* out, cudaStream_t st) {
     ProfileScope ps_("moe_permute", st);
+    const int np = (m.W + 255) / 256, kmax = k <= 2 ? 2 : k <= 4 ? 4 : 8;
+    if (dtype == 1 && (m.layout == 0 || m.dh % 8 == 0) && m.W % 8 == 0 && np <= 4 && k >= 1 && k <= 8) {
+        const int gv = grid_for(((size_t)B * m.banks + 1) / 2 * 32, 256);
+#define SLAUNCH(NP, KM)                                                                                               \
+        if (np == NP && kmax == KM) {                                                                                 \
+            scatter_rows_vec_kernel<NP, KM><<<gv, 256, 0, st>>>((const __nv_bfloat16*)x, m, B, k, slot_of, (int)routed, \
+                                                               (__nv_bfloat16*)out);                                  \
+            return cudaGetLastError();                                                                                \
+        }
+#define SLAUNCH_NP(NP) SLAUNCH(NP, 2) SLAUNCH(NP, 4) SLAUNCH(NP, 8)
+        SLAUNCH_NP(1) SLAUNCH_NP(2) SLAUNCH_NP(3) SLAUNCH_NP(4)
+#undef SLAUNCH_NP
+#undef SLAUNCH
+    }
     const int grid = grid_for((size_t)B * m.banks * 32, 256);
     if (dtype == 1)
         scatter_rows_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, m, B, k, slot_of, (int)routed,
