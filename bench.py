@@ -535,7 +535,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     # the backward step's inputs are X and dY (both copied in), its result dX (copied back)
     dYh = dY.cpu().pin_memory() if args.backward else None
     chunks = (api.RAMP_CHUNKS if args.e2e_chunks == "ramp" else int(args.e2e_chunks)) \
-        if not (args.backward or args.fp8) else 1
+        if not args.backward and isinstance(run, (api.StackRunner, api.Fp8StackRunner)) else 1
     if args.backward:
         host = lambda: run.run_host(Xh, Yh, Xd, Y, dYh, stream)
     elif chunks != 1:

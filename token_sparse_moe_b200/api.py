@@ -8,7 +8,7 @@ from __future__ import annotations
 
 import ctypes
 from dataclasses import dataclass, field
-from typing import Dict, List, Optional, Sequence
+from typing import Callable, Dict, List, Optional, Sequence
 
 import numpy as np
 import torch
@@ -297,6 +297,60 @@ def chunk_bounds(B: int, chunks) -> List[int]:
     return sorted(set(bounds))
 
 
+def run_host_pipelined(owner, run_rows: Callable, X_host: torch.Tensor, Y_host: torch.Tensor, X_dev: torch.Tensor,
+                       Y_dev: torch.Tensor, stream=None, chunks=1) -> torch.Tensor:
+    """End to end: pinned host X -> device, forward, device -> pinned host Y; run_rows(a, b, stream)
+    runs the forward on samples a .. b-1 of X_dev into Y_dev.
+
+    chunks == 1: all on `stream`.  Otherwise the batch is split along the samples (which are
+    independent, so every output is the same bits) and pipelined over three streams: the
+    host-to-device copy of chunk i+1 and the device-to-host copy of chunk i-1 run while chunk i
+    computes on `stream`.  chunks: a count of equal chunks, or a sequence of relative chunk sizes
+    (RAMP_CHUNKS: small first and last chunks, so that little copy time is left uncovered at either
+    end, and large ones between, so that few launches run on small batches).  All work of the call
+    lies between an event recorded on `stream` at entry and `stream`'s wait for the last copy, so
+    events on `stream` around the call time all of it; the next call's work on the same buffers
+    starts only after that.  owner keeps the two copy streams between calls."""
+    s = torch.cuda.current_stream() if stream is None else stream
+    B = X_host.shape[0]
+    bounds = chunk_bounds(B, chunks)
+    if len(bounds) <= 2:
+        with torch.cuda.stream(s):
+            X_dev.copy_(X_host, non_blocking=True)
+            run_rows(0, B, s)
+            Y_host.copy_(Y_dev, non_blocking=True)
+        return Y_host
+    if not hasattr(owner, "_pipe"):
+        owner._pipe = (torch.cuda.Stream(device=X_dev.device), torch.cuda.Stream(device=X_dev.device))
+    h2d, d2h = owner._pipe
+    n = len(bounds) - 1
+    start = torch.cuda.Event()
+    start.record(s)
+    h2d.wait_event(start)
+    done_in, done_out = [], []
+    for i in range(n):
+        a, b = bounds[i], bounds[i + 1]
+        with torch.cuda.stream(h2d):
+            X_dev[a:b].copy_(X_host[a:b], non_blocking=True)
+            e = torch.cuda.Event()
+            e.record(h2d)
+            done_in.append(e)
+    for i in range(n):
+        a, b = bounds[i], bounds[i + 1]
+        s.wait_event(done_in[i])
+        run_rows(a, b, s)
+        e = torch.cuda.Event()
+        e.record(s)
+        d2h.wait_event(e)
+        with torch.cuda.stream(d2h):
+            Y_host[a:b].copy_(Y_dev[a:b], non_blocking=True)
+            e2 = torch.cuda.Event()
+            e2.record(d2h)
+            done_out.append(e2)
+    s.wait_event(done_out[-1])
+    return Y_host
+
+
 class StackRunner:
     """Holds the C block array and a workspace so repeated stack forwards launch with no allocation."""
 
@@ -315,57 +369,12 @@ class StackRunner:
 
     def run_host(self, X_host: torch.Tensor, Y_host: torch.Tensor, X_dev: torch.Tensor, Y_dev: torch.Tensor,
                  stream=None, chunks=1) -> torch.Tensor:
-        """End to end: pinned host X -> device, stack forward, device -> pinned host Y.
-
-        chunks == 1: all on `stream`.  Otherwise the batch is split along the samples (which are
-        independent, so every output is the same bits) and pipelined over three streams: the
-        host-to-device copy of chunk i+1 and the device-to-host copy of chunk i-1 run while chunk i
-        computes on `stream`.  chunks: a count of equal chunks, or a sequence of relative chunk
-        sizes (RAMP_CHUNKS: small first and last chunks, so that little copy time is left
-        uncovered at either end, and large ones between, so that few launches run on small
-        batches).  All work of the call lies between an event recorded on `stream` at entry and
-        `stream`'s wait for the last copy, so events on `stream` around the call time all of it;
-        the next call's work on the same buffers starts only after that."""
-        s = torch.cuda.current_stream() if stream is None else stream
-        B = X_host.shape[0]
-        bounds = chunk_bounds(B, chunks)
-        if len(bounds) <= 2:
-            with torch.cuda.stream(s):
-                X_dev.copy_(X_host, non_blocking=True)
-                self(X_dev, Y_dev, s)
-                Y_host.copy_(Y_dev, non_blocking=True)
-            return Y_host
-        if not hasattr(self, "_pipe"):
-            self._pipe = (torch.cuda.Stream(device=X_dev.device), torch.cuda.Stream(device=X_dev.device))
-        h2d, d2h = self._pipe
-        chunks = len(bounds) - 1
-        start = torch.cuda.Event()
-        start.record(s)
-        h2d.wait_event(start)
-        done_in, done_out = [], []
-        for i in range(chunks):
-            a, b = bounds[i], bounds[i + 1]
-            with torch.cuda.stream(h2d):
-                X_dev[a:b].copy_(X_host[a:b], non_blocking=True)
-                e = torch.cuda.Event()
-                e.record(h2d)
-                done_in.append(e)
-        for i in range(chunks):
-            a, b = bounds[i], bounds[i + 1]
-            s.wait_event(done_in[i])
+        """End to end through tm_stack_forward, pipelined in sample chunks (run_host_pipelined)."""
+        def rows(a, b, s):
             sh = A.tm_shape(b - a, self.sh.T, self.sh.D, self.sh.H, self.sh.dtype, self.sh.eps)
             A.check(lib().tm_stack_forward(_p(X_dev[a:b]), self.arr, len(self.blocks), self.gap, ctypes.byref(sh),
                                            _p(Y_dev[a:b]), _p(self.ws), self.ws.numel(), _s(s)), "tm_stack_forward")
-            e = torch.cuda.Event()
-            e.record(s)
-            d2h.wait_event(e)
-            with torch.cuda.stream(d2h):
-                Y_host[a:b].copy_(Y_dev[a:b], non_blocking=True)
-                e2 = torch.cuda.Event()
-                e2.record(d2h)
-                done_out.append(e2)
-        s.wait_event(done_out[-1])
-        return Y_host
+        return run_host_pipelined(self, rows, X_host, Y_host, X_dev, Y_dev, stream, chunks)
 
 
 def stack_forward(X, blocks: Sequence[Block], gap: int, sh: A.tm_shape, Y=None, stream=None):
@@ -632,28 +641,31 @@ class Fp8StackRunner:
         self.xr = torch.empty(tok, dtype=torch.bfloat16, device=device)
         self.hist = [torch.empty(tok, dtype=torch.bfloat16, device=device) for _ in range(L - 1)]
 
-    def _sub(self, x, resid, extra, layout, c, y, stream):
-        A.check(lib().tm_sublayer_forward_fp8(_p(x), _p(resid), _p(extra), layout, ctypes.byref(self.sh),
+    def _sub(self, sh, x, resid, extra, layout, c, y, stream):
+        A.check(lib().tm_sublayer_forward_fp8(_p(x), _p(resid), _p(extra), layout, ctypes.byref(sh),
                                               ctypes.byref(c), _p(y), _p(self.ws), self.ws.numel(), _s(stream)),
                 "tm_sublayer_forward_fp8")
 
-    def __call__(self, X: torch.Tensor, Y: torch.Tensor, stream=None) -> torch.Tensor:
+    def rows(self, X: torch.Tensor, Y: torch.Tensor, a: int, b: int, stream=None) -> None:
+        """The stack on samples a .. b-1 of X into Y (the intermediates use the same rows)."""
         L = len(self.cs)
-        xs = [X] + self.hist + [Y]
+        sh = A.tm_shape(b - a, self.sh.T, self.sh.D, self.sh.H, self.sh.dtype, self.sh.eps)
+        xs = [X[a:b]] + [h[a:b] for h in self.hist] + [Y[a:b]]
+        xr = self.xr[a:b]
         for l in range(1, L + 1):
             cm, cr = self.cs[l - 1]
-            self._sub(xs[l - 1], xs[l - 1], None, A.TM_LAYOUT_MIXED, cm, self.xr, stream)
+            self._sub(sh, xs[l - 1], xs[l - 1], None, A.TM_LAYOUT_MIXED, cm, xr, stream)
             skip = xs[l - self.gap] if (self.gap > 0 and l % self.gap == 0 and l < L) else None
-            self._sub(self.xr, xs[l - 1], skip, A.TM_LAYOUT_ROWS, cr, xs[l], stream)
+            self._sub(sh, xr, xs[l - 1], skip, A.TM_LAYOUT_ROWS, cr, xs[l], stream)
+
+    def __call__(self, X: torch.Tensor, Y: torch.Tensor, stream=None) -> torch.Tensor:
+        self.rows(X, Y, 0, X.shape[0], stream)
         return Y
 
-    def run_host(self, X_host, Y_host, X_dev, Y_dev, stream=None):
-        s = torch.cuda.current_stream() if stream is None else stream
-        with torch.cuda.stream(s):
-            X_dev.copy_(X_host, non_blocking=True)
-            self(X_dev, Y_dev, s)
-            Y_host.copy_(Y_dev, non_blocking=True)
-        return Y_host
+    def run_host(self, X_host, Y_host, X_dev, Y_dev, stream=None, chunks=1):
+        """End to end, pipelined in sample chunks (run_host_pipelined)."""
+        return run_host_pipelined(self, lambda a, b, s: self.rows(X_dev, Y_dev, a, b, s), X_host, Y_host, X_dev,
+                                  Y_dev, stream, chunks)
 
 
 def _grads_c(grads: Dict[str, torch.Tensor]) -> A.tm_swiglu_grads:

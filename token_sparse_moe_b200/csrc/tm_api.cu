@@ -240,11 +240,11 @@ int dense_grid(const GemmParams& p) {
 bool env_is(const char* name, char v);
 
 // CTA pairs (M = 256 per tile, each SM streaming half of the weight rows) for the combine of bf16
-// rows: the kernel that streams the most weight rows per tile (the shared expert's down projection
-// beside its k + 1 source slabs) measured 7-10% faster so on the MoE stacks, while GEMM1 measured
-// the same and the routed GEMM2, whose epilogue bounds it, slower (a pair waits for the slower of
-// its two epilogues).  TM_PAIR=0 in the environment keeps one CTA per tile: the tests use it to show
-// that both forms give the same bits.
+// rows and the MoE shared expert's GEMM1: the combine (the shared expert's down projection beside
+// its k + 1 source slabs) measured 7-10% faster so on the MoE stacks, the shared GEMM1 of the large
+// stack up to 20%; the routed GEMM2, whose epilogue bounds it, was slower (a pair waits for the
+// slower of its two epilogues).  TM_PAIR=0 in the environment keeps one CTA per tile: the tests use
+// it to show that both forms give the same bits.
 bool use_pair(const Geo& g, int amode) {
     return g.dtype == TM_BF16 && amode != A_GATHER && !env_is("TM_PAIR", '0');
 }
@@ -289,7 +289,10 @@ tm_status gemm1_dense(const Geo& g, const void* x, const void* wg, const void* w
     if (!map_2d(&mg, wg, (uint64_t)g.banks * F, g.W, bn / 2) || !map_2d(&mu, wu, (uint64_t)g.banks * F, g.W, bn / 2) ||
         !map_2d(&mo, hidden, (uint64_t)g.banks * g.B, F, 32))
         return TM_ERR_CUDA;
-    return cuda_status(launch_grouped_gemm(bn, am, epi, ma, mg, mu, p, dense_grid(p), st, &mo));
+    // CTA pairs when the row factors come in (the MoE shared expert): measured 20% faster for the
+    // large stack's mixing shared GEMM1; the statistics warps of EPI_SWIGLU_NORM need the single form
+    const bool pair = use_pair(g, am) && epi == EPI_SWIGLU;
+    return cuda_status(launch_grouped_gemm(bn, am, epi, ma, mg, mu, p, sched0_grid(p, pair), st, &mo, pair));
 }
 
 // GEMM2 over dense hidden rows [banks*B, F] with the residual / combine epilogue into y (omap).

@@ -158,7 +158,9 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
     X(256, A_TMA_2D, EPI_SLOT_PERM, 0) X(192, A_TMA_2D, EPI_SLOT_PERM, 0) X(128, A_TMA_2D, EPI_SLOT_PERM, 0) \
     X(256, A_TMA_2D, EPI_SUM, 0) X(192, A_TMA_2D, EPI_SUM, 0) X(128, A_TMA_2D, EPI_SUM, 0) \
     X(64, A_TMA_3D, EPI_ROUTE, 0) X(64, A_TMA_MIX, EPI_ROUTE, 0) \
-    X(256, A_TMA_2D, EPI_SUM, 1) X(192, A_TMA_2D, EPI_SUM, 1) X(128, A_TMA_2D, EPI_SUM, 1)
+    X(256, A_TMA_2D, EPI_SUM, 1) X(192, A_TMA_2D, EPI_SUM, 1) X(128, A_TMA_2D, EPI_SUM, 1) \
+    X(256, A_TMA_3D, EPI_SWIGLU, 1) X(128, A_TMA_3D, EPI_SWIGLU, 1) \
+    X(256, A_TMA_MIX, EPI_SWIGLU, 1) X(128, A_TMA_MIX, EPI_SWIGLU, 1)
 
 cudaError_t launch_grouped_gemm_src(int bn, int a_mode, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                                     const CUtensorMap& tmB1, const CUtensorMap& tmS0, const CUtensorMap& tmS1,

@@ -130,6 +130,8 @@ struct GemmCfg {
                                           ? EPI_WARPS * 4096 : 0;
     // the row-statistics warps (6-9) of the router and of GEMM1 with the norm in the kernel
     static constexpr bool STATS = EPI == EPI_ROUTE || EPI == EPI_SWIGLU_NORM;
+    static_assert(!(PAIR && STATS), "the statistics warps wait on this CTA's own stage barriers, which the "
+                                    "pair-mode loads (completing on the leader's) never complete");
     // pair mode: as many stages as the shared memory holds, at most 8
     static constexpr int PAIR_STAGES_ = (232448 - 2304 - STG_BYTES_) / STAGE_BYTES;
     static constexpr int STAGES = PAIR ? (PAIR_STAGES_ > 8 ? 8 : PAIR_STAGES_)
