@@ -663,7 +663,7 @@ def main():
                     help="run the workload with this many blocks (small cases for profiler captures)")
     ap.add_argument("--e2e-chunks", default="ramp",
                     help="end-to-end leg: split the batch into this many equal chunks whose host copies overlap "
-                         "the compute, or 'ramp' (chunk sizes 1:4:16:8:2:1, small at both ends; forward only)")
+                         "the compute, or 'ramp' (chunk sizes 1:3:8:3:1, small at both ends; forward only)")
     ap.add_argument("--backward", action="store_true",
                     help="the dense block backward (training): its own line, not the forward metric's")
     ap.add_argument("--fp8", action="store_true",

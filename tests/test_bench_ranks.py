@@ -87,11 +87,11 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
 
 def test_end_to_end_chunk_bounds():
     """The pipelined end-to-end call's chunks: every sample in exactly one chunk, in order; the ramp
-    keeps the first and last chunks at 1/32 of the batch (the copy time left uncovered)."""
+    keeps the first and last chunks at 1/16 of the batch (the copy time left uncovered)."""
     from token_sparse_moe_b200 import api
-    assert api.chunk_bounds(16384, api.RAMP_CHUNKS) == [0, 512, 2560, 10752, 14848, 15872, 16384]
+    assert api.chunk_bounds(16384, api.RAMP_CHUNKS) == [0, 1024, 4096, 12288, 15360, 16384]
     assert api.chunk_bounds(8192, 8) == [1024 * i for i in range(9)]
-    assert api.chunk_bounds(10, api.RAMP_CHUNKS) == [0, 10]          # too small to split
+    assert api.chunk_bounds(9, api.RAMP_CHUNKS) == [0, 9]            # too small to split
     assert api.chunk_bounds(4096, 1) == [0, 4096]
     for B in (13, 100, 333, 4097):
         b = api.chunk_bounds(B, api.RAMP_CHUNKS)
