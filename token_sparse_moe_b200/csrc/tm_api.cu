@@ -289,8 +289,9 @@ tm_status gemm1_dense(const Geo& g, const void* x, const void* wg, const void* w
     if (!map_2d(&mg, wg, (uint64_t)g.banks * F, g.W, bn / 2) || !map_2d(&mu, wu, (uint64_t)g.banks * F, g.W, bn / 2) ||
         !map_2d(&mo, hidden, (uint64_t)g.banks * g.B, F, 32))
         return TM_ERR_CUDA;
-    // CTA pairs when the row factors come in (the MoE shared expert): measured 20% faster for the
-    // large stack's mixing shared GEMM1; the statistics warps of EPI_SWIGLU_NORM need the single form
+    // CTA pairs when the row factors come in (the MoE shared expert): up to 20% faster on the large
+    // stack.  With the row statistics in the kernel the pair form has to relay each stage's arrival
+    // to the peer's statistics warps, which measured 1.85x slower: the dense path keeps one CTA.
     const bool pair = use_pair(g, am) && epi == EPI_SWIGLU;
     return cuda_status(launch_grouped_gemm(bn, am, epi, ma, mg, mu, p, sched0_grid(p, pair), st, &mo, pair));
 }
