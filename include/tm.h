@@ -148,6 +148,20 @@ TM_API tm_status tm_model_forward(const void *groups, const void *w_group, const
                                   const tm_shape *shape, float *logits, void *workspace, size_t workspace_bytes,
                                   void *stream);
 
+/* Token Parallel ([digest] 2.5.3) exchange layouts.  Over P ranks, rank p holds the tokens
+ * p*Tp .. (p+1)*Tp-1 (Tp = T/P) for the reverting sub-layer and the head columns p*Dp .. (p+1)*Dp-1
+ * (Dp = D/P, whole heads) for the mixing sub-layer; an all-to-all buffer E [P][B][Tp][Dp] holds in
+ * chunk q the part for (sending) or from (receiving) rank q.  local_layout TM_TP_TOKEN_SHARD: the
+ * local tensor is the rank's token shard [B][Tp][D] = [B][Tp][P][Dp] (chunk q = the columns of rank
+ * q's heads); TM_TP_HEAD_SHARD: the rank's head-column shard of every token [B][T][Dp] = [B][P][Tp][Dp]
+ * (chunk q = rank q's tokens).  to_exchange != 0 copies local (src) -> E (dst), else E (src) ->
+ * local (dst).  A pure permutation (bit-exact); src and dst device memory, not overlapping, 16-byte
+ * aligned when Dp * element size is a multiple of 16. */
+#define TM_TP_TOKEN_SHARD 0
+#define TM_TP_HEAD_SHARD 1
+TM_API tm_status tm_tp_exchange_layout(const void *src, void *dst, int P, int B, int Tp, int Dp, tm_dtype dtype,
+                                       int local_layout, int to_exchange, void *stream);
+
 /* Revert ([digest] 2.3.1, Eq. 13-15), the inverse of Mix: Hm [B,H,T*D/H] -> X [B,T,D]. */
 TM_API tm_status tm_revert(const void *Hm, void *X, const tm_shape *shape, void *stream);
 

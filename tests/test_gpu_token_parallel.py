@@ -37,3 +37,23 @@ def test_token_parallel_shards_reproduce_the_stack(cfg, P):
     api.get_device_error()
     Yp = torch.cat(ys, dim=1)
     assert torch.equal(Yp.view(torch.int16), Y.view(torch.int16))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("T,D,H,P", [(16, 256, 16, 4), (6, 12, 3, 3), (48, 768, 48, 2), (10, 40, 10, 5)])
+def test_exchange_layouts_match_the_host_permutation(T, D, H, P, dtype):
+    """tm_tp_exchange_layout in all four uses against the host permutation, bit for bit (16-byte
+    pieces when a chunk row is a multiple of 16 bytes, single elements otherwise)."""
+    from test_token_parallel import HostLayouts
+    plan = TP.ShardPlan(T, D, H, P)
+    B = 37
+    g = torch.Generator().manual_seed(T * 1000 + D)
+    x = torch.randn((B, plan.Tp, D), generator=g).to(dtype)
+    r = torch.randn((B, T, plan.Dp), generator=g).to(dtype)
+    e = torch.randn((P, B, plan.Tp, plan.Dp), generator=g).to(dtype)
+    L = TP.LibraryLayouts
+    for fn, arg in (("pack_for_heads", x), ("unpack_heads", e), ("pack_for_tokens", r), ("unpack_tokens", e)):
+        want = getattr(HostLayouts, fn)(plan, arg)
+        got = getattr(L, fn)(plan, arg.to(DEV))
+        torch.cuda.synchronize()
+        assert torch.equal(got.cpu(), want), fn

@@ -18,6 +18,32 @@ from tm_synth import FFNSpec
 from token_sparse_moe_b200 import token_parallel as TP
 
 
+class HostLayouts:
+    """The four packing maps of the two exchanges as host permutations of CPU tensors (the ranks of
+    this test compute on the CPU; the library's tm_tp_exchange_layout is the device form, checked
+    against this one bit for bit in the GPU tests)."""
+
+    @staticmethod
+    def pack_for_heads(plan, x_local):
+        B = x_local.shape[0]
+        return x_local.reshape(B, plan.Tp, plan.P, plan.Dp).permute(2, 0, 1, 3).contiguous()
+
+    @staticmethod
+    def unpack_heads(plan, recv):
+        B = recv.shape[1]
+        return recv.permute(1, 0, 2, 3).reshape(B, plan.T, plan.Dp).contiguous()
+
+    @staticmethod
+    def pack_for_tokens(plan, r_local):
+        B = r_local.shape[0]
+        return r_local.reshape(B, plan.P, plan.Tp, plan.Dp).permute(1, 0, 2, 3).contiguous()
+
+    @staticmethod
+    def unpack_tokens(plan, recv):
+        B = recv.shape[1]
+        return recv.permute(1, 2, 0, 3).reshape(B, plan.Tp, plan.D).contiguous()
+
+
 class OracleStage:
     """A rank's two sub-layer computations done by the oracle (float64 torch tensors in and out)."""
 
@@ -59,7 +85,7 @@ def _rank(rank, world, kind, port, out_path):
         X = torch.from_numpy(S.to_f64(S.make_x(cfg)))
         t0, t1 = plan.tokens(rank)
         y = TP.forward_rank(OracleStage(cfg, plan, rank), plan, X[:, t0:t1].contiguous(), cfg.L, cfg.gap,
-                            TP.torch_exchange())
+                            TP.torch_exchange(), layouts=HostLayouts)
         parts = [torch.empty_like(y) for _ in range(world)]
         dist.all_gather(parts, y)
         if rank == 0:
@@ -87,15 +113,15 @@ def test_shard_plan_and_packing_round_trip():
     plan = TP.ShardPlan(T=6, D=12, H=3, P=3)
     B = 2
     X = torch.arange(B * 6 * 12, dtype=torch.float64).reshape(B, 6, 12)
-    sends = [TP.pack_for_heads(plan, X[:, slice(*plan.tokens(q))]) for q in range(3)]
+    sends = [HostLayouts.pack_for_heads(plan, X[:, slice(*plan.tokens(q))]) for q in range(3)]
     for p in range(3):
-        G = TP.unpack_heads(plan, torch.stack([sends[q][p] for q in range(3)]))
+        G = HostLayouts.unpack_heads(plan, torch.stack([sends[q][p] for q in range(3)]))
         c0, c1 = p * plan.Dp, (p + 1) * plan.Dp
         assert torch.equal(G, X[:, :, c0:c1])
     Rs = [X[:, :, p * plan.Dp:(p + 1) * plan.Dp] for p in range(3)]
-    sends = [TP.pack_for_tokens(plan, Rs[q]) for q in range(3)]
+    sends = [HostLayouts.pack_for_tokens(plan, Rs[q]) for q in range(3)]
     for p in range(3):
-        Xr = TP.unpack_tokens(plan, torch.stack([sends[q][p] for q in range(3)]))
+        Xr = HostLayouts.unpack_tokens(plan, torch.stack([sends[q][p] for q in range(3)]))
         assert torch.equal(Xr, X[:, slice(*plan.tokens(p))])
     with pytest.raises(ValueError):
         TP.ShardPlan(T=6, D=12, H=4, P=3)

@@ -11,6 +11,7 @@ TM_OK, TM_ERR_INVALID_ARG, TM_ERR_UNSUPPORTED, TM_ERR_WORKSPACE, TM_ERR_CUDA, TM
     TM_ERR_DEVICE_BOUNDS = range(7)
 TM_F32, TM_BF16 = 0, 1
 TM_LAYOUT_ROWS, TM_LAYOUT_MIXED = 0, 1
+TM_TP_TOKEN_SHARD, TM_TP_HEAD_SHARD = 0, 1
 
 # Every entry point declared in include/tm.h (the CPU test checks the library exports each one).
 EXPORTS = ["tm_status_string", "tm_version", "tm_sublayer_workspace_bytes", "tm_route_workspace_bytes",
@@ -25,7 +26,7 @@ EXPORTS = ["tm_status_string", "tm_version", "tm_sublayer_workspace_bytes", "tm_
            "tm_block_backward_workspace_bytes", "tm_block_backward", "tm_stack_backward_workspace_bytes",
            "tm_stack_backward", "tm_last_device_error_site", "tm_set_wait_limit_ns", "tm_selftest_wait",
            "tm_selftest_bucket_scatter", "tm_sublayer_fp8_workspace_bytes", "tm_sublayer_forward_fp8",
-           "tm_sparse_pertoken_moe_fp8"]
+           "tm_sparse_pertoken_moe_fp8", "tm_tp_exchange_layout"]
 
 
 class tm_shape(ctypes.Structure):
@@ -125,6 +126,7 @@ _SIGS = {
                                         _P]),
     "tm_sparse_pertoken_moe_fp8": (c_int, [_P, _P, c_int, POINTER(tm_shape), _P, POINTER(tm_moe_w8), _P, _P, c_size_t,
                                            _P]),
+    "tm_tp_exchange_layout": (c_int, [_P, _P, c_int, c_int, c_int, c_int, c_int, c_int, c_int, _P]),
     "tm_head_forward": (c_int, [_P, POINTER(tm_shape), _P, _P, _P]),
     "tm_model_workspace_bytes": (c_size_t, [POINTER(tm_shape), POINTER(tm_block), c_int, c_int]),
     "tm_model_forward": (c_int, [_P, _P, _P, c_int, POINTER(tm_block), c_int, c_int, _P, POINTER(tm_shape), _P, _P,

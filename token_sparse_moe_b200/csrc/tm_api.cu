@@ -1384,6 +1384,17 @@ tm_status tm_mix(const void* X, void* Hm, const tm_shape* shape, void* stream) {
                                       (cudaStream_t)stream));
 }
 
+tm_status tm_tp_exchange_layout(const void* src, void* dst, int P, int B, int Tp, int Dp, tm_dtype dtype,
+                                int local_layout, int to_exchange, void* stream) {
+    if (!src || !dst || src == dst || P < 1 || B < 1 || Tp < 1 || Dp < 1) return TM_ERR_INVALID_ARG;
+    if ((dtype != TM_F32 && dtype != TM_BF16) || (local_layout != TM_TP_TOKEN_SHARD && local_layout != TM_TP_HEAD_SHARD))
+        return TM_ERR_INVALID_ARG;
+    const int esz = dtype == TM_BF16 ? 2 : 4;
+    if (((size_t)Dp * esz) % 16 == 0 && (!al16(src) || !al16(dst))) return TM_ERR_INVALID_ARG;
+    return cuda_status(launch_tp_layout(src, dst, P, B, Tp, Dp, esz, local_layout == TM_TP_TOKEN_SHARD, to_exchange != 0,
+                                        (cudaStream_t)stream));
+}
+
 tm_status tm_revert(const void* Hm, void* X, const tm_shape* shape, void* stream) {
     tm_status s = check_shape(shape);
     if (s != TM_OK) return s;

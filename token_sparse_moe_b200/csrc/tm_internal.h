@@ -107,6 +107,9 @@ cudaError_t launch_quant_matrices(const void* w, const void* gain, int groups, s
 cudaError_t launch_quant_act_rows(const void* x, RowMap m, int B, float eps, uint8_t* q, float* rowscale,
                                   cudaStream_t st, const int32_t* slot_of = nullptr, int k = 0, size_t routed = 0,
                                   uint8_t* qpos = nullptr, float* scale_pos = nullptr);
+// Token Parallel: exchange buffer [P][B][Tp][Dp] <-> local [B][Tp][P][Dp] (cols_shard) or [B][P][Tp][Dp]
+cudaError_t launch_tp_layout(const void* src, void* dst, int P, int B, int Tp, int Dp, int esz, bool cols_shard,
+                             bool to_exchange, cudaStream_t st);
 cudaError_t launch_permute(int dtype, const void* src, void* dst, int B, int T, int D, int H, bool to_mixed,
                            cudaStream_t st);
 cudaError_t launch_fold_gain(int dtype, const void* w, const void* gain, void* out, size_t rows, int width,

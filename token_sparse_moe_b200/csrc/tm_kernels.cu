@@ -737,6 +737,48 @@ cudaError_t launch_scatter_rows(int dtype, const void* x, RowMap m, int B, int k
     return cudaGetLastError();
 }
 
+// Token Parallel exchange layouts: the all-to-all buffer E [P][B][Tp][Dp] (chunk q for / from rank
+// q) against a rank's local tensor, either its token shard of the full width, L [B][Tp][P][Dp]
+// (columns q * Dp .. of token t), or its head-column shard of every token, L [B][P][Tp][Dp] (token
+// q * Tp + t).  One 16-byte piece per thread when Dp * esz is a multiple of 16, else one element.
+template <typename V>
+__global__ void tp_layout_kernel(const V* __restrict__ src, V* __restrict__ dst, int P, int B, int Tp, int dv,
+                                 int cols_shard, int to_exchange) {
+    const size_t n = (size_t)P * B * Tp * dv;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        // i indexes the exchange layout: (q, b, t, j)
+        const int j = (int)(i % dv);
+        size_t r = i / dv;
+        const int t = (int)(r % Tp);
+        r /= Tp;
+        const int b = (int)(r % B);
+        const int q = (int)(r / B);
+        const size_t l = cols_shard ? (((size_t)b * Tp + t) * P + q) * dv + j : (((size_t)b * P + q) * Tp + t) * dv + j;
+        if (to_exchange) dst[i] = src[l];
+        else dst[l] = src[i];
+    }
+}
+
+cudaError_t launch_tp_layout(const void* src, void* dst, int P, int B, int Tp, int Dp, int esz, bool cols_shard,
+                             bool to_exchange, cudaStream_t st) {
+    ProfileScope ps_("tp_layout", st);
+    const size_t row = (size_t)Dp * esz;
+    if (row % 16 == 0) {
+        const int dv = (int)(row / 16);
+        tp_layout_kernel<uint4><<<grid_for((size_t)P * B * Tp * dv, 256), 256, 0, st>>>(
+            (const uint4*)src, (uint4*)dst, P, B, Tp, dv, cols_shard, to_exchange);
+    } else if (esz == 2) {
+        tp_layout_kernel<uint16_t><<<grid_for((size_t)P * B * Tp * Dp, 256), 256, 0, st>>>(
+            (const uint16_t*)src, (uint16_t*)dst, P, B, Tp, Dp, cols_shard, to_exchange);
+    } else if (esz == 4) {
+        tp_layout_kernel<uint32_t><<<grid_for((size_t)P * B * Tp * Dp, 256), 256, 0, st>>>(
+            (const uint32_t*)src, (uint32_t*)dst, P, B, Tp, Dp, cols_shard, to_exchange);
+    } else {
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t launch_permute(int dtype, const void* src, void* dst, int B, int T, int D, int H, bool to_mixed,
                            cudaStream_t st) {
     ProfileScope ps_(to_mixed ? "mix" : "revert", st);

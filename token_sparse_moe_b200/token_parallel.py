@@ -28,7 +28,10 @@ sharded stack gives the same bits as tm_stack_forward.
 
 The exchange is a callable send [P, ...] -> recv [P, ...] (chunk q of send goes to rank q; chunk q
 of recv came from rank q): torch.distributed's all_to_all_single between processes, or a local
-transpose of all ranks' chunks when every shard lives in one process.
+transpose of all ranks' chunks when every shard lives in one process.  The packing of a rank's
+tensors into the exchange layout and back is the library's tm_tp_exchange_layout (a permutation
+kernel); `layouts` may stand in another implementation of the same four maps (the CPU tests pass
+a host one, since their ranks compute on the CPU).
 """
 from __future__ import annotations
 
@@ -74,28 +77,45 @@ class ShardPlan:
 
 
 # ------------------------------------------------------------------ exchange layout
-def pack_for_heads(plan: ShardPlan, x_local: torch.Tensor) -> torch.Tensor:
-    """x_p [B, T/P, D] -> send [P, B, T/P, D/P]: chunk q = the columns of rank q's heads."""
-    B = x_local.shape[0]
-    return x_local.reshape(B, plan.Tp, plan.P, plan.Dp).permute(2, 0, 1, 3).contiguous()
+def _tp_layout(src: torch.Tensor, dst: torch.Tensor, plan: "ShardPlan", B: int, local_layout: int,
+               to_exchange: bool) -> torch.Tensor:
+    dt = A.TM_BF16 if src.dtype == torch.bfloat16 else A.TM_F32
+    A.check(api.lib().tm_tp_exchange_layout(api._p(src), api._p(dst), plan.P, B, plan.Tp, plan.Dp, dt, local_layout,
+                                            1 if to_exchange else 0, api._s(torch.cuda.current_stream())),
+            "tm_tp_exchange_layout")
+    return dst
 
 
-def unpack_heads(plan: ShardPlan, recv: torch.Tensor) -> torch.Tensor:
-    """recv [P, B, T/P, D/P] (chunk q: q's tokens) -> G_p [B, T, D/P] in token order."""
-    B = recv.shape[1]
-    return recv.permute(1, 0, 2, 3).reshape(B, plan.T, plan.Dp).contiguous()
+class LibraryLayouts:
+    """The four packing maps of the two exchanges, on the device (tm_tp_exchange_layout)."""
 
+    @staticmethod
+    def pack_for_heads(plan: "ShardPlan", x_local: torch.Tensor) -> torch.Tensor:
+        """x_p [B, T/P, D] -> send [P, B, T/P, D/P]: chunk q = the columns of rank q's heads."""
+        B = x_local.shape[0]
+        out = torch.empty((plan.P, B, plan.Tp, plan.Dp), dtype=x_local.dtype, device=x_local.device)
+        return _tp_layout(x_local.contiguous(), out, plan, B, A.TM_TP_TOKEN_SHARD, True)
 
-def pack_for_tokens(plan: ShardPlan, r_local: torch.Tensor) -> torch.Tensor:
-    """R_p [B, T, D/P] -> send [P, B, T/P, D/P]: chunk q = rank q's tokens."""
-    B = r_local.shape[0]
-    return r_local.reshape(B, plan.P, plan.Tp, plan.Dp).permute(1, 0, 2, 3).contiguous()
+    @staticmethod
+    def unpack_heads(plan: "ShardPlan", recv: torch.Tensor) -> torch.Tensor:
+        """recv [P, B, T/P, D/P] (chunk q: q's tokens) -> G_p [B, T, D/P] in token order."""
+        B = recv.shape[1]
+        out = torch.empty((B, plan.T, plan.Dp), dtype=recv.dtype, device=recv.device)
+        return _tp_layout(recv.contiguous(), out, plan, B, A.TM_TP_HEAD_SHARD, False)
 
+    @staticmethod
+    def pack_for_tokens(plan: "ShardPlan", r_local: torch.Tensor) -> torch.Tensor:
+        """R_p [B, T, D/P] -> send [P, B, T/P, D/P]: chunk q = rank q's tokens."""
+        B = r_local.shape[0]
+        out = torch.empty((plan.P, B, plan.Tp, plan.Dp), dtype=r_local.dtype, device=r_local.device)
+        return _tp_layout(r_local.contiguous(), out, plan, B, A.TM_TP_HEAD_SHARD, True)
 
-def unpack_tokens(plan: ShardPlan, recv: torch.Tensor) -> torch.Tensor:
-    """recv [P, B, T/P, D/P] (chunk q: the columns of q's heads) -> X_revert of p's tokens [B, T/P, D]."""
-    B = recv.shape[1]
-    return recv.permute(1, 2, 0, 3).reshape(B, plan.Tp, plan.D).contiguous()
+    @staticmethod
+    def unpack_tokens(plan: "ShardPlan", recv: torch.Tensor) -> torch.Tensor:
+        """recv [P, B, T/P, D/P] (chunk q: the columns of q's heads) -> X_revert of p's tokens [B, T/P, D]."""
+        B = recv.shape[1]
+        out = torch.empty((B, plan.Tp, plan.D), dtype=recv.dtype, device=recv.device)
+        return _tp_layout(recv.contiguous(), out, plan, B, A.TM_TP_TOKEN_SHARD, False)
 
 
 def skip_index(l: int, L: int, gap: int) -> Optional[int]:
@@ -131,31 +151,33 @@ class RankStage:
 
 # ------------------------------------------------------------------ drivers
 def forward_rank(stage, plan: ShardPlan, x_local: torch.Tensor, L: int, gap: int,
-                 exchange: Callable[[torch.Tensor], torch.Tensor]) -> torch.Tensor:
+                 exchange: Callable[[torch.Tensor], torch.Tensor], layouts=LibraryLayouts) -> torch.Tensor:
     """The stack on one rank: x_p [B, T/P, D] -> Y_p [B, T/P, D]; exchange(send) -> recv is the
     all-to-all between the ranks (every rank calls this with the same L and gap, so the exchanges
     pair up)."""
+    lay = layouts
     hist: List[torch.Tensor] = [x_local]
     for l in range(1, L + 1):
-        G = unpack_heads(plan, exchange(pack_for_heads(plan, hist[-1])))
+        G = lay.unpack_heads(plan, exchange(lay.pack_for_heads(plan, hist[-1])))
         R = stage.mixing(l - 1, G)
-        Xr = unpack_tokens(plan, exchange(pack_for_tokens(plan, R)))
+        Xr = lay.unpack_tokens(plan, exchange(lay.pack_for_tokens(plan, R)))
         s = skip_index(l, L, gap)
         hist.append(stage.reverting(l - 1, Xr, hist[-1], hist[s] if s is not None else None))
     return hist[-1]
 
 
 def forward_all_ranks(stages: Sequence, plan: ShardPlan, x_locals: Sequence[torch.Tensor], L: int,
-                      gap: int) -> List[torch.Tensor]:
+                      gap: int, layouts=LibraryLayouts) -> List[torch.Tensor]:
     """Every rank's share in one process (the exchange becomes a transpose of the ranks' chunks)."""
     P = plan.P
+    lay = layouts
     hist = [list(x_locals)]
     for l in range(1, L + 1):
-        sends = [pack_for_heads(plan, hist[-1][p]) for p in range(P)]
-        G = [unpack_heads(plan, torch.stack([sends[q][p] for q in range(P)])) for p in range(P)]
+        sends = [lay.pack_for_heads(plan, hist[-1][p]) for p in range(P)]
+        G = [lay.unpack_heads(plan, torch.stack([sends[q][p] for q in range(P)])) for p in range(P)]
         R = [stages[p].mixing(l - 1, G[p]) for p in range(P)]
-        sends = [pack_for_tokens(plan, R[p]) for p in range(P)]
-        Xr = [unpack_tokens(plan, torch.stack([sends[q][p] for q in range(P)])) for p in range(P)]
+        sends = [lay.pack_for_tokens(plan, R[p]) for p in range(P)]
+        Xr = [lay.unpack_tokens(plan, torch.stack([sends[q][p] for q in range(P)])) for p in range(P)]
         s = skip_index(l, L, gap)
         hist.append([stages[p].reverting(l - 1, Xr[p], hist[-1][p], hist[s][p] if s is not None else None)
                      for p in range(P)])
