@@ -211,11 +211,17 @@ __global__ void __launch_bounds__(1024) offsets_kernel(int32_t* counts, int bank
     for (int g = threadIdx.x; g < G; g += blockDim.x) {
         const int bank = g / E, e = g - bank * E;
         int run = 0;
-        for (int c = 0; c < nchunks; ++c) {
-            const size_t i = ((size_t)bank * nchunks + c) * E + e;
-            const int v = counts[i];
-            counts[i] = run;
-            run += v;
+        // sixteen chunks' counts loaded before any of them is rewritten, so the loads overlap
+        for (int c0 = 0; c0 < nchunks; c0 += 16) {
+            int v[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                v[c] = c0 + c < nchunks ? counts[((size_t)bank * nchunks + c0 + c) * E + e] : 0;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                if (c0 + c < nchunks) counts[((size_t)bank * nchunks + c0 + c) * E + e] = run;
+                run += v[c];
+            }
         }
         tot[g] = run;
     }
