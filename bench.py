@@ -16,9 +16,10 @@ Without --steps the step count is chosen from the warm-up steps' time so that th
 lasts about two seconds.  N > 1 (under torchrun): every rank runs its own batch (weak scaling,
 no data-path collective); the step time is the max over ranks.  --impl reference times the CPU
 float64 oracle on the host cores (rank 0 only) on a bounded sample of the workload.  The
-end-to-end leg copies each step's batch from pinned host memory and the result back, in C
-sample chunks pipelined against the compute (the result is checked bit for bit against the
-full-batch device run).  --batch and --layers run a smaller case of the same kernels (profiler
+end-to-end leg runs a stream of steps through the public API, each copying its batch from pinned
+host memory and its result back, the copies overlapping the neighbouring steps' compute
+(--e2e-mode step: each step alone, its copies overlapping its own compute in C sample chunks); the
+result is checked bit for bit against the full-batch device run.  --batch and --layers run a smaller case of the same kernels (profiler
 captures).  --fp8 and --backward print their own lines (the FP8 serving path, the dense block
 backward).
 """
@@ -547,18 +548,33 @@ def run_ours(args, cfg, rank, world, local_rank):
     with torch.cuda.stream(stream):
         run(X, Yref, stream)
     stream.synchronize()
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            host()
-        stream.synchronize()
-        eve = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
-        for i in range(Ke):
-            flush.zero_()
-            eve[i][0].record(stream)
-            host()
-            eve[i][1].record(stream)
-        stream.synchronize()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eve) / Ke, world, dev)
+    streamed = args.e2e_mode == "stream" and not args.backward and hasattr(run, "run_host_steps")
+    if streamed:
+        # a stream of Ke steps as a serving loop runs it: every step copies its batch in and its result
+        # out, each step's copies overlapping the neighbouring steps' compute (run_host_steps)
+        Xb, Yb = [Xd, torch.empty_like(X)], [torch.empty_like(X), torch.empty_like(X)]
+        with torch.cuda.stream(stream):
+            run.run_host_steps(Xh, Yh, Xb, Yb, 2, stream)
+            stream.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            run.run_host_steps(Xh, Yh, Xb, Yb, Ke, stream)
+            e1.record(stream)
+            stream.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, world, dev)
+    else:
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                host()
+            stream.synchronize()
+            eve = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+            for i in range(Ke):
+                flush.zero_()
+                eve[i][0].record(stream)
+                host()
+                eve[i][1].record(stream)
+            stream.synchronize()
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eve) / Ke, world, dev)
     e2e_exact = bool(torch.equal(Yh, Yref.cpu()))
     io_bytes = X.numel() * X.element_size()
     h2d_bytes = io_bytes * (2 if args.backward else 1)
@@ -629,7 +645,11 @@ def run_ours(args, cfg, rank, world, local_rank):
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(cfg.B, world, e2e_ms), "unit": "samples/s", "h2d_bytes_per_step": h2d_bytes,
                 "d2h_bytes_per_step": io_bytes, "ms_per_step": e2e_ms, "steps": Ke,
-                "chunks": list(chunks) if not isinstance(chunks, int) else chunks,
+                "mode": ("stream: Ke consecutive steps, each copying its batch in and its result out, the copies "
+                         "overlapping the neighbouring steps' compute (two device buffers each); one pair of "
+                         "events around the whole stream") if streamed else
+                        "one step at a time, its copies overlapping its own compute in sample chunks",
+                "chunks": None if streamed else (list(chunks) if not isinstance(chunks, int) else chunks),
                 "matches_device_result": e2e_exact},
         "gpu_launches": int(launches),
         "launches_per_step": launches / K,
@@ -661,6 +681,9 @@ def main():
                          "profiler captures; the line's workload string carries the B used)")
     ap.add_argument("--layers", type=int, default=None,
                     help="run the workload with this many blocks (small cases for profiler captures)")
+    ap.add_argument("--e2e-mode", choices=["stream", "step"], default="stream",
+                    help="end-to-end leg: a stream of steps whose copies overlap the neighbouring steps' compute "
+                         "(stream), or each step alone with its copies overlapping its own compute in chunks (step)")
     ap.add_argument("--e2e-chunks", default="ramp",
                     help="end-to-end leg: split the batch into this many equal chunks whose host copies overlap "
                          "the compute, or 'ramp' (chunk sizes 1:3:8:3:1, small at both ends; forward only)")

@@ -457,3 +457,32 @@ def test_workspace_too_small_is_reported():
                                        ctypes.byref(w), api._p(y), api._p(small_ws), 1024, api._s(None)), "call")
     assert e.value.status == A.TM_ERR_WORKSPACE
     api.get_device_error()
+
+
+@pytest.mark.parametrize("cfg", [MOE_SMALL[0], DENSE_SMALL[0]], ids=lambda c: c.name)
+def test_end_to_end_host_calls_give_the_device_bits(cfg):
+    """The end-to-end calls through pinned host memory: the chunked single step (equal chunks and
+    the ramp) and the stream of steps with double-buffered copies give the bits of the plain device
+    call on the same batch."""
+    c = cfg.with_(L=2, gap=1)
+    blocks = api.blocks_from_synth(c, DEV)
+    sh = api.config_shape(c)
+    run = api.StackRunner(blocks, sh, c.gap, DEV)
+    X = dev(S.make_x(c))
+    Y = torch.empty_like(X)
+    run(X, Y)
+    Xh = X.cpu().pin_memory()
+    s = torch.cuda.Stream()
+    for chunks in (1, 4, api.RAMP_CHUNKS):
+        Yh = torch.zeros_like(Xh).pin_memory()
+        with torch.cuda.stream(s):
+            run.run_host(Xh, Yh, torch.empty_like(X), torch.empty_like(X), s, chunks=chunks)
+        s.synchronize()
+        assert torch.equal(Yh.view(torch.int16), Y.cpu().view(torch.int16)), chunks
+    Yh = torch.zeros_like(Xh).pin_memory()
+    with torch.cuda.stream(s):
+        run.run_host_steps(Xh, Yh, [torch.empty_like(X), torch.empty_like(X)],
+                           [torch.empty_like(X), torch.empty_like(X)], 5, s)
+    s.synchronize()
+    api.get_device_error()
+    assert torch.equal(Yh.view(torch.int16), Y.cpu().view(torch.int16))

@@ -353,6 +353,50 @@ def run_host_pipelined(owner, run_rows: Callable, X_host: torch.Tensor, Y_host: 
     return Y_host
 
 
+def run_host_steps(owner, run_full: Callable, X_host: torch.Tensor, Y_host: torch.Tensor,
+                   X_bufs: Sequence[torch.Tensor], Y_bufs: Sequence[torch.Tensor], steps: int, stream=None) -> torch.Tensor:
+    """A stream of `steps` end-to-end steps, as a serving loop runs them: every step copies its batch
+    from pinned host memory to the device, runs the forward (run_full(X_dev, Y_dev, stream)) and copies
+    the result back, with two device buffers of each so that step i's copy-in and step i-1's copy-out
+    run on their own streams while step i-1 and step i compute.  Step i's copy-in waits for step i-2's
+    compute (which read the same buffer), step i's compute for step i-2's copy-out.  All of it lies
+    between an event recorded on `stream` at entry and `stream`'s wait for the last copy-out, so
+    events on `stream` around the call time the whole stream of steps.  Y_host holds the last step's
+    result.  owner keeps the two copy streams between calls."""
+    s = torch.cuda.current_stream() if stream is None else stream
+    if not hasattr(owner, "_pipe"):
+        owner._pipe = (torch.cuda.Stream(device=X_bufs[0].device), torch.cuda.Stream(device=X_bufs[0].device))
+    h2d, d2h = owner._pipe
+    start = torch.cuda.Event()
+    start.record(s)
+    h2d.wait_event(start)
+    d2h.wait_event(start)
+    comp, out = [], []
+    for i in range(steps):
+        b = i % 2
+        with torch.cuda.stream(h2d):
+            if i >= 2:
+                h2d.wait_event(comp[i - 2])
+            X_bufs[b].copy_(X_host, non_blocking=True)
+            e_in = torch.cuda.Event()
+            e_in.record(h2d)
+        s.wait_event(e_in)
+        if i >= 2:
+            s.wait_event(out[i - 2])
+        run_full(X_bufs[b], Y_bufs[b], s)
+        e_c = torch.cuda.Event()
+        e_c.record(s)
+        comp.append(e_c)
+        d2h.wait_event(e_c)
+        with torch.cuda.stream(d2h):
+            Y_host.copy_(Y_bufs[b], non_blocking=True)
+            e_o = torch.cuda.Event()
+            e_o.record(d2h)
+            out.append(e_o)
+    s.wait_event(out[-1])
+    return Y_host
+
+
 class StackRunner:
     """Holds the C block array and a workspace so repeated stack forwards launch with no allocation."""
 
@@ -377,6 +421,10 @@ class StackRunner:
             A.check(lib().tm_stack_forward(_p(X_dev[a:b]), self.arr, len(self.blocks), self.gap, ctypes.byref(sh),
                                            _p(Y_dev[a:b]), _p(self.ws), self.ws.numel(), _s(s)), "tm_stack_forward")
         return run_host_pipelined(self, rows, X_host, Y_host, X_dev, Y_dev, stream, chunks)
+
+    def run_host_steps(self, X_host, Y_host, X_bufs, Y_bufs, steps: int, stream=None) -> torch.Tensor:
+        """A stream of end-to-end steps, each step's copies overlapping its neighbours' compute."""
+        return run_host_steps(self, lambda x, y, s: self(x, y, s), X_host, Y_host, X_bufs, Y_bufs, steps, stream)
 
 
 def stack_forward(X, blocks: Sequence[Block], gap: int, sh: A.tm_shape, Y=None, stream=None):
@@ -621,6 +669,10 @@ class Fp8BlockRunner:
             Y_host.copy_(Y_dev, non_blocking=True)
         return Y_host
 
+    def run_host_steps(self, X_host, Y_host, X_bufs, Y_bufs, steps: int, stream=None) -> torch.Tensor:
+        """A stream of end-to-end steps, each step's copies overlapping its neighbours' compute."""
+        return run_host_steps(self, lambda x, y, s: self(x, y, s), X_host, Y_host, X_bufs, Y_bufs, steps, stream)
+
 
 class Fp8StackRunner:
     """A stack on the FP8 path, one tm_sublayer_forward_fp8 call per sub-layer, with the inter-residual
@@ -668,6 +720,10 @@ class Fp8StackRunner:
         """End to end, pipelined in sample chunks (run_host_pipelined)."""
         return run_host_pipelined(self, lambda a, b, s: self.rows(X_dev, Y_dev, a, b, s), X_host, Y_host, X_dev,
                                   Y_dev, stream, chunks)
+
+    def run_host_steps(self, X_host, Y_host, X_bufs, Y_bufs, steps: int, stream=None) -> torch.Tensor:
+        """A stream of end-to-end steps, each step's copies overlapping its neighbours' compute."""
+        return run_host_steps(self, lambda x, y, s: self(x, y, s), X_host, Y_host, X_bufs, Y_bufs, steps, stream)
 
 
 def _grads_c(grads: Dict[str, torch.Tensor]) -> A.tm_swiglu_grads:
