@@ -1,4 +1,5 @@
-"""FP8 E4M3 serving path of the dense per-token SwiGLU FFN: the float64 oracle.
+"""FP8 E4M3 serving path of the per-token FFNs (dense SwiGLU banks and Sparse-Pertoken MoE banks):
+the float64 oracle.
 
 TEST INFRASTRUCTURE ONLY, like the rest of this package: imported by the tests, the smoke
 check and the benchmark's CPU leg, never by the library, and sharing no code or table with it.
@@ -29,6 +30,10 @@ quantization of a model trained in bf16.  The page names the format only; the re
     up_n likewise, with rms taken over the unquantized row exactly as in the bf16 path.  The
     SwiGLU, the down projection and the residual are those of the bf16 path (the down
     projection keeps its bf16 weights): GEMM1 carries two thirds of the FFN's flops.
+  * MoE banks: every expert (the k routed ones a row reaches and the shared one) is such an FFN,
+    its gate and up matrices quantized with one scale each (per (bank, expert)); a row is
+    quantized once for all of them; the router is not quantized, so the routing (top-k, gates
+    alpha * p) is the bf16 path's.
 """
 from __future__ import annotations
 
