@@ -41,6 +41,8 @@ CASES = [
     small("fp8moe_ns", 260, 8, 384, 4, moe(16, 4, 128, 256), moe(6, 3, 256, 128)),
     # 24 experts: the CUDA-core router
     small("fp8moe_e24", 170, 8, 256, 8, moe(24, 3, 128, 128), moe(24, 2, 128, 128)),
+    # degenerate routing: k = E (every row reaches every expert) and a single expert
+    small("fp8moe_kE", 200, 8, 256, 8, moe(4, 4, 128, 128, 1.0), moe(1, 1, 128, 128, 2.0)),
 ]
 
 

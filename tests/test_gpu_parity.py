@@ -486,3 +486,40 @@ def test_end_to_end_host_calls_give_the_device_bits(cfg):
     s.synchronize()
     api.get_device_error()
     assert torch.equal(Yh.view(torch.int16), Y.cpu().view(torch.int16))
+
+
+MOE_DEGENERATE = [
+    # k = E: every row reaches every expert (the dense softmax mixture of [digest] Eq. 19 with alpha = 1)
+    small("moe_k_eq_E", 200, 8, 256, 8, "bf16", moe(4, 4, 128, 128, 1.0), moe(3, 3, 64, 128, 1.0)),
+    # one expert, top-1: softmax over one logit is 1, so the gate is alpha for every row
+    small("moe_E1", 170, 8, 256, 8, "bf16", moe(1, 1, 128, 128, 2.0), moe(1, 1, 128, 64, 2.0)),
+]
+
+
+@pytest.mark.parametrize("sub", [0, 1])
+@pytest.mark.parametrize("cfg", MOE_DEGENERATE, ids=lambda c: c.name)
+def test_moe_degenerate_routing(cfg, sub):
+    """The routing's degenerate cases, every row of the sub-layer against the oracle: k = E (no
+    choice is made, every bucket holds all rows) and E = 1; the GPU's expert sets equal the oracle's
+    (no near tie can change a set that contains every expert)."""
+    X, R = inputs(cfg)
+    sw = api.sublayer_from_synth(cfg, 0, sub, DEV, 1.0)
+    sh = api.config_shape(cfg)
+    layout = A.TM_LAYOUT_MIXED if sub == 0 else A.TM_LAYOUT_ROWS
+    r = api.route_topk(dev(X), layout, sh, sw)
+    y = to_np(api.sparse_pertoken_moe(dev(X), dev(R), layout, sh, sw))
+    api.get_device_error()
+    spec = cfg.ffn(sub)
+    assert spec.k == spec.E
+    gi = np.sort(r["idx"].cpu().numpy(), -1)
+    assert np.array_equal(gi, np.broadcast_to(np.arange(spec.E), gi.shape))     # every expert, every row
+    assert np.all(np.isinf(r["gap"].cpu().numpy()))                            # no expert left out
+    X64, R64 = S.to_f64(X), S.to_f64(R)
+    rows = O.mix(X64, cfg.H) if sub == 0 else X64
+    res = R64 if sub == 1 else O.mix(R64, cfg.H)
+    o = oracle_sublayer(cfg, 0, sub, rows, 1.0)["out"] + res
+    c = routed_abs_contrib(cfg, 0, sub, rows, 1.0)
+    if sub == 0:
+        o, c = O.revert(o, cfg.T), O.revert(c, cfg.T)
+    e = err_moe_delta(y, o, R64, c, cfg.dtype)
+    assert e <= tol(cfg.dtype), e
