@@ -57,3 +57,25 @@ def test_exchange_layouts_match_the_host_permutation(T, D, H, P, dtype):
         got = getattr(L, fn)(plan, arg.to(DEV))
         torch.cuda.synchronize()
         assert torch.equal(got.cpu(), want), fn
+
+
+def test_rank_stage_runs_sample_chunks():
+    """A rank's sub-layers on a chunk of its samples (the overlapped schedule's unit of work) give
+    the bits of the same rows in the whole-batch call."""
+    cfg = CASES[0]
+    blocks = api.blocks_from_synth(cfg, DEV)
+    sh = api.config_shape(cfg)
+    plan = TP.ShardPlan(cfg.T, cfg.D, cfg.H, 2)
+    st = TP.RankStage(blocks, plan, 1, sh, DEV)
+    g = torch.Generator().manual_seed(5)
+    G = torch.randn((cfg.B, plan.T, plan.Dp), generator=g).to(torch.bfloat16).to(DEV)
+    Xr = torch.randn((cfg.B, plan.Tp, plan.D), generator=g).to(torch.bfloat16).to(DEV)
+    x = torch.randn((cfg.B, plan.Tp, plan.D), generator=g).to(torch.bfloat16).to(DEV)
+    R = st.mixing(0, G).clone()
+    Y = st.reverting(0, Xr, x, None).clone()
+    a, b = 37, 211
+    Rc = st.mixing(0, G[a:b].contiguous())
+    Yc = st.reverting(0, Xr[a:b].contiguous(), x[a:b].contiguous(), None)
+    api.get_device_error()
+    assert torch.equal(Rc.view(torch.int16), R[a:b].view(torch.int16))
+    assert torch.equal(Yc.view(torch.int16), Y[a:b].view(torch.int16))

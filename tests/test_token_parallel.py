@@ -74,7 +74,7 @@ def _cfg(kind):
                     mix=FFNSpec("dense", hidden=32), rev=FFNSpec("dense", hidden=16))
 
 
-def _rank(rank, world, kind, port, out_path):
+def _rank(rank, world, kind, port, out_path, overlapped=False):
     import torch.distributed as dist
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
@@ -84,8 +84,12 @@ def _rank(rank, world, kind, port, out_path):
         plan = TP.ShardPlan(cfg.T, cfg.D, cfg.H, world)
         X = torch.from_numpy(S.to_f64(S.make_x(cfg)))
         t0, t1 = plan.tokens(rank)
-        y = TP.forward_rank(OracleStage(cfg, plan, rank), plan, X[:, t0:t1].contiguous(), cfg.L, cfg.gap,
-                            TP.torch_exchange(), layouts=HostLayouts)
+        if overlapped:
+            y = TP.forward_rank_overlapped(OracleStage(cfg, plan, rank), plan, X[:, t0:t1].contiguous(), cfg.L,
+                                           cfg.gap, TP.torch_exchange_async(), chunks=3, layouts=HostLayouts)
+        else:
+            y = TP.forward_rank(OracleStage(cfg, plan, rank), plan, X[:, t0:t1].contiguous(), cfg.L, cfg.gap,
+                                TP.torch_exchange(), layouts=HostLayouts)
         parts = [torch.empty_like(y) for _ in range(world)]
         dist.all_gather(parts, y)
         if rank == 0:
@@ -94,12 +98,15 @@ def _rank(rank, world, kind, port, out_path):
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("overlapped", [False, True], ids=["plain", "overlapped"])
 @pytest.mark.parametrize("kind", ["moe", "dense"])
-def test_token_parallel_two_ranks_equal_the_unsharded_stack(kind, tmp_path):
+def test_token_parallel_two_ranks_equal_the_unsharded_stack(kind, overlapped, tmp_path):
+    """Also with the exchanges issued asynchronously in three sample chunks, each chunk's compute
+    starting when its own exchange has landed (forward_rank_overlapped)."""
     import torch.multiprocessing as mp
     out = str(tmp_path / "y.pt")
-    port = 29600 + (os.getpid() % 200) + (0 if kind == "moe" else 1)
-    mp.spawn(_rank, args=(2, kind, port, out), nprocs=2, join=True)
+    port = 29600 + (os.getpid() % 200) + (0 if kind == "moe" else 1) + (2 if overlapped else 0)
+    mp.spawn(_rank, args=(2, kind, port, out, overlapped), nprocs=2, join=True)
     cfg = _cfg(kind)
     ref = oracle.run_stack(cfg, storage=cfg.dtype)["Y"]
     got = torch.load(out).numpy()

@@ -140,13 +140,20 @@ class RankStage:
                 [api.sublayer_workspace_bytes(self.sh_rev, A.TM_LAYOUT_ROWS, s) for s in self.rev])
         self.ws = torch.empty(n, dtype=torch.uint8, device=device)
 
+    @staticmethod
+    def _rows(sh: A.tm_shape, B: int) -> A.tm_shape:
+        return sh if B == sh.B else A.tm_shape(B, sh.T, sh.D, sh.H, sh.dtype, sh.eps)
+
     def mixing(self, l: int, G: torch.Tensor) -> torch.Tensor:
-        """Mixing sub-layer of block l on p's heads: R_p = Revert(FFN(Norm(Mix(G_p))) + Mix(G_p))."""
-        return api.sublayer_forward(G, G, None, A.TM_LAYOUT_MIXED, self.sh_mix, self.mix[l], workspace=self.ws)
+        """Mixing sub-layer of block l on p's heads: R_p = Revert(FFN(Norm(Mix(G_p))) + Mix(G_p)) (any
+        number of samples up to the stage's B)."""
+        return api.sublayer_forward(G, G, None, A.TM_LAYOUT_MIXED, self._rows(self.sh_mix, G.shape[0]), self.mix[l],
+                                    workspace=self.ws)
 
     def reverting(self, l: int, Xr: torch.Tensor, x: torch.Tensor, extra: Optional[torch.Tensor]) -> torch.Tensor:
         """Reverting sub-layer of block l on p's tokens: FFN(Norm(X_rev)) + x (+ inter-residual)."""
-        return api.sublayer_forward(Xr, x, extra, A.TM_LAYOUT_ROWS, self.sh_rev, self.rev[l], workspace=self.ws)
+        return api.sublayer_forward(Xr, x, extra, A.TM_LAYOUT_ROWS, self._rows(self.sh_rev, Xr.shape[0]), self.rev[l],
+                                    workspace=self.ws)
 
 
 # ------------------------------------------------------------------ drivers
@@ -166,6 +173,40 @@ def forward_rank(stage, plan: ShardPlan, x_local: torch.Tensor, L: int, gap: int
     return hist[-1]
 
 
+def forward_rank_overlapped(stage, plan: ShardPlan, x_local: torch.Tensor, L: int, gap: int, exchange_async,
+                            chunks: int = 2, layouts=LibraryLayouts) -> torch.Tensor:
+    """forward_rank with each block's two exchanges split into sample chunks and overlapped with the
+    compute: every chunk's token->head exchange is issued at once; chunk c's mixing sub-layer runs
+    as soon as its exchange has landed, while the later chunks' exchanges are in flight, and its
+    head->token exchange is issued right after it, in flight while chunk c+1 mixes; the reverting
+    sub-layer of chunk c follows its exchange.  exchange_async(send) -> (recv, handle), handle.wait()
+    before recv is used (torch_exchange_async: NCCL's own stream beside the compute).  Samples are
+    independent, so the result is the bits of forward_rank; every rank issues the same exchanges in
+    the same order."""
+    lay = layouts
+    B = x_local.shape[0]
+    n = max(1, min(chunks, B))
+    bounds = [B * i // n for i in range(n + 1)]
+    spans = [(bounds[i], bounds[i + 1]) for i in range(n) if bounds[i + 1] > bounds[i]]
+    hist: List[torch.Tensor] = [x_local]
+    for l in range(1, L + 1):
+        x = hist[-1]
+        first = [exchange_async(lay.pack_for_heads(plan, x[a:b])) for a, b in spans]
+        second = []
+        for recv, h in first:
+            h.wait()
+            R = stage.mixing(l - 1, lay.unpack_heads(plan, recv))
+            second.append(exchange_async(lay.pack_for_tokens(plan, R)))
+        s = skip_index(l, L, gap)
+        outs = []
+        for (a, b), (recv, h) in zip(spans, second):
+            h.wait()
+            Xr = lay.unpack_tokens(plan, recv)
+            outs.append(stage.reverting(l - 1, Xr, x[a:b], hist[s][a:b] if s is not None else None))
+        hist.append(torch.cat(outs, dim=0))
+    return hist[-1]
+
+
 def forward_all_ranks(stages: Sequence, plan: ShardPlan, x_locals: Sequence[torch.Tensor], L: int,
                       gap: int, layouts=LibraryLayouts) -> List[torch.Tensor]:
     """Every rank's share in one process (the exchange becomes a transpose of the ranks' chunks)."""
@@ -182,6 +223,16 @@ def forward_all_ranks(stages: Sequence, plan: ShardPlan, x_locals: Sequence[torc
         hist.append([stages[p].reverting(l - 1, Xr[p], hist[-1][p], hist[s][p] if s is not None else None)
                      for p in range(P)])
     return hist[-1]
+
+
+def torch_exchange_async(group=None):
+    """The all-to-all of torch.distributed issued asynchronously: send -> (recv, handle)."""
+    import torch.distributed as dist
+
+    def ex(send: torch.Tensor):
+        recv = torch.empty_like(send)
+        return recv, dist.all_to_all_single(recv, send, group=group, async_op=True)
+    return ex
 
 
 def torch_exchange(group=None) -> Callable[[torch.Tensor], torch.Tensor]:
