@@ -107,10 +107,6 @@ def quantize_rows(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
     return e4m3_encode(np.ldexp(x32.astype(np.float64), -e[:, None])), s
 
 
-def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
-    return e4m3_decode(codes) * np.asarray(scales, dtype=np.float64)[:, None]
-
-
 def quantize_matrix(w: np.ndarray) -> Tuple[np.ndarray, np.float32]:
     """E4M3 quantization of a whole matrix with one power-of-two scale (as quantize_rows)."""
     w32 = np.asarray(w, dtype=np.float32)
