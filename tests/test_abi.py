@@ -51,6 +51,9 @@ int main(void) {
   P(tm_swiglu_w8, q_gate) P(tm_swiglu_w8, s_up) P(tm_swiglu_w8, w_down) P(tm_block_fp8, rev)
   printf("tm_swiglu_grads %zu\ntm_block_grads %zu\n", sizeof(tm_swiglu_grads), sizeof(tm_block_grads));
   P(tm_swiglu_grads, dw_up) P(tm_swiglu_grads, dw_down) P(tm_block_grads, rev)
+  printf("tm_moe_w8 %zu\ntm_sublayer8 %zu\n", sizeof(tm_moe_w8), sizeof(tm_sublayer8));
+  P(tm_moe_w8, alpha) P(tm_moe_w8, w_router) P(tm_moe_w8, se_up) P(tm_moe_w8, we_down) P(tm_moe_w8, ss_up)
+  P(tm_moe_w8, ws_down) P(tm_sublayer8, dense) P(tm_sublayer8, moe)
   return 0;
 }
 ''')
@@ -73,6 +76,11 @@ int main(void) {
         "tm_swiglu_grads.dw_up": A.tm_swiglu_grads.dw_up.offset,
         "tm_swiglu_grads.dw_down": A.tm_swiglu_grads.dw_down.offset,
         "tm_block_grads.rev": A.tm_block_grads.rev.offset,
+        "tm_moe_w8": ctypes.sizeof(A.tm_moe_w8), "tm_sublayer8": ctypes.sizeof(A.tm_sublayer8),
+        "tm_moe_w8.alpha": A.tm_moe_w8.alpha.offset, "tm_moe_w8.w_router": A.tm_moe_w8.w_router.offset,
+        "tm_moe_w8.se_up": A.tm_moe_w8.se_up.offset, "tm_moe_w8.we_down": A.tm_moe_w8.we_down.offset,
+        "tm_moe_w8.ss_up": A.tm_moe_w8.ss_up.offset, "tm_moe_w8.ws_down": A.tm_moe_w8.ws_down.offset,
+        "tm_sublayer8.dense": A.tm_sublayer8.dense.offset, "tm_sublayer8.moe": A.tm_sublayer8.moe.offset,
     }
     assert {k: int(v) for k, v in got.items()} == want
 
