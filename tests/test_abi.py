@@ -54,6 +54,7 @@ int main(void) {
   printf("tm_moe_w8 %zu\ntm_sublayer8 %zu\n", sizeof(tm_moe_w8), sizeof(tm_sublayer8));
   P(tm_moe_w8, alpha) P(tm_moe_w8, w_router) P(tm_moe_w8, se_up) P(tm_moe_w8, we_down) P(tm_moe_w8, ss_up)
   P(tm_moe_w8, ws_down) P(tm_sublayer8, dense) P(tm_sublayer8, moe)
+  printf("TM_TP_TOKEN_SHARD %d\nTM_TP_HEAD_SHARD %d\n", TM_TP_TOKEN_SHARD, TM_TP_HEAD_SHARD);
   return 0;
 }
 ''')
@@ -81,6 +82,7 @@ int main(void) {
         "tm_moe_w8.se_up": A.tm_moe_w8.se_up.offset, "tm_moe_w8.we_down": A.tm_moe_w8.we_down.offset,
         "tm_moe_w8.ss_up": A.tm_moe_w8.ss_up.offset, "tm_moe_w8.ws_down": A.tm_moe_w8.ws_down.offset,
         "tm_sublayer8.dense": A.tm_sublayer8.dense.offset, "tm_sublayer8.moe": A.tm_sublayer8.moe.offset,
+        "TM_TP_TOKEN_SHARD": A.TM_TP_TOKEN_SHARD, "TM_TP_HEAD_SHARD": A.TM_TP_HEAD_SHARD,
     }
     assert {k: int(v) for k, v in got.items()} == want
 
