@@ -289,3 +289,19 @@ def test_fp8_moe_workspace_and_validation(name):
         assert lib.tm_sublayer_fp8_workspace_bytes(ctypes.byref(sh), layout, ctypes.byref(bad)) == 0
         assert lib.tm_sublayer_forward_fp8(x, None, None, layout, ctypes.byref(sh), ctypes.byref(bad), y, ws, n8,
                                            None) == A.TM_ERR_UNSUPPORTED
+
+
+def test_tp_exchange_layout_validation():
+    """tm_tp_exchange_layout refuses bad arguments on the host, before any launch."""
+    lib = A.load()
+    src, dst = ctypes.c_void_p(0x200000), ctypes.c_void_p(0x400000)
+    bad = [
+        (src, dst, 0, 4, 2, 64, A.TM_BF16, A.TM_TP_TOKEN_SHARD, 1),      # P < 1
+        (src, src, 2, 4, 2, 64, A.TM_BF16, A.TM_TP_TOKEN_SHARD, 1),      # in place
+        (src, dst, 2, 4, 2, 64, A.TM_BF16, 7, 1),                        # unknown layout
+        (src, dst, 2, 4, 2, 64, 5, A.TM_TP_HEAD_SHARD, 0),               # unknown dtype
+        (ctypes.c_void_p(0x200002), dst, 2, 4, 2, 64, A.TM_BF16, A.TM_TP_HEAD_SHARD, 0),   # misaligned
+        (None, dst, 2, 4, 2, 64, A.TM_F32, A.TM_TP_HEAD_SHARD, 0),       # null
+    ]
+    for args in bad:
+        assert lib.tm_tp_exchange_layout(*args, None) == A.TM_ERR_INVALID_ARG, args
