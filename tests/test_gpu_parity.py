@@ -55,6 +55,8 @@ MOE_SMALL = [
     small("moe_ns", 260, 8, 384, 4, "bf16", moe(16, 4, 128, 256), moe(6, 3, 64, 64)),
     # 24 experts: the CUDA-core router; mixed rows then reach GEMM1 through the bucket-order copy
     small("moe_e24", 170, 8, 256, 8, "bf16", moe(24, 3, 64, 64), moe(24, 2, 64, 128)),
+    # head width 64: four 16-column pieces per token in the Mix geometry
+    small("moe_dh64", 150, 8, 256, 4, "bf16", moe(8, 2, 128, 128), moe(4, 2, 64, 128)),
     small("moe_f32", 150, 8, 64, 8, "f32", moe(4, 2, 64, 32), moe(8, 3, 32, 64)),
 ]
 
