@@ -267,16 +267,31 @@ __global__ void __launch_bounds__(kRouterChunk) scatter_kernel(const int32_t* __
                                                                const float* __restrict__ gate, float* __restrict__ inv_pos,
                                                                float* __restrict__ gate_pos) {
     __shared__ int wcount[kRouterChunk / 32][64];
+    __shared__ int base[64];   // per expert: the bucket's offset plus the earlier chunks' rows
     const int bank = blockIdx.y, chunk = blockIdx.x, nchunks = gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = chunk * kRouterChunk + threadIdx.x;
     const bool valid = b < B;
     const size_t rowi = (size_t)b * banks + bank;
+    // every global load the block needs is issued here, before any of it is used
+    if (threadIdx.x < E)
+        base[threadIdx.x] = bucket_offsets[bank * E + threadIdx.x] +
+                            chunk_prefix[((size_t)bank * nchunks + chunk) * E + threadIdx.x];
     int my[8], rank[8];
+    float gv[8];
+    float irs = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) { my[j] = -1; rank[j] = 0; }
-    if (valid)
-        for (int j = 0; j < k; ++j) my[j] = idx[rowi * k + j];
+    for (int j = 0; j < 8; ++j) { my[j] = -1; rank[j] = 0; gv[j] = 0.f; }
+    if (valid) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (j < k) {
+                my[j] = idx[rowi * k + j];
+                if (gate_pos) gv[j] = gate[rowi * k + j];
+            }
+        }
+        if (inv_pos) irs = inv_rms[rowi];
+    }
     const unsigned lt_mask = (1u << lane) - 1u;
     for (int e = 0; e < E; ++e) {
         bool has = false;
@@ -292,13 +307,15 @@ __global__ void __launch_bounds__(kRouterChunk) scatter_kernel(const int32_t* __
     if (!valid) return;
     // positions must fall inside the caller's bucket_rows (limit entries): a table that does not
     // match the choices is reported, never written out of range
-    for (int j = 0; j < k; ++j) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        if (j >= k) break;
         const int e = my[j];
         if (e < 0 || e >= E) {
             record_error(ERR_BOUNDS, 0x500);
             continue;
         }
-        int pos = bucket_offsets[bank * E + e] + chunk_prefix[((size_t)bank * nchunks + chunk) * E + e] + rank[j];
+        int pos = base[e] + rank[j];
         for (int w = 0; w < warp; ++w) pos += wcount[w][e];
         if (pos < 0 || pos >= limit) {
             record_error(ERR_BOUNDS, 0x501);
@@ -311,8 +328,8 @@ __global__ void __launch_bounds__(kRouterChunk) scatter_kernel(const int32_t* __
         if (perm) perm[pos] = (int32_t)(((size_t)bank * k + j) * B + b);
         // (optional) the row's 1/rms and the choice's gate by bucket position, so that the routed
         // GEMMs read them as contiguous per-row values
-        if (inv_pos) inv_pos[pos] = inv_rms[rowi];
-        if (gate_pos) gate_pos[pos] = gate[rowi * k + j];
+        if (inv_pos) inv_pos[pos] = irs;
+        if (gate_pos) gate_pos[pos] = gv[j];
     }
 }
 
