@@ -634,9 +634,9 @@ tm_status run_moe(const Geo& g, const void* x, const void* resid, const void* ex
     } else {
         // MoEPermute: copy the routed rows into bucket order (the slot buffer, [routed, W], is free
         // until the routed GEMM2 writes it), then GEMM1 reads A as contiguous rows through a 2-D
-        // tensor map.  (Gathering the rows inside GEMM1 instead, by tile::gather4 TMA loads of
-        // one-row boxes, measured 2.2x slower for GEMM1 than this copy plus one 16 KB box per K slab:
-        // every N tile gathers its A rows again, 32 four-row operations per slab.)
+        // tensor map.  (Gathering the rows inside GEMM1 instead measured slower than this copy plus one
+        // 16 KB box per K slab: by tile::gather4 TMA loads of one-row boxes 2.2x, by the gatherer
+        // warps' cp.async 3-6x; every N tile gathers its A rows again.)
         const int bn = pick_bn_swiglu(Fe);
         p.n_tiles = p.N / bn;
         CUtensorMap ma, mg, mu, mo;
