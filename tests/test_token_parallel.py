@@ -1,4 +1,4 @@
-"""Token Parallel on the CPU: two gloo ranks exchange their shards with all_to_all_single.
+"""Token Parallel on the CPU: two or three gloo ranks exchange their shards with all_to_all_single.
 
 Each rank holds half of the tokens and half of the heads of a small stack and runs the exchange
 schedule and shard packing of token_sparse_moe_b200.token_parallel; the compute of each rank's
@@ -67,6 +67,10 @@ class OracleStage:
 
 
 def _cfg(kind):
+    if kind == "moe3":
+        # three ranks: 6 tokens and 6 heads, two of each per rank
+        spec = FFNSpec("moe", E=3, k=2, hidden_e=16, hidden_s=16, alpha=1.5)
+        return S.Config("tp_moe3", B=18, T=6, D=24, H=6, L=2, gap=1, dtype="bf16", mix=spec, rev=spec)
     if kind == "moe":
         spec = FFNSpec("moe", E=4, k=2, hidden_e=16, hidden_s=16, alpha=2.0)
         return S.Config("tp_moe", B=24, T=4, D=32, H=4, L=3, gap=2, dtype="bf16", mix=spec, rev=spec)
@@ -99,14 +103,15 @@ def _rank(rank, world, kind, port, out_path, overlapped=False):
 
 
 @pytest.mark.parametrize("overlapped", [False, True], ids=["plain", "overlapped"])
-@pytest.mark.parametrize("kind", ["moe", "dense"])
-def test_token_parallel_two_ranks_equal_the_unsharded_stack(kind, overlapped, tmp_path):
+@pytest.mark.parametrize("kind", ["moe", "dense", "moe3"])
+def test_token_parallel_ranks_equal_the_unsharded_stack(kind, overlapped, tmp_path):
     """Also with the exchanges issued asynchronously in three sample chunks, each chunk's compute
-    starting when its own exchange has landed (forward_rank_overlapped)."""
+    starting when its own exchange has landed (forward_rank_overlapped); moe3 runs three ranks."""
     import torch.multiprocessing as mp
     out = str(tmp_path / "y.pt")
-    port = 29600 + (os.getpid() % 200) + (0 if kind == "moe" else 1) + (2 if overlapped else 0)
-    mp.spawn(_rank, args=(2, kind, port, out, overlapped), nprocs=2, join=True)
+    world = 3 if kind == "moe3" else 2
+    port = 29600 + (os.getpid() % 200) + {"moe": 0, "dense": 1, "moe3": 4}[kind] + (2 if overlapped else 0) * 3
+    mp.spawn(_rank, args=(world, kind, port, out, overlapped), nprocs=world, join=True)
     cfg = _cfg(kind)
     ref = oracle.run_stack(cfg, storage=cfg.dtype)["Y"]
     got = torch.load(out).numpy()
