@@ -1,6 +1,6 @@
 """Token Parallel on the CPU: two or three gloo ranks exchange their shards with all_to_all_single.
 
-Each rank holds half of the tokens and half of the heads of a small stack and runs the exchange
+Each rank holds its share of the tokens and of the heads of a small stack and runs the exchange
 schedule and shard packing of token_sparse_moe_b200.token_parallel; the compute of each rank's
 sub-layers is the float64 oracle here (this test has no GPU), with the model's bf16 storage
 rounding.  Gathered over the ranks, the result must equal the oracle's unsharded stack exactly:
