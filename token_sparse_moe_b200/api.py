@@ -7,7 +7,7 @@ here, by the caller side of the C ABI) and the CUDA stream.
 from __future__ import annotations
 
 import ctypes
-from dataclasses import dataclass, field
+from dataclasses import dataclass
 from typing import Callable, Dict, List, Optional, Sequence
 
 import numpy as np
