@@ -305,3 +305,26 @@ def test_tp_exchange_layout_validation():
     ]
     for args in bad:
         assert lib.tm_tp_exchange_layout(*args, None) == A.TM_ERR_INVALID_ARG, args
+
+
+def test_empty_batch_is_refused_everywhere():
+    """B = 0 (an empty batch) is an invalid shape for every entry point that takes one, refused on
+    the host before any launch; so are a non-positive token count and an eps that is negative."""
+    lib = A.load()
+    cfg = S.CONFIGS["moe_stack_bf16"]
+    x, y, ws = ctypes.c_void_p(0x200000), ctypes.c_void_p(0x400000), ctypes.c_void_p(0x800000)
+    for bad in (api.shape(0, cfg.T, cfg.D, cfg.H, "bf16"), api.shape(cfg.B, 0, cfg.D, cfg.H, "bf16"),
+                api.shape(cfg.B, cfg.T, cfg.D, cfg.H, "bf16", eps=-1.0)):
+        blk = A.tm_block(_fake_sub(cfg, 0).c(), _fake_sub(cfg, 1).c())
+        assert lib.tm_stack_forward(x, ctypes.byref(blk), 1, 0, ctypes.byref(bad), y, ws, 1 << 30,
+                                    None) == A.TM_ERR_INVALID_ARG
+        assert lib.tm_block_forward(x, ctypes.byref(blk), ctypes.byref(bad), y, None, ws, 1 << 30,
+                                    None) == A.TM_ERR_INVALID_ARG
+        mw = _fake_sub(cfg, 1).moe_c()
+        assert lib.tm_sparse_pertoken_moe(x, None, A.TM_LAYOUT_ROWS, ctypes.byref(bad), None, ctypes.byref(mw), y, ws,
+                                          1 << 30, None) == A.TM_ERR_INVALID_ARG
+        s8 = _fake_moe8(cfg, 1).sub_c()
+        assert lib.tm_sublayer_forward_fp8(x, None, None, A.TM_LAYOUT_ROWS, ctypes.byref(bad), ctypes.byref(s8), y, ws,
+                                           1 << 30, None) == A.TM_ERR_INVALID_ARG
+        assert lib.tm_sublayer_fp8_workspace_bytes(ctypes.byref(bad), A.TM_LAYOUT_ROWS, ctypes.byref(s8)) == 0
+        assert lib.tm_route_workspace_bytes(ctypes.byref(bad), A.TM_LAYOUT_ROWS, ctypes.byref(mw)) == 0
