@@ -81,8 +81,12 @@ def rmsnorm(x: np.ndarray, eps: float, gain: Optional[np.ndarray] = None) -> np.
 
 
 def silu(z: np.ndarray) -> np.ndarray:
-    """Swish with beta = 1.  [digest] 2.3.2, Eq. 17."""
-    return z / (1.0 + np.exp(-z))
+    """Swish with beta = 1.  [digest] 2.3.2, Eq. 17.
+
+    For z below about -709, exp(-z) overflows to inf and z / inf gives the limit 0; the overflow is
+    expected there and not reported."""
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
 
 
 def swiglu(n: np.ndarray, w_gate: np.ndarray, w_up: np.ndarray, w_down: np.ndarray) -> np.ndarray:
