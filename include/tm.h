@@ -155,8 +155,10 @@ TM_API tm_status tm_model_forward(const void *groups, const void *w_group, const
  * local tensor is the rank's token shard [B][Tp][D] = [B][Tp][P][Dp] (chunk q = the columns of rank
  * q's heads); TM_TP_HEAD_SHARD: the rank's head-column shard of every token [B][T][Dp] = [B][P][Tp][Dp]
  * (chunk q = rank q's tokens).  to_exchange != 0 copies local (src) -> E (dst), else E (src) ->
- * local (dst).  A pure permutation (bit-exact); src and dst device memory, not overlapping, 16-byte
- * aligned when Dp * element size is a multiple of 16. */
+ * local (dst).  A pure permutation (bit-exact); src and dst device memory, not overlapping, aligned
+ * to the element size, and to 16 bytes when Dp * element size is a multiple of 16.  TM_ERR_INVALID_ARG
+ * (nothing launched) for a null, equal or misaligned pointer, a size below 1, a dtype other than f32
+ * or bf16, or an unknown layout. */
 #define TM_TP_TOKEN_SHARD 0
 #define TM_TP_HEAD_SHARD 1
 TM_API tm_status tm_tp_exchange_layout(const void *src, void *dst, int P, int B, int Tp, int Dp, tm_dtype dtype,

@@ -302,6 +302,8 @@ def test_tp_exchange_layout_validation():
         (src, dst, 2, 4, 2, 64, 5, A.TM_TP_HEAD_SHARD, 0),               # unknown dtype
         (ctypes.c_void_p(0x200002), dst, 2, 4, 2, 64, A.TM_BF16, A.TM_TP_HEAD_SHARD, 0),   # misaligned
         (None, dst, 2, 4, 2, 64, A.TM_F32, A.TM_TP_HEAD_SHARD, 0),       # null
+        (src, ctypes.c_void_p(0x400002), 2, 4, 2, 3, A.TM_F32, A.TM_TP_TOKEN_SHARD, 1),  # f32 element path, 2-byte aligned
+        (ctypes.c_void_p(0x200001), dst, 2, 4, 2, 3, A.TM_BF16, A.TM_TP_TOKEN_SHARD, 0),  # bf16 element path, odd address
     ]
     for args in bad:
         assert lib.tm_tp_exchange_layout(*args, None) == A.TM_ERR_INVALID_ARG, args

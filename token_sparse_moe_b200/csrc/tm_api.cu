@@ -1390,6 +1390,8 @@ tm_status tm_tp_exchange_layout(const void* src, void* dst, int P, int B, int Tp
     if ((dtype != TM_F32 && dtype != TM_BF16) || (local_layout != TM_TP_TOKEN_SHARD && local_layout != TM_TP_HEAD_SHARD))
         return TM_ERR_INVALID_ARG;
     const int esz = dtype == TM_BF16 ? 2 : 4;
+    if (((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & (uintptr_t)(esz - 1)) != 0)
+        return TM_ERR_INVALID_ARG;
     if (((size_t)Dp * esz) % 16 == 0 && (!al16(src) || !al16(dst))) return TM_ERR_INVALID_ARG;
     return cuda_status(launch_tp_layout(src, dst, P, B, Tp, Dp, esz, local_layout == TM_TP_TOKEN_SHARD, to_exchange != 0,
                                         (cudaStream_t)stream));
