@@ -330,3 +330,17 @@ def test_empty_batch_is_refused_everywhere():
                                            1 << 30, None) == A.TM_ERR_INVALID_ARG
         assert lib.tm_sublayer_fp8_workspace_bytes(ctypes.byref(bad), A.TM_LAYOUT_ROWS, ctypes.byref(s8)) == 0
         assert lib.tm_route_workspace_bytes(ctypes.byref(bad), A.TM_LAYOUT_ROWS, ctypes.byref(mw)) == 0
+
+
+def test_elementwise_utilities_refuse_misaligned_pointers():
+    """tm_mix, tm_revert and tm_tokenize_stub take element-aligned pointers; one that is not aligned
+    to its element is refused on the host (an element-wise kernel would fault on it)."""
+    lib = A.load()
+    a, b = ctypes.c_void_p(0x200000), ctypes.c_void_p(0x400000)
+    for dtype, off in (("f32", 2), ("bf16", 1)):
+        sh = api.shape(4, 8, 16, 4, dtype)
+        odd = ctypes.c_void_p(0x400000 + off)
+        assert lib.tm_mix(a, odd, ctypes.byref(sh), None) == A.TM_ERR_INVALID_ARG
+        assert lib.tm_revert(odd, b, ctypes.byref(sh), None) == A.TM_ERR_INVALID_ARG
+        assert lib.tm_tokenize_stub(a, a, a, 4, ctypes.byref(sh), odd, None) == A.TM_ERR_INVALID_ARG
+        assert lib.tm_tokenize_stub(odd, a, a, 4, ctypes.byref(sh), b, None) == A.TM_ERR_INVALID_ARG

@@ -14,6 +14,10 @@ namespace {
 
 // ------------------------------------------------------------------ small utilities
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// aligned to one element of the shape's dtype (the element-wise kernels' only requirement)
+inline bool al_elem(const void* p, int dtype) {
+    return (reinterpret_cast<uintptr_t>(p) & (dtype == TM_BF16 ? 1u : 3u)) == 0;
+}
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Carve {
@@ -1341,6 +1345,9 @@ tm_status tm_tokenize_stub(const void* groups, const void* w_group, const void* 
     if (s != TM_OK) return s;
     if (!groups || !w_global || !X_out || dg <= 0 || shape->T < 2) return TM_ERR_INVALID_ARG;
     if (!w_group) return TM_ERR_INVALID_ARG;
+    if (!al_elem(groups, shape->dtype) || !al_elem(w_group, shape->dtype) || !al_elem(w_global, shape->dtype) ||
+        !al_elem(X_out, shape->dtype))
+        return TM_ERR_INVALID_ARG;
     return cuda_status(launch_tokenize(shape->dtype, groups, w_group, w_global, dg, shape->B, shape->T, shape->D, X_out,
                                        (cudaStream_t)stream));
 }
@@ -1379,7 +1386,7 @@ tm_status tm_model_forward(const void* groups, const void* w_group, const void* 
 tm_status tm_mix(const void* X, void* Hm, const tm_shape* shape, void* stream) {
     tm_status s = check_shape(shape);
     if (s != TM_OK) return s;
-    if (!X || !Hm || X == Hm) return TM_ERR_INVALID_ARG;
+    if (!X || !Hm || X == Hm || !al_elem(X, shape->dtype) || !al_elem(Hm, shape->dtype)) return TM_ERR_INVALID_ARG;
     return cuda_status(launch_permute(shape->dtype, X, Hm, shape->B, shape->T, shape->D, shape->H, true,
                                       (cudaStream_t)stream));
 }
@@ -1400,7 +1407,7 @@ tm_status tm_tp_exchange_layout(const void* src, void* dst, int P, int B, int Tp
 tm_status tm_revert(const void* Hm, void* X, const tm_shape* shape, void* stream) {
     tm_status s = check_shape(shape);
     if (s != TM_OK) return s;
-    if (!X || !Hm || X == Hm) return TM_ERR_INVALID_ARG;
+    if (!X || !Hm || X == Hm || !al_elem(X, shape->dtype) || !al_elem(Hm, shape->dtype)) return TM_ERR_INVALID_ARG;
     return cuda_status(launch_permute(shape->dtype, Hm, X, shape->B, shape->T, shape->D, shape->H, false,
                                       (cudaStream_t)stream));
 }
