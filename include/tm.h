@@ -9,7 +9,8 @@
  *            block diagram and the list of paper-faithful choices.
  *
  * Conventions shared by every call:
- *   - Every tensor pointer is caller-owned DEVICE memory, 16-byte aligned, in
+ *   - Every tensor pointer is caller-owned DEVICE memory, 16-byte aligned (the
+ *     element-wise utilities below ask only for one element's alignment), in
  *     row-major (C) order with the shape given beside it.  The library never
  *     allocates device memory and never frees caller memory; scratch space is
  *     the caller's `workspace`, sized by the *_workspace_bytes queries.
@@ -122,15 +123,17 @@ TM_API size_t tm_workspace_bytes(const tm_shape *shape, const tm_block *blocks, 
  * layer per group: X[b,0] = w_global . concat_g groups[b,g]  (the global token),
  * X[b,t] = w_group[t-1] . groups[b,t-1] for t = 1..T-1.
  * groups [B, T-1, dg]; w_group [T-1, D, dg]; w_global [D, (T-1)*dg]; X_out [B,T,D].
- * A boundary utility (plain CUDA-core kernel), not part of the timed path. */
+ * A boundary utility (plain CUDA-core kernel), not part of the timed path; pointers aligned to
+ * one element suffice.  TM_ERR_INVALID_ARG for a null or misaligned pointer, dg < 1 or T < 2. */
 TM_API tm_status tm_tokenize_stub(const void *groups, const void *w_group, const void *w_global, int dg,
                            const tm_shape *shape, void *X_out, void *stream);
 
 /* Mix ([digest] 2.3.1, Eq. 9-11): Hm[b, h, t*dh + j] = X[b, t, h*dh + j],
- * X [B,T,D] -> Hm [B, H, T*D/H].  A test/API utility: the fused path never calls it. */
+ * X [B,T,D] -> Hm [B, H, T*D/H].  A test/API utility: the fused path never calls it.  Pointers
+ * aligned to one element suffice; TM_ERR_INVALID_ARG for a null, equal or misaligned pointer. */
 TM_API tm_status tm_mix(const void *X, void *Hm, const tm_shape *shape, void *stream);
 
-/* Scoring head ([readme] block diagram: "mean-pool over tokens -> projection head -> logit",
+/* Scoring head ([readme] block diagram: the tokens are mean-pooled, then projected to one logit;
  * bias off as the reproduction's default): logits[b] = (1/T) sum_t sum_d X[b,t,d] * w_head[d],
  * fp32 accumulation.  X [B,T,D] and w_head [D] in the shape's dtype; logits [B] fp32.
  * An HBM-bound reduction kernel (one warp per sample). */
@@ -164,7 +167,8 @@ TM_API tm_status tm_model_forward(const void *groups, const void *w_group, const
 TM_API tm_status tm_tp_exchange_layout(const void *src, void *dst, int P, int B, int Tp, int Dp, tm_dtype dtype,
                                        int local_layout, int to_exchange, void *stream);
 
-/* Revert ([digest] 2.3.1, Eq. 13-15), the inverse of Mix: Hm [B,H,T*D/H] -> X [B,T,D]. */
+/* Revert ([digest] 2.3.1, Eq. 13-15), the inverse of Mix: Hm [B,H,T*D/H] -> X [B,T,D].  Same
+ * pointer rules as tm_mix. */
 TM_API tm_status tm_revert(const void *Hm, void *X, const tm_shape *shape, void *stream);
 
 /* Router of a Sparse-Pertoken MoE sub-layer ([digest] 2.4.1 Eq. 19, 2.4.3 Eq. 21)
@@ -253,8 +257,8 @@ TM_API tm_status tm_block_forward(const void *X, const tm_block *block, const tm
 TM_API tm_status tm_stack_step(const void *X, const void *X_skip, const tm_block *block, const tm_shape *shape,
                                void *Y, void *X_revert_opt, void *workspace, size_t workspace_bytes, void *stream);
 
-/* L blocks with the inter-residual of [digest] 2.3.4 ([readme]: "at gap 2, excluded
- * from the final layer"): X_l = Block_l(X_{l-1}); X_l += X_{l-gap} when gap > 0,
+/* L blocks with the inter-residual of [digest] 2.3.4 ([readme]: every second layer, none
+ * after the final one): X_l = Block_l(X_{l-1}); X_l += X_{l-gap} when gap > 0,
  * l % gap == 0 and l < L (layers counted from 1).  Y = X_L.  Y must not alias X. */
 TM_API tm_status tm_stack_forward(const void *X, const tm_block *blocks, int L, int inter_residual_gap,
                            const tm_shape *shape, void *Y, void *workspace, size_t workspace_bytes,

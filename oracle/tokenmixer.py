@@ -15,7 +15,7 @@ Sources (two of the pages on TokenMixer-Large):
 Readings where the pages are silent or garbled (each one is listed with its
 reason in the design notes of the repository):
   * pre-norm sub-layers  out = FFN(RMSNorm(in)) + residual  ([readme] block
-    diagram; [digest] 2.3.3 "Pre-Norm replaces Post-Norm"), not the post-norm
+    diagram; [digest] 2.3.3, which moves the norm in front of the FFN), not the post-norm
     form printed in Eq. 8/12/16;
   * Revert is the exact inverse of Mix (Eq. 13 prints the same head index twice);
   * Swish is SiLU (beta = 1);
@@ -75,7 +75,7 @@ def revert(Hn: np.ndarray, T: int) -> np.ndarray:
 
 # ------------------------------------------------------------------ norm / FFN
 def rmsnorm(x: np.ndarray, eps: float, gain: Optional[np.ndarray] = None) -> np.ndarray:
-    """RMSNorm over the last axis, no mean-centering.  [digest] 2.3.3; [readme] "RMSNorm + no bias"."""
+    """RMSNorm over the last axis, no mean-centering.  [digest] 2.3.3; [readme] (RMSNorm, no bias terms)."""
     r = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
     return r if gain is None else r * gain
 
@@ -92,7 +92,7 @@ def silu(z: np.ndarray) -> np.ndarray:
 def swiglu(n: np.ndarray, w_gate: np.ndarray, w_up: np.ndarray, w_down: np.ndarray) -> np.ndarray:
     """FC_down(Swish(FC_gate n) * FC_up n), weights in [out, in] layout, no bias.
 
-    [digest] 2.3.2, Eq. 17-18 (bias terms dropped: [readme] "Bias defaults to off").
+    [digest] 2.3.2, Eq. 17-18 (bias terms dropped: the [readme] reproduction leaves them off by default).
     n: [R, W]; w_gate, w_up: [F, W]; w_down: [W, F]  ->  [R, W].
     """
     g = n @ w_gate.T
@@ -203,7 +203,7 @@ def sublayer(rows: np.ndarray, bank_w: Callable[[int], Weights], spec, eps: floa
     """FFN(RMSNorm(row)) for every row of every bank, without the residual.
 
     rows: [R, banks, W].  Bank j owns its own weights (parameter isolation,
-    [digest] 2.3.2 and 2.4.2 "per-token").  Returns out [R, banks, W] and, for
+    [digest] 2.3.2 and 2.4.2, per-token weights).  Returns out [R, banks, W] and, for
     MoE, the routing of each bank.  forced_idx [R, banks, k] (MoE only): teacher-forced
     routing, see sp_moe.
     """
@@ -254,8 +254,8 @@ def block_forward(X: np.ndarray, cfg, layer: int, bank_w: Callable[[int, int, in
 
 def stack_forward(X: np.ndarray, cfg, bank_w: Callable[[int, int, int], Weights],
                   gains: Optional[List] = None, keep: bool = False, storage=None) -> Dict[str, object]:
-    """L blocks with the inter-residual.  [digest] 2.3.4; [readme] "inter-residual at gap 2
-    with the last layer excluded":  X_l = Block_l(X_{l-1}); X_l += X_{l-gap} when
+    """L blocks with the inter-residual.  [digest] 2.3.4; [readme] (inter-residual every 2 layers,
+    none after the final one):  X_l = Block_l(X_{l-1}); X_l += X_{l-gap} when
     gap > 0, l % gap == 0 and l < L (layers counted from 1)."""
     hist = [X]
     blocks = []
