@@ -7,7 +7,6 @@ from __future__ import annotations
 
 from functools import lru_cache
 
-import numpy as np
 
 import tm_synth
 from . import tokenmixer

@@ -4,7 +4,6 @@ rounding bound of a 3-bit mantissa, and the special case in which quantization i
 the FP8 FFN must equal the bf16 oracle's FFN.
 """
 import numpy as np
-import pytest
 import torch
 
 from oracle import fp8 as F

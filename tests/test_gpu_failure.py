@@ -9,7 +9,6 @@ host-made table that under-counts the routed rows: the positions past the bucket
 reported as TM_ERR_DEVICE_BOUNDS and left unwritten (guard entries past the array keep their
 values).  In both cases the context stays usable: an ordinary call afterwards succeeds.
 """
-import ctypes
 
 import numpy as np
 import pytest

@@ -6,7 +6,6 @@ import numpy as np
 
 import oracle
 import tm_synth as S
-from oracle import tokenmixer as O
 from parity_util import GAP_TOL, err_stored, force_near_ties, oracle_stack_forced, rms
 from tm_synth import FFNSpec
 

@@ -10,13 +10,12 @@ this file last; it must pass on its own in a fresh process as well.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
 import tm_synth as S
 from tm_synth import FFNSpec
-from token_sparse_moe_b200 import TMError, api
+from token_sparse_moe_b200 import api
 from token_sparse_moe_b200 import _abi as A
 
 DEV = "cuda:0"

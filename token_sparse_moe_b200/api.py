@@ -412,7 +412,6 @@ class StackRunner:
                                        _p(self.ws), self.ws.numel(), _s(stream)), "tm_stack_forward")
         return Y
 
-
     def run_host(self, X_host: torch.Tensor, Y_host: torch.Tensor, X_dev: torch.Tensor, Y_dev: torch.Tensor,
                  stream=None, chunks=1) -> torch.Tensor:
         """End to end through tm_stack_forward, pipelined in sample chunks (run_host_pipelined)."""
