@@ -26,6 +26,8 @@
  *     is touched.  A kernel that hits a bounded-wait timeout or a bounds check
  *     records it in a device error word (it never traps); read it with
  *     tm_get_device_error.
+ *   - Size limits: T * D < 2^31 elements per sample and B * banks <= 2^28 rows
+ *     per sub-layer (TM_ERR_UNSUPPORTED beyond them).
  *   - Results are deterministic: the same inputs give the same output bits.
  *   - Calls that share a workspace must not overlap on the GPU.
  */

@@ -344,3 +344,20 @@ def test_elementwise_utilities_refuse_misaligned_pointers():
         assert lib.tm_revert(odd, b, ctypes.byref(sh), None) == A.TM_ERR_INVALID_ARG
         assert lib.tm_tokenize_stub(a, a, a, 4, ctypes.byref(sh), odd, None) == A.TM_ERR_INVALID_ARG
         assert lib.tm_tokenize_stub(odd, a, a, 4, ctypes.byref(sh), b, None) == A.TM_ERR_INVALID_ARG
+
+
+def test_sizes_past_32_bit_indexing_are_unsupported():
+    """Shapes whose per-sample element count or per-sub-layer row count would overflow the kernels'
+    32-bit indices and tensor-map coordinates are refused on the host as unsupported."""
+    lib = A.load()
+    a, b = ctypes.c_void_p(0x200000), ctypes.c_void_p(0x400000)
+    wide = api.shape(2, 65536, 65536, 64, "bf16")          # T * D = 2^32 elements per sample
+    assert lib.tm_mix(a, b, ctypes.byref(wide), None) == A.TM_ERR_UNSUPPORTED
+    cfg = S.CONFIGS["moe_stack_bf16"]
+    many = api.shape((1 << 28) // cfg.T + 1, cfg.T, cfg.D, cfg.H, "bf16")   # B * T > 2^28 rows
+    blk = A.tm_block(_fake_sub(cfg, 0).c(), _fake_sub(cfg, 1).c())
+    assert lib.tm_workspace_bytes(ctypes.byref(many), ctypes.byref(blk), 1, 0) == 0
+    assert lib.tm_block_forward(a, ctypes.byref(blk), ctypes.byref(many), b, None, a, 1 << 30,
+                                None) == A.TM_ERR_UNSUPPORTED
+    ok = api.shape((1 << 28) // cfg.T, cfg.T, cfg.D, cfg.H, "bf16")
+    assert lib.tm_workspace_bytes(ctypes.byref(ok), ctypes.byref(blk), 1, 0) > 0

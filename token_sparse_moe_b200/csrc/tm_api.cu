@@ -111,6 +111,8 @@ tm_status check_shape(const tm_shape* s) {
     if (s->B <= 0 || s->T <= 0 || s->D <= 0 || s->H <= 0 || s->D % s->H != 0) return TM_ERR_INVALID_ARG;
     if (s->dtype != TM_F32 && s->dtype != TM_BF16) return TM_ERR_INVALID_ARG;
     if (!(s->eps >= 0.f) || !isfinite(s->eps)) return TM_ERR_INVALID_ARG;
+    // a sample's T * D elements are indexed with 32-bit integers inside the kernels
+    if ((long long)s->T * s->D > INT32_MAX) return TM_ERR_UNSUPPORTED;
     return TM_OK;
 }
 
@@ -126,6 +128,8 @@ tm_status make_geo(const tm_shape* s, int layout, int banks, int width, Geo* g) 
     } else {
         return TM_ERR_INVALID_ARG;
     }
+    // row counts (B * banks, times k <= 8 for the routed rows) are 32-bit tensor-map coordinates
+    if ((long long)s->B * banks > (1LL << 28)) return TM_ERR_UNSUPPORTED;
     const int V = s->dtype == TM_BF16 ? 8 : 4;   // elements per 16-byte vector
     if (width % V != 0) return TM_ERR_UNSUPPORTED;
     if (layout == TM_LAYOUT_MIXED && dh % V != 0) return TM_ERR_UNSUPPORTED;
