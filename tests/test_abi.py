@@ -361,3 +361,12 @@ def test_sizes_past_32_bit_indexing_are_unsupported():
                                 None) == A.TM_ERR_UNSUPPORTED
     ok = api.shape((1 << 28) // cfg.T, cfg.T, cfg.D, cfg.H, "bf16")
     assert lib.tm_workspace_bytes(ctypes.byref(ok), ctypes.byref(blk), 1, 0) > 0
+
+
+def test_binding_refuses_host_tensors():
+    """The binding passes only device addresses to the library: a host tensor raises before any call."""
+    import torch
+    with pytest.raises(ValueError):
+        api._p(torch.zeros(4))
+    assert api._p(None) is None
+    assert api._p(_FakeTensor(0x1230)).value == 0x1230

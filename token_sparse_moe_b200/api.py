@@ -20,7 +20,13 @@ _TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
 
 
 def _p(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a tensor for the C ABI, which reads and writes device memory only: a host
+    tensor is refused here (its address would reach a kernel)."""
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor) and not t.is_cuda:
+        raise ValueError(f"libtm takes device tensors; got one on {t.device}")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _s(stream) -> ctypes.c_void_p:
