@@ -83,7 +83,9 @@ typedef struct {
  * w_router [banks, E, width], E routed SwiGLU experts we_gate/we_up
  * [banks, E, hidden_e, width], we_down [banks, E, width, hidden_e], and one
  * always-on shared expert ws_gate/ws_up [banks, hidden_s, width], ws_down
- * [banks, width, hidden_s] (hidden_s == 0: no shared expert, ws_* ignored).
+ * [banks, width, hidden_s].  hidden_s == 0 (no shared expert, ws_* ignored) is accepted by
+ * tm_route_topk only: the forward calls return TM_ERR_UNSUPPORTED for it (the method's MoE always
+ * has the shared expert, and the combine runs as that expert's down projection).
  * Output = alpha * sum_{top-k e} softmax(router logits)_e * Expert_e + Shared. */
 typedef struct {
     int banks, width, E, k, hidden_e, hidden_s;

@@ -370,3 +370,23 @@ def test_binding_refuses_host_tensors():
         api._p(torch.zeros(4))
     assert api._p(None) is None
     assert api._p(_FakeTensor(0x1230)).value == 0x1230
+
+
+def test_moe_without_shared_expert_routes_but_has_no_forward():
+    """hidden_s = 0 (no shared expert): tm_route_topk takes it (its workspace query answers), every
+    forward call refuses it as unsupported before any launch."""
+    lib = A.load()
+    cfg = S.CONFIGS["moe_stack_bf16"]
+    spec = cfg.ffn(1)
+    x, y, ws = ctypes.c_void_p(0x200000), ctypes.c_void_p(0x400000), ctypes.c_void_p(0x800000)
+    sh = api.shape(cfg.B, cfg.T, cfg.D, cfg.H, "bf16")
+    w = A.tm_moe_w(cfg.T, cfg.D, spec.E, spec.k, spec.hidden_e, 0, spec.alpha, 0x100000, 0x200000, 0x300000, 0x400000,
+                   None, None, None)
+    assert lib.tm_route_workspace_bytes(ctypes.byref(sh), A.TM_LAYOUT_ROWS, ctypes.byref(w)) > 0
+    assert lib.tm_sublayer_workspace_bytes(ctypes.byref(sh), A.TM_LAYOUT_ROWS,
+                                           ctypes.byref(A.tm_sublayer(None, 1, A.tm_swiglu_w(), w))) == 0
+    assert lib.tm_sparse_pertoken_moe(x, None, A.TM_LAYOUT_ROWS, ctypes.byref(sh), None, ctypes.byref(w), y, ws,
+                                      1 << 30, None) == A.TM_ERR_UNSUPPORTED
+    sub = A.tm_sublayer(None, 1, A.tm_swiglu_w(), w)
+    assert lib.tm_sublayer_forward(x, None, None, A.TM_LAYOUT_ROWS, ctypes.byref(sh), ctypes.byref(sub), y, ws,
+                                   1 << 30, None) == A.TM_ERR_UNSUPPORTED
