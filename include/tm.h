@@ -219,6 +219,13 @@ TM_API tm_status tm_route_topk_noalloc(const void *x, tm_layout layout, const tm
                                        int32_t *bucket_offsets, int32_t *bucket_rows, int32_t *slot_of,
                                        void *stream);
 
+/* Sizes the sub-layer, block and stack calls take (others return TM_ERR_UNSUPPORTED before any
+ * launch): row width and hidden widths multiples of 64 (bf16) or 32 (f32); on mixed rows a head
+ * width D/H that is a multiple of 8 (bf16) or 4 (f32), and of 16 for a bf16 MoE sub-layer; MoE:
+ * E <= 32, k <= 8, banks * E <= 4096, a shared expert (hidden_s > 0), and the router's shared
+ * memory within 220 KB: ep * (width + 4) * 4 + 16 * max(32 / ep, 4) * width * (element bytes), ep =
+ * E rounded up to a power of two of at least 4 (width 768 with E = 16 takes 144 KB). */
+
 /* Dense per-token SwiGLU sub-layer with pre-RMSNorm and residual
  * ([readme] block diagram; [digest] 2.3.2-2.3.3):
  *   y_row = SwiGLU_bank(RMSNorm(x_row) * gain) + residual_row

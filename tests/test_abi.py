@@ -390,3 +390,24 @@ def test_moe_without_shared_expert_routes_but_has_no_forward():
     sub = A.tm_sublayer(None, 1, A.tm_swiglu_w(), w)
     assert lib.tm_sublayer_forward(x, None, None, A.TM_LAYOUT_ROWS, ctypes.byref(sh), ctypes.byref(sub), y, ws,
                                    1 << 30, None) == A.TM_ERR_UNSUPPORTED
+
+
+def test_bf16_moe_on_mixed_rows_with_narrow_heads_is_refused_before_launch():
+    """A bf16 MoE sub-layer on mixed rows whose head width is not a multiple of 16 (here 8) is
+    refused by the host checks (its combine reads the residual through a tensor map); the router
+    alone still takes those rows."""
+    lib = A.load()
+    T, D, H, E, k = 8, 64, 8, 4, 2
+    W = T * D // H
+    x, y, ws = ctypes.c_void_p(0x200000), ctypes.c_void_p(0x400000), ctypes.c_void_p(0x800000)
+    sh = api.shape(256, T, D, H, "bf16")
+    w = A.tm_moe_w(H, W, E, k, 64, 64, 2.0, 0x100000, 0x200000, 0x300000, 0x400000, 0x500000, 0x600000, 0x700000)
+    sub = A.tm_sublayer(None, 1, A.tm_swiglu_w(), w)
+    assert lib.tm_route_workspace_bytes(ctypes.byref(sh), A.TM_LAYOUT_MIXED, ctypes.byref(w)) > 0
+    assert lib.tm_sublayer_workspace_bytes(ctypes.byref(sh), A.TM_LAYOUT_MIXED, ctypes.byref(sub)) == 0
+    assert lib.tm_sparse_pertoken_moe(x, None, A.TM_LAYOUT_MIXED, ctypes.byref(sh), None, ctypes.byref(w), y, ws,
+                                      1 << 30, None) == A.TM_ERR_UNSUPPORTED
+    # the same shapes on rows (the reverting layout) pass the checks: only the workspace is short
+    wr = A.tm_moe_w(T, D, E, k, 64, 64, 2.0, 0x100000, 0x200000, 0x300000, 0x400000, 0x500000, 0x600000, 0x700000)
+    assert lib.tm_sparse_pertoken_moe(x, None, A.TM_LAYOUT_ROWS, ctypes.byref(sh), None, ctypes.byref(wr), y, ws,
+                                      16, None) == A.TM_ERR_WORKSPACE

@@ -980,6 +980,9 @@ tm_status check_sublayer(const tm_shape* shape, int layout, const tm_sublayer* s
     if (sub->is_moe) {
         s = check_moe(*g, &sub->moe);
         if (s == TM_OK && sub->moe.hidden_s == 0) s = TM_ERR_UNSUPPORTED;
+        // the bf16 combine reads the residual through a tensor map: mixed rows need 16-column head
+        // pieces (refused here, before the routing and the GEMMs are launched)
+        if (s == TM_OK && g->dtype == TM_BF16 && gemm1_amode(*g) == A_GATHER) s = TM_ERR_UNSUPPORTED;
         return s;
     }
     return check_dense(*g, &sub->dense);
