@@ -363,11 +363,23 @@ def test_sizes_past_32_bit_indexing_are_unsupported():
     assert lib.tm_workspace_bytes(ctypes.byref(ok), ctypes.byref(blk), 1, 0) > 0
 
 
-def test_binding_refuses_host_tensors():
-    """The binding passes only device addresses to the library: a host tensor raises before any call."""
+def test_binding_refuses_host_tensors_and_strided_views():
+    """The binding passes only addresses of dense device tensors to the library: a host tensor or a
+    strided view raises before any call (a tensor that claims to be on the device stands in for one
+    here); a slice along the leading axis is dense and passes."""
     import torch
-    with pytest.raises(ValueError):
+
+    class _OnDevice(torch.Tensor):
+        @property
+        def is_cuda(self):
+            return True
+
+    with pytest.raises(ValueError, match="device"):
         api._p(torch.zeros(4))
+    with pytest.raises(ValueError, match="contiguous"):
+        api._p(torch.zeros(4, 6).t().as_subclass(_OnDevice))
+    rows = torch.zeros(4, 6).as_subclass(_OnDevice)
+    assert api._p(rows[1:3]).value == rows.data_ptr() + 6 * 4
     assert api._p(None) is None
     assert api._p(_FakeTensor(0x1230)).value == 0x1230
 

@@ -20,12 +20,16 @@ _TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
 
 
 def _p(t: Optional[torch.Tensor]):
-    """Device address of a tensor for the C ABI, which reads and writes device memory only: a host
-    tensor is refused here (its address would reach a kernel)."""
+    """Device address of a tensor for the C ABI, which reads and writes device memory only and takes
+    every tensor dense in row-major order: a host tensor or a strided view is refused here (its
+    address would reach a kernel that reads it as something else)."""
     if t is None:
         return None
-    if isinstance(t, torch.Tensor) and not t.is_cuda:
-        raise ValueError(f"libtm takes device tensors; got one on {t.device}")
+    if isinstance(t, torch.Tensor):
+        if not t.is_cuda:
+            raise ValueError(f"libtm takes device tensors; got one on {t.device}")
+        if not t.is_contiguous():
+            raise ValueError(f"libtm takes contiguous tensors; got strides {t.stride()} for shape {tuple(t.shape)}")
     return ctypes.c_void_p(t.data_ptr())
 
 
