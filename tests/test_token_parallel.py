@@ -73,7 +73,8 @@ def _cfg(kind):
         return S.Config("tp_moe3", B=18, T=6, D=24, H=6, L=2, gap=1, dtype="bf16", mix=spec, rev=spec)
     if kind == "moe":
         spec = FFNSpec("moe", E=4, k=2, hidden_e=16, hidden_s=16, alpha=2.0)
-        return S.Config("tp_moe", B=24, T=4, D=32, H=4, L=3, gap=2, dtype="bf16", mix=spec, rev=spec)
+        # 25 samples: the overlapped schedule's three chunks are ragged (8, 8, 9)
+        return S.Config("tp_moe", B=25, T=4, D=32, H=4, L=3, gap=2, dtype="bf16", mix=spec, rev=spec)
     return S.Config("tp_dense", B=24, T=4, D=32, H=2, L=2, gap=1, dtype="bf16",
                     mix=FFNSpec("dense", hidden=32), rev=FFNSpec("dense", hidden=16))
 
